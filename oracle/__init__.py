@@ -1,0 +1,194 @@
+"""CPU oracle for 3D Block Sparse Attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The product path (the CUDA library and its
+Python binding) never calls it, and it never calls the product path.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64, OpenMP), which restates
+the method from the pages:
+
+* "LongCat-Video Technical Report" (paper summary page), section
+  "Block Sparse Attention (BSA)" -- 3D block partitioning, pooled block
+  similarity S_pool = Q_pool K_pool^T / sqrt(d), top-r key blocks per query
+  block, softmax(QK^T/sqrt(d)) V with non-selected positions at -inf;
+  section "Block Attention with KV-Cache for Efficient Multi-Task Inference" --
+  condition tokens attend only to condition tokens.
+* "LongCat-Video Technical Report #" (detail page), section
+  "3D Block Sparse Attention" -- chunk shape [4,4,8], Top-K / CDF modes.
+
+Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
+against hand-derived fixtures (``tests/golden/``), library routines (numpy
+sorting, reshaping and matmul), brute force on tiny inputs, closed forms and
+invariants. Beyond those pins, full-size outputs are "parity unpinned" except
+through the invariants, which the tests also check on sampled rows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+CHUNK = (4, 4, 8)
+CN = 128
+
+c_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so (gcc, -O2, OpenMP). Portable flags: no -march."""
+    src = os.path.join(_HERE, "oracle.c")
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(src):
+        tmp = _SO + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-D_GNU_SOURCE", "-o", tmp, src, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_SO)
+            vp, i32, i64, dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+            lib.oracle_token_of.restype = i64
+            lib.oracle_token_of.argtypes = [i32, i32, i32, i64, i32]
+            lib.oracle_rearrange.restype = i32
+            lib.oracle_rearrange.argtypes = [vp, i32, i32, i32, i32, i32, vp]
+            lib.oracle_pool.restype = i32
+            lib.oracle_pool.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp]
+            lib.oracle_scores.restype = i32
+            lib.oracle_scores.argtypes = [vp, vp, i32, i32, i32, dbl, i32, vp]
+            lib.oracle_select.restype = i64
+            lib.oracle_select.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, dbl, dbl, i32,
+                                          vp, vp, i64]
+            lib.oracle_attend.restype = i32
+            lib.oracle_attend.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, dbl, vp, vp, vp,
+                                          i64, vp, vp]
+            lib.oracle_dense.restype = i32
+            lib.oracle_dense.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, dbl, i32, vp, i64,
+                                         vp, vp]
+            lib.oracle_num_threads.restype = i32
+            lib.oracle_num_threads.argtypes = []
+            _lib = lib
+    return _lib
+
+
+def _u16(a):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, "inputs are bf16 bit patterns (uint16)"
+    return a
+
+
+def _check(rc, what):
+    if rc < 0:
+        raise ValueError(f"{what} failed ({rc})")
+    return rc
+
+
+def num_threads() -> int:
+    return _load().oracle_num_threads()
+
+
+def token_of(T, H, W, c, l) -> int:
+    return _load().oracle_token_of(T, H, W, c, l)
+
+
+def rearrange(x, T, H, W):
+    """THW order [B, heads, N, d] -> chunk-major [B, heads, Nc, 128, d] (bf16 bits)."""
+    x = _u16(x)
+    B, Hh, N, d = x.shape
+    out = np.empty((B, Hh, N // CN, CN, d), dtype=np.uint16)
+    _check(_load().oracle_rearrange(x.ctypes.data, B * Hh, T, H, W, d, out.ctypes.data),
+           "oracle_rearrange")
+    return out
+
+
+def pool(x, T, H, W, fp32=False):
+    """Chunk means [B, heads, Nc, d] (float64; float-valued when fp32)."""
+    x = _u16(x)
+    B, Hh, N, d = x.shape
+    out = np.empty((B, Hh, N // CN, d), dtype=np.float64)
+    _check(_load().oracle_pool(x.ctypes.data, B * Hh, T, H, W, d, int(fp32), out.ctypes.data),
+           "oracle_pool")
+    return out
+
+
+def scores(qp, kp, scale, fp32=False):
+    """Pooled scores [B, heads, Nc, Nc] = qp kp^T * scale."""
+    qp = np.ascontiguousarray(qp, dtype=np.float64)
+    kp = np.ascontiguousarray(kp, dtype=np.float64)
+    B, Hh, Nc, d = qp.shape
+    out = np.empty((B, Hh, Nc, Nc), dtype=np.float64)
+    _check(_load().oracle_scores(qp.ctypes.data, kp.ctypes.data, B * Hh, Nc, d, float(scale),
+                                 int(fp32), out.ctypes.data), "oracle_scores")
+    return out
+
+
+def select(S, T, H, W, mode="topk", topk=0, cdf_p=0.9, cap_frac=0.25, t_cond=0, fp32=False):
+    """CSR (row_ptr int32 [rows+1], col_idx int32 [nnz]) of the selected chunks."""
+    S = np.ascontiguousarray(S, dtype=np.float64)
+    B, Hh, Nc, _ = S.shape
+    rows = B * Hh * Nc
+    row_ptr = np.zeros(rows + 1, dtype=np.int32)
+    col_cap = rows * Nc
+    col_idx = np.empty(col_cap, dtype=np.int32)
+    nnz = _check(_load().oracle_select(S.ctypes.data, B * Hh, T, H, W, int(t_cond),
+                                       0 if mode == "topk" else 1, int(topk), float(cdf_p),
+                                       float(cap_frac), int(fp32), row_ptr.ctypes.data,
+                                       col_idx.ctypes.data, col_cap), "oracle_select")
+    return row_ptr, col_idx[:nnz].copy()
+
+
+def plan(q, k, T, H, W, scale, mode="topk", topk=0, cdf_p=0.9, cap_frac=0.25, t_cond=0,
+         fp32=False):
+    """pool -> scores -> select; returns (row_ptr, col_idx, S)."""
+    S = scores(pool(q, T, H, W, fp32), pool(k, T, H, W, fp32), scale, fp32)
+    rp, ci = select(S, T, H, W, mode, topk, cdf_p, cap_frac, t_cond, fp32)
+    return rp, ci, S
+
+
+def attend(q, k, v, T, H, W, scale, row_ptr, col_idx, rows, want_lse=True):
+    """Sparse attention for the listed CSR rows: out [n, 128, d] f64, lse [n, 128]."""
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    B, Hh, N, d = q.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    rp = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    ci = np.ascontiguousarray(col_idx, dtype=np.int32)
+    if ci.size == 0:
+        ci = np.zeros(1, dtype=np.int32)
+    out = np.empty((rows.size, CN, d), dtype=np.float64)
+    lse = np.empty((rows.size, CN), dtype=np.float64) if want_lse else None
+    _check(_load().oracle_attend(q.ctypes.data, k.ctypes.data, v.ctypes.data, B * Hh, T, H, W, d,
+                                 float(scale), rp.ctypes.data, ci.ctypes.data, rows.ctypes.data,
+                                 rows.size, out.ctypes.data,
+                                 lse.ctypes.data if lse is not None else None), "oracle_attend")
+    return out, lse
+
+
+def dense(q, k, v, T, H, W, scale, qtok, t_cond=0, want_lse=True):
+    """Dense (optionally block-causal) attention for global query ids bh*N + token."""
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    B, Hh, N, d = q.shape
+    qtok = np.ascontiguousarray(qtok, dtype=np.int64)
+    out = np.empty((qtok.size, d), dtype=np.float64)
+    lse = np.empty(qtok.size, dtype=np.float64) if want_lse else None
+    _check(_load().oracle_dense(q.ctypes.data, k.ctypes.data, v.ctypes.data, B * Hh, T, H, W, d,
+                                float(scale), int(t_cond), qtok.ctypes.data, qtok.size,
+                                out.ctypes.data, lse.ctypes.data if lse is not None else None),
+           "oracle_dense")
+    return out, lse
+
+
+def chunk_tokens(T, H, W, c):
+    """Token indices (THW order) of the 128 local tokens of chunk c."""
+    return np.array([token_of(T, H, W, c, l) for l in range(CN)], dtype=np.int64)

@@ -1,0 +1,383 @@
+/*
+ * CPU ORACLE for 3D Block Sparse Attention (BSA) -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, obviously-correct restatement of what the method computes, used
+ * only by the tests, by the benchmark's CPU-baseline leg and by the package's
+ * smoke check. It shares no code, header, table or helper with the CUDA path.
+ * Floating point is fp64 unless a function's `fp32` flag asks for the single
+ * precision decision mode (selection decided in the GPU kernel's precision).
+ *
+ * Sources (page titles and sections):
+ *   [P1] "LongCat-Video Technical Report" (paper summary page), section
+ *        "Block Sparse Attention (BSA)": 3D block partitioning, pooled block
+ *        similarity, top-r selection, masked softmax attention; section
+ *        "Block Attention with KV-Cache for Efficient Multi-Task Inference":
+ *        condition tokens attend only to condition tokens, noisy tokens to all.
+ *   [P3] "LongCat-Video Technical Report #" (detail page), section
+ *        "3D Block Sparse Attention": default chunk shape [4,4,8], Top-K and
+ *        CDF-threshold selection modes.
+ *
+ * Readings where the pages are loose (each also listed in the design notes):
+ *   - chunk shape (T,H,W) = (4,4,8), 128 tokens, for queries and keys alike;
+ *   - chunk index is 0-based over the rearranged sequence: chunk c holds the
+ *     tokens of block (ct,ch,cw) with c = (ct*NH + ch)*NW + cw and local index
+ *     (lt*4 + lh)*8 + lw (block order [N_T,N_H,N_W], intra-block order [t,h,w]);
+ *   - masked logits are -inf, i.e. an exact softmax over the selected keys;
+ *   - ties in selection go to the lower chunk index;
+ *   - CDF: softmax of the pooled scores over the candidate set, descending
+ *     order, smallest prefix with mass >= p, capped at max(1, floor(cap*|A|));
+ *   - block-causal: a query chunk whose frames all lie below t_cond may only
+ *     select condition chunks; other query chunks select among all chunks.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define CT 4
+#define CH 4
+#define CW 8
+#define CN (CT * CH * CW)
+
+static inline double bf16_to_double(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* [P1] 3D block partitioning: token index (THW order) of local token `l` of
+ * chunk `c`. */
+int64_t oracle_token_of(int T, int H, int W, int64_t c, int l) {
+    const int NH = H / CH, NW = W / CW;
+    const int64_t ct = c / ((int64_t)NH * NW);
+    const int ch = (int)((c / NW) % NH);
+    const int cw = (int)(c % NW);
+    const int lt = l / (CH * CW), lh = (l / CW) % CH, lw = l % CW;
+    const int64_t t = ct * CT + lt, h = (int64_t)ch * CH + lh, w = (int64_t)cw * CW + lw;
+    (void)T;
+    return (t * H + h) * W + w;
+}
+
+static int grid_ok(int T, int H, int W) {
+    return T > 0 && H > 0 && W > 0 && T % CT == 0 && H % CH == 0 && W % CW == 0;
+}
+
+/* [P1] "tokens are rearranged in memory so that all tokens within a block are
+ * contiguous": out[bh][c][l][:] = x[bh][token_of(c,l)][:] (bf16 bits copied). */
+int oracle_rearrange(const uint16_t* x, int BH, int T, int H, int W, int d, uint16_t* out) {
+    if (!x || !out || BH <= 0 || d <= 0 || !grid_ok(T, H, W)) return -1;
+    const int64_t N = (int64_t)T * H * W, Nc = N / CN;
+    for (int bh = 0; bh < BH; ++bh)
+        for (int64_t c = 0; c < Nc; ++c)
+            for (int l = 0; l < CN; ++l) {
+                const int64_t tok = oracle_token_of(T, H, W, c, l);
+                memcpy(out + (((int64_t)bh * Nc + c) * CN + l) * d, x + ((int64_t)bh * N + tok) * d,
+                       sizeof(uint16_t) * (size_t)d);
+            }
+    return 0;
+}
+
+/* [P1] pooled representations: mean of the n = 128 token vectors of a chunk.
+ * pooled[bh][c][:]. fp32 != 0: accumulate in float in local-token order. */
+int oracle_pool(const uint16_t* x, int BH, int T, int H, int W, int d, int fp32, double* pooled) {
+    if (!x || !pooled || BH <= 0 || d <= 0 || !grid_ok(T, H, W)) return -1;
+    const int64_t N = (int64_t)T * H * W, Nc = N / CN;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int bh = 0; bh < BH; ++bh)
+        for (int64_t c = 0; c < Nc; ++c) {
+            double* o = pooled + ((int64_t)bh * Nc + c) * d;
+            for (int e = 0; e < d; ++e) {
+                double acc = 0.0;
+                float accf = 0.0f;
+                for (int l = 0; l < CN; ++l) {
+                    const double v = bf16_to_double(x[((int64_t)bh * N + oracle_token_of(T, H, W, c, l)) * d + e]);
+                    if (fp32) accf += (float)v; else acc += v;
+                }
+                o[e] = fp32 ? (double)(accf * (1.0f / CN)) : acc / CN;
+            }
+        }
+    return 0;
+}
+
+/* [P1] S_pool = Q_pool K_pool^T / sqrt(d) (scale passed in). S[bh][i][m]. */
+int oracle_scores(const double* qp, const double* kp, int BH, int Nc, int d, double scale,
+                  int fp32, double* S) {
+    if (!qp || !kp || !S || BH <= 0 || Nc <= 0 || d <= 0) return -1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int bh = 0; bh < BH; ++bh)
+        for (int i = 0; i < Nc; ++i) {
+            const double* q = qp + ((int64_t)bh * Nc + i) * d;
+            for (int m = 0; m < Nc; ++m) {
+                const double* k = kp + ((int64_t)bh * Nc + m) * d;
+                double s;
+                if (fp32) {
+                    float a = 0.0f;
+                    for (int e = 0; e < d; ++e) a += (float)q[e] * (float)k[e];
+                    s = (double)(a * (float)scale);
+                } else {
+                    double a = 0.0;
+                    for (int e = 0; e < d; ++e) a += q[e] * k[e];
+                    s = a * scale;
+                }
+                S[((int64_t)bh * Nc + i) * Nc + m] = s;
+            }
+        }
+    return 0;
+}
+
+/* [P1] block-causal attention: a chunk is a condition chunk when every frame of
+ * it lies below t_cond. */
+static int is_condition_chunk(int H, int W, int64_t c, int t_cond) {
+    const int64_t ct = c / ((int64_t)(H / CH) * (W / CW));
+    return (ct * CT + CT - 1) < t_cond;
+}
+
+typedef struct {
+    double s;
+    int idx;
+} cand_t;
+
+/* descending score, then ascending index */
+static int cand_cmp(const void* a, const void* b) {
+    const cand_t* x = (const cand_t*)a;
+    const cand_t* y = (const cand_t*)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    return (x->idx > y->idx) - (x->idx < y->idx);
+}
+
+static int int_cmp(const void* a, const void* b) {
+    const int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+    return (x > y) - (x < y);
+}
+
+/*
+ * Block selection over the scores S[bh][i][m] -> CSR in row order (bh, i).
+ * mode 0 = top-k ([P1] top-r; [P3] Top-K), mode 1 = CDF ([P3] CDF threshold;
+ * [P1] "CDF-p mode": descending pooled scores until the cumulative softmax of
+ * the scores reaches p). k is clamped to |A(i)|. fp32 != 0 takes the CDF
+ * decision in float arithmetic (scores are already float-valued then).
+ * Column indices of a row are written in ascending order.
+ * Returns nnz >= 0, or -1 on bad arguments, -2 if col_cap is too small.
+ */
+int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, int mode,
+                      int topk, double cdf_p, double cap_frac, int fp32, int32_t* row_ptr,
+                      int32_t* col_idx, int64_t col_cap) {
+    if (!S || !row_ptr || !col_idx || BH <= 0 || !grid_ok(T, H, W) || t_cond < 0 ||
+        t_cond % CT != 0 || (mode != 0 && mode != 1) || (mode == 0 && topk <= 0))
+        return -1;
+    const int Nc = (int)((int64_t)T * H * W / CN);
+    cand_t* cand = (cand_t*)malloc(sizeof(cand_t) * (size_t)Nc);
+    int32_t* pick = (int32_t*)malloc(sizeof(int32_t) * (size_t)Nc);
+    if (!cand || !pick) {
+        free(cand);
+        free(pick);
+        return -1;
+    }
+    int64_t nnz = 0;
+    row_ptr[0] = 0;
+    for (int bh = 0; bh < BH; ++bh) {
+        for (int i = 0; i < Nc; ++i) {
+            const double* row = S + ((int64_t)bh * Nc + i) * Nc;
+            const int q_cond = t_cond > 0 && is_condition_chunk(H, W, i, t_cond);
+            int na = 0;
+            for (int m = 0; m < Nc; ++m) {
+                if (q_cond && !is_condition_chunk(H, W, m, t_cond)) continue;
+                cand[na].s = row[m];
+                cand[na].idx = m;
+                ++na;
+            }
+            qsort(cand, (size_t)na, sizeof(cand_t), cand_cmp);
+            int count;
+            if (mode == 0) {
+                count = topk < na ? topk : na;
+            } else {
+                /* softmax over A(i) of the scores, in the chosen precision */
+                int mstar = na;
+                if (fp32) {
+                    const float mx = (float)cand[0].s;
+                    float z = 0.0f;
+                    for (int a = 0; a < na; ++a) z += expf((float)cand[a].s - mx);
+                    float cum = 0.0f;
+                    for (int a = 0; a < na; ++a) {
+                        cum += expf((float)cand[a].s - mx) / z;
+                        if (cum >= (float)cdf_p) { mstar = a + 1; break; }
+                    }
+                } else {
+                    const double mx = cand[0].s;
+                    double z = 0.0;
+                    for (int a = 0; a < na; ++a) z += exp(cand[a].s - mx);
+                    double cum = 0.0;
+                    for (int a = 0; a < na; ++a) {
+                        cum += exp(cand[a].s - mx) / z;
+                        if (cum >= cdf_p) { mstar = a + 1; break; }
+                    }
+                }
+                int cap = (int)floor(cap_frac * na);
+                if (cap < 1) cap = 1;
+                count = mstar < cap ? mstar : cap;
+            }
+            if (nnz + count > col_cap) {
+                free(cand);
+                free(pick);
+                return -2;
+            }
+            for (int a = 0; a < count; ++a) pick[a] = cand[a].idx;
+            qsort(pick, (size_t)count, sizeof(int32_t), int_cmp);
+            memcpy(col_idx + nnz, pick, sizeof(int32_t) * (size_t)count);
+            nnz += count;
+            row_ptr[(int64_t)bh * Nc + i + 1] = (int32_t)nnz;
+        }
+    }
+    free(cand);
+    free(pick);
+    return nnz;
+}
+
+/*
+ * [P1] sparse attention: O = softmax(Q K^T / sqrt(d) with non-selected logits
+ * at -inf) V, evaluated for the query chunks listed in rows[] (row r = bh*Nc+i)
+ * over the tokens of the chunks in CSR row r. All arithmetic in fp64.
+ * out[n][l][:] is the output of local query l of rows[n]; lse[n][l] is the
+ * natural-log log-sum-exp of the scaled logits (nullable). A row with no
+ * selected chunk yields zeros and lse = -inf.
+ */
+int oracle_attend(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int T, int H,
+                  int W, int d, double scale, const int32_t* row_ptr, const int32_t* col_idx,
+                  const int64_t* rows, int64_t n_rows, double* out, double* lse) {
+    if (!q || !k || !v || !row_ptr || !col_idx || !rows || !out || BH <= 0 || d <= 0 ||
+        !grid_ok(T, H, W))
+        return -1;
+    const int64_t N = (int64_t)T * H * W, Nc = N / CN;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double* kd = NULL;
+        double* vd = NULL;
+        double* s = NULL;
+        double* qd = (double*)malloc(sizeof(double) * (size_t)d);
+        int64_t cap_keys = 0;
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t n = 0; n < n_rows; ++n) {
+            const int64_t r = rows[n];
+            if (r < 0 || r >= (int64_t)BH * Nc) { bad = 1; continue; }
+            const int64_t bh = r / Nc, i = r % Nc;
+            const int64_t beg = row_ptr[r], end = row_ptr[r + 1];
+            const int64_t nk = (end - beg) * CN;
+            if (nk > cap_keys) {
+                free(kd); free(vd); free(s);
+                kd = (double*)malloc(sizeof(double) * (size_t)(nk * d));
+                vd = (double*)malloc(sizeof(double) * (size_t)(nk * d));
+                s = (double*)malloc(sizeof(double) * (size_t)nk);
+                cap_keys = nk;
+            }
+            /* keys: every token of every selected chunk */
+            for (int64_t e = beg; e < end; ++e) {
+                const int64_t c = col_idx[e];
+                for (int l = 0; l < CN; ++l) {
+                    const int64_t tok = oracle_token_of(T, H, W, c, l);
+                    const int64_t j = (e - beg) * CN + l;
+                    for (int x = 0; x < d; ++x) {
+                        kd[j * d + x] = bf16_to_double(k[(bh * N + tok) * d + x]);
+                        vd[j * d + x] = bf16_to_double(v[(bh * N + tok) * d + x]);
+                    }
+                }
+            }
+            for (int lq = 0; lq < CN; ++lq) {
+                const int64_t qtok = oracle_token_of(T, H, W, i, lq);
+                for (int x = 0; x < d; ++x) qd[x] = bf16_to_double(q[(bh * N + qtok) * d + x]);
+                double* o = out + (n * CN + lq) * d;
+                if (nk == 0) {
+                    for (int x = 0; x < d; ++x) o[x] = 0.0;
+                    if (lse) lse[n * CN + lq] = -INFINITY;
+                    continue;
+                }
+                double mx = -INFINITY;
+                for (int64_t j = 0; j < nk; ++j) {
+                    double a = 0.0;
+                    for (int x = 0; x < d; ++x) a += qd[x] * kd[j * d + x];
+                    s[j] = a * scale;
+                    if (s[j] > mx) mx = s[j];
+                }
+                double z = 0.0;
+                for (int64_t j = 0; j < nk; ++j) {
+                    s[j] = exp(s[j] - mx);
+                    z += s[j];
+                }
+                for (int x = 0; x < d; ++x) o[x] = 0.0;
+                for (int64_t j = 0; j < nk; ++j) {
+                    const double w = s[j] / z;
+                    for (int x = 0; x < d; ++x) o[x] += w * vd[j * d + x];
+                }
+                if (lse) lse[n * CN + lq] = mx + log(z);
+            }
+        }
+        free(kd); free(vd); free(s); free(qd);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Dense attention over the token sequence in THW order, with the block-causal
+ * rule of [P1] ("Block Attention with KV-Cache"): a query in a frame below
+ * t_cond attends to the keys of frames below t_cond; every other query attends
+ * to all keys (t_cond = 0: plain dense attention). qtok[n] = bh*N + token.
+ * out[n][:], lse[n] (nullable). fp64.
+ */
+int oracle_dense(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int T, int H,
+                 int W, int d, double scale, int t_cond, const int64_t* qtok, int64_t n_q,
+                 double* out, double* lse) {
+    if (!q || !k || !v || !qtok || !out || BH <= 0 || T <= 0 || H <= 0 || W <= 0 || d <= 0 ||
+        t_cond < 0)
+        return -1;
+    const int64_t N = (int64_t)T * H * W, HW = (int64_t)H * W;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)N);
+        double* qd = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t n = 0; n < n_q; ++n) {
+            const int64_t g = qtok[n];
+            if (g < 0 || g >= (int64_t)BH * N) { bad = 1; continue; }
+            const int64_t bh = g / N, tok = g % N;
+            const int64_t t = tok / HW;
+            const int64_t nkeys = (t_cond > 0 && t < t_cond) ? (int64_t)t_cond * HW : N;
+            for (int x = 0; x < d; ++x) qd[x] = bf16_to_double(q[g * d + x]);
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < nkeys; ++j) {
+                const uint16_t* kr = k + (bh * N + j) * d;
+                double a = 0.0;
+                for (int x = 0; x < d; ++x) a += qd[x] * bf16_to_double(kr[x]);
+                s[j] = a * scale;
+                if (s[j] > mx) mx = s[j];
+            }
+            double z = 0.0;
+            for (int64_t j = 0; j < nkeys; ++j) {
+                s[j] = exp(s[j] - mx);
+                z += s[j];
+            }
+            double* o = out + n * d;
+            for (int x = 0; x < d; ++x) o[x] = 0.0;
+            for (int64_t j = 0; j < nkeys; ++j) {
+                const uint16_t* vr = v + (bh * N + j) * d;
+                const double w = s[j] / z;
+                for (int x = 0; x < d; ++x) o[x] += w * bf16_to_double(vr[x]);
+            }
+            if (lse) lse[n] = mx + log(z);
+        }
+        free(s);
+        free(qd);
+    }
+    return bad ? -1 : 0;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

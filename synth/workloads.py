@@ -1,0 +1,66 @@
+"""The five synthetic workloads (shapes, selection settings, generator knobs).
+
+Each workload stands in for a latent grid of the video DiT's refinement stage
+("LongCat-Video Technical Report", sections "Block Sparse Attention (BSA)" and
+"Efficiency Results": 480p / 720p generation, 93.75% sparsity, i.e. r = N_k/16
+key chunks per query chunk). No dataset is involved; the inputs are the seeded
+smooth fields of ``synth.c``.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, replace
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    heads: int
+    T: int
+    H: int
+    W: int
+    d: int
+    mode: str = "topk"          # "topk" | "cdf"
+    topk: int = 0
+    cdf_p: float = 0.9
+    cdf_cap_frac: float = 0.25
+    t_cond: int = 0             # latent frames of condition tokens (block-causal mask)
+    tfreq_mult: float = 1.0     # temporal frequency multiplier of the smooth field
+    seed: int = 0
+    cond_seed: int = 1
+
+    @property
+    def N(self) -> int:
+        return self.T * self.H * self.W
+
+    @property
+    def Nc(self) -> int:
+        return (self.T // 4) * (self.H // 4) * (self.W // 8)
+
+    @property
+    def n_cond(self) -> int:
+        """Condition chunks: chunks whose 4 frames all lie below t_cond."""
+        return (self.t_cond // 4) * (self.H // 4) * (self.W // 8)
+
+    @property
+    def rows(self) -> int:
+        return self.B * self.heads * self.Nc
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+WORKLOADS = {
+    # 512 tokens, 4 chunks, keep 2
+    "tiny": Workload("tiny", B=1, heads=2, T=4, H=8, W=16, d=64, topk=2),
+    # 480p-like: 28,672 tokens, 224 chunks, keep 14
+    "480p": Workload("480p", B=1, heads=32, T=16, H=32, W=56, d=128, topk=14),
+    # 720p-like refinement grid: 92,160 tokens, 720 chunks, keep 45
+    "720p": Workload("720p", B=1, heads=32, T=24, H=48, W=80, d=128, topk=45),
+    # long video: 215,040 tokens, 1,680 chunks, keep 105, faster motion
+    "long": Workload("long", B=1, heads=32, T=56, H=48, W=80, d=128, topk=105,
+                     tfreq_mult=2.0),
+    # block-causal video continuation with CDF selection (p = 0.9, cap 25%)
+    "causal_cdf": Workload("causal_cdf", B=2, heads=32, T=24, H=48, W=80, d=128,
+                           mode="cdf", cdf_p=0.9, cdf_cap_frac=0.25, t_cond=8),
+}
