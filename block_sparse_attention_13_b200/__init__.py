@@ -1,0 +1,247 @@
+"""B200 (sm_100a) 3D Block Sparse Attention -- Python binding of libbsa.so.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels (include/bsa.h documents the C ABI). PyTorch supplies device memory
+and streams. There is no CPU fallback: if libbsa.so is missing or cannot be
+loaded, every call raises.
+
+Method: "LongCat-Video Technical Report" (paper summary page), section
+"Block Sparse Attention (BSA)"; "LongCat-Video Technical Report #" (detail
+page), section "3D Block Sparse Attention".
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsa.so")
+
+BSA_OK = 0
+BSA_ERR_INVALID_ARG = 1
+BSA_ERR_SHAPE = 2
+BSA_ERR_UNSUPPORTED = 3
+BSA_ERR_ALIGNMENT = 4
+BSA_ERR_WORKSPACE_TOO_SMALL = 5
+BSA_ERR_CUDA = 6
+BSA_ERR_DEVICE_BAD_INDEX = 7
+BSA_ERR_DEVICE_TIMEOUT = 8
+BSA_ERR_CAPACITY = 9
+
+BSA_SEL_TOPK = 0
+BSA_SEL_CDF = 1
+
+EXPORTED = ("bsa_version", "bsa_status_string", "bsa_workspace_size", "bsa_plan_sizes",
+            "bsa_plan", "bsa_forward", "bsa_forward_ex", "bsa_read_status", "bsa_rearrange",
+            "bsa_pool", "bsa_scores", "bsa_selftest_timeout")
+
+
+class BsaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+
+
+class bsa_params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("heads", ctypes.c_int32), ("T", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("W", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("chunk_t", ctypes.c_int32), ("chunk_h", ctypes.c_int32),
+                ("chunk_w", ctypes.c_int32), ("scale", ctypes.c_float), ("mode", ctypes.c_int32),
+                ("topk", ctypes.c_int32), ("cdf_p", ctypes.c_float),
+                ("cdf_cap_frac", ctypes.c_float), ("t_cond", ctypes.c_int32)]
+
+
+def make_params(B, heads, T, H, W, d, mode="topk", topk=1, cdf_p=0.9, cdf_cap_frac=0.25,
+                t_cond=0, scale=0.0) -> bsa_params:
+    return bsa_params(B, heads, T, H, W, d, 4, 4, 8, float(scale),
+                      BSA_SEL_TOPK if mode == "topk" else BSA_SEL_CDF, int(topk), float(cdf_p),
+                      float(cdf_cap_frac), int(t_cond))
+
+
+def params_for(wl) -> bsa_params:
+    """Parameters of a workload description (anything with the Workload fields)."""
+    return make_params(wl.B, wl.heads, wl.T, wl.H, wl.W, wl.d, wl.mode, wl.topk, wl.cdf_p,
+                       wl.cdf_cap_frac, wl.t_cond)
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libbsa.so (raises if it is missing)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libbsa.so not built ({LIB_PATH}); run "
+                               "block_sparse_attention_13_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(bsa_params)
+        vp, i32, i64, sz, u64 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t,
+                                 ctypes.c_uint64)
+        sigs = {
+            "bsa_version": (i32, []),
+            "bsa_status_string": (ctypes.c_char_p, [i32]),
+            "bsa_workspace_size": (sz, [P]),
+            "bsa_plan_sizes": (i32, [P, ctypes.POINTER(i64), ctypes.POINTER(i64)]),
+            "bsa_plan": (i32, [P, vp, vp, vp, sz, vp, vp, i64, vp]),
+            "bsa_forward": (i32, [P, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, vp]),
+            "bsa_forward_ex": (i32, [P, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, u64, i32, vp]),
+            "bsa_read_status": (i32, [vp, vp]),
+            "bsa_rearrange": (i32, [P, vp, vp, i32, vp]),
+            "bsa_pool": (i32, [P, vp, vp, vp]),
+            "bsa_scores": (i32, [P, vp, vp, vp, vp]),
+            "bsa_selftest_timeout": (i32, [vp, u64, vp]),
+        }
+        for name, (res, args) in sigs.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().bsa_status_string(int(code)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != BSA_OK:
+        raise BsaError(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ------------------------------------------------------------------ C-ABI mirrors
+
+def bsa_version() -> int:
+    return lib().bsa_version()
+
+
+def bsa_workspace_size(p: bsa_params) -> int:
+    n = lib().bsa_workspace_size(ctypes.byref(p))
+    if n == 0:
+        raise BsaError(BSA_ERR_INVALID_ARG, "bsa_workspace_size")
+    return n
+
+
+def bsa_plan_sizes(p: bsa_params):
+    rows, nnz = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().bsa_plan_sizes(ctypes.byref(p), ctypes.byref(rows), ctypes.byref(nnz)),
+           "bsa_plan_sizes")
+    return rows.value, nnz.value
+
+
+def bsa_plan(p, q, k, workspace, row_ptr, col_idx, stream=None):
+    _check(lib().bsa_plan(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _ptr(row_ptr),
+                          _ptr(col_idx), col_idx.numel(), _stream(stream)), "bsa_plan")
+
+
+def bsa_forward(p, q, k, v, row_ptr, col_idx, workspace, out, lse=None, stream=None):
+    _check(lib().bsa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
+                             _ptr(col_idx), col_idx.numel(), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse),
+                             _stream(stream)), "bsa_forward")
+
+
+def bsa_forward_ex(p, q, k, v, row_ptr, col_idx, workspace, out, lse=None, timeout_ns=0,
+                   debug_flags=0, stream=None):
+    _check(lib().bsa_forward_ex(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
+                                _ptr(col_idx), col_idx.numel(), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _ptr(out),
+                                _ptr(lse), int(timeout_ns), int(debug_flags), _stream(stream)),
+           "bsa_forward_ex")
+
+
+def bsa_read_status(workspace, stream=None) -> int:
+    return lib().bsa_read_status(_ptr(workspace), _stream(stream))
+
+
+def bsa_rearrange(p, x, out, inverse=False, stream=None):
+    _check(lib().bsa_rearrange(ctypes.byref(p), _ptr(x), _ptr(out), 1 if inverse else 0,
+                               _stream(stream)), "bsa_rearrange")
+
+
+def bsa_pool(p, x, pooled, stream=None):
+    _check(lib().bsa_pool(ctypes.byref(p), _ptr(x), _ptr(pooled), _stream(stream)), "bsa_pool")
+
+
+def bsa_scores(p, qp, kp, S, stream=None):
+    _check(lib().bsa_scores(ctypes.byref(p), _ptr(qp), _ptr(kp), _ptr(S), _stream(stream)),
+           "bsa_scores")
+
+
+def bsa_selftest_timeout(workspace, timeout_ns, stream=None):
+    _check(lib().bsa_selftest_timeout(_ptr(workspace), int(timeout_ns), _stream(stream)),
+           "bsa_selftest_timeout")
+
+
+# ------------------------------------------------------------------ convenience
+
+@dataclass
+class Plan:
+    params: bsa_params
+    workspace: "object"
+    row_ptr: "object"
+    col_idx: "object"
+
+
+def allocate(p: bsa_params, device="cuda"):
+    """Workspace and CSR buffers for `p` (torch device tensors)."""
+    import torch
+    rows, nnz = bsa_plan_sizes(p)
+    ws = torch.empty(bsa_workspace_size(p), dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return Plan(p, ws, torch.empty(rows + 1, dtype=torch.int32, device=device),
+                torch.empty(max(nnz, 1), dtype=torch.int32, device=device))
+
+
+def plan(p: bsa_params, q, k, buffers: Plan | None = None, stream=None) -> Plan:
+    buffers = buffers or allocate(p, q.device)
+    bsa_plan(p, q, k, buffers.workspace, buffers.row_ptr, buffers.col_idx, stream)
+    return buffers
+
+
+def forward(pl: Plan, q, k, v, out=None, lse=None, stream=None):
+    import torch
+    out = torch.empty_like(q) if out is None else out
+    bsa_forward(pl.params, q, k, v, pl.row_ptr, pl.col_idx, pl.workspace, out, lse, stream)
+    return out
+
+
+def block_sparse_attention(q, k, v, topk=None, mode="topk", cdf_p=0.9, cdf_cap_frac=0.25,
+                           t_cond=0, grid=None, want_lse=False):
+    """One call: plan + forward for q, k, v [B, heads, T*H*W, d] bf16 on the GPU.
+
+    grid = (T, H, W) of the latent video. Returns out (and lse if asked).
+    """
+    import torch
+    B, heads, N, d = q.shape
+    T, H, W = grid
+    assert T * H * W == N
+    if topk is None:
+        topk = max(1, ((T // 4) * (H // 4) * (W // 8)) // 16)
+    p = make_params(B, heads, T, H, W, d, mode, topk, cdf_p, cdf_cap_frac, t_cond)
+    pl = plan(p, q, k)
+    lse = torch.empty((B, heads, N), dtype=torch.float32, device=q.device) if want_lse else None
+    out = forward(pl, q, k, v, lse=lse)
+    rc = bsa_read_status(pl.workspace)
+    _check(rc, "device status")
+    return (out, lse) if want_lse else out
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,268 @@
+// C ABI of the block sparse attention library: argument checking, workspace
+// layout and the launch sequence of each entry point. See include/bsa.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "bsa_internal.cuh"
+#include "bsa_ptx.cuh"
+
+namespace bsa {
+
+static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+WsLayout ws_layout(const Dims& g, const bsa_params& p) {
+    WsLayout L{};
+    size_t off = 0;
+    L.status = off;
+    off += 256;
+    const size_t pool_bytes = round_up((size_t)g.BH * g.Nc * g.d * sizeof(float), 256);
+    L.qpool = off;
+    off += pool_bytes;
+    L.kpool = off;
+    off += pool_bytes;
+    L.scores = off;
+    off += round_up((size_t)g.BH * g.Nc * g.Nc * sizeof(float), 256);
+    L.pad_stride = 0;
+    L.counts = L.padded = off;
+    if (p.mode == BSA_SEL_CDF) {
+        int cap = (int)std::floor((double)p.cdf_cap_frac * g.Nc);
+        if (cap < 1) cap = 1;
+        if (cap > g.Nc) cap = g.Nc;
+        L.pad_stride = cap;
+        L.counts = off;
+        off += round_up((size_t)g.rows * sizeof(int32_t), 256);
+        L.padded = off;
+        off += round_up((size_t)g.rows * cap * sizeof(int32_t), 256);
+    }
+    L.total = off;
+    return L;
+}
+
+// Validates `p` and fills the derived sizes. Host only, no CUDA calls.
+static int make_dims(const bsa_params* p, Dims* g) {
+    if (!p || !g) return BSA_ERR_INVALID_ARG;
+    if (p->B <= 0 || p->heads <= 0 || p->T <= 0 || p->H <= 0 || p->W <= 0 || p->d <= 0)
+        return BSA_ERR_SHAPE;
+    if (p->chunk_t != kChunkT || p->chunk_h != kChunkH || p->chunk_w != kChunkW)
+        return BSA_ERR_UNSUPPORTED;
+    if (p->d != 64 && p->d != 128) return BSA_ERR_UNSUPPORTED;
+    if (p->T % kChunkT || p->H % kChunkH || p->W % kChunkW) return BSA_ERR_SHAPE;
+    if (p->t_cond < 0 || p->t_cond % kChunkT || p->t_cond > p->T) return BSA_ERR_SHAPE;
+    if (!(std::isfinite(p->scale)) || p->scale < 0.f) return BSA_ERR_INVALID_ARG;
+    if (p->mode == BSA_SEL_TOPK) {
+        if (p->topk < 1) return BSA_ERR_INVALID_ARG;
+    } else if (p->mode == BSA_SEL_CDF) {
+        if (!(p->cdf_p > 0.f && p->cdf_p <= 1.f)) return BSA_ERR_INVALID_ARG;
+        if (!(p->cdf_cap_frac > 0.f && p->cdf_cap_frac <= 1.f)) return BSA_ERR_INVALID_ARG;
+    } else {
+        return BSA_ERR_INVALID_ARG;
+    }
+    g->B = p->B;
+    g->heads = p->heads;
+    g->T = p->T;
+    g->H = p->H;
+    g->W = p->W;
+    g->d = p->d;
+    g->NT = p->T / kChunkT;
+    g->NH = p->H / kChunkH;
+    g->NW = p->W / kChunkW;
+    const int64_t nc = (int64_t)g->NT * g->NH * g->NW;
+    g->N = (int64_t)p->T * p->H * p->W;
+    g->BH = (int64_t)p->B * p->heads;
+    // Limits of this implementation: selection keeps a row of scores in one
+    // warp's registers (Nc <= 2048), grids index batch*heads in y (<= 65535),
+    // and CSR offsets are int32.
+    if (nc > 2048 || g->BH > 65535) return BSA_ERR_UNSUPPORTED;
+    g->Nc = (int)nc;
+    g->rows = g->BH * g->Nc;
+    if (g->rows * (int64_t)g->Nc > INT32_MAX) return BSA_ERR_UNSUPPORTED;
+    g->n_cond = (p->t_cond / kChunkT) * g->NH * g->NW;
+    g->scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt((float)p->d);
+    return BSA_OK;
+}
+
+static int64_t max_nnz_of(const Dims& g, const bsa_params& p) {
+    if (p.mode == BSA_SEL_TOPK) {
+        const int64_t kc = p.topk < g.n_cond ? p.topk : g.n_cond;
+        const int64_t kn = p.topk < g.Nc ? p.topk : g.Nc;
+        return g.BH * ((int64_t)g.n_cond * kc + (int64_t)(g.Nc - g.n_cond) * kn);
+    }
+    int64_t total = 0;
+    for (int which = 0; which < 2; ++which) {
+        const int na = which == 0 ? g.n_cond : g.Nc;
+        const int64_t nrows = which == 0 ? g.n_cond : g.Nc - g.n_cond;
+        if (nrows == 0) continue;
+        int cap = (int)std::floor((double)p.cdf_cap_frac * na);
+        if (cap < 1) cap = 1;
+        total += nrows * cap;
+    }
+    return g.BH * total;
+}
+
+static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+static int cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
+
+static int device_ok() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return BSA_ERR_CUDA;
+    return major == 10 ? BSA_OK : BSA_ERR_UNSUPPORTED;
+}
+
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" {
+
+int bsa_version(void) { return 100; }
+
+const char* bsa_status_string(int s) {
+    switch (s) {
+        case BSA_OK: return "ok";
+        case BSA_ERR_INVALID_ARG: return "invalid argument";
+        case BSA_ERR_SHAPE: return "unsupported shape (T%4, H%4, W%8, t_cond%4 must be 0)";
+        case BSA_ERR_UNSUPPORTED: return "unsupported configuration or device";
+        case BSA_ERR_ALIGNMENT: return "tensor pointer not 16-byte aligned";
+        case BSA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case BSA_ERR_CUDA: return "CUDA call or launch failed";
+        case BSA_ERR_DEVICE_BAD_INDEX: return "device saw an out-of-range CSR index";
+        case BSA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case BSA_ERR_CAPACITY: return "col_idx capacity too small";
+        default: return "unknown status";
+    }
+}
+
+size_t bsa_workspace_size(const bsa_params* p) {
+    Dims g;
+    if (make_dims(p, &g) != BSA_OK) return 0;
+    return ws_layout(g, *p).total;
+}
+
+int bsa_plan_sizes(const bsa_params* p, int64_t* n_rows, int64_t* max_nnz) {
+    Dims g;
+    const int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!n_rows || !max_nnz) return BSA_ERR_INVALID_ARG;
+    *n_rows = g.rows;
+    *max_nnz = max_nnz_of(g, *p);
+    return BSA_OK;
+}
+
+int bsa_plan(const bsa_params* p, const void* q, const void* k, void* workspace, size_t ws_bytes,
+             int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, void* stream) {
+    Dims g;
+    int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!q || !k || !workspace || !row_ptr || !col_idx) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(workspace) || !aligned16(row_ptr) ||
+        !aligned16(col_idx))
+        return BSA_ERR_ALIGNMENT;
+    const WsLayout L = ws_layout(g, *p);
+    if (ws_bytes < L.total) return BSA_ERR_WORKSPACE_TOO_SMALL;
+    if (col_capacity < max_nnz_of(g, *p)) return BSA_ERR_CAPACITY;
+    if ((rc = device_ok()) != BSA_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    float* qp = reinterpret_cast<float*>(ws + L.qpool);
+    float* kp = reinterpret_cast<float*>(ws + L.kpool);
+    float* S = reinterpret_cast<float*>(ws + L.scores);
+    uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+    if ((rc = cuda_status(launch_pool(g, q, k, qp, kp, st))) != BSA_OK) return rc;
+    if ((rc = cuda_status(launch_scores(g, qp, kp, S, st))) != BSA_OK) return rc;
+    return cuda_status(launch_select(g, *p, S, row_ptr, col_idx, col_capacity,
+                                     reinterpret_cast<int32_t*>(ws + L.counts),
+                                     reinterpret_cast<int32_t*>(ws + L.padded), L.pad_stride,
+                                     status, st));
+}
+
+// Internal: forward with a custom wait limit and debug flags (used by the
+// binding's fault tests). Same contract as bsa_forward otherwise.
+int bsa_forward_ex(const bsa_params* p, const void* q, const void* k, const void* v,
+                   const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
+                   void* workspace, size_t ws_bytes, void* out, float* lse, uint64_t timeout_ns,
+                   int debug_flags, void* stream) {
+    Dims g;
+    int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!q || !k || !v || !row_ptr || !col_idx || !workspace || !out || col_capacity < 0)
+        return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(workspace) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return BSA_ERR_ALIGNMENT;
+    if (ws_bytes < 256) return BSA_ERR_WORKSPACE_TOO_SMALL;
+    if ((rc = device_ok()) != BSA_OK) return rc;
+    uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace));
+    return cuda_status(launch_forward(g, q, k, v, row_ptr, col_idx, col_capacity, out, lse, status,
+                                      timeout_ns ? timeout_ns : kDefaultTimeoutNs, debug_flags,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_forward(const bsa_params* p, const void* q, const void* k, const void* v,
+                const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
+                void* workspace, size_t ws_bytes, void* out, float* lse, void* stream) {
+    return bsa_forward_ex(p, q, k, v, row_ptr, col_idx, col_capacity, workspace, ws_bytes, out,
+                          lse, 0, 0, stream);
+}
+
+int bsa_read_status(void* workspace, void* stream) {
+    if (!workspace) return BSA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return BSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return BSA_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof(word), st) != cudaSuccess) return BSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return BSA_ERR_CUDA;
+    if (word & kStatusTimeout) return BSA_ERR_DEVICE_TIMEOUT;
+    if (word & kStatusBadIndex) return BSA_ERR_DEVICE_BAD_INDEX;
+    if (word & kStatusCapacity) return BSA_ERR_CAPACITY;
+    return BSA_OK;
+}
+
+int bsa_rearrange(const bsa_params* p, const void* x, void* out, int inverse, void* stream) {
+    Dims g;
+    int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!x || !out || (inverse != 0 && inverse != 1)) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out)) return BSA_ERR_ALIGNMENT;
+    if ((rc = device_ok()) != BSA_OK) return rc;
+    return cuda_status(launch_rearrange(g, x, out, inverse, static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_pool(const bsa_params* p, const void* x, float* pooled, void* stream) {
+    Dims g;
+    int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!x || !pooled) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(pooled)) return BSA_ERR_ALIGNMENT;
+    if ((rc = device_ok()) != BSA_OK) return rc;
+    return cuda_status(launch_pool(g, x, nullptr, pooled, nullptr, static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_scores(const bsa_params* p, const float* qp, const float* kp, float* S, void* stream) {
+    Dims g;
+    int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!qp || !kp || !S) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(qp) || !aligned16(kp) || !aligned16(S)) return BSA_ERR_ALIGNMENT;
+    if ((rc = device_ok()) != BSA_OK) return rc;
+    return cuda_status(launch_scores(g, qp, kp, S, static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_selftest_timeout(void* workspace, uint64_t timeout_ns, void* stream) {
+    if (!workspace || timeout_ns == 0) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return BSA_ERR_ALIGNMENT;
+    int rc = device_ok();
+    if (rc != BSA_OK) return rc;
+    return cuda_status(launch_selftest_timeout(static_cast<uint32_t*>(workspace), timeout_ns,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,55 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../include/bsa.h"
+
+namespace bsa {
+
+constexpr int kChunkT = 4, kChunkH = 4, kChunkW = 8;
+constexpr int kChunkTokens = kChunkT * kChunkH * kChunkW;  // 128
+
+// Derived sizes of one call.
+struct Dims {
+    int B, heads, T, H, W, d;
+    int NT, NH, NW, Nc;
+    int64_t N, BH, rows;
+    int n_cond;      // condition chunks per (batch, head); 0 without block-causal mask
+    float scale;
+};
+
+// Workspace layout (byte offsets), identical for plan and forward.
+struct WsLayout {
+    size_t status;   // uint32 status word (+ padding to 256)
+    size_t qpool;    // float [BH][Nc][d]
+    size_t kpool;    // float [BH][Nc][d]
+    size_t scores;   // float [BH][Nc][Nc]
+    size_t counts;   // int32 [rows]            (CDF only)
+    size_t padded;   // int32 [rows][pad_stride] (CDF only)
+    int pad_stride;  // max chunks a CDF row may keep
+    size_t total;
+};
+
+WsLayout ws_layout(const Dims& g, const bsa_params& p);
+
+// Launchers (return cudaError_t of the launch).
+cudaError_t launch_pool(const Dims& g, const void* x0, const void* x1, float* p0, float* p1,
+                        cudaStream_t st);
+cudaError_t launch_rearrange(const Dims& g, const void* src, void* dst, int inverse,
+                             cudaStream_t st);
+cudaError_t launch_scores(const Dims& g, const float* qp, const float* kp, float* S,
+                          cudaStream_t st);
+cudaError_t launch_select(const Dims& g, const bsa_params& p, const float* S, int32_t* row_ptr,
+                          int32_t* col_idx, int64_t col_cap, int32_t* counts, int32_t* padded,
+                          int pad_stride, uint32_t* status, cudaStream_t st);
+cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const void* v,
+                           const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
+                           void* out, float* lse, uint32_t* status, uint64_t timeout_ns,
+                           int debug_flags, cudaStream_t st);
+cudaError_t launch_selftest_timeout(uint32_t* status, uint64_t timeout_ns, cudaStream_t st);
+
+// Default limit of every device-side wait (2 s of global time).
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+
+}  // namespace bsa

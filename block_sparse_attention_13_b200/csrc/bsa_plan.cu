@@ -1,0 +1,484 @@
+// Block selection kernels: 3D gather + chunk mean-pool, pooled scores,
+// warp-level top-k / CDF selection into CSR, and the 3D rearrangement.
+//
+// Method ("LongCat-Video Technical Report", section "Block Sparse Attention
+// (BSA)"): Q_pool / K_pool are block means over the n tokens of each 3D block,
+// S_pool = Q_pool K_pool^T / sqrt(d), and each query block keeps the r key
+// blocks with the highest scores. "LongCat-Video Technical Report #", section
+// "3D Block Sparse Attention": chunk shape [4,4,8]; Top-K and CDF-threshold
+// selection. Block-causal candidates: "LongCat-Video Technical Report",
+// section "Block Attention with KV-Cache for Efficient Multi-Task Inference".
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "bsa_internal.cuh"
+#include "bsa_ptx.cuh"
+
+namespace bsa {
+
+namespace {
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void add_bf16x2(float& a, float& b, uint32_t u) {
+    a += __uint_as_float(u << 16);
+    b += __uint_as_float(u & 0xFFFF0000u);
+}
+
+// ------------------------------------------------------------------------
+// Gather + mean-pool. One CTA per (chunk, batch*head, tensor). A chunk is 16
+// contiguous segments (lt, lh) of 8 tokens (lw = 0..7); consecutive threads
+// read consecutive 16-byte vectors, so every warp load is one contiguous
+// 512-byte run. Each thread always covers the same 8 channels and sums them
+// over its tokens in fp32; a shared-memory pass finishes the 128-token sum.
+template <int D>
+__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ x0,
+                                                   const __nv_bfloat16* __restrict__ x1,
+                                                   float* __restrict__ p0, float* __restrict__ p1,
+                                                   int H, int W, int NH, int NW, int Nc,
+                                                   int64_t N) {
+    constexpr int VPT = D / 8;               // 16-byte vectors per token row
+    constexpr int ITERS = 128 * VPT / 256;   // vectors per thread
+    constexpr int GROUPS = 256 / VPT;        // threads that share one channel group
+    __shared__ float red[GROUPS][D + 1];
+
+    const __nv_bfloat16* x = blockIdx.z ? x1 : x0;
+    float* pooled = blockIdx.z ? p1 : p0;
+    const int c = blockIdx.x;
+    const int64_t bh = blockIdx.y;
+    const int ct = c / (NH * NW), ch = (c / NW) % NH, cw = c % NW;
+    const int tid = threadIdx.x;
+    const int dvec = tid % VPT;
+
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    const __nv_bfloat16* base = x + bh * N * D;
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+        const int v = it * 256 + tid;
+        const int l = v / VPT;  // local token (lt*4 + lh)*8 + lw
+        const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
+        const int64_t tok =
+            ((int64_t)(ct * kChunkT + lt) * H + (ch * kChunkH + lh)) * W + cw * kChunkW + lw;
+        const uint4 u = ld_nc_v4(base + tok * D + dvec * 8);
+        add_bf16x2(acc[0], acc[1], u.x);
+        add_bf16x2(acc[2], acc[3], u.y);
+        add_bf16x2(acc[4], acc[5], u.z);
+        add_bf16x2(acc[6], acc[7], u.w);
+    }
+    const int grp = tid / VPT;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[grp][dvec * 8 + e] = acc[e];
+    __syncthreads();
+    if (tid < D) {
+        float s = 0.f;
+#pragma unroll
+        for (int g2 = 0; g2 < GROUPS; ++g2) s += red[g2][tid];
+        pooled[(bh * Nc + c) * D + tid] = s * (1.0f / kChunkTokens);
+    }
+}
+
+// ------------------------------------------------------------------------
+// 3D rearrangement: a (lt, lh) segment of 8 tokens is contiguous both in the
+// [T,H,W] layout and in the chunk-major layout, so the copy is two streams of
+// contiguous 16-byte vectors.
+template <int D>
+__global__ void __launch_bounds__(256) rearrange_kernel(const __nv_bfloat16* __restrict__ src,
+                                                        __nv_bfloat16* __restrict__ dst, int H,
+                                                        int W, int NH, int NW, int Nc, int64_t N,
+                                                        int inverse) {
+    constexpr int VPT = D / 8;
+    constexpr int ITERS = 128 * VPT / 256;
+    const int c = blockIdx.x;
+    const int64_t bh = blockIdx.y;
+    const int ct = c / (NH * NW), ch = (c / NW) % NH, cw = c % NW;
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+        const int v = it * 256 + threadIdx.x;
+        const int l = v / VPT, dv = v % VPT;
+        const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
+        const int64_t tok =
+            ((int64_t)(ct * kChunkT + lt) * H + (ch * kChunkH + lh)) * W + cw * kChunkW + lw;
+        const int64_t thw = (bh * N + tok) * D + dv * 8;
+        const int64_t blk = ((bh * Nc + c) * kChunkTokens + l) * D + dv * 8;
+        const int64_t s_off = inverse ? blk : thw;
+        const int64_t d_off = inverse ? thw : blk;
+        *reinterpret_cast<uint4*>(dst + d_off) = ld_nc_v4(src + s_off);
+    }
+}
+
+// ------------------------------------------------------------------------
+// Pooled scores S[bh][i][m] = <qp[i], kp[m]> * scale in fp32 FMA. 64x64 output
+// tile per CTA, 4x4 register micro-tile per thread, operands staged
+// transposed in shared memory 32 channels at a time.
+__global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ qp,
+                                                     const float* __restrict__ kp,
+                                                     float* __restrict__ S, int Nc, int D,
+                                                     float scale) {
+    constexpr int BT = 64, BK = 32, LD = BT + 4;
+    __shared__ __align__(16) float As[BK][LD];
+    __shared__ __align__(16) float Bs[BK][LD];
+    const int64_t bh = blockIdx.z;
+    const int i0 = blockIdx.y * BT, m0 = blockIdx.x * BT;
+    const float* A = qp + bh * (int64_t)Nc * D;
+    const float* Bm = kp + bh * (int64_t)Nc * D;
+    const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+
+    for (int k0 = 0; k0 < D; k0 += BK) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int idx = tid + 256 * j;  // 512 float4 per 64x32 tile
+            const int r = idx / (BK / 4), kq = idx % (BK / 4);
+            float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
+            if (i0 + r < Nc) va = *reinterpret_cast<const float4*>(A + (int64_t)(i0 + r) * D + k0 + kq * 4);
+            if (m0 + r < Nc) vb = *reinterpret_cast<const float4*>(Bm + (int64_t)(m0 + r) * D + k0 + kq * 4);
+            As[kq * 4 + 0][r] = va.x; As[kq * 4 + 1][r] = va.y;
+            As[kq * 4 + 2][r] = va.z; As[kq * 4 + 3][r] = va.w;
+            Bs[kq * 4 + 0][r] = vb.x; Bs[kq * 4 + 1][r] = vb.y;
+            Bs[kq * 4 + 2][r] = vb.z; Bs[kq * 4 + 3][r] = vb.w;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < BK; ++kk) {
+            const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+            const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
+        }
+        __syncthreads();
+    }
+    float* out = S + bh * (int64_t)Nc * Nc;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const int i = i0 + ty * 4 + p;
+        if (i >= Nc) continue;
+        const int m = m0 + tx * 4;
+        float* o = out + (int64_t)i * Nc + m;
+        if ((Nc & 3) == 0 && m + 3 < Nc) {
+            *reinterpret_cast<float4*>(o) = make_float4(acc[p][0] * scale, acc[p][1] * scale,
+                                                        acc[p][2] * scale, acc[p][3] * scale);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (m + q < Nc) o[q] = acc[p][q] * scale;
+        }
+    }
+}
+
+// ------------------------------------------------------------------------
+// Selection: one warp per CSR row. Scores become order-preserving 32-bit keys
+// (larger score -> larger key; invalid slots are 0, below every real key).
+// The k-th largest key is found by a 32-step bitwise search with warp
+// reductions; rows are then emitted in ascending chunk order with ballots,
+// keeping the lowest indices among keys equal to the threshold.
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+template <int MAXJ>
+__device__ __forceinline__ uint32_t kth_largest_key(const uint32_t (&key)[MAXJ], int k) {
+    uint32_t v = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t t = v | (1u << bit);
+        int c = 0;
+#pragma unroll
+        for (int j = 0; j < MAXJ; ++j) c += key[j] >= t;
+        c = __reduce_add_sync(0xffffffffu, c);
+        if (c >= k) v = t;
+    }
+    return v;
+}
+
+template <int MAXJ>
+__global__ void __launch_bounds__(256) select_kernel(
+    const float* __restrict__ S, int Nc, int n_cond, int64_t rows, int mode, int topk,
+    float cdf_p, float cap_frac, int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
+    int64_t col_cap, int32_t* __restrict__ counts, int32_t* __restrict__ padded, int pad_stride,
+    uint32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (w >= rows) return;
+    const int64_t bh = w / Nc;
+    const int i = (int)(w % Nc);
+    const int na = (n_cond > 0 && i < n_cond) ? n_cond : Nc;  // candidates are [0, na)
+    const float* srow = S + w * (int64_t)Nc;
+
+    uint32_t key[MAXJ];
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int m = j * 32 + lane;
+        key[j] = (m < na) ? order_key(srow[m]) : 0u;
+    }
+
+    int count;
+    if (mode == BSA_SEL_TOPK) {
+        count = topk < na ? topk : na;
+    } else {
+        // softmax over A(i) in fp32; shortest descending prefix with mass >= p
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < MAXJ; ++j)
+            if (key[j]) mx = fmaxf(mx, key_value(key[j]));
+        mx = warp_max(mx);
+        float e[MAXJ];
+        float z = 0.f;
+#pragma unroll
+        for (int j = 0; j < MAXJ; ++j) {
+            e[j] = key[j] ? expf(key_value(key[j]) - mx) : 0.f;
+            z += e[j];
+        }
+        z = warp_sum(z);
+        const float target = cdf_p * z;
+        uint32_t v = 0;
+        for (int bit = 31; bit >= 0; --bit) {
+            const uint32_t t = v | (1u << bit);
+            float msum = 0.f;
+#pragma unroll
+            for (int j = 0; j < MAXJ; ++j) msum += (key[j] >= t) ? e[j] : 0.f;
+            msum = warp_sum(msum);
+            if (msum >= target) v = t;
+        }
+        int mstar = na;
+        if (v != 0) {
+            int cgt = 0, ceq = 0;
+            float mgt = 0.f;
+#pragma unroll
+            for (int j = 0; j < MAXJ; ++j) {
+                cgt += key[j] > v;
+                ceq += key[j] == v;
+                mgt += (key[j] > v) ? e[j] : 0.f;
+            }
+            cgt = __reduce_add_sync(0xffffffffu, cgt);
+            ceq = __reduce_add_sync(0xffffffffu, ceq);
+            mgt = warp_sum(mgt);
+            const float ev = expf(key_value(v) - mx);
+            int needed = 0;
+            float cum = mgt;
+            while (needed < ceq) {  // equal scores, taken in index order
+                cum += ev;
+                ++needed;
+                if (cum >= target) break;
+            }
+            mstar = cgt + needed;
+        }
+        // same double-precision formula as the host's workspace sizing
+        int cap = (int)floor((double)cap_frac * (double)na);
+        if (cap < 1) cap = 1;
+        if (cap > pad_stride) cap = pad_stride;
+        count = mstar < cap ? mstar : cap;
+    }
+
+    // emit the top-`count` chunks by (score desc, index asc), ascending
+    const uint32_t v = kth_largest_key(key, count);
+    int cgt = 0;
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) cgt += key[j] > v;
+    cgt = __reduce_add_sync(0xffffffffu, cgt);
+    const int need_eq = count - cgt;
+
+    int32_t* dst;
+    int64_t off;
+    if (mode == BSA_SEL_TOPK) {
+        const int kc = topk < n_cond ? topk : n_cond;
+        const int kn = topk < Nc ? topk : Nc;
+        const int64_t per_bh = (int64_t)n_cond * kc + (int64_t)(Nc - n_cond) * kn;
+        off = bh * per_bh + (i < n_cond ? (int64_t)i * kc : (int64_t)n_cond * kc + (int64_t)(i - n_cond) * kn);
+        if (off + count > col_cap) {
+            if (lane == 0) atomicOr(status, kStatusCapacity);
+            return;
+        }
+        dst = col_idx + off;
+        if (lane == 0) {
+            row_ptr[w + 1] = (int32_t)(off + count);
+            if (w == 0) row_ptr[0] = 0;
+        }
+    } else {
+        dst = padded + w * (int64_t)pad_stride;
+        if (lane == 0) counts[w] = count;
+    }
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int run_sel = 0, run_eq = 0;
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        if (j * 32 >= na) break;
+        const bool gt = key[j] > v;
+        const bool eq = key[j] == v;
+        const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+        const int eq_before = run_eq + __popc(eqb & lt_mask);
+        const bool sel = gt || (eq && eq_before < need_eq);
+        const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+        if (sel) dst[run_sel + __popc(sb & lt_mask)] = j * 32 + lane;
+        run_sel += __popc(sb);
+        run_eq += __popc(eqb);
+    }
+}
+
+// Exclusive scan of CDF row counts into row_ptr (one CTA).
+__global__ void __launch_bounds__(1024) scan_counts_kernel(const int32_t* __restrict__ counts,
+                                                          int64_t rows, int32_t* __restrict__ row_ptr) {
+    __shared__ int64_t warp_tot[32];
+    const int tid = threadIdx.x;
+    const int64_t per = (rows + 1023) / 1024;
+    const int64_t beg = tid * per;
+    const int64_t end = beg + per < rows ? beg + per : rows;
+    int64_t local = 0;
+    for (int64_t r = beg; r < end; ++r) local += counts[r];
+    // inclusive scan of `local` over the block
+    int64_t x = local;
+    const int lane = tid & 31, wid = tid >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+        int64_t t = warp_tot[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        warp_tot[lane] = t;
+    }
+    __syncthreads();
+    int64_t run = x - local + (wid > 0 ? warp_tot[wid - 1] : 0);
+    for (int64_t r = beg; r < end; ++r) {
+        run += counts[r];
+        row_ptr[r + 1] = (int32_t)run;
+    }
+    if (tid == 0) row_ptr[0] = 0;
+}
+
+// Copy each padded CDF row to its CSR position (one warp per row).
+__global__ void __launch_bounds__(256) compact_kernel(const int32_t* __restrict__ counts,
+                                                      const int32_t* __restrict__ padded,
+                                                      int pad_stride, int64_t rows,
+                                                      const int32_t* __restrict__ row_ptr,
+                                                      int32_t* __restrict__ col_idx,
+                                                      int64_t col_cap, uint32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (w >= rows) return;
+    const int64_t off = row_ptr[w];
+    const int n = counts[w];
+    if (off + n > col_cap) {
+        if (lane == 0) atomicOr(status, kStatusCapacity);
+        return;
+    }
+    for (int e = lane; e < n; e += 32) col_idx[off + e] = padded[w * (int64_t)pad_stride + e];
+}
+
+// One CTA waits on an mbarrier that nothing arrives at; the bounded wait
+// expires, records the timeout and the kernel returns normally.
+__global__ void selftest_timeout_kernel(uint32_t* status, uint64_t timeout_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, &abort_flag, status, timeout_ns);
+    __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_pool(const Dims& g, const void* x0, const void* x1, float* p0, float* p1,
+                        cudaStream_t st) {
+    dim3 grid(g.Nc, (unsigned)g.BH, x1 ? 2 : 1);
+    const auto* a = static_cast<const __nv_bfloat16*>(x0);
+    const auto* b = static_cast<const __nv_bfloat16*>(x1 ? x1 : x0);
+    if (g.d == 128)
+        pool_kernel<128><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, g.H, g.W, g.NH, g.NW, g.Nc, g.N);
+    else
+        pool_kernel<64><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, g.H, g.W, g.NH, g.NW, g.Nc, g.N);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rearrange(const Dims& g, const void* src, void* dst, int inverse,
+                             cudaStream_t st) {
+    dim3 grid(g.Nc, (unsigned)g.BH);
+    const auto* s = static_cast<const __nv_bfloat16*>(src);
+    auto* d = static_cast<__nv_bfloat16*>(dst);
+    if (g.d == 128)
+        rearrange_kernel<128><<<grid, 256, 0, st>>>(s, d, g.H, g.W, g.NH, g.NW, g.Nc, g.N, inverse);
+    else
+        rearrange_kernel<64><<<grid, 256, 0, st>>>(s, d, g.H, g.W, g.NH, g.NW, g.Nc, g.N, inverse);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scores(const Dims& g, const float* qp, const float* kp, float* S,
+                          cudaStream_t st) {
+    dim3 grid((g.Nc + 63) / 64, (g.Nc + 63) / 64, (unsigned)g.BH);
+    scores_kernel<<<grid, 256, 0, st>>>(qp, kp, S, g.Nc, g.d, g.scale);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select(const Dims& g, const bsa_params& p, const float* S, int32_t* row_ptr,
+                          int32_t* col_idx, int64_t col_cap, int32_t* counts, int32_t* padded,
+                          int pad_stride, uint32_t* status, cudaStream_t st) {
+    const unsigned blocks = (unsigned)((g.rows + 7) / 8);
+    const int mode = p.mode;
+#define BSA_SELECT(MJ)                                                                       \
+    select_kernel<MJ><<<blocks, 256, 0, st>>>(S, g.Nc, g.n_cond, g.rows, mode, p.topk,      \
+                                              p.cdf_p, p.cdf_cap_frac, row_ptr, col_idx,    \
+                                              col_cap, counts, padded, pad_stride, status)
+    if (g.Nc <= 32) BSA_SELECT(1);
+    else if (g.Nc <= 256) BSA_SELECT(8);
+    else if (g.Nc <= 1024) BSA_SELECT(32);
+    else if (g.Nc <= 2048) BSA_SELECT(64);
+    else return cudaErrorInvalidValue;
+#undef BSA_SELECT
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || mode == BSA_SEL_TOPK) return e;
+    scan_counts_kernel<<<1, 1024, 0, st>>>(counts, g.rows, row_ptr);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    compact_kernel<<<blocks, 256, 0, st>>>(counts, padded, pad_stride, g.rows, row_ptr, col_idx,
+                                           col_cap, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_timeout(uint32_t* status, uint64_t timeout_ns, cudaStream_t st) {
+    selftest_timeout_kernel<<<1, 32, 0, st>>>(status, timeout_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace bsa

@@ -1,0 +1,167 @@
+/*
+ * bsa.h -- C ABI of the B200 (sm_100a) 3D Block Sparse Attention library.
+ *
+ * The operation is the 3D Block Sparse Attention (BSA) of a video diffusion
+ * transformer, as described on the pages:
+ *   [P1] "LongCat-Video Technical Report" (paper summary page), section
+ *        "Block Sparse Attention (BSA)" -- 3D block partitioning, pooled block
+ *        similarity, top-r key blocks per query block, masked softmax
+ *        attention; section "Block Attention with KV-Cache for Efficient
+ *        Multi-Task Inference" -- condition tokens attend only among themselves.
+ *   [P3] "LongCat-Video Technical Report #" (detail page), section
+ *        "3D Block Sparse Attention" -- default chunk shape [4,4,8], Top-K and
+ *        CDF-threshold selection; section "开源实现" (open-source kernels) --
+ *        gating-score, varlen forward and 3D rearrange kernels.
+ *
+ * Conventions for every entry point:
+ *   - Tensors Q, K, V, O are bf16, contiguous [B, heads, T*H*W, d], tokens in
+ *     [T,H,W] order (t slowest, w fastest). DEVICE pointers, 16-byte aligned.
+ *   - Chunk c of a (batch, head) covers the (4,4,8) block (ct, ch, cw) with
+ *     c = (ct*(H/4) + ch)*(W/8) + cw; its local token l = (lt*4 + lh)*8 + lw.
+ *   - CSR rows are ordered (batch, head, query chunk); row r's key chunks are
+ *     col_idx[row_ptr[r] .. row_ptr[r+1]), ascending. int32, DEVICE memory.
+ *   - The caller allocates and owns every buffer. The library never allocates
+ *     device memory and holds no global state beyond cached driver entry points.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Launches are
+ *     asynchronous; errors found on the device are read with bsa_read_status.
+ *   - Return value: BSA_OK (0) or a bsa_status code. No exception crosses the ABI.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BSA_API __attribute__((visibility("default")))
+#else
+#define BSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BSA_OK = 0,
+    BSA_ERR_INVALID_ARG = 1,         /* null pointer, bad enum, k < 1, p outside (0,1] ...   */
+    BSA_ERR_SHAPE = 2,               /* T%4, H%4, W%8 or t_cond%4 != 0, sizes <= 0 ...        */
+    BSA_ERR_UNSUPPORTED = 3,         /* d not in {64,128}, chunk shape != (4,4,8), no sm_100  */
+    BSA_ERR_ALIGNMENT = 4,           /* a tensor pointer is not 16-byte aligned               */
+    BSA_ERR_WORKSPACE_TOO_SMALL = 5, /* ws_bytes < bsa_workspace_size()                       */
+    BSA_ERR_CUDA = 6,                /* a CUDA runtime/driver call or launch failed           */
+    BSA_ERR_DEVICE_BAD_INDEX = 7,    /* device saw an out-of-range CSR row or column index    */
+    BSA_ERR_DEVICE_TIMEOUT = 8,      /* a bounded device-side wait expired                    */
+    BSA_ERR_CAPACITY = 9             /* col_idx capacity smaller than the selection needs     */
+} bsa_status;
+
+typedef enum { BSA_SEL_TOPK = 0, BSA_SEL_CDF = 1 } bsa_select_mode;
+
+typedef struct {
+    int32_t B, heads, T, H, W, d; /* d in {64,128}; T%4 == H%4 == W%8 == 0                 */
+    int32_t chunk_t, chunk_h, chunk_w; /* must be 4,4,8 ([P3] default chunk shape)          */
+    float scale;        /* softmax scale; 0 means 1/sqrt(d) ([P1] scaled dot product)     */
+    int32_t mode;       /* bsa_select_mode                                                */
+    int32_t topk;       /* TOPK: key chunks kept per query chunk (clamped to |A(i)|)      */
+    float cdf_p;        /* CDF: cumulative pooled-softmax mass to reach, in (0,1]          */
+    float cdf_cap_frac; /* CDF: at most max(1, floor(cap_frac*|A(i)|)) chunks, in (0,1]   */
+    int32_t t_cond;     /* leading latent frames holding condition tokens; 0 = none; %4==0 */
+} bsa_params;
+
+/* Library version: major*10000 + minor*100 + patch. */
+BSA_API int bsa_version(void);
+
+/* Text for a status code (static storage; never NULL). */
+BSA_API const char* bsa_status_string(int status);
+
+/* Bytes of device workspace that bsa_plan / bsa_forward need for `p`
+ * (status word, pooled Q/K in fp32, pooled scores, CDF scratch). 0 if `p` is
+ * invalid. The same workspace serves both calls. */
+BSA_API size_t bsa_workspace_size(const bsa_params* p);
+
+/* CSR sizes for `p`: *n_rows = B*heads*Nc; *max_nnz = col_idx capacity that
+ * always suffices (exact for TOPK; upper bound for CDF). Host-only call. */
+BSA_API int bsa_plan_sizes(const bsa_params* p, int64_t* n_rows, int64_t* max_nnz);
+
+/*
+ * Block selection ([P1] pooled block similarity + top-r; [P3] Top-K / CDF):
+ *   1. mean-pool every (4,4,8) chunk of Q and K in fp32 ([P1] Q_pool, K_pool);
+ *   2. pooled scores S[i,m] = <Q_pool[i], K_pool[m]> * scale in fp32;
+ *   3. candidates A(i): all chunks, or -- when t_cond > 0 and chunk i lies
+ *      entirely in frames < t_cond -- the condition chunks only ([P1] block
+ *      attention for condition tokens);
+ *   4. TOPK: the topk highest scores of A(i), ties to the lower chunk index;
+ *      CDF: softmax of S over A(i), descending order (ties to the lower
+ *      index), the shortest prefix with mass >= cdf_p, at most
+ *      max(1, floor(cdf_cap_frac*|A(i)|)) chunks.
+ * q, k: device bf16 [B,heads,N,d]. workspace: device, >= bsa_workspace_size.
+ * row_ptr: device int32 [n_rows+1]; col_idx: device int32 [col_capacity],
+ * written ascending per row. Errors: INVALID_ARG, SHAPE, UNSUPPORTED,
+ * ALIGNMENT, WORKSPACE_TOO_SMALL, CAPACITY (host-detectable: col_capacity <
+ * max_nnz), CUDA.
+ */
+BSA_API int bsa_plan(const bsa_params* p, const void* q, const void* k, void* workspace,
+             size_t ws_bytes, int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+             void* stream);
+
+/*
+ * Sparse attention over the selected chunks ([P1] O = softmax(QK^T/sqrt(d)
+ * with non-selected positions at -inf) V): for every query token of chunk i,
+ * an exact softmax over the 128*|row i| keys of the chunks in CSR row i, with
+ * bf16 tensor-core products, fp32 accumulation and fp32 online softmax.
+ * q, k, v: device bf16 [B,heads,N,d]; out: device bf16, same shape, written in
+ * [T,H,W] token order (the inverse 3D rearrangement is fused). lse: nullable
+ * device fp32 [B,heads,N], natural-log log-sum-exp of the scaled logits per
+ * query (-inf for an empty row). row_ptr/col_idx: CSR as written by bsa_plan,
+ * or any caller CSR with col_capacity entries; rows or columns out of range
+ * are skipped (their output is zero) and reported as DEVICE_BAD_INDEX by
+ * bsa_read_status. Errors: INVALID_ARG, SHAPE, UNSUPPORTED, ALIGNMENT,
+ * WORKSPACE_TOO_SMALL, CUDA.
+ */
+BSA_API int bsa_forward(const bsa_params* p, const void* q, const void* k, const void* v,
+                const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
+                void* workspace, size_t ws_bytes, void* out, float* lse, void* stream);
+
+/* bsa_forward with an explicit limit for every device-side wait (timeout_ns;
+ * 0 = the default of 2 s) and debug flags (bit 0: the MMA warp withholds its
+ * first "scores ready" signal, so the softmax warps' bounded wait expires and
+ * the kernel reports DEVICE_TIMEOUT without faulting or hanging; used by the
+ * failure-detection tests). Same contract as bsa_forward otherwise. */
+BSA_API int bsa_forward_ex(const bsa_params* p, const void* q, const void* k, const void* v,
+                   const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
+                   void* workspace, size_t ws_bytes, void* out, float* lse, uint64_t timeout_ns,
+                   int debug_flags, void* stream);
+
+/* Synchronise `stream`, return the first device-side error recorded in the
+ * workspace status word since the last call (BSA_OK if none) and clear it. */
+BSA_API int bsa_read_status(void* workspace, void* stream);
+
+/*
+ * 3D rearrangement ([P1] "tokens ... rearranged in memory so that all tokens
+ * within a block are contiguous"; [P3] rearrange_THW_to_3d_block and its
+ * inverse). inverse = 0: x in [T,H,W] token order -> out chunk-major
+ * [B,heads,Nc,128,d]; inverse = 1: chunk-major -> [T,H,W]. bf16, device,
+ * 16-byte aligned, non-overlapping. A bit-exact permutation.
+ */
+BSA_API int bsa_rearrange(const bsa_params* p, const void* x, void* out, int inverse, void* stream);
+
+/* Chunk mean-pool ([P1] Q_pool / K_pool) of one tensor: x bf16 [B,heads,N,d]
+ * -> pooled fp32 [B,heads,Nc,d] (device). The same kernel bsa_plan runs. */
+BSA_API int bsa_pool(const bsa_params* p, const void* x, float* pooled, void* stream);
+
+/* Pooled scores ([P1] S_pool = Q_pool K_pool^T / sqrt(d); [P3] gating-score
+ * kernel): qp, kp fp32 [B,heads,Nc,d] -> S fp32 [B,heads,Nc,Nc] (device),
+ * S = <qp_i, kp_m> * scale. The same kernel bsa_plan runs. */
+BSA_API int bsa_scores(const bsa_params* p, const float* qp, const float* kp, float* S, void* stream);
+
+/* Device self-test of the bounded-wait machinery: launches one CTA that waits
+ * on a barrier nothing arrives at, for at most timeout_ns, then records
+ * DEVICE_TIMEOUT in the workspace status word and returns. The context stays
+ * usable. workspace: device, >= 256 bytes. */
+BSA_API int bsa_selftest_timeout(void* workspace, uint64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H_ */

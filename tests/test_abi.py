@@ -1,0 +1,162 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol that
+include/bsa.h declares, and its host-side argument checks return the
+documented status codes before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_13_b200 as bsa
+from block_sparse_attention_13_b200 import build as bsa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    bsa_build.build()
+    return bsa.lib()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "bsa.h")).read()
+    return re.findall(r"^BSA_API\s+[\w\s\*]+?\b(bsa_\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_binding_names():
+    names = declared_symbols()
+    assert len(names) == len(set(names)) >= 12
+    assert set(names) == set(bsa.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_library_exports_nothing_else():
+    out = os.popen(f"nm -D --defined-only {bsa.LIB_PATH}").read()
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert exported == set(declared_symbols())
+
+
+def test_version_and_strings(L):
+    assert bsa.bsa_version() == 100
+    for code in range(0, 10):
+        s = bsa.status_string(code)
+        assert s and s != "unknown status"
+    assert bsa.status_string(99) == "unknown status"
+
+
+def P(**kw):
+    base = dict(B=1, heads=2, T=4, H=8, W=16, d=64, mode="topk", topk=2)
+    base.update(kw)
+    return bsa.make_params(**base)
+
+
+def rc_sizes(p):
+    rows, nnz = ctypes.c_int64(), ctypes.c_int64()
+    return bsa.lib().bsa_plan_sizes(ctypes.byref(p), ctypes.byref(rows), ctypes.byref(nnz)), \
+        rows.value, nnz.value
+
+
+def test_plan_sizes_topk_and_cdf(L):
+    rc, rows, nnz = rc_sizes(P())
+    assert (rc, rows, nnz) == (0, 8, 16)
+    # 720p-like: 32 heads x 720 chunks, keep 45
+    rc, rows, nnz = rc_sizes(P(heads=32, T=24, H=48, W=80, d=128, topk=45))
+    assert (rc, rows, nnz) == (0, 23040, 23040 * 45)
+    # block-causal CDF: 240 condition rows capped at 60, 480 noisy rows capped at 180
+    rc, rows, nnz = rc_sizes(P(B=2, heads=32, T=24, H=48, W=80, d=128, mode="cdf", t_cond=8))
+    assert (rc, rows, nnz) == (0, 46080, 64 * (240 * 60 + 480 * 180))
+    # block-causal top-k clamps condition rows to the 240 condition chunks
+    rc, rows, nnz = rc_sizes(P(heads=1, T=24, H=48, W=80, d=128, topk=300, t_cond=8))
+    assert (rc, nnz) == (0, 240 * 240 + 480 * 300)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=6), bsa.BSA_ERR_SHAPE),
+    (dict(H=6), bsa.BSA_ERR_SHAPE),
+    (dict(W=12), bsa.BSA_ERR_SHAPE),
+    (dict(B=0), bsa.BSA_ERR_SHAPE),
+    (dict(d=96), bsa.BSA_ERR_UNSUPPORTED),
+    (dict(t_cond=2), bsa.BSA_ERR_SHAPE),
+    (dict(t_cond=8), bsa.BSA_ERR_SHAPE),
+    (dict(topk=0), bsa.BSA_ERR_INVALID_ARG),
+    (dict(mode="cdf", cdf_p=0.0), bsa.BSA_ERR_INVALID_ARG),
+    (dict(mode="cdf", cdf_p=1.5), bsa.BSA_ERR_INVALID_ARG),
+    (dict(mode="cdf", cdf_cap_frac=0.0), bsa.BSA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), bsa.BSA_ERR_INVALID_ARG),
+    (dict(T=4 * 64, H=4 * 8, W=8 * 8), bsa.BSA_ERR_UNSUPPORTED),  # Nc = 4096 > 2048
+])
+def test_invalid_params(L, kw, code):
+    p = P(**kw)
+    assert rc_sizes(p)[0] == code
+    assert bsa.lib().bsa_workspace_size(ctypes.byref(p)) == 0
+
+
+def test_chunk_shape_other_than_448_unsupported(L):
+    p = P()
+    p.chunk_w = 4
+    assert rc_sizes(p)[0] == bsa.BSA_ERR_UNSUPPORTED
+
+
+def test_workspace_size_layout(L):
+    p = P(heads=32, T=24, H=48, W=80, d=128, topk=45)
+    n = bsa.bsa_workspace_size(p)
+    pool = 32 * 720 * 128 * 4
+    assert n == 256 + 2 * pool + 32 * 720 * 720 * 4
+    pc = P(B=2, heads=32, T=24, H=48, W=80, d=128, mode="cdf", t_cond=8)
+    assert bsa.bsa_workspace_size(pc) > n
+
+
+FAKE = 0x10000  # a 16-byte aligned address that is never dereferenced
+
+
+def vp(x):
+    return ctypes.c_void_p(x)
+
+
+def test_plan_host_checks_before_any_cuda_call(L):
+    p = P()
+    ws = bsa.bsa_workspace_size(p)
+    f = L.bsa_plan
+    pp = ctypes.byref(p)
+    assert f(None, vp(FAKE), vp(FAKE), vp(FAKE), ws, vp(FAKE), vp(FAKE), 16, None) == \
+        bsa.BSA_ERR_INVALID_ARG
+    assert f(pp, None, vp(FAKE), vp(FAKE), ws, vp(FAKE), vp(FAKE), 16, None) == \
+        bsa.BSA_ERR_INVALID_ARG
+    assert f(pp, vp(FAKE + 8), vp(FAKE), vp(FAKE), ws, vp(FAKE), vp(FAKE), 16, None) == \
+        bsa.BSA_ERR_ALIGNMENT
+    assert f(pp, vp(FAKE), vp(FAKE), vp(FAKE), ws - 1, vp(FAKE), vp(FAKE), 16, None) == \
+        bsa.BSA_ERR_WORKSPACE_TOO_SMALL
+    assert f(pp, vp(FAKE), vp(FAKE), vp(FAKE), ws, vp(FAKE), vp(FAKE), 15, None) == \
+        bsa.BSA_ERR_CAPACITY
+
+
+def test_forward_host_checks_before_any_cuda_call(L):
+    p = P()
+    f = L.bsa_forward
+    pp = ctypes.byref(p)
+    a = [vp(FAKE)] * 5
+    assert f(pp, *a, 16, vp(FAKE), 256, None, None, None) == bsa.BSA_ERR_INVALID_ARG
+    assert f(pp, vp(FAKE), vp(FAKE), vp(FAKE + 4), vp(FAKE), vp(FAKE), 16, vp(FAKE), 256,
+             vp(FAKE), None, None) == bsa.BSA_ERR_ALIGNMENT
+    assert f(pp, *a, 16, vp(FAKE), 255, vp(FAKE), None, None) == \
+        bsa.BSA_ERR_WORKSPACE_TOO_SMALL
+    assert f(pp, *a, -1, vp(FAKE), 256, vp(FAKE), None, None) == bsa.BSA_ERR_INVALID_ARG
+
+
+def test_no_cpu_fallback_without_a_gpu(L):
+    """With valid arguments and no usable GPU the call fails loudly."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    p = P()
+    ws = bsa.bsa_workspace_size(p)
+    rc = L.bsa_plan(ctypes.byref(p), vp(FAKE), vp(FAKE), vp(FAKE), ws, vp(FAKE), vp(FAKE), 16,
+                    None)
+    assert rc == bsa.BSA_ERR_CUDA
+    with pytest.raises(bsa.BsaError):
+        bsa.bsa_plan_sizes(P(T=6))

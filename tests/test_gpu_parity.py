@@ -1,0 +1,222 @@
+"""GPU parity: every stage of the CUDA path against the CPU oracle on the same
+seeded inputs (marked gpu; needs a B200).
+
+Bars (from the method's targets): rearrangement bit-exact; pooled means within
+1e-6 absolute of fp64; pooled scores within 1e-5 relative; chunk selection
+bit-exact except near-ties within 1e-5 relative (tests/parity.py); attention
+max-abs <= 2e-2 and mean-abs <= 2e-3 against the fp64 oracle evaluated on the
+GPU's own CSR (so selection and attention errors stay separate).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity import ATT_MAX_ABS, ATT_MEAN_ABS, compare_attention, compare_csr, rows_of
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import block_sparse_attention_13_b200 as bsa  # noqa: E402
+
+W = synth.WORKLOADS
+
+# small cases that span several score tiles, a ragged tail and both head dims
+SMALL = {
+    "tiny": W["tiny"],
+    "ragged60_d64": W["tiny"].with_(name="ragged60_d64", heads=3, T=8, H=24, W=40, d=64, topk=5),
+    "ragged135_d128": W["tiny"].with_(name="ragged135_d128", heads=2, T=12, H=20, W=72, d=128,
+                                      topk=9),
+    "causal_topk": W["tiny"].with_(name="causal_topk", heads=2, T=16, H=16, W=32, d=128, topk=6,
+                                   t_cond=8),
+    "causal_cdf_small": W["tiny"].with_(name="causal_cdf_small", B=2, heads=2, T=16, H=16, W=32,
+                                        d=128, mode="cdf", cdf_p=0.9, cdf_cap_frac=0.25,
+                                        t_cond=8),
+    "cdf_nocap": W["tiny"].with_(name="cdf_nocap", heads=2, T=8, H=16, W=32, d=64, mode="cdf",
+                                 cdf_p=0.5, cdf_cap_frac=1.0),
+}
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).cuda()
+
+
+def host_f32(t):
+    return t.float().cpu().numpy()
+
+
+def run_gpu(wl, q, k, v):
+    p = bsa.params_for(wl)
+    pl = bsa.allocate(p)
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    bsa.bsa_plan(p, qd, kd, pl.workspace, pl.row_ptr, pl.col_idx)
+    out = torch.empty_like(qd)
+    lse = torch.empty((wl.B, wl.heads, wl.N), dtype=torch.float32, device="cuda")
+    bsa.bsa_forward(p, qd, kd, vd, pl.row_ptr, pl.col_idx, pl.workspace, out, lse)
+    status = bsa.bsa_read_status(pl.workspace)
+    rp = pl.row_ptr.cpu().numpy()
+    ci = pl.col_idx[: int(rp[-1])].cpu().numpy()
+    return rp, ci, out, lse, status
+
+
+def gather_rows(x_bhnd, wl, rows):
+    """[B,Hh,N,d] (numpy) -> [len(rows), 128, d] in chunk-local order."""
+    flat = x_bhnd.reshape(wl.B * wl.heads, wl.N, -1)
+    return np.stack([flat[r // wl.Nc][oracle.chunk_tokens(wl.T, wl.H, wl.W, r % wl.Nc)]
+                     for r in rows])
+
+
+def check_case(wl, rows=None):
+    q, k, v = synth.make_qkv(wl)
+    scale = 1.0 / math.sqrt(wl.d)
+    rp, ci, out, lse, status = run_gpu(wl, q, k, v)
+    assert status == bsa.BSA_OK, bsa.status_string(status)
+    # selection: oracle decides in fp32 (the kernel's precision); ties judged in fp64
+    o_rp, o_ci, _ = oracle.plan(q, k, wl.T, wl.H, wl.W, scale, wl.mode, wl.topk, wl.cdf_p,
+                                wl.cdf_cap_frac, wl.t_cond, fp32=True)
+    S64 = oracle.scores(oracle.pool(q, wl.T, wl.H, wl.W), oracle.pool(k, wl.T, wl.H, wl.W), scale)
+    n_checked, n_diff = compare_csr(rp, ci, o_rp, o_ci, S64, wl.Nc, wl.n_cond, wl.mode,
+                                    wl.cdf_p, wl.cdf_cap_frac)
+    assert n_diff <= max(1, n_checked // 100), f"{n_diff} of {n_checked} rows differ (ties)"
+    # attention on the GPU's own CSR
+    if rows is None:
+        rows = np.arange(wl.rows)
+    o_out, o_lse = oracle.attend(q, k, v, wl.T, wl.H, wl.W, scale, rp, ci, rows)
+    g_out = gather_rows(host_f32(out), wl, rows)
+    mx, mean = compare_attention(g_out, o_out)
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+    g_lse = gather_rows(lse.cpu().numpy()[..., None], wl, rows)[..., 0]
+    np.testing.assert_allclose(g_lse, o_lse, rtol=0, atol=2e-3)
+    return dict(rows_diff=n_diff, max_abs=mx, mean_abs=mean)
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_small_cases_all_rows(name):
+    check_case(SMALL[name])
+
+
+def test_rearrange_bit_exact_and_inverse():
+    for wl in (SMALL["ragged60_d64"], SMALL["ragged135_d128"]):
+        q, _, _ = synth.make_qkv(wl)
+        p = bsa.params_for(wl)
+        x = dev(q)
+        blk = torch.empty_like(x)
+        bsa.bsa_rearrange(p, x, blk)
+        back = torch.empty_like(x)
+        bsa.bsa_rearrange(p, blk, back, inverse=True)
+        torch.cuda.synchronize()
+        got = blk.view(torch.int16).cpu().numpy().view(np.uint16).reshape(
+            wl.B, wl.heads, wl.Nc, 128, wl.d)
+        np.testing.assert_array_equal(got, oracle.rearrange(q, wl.T, wl.H, wl.W))
+        assert torch.equal(back.view(torch.int16), x.view(torch.int16))
+
+
+def test_pool_and_scores_match_oracle():
+    wl = SMALL["ragged135_d128"]
+    q, k, _ = synth.make_qkv(wl)
+    p = bsa.params_for(wl)
+    qp = torch.empty((wl.B, wl.heads, wl.Nc, wl.d), dtype=torch.float32, device="cuda")
+    kp = torch.empty_like(qp)
+    bsa.bsa_pool(p, dev(q), qp)
+    bsa.bsa_pool(p, dev(k), kp)
+    S = torch.empty((wl.B, wl.heads, wl.Nc, wl.Nc), dtype=torch.float32, device="cuda")
+    bsa.bsa_scores(p, qp, kp, S)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(qp.cpu().numpy(), oracle.pool(q, wl.T, wl.H, wl.W), rtol=0,
+                               atol=1e-6)
+    scale = 1 / math.sqrt(wl.d)
+    S_or = oracle.scores(qp.cpu().numpy().astype(np.float64),
+                         kp.cpu().numpy().astype(np.float64), scale)
+    err = np.abs(S.cpu().numpy() - S_or)
+    assert err.max() <= 1e-5 * np.abs(S_or).max()
+
+
+def test_all_chunks_equals_dense_oracle():
+    wl = W["tiny"].with_(T=8, H=16, W=32, d=64, heads=2)  # 32 chunks
+    wl = wl.with_(topk=wl.Nc)
+    q, k, v = synth.make_qkv(wl)
+    rp, ci, out, lse, status = run_gpu(wl, q, k, v)
+    assert status == bsa.BSA_OK
+    assert np.all(np.diff(rp) == wl.Nc)
+    ids = np.arange(0, wl.B * wl.heads * wl.N, 7)
+    ref, ref_lse = oracle.dense(q, k, v, wl.T, wl.H, wl.W, 1 / math.sqrt(wl.d), ids)
+    got = host_f32(out).reshape(-1, wl.d)[ids]
+    assert np.abs(got - ref).max() <= ATT_MAX_ABS and np.abs(got - ref).mean() <= ATT_MEAN_ABS
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(-1)[ids], ref_lse, atol=2e-3, rtol=0)
+
+
+def test_caller_csr_empty_and_out_of_range_rows():
+    wl = W["tiny"]  # 8 rows of 4 chunks
+    q, k, v = synth.make_qkv(wl)
+    p = bsa.params_for(wl)
+    pl = bsa.allocate(p)
+    # rows: [0,3] [] [1] [2,3] [3,7] [] [0,1] [2]; chunk 7 does not exist (Nc = 4)
+    rp = np.array([0, 2, 2, 3, 5, 7, 7, 9, 10], dtype=np.int32)
+    ci = np.array([0, 3, 1, 2, 3, 3, 7, 0, 1, 2], dtype=np.int32)
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    out = torch.full_like(qd, 7.0)
+    lse = torch.zeros((1, 2, wl.N), dtype=torch.float32, device="cuda")
+    bsa.bsa_forward(p, qd, kd, vd, torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda(),
+                    pl.workspace, out, lse)
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_ERR_DEVICE_BAD_INDEX
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_OK  # cleared by the read
+    g = host_f32(out)
+    g_lse = lse.cpu().numpy()[..., None]
+    # the out-of-range chunk is skipped: row 4 attends to chunk 3 only
+    rp_o = np.array([0, 2, 2, 3, 5, 6, 6, 8, 9], dtype=np.int32)
+    ci_o = np.array([0, 3, 1, 2, 3, 3, 0, 1, 2], dtype=np.int32)
+    good = [0, 2, 3, 4, 6, 7]
+    o_out, o_lse = oracle.attend(q, k, v, wl.T, wl.H, wl.W, 1 / math.sqrt(wl.d), rp_o, ci_o, good)
+    mx, mean = compare_attention(gather_rows(g, wl, good), o_out)
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS
+    np.testing.assert_allclose(gather_rows(g_lse, wl, good)[..., 0], o_lse, rtol=0, atol=2e-3)
+    for r in (1, 5):  # empty rows: zeros and lse = -inf
+        assert np.all(gather_rows(g, wl, [r]) == 0)
+        assert np.all(np.isneginf(gather_rows(g_lse, wl, [r])))
+
+
+def test_row_ptr_out_of_range_is_rejected_not_read():
+    wl = W["tiny"]
+    q, k, v = synth.make_qkv(wl)
+    p = bsa.params_for(wl)
+    pl = bsa.allocate(p)
+    rp = torch.tensor([0, 2, 4, 6, 8, 1 << 30, 12, 14, 16], dtype=torch.int32, device="cuda")
+    ci = torch.zeros(16, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(dev(q))
+    bsa.bsa_forward(p, dev(q), dev(k), dev(v), rp, ci, pl.workspace, out)
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_ERR_DEVICE_BAD_INDEX
+
+
+def test_deterministic():
+    wl = SMALL["causal_cdf_small"]
+    q, k, v = synth.make_qkv(wl)
+    a = run_gpu(wl, q, k, v)
+    b = run_gpu(wl, q, k, v)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    assert torch.equal(a[2].view(torch.int16), b[2].view(torch.int16))
+
+
+def test_bounded_wait_selftest_reports_timeout():
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    bsa.bsa_selftest_timeout(ws, 20_000_000)  # 20 ms
+    assert bsa.bsa_read_status(ws) == bsa.BSA_ERR_DEVICE_TIMEOUT
+    check_case(SMALL["tiny"])  # the context is still usable
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def _sample_rows(wl, per_head, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = []
+    for bh in range(wl.B * wl.heads):
+        rows.extend(bh * wl.Nc + rng.choice(wl.Nc, size=min(per_head, wl.Nc), replace=False))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+@pytest.mark.parametrize("name,per_head", [("480p", 8), ("720p", 4), ("long", 2),
+                                           ("causal_cdf", 2)])
+def test_full_size_workloads(name, per_head):
+    wl = W[name]
+    check_case(wl, rows=_sample_rows(wl, per_head))
