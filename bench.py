@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the 3D block sparse attention hot path on B200.
+
+One step = bsa_plan (chunk gather + mean-pool, pooled scores, selection into
+CSR) + bsa_forward (block-sparse attention) over one synthetic batch of the
+chosen workload (default: the 720p-like refinement grid, 93.75% sparse),
+inputs resident in HBM. Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 720p]
+  python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Multi-GPU: one process per GPU (torchrun); every rank runs an independent
+problem (its own batch element), there is no collective on the data path;
+timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "BSA fwd ms/call and executed TFLOPS (% of bf16 peak) at 720p grid, 93.75% sparse"
+UNIT = "TFLOP/s"
+KERNEL_SRC = os.path.join(ROOT, "block_sparse_attention_13_b200", "csrc", "bsa_attn.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "bsa_fwd_traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="720p")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (smaller cases for profiling)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk.get("bf16_tflops", 1590.0), pk.get("hbm_gbs", 6650.0), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(os.path.dirname(KERNEL_SRC))):
+        if f in ("bsa_attn.cu", "bsa_ptx.cuh"):
+            with open(os.path.join(os.path.dirname(KERNEL_SRC), f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(workload):
+    """DRAM bytes per forward launch from a committed ncu capture, if the
+    kernel source is unchanged since that capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        rec = json.load(f)
+    ent = rec.get(workload)
+    if not ent or ent.get("kernel_hash") != kernel_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+def exec_flops(wl, nnz):
+    """Executed attention FLOPs: QK^T and PV over 128x128 tiles of kept chunks."""
+    return 4.0 * wl.d * 128 * 128 * nnz
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------- CPU oracle leg
+
+def cpu_oracle_sample(wl, q, k, v, target_s):
+    """Time the oracle (as it stands) on a bounded sample and extrapolate the
+    full step: plan on one head, attention on a seeded sample of query chunks."""
+    import numpy as np
+    import oracle
+
+    scale = 1.0 / math.sqrt(wl.d)
+    qh, kh = q[:1, :1], k[:1, :1]
+    t0 = time.perf_counter()
+    rp, ci, _ = oracle.plan(qh, kh, wl.T, wl.H, wl.W, scale, wl.mode, wl.topk, wl.cdf_p,
+                            wl.cdf_cap_frac, min(wl.t_cond, wl.T))
+    t_plan_head = time.perf_counter() - t0
+    # attention rows of head 0, grown until the sample takes ~target_s
+    rng = np.random.default_rng(0)
+    order = rng.permutation(wl.Nc)
+    n, t_att, done = 4, 0.0, 0
+    while True:
+        rows = np.sort(order[done:done + n])
+        t0 = time.perf_counter()
+        oracle.attend(qh, kh, v[:1, :1], wl.T, wl.H, wl.W, scale, rp, ci, rows, want_lse=False)
+        t_att += time.perf_counter() - t0
+        done += len(rows)
+        if t_att + t_plan_head >= target_s or done >= wl.Nc:
+            break
+        n = min(wl.Nc - done, max(4, int(n * 2)))
+    sample_nnz = int(sum(rp[r + 1] - rp[r] for r in order[:done]))
+    t_per_chunk_pair = t_att / max(sample_nnz, 1)
+    full_nnz = int(rp[-1]) * wl.B * wl.heads   # head 0's selection size as the estimate
+    t_full = t_plan_head * wl.B * wl.heads + t_per_chunk_pair * full_nnz
+    value = exec_flops(wl, full_nnz) / t_full / 1e12
+    return {
+        "value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+        "sample": (f"plan on 1 of {wl.B * wl.heads} (batch,head) pairs + attention on {done} of "
+                   f"{wl.rows} query chunks; full step extrapolated linearly "
+                   f"({t_full:.1f} s)"),
+        "sample_seconds": round(t_plan_head + t_att, 2),
+        "est_full_step_s": t_full,
+    }
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return 0
+    import numpy as np  # noqa: F401
+    import synth
+    q, k, v = synth.make_qkv(wl.with_(B=1, heads=1))
+    per_step = max(1.0, min(args.cpu_seconds, 100.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    cb = None
+    for s in range(args.warmup + args.steps):
+        cb = cpu_oracle_sample(wl, q, k, v, per_step)
+        if s >= args.warmup:
+            vals.append(cb["value"])
+    value = statistics.median(vals)
+    cb["value"] = value
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": cb["est_full_step_s"] * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, world),
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, world):
+    return {"workload": wl.name, "B": wl.B, "heads": wl.heads, "grid_thw": [wl.T, wl.H, wl.W],
+            "d": wl.d, "chunk_thw": [4, 4, 8], "mode": wl.mode,
+            "topk": wl.topk if wl.mode == "topk" else None,
+            "cdf_p": wl.cdf_p if wl.mode == "cdf" else None,
+            "t_cond": wl.t_cond, "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2 (Q+K+V per step "
+                  f"{3 * wl.B * wl.heads * wl.N * wl.d * 2 / 1e9:.2f} GB)"}
+
+
+# ---------------------------------------------------------------------- GPU leg
+
+def main():
+    args = parse()
+    import synth
+    wl = synth.WORKLOADS[args.workload]
+    if args.heads:
+        wl = wl.with_(heads=args.heads, name=f"{wl.name}_h{args.heads}")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, wl, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import block_sparse_attention_13_b200 as bsa
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    # inputs: this rank's own problem (batch offset = rank), pinned host + device copies
+    q_np, k_np, v_np = synth.make_qkv(wl, batch_offset=rank * wl.B)
+    host = [torch.from_numpy(a).view(torch.bfloat16).pin_memory() for a in (q_np, k_np, v_np)]
+    q, k, v = (h.to("cuda", non_blocking=False) for h in host)
+    p = bsa.params_for(wl)
+    pl = bsa.allocate(p)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        bsa.bsa_plan(p, q, k, pl.workspace, pl.row_ptr, pl.col_idx)
+        bsa.bsa_forward(p, q, k, v, pl.row_ptr, pl.col_idx, pl.workspace, out)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    rc = bsa.bsa_read_status(pl.workspace)
+    if rc != bsa.BSA_OK:
+        print(json.dumps({"error": f"device status {bsa.status_string(rc)}"}), flush=True)
+        return 1
+    nnz = int(pl.row_ptr[-1].item())
+    flops = exec_flops(wl, nnz)
+
+    # ---- timed region: K steps, per-kernel events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            bsa.bsa_plan(p, q, k, pl.workspace, pl.row_ptr, pl.col_idx)
+            ev[s][1].record(stream)
+            bsa.bsa_forward(p, q, k, v, pl.row_ptr, pl.col_idx, pl.workspace, out)
+            ev[s][2].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    clocks = clk.summary()
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    plan_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    ms_per_step = total_ms / args.steps
+    rc = bsa.bsa_read_status(pl.workspace)
+    launches_per_step = 4 if wl.mode == "topk" else 6   # pool, scores, select(+scan, compact), fwd
+    total_flops = sum_over_ranks(flops * args.steps)
+    value = total_flops / (total_ms / 1e3) / 1e12
+
+    # ---- end to end through the C ABI with host buffers (pinned), per step:
+    # H2D of q, k, v; plan; forward; D2H of the output
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e_s.record(stream)
+    for _ in range(max(args.e2e_steps, 1)):
+        q.copy_(host[0], non_blocking=True)
+        k.copy_(host[1], non_blocking=True)
+        v.copy_(host[2], non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+    e_e.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e)) / max(args.e2e_steps, 1)
+    e2e_value = sum_over_ranks(flops) / (e2e_ms / 1e3) / 1e12
+    h2d = sum(h.numel() * h.element_size() for h in host)
+    d2h = out_host.numel() * out_host.element_size()
+
+    # ---- dense comparator at the same shape (torch SDPA as dispatched)
+    dense = None
+    if not args.no_dense and rank == 0 and wl.t_cond == 0:
+        import torch.nn.functional as F
+        F.scaled_dot_product_attention(q, k, v)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            F.scaled_dot_product_attention(q, k, v)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        dense_ms = statistics.median(ts)
+        dense = {"sdpa_ms": dense_ms, "bsa_step_ms": ms_per_step,
+                 "speedup": dense_ms / ms_per_step,
+                 "dense_tflops": 4.0 * wl.B * wl.heads * wl.N * wl.N * wl.d / dense_ms / 1e9}
+
+    peak_tf, peak_hbm, peak_src = load_peaks()
+    fwd_tflops = flops / (fwd_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "achieved": fwd_tflops, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": fwd_tflops / peak_tf, "traffic": load_traffic(wl.name),
+                "kernel": "bsa_fwd_kernel", "peak_source": f"{peak_src} bf16 (burst)",
+                "algorithmic_flops_per_launch": flops}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(wl, q_np, k_np, v_np, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": workload_config(wl, world),
+            "plan_ms": plan_ms, "fwd_ms": fwd_ms, "fwd_exec_tflops": fwd_tflops,
+            "nnz": nnz, "sparsity": 1.0 - nnz / (wl.B * wl.heads * wl.Nc * wl.Nc),
+            "dense_equiv_tflops": 4.0 * wl.B * wl.heads * wl.N * wl.N * wl.d / ms_per_step / 1e9,
+            "dense": dense, "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks, "device_status": bsa.status_string(rc),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0 if rc == bsa.BSA_OK else 1
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -8,22 +8,24 @@
 // section "3D Block Sparse Attention": online softmax over variable-length
 // block lists), bf16 tensor-core products and fp32 accumulation.
 //
-// One CTA owns one query chunk (128 queries = one M=128 MMA tile). Q, K, V and
-// O are addressed directly in [T,H,W] token order through 5-D TMA maps whose
-// box (64 ch, 8 w, 4 h, 4 t) lands a (4,4,8) chunk in shared memory already in
+// A query chunk (128 queries) is one M=128 MMA tile. Q, K, V and O are
+// addressed directly in [T,H,W] token order through 5-D TMA maps whose box
+// (64 ch, 8 w, 4 h, 4 t) lands a (4,4,8) chunk in shared memory already in
 // chunk-local order, so neither the forward rearrangement nor its inverse
 // costs a pass over HBM.
 //
-// Roles (192 threads): warps 0-3 softmax + epilogue (thread m owns query row m
-// = TMEM lane m); warp 4 TMA producer; warp 5 TMEM allocator + MMA issuer.
-// TMEM (256 columns): S = Q K^T at [0,128) fp32; P = softmax numerators are
-// written back over S as packed bf16 (64 columns) and feed the PV MMA as the
-// TMEM A operand; O accumulates at [128, 128+d). Per chunk the MMA warp issues
-// S (SS MMA), waits for P, issues O += P V (TS MMA) and waits for it before
-// the next S overwrites P. Two CTAs share an SM (<100 KB smem, 256 TMEM
-// columns, <=168 registers each), so one CTA's softmax overlaps the other's
-// MMAs. O is rescaled in TMEM only when the running max grows by more than
-// 2^8 (exact: the final normalisation uses the same reference max).
+// One CTA per SM holds two query chunks (tiles 0 and 1: consecutive CSR rows,
+// so usually neighbours in the same head, whose key chunks share L2). Roles
+// (320 threads): warps 0-3 and 4-7 are the softmax + epilogue warpgroups of
+// tiles 0 and 1 (thread m of a group owns query row m = TMEM lane m); warp 8
+// is the TMA producer; warp 9 allocates TMEM and issues the MMAs.
+// TMEM (512 columns): S0, S1 = Q K^T fp32 at [0,128) and [128,256); the
+// softmax numerators P are written back over the first 64 columns of S as
+// packed bf16 and feed the PV MMA as its TMEM A operand; O0, O1 accumulate at
+// [256,384) and [384,512). The MMA warp alternates tiles (PV0, S0', PV1, S1'),
+// so one tile's softmax overlaps the other tile's MMAs. O is rescaled in TMEM
+// only when the running max grows by more than 2^8 (exact: the final
+// normalisation uses the same reference max).
 //
 // Every mbarrier wait is bounded; on expiry the CTA records a timeout in the
 // status word, drains its in-flight TMA and MMA work, frees TMEM and returns.
@@ -43,15 +45,19 @@ struct AttnCfg {
     static constexpr int kHalfBytes = 128 * 64 * 2;  // one TMA box: 128 tokens x 64 channels
     static constexpr int kHalves = D / 64;
     static constexpr int kTileBytes = kHalves * kHalfBytes;
-    static constexpr int kQ = 0;
-    static constexpr int kK = kTileBytes;
-    static constexpr int kV = 2 * kTileBytes;
-    static constexpr int kCtl = 3 * kTileBytes;
-    static constexpr int kSmemBytes = kCtl + 256 + 1024;  // + control block + alignment slack
-    static constexpr uint32_t kTmemCols = 256;
-    static constexpr uint32_t kSCol = 0;
-    static constexpr uint32_t kOCol = 128;
-    static constexpr int kThreads = 192;
+    // shared memory: Q0 Q1 K0 K1 V0 V1 (one buffer each per tile), control block
+    static constexpr int q_off(int t) { return t * kTileBytes; }
+    static constexpr int k_off(int t) { return (2 + t) * kTileBytes; }
+    static constexpr int v_off(int t) { return (4 + t) * kTileBytes; }
+    static constexpr int kCtl = 6 * kTileBytes;
+    static constexpr int kSmemBytes = kCtl + 512 + 1024;  // + control block + alignment slack
+    // tensor memory: S0 S1 (fp32 128x128; P is written over S as bf16) O0 O1
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t s_col(int t) { return t * 128; }
+    static constexpr uint32_t o_col(int t) { return 256 + t * 128; }
+    static constexpr int kThreads = 320;  // softmax WG0, softmax WG1, TMA warp, MMA warp
+    static constexpr int kTmaWarp = 8;
+    static constexpr int kMmaWarp = 9;
 };
 
 struct FwdArgs {
@@ -63,16 +69,24 @@ struct FwdArgs {
     uint32_t* status;
     int H, W, NH, NW, Nc;
     int64_t N;
+    int64_t rows;
     float scale_log2;  // softmax scale * log2(e)
     uint64_t timeout_ns;
-    int debug_flags;   // bit 0: withhold the first S-ready signal (timeout test)
+    int debug_flags;   // bit 0: withhold the first S-ready signal (timeout test);
+                       // bit 1: count finished CTAs in status[8]
+};
+
+struct __align__(8) TileBars {
+    uint64_t q_full, k_full, k_empty, v_full, v_empty, s_full, p_full, o_full;
 };
 
 struct __align__(8) Ctl {
-    uint64_t q_full, k_full, k_empty, v_full, v_empty, s_full, p_full, o_full, aux;
+    TileBars tb[2];
+    uint64_t aux;
+    int64_t beg[2], end[2];
+    int n_valid[2];
     uint32_t tmem_base;
     int abort_flag;
-    int n_valid;
 };
 
 // Wait used only while draining after an abort: ignores the abort flag.
@@ -101,8 +115,35 @@ __device__ __forceinline__ bool bar_red_and(int id, int nthreads, bool pred) {
     return r != 0;
 }
 
+__device__ __forceinline__ void chunk_origin(int c, int NH, int NW, int& t0, int& h0, int& w0) {
+    t0 = (c / (NH * NW)) * kChunkT;
+    h0 = ((c / NW) % NH) * kChunkH;
+    w0 = (c % NW) * kChunkW;
+}
+
+// Code of a wait site for the timeout record: role (1 TMA, 2 MMA, 3 softmax),
+// barrier, tile and key-chunk step.
+__device__ __forceinline__ uint32_t site(int role, int bar, int tile, int step) {
+    return static_cast<uint32_t>((role * 100 + bar * 10 + tile) * 10000 + (step < 9999 ? step : 9999));
+}
+
+// Next valid chunk index of a CSR row, starting at *e (advanced past it).
+__device__ __forceinline__ int next_chunk(const int32_t* col_idx, int64_t* e, int64_t end, int Nc) {
+    while (*e < end) {
+        const int c = col_idx[(*e)++];
+        if (c >= 0 && c < Nc) return c;
+    }
+    return -1;
+}
+
+// Two query chunks ("tiles" 0 and 1, CSR rows 2*blockIdx.x and 2*blockIdx.x+1)
+// per CTA, one CTA per SM. The MMA warp issues, per key-chunk step j,
+//   PV0(j), S0(j+1), PV1(j), S1(j+1)
+// so each tile's softmax runs while the tensor core works on the other tile.
+// S(j+1) is queued right behind the PV(j) that reads P from the same TMEM
+// columns: tcgen05 MMAs of one CTA execute in issue order.
 template <int D>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(320, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const FwdArgs a) {
@@ -111,51 +152,51 @@ __global__ void __launch_bounds__(192, 2)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     Ctl* ctl = reinterpret_cast<Ctl*>(smem + C::kCtl);
-    const uint32_t sQ = smem_u32(smem + C::kQ);
-    const uint32_t sK = smem_u32(smem + C::kK);
-    const uint32_t sV = smem_u32(smem + C::kV);
-
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t row = blockIdx.x;
-    const int64_t bh = row / a.Nc;
-    const int qc = static_cast<int>(row % a.Nc);
-    const int q_t = (qc / (a.NH * a.NW)) * kChunkT;
-    const int q_h = ((qc / a.NW) % a.NH) * kChunkH;
-    const int q_w = (qc % a.NW) * kChunkW;
-
-    // Row extent; an invalid row is treated as empty and reported.
-    int64_t beg = a.row_ptr[row], end = a.row_ptr[row + 1];
-    const bool row_ok = beg >= 0 && end >= beg && end <= a.col_cap && end - beg <= a.Nc;
-    if (!row_ok) beg = end = 0;
 
     if (threadIdx.x == 0) {
-        mbar_init(&ctl->q_full, 1);
-        mbar_init(&ctl->k_full, 1);
-        mbar_init(&ctl->k_empty, 1);
-        mbar_init(&ctl->v_full, 1);
-        mbar_init(&ctl->v_empty, 1);
-        mbar_init(&ctl->s_full, 1);
-        mbar_init(&ctl->p_full, 128);
-        mbar_init(&ctl->o_full, 1);
+        bool bad = false;
+        for (int t = 0; t < 2; ++t) {
+            TileBars& b = ctl->tb[t];
+            mbar_init(&b.q_full, 1);
+            mbar_init(&b.k_full, 1);
+            mbar_init(&b.k_empty, 1);
+            mbar_init(&b.v_full, 1);
+            mbar_init(&b.v_empty, 1);
+            mbar_init(&b.s_full, 1);
+            mbar_init(&b.p_full, 128);
+            mbar_init(&b.o_full, 1);
+            const int64_t row = 2 * static_cast<int64_t>(blockIdx.x) + t;
+            int64_t beg = 0, end = 0;
+            if (row < a.rows) {
+                beg = a.row_ptr[row];
+                end = a.row_ptr[row + 1];
+                if (!(beg >= 0 && end >= beg && end <= a.col_cap && end - beg <= a.Nc)) {
+                    bad = true;
+                    beg = end = 0;
+                }
+            }
+            int nv = 0;
+            for (int64_t e = beg; e < end; ++e) {
+                const int c = a.col_idx[e];
+                if (c >= 0 && c < a.Nc) ++nv; else bad = true;
+            }
+            ctl->beg[t] = beg;
+            ctl->end[t] = end;
+            ctl->n_valid[t] = nv;
+        }
         mbar_init(&ctl->aux, 1);
         ctl->abort_flag = 0;
-        int nv = 0;
-        bool bad = !row_ok;
-        for (int64_t e = beg; e < end; ++e) {
-            const int c = a.col_idx[e];
-            if (c >= 0 && c < a.Nc) ++nv; else bad = true;
-        }
-        ctl->n_valid = nv;
         if (bad) atomicOr(a.status, kStatusBadIndex);
         fence_mbar_init();
         fence_proxy_async_smem();
     }
-    if (warp == 5) {
+    if (warp == C::kMmaWarp) {
         tmem_alloc(&ctl->tmem_base, C::kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == C::kTmaWarp && lane == 0) {
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
@@ -165,92 +206,131 @@ __global__ void __launch_bounds__(192, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
-    const int n_valid = ctl->n_valid;
+    const int n0 = ctl->n_valid[0], n1 = ctl->n_valid[1];
+    const int nmax = n0 > n1 ? n0 : n1;
     volatile int* abort_flag = &ctl->abort_flag;
     const uint64_t tmo = a.timeout_ns;
 
-    if (warp == 4) {
+    if (warp == C::kTmaWarp) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0 && n_valid > 0) {
-            mbar_arrive_expect_tx(&ctl->q_full, C::kTileBytes);
+        if (lane == 0 && nmax > 0) {
+            const int n[2] = {n0, n1};
+            int64_t e[2] = {ctl->beg[0], ctl->beg[1]};
+            const int64_t end[2] = {ctl->end[0], ctl->end[1]};
+            int bh[2], ct[2], chh[2], cw[2];
+            for (int t = 0; t < 2; ++t) {
+                const int64_t row = 2 * static_cast<int64_t>(blockIdx.x) + t;
+                bh[t] = static_cast<int>(row / a.Nc);
+                if (n[t] == 0) continue;
+                chunk_origin(static_cast<int>(row % a.Nc), a.NH, a.NW, ct[t], chh[t], cw[t]);
+                mbar_arrive_expect_tx(&ctl->tb[t].q_full, C::kTileBytes);
 #pragma unroll
-            for (int h = 0; h < C::kHalves; ++h)
-                tma_load_5d(&tm_q, sQ + h * C::kHalfBytes, &ctl->q_full, h * 64, q_w, q_h, q_t,
-                            static_cast<int>(bh));
-            int nk = 0, nv = 0;
+                for (int h = 0; h < C::kHalves; ++h)
+                    tma_load_5d(&tm_q, smem_u32(smem + C::q_off(t)) + h * C::kHalfBytes,
+                                &ctl->tb[t].q_full, h * 64, cw[t], chh[t], ct[t], bh[t]);
+            }
+            int nk[2] = {0, 0}, nvv[2] = {0, 0};
+            int kt[2], kh[2], kw[2];
             bool aborted = false;
-            for (int64_t e = beg; e < end; ++e) {
-                const int c = a.col_idx[e];
-                if (c < 0 || c >= a.Nc) continue;
-                const int kt = (c / (a.NH * a.NW)) * kChunkT;
-                const int kh = ((c / a.NW) % a.NH) * kChunkH;
-                const int kw = (c % a.NW) * kChunkW;
-                if (nk > 0 && !mbar_wait(&ctl->k_empty, (nk - 1) & 1, abort_flag, a.status, tmo)) {
-                    aborted = true;
-                    break;
-                }
-                mbar_arrive_expect_tx(&ctl->k_full, C::kTileBytes);
+            for (int j = 0; j < nmax && !aborted; ++j) {
+                for (int t = 0; t < 2 && !aborted; ++t) {
+                    if (j >= n[t]) continue;
+                    const int c = next_chunk(a.col_idx, &e[t], end[t], a.Nc);
+                    chunk_origin(c, a.NH, a.NW, kt[t], kh[t], kw[t]);
+                    TileBars& b = ctl->tb[t];
+                    if (j > 0 && !mbar_wait(&b.k_empty, (j - 1) & 1, abort_flag, a.status, tmo, site(1, 1, t, j))) {
+                        aborted = true;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&b.k_full, C::kTileBytes);
 #pragma unroll
-                for (int h = 0; h < C::kHalves; ++h)
-                    tma_load_5d(&tm_k, sK + h * C::kHalfBytes, &ctl->k_full, h * 64, kw, kh, kt,
-                                static_cast<int>(bh));
-                ++nk;
-                if (nv > 0 && !mbar_wait(&ctl->v_empty, (nv - 1) & 1, abort_flag, a.status, tmo)) {
-                    aborted = true;
-                    break;
+                    for (int h = 0; h < C::kHalves; ++h)
+                        tma_load_5d(&tm_k, smem_u32(smem + C::k_off(t)) + h * C::kHalfBytes,
+                                    &b.k_full, h * 64, kw[t], kh[t], kt[t], bh[t]);
+                    ++nk[t];
                 }
-                mbar_arrive_expect_tx(&ctl->v_full, C::kTileBytes);
+                for (int t = 0; t < 2 && !aborted; ++t) {
+                    if (j >= n[t]) continue;
+                    TileBars& b = ctl->tb[t];
+                    if (j > 0 && !mbar_wait(&b.v_empty, (j - 1) & 1, abort_flag, a.status, tmo, site(1, 2, t, j))) {
+                        aborted = true;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&b.v_full, C::kTileBytes);
 #pragma unroll
-                for (int h = 0; h < C::kHalves; ++h)
-                    tma_load_5d(&tm_v, sV + h * C::kHalfBytes, &ctl->v_full, h * 64, kw, kh, kt,
-                                static_cast<int>(bh));
-                ++nv;
+                    for (int h = 0; h < C::kHalves; ++h)
+                        tma_load_5d(&tm_v, smem_u32(smem + C::v_off(t)) + h * C::kHalfBytes,
+                                    &b.v_full, h * 64, kw[t], kh[t], kt[t], bh[t]);
+                    ++nvv[t];
+                }
             }
             if (aborted || *abort_flag) {
                 // let the copies already issued land before shared memory is released
-                drain_wait(&ctl->q_full, 0, tmo);
-                if (nk > 0) drain_wait(&ctl->k_full, (nk - 1) & 1, tmo);
-                if (nv > 0) drain_wait(&ctl->v_full, (nv - 1) & 1, tmo);
+                for (int t = 0; t < 2; ++t) {
+                    if (n[t] == 0) continue;
+                    drain_wait(&ctl->tb[t].q_full, 0, tmo);
+                    if (nk[t] > 0) drain_wait(&ctl->tb[t].k_full, (nk[t] - 1) & 1, tmo);
+                    if (nvv[t] > 0) drain_wait(&ctl->tb[t].v_full, (nvv[t] - 1) & 1, tmo);
+                }
             }
         }
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == C::kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && n_valid > 0) {
+        if (lane == 0 && nmax > 0) {
             constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);  // Q, K both K-major
             constexpr uint32_t kIdO = idesc_bf16_f32(128, D, 0, 1);    // P from TMEM, V MN-major
-            const uint32_t tS = tmem + C::kSCol;
-            const uint32_t tO = tmem + C::kOCol;
-            bool aborted = !mbar_wait(&ctl->q_full, 0, abort_flag, a.status, tmo);
-            bool issued = false;
-            for (int it = 0; it < n_valid && !aborted; ++it) {
-                if (!mbar_wait(&ctl->k_full, it & 1, abort_flag, a.status, tmo)) { aborted = true; break; }
+            const int n[2] = {n0, n1};
+            bool aborted = false, issued = false;
+            for (int t = 0; t < 2 && !aborted; ++t)
+                if (n[t] > 0 && !mbar_wait(&ctl->tb[t].q_full, 0, abort_flag, a.status, tmo, site(2, 0, t, 0)))
+                    aborted = true;
+            auto issue_s = [&](int t, int j) -> bool {
+                TileBars& b = ctl->tb[t];
+                if (!mbar_wait(&b.k_full, j & 1, abort_flag, a.status, tmo, site(2, 1, t, j))) return false;
                 tc_fence_after();
+                const uint32_t sq = smem_u32(smem + C::q_off(t));
+                const uint32_t sk = smem_u32(smem + C::k_off(t));
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-                    mma_ss(tS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024),
-                           kIdS, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::s_col(t), sdesc_sw128(sq + off, 16, 1024),
+                           sdesc_sw128(sk + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
                 }
                 issued = true;
-                tc_commit(&ctl->k_empty);
-                if (!((a.debug_flags & 1) && it == 0)) tc_commit(&ctl->s_full);
-                if (!mbar_wait(&ctl->p_full, it & 1, abort_flag, a.status, tmo)) { aborted = true; break; }
+                tc_commit(&b.k_empty);
+                if (!((a.debug_flags & 1) && j == 0 && t == 0)) tc_commit(&b.s_full);
+                return true;
+            };
+            auto issue_pv = [&](int t, int j) -> bool {
+                TileBars& b = ctl->tb[t];
+                if (!mbar_wait(&b.p_full, j & 1, abort_flag, a.status, tmo, site(2, 3, t, j))) return false;
                 tc_fence_after();
-                if (!mbar_wait(&ctl->v_full, it & 1, abort_flag, a.status, tmo)) { aborted = true; break; }
+                if (!mbar_wait(&b.v_full, j & 1, abort_flag, a.status, tmo, site(2, 2, t, j))) return false;
                 tc_fence_after();
+                const uint32_t sv = smem_u32(smem + C::v_off(t));
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tO, tS + kk * 8, sdesc_sw128(sV + kk * 2048, C::kHalfBytes, 1024), kIdO,
-                           (it > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(&ctl->v_empty);
-                // P lives in the S columns: the next S may only start once PV has read it.
-                if (it + 1 < n_valid &&
-                    !mbar_wait(&ctl->v_empty, it & 1, abort_flag, a.status, tmo)) { aborted = true; break; }
+                    mma_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
+                           sdesc_sw128(sv + kk * 2048, C::kHalfBytes, 1024), kIdO,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&b.v_empty);
+                return true;
+            };
+            for (int t = 0; t < 2 && !aborted; ++t)
+                if (n[t] > 0 && !issue_s(t, 0)) aborted = true;
+            for (int j = 0; j < nmax && !aborted; ++j) {
+                for (int t = 0; t < 2 && !aborted; ++t) {
+                    if (j >= n[t]) continue;
+                    if (!issue_pv(t, j)) { aborted = true; break; }
+                    if (j + 1 < n[t]) {
+                        if (!issue_s(t, j + 1)) { aborted = true; break; }
+                    } else {
+                        tc_commit(&ctl->tb[t].o_full);
+                    }
+                }
             }
-            if (!aborted) {
-                tc_commit(&ctl->o_full);
-            } else if (issued) {
+            if (aborted && issued) {
                 tc_commit(&ctl->aux);
                 drain_wait(&ctl->aux, 0, tmo);
             }
@@ -258,35 +338,64 @@ __global__ void __launch_bounds__(192, 2)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        const int m = threadIdx.x;  // query row = TMEM lane
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t tS = tmem + lane_off + C::kSCol;
-        const uint32_t tO = tmem + lane_off + C::kOCol;
+        const int t = warp >> 2;                     // tile of this warpgroup
+        const int m = threadIdx.x & 127;             // query row = TMEM lane
+        const int n_t = t ? n1 : n0;
+        TileBars& b = ctl->tb[t];
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + C::s_col(t);
+        const uint32_t tO = tmem + lane_off + C::o_col(t);
         const float c2 = a.scale_log2;
-        float m_run = -INFINITY, l_run = 0.f;
+        float m_run = -INFINITY;
+        float2 l2 = make_float2(0.f, 0.f);
         bool ok = true;
-        for (int it = 0; it < n_valid; ++it) {
-            const bool got = mbar_wait(&ctl->s_full, it & 1, abort_flag, a.status, tmo);
+        for (int it = 0; it < n_t; ++it) {
+            const bool got = mbar_wait(&b.s_full, it & 1, abort_flag, a.status, tmo, site(3, 4, t, it));
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
-            float mx = -INFINITY;
+            uint32_t s[128];
+            tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(s + 0));
+            tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
+            tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(s + 64));
+            tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(s + 96));
+            tmem_wait_ld();
+            float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
+            float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                uint32_t s[32];
-                tmem_ld32(tS + g * 32, s);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(s[j]));
+            for (int j = 4; j < 128; j += 4) {
+                mx0 = fmaxf(mx0, __uint_as_float(s[j]));
+                mx1 = fmaxf(mx1, __uint_as_float(s[j + 1]));
+                mx2 = fmaxf(mx2, __uint_as_float(s[j + 2]));
+                mx3 = fmaxf(mx3, __uint_as_float(s[j + 3]));
             }
-            const float m_new = mx * c2;
-            if (it == 0) {
-                m_run = m_new;
-            } else if (m_new > m_run + 8.0f) {
-                // O holds the chunks before this one (their PV completed before S was
-                // signalled); rescale it to the new reference max.
-                const float alpha = ex2_approx(m_run - m_new);
-                l_run *= alpha;
+            const float m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c2;
+            // Lazy rescale: move the reference max only when it grows by > 2^8.
+            const bool rescale = it > 0 && m_new > m_run + 8.0f;
+            const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
+            if (it == 0 || rescale) m_run = m_new;
+            l2.x *= alpha;
+            l2.y *= alpha;
+            const float2 cc = make_float2(c2, c2);
+            const float2 nm = make_float2(-m_run, -m_run);
+            uint32_t pk[64];
 #pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                const float2 x = __ffma2_rn(
+                    make_float2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), cc, nm);
+                const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                l2 = __fadd2_rn(l2, pp);
+                pk[j] = pack_bf16x2(pp.x, pp.y);
+            }
+            // P over S columns [0, 64): every S value is already in registers
+            tmem_st32(tS + 0, *reinterpret_cast<const uint32_t(*)[32]>(pk + 0));
+            tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
+            // tcgen05.ld/st are warp-collective (.sync.aligned): the branch must be
+            // taken by the whole warp, each row scaling by its own alpha (1 if its
+            // reference max did not move).
+            if (__any_sync(0xffffffffu, rescale)) {
+                // O holds the chunks before this one (their PV completed before S was
+                // signalled, and the next PV waits for P): rescale it to the new max.
+#pragma unroll 1
                 for (int g = 0; g < D / 32; ++g) {
                     uint32_t o[32];
                     tmem_ld32(tO + g * 32, o);
@@ -295,84 +404,77 @@ __global__ void __launch_bounds__(192, 2)
                     for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
                     tmem_st32(tO + g * 32, o);
                 }
-                tmem_wait_st();
-                m_run = m_new;
-            }
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                uint32_t s[32];
-                tmem_ld32(tS + g * 32, s);
-                tmem_wait_ld();
-                uint32_t pk[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * j]), c2, -m_run));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * j + 1]), c2, -m_run));
-                    l_run += p0 + p1;
-                    pk[j] = pack_bf16x2(p0, p1);
-                }
-                tmem_st16(tS + g * 16, pk);  // P columns [16g, 16g+16) were read as S already
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&ctl->p_full);
+            mbar_arrive(&b.p_full);
         }
-        if (ok && n_valid > 0) {
-            const bool got = mbar_wait(&ctl->o_full, 0, abort_flag, a.status, tmo);
+        const float l_run = l2.x + l2.y;
+        if (ok && n_t > 0) {
+            const bool got = mbar_wait(&b.o_full, 0, abort_flag, a.status, tmo, site(3, 5, t, 0));
             ok = __all_sync(0xffffffffu, got);
         }
-        const bool all_ok = bar_red_and(1, 128, ok);
-        const int lt = m >> 5, lh = (m >> 3) & 3, lw = m & 7;
-        const int64_t tok = (static_cast<int64_t>(q_t + lt) * a.H + (q_h + lh)) * a.W + q_w + lw;
-        if (all_ok && n_valid > 0) {
-            tc_fence_after();
-            const float inv_l = 1.0f / l_run;
-            uint8_t* stage = smem + C::kQ;  // Q is dead once O is final
+        const bool all_ok = bar_red_and(1 + t, 128, ok);
+        const int64_t row = 2 * static_cast<int64_t>(blockIdx.x) + t;
+        if (row < a.rows) {
+            const int64_t bh = row / a.Nc;
+            int q_t, q_h, q_w;
+            chunk_origin(static_cast<int>(row % a.Nc), a.NH, a.NW, q_t, q_h, q_w);
+            const int lt = m >> 5, lh = (m >> 3) & 3, lw = m & 7;
+            const int64_t tok =
+                (static_cast<int64_t>(q_t + lt) * a.H + (q_h + lh)) * a.W + q_w + lw;
+            if (all_ok && n_t > 0) {
+                tc_fence_after();
+                const float inv_l = 1.0f / l_run;
+                uint8_t* stage = smem + C::q_off(t);  // Q of this tile is dead once O is final
 #pragma unroll
-            for (int g = 0; g < D / 32; ++g) {
-                uint32_t o[32];
-                tmem_ld32(tO + g * 32, o);
-                tmem_wait_ld();
-                const int half = (g * 32) / 64;
-                const int chunk0 = ((g * 32) % 64) / 8;
+                for (int g = 0; g < D / 32; ++g) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + g * 32, o);
+                    tmem_wait_ld();
+                    const int half = (g * 32) / 64;
+                    const int chunk0 = ((g * 32) % 64) / 8;
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint4 val;
-                    val.x = pack_bf16x2(__uint_as_float(o[c4 * 8 + 0]) * inv_l, __uint_as_float(o[c4 * 8 + 1]) * inv_l);
-                    val.y = pack_bf16x2(__uint_as_float(o[c4 * 8 + 2]) * inv_l, __uint_as_float(o[c4 * 8 + 3]) * inv_l);
-                    val.z = pack_bf16x2(__uint_as_float(o[c4 * 8 + 4]) * inv_l, __uint_as_float(o[c4 * 8 + 5]) * inv_l);
-                    val.w = pack_bf16x2(__uint_as_float(o[c4 * 8 + 6]) * inv_l, __uint_as_float(o[c4 * 8 + 7]) * inv_l);
-                    const int chunk = chunk0 + c4;
-                    *reinterpret_cast<uint4*>(stage + half * C::kHalfBytes + m * 128 +
-                                              ((chunk ^ (m & 7)) << 4)) = val;
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        uint4 val;
+                        val.x = pack_bf16x2(__uint_as_float(o[c4 * 8 + 0]) * inv_l, __uint_as_float(o[c4 * 8 + 1]) * inv_l);
+                        val.y = pack_bf16x2(__uint_as_float(o[c4 * 8 + 2]) * inv_l, __uint_as_float(o[c4 * 8 + 3]) * inv_l);
+                        val.z = pack_bf16x2(__uint_as_float(o[c4 * 8 + 4]) * inv_l, __uint_as_float(o[c4 * 8 + 5]) * inv_l);
+                        val.w = pack_bf16x2(__uint_as_float(o[c4 * 8 + 6]) * inv_l, __uint_as_float(o[c4 * 8 + 7]) * inv_l);
+                        const int chunk = chunk0 + c4;
+                        *reinterpret_cast<uint4*>(stage + half * C::kHalfBytes + m * 128 +
+                                                  ((chunk ^ (m & 7)) << 4)) = val;
+                    }
                 }
-            }
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (m == 0) {
+                fence_proxy_async_smem();
+                named_bar_sync(1 + t, 128);
+                if (m == 0) {
 #pragma unroll
-                for (int h = 0; h < C::kHalves; ++h)
-                    tma_store_5d(&tm_o, sQ + h * C::kHalfBytes, h * 64, q_w, q_h, q_t,
-                                 static_cast<int>(bh));
-                tma_store_commit_and_wait_all();
-            }
-            if (a.lse) a.lse[bh * a.N + tok] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
-        } else if (all_ok) {
-            // empty (or rejected) row: zeros, lse = -inf
-            uint4 z = make_uint4(0u, 0u, 0u, 0u);
-            uint4* dst = reinterpret_cast<uint4*>(a.out + (bh * a.N + tok) * D);
+                    for (int h = 0; h < C::kHalves; ++h)
+                        tma_store_5d(&tm_o, smem_u32(stage) + h * C::kHalfBytes, h * 64, q_w, q_h,
+                                     q_t, static_cast<int>(bh));
+                    tma_store_commit_and_wait_all();
+                }
+                if (a.lse)
+                    a.lse[bh * a.N + tok] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+            } else if (all_ok) {
+                // empty (or rejected) row: zeros, lse = -inf
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                uint4* dst = reinterpret_cast<uint4*>(a.out + (bh * a.N + tok) * D);
 #pragma unroll
-            for (int j = 0; j < D / 8; ++j) dst[j] = z;
-            if (a.lse) a.lse[bh * a.N + tok] = -INFINITY;
+                for (int j = 0; j < D / 8; ++j) dst[j] = z;
+                if (a.lse) a.lse[bh * a.N + tok] = -INFINITY;
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == C::kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
+    if ((a.debug_flags & 2) && threadIdx.x == 0) atomicAdd(a.status + 8, 1u);
 }
 
 // 5-D tiled map over a [BH][T][H][W][D] bf16 tensor with a (64,8,4,4,1) box and
@@ -426,7 +528,8 @@ cudaError_t launch_fwd_d(const Dims& g, const CUtensorMap& mq, const CUtensorMap
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    bsa_fwd_kernel<D><<<(unsigned)g.rows, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mo, args);
+    const unsigned grid = static_cast<unsigned>((g.rows + 1) / 2);
+    bsa_fwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mo, args);
     return cudaGetLastError();
 }
 
@@ -453,6 +556,7 @@ cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const vo
     args.NW = g.NW;
     args.Nc = g.Nc;
     args.N = g.N;
+    args.rows = g.rows;
     args.scale_log2 = g.scale * 1.4426950408889634f;
     args.timeout_ns = timeout_ns;
     args.debug_flags = debug_flags;

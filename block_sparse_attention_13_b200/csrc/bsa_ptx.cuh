@@ -62,10 +62,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait for phase `parity` of `bar` to complete. Gives up when *abort_flag is
 // set by another thread of the CTA, or after timeout_ns of global time, in
-// which case it sets *abort_flag and the timeout bit of the device status.
+// which case it sets *abort_flag and the timeout bit of the device status and
+// records where it gave up: status[1] counts expired waits; the first one
+// stores its site code, CTA index and parity in status[3..5].
 // Returns true when the phase completed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status, uint64_t timeout_ns) {
+                                          uint32_t* status, uint64_t timeout_ns, uint32_t site = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
@@ -74,6 +76,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         if (global_timer_ns() - t0 > timeout_ns) {
             *abort_flag = 1;
             atomicOr(status, kStatusTimeout);
+            atomicAdd(status + 1, 1u);
+            if (atomicCAS(status + 2, 0u, 1u) == 0u) {
+                status[3] = site;
+                status[4] = blockIdx.x;
+                status[5] = parity;
+            }
             return false;
         }
     }

@@ -68,8 +68,8 @@ def gather_rows(x_bhnd, wl, rows):
                      for r in rows])
 
 
-def check_case(wl, rows=None):
-    q, k, v = synth.make_qkv(wl)
+def check_case(wl, rows=None, qkv=None):
+    q, k, v = synth.make_qkv(wl) if qkv is None else qkv
     scale = 1.0 / math.sqrt(wl.d)
     rp, ci, out, lse, status = run_gpu(wl, q, k, v)
     assert status == bsa.BSA_OK, bsa.status_string(status)
@@ -95,6 +95,29 @@ def check_case(wl, rows=None):
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_small_cases_all_rows(name):
     check_case(SMALL[name])
+
+
+def _f32_to_bf16_bits(a):
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def test_long_rows_divergent_rescale():
+    """Rows of 180 chunks where K grows with the chunk index, so every query
+    row's running max jumps by more than 2^8 at its own chunk: the lazy O
+    rescale is needed by some rows of a warp and not by others."""
+    wl = W["tiny"].with_(name="long_rows", heads=2, T=16, H=32, W=56, d=128, topk=180)
+    q, k, v = synth.make_qkv(wl)
+    kf = synth.bf16_bits_to_f32(k).reshape(wl.B, wl.heads, wl.T // 4, 4, wl.H // 4, 4,
+                                           wl.W // 8, 8, wl.d).copy()
+    NH, NW = wl.H // 4, wl.W // 8
+    for ct in range(wl.T // 4):
+        for ch in range(NH):
+            for cw in range(NW):
+                c = (ct * NH + ch) * NW + cw
+                kf[:, :, ct, :, ch, :, cw] *= 0.5 + 4.0 * c / wl.Nc
+    k2 = _f32_to_bf16_bits(kf.reshape(k.shape))
+    check_case(wl, rows=np.arange(0, wl.rows, 19), qkv=(q, k2, v))
 
 
 def test_rearrange_bit_exact_and_inverse():
