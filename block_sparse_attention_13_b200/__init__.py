@@ -34,8 +34,8 @@ BSA_SEL_TOPK = 0
 BSA_SEL_CDF = 1
 
 EXPORTED = ("bsa_version", "bsa_status_string", "bsa_workspace_size", "bsa_plan_sizes",
-            "bsa_plan", "bsa_forward", "bsa_forward_ex", "bsa_read_status", "bsa_rearrange",
-            "bsa_pool", "bsa_scores", "bsa_selftest_timeout")
+            "bsa_plan", "bsa_plan_noalloc", "bsa_forward", "bsa_forward_ex", "bsa_read_status",
+            "bsa_rearrange", "bsa_pool", "bsa_scores", "bsa_selftest_timeout")
 
 
 class BsaError(RuntimeError):
@@ -86,6 +86,7 @@ def lib():
             "bsa_workspace_size": (sz, [P]),
             "bsa_plan_sizes": (i32, [P, ctypes.POINTER(i64), ctypes.POINTER(i64)]),
             "bsa_plan": (i32, [P, vp, vp, vp, sz, vp, vp, i64, vp]),
+            "bsa_plan_noalloc": (i32, [P, vp, vp, vp, vp, i64, vp]),
             "bsa_forward": (i32, [P, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, vp]),
             "bsa_forward_ex": (i32, [P, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, u64, i32, vp]),
             "bsa_read_status": (i32, [vp, vp]),
@@ -148,6 +149,14 @@ def bsa_plan(p, q, k, workspace, row_ptr, col_idx, stream=None):
     _check(lib().bsa_plan(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _ptr(row_ptr),
                           _ptr(col_idx), col_idx.numel(), _stream(stream)), "bsa_plan")
+
+
+def bsa_plan_noalloc(p, q, k, row_ptr, col_idx, stream=None):
+    """bsa_plan with the library's fixed scratch array instead of a workspace,
+    for callers that cannot allocate device memory (see include/bsa.h)."""
+    _check(lib().bsa_plan_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(row_ptr),
+                                  _ptr(col_idx), col_idx.numel(), _stream(stream)),
+           "bsa_plan_noalloc")
 
 
 def bsa_forward(p, q, k, v, row_ptr, col_idx, workspace, out, lse=None, stream=None):

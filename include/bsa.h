@@ -122,6 +122,33 @@ BSA_API int bsa_forward(const bsa_params* p, const void* q, const void* k, const
                 const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
                 void* workspace, size_t ws_bytes, void* out, float* lse, void* stream);
 
+/*
+ * bsa_plan without a caller workspace: the same selection as bsa_plan, with
+ * its scratch held in a fixed array inside this library, for callers that
+ * cannot allocate device memory (a plug-in whose host engine owns the memory
+ * budget and passes only input and output tensors, or a latency-critical
+ * caller that must not call cudaMalloc/cudaFree because they can synchronise
+ * the device). The paper has no counterpart; this is an interface convenience.
+ *   - Limit: 32 MiB of scratch (bsa_workspace_size(p) must not exceed it,
+ *     about the 480p-like grid with 32 heads); larger plans return
+ *     BSA_ERR_WORKSPACE_TOO_SMALL before any CUDA call. The array occupies
+ *     32 MiB on every GPU that loads this library's device code, until exit.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call reuses the same array, which keeps the previous call's
+ *     contents; the call clears the part that must start at zero. Calls whose
+ *     work overlaps on the GPU (e.g. on two streams without ordering) race on
+ *     the array: serialise them.
+ *   - Device-side errors are not kept for bsa_read_status (the status block
+ *     lives in the shared array); the one the plan can raise (CAPACITY) is
+ *     rejected on the host first.
+ * Arguments and other errors as for bsa_plan.
+ */
+BSA_API int bsa_plan_noalloc(const bsa_params* p, const void* q, const void* k, int32_t* row_ptr,
+                             int32_t* col_idx, int64_t col_capacity, void* stream);
+
 /* bsa_forward with an explicit limit for every device-side wait (timeout_ns;
  * 0 = the default of 2 s) and debug flags (bit 0: the MMA warp withholds its
  * first "scores ready" signal, so the softmax warps' bounded wait expires and
