@@ -229,6 +229,25 @@ def workload_config(wl, world):
                   f"{3 * wl.B * wl.heads * wl.N * wl.d * 2 / 1e9:.2f} GB)"}
 
 
+# ---------------------------------------------------------------------- ranks
+
+def shard_batch_offset(rank, wl):
+    """Batch index of this rank's first element: every rank runs its own
+    independent problem (weak scaling, no data exchange)."""
+    return rank * wl.B
+
+
+def reduce_over_ranks(value, op, world, device):
+    """MAX or SUM of a scalar over ranks (plumbing for the timing only)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------------- GPU leg
 
 def main():
@@ -260,21 +279,13 @@ def main():
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_over_ranks(x, "max", world, "cuda")
 
     def sum_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
+        return reduce_over_ranks(x, "sum", world, "cuda")
 
     # inputs: this rank's own problem (batch offset = rank), pinned host + device copies
-    q_np, k_np, v_np = synth.make_qkv(wl, batch_offset=rank * wl.B)
+    q_np, k_np, v_np = synth.make_qkv(wl, batch_offset=shard_batch_offset(rank, wl))
     host = [torch.from_numpy(a).view(torch.bfloat16).pin_memory() for a in (q_np, k_np, v_np)]
     q, k, v = (h.to("cuda", non_blocking=False) for h in host)
     p = bsa.params_for(wl)
