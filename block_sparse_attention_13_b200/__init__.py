@@ -35,7 +35,8 @@ BSA_SEL_CDF = 1
 
 EXPORTED = ("bsa_version", "bsa_status_string", "bsa_workspace_size", "bsa_plan_sizes",
             "bsa_plan", "bsa_plan_noalloc", "bsa_forward", "bsa_forward_ex", "bsa_read_status",
-            "bsa_rearrange", "bsa_pool", "bsa_scores", "bsa_selftest_timeout")
+            "bsa_rearrange", "bsa_pool", "bsa_scores", "bsa_selftest_exp2",
+            "bsa_selftest_timeout")
 
 
 class BsaError(RuntimeError):
@@ -93,6 +94,7 @@ def lib():
             "bsa_rearrange": (i32, [P, vp, vp, i32, vp]),
             "bsa_pool": (i32, [P, vp, vp, vp]),
             "bsa_scores": (i32, [P, vp, vp, vp, vp]),
+            "bsa_selftest_exp2": (i32, [vp, vp, vp, i64, vp]),
             "bsa_selftest_timeout": (i32, [vp, u64, vp]),
         }
         for name, (res, args) in sigs.items():
@@ -191,6 +193,11 @@ def bsa_pool(p, x, pooled, stream=None):
 def bsa_scores(p, qp, kp, S, stream=None):
     _check(lib().bsa_scores(ctypes.byref(p), _ptr(qp), _ptr(kp), _ptr(S), _stream(stream)),
            "bsa_scores")
+
+
+def bsa_selftest_exp2(x, y_poly, y_mufu, stream=None):
+    _check(lib().bsa_selftest_exp2(_ptr(x), _ptr(y_poly), _ptr(y_mufu), x.numel(),
+                                   _stream(stream)), "bsa_selftest_exp2")
 
 
 def bsa_selftest_timeout(workspace, timeout_ns, stream=None):

@@ -256,6 +256,13 @@ int bsa_scores(const bsa_params* p, const float* qp, const float* kp, float* S, 
     return cuda_status(launch_scores(g, qp, kp, S, static_cast<cudaStream_t>(stream)));
 }
 
+int bsa_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n, void* stream) {
+    if (!x || !y_poly || !y_mufu || n < 0 || (n & 1)) return BSA_ERR_INVALID_ARG;
+    const int rc = device_ok();
+    if (rc != BSA_OK) return rc;
+    return cuda_status(launch_exp2_selftest(x, y_poly, y_mufu, n, static_cast<cudaStream_t>(stream)));
+}
+
 int bsa_selftest_timeout(void* workspace, uint64_t timeout_ns, void* stream) {
     if (!workspace || timeout_ns == 0) return BSA_ERR_INVALID_ARG;
     if (!aligned16(workspace)) return BSA_ERR_ALIGNMENT;

@@ -40,6 +40,13 @@ namespace bsa {
 
 namespace {
 
+// Every kPolyEvery-th pair of softmax exponentials is evaluated by the FMA-pipe
+// polynomial instead of the MUFU unit (0 = all on MUFU).
+#ifndef BSA_POLY_EVERY
+#define BSA_POLY_EVERY 4
+#endif
+constexpr int kPolyEvery = BSA_POLY_EVERY;
+
 template <int D>
 struct AttnCfg {
     static constexpr int kHalfBytes = 128 * 64 * 2;  // one TMA box: 128 tokens x 64 channels
@@ -50,7 +57,9 @@ struct AttnCfg {
     static constexpr int k_off(int t) { return (2 + t) * kTileBytes; }
     static constexpr int v_off(int t) { return (4 + t) * kTileBytes; }
     static constexpr int kCtl = 6 * kTileBytes;
-    static constexpr int kSmemBytes = kCtl + 512 + 1024;  // + control block + alignment slack
+    static constexpr int kMaxChunks = 2048;                // Nc limit of the library
+    static constexpr int kList = kCtl + 512;               // uint16 chunk lists of both tiles
+    static constexpr int kSmemBytes = kList + 2 * kMaxChunks * 2 + 1024;  // + alignment slack
     // tensor memory: S0 S1 (fp32 128x128; P is written over S as bf16) O0 O1
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t s_col(int t) { return t * 128; }
@@ -83,7 +92,6 @@ struct __align__(8) TileBars {
 struct __align__(8) Ctl {
     TileBars tb[2];
     uint64_t aux;
-    int64_t beg[2], end[2];
     int n_valid[2];
     uint32_t tmem_base;
     int abort_flag;
@@ -127,15 +135,6 @@ __device__ __forceinline__ uint32_t site(int role, int bar, int tile, int step) 
     return static_cast<uint32_t>((role * 100 + bar * 10 + tile) * 10000 + (step < 9999 ? step : 9999));
 }
 
-// Next valid chunk index of a CSR row, starting at *e (advanced past it).
-__device__ __forceinline__ int next_chunk(const int32_t* col_idx, int64_t* e, int64_t end, int Nc) {
-    while (*e < end) {
-        const int c = col_idx[(*e)++];
-        if (c >= 0 && c < Nc) return c;
-    }
-    return -1;
-}
-
 // Two query chunks ("tiles" 0 and 1, CSR rows 2*blockIdx.x and 2*blockIdx.x+1)
 // per CTA, one CTA per SM. The MMA warp issues, per key-chunk step j,
 //   PV0(j), S0(j+1), PV1(j), S1(j+1)
@@ -155,8 +154,9 @@ __global__ void __launch_bounds__(320, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    uint16_t* lists = reinterpret_cast<uint16_t*>(smem + C::kList);  // [2][kMaxChunks]
+
     if (threadIdx.x == 0) {
-        bool bad = false;
         for (int t = 0; t < 2; ++t) {
             TileBars& b = ctl->tb[t];
             mbar_init(&b.q_full, 1);
@@ -167,6 +167,18 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(&b.s_full, 1);
             mbar_init(&b.p_full, 128);
             mbar_init(&b.o_full, 1);
+        }
+        mbar_init(&ctl->aux, 1);
+        ctl->abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == C::kTmaWarp) {
+        // Stage each tile's chunk list in shared memory (coalesced reads, out-of-range
+        // rows and columns dropped and reported), so no global load sits between a
+        // freed K/V buffer and the TMA load that refills it.
+        bool bad = false;
+        for (int t = 0; t < 2; ++t) {
             const int64_t row = 2 * static_cast<int64_t>(blockIdx.x) + t;
             int64_t beg = 0, end = 0;
             if (row < a.rows) {
@@ -177,30 +189,30 @@ __global__ void __launch_bounds__(320, 1)
                     beg = end = 0;
                 }
             }
-            int nv = 0;
-            for (int64_t e = beg; e < end; ++e) {
-                const int c = a.col_idx[e];
-                if (c >= 0 && c < a.Nc) ++nv; else bad = true;
+            int cnt = 0;
+            for (int64_t e0 = beg; e0 < end; e0 += 32) {
+                const int64_t e = e0 + lane;
+                const int c = e < end ? a.col_idx[e] : 0;
+                const bool valid = e < end && c >= 0 && c < a.Nc;
+                if (e < end && !valid) bad = true;
+                const uint32_t vb = __ballot_sync(0xffffffffu, valid);
+                if (valid) lists[t * C::kMaxChunks + cnt + __popc(vb & ((1u << lane) - 1u))] =
+                    static_cast<uint16_t>(c);
+                cnt += __popc(vb);
             }
-            ctl->beg[t] = beg;
-            ctl->end[t] = end;
-            ctl->n_valid[t] = nv;
+            if (lane == 0) ctl->n_valid[t] = cnt;
         }
-        mbar_init(&ctl->aux, 1);
-        ctl->abort_flag = 0;
-        if (bad) atomicOr(a.status, kStatusBadIndex);
-        fence_mbar_init();
-        fence_proxy_async_smem();
+        if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.status, kStatusBadIndex);
+        if (lane == 0) {
+            prefetch_tensormap(&tm_q);
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+            prefetch_tensormap(&tm_o);
+        }
     }
     if (warp == C::kMmaWarp) {
         tmem_alloc(&ctl->tmem_base, C::kTmemCols);
         tmem_relinquish();
-    }
-    if (warp == C::kTmaWarp && lane == 0) {
-        prefetch_tensormap(&tm_q);
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
-        prefetch_tensormap(&tm_o);
     }
     tc_fence_before();
     __syncthreads();
@@ -215,8 +227,6 @@ __global__ void __launch_bounds__(320, 1)
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && nmax > 0) {
             const int n[2] = {n0, n1};
-            int64_t e[2] = {ctl->beg[0], ctl->beg[1]};
-            const int64_t end[2] = {ctl->end[0], ctl->end[1]};
             int bh[2], ct[2], chh[2], cw[2];
             for (int t = 0; t < 2; ++t) {
                 const int64_t row = 2 * static_cast<int64_t>(blockIdx.x) + t;
@@ -229,41 +239,46 @@ __global__ void __launch_bounds__(320, 1)
                     tma_load_5d(&tm_q, smem_u32(smem + C::q_off(t)) + h * C::kHalfBytes,
                                 &ctl->tb[t].q_full, h * 64, cw[t], chh[t], ct[t], bh[t]);
             }
+            // The MMA warp frees buffers in the order PV0(j-1), S0(j), PV1(j-1), S1(j)
+            // (its issue order), so the loads go out in that order too: V0(j),
+            // K0(j+1), V1(j), K1(j+1). Each wait depends only on loads issued by
+            // earlier steps of this loop.
             int nk[2] = {0, 0}, nvv[2] = {0, 0};
-            int kt[2], kh[2], kw[2];
-            bool aborted = false;
-            for (int j = 0; j < nmax && !aborted; ++j) {
-                for (int t = 0; t < 2 && !aborted; ++t) {
-                    if (j >= n[t]) continue;
-                    const int c = next_chunk(a.col_idx, &e[t], end[t], a.Nc);
-                    chunk_origin(c, a.NH, a.NW, kt[t], kh[t], kw[t]);
-                    TileBars& b = ctl->tb[t];
-                    if (j > 0 && !mbar_wait(&b.k_empty, (j - 1) & 1, abort_flag, a.status, tmo, site(1, 1, t, j))) {
-                        aborted = true;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&b.k_full, C::kTileBytes);
+            auto load_k = [&](int t, int j) -> bool {
+                if (j >= n[t]) return true;
+                TileBars& b = ctl->tb[t];
+                if (j > 0 && !mbar_wait(&b.k_empty, (j - 1) & 1, abort_flag, a.status, tmo,
+                                        site(1, 1, t, j)))
+                    return false;
+                int kt, kh, kw;
+                chunk_origin(lists[t * C::kMaxChunks + j], a.NH, a.NW, kt, kh, kw);
+                mbar_arrive_expect_tx(&b.k_full, C::kTileBytes);
 #pragma unroll
-                    for (int h = 0; h < C::kHalves; ++h)
-                        tma_load_5d(&tm_k, smem_u32(smem + C::k_off(t)) + h * C::kHalfBytes,
-                                    &b.k_full, h * 64, kw[t], kh[t], kt[t], bh[t]);
-                    ++nk[t];
-                }
-                for (int t = 0; t < 2 && !aborted; ++t) {
-                    if (j >= n[t]) continue;
-                    TileBars& b = ctl->tb[t];
-                    if (j > 0 && !mbar_wait(&b.v_empty, (j - 1) & 1, abort_flag, a.status, tmo, site(1, 2, t, j))) {
-                        aborted = true;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&b.v_full, C::kTileBytes);
+                for (int h = 0; h < C::kHalves; ++h)
+                    tma_load_5d(&tm_k, smem_u32(smem + C::k_off(t)) + h * C::kHalfBytes, &b.k_full,
+                                h * 64, kw, kh, kt, bh[t]);
+                ++nk[t];
+                return true;
+            };
+            auto load_v = [&](int t, int j) -> bool {
+                if (j >= n[t]) return true;
+                TileBars& b = ctl->tb[t];
+                if (j > 0 && !mbar_wait(&b.v_empty, (j - 1) & 1, abort_flag, a.status, tmo,
+                                        site(1, 2, t, j)))
+                    return false;
+                int vt, vh, vw;
+                chunk_origin(lists[t * C::kMaxChunks + j], a.NH, a.NW, vt, vh, vw);
+                mbar_arrive_expect_tx(&b.v_full, C::kTileBytes);
 #pragma unroll
-                    for (int h = 0; h < C::kHalves; ++h)
-                        tma_load_5d(&tm_v, smem_u32(smem + C::v_off(t)) + h * C::kHalfBytes,
-                                    &b.v_full, h * 64, kw[t], kh[t], kt[t], bh[t]);
-                    ++nvv[t];
-                }
-            }
+                for (int h = 0; h < C::kHalves; ++h)
+                    tma_load_5d(&tm_v, smem_u32(smem + C::v_off(t)) + h * C::kHalfBytes, &b.v_full,
+                                h * 64, vw, vh, vt, bh[t]);
+                ++nvv[t];
+                return true;
+            };
+            bool aborted = !(load_k(0, 0) && load_k(1, 0));
+            for (int j = 0; j < nmax && !aborted; ++j)
+                aborted = !(load_v(0, j) && load_k(0, j + 1) && load_v(1, j) && load_k(1, j + 1));
             if (aborted || *abort_flag) {
                 // let the copies already issued land before shared memory is released
                 for (int t = 0; t < 2; ++t) {
@@ -347,7 +362,7 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t tO = tmem + lane_off + C::o_col(t);
         const float c2 = a.scale_log2;
         float m_run = -INFINITY;
-        float2 l2 = make_float2(0.f, 0.f);
+        float2 l2 = make_float2(0.f, 0.f), l2b = make_float2(0.f, 0.f);
         bool ok = true;
         for (int it = 0; it < n_t; ++it) {
             const bool got = mbar_wait(&b.s_full, it & 1, abort_flag, a.status, tmo, site(3, 4, t, it));
@@ -362,19 +377,21 @@ __global__ void __launch_bounds__(320, 1)
             float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
             float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
 #pragma unroll
-            for (int j = 4; j < 128; j += 4) {
-                mx0 = fmaxf(mx0, __uint_as_float(s[j]));
-                mx1 = fmaxf(mx1, __uint_as_float(s[j + 1]));
-                mx2 = fmaxf(mx2, __uint_as_float(s[j + 2]));
-                mx3 = fmaxf(mx3, __uint_as_float(s[j + 3]));
+            for (int j = 4; j < 128; j += 8) {
+                mx0 = fmax3(mx0, __uint_as_float(s[j]), __uint_as_float(s[j + 1]));
+                mx1 = fmax3(mx1, __uint_as_float(s[j + 2]), __uint_as_float(s[j + 3]));
+                mx2 = fmax3(mx2, __uint_as_float(s[j + 4]), __uint_as_float(s[j + 5]));
+                mx3 = fmax3(mx3, __uint_as_float(s[j + 6]), __uint_as_float(s[j + 7]));
             }
-            const float m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c2;
+            const float m_new = fmax3(fmaxf(mx0, mx1), mx2, mx3) * c2;
             // Lazy rescale: move the reference max only when it grows by > 2^8.
             const bool rescale = it > 0 && m_new > m_run + 8.0f;
             const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
             if (it == 0 || rescale) m_run = m_new;
             l2.x *= alpha;
             l2.y *= alpha;
+            l2b.x *= alpha;
+            l2b.y *= alpha;
             const float2 cc = make_float2(c2, c2);
             const float2 nm = make_float2(-m_run, -m_run);
             uint32_t pk[64];
@@ -382,8 +399,11 @@ __global__ void __launch_bounds__(320, 1)
             for (int j = 0; j < 64; ++j) {
                 const float2 x = __ffma2_rn(
                     make_float2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), cc, nm);
-                const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                l2 = __fadd2_rn(l2, pp);
+                // alternate pairs between the MUFU unit and the FMA-pipe polynomial
+                const float2 pp = (kPolyEvery > 0 && j % kPolyEvery == 0)
+                                      ? exp2_poly2(x)
+                                      : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                if (j & 1) l2b = __fadd2_rn(l2b, pp); else l2 = __fadd2_rn(l2, pp);
                 pk[j] = pack_bf16x2(pp.x, pp.y);
             }
             // P over S columns [0, 64): every S value is already in registers
@@ -409,7 +429,7 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_before();
             mbar_arrive(&b.p_full);
         }
-        const float l_run = l2.x + l2.y;
+        const float l_run = (l2.x + l2.y) + (l2b.x + l2b.y);
         if (ok && n_t > 0) {
             const bool got = mbar_wait(&b.o_full, 0, abort_flag, a.status, tmo, site(3, 5, t, 0));
             ok = __all_sync(0xffffffffu, got);
@@ -533,7 +553,28 @@ cudaError_t launch_fwd_d(const Dims& g, const CUtensorMap& mq, const CUtensorMap
     return cudaGetLastError();
 }
 
+__global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y_poly,
+                                     float* __restrict__ y_mufu, int64_t n) {
+    const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 2;
+    if (i + 1 < n) {
+        const float2 v = make_float2(x[i], x[i + 1]);
+        const float2 p = exp2_poly2(v);
+        y_poly[i] = p.x;
+        y_poly[i + 1] = p.y;
+        y_mufu[i] = ex2_approx(v.x);
+        y_mufu[i + 1] = ex2_approx(v.y);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, int64_t n,
+                                 cudaStream_t st) {
+    const int64_t pairs = n / 2;
+    if (pairs == 0) return cudaSuccess;
+    exp2_selftest_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, st>>>(x, y_poly, y_mufu, n);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const void* v,
                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,

@@ -47,6 +47,8 @@ cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const vo
                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
                            void* out, float* lse, uint32_t* status, uint64_t timeout_ns,
                            int debug_flags, cudaStream_t st);
+cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, int64_t n,
+                                 cudaStream_t st);
 cudaError_t launch_selftest_timeout(uint32_t* status, uint64_t timeout_ns, cudaStream_t st);
 
 // Default limit of every device-side wait (2 s of global time).

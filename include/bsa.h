@@ -181,6 +181,13 @@ BSA_API int bsa_pool(const bsa_params* p, const void* x, float* pooled, void* st
  * S = <qp_i, kp_m> * scale. The same kernel bsa_plan runs. */
 BSA_API int bsa_scores(const bsa_params* p, const float* qp, const float* kp, float* S, void* stream);
 
+/* Device self-test of the softmax exponentials: for n (even) floats x, writes
+ * the FMA-pipe polynomial 2^x that the forward kernel uses for part of the
+ * softmax numerators into y_poly, and the MUFU ex2.approx value into y_mufu.
+ * Device pointers. Used to check the polynomial against exact 2^x. */
+BSA_API int bsa_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n,
+                              void* stream);
+
 /* Device self-test of the bounded-wait machinery: launches one CTA that waits
  * on a barrier nothing arrives at, for at most timeout_ns, then records
  * DEVICE_TIMEOUT in the workspace status word and returns. The context stays
