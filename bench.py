@@ -37,7 +37,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "bsa_fwd_traffic.json")
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="720p")
     ap.add_argument("--heads", type=int, default=0,
@@ -90,7 +90,7 @@ def exec_flops(wl, nnz):
 class ClockSampler:
     """nvidia-smi clock/throttle samples during the timed region."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -120,7 +120,10 @@ class ClockSampler:
                 self.proc.kill()
             self.fh.close()
 
-    def summary(self):
+    def summary(self, t_begin=None, t_end=None):
+        """Median SM clock and throttle reasons over the samples taken between
+        host times t_begin and t_end (seconds since the epoch)."""
+        import datetime
         if self.proc is None or not os.path.exists(self.path):
             return None
         sm, mx, reasons = [], [], set()
@@ -128,14 +131,18 @@ class ClockSampler:
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    clk, cmax = float(parts[2]), float(parts[3])
                 except ValueError:
                     continue
-                for nm, val in zip(names, parts[5:9]):
+                if t_begin is not None and not (t_begin <= ts <= t_end):
+                    continue
+                sm.append(clk)
+                mx.append(cmax)
+                for nm, val in zip(names, parts[6:10]):
                     if val.lower() == "active":
                         reasons.add(nm)
         try:
@@ -313,6 +320,8 @@ def main():
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        time.sleep(0.5)  # let the sampler start before the timed region
+        host_t0 = time.time()
         t_start.record(stream)
         for s in range(args.steps):
             ev[s][0].record(stream)
@@ -322,8 +331,9 @@ def main():
             ev[s][2].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
+        host_t1 = time.time()
         barrier()
-    clocks = clk.summary()
+    clocks = clk.summary(host_t0, host_t1)
     total_ms = max_over_ranks(t_start.elapsed_time(t_end))
     plan_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
