@@ -120,6 +120,13 @@ def test_long_rows_divergent_rescale():
     check_case(wl, rows=np.arange(0, wl.rows, 19), qkv=(q, k2, v))
 
 
+def test_rows_longer_than_the_staged_chunk_list():
+    """Rows of 420 chunks: the forward kernel stages the first 384 chunk indices
+    of a row in shared memory and reads the rest from col_idx."""
+    wl = W["720p"].with_(name="long_rows_420", heads=1, topk=420)
+    check_case(wl, rows=np.arange(0, wl.rows, 97))
+
+
 def test_rearrange_bit_exact_and_inverse():
     for wl in (SMALL["ragged60_d64"], SMALL["ragged135_d128"]):
         q, _, _ = synth.make_qkv(wl)
