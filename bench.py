@@ -171,7 +171,7 @@ def cpu_oracle_sample(wl, q, k, v, target_s):
     t_plan_head = time.perf_counter() - t0
     # attention rows of head 0, grown until the sample takes ~target_s
     rng = np.random.default_rng(0)
-    order = rng.permutation(wl.Nc)
+    order = wl.q_skip + rng.permutation(wl.Nq)   # only the computed query chunks
     n, t_att, done = 4, 0.0, 0
     while True:
         rows = np.sort(order[done:done + n])
@@ -179,12 +179,13 @@ def cpu_oracle_sample(wl, q, k, v, target_s):
         oracle.attend(qh, kh, v[:1, :1], wl.T, wl.H, wl.W, scale, rp, ci, rows, want_lse=False)
         t_att += time.perf_counter() - t0
         done += len(rows)
-        if t_att + t_plan_head >= target_s or done >= wl.Nc:
+        if t_att + t_plan_head >= target_s or done >= wl.Nq:
             break
-        n = min(wl.Nc - done, max(4, int(n * 2)))
+        n = min(wl.Nq - done, max(4, int(n * 2)))
     sample_nnz = int(sum(rp[r + 1] - rp[r] for r in order[:done]))
     t_per_chunk_pair = t_att / max(sample_nnz, 1)
-    full_nnz = int(rp[-1]) * wl.B * wl.heads   # head 0's selection size as the estimate
+    # head 0's selection size over the computed rows as the estimate
+    full_nnz = int(rp[-1] - rp[wl.q_skip]) * wl.B * wl.heads
     t_full = t_plan_head * wl.B * wl.heads + t_per_chunk_pair * full_nnz
     value = exec_flops(wl, full_nnz) / t_full / 1e12
     return {
@@ -231,7 +232,7 @@ def workload_config(wl, world):
             "d": wl.d, "chunk_thw": [4, 4, 8], "mode": wl.mode,
             "topk": wl.topk if wl.mode == "topk" else None,
             "cdf_p": wl.cdf_p if wl.mode == "cdf" else None,
-            "t_cond": wl.t_cond, "parallelism": f"replicas{world}",
+            "t_cond": wl.t_cond, "q_begin": wl.q_begin, "parallelism": f"replicas{world}",
             "l2": "inputs larger than L2 (Q+K+V per step "
                   f"{3 * wl.B * wl.heads * wl.N * wl.d * 2 / 1e9:.2f} GB)"}
 
@@ -401,8 +402,9 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": workload_config(wl, world),
             "plan_ms": plan_ms, "fwd_ms": fwd_ms, "fwd_exec_tflops": fwd_tflops,
-            "nnz": nnz, "sparsity": 1.0 - nnz / (wl.B * wl.heads * wl.Nc * wl.Nc),
-            "dense_equiv_tflops": 4.0 * wl.B * wl.heads * wl.N * wl.N * wl.d / ms_per_step / 1e9,
+            "nnz": nnz, "sparsity": 1.0 - nnz / (wl.B * wl.heads * wl.Nq * wl.Nc),
+            "dense_equiv_tflops": 4.0 * wl.B * wl.heads * wl.Nq * 128 * wl.N * wl.d
+            / ms_per_step / 1e9,
             "dense": dense, "roofline": roofline, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

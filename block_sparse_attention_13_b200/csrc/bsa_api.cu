@@ -18,13 +18,12 @@ WsLayout ws_layout(const Dims& g, const bsa_params& p) {
     size_t off = 0;
     L.status = off;
     off += 256;
-    const size_t pool_bytes = round_up((size_t)g.BH * g.Nc * g.d * sizeof(float), 256);
     L.qpool = off;
-    off += pool_bytes;
+    off += round_up((size_t)g.BH * g.Nq * g.d * sizeof(float), 256);
     L.kpool = off;
-    off += pool_bytes;
+    off += round_up((size_t)g.BH * g.Nc * g.d * sizeof(float), 256);
     L.scores = off;
-    off += round_up((size_t)g.BH * g.Nc * g.Nc * sizeof(float), 256);
+    off += round_up((size_t)g.BH * g.Nq * g.Nc * sizeof(float), 256);
     L.pad_stride = 0;
     L.counts = L.padded = off;
     if (p.mode == BSA_SEL_CDF) {
@@ -51,6 +50,7 @@ static int make_dims(const bsa_params* p, Dims* g) {
     if (p->d != 64 && p->d != 128) return BSA_ERR_UNSUPPORTED;
     if (p->T % kChunkT || p->H % kChunkH || p->W % kChunkW) return BSA_ERR_SHAPE;
     if (p->t_cond < 0 || p->t_cond % kChunkT || p->t_cond > p->T) return BSA_ERR_SHAPE;
+    if (p->q_begin < 0 || p->q_begin % kChunkT || p->q_begin >= p->T) return BSA_ERR_SHAPE;
     if (!(std::isfinite(p->scale)) || p->scale < 0.f) return BSA_ERR_INVALID_ARG;
     if (p->mode == BSA_SEL_TOPK) {
         if (p->topk < 1) return BSA_ERR_INVALID_ARG;
@@ -77,23 +77,30 @@ static int make_dims(const bsa_params* p, Dims* g) {
     // and CSR offsets are int32.
     if (nc > 2048 || g->BH > 65535) return BSA_ERR_UNSUPPORTED;
     g->Nc = (int)nc;
-    g->rows = g->BH * g->Nc;
+    g->q_skip = (p->q_begin / kChunkT) * g->NH * g->NW;
+    g->Nq = g->Nc - g->q_skip;
+    g->rows = g->BH * g->Nq;
     if (g->rows * (int64_t)g->Nc > INT32_MAX) return BSA_ERR_UNSUPPORTED;
     g->n_cond = (p->t_cond / kChunkT) * g->NH * g->NW;
     g->scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt((float)p->d);
     return BSA_OK;
 }
 
+// Computed rows per (batch, head) that are condition rows (candidates: the
+// n_cond condition chunks) and noisy rows (candidates: all chunks).
+static int64_t cond_rows(const Dims& g) { return g.n_cond > g.q_skip ? g.n_cond - g.q_skip : 0; }
+static int64_t noisy_rows(const Dims& g) { return g.Nq - cond_rows(g); }
+
 static int64_t max_nnz_of(const Dims& g, const bsa_params& p) {
     if (p.mode == BSA_SEL_TOPK) {
         const int64_t kc = p.topk < g.n_cond ? p.topk : g.n_cond;
         const int64_t kn = p.topk < g.Nc ? p.topk : g.Nc;
-        return g.BH * ((int64_t)g.n_cond * kc + (int64_t)(g.Nc - g.n_cond) * kn);
+        return g.BH * (cond_rows(g) * kc + noisy_rows(g) * kn);
     }
     int64_t total = 0;
     for (int which = 0; which < 2; ++which) {
         const int na = which == 0 ? g.n_cond : g.Nc;
-        const int64_t nrows = which == 0 ? g.n_cond : g.Nc - g.n_cond;
+        const int64_t nrows = which == 0 ? cond_rows(g) : noisy_rows(g);
         if (nrows == 0) continue;
         int cap = (int)std::floor((double)p.cdf_cap_frac * na);
         if (cap < 1) cap = 1;

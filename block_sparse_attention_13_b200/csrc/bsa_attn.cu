@@ -77,6 +77,7 @@ struct FwdArgs {
     float* lse;
     uint32_t* status;
     int H, W, NH, NW, Nc;
+    int q_skip, Nq;    // CSR row r is query chunk q_skip + r % Nq of (batch, head) r / Nq
     int64_t N;
     int64_t rows;
     float scale_log2;  // softmax scale * log2(e)
@@ -230,9 +231,9 @@ __global__ void __launch_bounds__(320, 1)
             int bh[2], ct[2], chh[2], cw[2];
             for (int t = 0; t < 2; ++t) {
                 const int64_t row = 2 * static_cast<int64_t>(blockIdx.x) + t;
-                bh[t] = static_cast<int>(row / a.Nc);
+                bh[t] = static_cast<int>(row / a.Nq);
                 if (n[t] == 0) continue;
-                chunk_origin(static_cast<int>(row % a.Nc), a.NH, a.NW, ct[t], chh[t], cw[t]);
+                chunk_origin(a.q_skip + static_cast<int>(row % a.Nq), a.NH, a.NW, ct[t], chh[t], cw[t]);
                 mbar_arrive_expect_tx(&ctl->tb[t].q_full, C::kTileBytes);
 #pragma unroll
                 for (int h = 0; h < C::kHalves; ++h)
@@ -437,9 +438,9 @@ __global__ void __launch_bounds__(320, 1)
         const bool all_ok = bar_red_and(1 + t, 128, ok);
         const int64_t row = 2 * static_cast<int64_t>(blockIdx.x) + t;
         if (row < a.rows) {
-            const int64_t bh = row / a.Nc;
+            const int64_t bh = row / a.Nq;
             int q_t, q_h, q_w;
-            chunk_origin(static_cast<int>(row % a.Nc), a.NH, a.NW, q_t, q_h, q_w);
+            chunk_origin(a.q_skip + static_cast<int>(row % a.Nq), a.NH, a.NW, q_t, q_h, q_w);
             const int lt = m >> 5, lh = (m >> 3) & 3, lw = m & 7;
             const int64_t tok =
                 (static_cast<int64_t>(q_t + lt) * a.H + (q_h + lh)) * a.W + q_w + lw;
@@ -596,6 +597,8 @@ cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const vo
     args.NH = g.NH;
     args.NW = g.NW;
     args.Nc = g.Nc;
+    args.q_skip = g.q_skip;
+    args.Nq = g.Nq;
     args.N = g.N;
     args.rows = g.rows;
     args.scale_log2 = g.scale * 1.4426950408889634f;

@@ -16,6 +16,8 @@ struct Dims {
     int NT, NH, NW, Nc;
     int64_t N, BH, rows;
     int n_cond;      // condition chunks per (batch, head); 0 without block-causal mask
+    int q_skip;      // query chunks before q_begin (not computed)
+    int Nq;          // query chunks computed per (batch, head): Nc - q_skip
     float scale;
 };
 

@@ -37,12 +37,14 @@ __device__ __forceinline__ void add_bf16x2(float& a, float& b, uint32_t u) {
 // read consecutive 16-byte vectors, so every warp load is one contiguous
 // 512-byte run. Each thread always covers the same 8 channels and sums them
 // over its tokens in fp32; a shared-memory pass finishes the 128-token sum.
+// Tensor z (blockIdx.z) pools chunks [c_begin_z, c_begin_z + n_z) into rows
+// 0 .. n_z-1 of its output.
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ x0,
                                                    const __nv_bfloat16* __restrict__ x1,
                                                    float* __restrict__ p0, float* __restrict__ p1,
-                                                   int H, int W, int NH, int NW, int Nc,
-                                                   int64_t N) {
+                                                   int c_begin0, int n0, int c_begin1, int n1,
+                                                   int H, int W, int NH, int NW, int64_t N) {
     constexpr int VPT = D / 8;               // 16-byte vectors per token row
     constexpr int ITERS = 128 * VPT / 256;   // vectors per thread
     constexpr int GROUPS = 256 / VPT;        // threads that share one channel group
@@ -50,7 +52,9 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 
     const __nv_bfloat16* x = blockIdx.z ? x1 : x0;
     float* pooled = blockIdx.z ? p1 : p0;
-    const int c = blockIdx.x;
+    const int n_out = blockIdx.z ? n1 : n0;
+    if (static_cast<int>(blockIdx.x) >= n_out) return;
+    const int c = (blockIdx.z ? c_begin1 : c_begin0) + blockIdx.x;
     const int64_t bh = blockIdx.y;
     const int ct = c / (NH * NW), ch = (c / NW) % NH, cw = c % NW;
     const int tid = threadIdx.x;
@@ -81,7 +85,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
         float s = 0.f;
 #pragma unroll
         for (int g2 = 0; g2 < GROUPS; ++g2) s += red[g2][tid];
-        pooled[(bh * Nc + c) * D + tid] = s * (1.0f / kChunkTokens);
+        pooled[(bh * n_out + blockIdx.x) * D + tid] = s * (1.0f / kChunkTokens);
     }
 }
 
@@ -120,15 +124,15 @@ __global__ void __launch_bounds__(256) rearrange_kernel(const __nv_bfloat16* __r
 // transposed in shared memory 32 channels at a time.
 __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ qp,
                                                      const float* __restrict__ kp,
-                                                     float* __restrict__ S, int Nc, int D,
-                                                     float scale) {
+                                                     float* __restrict__ S, int Nq, int Nk,
+                                                     int D, float scale) {
     constexpr int BT = 64, BK = 32, LD = BT + 4;
     __shared__ __align__(16) float As[BK][LD];
     __shared__ __align__(16) float Bs[BK][LD];
     const int64_t bh = blockIdx.z;
     const int i0 = blockIdx.y * BT, m0 = blockIdx.x * BT;
-    const float* A = qp + bh * (int64_t)Nc * D;
-    const float* Bm = kp + bh * (int64_t)Nc * D;
+    const float* A = qp + bh * (int64_t)Nq * D;
+    const float* Bm = kp + bh * (int64_t)Nk * D;
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
     float acc[4][4];
 #pragma unroll
@@ -142,8 +146,8 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ q
             const int idx = tid + 256 * j;  // 512 float4 per 64x32 tile
             const int r = idx / (BK / 4), kq = idx % (BK / 4);
             float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
-            if (i0 + r < Nc) va = *reinterpret_cast<const float4*>(A + (int64_t)(i0 + r) * D + k0 + kq * 4);
-            if (m0 + r < Nc) vb = *reinterpret_cast<const float4*>(Bm + (int64_t)(m0 + r) * D + k0 + kq * 4);
+            if (i0 + r < Nq) va = *reinterpret_cast<const float4*>(A + (int64_t)(i0 + r) * D + k0 + kq * 4);
+            if (m0 + r < Nk) vb = *reinterpret_cast<const float4*>(Bm + (int64_t)(m0 + r) * D + k0 + kq * 4);
             As[kq * 4 + 0][r] = va.x; As[kq * 4 + 1][r] = va.y;
             As[kq * 4 + 2][r] = va.z; As[kq * 4 + 3][r] = va.w;
             Bs[kq * 4 + 0][r] = vb.x; Bs[kq * 4 + 1][r] = vb.y;
@@ -162,20 +166,20 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ q
         }
         __syncthreads();
     }
-    float* out = S + bh * (int64_t)Nc * Nc;
+    float* out = S + bh * (int64_t)Nq * Nk;
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
         const int i = i0 + ty * 4 + p;
-        if (i >= Nc) continue;
+        if (i >= Nq) continue;
         const int m = m0 + tx * 4;
-        float* o = out + (int64_t)i * Nc + m;
-        if ((Nc & 3) == 0 && m + 3 < Nc) {
+        float* o = out + (int64_t)i * Nk + m;
+        if ((Nk & 3) == 0 && m + 3 < Nk) {
             *reinterpret_cast<float4*>(o) = make_float4(acc[p][0] * scale, acc[p][1] * scale,
                                                         acc[p][2] * scale, acc[p][3] * scale);
         } else {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                if (m + q < Nc) o[q] = acc[p][q] * scale;
+                if (m + q < Nk) o[q] = acc[p][q] * scale;
         }
     }
 }
@@ -224,15 +228,16 @@ __device__ __forceinline__ uint32_t kth_largest_key(const uint32_t (&key)[MAXJ],
 
 template <int MAXJ>
 __global__ void __launch_bounds__(256) select_kernel(
-    const float* __restrict__ S, int Nc, int n_cond, int64_t rows, int mode, int topk,
+    const float* __restrict__ S, int Nc, int n_cond, int q_skip, int64_t rows, int mode, int topk,
     float cdf_p, float cap_frac, int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
     int64_t col_cap, int32_t* __restrict__ counts, int32_t* __restrict__ padded, int pad_stride,
     uint32_t* status) {
     const int lane = threadIdx.x & 31;
     const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (w >= rows) return;
-    const int64_t bh = w / Nc;
-    const int i = (int)(w % Nc);
+    const int Nq = Nc - q_skip;                 // computed query chunks per (batch, head)
+    const int64_t bh = w / Nq;
+    const int i = q_skip + (int)(w % Nq);       // query chunk of this row
     const int na = (n_cond > 0 && i < n_cond) ? n_cond : Nc;  // candidates are [0, na)
     const float* srow = S + w * (int64_t)Nc;
 
@@ -314,8 +319,12 @@ __global__ void __launch_bounds__(256) select_kernel(
     if (mode == BSA_SEL_TOPK) {
         const int kc = topk < n_cond ? topk : n_cond;
         const int kn = topk < Nc ? topk : Nc;
-        const int64_t per_bh = (int64_t)n_cond * kc + (int64_t)(Nc - n_cond) * kn;
-        off = bh * per_bh + (i < n_cond ? (int64_t)i * kc : (int64_t)n_cond * kc + (int64_t)(i - n_cond) * kn);
+        // rows of a (batch, head): condition rows q_skip .. n_cond-1, then noisy rows
+        const int c_rows = n_cond > q_skip ? n_cond - q_skip : 0;
+        const int first_noisy = n_cond > q_skip ? n_cond : q_skip;
+        const int64_t per_bh = (int64_t)c_rows * kc + (int64_t)(Nc - first_noisy) * kn;
+        off = bh * per_bh + (i < n_cond ? (int64_t)(i - q_skip) * kc
+                                        : (int64_t)c_rows * kc + (int64_t)(i - first_noisy) * kn);
         if (off + count > col_cap) {
             if (lane == 0) atomicOr(status, kStatusCapacity);
             return;
@@ -422,13 +431,18 @@ __global__ void selftest_timeout_kernel(uint32_t* status, uint64_t timeout_ns) {
 
 cudaError_t launch_pool(const Dims& g, const void* x0, const void* x1, float* p0, float* p1,
                         cudaStream_t st) {
+    // with two tensors (plan): x0 = Q pools the computed query chunks, x1 = K
+    // pools every chunk; with one tensor it pools every chunk of x0
     dim3 grid(g.Nc, (unsigned)g.BH, x1 ? 2 : 1);
     const auto* a = static_cast<const __nv_bfloat16*>(x0);
     const auto* b = static_cast<const __nv_bfloat16*>(x1 ? x1 : x0);
+    const int c0 = x1 ? g.q_skip : 0, n0 = x1 ? g.Nq : g.Nc;
     if (g.d == 128)
-        pool_kernel<128><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, g.H, g.W, g.NH, g.NW, g.Nc, g.N);
+        pool_kernel<128><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, c0, n0, 0, g.Nc, g.H, g.W,
+                                               g.NH, g.NW, g.N);
     else
-        pool_kernel<64><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, g.H, g.W, g.NH, g.NW, g.Nc, g.N);
+        pool_kernel<64><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, c0, n0, 0, g.Nc, g.H, g.W,
+                                              g.NH, g.NW, g.N);
     return cudaGetLastError();
 }
 
@@ -446,8 +460,8 @@ cudaError_t launch_rearrange(const Dims& g, const void* src, void* dst, int inve
 
 cudaError_t launch_scores(const Dims& g, const float* qp, const float* kp, float* S,
                           cudaStream_t st) {
-    dim3 grid((g.Nc + 63) / 64, (g.Nc + 63) / 64, (unsigned)g.BH);
-    scores_kernel<<<grid, 256, 0, st>>>(qp, kp, S, g.Nc, g.d, g.scale);
+    dim3 grid((g.Nc + 63) / 64, (g.Nq + 63) / 64, (unsigned)g.BH);
+    scores_kernel<<<grid, 256, 0, st>>>(qp, kp, S, g.Nq, g.Nc, g.d, g.scale);
     return cudaGetLastError();
 }
 
@@ -457,7 +471,7 @@ cudaError_t launch_select(const Dims& g, const bsa_params& p, const float* S, in
     const unsigned blocks = (unsigned)((g.rows + 7) / 8);
     const int mode = p.mode;
 #define BSA_SELECT(MJ)                                                                       \
-    select_kernel<MJ><<<blocks, 256, 0, st>>>(S, g.Nc, g.n_cond, g.rows, mode, p.topk,      \
+    select_kernel<MJ><<<blocks, 256, 0, st>>>(S, g.Nc, g.n_cond, g.q_skip, g.rows, mode, p.topk, \
                                               p.cdf_p, p.cdf_cap_frac, row_ptr, col_idx,    \
                                               col_cap, counts, padded, pad_stride, status)
     if (g.Nc <= 32) BSA_SELECT(1);

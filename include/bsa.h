@@ -66,6 +66,15 @@ typedef struct {
     float cdf_p;        /* CDF: cumulative pooled-softmax mass to reach, in (0,1]          */
     float cdf_cap_frac; /* CDF: at most max(1, floor(cap_frac*|A(i)|)) chunks, in (0,1]   */
     int32_t t_cond;     /* leading latent frames holding condition tokens; 0 = none; %4==0 */
+    int32_t q_begin;    /* first latent frame whose queries are computed; 0 = all; %4==0, < T.
+                         * Query chunks of earlier frames are neither read nor written and
+                         * get no CSR row: with q_begin = t_cond this is the KV-cached
+                         * video-continuation step of [P1] "Block Attention with KV-Cache":
+                         * only the noisy queries are evaluated, against the cached
+                         * condition K/V plus the noisy K/V, which stay in one
+                         * [B,heads,T*H*W,d] buffer. Row r of the CSR is query chunk
+                         * q_begin/4*(H/4)*(W/8) + r % Nq of (batch, head) r / Nq, where
+                         * Nq = Nc - q_begin/4*(H/4)*(W/8). */
 } bsa_params;
 
 /* Library version: major*10000 + minor*100 + patch. */
@@ -79,7 +88,8 @@ BSA_API const char* bsa_status_string(int status);
  * invalid. The same workspace serves both calls. */
 BSA_API size_t bsa_workspace_size(const bsa_params* p);
 
-/* CSR sizes for `p`: *n_rows = B*heads*Nc; *max_nnz = col_idx capacity that
+/* CSR sizes for `p`: *n_rows = B*heads*Nq (Nq = query chunks from q_begin on,
+ * Nc when q_begin = 0); *max_nnz = col_idx capacity that
  * always suffices (exact for TOPK; upper bound for CDF). Host-only call. */
 BSA_API int bsa_plan_sizes(const bsa_params* p, int64_t* n_rows, int64_t* max_nnz);
 
@@ -177,8 +187,9 @@ BSA_API int bsa_rearrange(const bsa_params* p, const void* x, void* out, int inv
 BSA_API int bsa_pool(const bsa_params* p, const void* x, float* pooled, void* stream);
 
 /* Pooled scores ([P1] S_pool = Q_pool K_pool^T / sqrt(d); [P3] gating-score
- * kernel): qp, kp fp32 [B,heads,Nc,d] -> S fp32 [B,heads,Nc,Nc] (device),
- * S = <qp_i, kp_m> * scale. The same kernel bsa_plan runs. */
+ * kernel): qp fp32 [B,heads,Nq,d], kp fp32 [B,heads,Nc,d] -> S fp32
+ * [B,heads,Nq,Nc] (device), S = <qp_i, kp_m> * scale (Nq = Nc when
+ * q_begin = 0). The same kernel bsa_plan runs. */
 BSA_API int bsa_scores(const bsa_params* p, const float* qp, const float* kp, float* S, void* stream);
 
 /* Device self-test of the softmax exponentials: for n (even) floats x, writes

@@ -25,6 +25,7 @@ class Workload:
     cdf_p: float = 0.9
     cdf_cap_frac: float = 0.25
     t_cond: int = 0             # latent frames of condition tokens (block-causal mask)
+    q_begin: int = 0            # first latent frame whose queries are computed (KV-cached step)
     tfreq_mult: float = 1.0     # temporal frequency multiplier of the smooth field
     seed: int = 0
     cond_seed: int = 1
@@ -43,8 +44,18 @@ class Workload:
         return (self.t_cond // 4) * (self.H // 4) * (self.W // 8)
 
     @property
+    def q_skip(self) -> int:
+        """Query chunks before q_begin (not computed)."""
+        return (self.q_begin // 4) * (self.H // 4) * (self.W // 8)
+
+    @property
+    def Nq(self) -> int:
+        """Query chunks computed per (batch, head)."""
+        return self.Nc - self.q_skip
+
+    @property
     def rows(self) -> int:
-        return self.B * self.heads * self.Nc
+        return self.B * self.heads * self.Nq
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -63,4 +74,8 @@ WORKLOADS = {
     # block-causal video continuation with CDF selection (p = 0.9, cap 25%)
     "causal_cdf": Workload("causal_cdf", B=2, heads=32, T=24, H=48, W=80, d=128,
                            mode="cdf", cdf_p=0.9, cdf_cap_frac=0.25, t_cond=8),
+    # the same video-continuation input at a later denoising step: the condition
+    # frames' K/V are cached, only the noisy queries (frames >= 8) are computed
+    "causal_cdf_kv": Workload("causal_cdf_kv", B=2, heads=32, T=24, H=48, W=80, d=128,
+                              mode="cdf", cdf_p=0.9, cdf_cap_frac=0.25, t_cond=8, q_begin=8),
 }

@@ -75,7 +75,23 @@ def test_plan_sizes_topk_and_cdf(L):
     assert (rc, nnz) == (0, 240 * 240 + 480 * 300)
 
 
+def test_plan_sizes_kv_cached_step(L):
+    # causal_cdf with only the noisy queries (frames >= 8): 480 of 720 rows per head
+    rc, rows, nnz = rc_sizes(P(B=2, heads=32, T=24, H=48, W=80, d=128, mode="cdf", t_cond=8,
+                               q_begin=8))
+    assert (rc, rows, nnz) == (0, 64 * 480, 64 * 480 * 180)
+    # q_begin inside the condition frames: 120 condition rows (k clamped to 240) + 480 noisy
+    rc, rows, nnz = rc_sizes(P(heads=1, T=24, H=48, W=80, d=128, topk=300, t_cond=8, q_begin=4))
+    assert (rc, rows, nnz) == (0, 600, 120 * 240 + 480 * 300)
+    p = P(heads=32, T=24, H=48, W=80, d=128, topk=45, q_begin=8)
+    assert bsa.bsa_workspace_size(p) == 256 + 32 * 480 * 128 * 4 + 32 * 720 * 128 * 4 + \
+        32 * 480 * 720 * 4
+
+
 @pytest.mark.parametrize("kw,code", [
+    (dict(q_begin=2), bsa.BSA_ERR_SHAPE),
+    (dict(q_begin=4), bsa.BSA_ERR_SHAPE),     # q_begin must leave at least one frame (T = 4)
+    (dict(q_begin=-4), bsa.BSA_ERR_SHAPE),
     (dict(T=6), bsa.BSA_ERR_SHAPE),
     (dict(H=6), bsa.BSA_ERR_SHAPE),
     (dict(W=12), bsa.BSA_ERR_SHAPE),

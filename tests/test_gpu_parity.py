@@ -127,6 +127,58 @@ def test_rows_longer_than_the_staged_chunk_list():
     check_case(wl, rows=np.arange(0, wl.rows, 97))
 
 
+@pytest.mark.parametrize("case", ["cdf_noisy_only", "topk_part_condition"])
+def test_kv_cached_step_equals_rows_of_the_full_computation(case):
+    """q_begin: only query chunks from frame q_begin on are computed (the
+    KV-cached video-continuation step). Their CSR rows and outputs must equal
+    those rows of the full block-causal computation; skipped queries are not
+    read (they hold NaN here) and their outputs are not written."""
+    if case == "cdf_noisy_only":
+        wl = SMALL["causal_cdf_small"].with_(q_begin=8)
+    else:
+        wl = SMALL["causal_topk"].with_(q_begin=4, topk=20)
+    full = wl.with_(q_begin=0)
+    q, k, v = synth.make_qkv(wl)
+    HW = wl.H * wl.W
+    q_nan = q.copy()
+    q_nan[:, :, : wl.q_begin * HW] = 0x7FC0          # bf16 NaN in the skipped query frames
+    p = bsa.params_for(wl)
+    pl = bsa.allocate(p)
+    qd, kd, vd = dev(q_nan), dev(k), dev(v)
+    bsa.bsa_plan(p, qd, kd, pl.workspace, pl.row_ptr, pl.col_idx)
+    out = torch.full_like(qd, 3.0)
+    lse = torch.full((wl.B, wl.heads, wl.N), 5.0, dtype=torch.float32, device="cuda")
+    bsa.bsa_forward(p, qd, kd, vd, pl.row_ptr, pl.col_idx, pl.workspace, out, lse)
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_OK
+    rp = pl.row_ptr.cpu().numpy()
+    ci = pl.col_idx[: int(rp[-1])].cpu().numpy()
+    assert len(rp) == wl.rows + 1
+    scale = 1.0 / math.sqrt(wl.d)
+    o_rp, o_ci, _ = oracle.plan(q, k, wl.T, wl.H, wl.W, scale, wl.mode, wl.topk, wl.cdf_p,
+                                wl.cdf_cap_frac, wl.t_cond, fp32=True)
+    # place the GPU's rows at their positions in the full plan (the oracle's rows elsewhere)
+    # and judge the selection with the same tie rules as the full computation
+    full_rows = np.array([(r // wl.Nq) * wl.Nc + wl.q_skip + r % wl.Nq for r in range(wl.rows)])
+    merged = rows_of(o_rp, o_ci)
+    for r, g in enumerate(rows_of(rp, ci)):
+        merged[full_rows[r]] = g
+    m_rp = np.concatenate([[0], np.cumsum([len(x) for x in merged])]).astype(np.int32)
+    m_ci = np.concatenate(merged).astype(np.int32)
+    S64 = oracle.scores(oracle.pool(q, wl.T, wl.H, wl.W), oracle.pool(k, wl.T, wl.H, wl.W), scale)
+    n_checked, n_diff = compare_csr(m_rp, m_ci, o_rp, o_ci, S64, wl.Nc, wl.n_cond, wl.mode,
+                                    wl.cdf_p, wl.cdf_cap_frac, rows=full_rows)
+    assert n_diff <= max(1, wl.rows // 100), f"{n_diff} of {wl.rows} rows differ (ties)"
+    o_out, o_lse = oracle.attend(q, k, v, wl.T, wl.H, wl.W, scale, m_rp, m_ci, full_rows)
+    g_out = gather_rows(host_f32(out), full, full_rows)
+    mx, mean = compare_attention(g_out, o_out)
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+    g_lse = gather_rows(lse.cpu().numpy()[..., None], full, full_rows)[..., 0]
+    np.testing.assert_allclose(g_lse, o_lse, rtol=0, atol=2e-3)
+    # skipped query frames: outputs untouched
+    assert torch.all(out[:, :, : wl.q_begin * HW] == 3.0)
+    assert torch.all(lse[:, :, : wl.q_begin * HW] == 5.0)
+
+
 def test_rearrange_bit_exact_and_inverse():
     for wl in (SMALL["ragged60_d64"], SMALL["ragged135_d128"]):
         q, _, _ = synth.make_qkv(wl)
