@@ -77,6 +77,9 @@ def _load():
             lib.oracle_dense.restype = i32
             lib.oracle_dense.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, dbl, i32, vp, i64,
                                          vp, vp]
+            lib.oracle_attend_bwd.restype = i32
+            lib.oracle_attend_bwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, dbl, vp, vp,
+                                              vp, i64, vp, vp, vp]
             lib.oracle_num_threads.restype = i32
             lib.oracle_num_threads.argtypes = []
             _lib = lib
@@ -173,6 +176,40 @@ def attend(q, k, v, T, H, W, scale, row_ptr, col_idx, rows, want_lse=True):
                                  rows.size, out.ctypes.data,
                                  lse.ctypes.data if lse is not None else None), "oracle_attend")
     return out, lse
+
+
+def _f64(a):
+    """bf16 bit patterns (uint16) widened exactly, or float arrays as float64."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return np.ascontiguousarray((a.astype(np.uint32) << 16).view(np.float32), dtype=np.float64)
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def attend_bwd(q, k, v, dout, T, H, W, scale, row_ptr, col_idx, rows):
+    """Gradients of ``attend`` for upstream gradient ``dout`` (same shape as q).
+
+    Inputs: bf16 bit patterns (uint16) or float arrays [B, heads, N, d].
+    Returns dq_rows [n, 128, d] for the listed CSR rows and dk, dv [B, heads, N, d]
+    holding the contributions of those rows (complete for every key chunk whose
+    selecting rows are all listed). float64 throughout.
+    """
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Hh, N, d = q.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    rp = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    ci = np.ascontiguousarray(col_idx, dtype=np.int32)
+    if ci.size == 0:
+        ci = np.zeros(1, dtype=np.int32)
+    dq = np.empty((rows.size, CN, d), dtype=np.float64)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    _check(_load().oracle_attend_bwd(q.ctypes.data, k.ctypes.data, v.ctypes.data,
+                                     dout.ctypes.data, B * Hh, T, H, W, d, float(scale),
+                                     rp.ctypes.data, ci.ctypes.data, rows.ctypes.data, rows.size,
+                                     dq.ctypes.data, dk.ctypes.data, dv.ctypes.data),
+           "oracle_attend_bwd")
+    return dq, dk, dv
 
 
 def dense(q, k, v, T, H, W, scale, qtok, t_cond=0, want_lse=True):

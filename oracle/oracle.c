@@ -373,6 +373,125 @@ int oracle_dense(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH
     return bad ? -1 : 0;
 }
 
+/*
+ * Gradients of the block-sparse attention of oracle_attend ([P1] "Block Sparse
+ * Attention (BSA)", sparse attention computation: O = softmax(QK^T/sqrt(d) with
+ * non-selected logits at -inf) V; [P3] section "开源实现" lists the backward
+ * kernels of the trainable BSA) for a scalar loss L whose gradient with
+ * respect to O is dout. For a query token q with keys J (every token of the
+ * chunks in its CSR row), written out by the chain rule through the softmax:
+ *   P[q,j]  = exp(s[q,j] - LSE[q]),   s[q,j] = scale * <q, k_j>
+ *   O[q]    = sum_j P[q,j] v_j
+ *   dV[j]  += P[q,j] dout[q]
+ *   dP[q,j] = <dout[q], v_j>
+ *   Dq      = <dout[q], O[q]>          (= sum_j P[q,j] dP[q,j])
+ *   dS[q,j] = P[q,j] (dP[q,j] - Dq)
+ *   dQ[q]   = scale * sum_j dS[q,j] k_j
+ *   dK[j]  += scale * dS[q,j] q
+ * Inputs are fp64 [BH][N][d] in THW token order (callers widen bf16 exactly),
+ * so the same routine serves finite-difference checks. The rows listed in
+ * rows[] (r = bh*Nc + i) are processed: dq_rows[n][l][:] receives dQ of local
+ * query l of rows[n]; dk and dv ([BH][N][d], zeroed by the caller) accumulate
+ * the contributions of those rows only (complete for a key chunk when every
+ * row that selects it is listed). A row with no selected chunk contributes
+ * nothing and has dQ = 0. All arithmetic in fp64.
+ */
+int oracle_attend_bwd(const double* q, const double* k, const double* v, const double* dout,
+                      int BH, int T, int H, int W, int d, double scale, const int32_t* row_ptr,
+                      const int32_t* col_idx, const int64_t* rows, int64_t n_rows,
+                      double* dq_rows, double* dk, double* dv) {
+    if (!q || !k || !v || !dout || !row_ptr || !col_idx || !rows || !dq_rows || !dk || !dv ||
+        BH <= 0 || d <= 0 || !grid_ok(T, H, W))
+        return -1;
+    const int64_t N = (int64_t)T * H * W, Nc = N / CN;
+    for (int64_t n = 0; n < n_rows; ++n)
+        if (rows[n] < 0 || rows[n] >= (int64_t)BH * Nc) return -1;
+    int64_t cap_keys = 0;
+    int64_t* ktok = NULL;  /* token index of each key of the row */
+    double* P = NULL;      /* [128][nk] softmax weights */
+    double* dS = NULL;     /* [128][nk] */
+    for (int64_t n = 0; n < n_rows; ++n) {
+        const int64_t r = rows[n];
+        const int64_t bh = r / Nc, i = r % Nc;
+        const int64_t beg = row_ptr[r], end = row_ptr[r + 1];
+        const int64_t nk = (end - beg) * CN;
+        double* dqr = dq_rows + n * CN * d;
+        if (nk <= 0) {
+            for (int64_t x = 0; x < (int64_t)CN * d; ++x) dqr[x] = 0.0;
+            continue;
+        }
+        if (nk > cap_keys) {
+            free(ktok); free(P); free(dS);
+            ktok = (int64_t*)malloc(sizeof(int64_t) * (size_t)nk);
+            P = (double*)malloc(sizeof(double) * (size_t)(CN * nk));
+            dS = (double*)malloc(sizeof(double) * (size_t)(CN * nk));
+            cap_keys = nk;
+        }
+        for (int64_t e = beg; e < end; ++e)
+            for (int l = 0; l < CN; ++l)
+                ktok[(e - beg) * CN + l] = bh * N + oracle_token_of(T, H, W, col_idx[e], l);
+        /* per query: softmax weights, O, D, dS and dQ */
+#pragma omp parallel for schedule(static)
+        for (int lq = 0; lq < CN; ++lq) {
+            const double* qr = q + (bh * N + oracle_token_of(T, H, W, i, lq)) * d;
+            const double* gr = dout + (bh * N + oracle_token_of(T, H, W, i, lq)) * d;
+            double* p = P + (int64_t)lq * nk;
+            double* ds = dS + (int64_t)lq * nk;
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < nk; ++j) {
+                const double* kr = k + ktok[j] * d;
+                double a = 0.0;
+                for (int x = 0; x < d; ++x) a += qr[x] * kr[x];
+                p[j] = a * scale;
+                if (p[j] > mx) mx = p[j];
+            }
+            double z = 0.0;
+            for (int64_t j = 0; j < nk; ++j) {
+                p[j] = exp(p[j] - mx);
+                z += p[j];
+            }
+            for (int64_t j = 0; j < nk; ++j) p[j] /= z;
+            /* D = <dout, O> with O = sum_j P v_j; dP[j] = <dout, v_j> kept in ds */
+            double D = 0.0;
+            for (int64_t j = 0; j < nk; ++j) {
+                const double* vr = v + ktok[j] * d;
+                double a = 0.0;
+                for (int x = 0; x < d; ++x) a += gr[x] * vr[x];
+                ds[j] = a;
+                D += p[j] * a;
+            }
+            double* dqq = dqr + (int64_t)lq * d;
+            for (int x = 0; x < d; ++x) dqq[x] = 0.0;
+            for (int64_t j = 0; j < nk; ++j) {
+                ds[j] = p[j] * (ds[j] - D);
+                const double* kr = k + ktok[j] * d;
+                for (int x = 0; x < d; ++x) dqq[x] += ds[j] * kr[x];
+            }
+            for (int x = 0; x < d; ++x) dqq[x] *= scale;
+        }
+        /* per key: dV and dK contributions of this row's queries (keys of one
+           row are distinct tokens, so the updates do not collide) */
+#pragma omp parallel for schedule(static)
+        for (int64_t j = 0; j < nk; ++j) {
+            double* dkr = dk + ktok[j] * d;
+            double* dvr = dv + ktok[j] * d;
+            for (int lq = 0; lq < CN; ++lq) {
+                const int64_t qt = bh * N + oracle_token_of(T, H, W, i, lq);
+                const double pw = P[(int64_t)lq * nk + j];
+                const double sw = dS[(int64_t)lq * nk + j] * scale;
+                const double* qr = q + qt * d;
+                const double* gr = dout + qt * d;
+                for (int x = 0; x < d; ++x) {
+                    dvr[x] += pw * gr[x];
+                    dkr[x] += sw * qr[x];
+                }
+            }
+        }
+    }
+    free(ktok); free(P); free(dS);
+    return 0;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     extern int omp_get_max_threads(void);

@@ -53,7 +53,7 @@ def _load():
     return _lib
 
 
-TENSOR_Q, TENSOR_K, TENSOR_V = 0, 1, 2
+TENSOR_Q, TENSOR_K, TENSOR_V, TENSOR_DO = 0, 1, 2, 3
 
 
 def field_bf16(B, heads, T, H, W, d, seed, tensor, rms_norm, tfreq_mult=1.0,
@@ -84,6 +84,15 @@ def make_qkv(wl: "Workload", seed: int | None = None, batch_offset: int = 0):
                    rms_norm=(tensor != TENSOR_V), tfreq_mult=wl.tfreq_mult,
                    cond_frames=wl.t_cond, cond_seed=wl.cond_seed, b_offset=batch_offset)
         for tensor in (TENSOR_Q, TENSOR_K, TENSOR_V))
+
+
+def make_dout(wl: "Workload", seed: int | None = None, batch_offset: int = 0):
+    """Upstream gradient dO for the backward (uint16 bf16 bits, [B, heads, N, d]):
+    a smooth field of its own stream, not normalised (like V)."""
+    s = wl.seed if seed is None else seed
+    return field_bf16(wl.B, wl.heads, wl.T, wl.H, wl.W, wl.d, s, TENSOR_DO, rms_norm=False,
+                      tfreq_mult=wl.tfreq_mult, cond_frames=wl.t_cond, cond_seed=wl.cond_seed,
+                      b_offset=batch_offset)
 
 
 def bf16_bits_to_f32(a: np.ndarray) -> np.ndarray:
