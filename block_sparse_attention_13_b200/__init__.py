@@ -36,7 +36,7 @@ BSA_SEL_CDF = 1
 EXPORTED = ("bsa_version", "bsa_status_string", "bsa_workspace_size", "bsa_plan_sizes",
             "bsa_plan", "bsa_plan_noalloc", "bsa_forward", "bsa_forward_ex", "bsa_read_status",
             "bsa_rearrange", "bsa_pool", "bsa_scores", "bsa_selftest_exp2",
-            "bsa_selftest_timeout")
+            "bsa_selftest_timeout", "bsa_backward_workspace_size", "bsa_backward")
 
 
 class BsaError(RuntimeError):
@@ -97,6 +97,9 @@ def lib():
             "bsa_scores": (i32, [P, vp, vp, vp, vp]),
             "bsa_selftest_exp2": (i32, [vp, vp, vp, i64, vp]),
             "bsa_selftest_timeout": (i32, [vp, u64, vp]),
+            "bsa_backward_workspace_size": (sz, [P]),
+            "bsa_backward": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, vp,
+                                   vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -178,6 +181,21 @@ def bsa_forward_ex(p, q, k, v, row_ptr, col_idx, workspace, out, lse=None, timeo
            "bsa_forward_ex")
 
 
+def bsa_backward_workspace_size(p: bsa_params) -> int:
+    n = lib().bsa_backward_workspace_size(ctypes.byref(p))
+    if n == 0:
+        raise BsaError(BSA_ERR_INVALID_ARG, "bsa_backward_workspace_size")
+    return n
+
+
+def bsa_backward(p, q, k, v, out, lse, dout, row_ptr, col_idx, workspace, dq, dk, dv,
+                 stream=None):
+    _check(lib().bsa_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                              _ptr(dout), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)), "bsa_backward")
+
+
 def bsa_read_status(workspace, stream=None) -> int:
     return lib().bsa_read_status(_ptr(workspace), _stream(stream))
 
@@ -237,6 +255,27 @@ def forward(pl: Plan, q, k, v, out=None, lse=None, stream=None):
     out = torch.empty_like(q) if out is None else out
     bsa_forward(pl.params, q, k, v, pl.row_ptr, pl.col_idx, pl.workspace, out, lse, stream)
     return out
+
+
+def backward_workspace(p: bsa_params, device="cuda"):
+    """Device workspace for bsa_backward (status block zeroed)."""
+    import torch
+    ws = torch.empty(bsa_backward_workspace_size(p), dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def backward(pl: Plan, q, k, v, out, lse, dout, workspace=None, dq=None, dk=None, dv=None,
+             stream=None):
+    """dq, dk, dv of forward(pl, q, k, v) for upstream gradient dout."""
+    import torch
+    workspace = backward_workspace(pl.params, q.device) if workspace is None else workspace
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    bsa_backward(pl.params, q, k, v, out, lse, dout, pl.row_ptr, pl.col_idx, workspace, dq, dk,
+                 dv, stream)
+    return dq, dk, dv, workspace
 
 
 def block_sparse_attention(q, k, v, topk=None, mode="topk", cdf_p=0.9, cdf_cap_frac=0.25,

@@ -218,6 +218,33 @@ int bsa_forward(const bsa_params* p, const void* q, const void* k, const void* v
                           lse, 0, 0, stream);
 }
 
+size_t bsa_backward_workspace_size(const bsa_params* p) {
+    Dims g;
+    if (make_dims(p, &g) != BSA_OK) return 0;
+    return bwd_layout(g).total;
+}
+
+int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* v,
+                 const void* out, const float* lse, const void* dout, const int32_t* row_ptr,
+                 const int32_t* col_idx, int64_t col_capacity, void* workspace, size_t ws_bytes,
+                 void* dq, void* dk, void* dv, void* stream) {
+    Dims g;
+    int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!q || !k || !v || !out || !lse || !dout || !row_ptr || !col_idx || !workspace || !dq ||
+        !dk || !dv || col_capacity < 0)
+        return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return BSA_ERR_ALIGNMENT;
+    if (ws_bytes < bwd_layout(g).total) return BSA_ERR_WORKSPACE_TOO_SMALL;
+    if ((rc = device_ok()) != BSA_OK) return rc;
+    return cuda_status(launch_backward(g, q, k, v, out, lse, dout, row_ptr, col_idx, col_capacity,
+                                       workspace, dq, dk, dv, kDefaultTimeoutNs,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 int bsa_read_status(void* workspace, void* stream) {
     if (!workspace) return BSA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

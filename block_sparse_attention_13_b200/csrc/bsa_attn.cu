@@ -98,44 +98,6 @@ struct __align__(8) Ctl {
     int abort_flag;
 };
 
-// Wait used only while draining after an abort: ignores the abort flag.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > timeout_ns) return;
-    }
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&h);
-}
-
-__device__ __forceinline__ bool bar_red_and(int id, int nthreads, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.and.pred p, %2, %3, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(r)
-        : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
-        : "memory");
-    return r != 0;
-}
-
-__device__ __forceinline__ void chunk_origin(int c, int NH, int NW, int& t0, int& h0, int& w0) {
-    t0 = (c / (NH * NW)) * kChunkT;
-    h0 = ((c / NW) % NH) * kChunkH;
-    w0 = (c % NW) * kChunkW;
-}
-
-// Code of a wait site for the timeout record: role (1 TMA, 2 MMA, 3 softmax),
-// barrier, tile and key-chunk step.
-__device__ __forceinline__ uint32_t site(int role, int bar, int tile, int step) {
-    return static_cast<uint32_t>((role * 100 + bar * 10 + tile) * 10000 + (step < 9999 ? step : 9999));
-}
-
 // Two query chunks ("tiles" 0 and 1, CSR rows 2*blockIdx.x and 2*blockIdx.x+1)
 // per CTA, one CTA per SM. The MMA warp issues, per key-chunk step j,
 //   PV0(j), S0(j+1), PV1(j), S1(j+1)
@@ -498,6 +460,8 @@ __global__ void __launch_bounds__(320, 1)
     if ((a.debug_flags & 2) && threadIdx.x == 0) atomicAdd(a.status + 8, 1u);
 }
 
+}  // namespace
+
 // 5-D tiled map over a [BH][T][H][W][D] bf16 tensor with a (64,8,4,4,1) box and
 // 128-byte swizzle: one box is 128 tokens of one chunk x 64 channels.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -505,7 +469,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn get_encode_fn() {
+static EncodeTiledFn get_encode_fn() {
     static EncodeTiledFn fn = nullptr;
     static bool tried = false;
     if (!tried) {
@@ -535,6 +499,8 @@ bool make_chunk_map(CUtensorMap* tm, const void* base, const Dims& g) {
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }
+
+namespace {
 
 template <int D>
 cudaError_t launch_fwd_d(const Dims& g, const CUtensorMap& mq, const CUtensorMap& mk,

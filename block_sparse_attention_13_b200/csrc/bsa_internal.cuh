@@ -1,5 +1,6 @@
 // Internal declarations shared by the library's translation units.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -9,6 +10,21 @@ namespace bsa {
 
 constexpr int kChunkT = 4, kChunkH = 4, kChunkW = 8;
 constexpr int kChunkTokens = kChunkT * kChunkH * kChunkW;  // 128
+
+// Token-space origin (t, h, w) of chunk c.
+__host__ __device__ __forceinline__ void chunk_origin(int c, int NH, int NW, int& t0, int& h0,
+                                                      int& w0) {
+    t0 = (c / (NH * NW)) * kChunkT;
+    h0 = ((c / NW) % NH) * kChunkH;
+    w0 = (c % NW) * kChunkW;
+}
+
+// Code of a wait site for the timeout record: role (1 TMA, 2 MMA, 3 softmax),
+// barrier, tile and step.
+__host__ __device__ __forceinline__ uint32_t site(int role, int bar, int tile, int step) {
+    return static_cast<uint32_t>((role * 100 + bar * 10 + tile) * 10000 +
+                                 (step < 9999 ? step : 9999));
+}
 
 // Derived sizes of one call.
 struct Dims {
@@ -35,6 +51,22 @@ struct WsLayout {
 
 WsLayout ws_layout(const Dims& g, const bsa_params& p);
 
+// Backward workspace layout (byte offsets).
+struct BwdLayout {
+    size_t status;   // uint32 status word (+ padding to 256)
+    size_t aux;      // float [BH][Nq][2][128]: LSE * log2(e), <dO, O>
+    size_t bitmap;   // uint32 [BH*Nc][words]: query rows per key chunk
+    size_t rawcnt;   // int32 [BH*Nc]: entries per key chunk (duplicate check)
+    size_t cnt;      // int32 [BH*Nc]: distinct rows per key chunk
+    size_t col_ptr;  // int32 [BH*Nc + 1]
+    size_t row_idx;  // int32 [idx_cap]
+    int words;       // ceil(Nq / 32)
+    int64_t idx_cap; // BH * Nq * Nc
+    size_t total;
+};
+
+BwdLayout bwd_layout(const Dims& g);
+
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_pool(const Dims& g, const void* x0, const void* x1, float* p0, float* p1,
                         cudaStream_t st);
@@ -49,6 +81,15 @@ cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const vo
                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
                            void* out, float* lse, uint32_t* status, uint64_t timeout_ns,
                            int debug_flags, cudaStream_t st);
+// 5-D TMA map over a [BH][T][H][W][d] bf16 tensor whose box is one (4,4,8)
+// chunk x 64 channels (128-byte swizzle). False if the driver call failed.
+bool make_chunk_map(CUtensorMap* tm, const void* base, const Dims& g);
+cudaError_t launch_scan_counts(const int32_t* counts, int64_t n, int32_t* ptr, cudaStream_t st);
+cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const void* v,
+                            const void* out, const float* lse, const void* dout,
+                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
+                            void* workspace, void* dq, void* dk, void* dv, uint64_t timeout_ns,
+                            cudaStream_t st);
 cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, int64_t n,
                                  cudaStream_t st);
 cudaError_t launch_selftest_timeout(uint32_t* status, uint64_t timeout_ns, cudaStream_t st);

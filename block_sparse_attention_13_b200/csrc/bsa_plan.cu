@@ -490,6 +490,11 @@ cudaError_t launch_select(const Dims& g, const bsa_params& p, const float* S, in
     return cudaGetLastError();
 }
 
+cudaError_t launch_scan_counts(const int32_t* counts, int64_t n, int32_t* ptr, cudaStream_t st) {
+    scan_counts_kernel<<<1, 1024, 0, st>>>(counts, n, ptr);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_selftest_timeout(uint32_t* status, uint64_t timeout_ns, cudaStream_t st) {
     selftest_timeout_kernel<<<1, 32, 0, st>>>(status, timeout_ns);
     return cudaGetLastError();

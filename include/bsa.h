@@ -133,6 +133,42 @@ BSA_API int bsa_forward(const bsa_params* p, const void* q, const void* k, const
                 void* workspace, size_t ws_bytes, void* out, float* lse, void* stream);
 
 /*
+ * Bytes of device workspace that bsa_backward needs for `p` (0 if `p` is
+ * invalid): a status block, LSE and <dO,O> per computed query token, and the
+ * column-major (CSC) copy of a block mask of at most one entry per (row, key
+ * chunk) pair. Host-only call.
+ */
+BSA_API size_t bsa_backward_workspace_size(const bsa_params* p);
+
+/*
+ * Gradients of bsa_forward for an upstream gradient dout ([P1] sparse
+ * attention O = softmax(QK^T*scale, non-selected positions at -inf) V; [P3]
+ * "开源实现": the trainable BSA's backward kernels and block-mask transpose).
+ * With P = exp(QK^T*scale - lse) over the selected keys and D = <dout, out>
+ * per query: dV = P^T dout, dS = P * (dout V^T - D), dQ = scale dS K,
+ * dK = scale dS^T Q, each summed over the chunks of the CSR only. The block
+ * selection itself has no gradient.
+ * q, k, v, out, dout: device bf16 [B,heads,N,d] (out and lse exactly as
+ * bsa_forward wrote them for the same CSR). lse: device fp32 [B,heads,N].
+ * dq, dk, dv: device bf16 [B,heads,N,d], written in [T,H,W] token order:
+ * every computed query chunk of dq (query chunks before q_begin are not
+ * written; an empty CSR row gives zeros) and every key chunk of dk and dv
+ * (zeros for a key chunk that no row selected). Results are deterministic
+ * (no atomic accumulation). row_ptr/col_idx/col_capacity: the CSR given to
+ * bsa_forward; rows or columns out of range, and a chunk listed twice in one
+ * row, are reported as DEVICE_BAD_INDEX by bsa_read_status(workspace) (the
+ * affected gradients are then not meaningful). workspace: device, >=
+ * bsa_backward_workspace_size(p), 16-byte aligned, owned by the caller; its
+ * first bytes are the status block that bsa_read_status reads. Errors:
+ * INVALID_ARG, SHAPE, UNSUPPORTED, ALIGNMENT, WORKSPACE_TOO_SMALL, CUDA.
+ */
+BSA_API int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* v,
+                         const void* out, const float* lse, const void* dout,
+                         const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
+                         void* workspace, size_t ws_bytes, void* dq, void* dk, void* dv,
+                         void* stream);
+
+/*
  * bsa_plan without a caller workspace: the same selection as bsa_plan, with
  * its scratch held in a fixed array inside this library, for callers that
  * cannot allocate device memory (a plug-in whose host engine owns the memory

@@ -164,6 +164,35 @@ def test_forward_host_checks_before_any_cuda_call(L):
     assert f(pp, *a, -1, vp(FAKE), 256, vp(FAKE), None, None) == bsa.BSA_ERR_INVALID_ARG
 
 
+def test_backward_workspace_size_layout(L):
+    p = P(heads=32, T=24, H=48, W=80, d=128, topk=45)
+    rows, cols, words = 32 * 720, 32 * 720, 23
+    r256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    expect = 256 + r256(rows * 256 * 4) + r256(cols * words * 4) + 2 * r256(cols * 4) + \
+        r256((cols + 1) * 4) + r256(rows * 720 * 4)
+    assert bsa.bsa_backward_workspace_size(p) == expect
+    assert bsa.lib().bsa_backward_workspace_size(ctypes.byref(P(T=6))) == 0
+
+
+def test_backward_host_checks_before_any_cuda_call(L):
+    p = P()
+    ws = bsa.bsa_backward_workspace_size(p)
+    f = L.bsa_backward
+    pp = ctypes.byref(p)
+    x = vp(FAKE)
+    # q, k, v, out, lse, dout, row_ptr, col_idx, cap, ws, ws_bytes, dq, dk, dv, stream
+    assert f(pp, x, x, x, x, None, x, x, x, 16, x, ws, x, x, x, None) == bsa.BSA_ERR_INVALID_ARG
+    assert f(pp, x, x, x, x, x, x, x, x, -1, x, ws, x, x, x, None) == bsa.BSA_ERR_INVALID_ARG
+    assert f(pp, x, x, x, x, x, x, x, x, 16, x, ws, x, vp(FAKE + 8), x, None) == \
+        bsa.BSA_ERR_ALIGNMENT
+    assert f(pp, x, x, x, x, vp(FAKE + 2), x, x, x, 16, x, ws, x, x, x, None) == \
+        bsa.BSA_ERR_ALIGNMENT
+    assert f(pp, x, x, x, x, x, x, x, x, 16, x, ws - 1, x, x, x, None) == \
+        bsa.BSA_ERR_WORKSPACE_TOO_SMALL
+    assert f(ctypes.byref(P(T=6)), x, x, x, x, x, x, x, x, 16, x, ws, x, x, x, None) == \
+        bsa.BSA_ERR_SHAPE
+
+
 def test_no_cpu_fallback_without_a_gpu(L):
     """With valid arguments and no usable GPU the call fails loudly."""
     import torch

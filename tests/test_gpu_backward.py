@@ -1,0 +1,202 @@
+"""GPU parity of the backward (dQ, dK, dV) against the fp64 oracle, through
+the C ABI. The oracle runs on the GPU's own CSR with its own exact forward
+(P, O, D in fp64); the GPU recomputes P from its bf16-path LSE and takes D
+from its bf16 output, so the bars below absorb bf16 rounding of P, dS and the
+outputs (relative to the gradients' own scale)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity import rows_of
+from test_gpu_parity import SMALL, W, dev, gather_rows, host_f32
+
+pytestmark = pytest.mark.gpu
+
+import block_sparse_attention_13_b200 as bsa  # noqa: E402
+
+# bars: max |gpu - ref| / max |ref| and mean |gpu - ref| / mean |ref|, per tensor
+BWD_MAX_REL = 2e-2
+BWD_MEAN_REL = 1e-2
+
+
+def rel_errors(g, o):
+    g = np.asarray(g, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    err = np.abs(g - o)
+    return float(err.max() / max(np.abs(o).max(), 1e-30)), \
+        float(err.mean() / max(np.abs(o).mean(), 1e-30))
+
+
+def gpu_fwd_bwd(wl, q, k, v, g, csr=None, sentinel=None):
+    """Plan (or the caller's CSR), forward with LSE, backward. Returns host
+    CSR, device out/lse/dq/dk/dv and the two status codes."""
+    p = bsa.params_for(wl)
+    qd, kd, vd, gd = dev(q), dev(k), dev(v), dev(g)
+    if csr is None:
+        pl = bsa.allocate(p)
+        bsa.bsa_plan(p, qd, kd, pl.workspace, pl.row_ptr, pl.col_idx)
+    else:
+        pl = bsa.allocate(p)
+        rp, ci = csr
+        pl.row_ptr.copy_(torch.from_numpy(np.asarray(rp, dtype=np.int32)))
+        pl.col_idx = torch.from_numpy(np.asarray(ci, dtype=np.int32).copy()).cuda() \
+            if len(ci) else torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(qd)
+    lse = torch.empty((wl.B, wl.heads, wl.N), dtype=torch.float32, device="cuda")
+    bsa.bsa_forward(p, qd, kd, vd, pl.row_ptr, pl.col_idx, pl.workspace, out, lse)
+    st_f = bsa.bsa_read_status(pl.workspace)
+    ws = bsa.backward_workspace(p)
+    fill = float("nan") if sentinel is None else sentinel
+    dq, dk, dv = (torch.full_like(qd, fill) for _ in range(3))
+    bsa.bsa_backward(p, qd, kd, vd, out, lse, gd, pl.row_ptr, pl.col_idx, ws, dq, dk, dv)
+    st_b = bsa.bsa_read_status(ws)
+    rp = pl.row_ptr.cpu().numpy()
+    ci = pl.col_idx[: int(rp[-1])].cpu().numpy()
+    return rp, ci, out, lse, dq, dk, dv, st_f, st_b
+
+
+def check_bwd(wl, csr=None):
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    scale = 1.0 / math.sqrt(wl.d)
+    rp, ci, out, lse, dq, dk, dv, st_f, st_b = gpu_fwd_bwd(wl, q, k, v, g, csr)
+    assert st_f == bsa.BSA_OK and st_b == bsa.BSA_OK, (st_f, st_b)
+    rows = np.arange(wl.rows)
+    o_dq, o_dk, o_dv = oracle.attend_bwd(q, k, v, g, wl.T, wl.H, wl.W, scale, rp, ci, rows)
+    errs = {
+        "dq": rel_errors(gather_rows(host_f32(dq), wl, rows), o_dq),
+        "dk": rel_errors(host_f32(dk), o_dk),
+        "dv": rel_errors(host_f32(dv), o_dv),
+    }
+    for name, (mx, mean) in errs.items():
+        assert mx <= BWD_MAX_REL and mean <= BWD_MEAN_REL, (name, errs)
+    return errs
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_backward_small_cases(name):
+    check_bwd(SMALL[name])
+
+
+def test_backward_all_chunks_selected():
+    wl = W["tiny"].with_(T=8, H=16, W=32, d=128, heads=2)
+    check_bwd(wl.with_(topk=wl.Nc))
+
+
+def test_backward_empty_rows_and_unselected_key_chunks():
+    """Caller CSR with empty rows and key chunks that no row selects: the dQ of
+    an empty row and the dK/dV of an unselected chunk are exact zeros."""
+    wl = W["tiny"].with_(T=8, H=16, W=32, d=64, heads=2)   # 32 chunks per head
+    rng = np.random.default_rng(3)
+    rows = []
+    for r in range(wl.rows):
+        if r % 7 == 3:
+            rows.append([])
+        else:
+            rows.append(sorted(rng.choice(np.arange(0, wl.Nc, 2), size=int(rng.integers(1, 6)),
+                                          replace=False)))   # odd chunks never selected
+    rp = np.concatenate([[0], np.cumsum([len(x) for x in rows])]).astype(np.int32)
+    ci = np.concatenate([np.asarray(x, dtype=np.int32) for x in rows])
+    check_bwd(wl, csr=(rp, ci))
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    _, _, _, _, dq, dk, dv, _, st_b = gpu_fwd_bwd(wl, q, k, v, g, csr=(rp, ci))
+    assert st_b == bsa.BSA_OK
+    for r in range(wl.rows):
+        if not rows[r]:
+            toks = oracle.chunk_tokens(wl.T, wl.H, wl.W, r % wl.Nc)
+            assert torch.all(dq.view(-1, wl.N, wl.d)[r // wl.Nc, toks] == 0)
+    for c in range(1, wl.Nc, 2):
+        toks = oracle.chunk_tokens(wl.T, wl.H, wl.W, c)
+        assert torch.all(dk.view(-1, wl.N, wl.d)[:, toks] == 0)
+        assert torch.all(dv.view(-1, wl.N, wl.d)[:, toks] == 0)
+
+
+def test_backward_duplicate_chunk_in_row_is_reported():
+    wl = W["tiny"].with_(T=8, H=16, W=32, d=64, heads=1)
+    rows = [[c, (c + 1) % wl.Nc] for c in range(wl.Nc)]
+    rows[5] = [2, 2, 9]                                        # duplicate entry
+    rp = np.concatenate([[0], np.cumsum([len(x) for x in rows])]).astype(np.int32)
+    ci = np.concatenate([np.asarray(x, dtype=np.int32) for x in rows])
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    *_, st_b = gpu_fwd_bwd(wl, q, k, v, g, csr=(rp, ci))
+    assert st_b == bsa.BSA_ERR_DEVICE_BAD_INDEX
+
+
+def test_backward_kv_cached_rows():
+    """q_begin: the backward of the computed rows only. dQ of skipped query
+    frames is not written; dK/dV hold the contributions of the computed rows."""
+    wl = SMALL["causal_cdf_small"].with_(q_begin=8)
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    scale = 1.0 / math.sqrt(wl.d)
+    rp, ci, out, lse, dq, dk, dv, st_f, st_b = gpu_fwd_bwd(wl, q, k, v, g, sentinel=7.0)
+    assert st_f == bsa.BSA_OK and st_b == bsa.BSA_OK
+    full = wl.with_(q_begin=0)
+    full_rows = np.array([(r // wl.Nq) * wl.Nc + wl.q_skip + r % wl.Nq for r in range(wl.rows)])
+    merged = [np.zeros(0, dtype=np.int32)] * (wl.B * wl.heads * wl.Nc)
+    for r, x in enumerate(rows_of(rp, ci)):
+        merged[full_rows[r]] = x
+    m_rp = np.concatenate([[0], np.cumsum([len(x) for x in merged])]).astype(np.int32)
+    m_ci = np.concatenate(merged).astype(np.int32)
+    o_dq, o_dk, o_dv = oracle.attend_bwd(q, k, v, g, wl.T, wl.H, wl.W, scale, m_rp, m_ci,
+                                         full_rows)
+    for name, (gx, ox) in {"dq": (gather_rows(host_f32(dq), full, full_rows), o_dq),
+                           "dk": (host_f32(dk), o_dk), "dv": (host_f32(dv), o_dv)}.items():
+        mx, mean = rel_errors(gx, ox)
+        assert mx <= BWD_MAX_REL and mean <= BWD_MEAN_REL, (name, mx, mean)
+    HW = wl.H * wl.W
+    assert torch.all(dq[:, :, : wl.q_begin * HW] == 7.0)
+
+
+def test_backward_deterministic():
+    wl = SMALL["ragged135_d128"]
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    a = gpu_fwd_bwd(wl, q, k, v, g)
+    b = gpu_fwd_bwd(wl, q, k, v, g)
+    for x, y in zip(a[4:7], b[4:7]):
+        assert torch.equal(x.view(torch.int16), y.view(torch.int16))
+
+
+def test_backward_full_size_720p_sampled():
+    """Full 720p grid, 32 heads, in the launch configuration of the benchmark:
+    dQ of sampled rows and dK/dV of sampled key chunks of (batch 0, head 0)
+    against the oracle, plus the invariants sum(dK) = 0 and sum(dV) = sum(dO)
+    per head (every row is non-empty under top-k)."""
+    wl = W["720p"]
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    scale = 1.0 / math.sqrt(wl.d)
+    rp, ci, out, lse, dq, dk, dv, st_f, st_b = gpu_fwd_bwd(wl, q, k, v, g)
+    assert st_f == bsa.BSA_OK and st_b == bsa.BSA_OK
+    # invariants on every head, from the GPU's bf16 gradients
+    dkf = dk.float().view(wl.heads, wl.N, wl.d)
+    dvf = dv.float().view(wl.heads, wl.N, wl.d)
+    gf = torch.from_numpy(synth.bf16_bits_to_f32(g)).cuda().view(wl.heads, wl.N, wl.d)
+    sk = dkf.sum(1).abs().max() / dkf.abs().sum(1).max()
+    sv = (dvf.sum(1) - gf.sum(1)).abs().max() / gf.abs().sum(1).max()
+    assert sk < 1e-3 and sv < 1e-3, (float(sk), float(sv))
+    # oracle on (batch 0, head 0)
+    q0, k0, v0, g0 = (x[:, :1] for x in (q, k, v, g))
+    rp0 = rp[: wl.Nc + 1]
+    ci0 = ci[: int(rp0[-1])]
+    rng = np.random.default_rng(11)
+    sample_rows = np.sort(rng.choice(wl.Nc, size=3, replace=False))
+    col = int(ci0[int(rng.integers(0, len(ci0)))])
+    col_rows = np.array([r for r in range(wl.Nc) if col in ci0[rp0[r]:rp0[r + 1]]])
+    rows = np.unique(np.concatenate([sample_rows, col_rows]))
+    w1 = wl.with_(heads=1)
+    o_dq, o_dk, o_dv = oracle.attend_bwd(q0, k0, v0, g0, wl.T, wl.H, wl.W, scale, rp0, ci0, rows)
+    sel = np.isin(rows, sample_rows)
+    mx, mean = rel_errors(gather_rows(host_f32(dq[:, :1]), w1, sample_rows), o_dq[sel])
+    assert mx <= BWD_MAX_REL and mean <= BWD_MEAN_REL, ("dq", mx, mean)
+    toks = oracle.chunk_tokens(wl.T, wl.H, wl.W, col)
+    for name, gx, ox in (("dk", dk, o_dk), ("dv", dv, o_dv)):
+        mx, mean = rel_errors(host_f32(gx[0, 0, toks]), ox[0, 0, toks])
+        assert mx <= BWD_MAX_REL and mean <= BWD_MEAN_REL, (name, col, mx, mean)
