@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time bsa_backward (dQ, dK, dV) on the same plan")
+    ap.add_argument("--bwd-steps", type=int, default=20)
     return ap.parse_args()
 
 
@@ -237,6 +240,51 @@ def workload_config(wl, world):
                   f"{3 * wl.B * wl.heads * wl.N * wl.d * 2 / 1e9:.2f} GB)"}
 
 
+# ---------------------------------------------------------------------- backward
+
+def time_backward(args, wl, p, pl, q, k, v, stream, peak_tf):
+    """bsa_backward on the plan of the timed forward: forward once with LSE,
+    then K timed backward calls (events on the launching stream). Algorithmic
+    FLOPs are the five products of the gradient (S, dP, dV, dS K, dS^T Q:
+    2.5x the forward's); the kernels execute seven (S and dP are recomputed
+    once for dQ and once for dK/dV)."""
+    import torch
+    import synth
+    import block_sparse_attention_13_b200 as bsa
+    g_np = synth.make_dout(wl, batch_offset=shard_batch_offset(
+        int(os.environ.get("RANK", "0")), wl))
+    dout = torch.from_numpy(g_np).view(torch.bfloat16).to("cuda")
+    out = torch.empty_like(q)
+    lse = torch.empty((wl.B, wl.heads, wl.N), dtype=torch.float32, device="cuda")
+    bsa.bsa_plan(p, q, k, pl.workspace, pl.row_ptr, pl.col_idx)
+    bsa.bsa_forward(p, q, k, v, pl.row_ptr, pl.col_idx, pl.workspace, out, lse)
+    ws = bsa.backward_workspace(p)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def bwd():
+        bsa.bsa_backward(p, q, k, v, out, lse, dout, pl.row_ptr, pl.col_idx, ws, dq, dk, dv)
+
+    for _ in range(max(3, args.warmup)):
+        bwd()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.bwd_steps)]
+    for a, b in evs:
+        a.record(stream)
+        bwd()
+        b.record(stream)
+    torch.cuda.synchronize()
+    rc = bsa.bsa_read_status(ws)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    nnz = int(pl.row_ptr[-1].item())
+    alg = 2.5 * exec_flops(wl, nnz)
+    executed = 3.5 * exec_flops(wl, nnz)
+    return {"bwd_ms": ms, "steps": args.bwd_steps, "algorithmic_flops": alg,
+            "executed_flops": executed, "alg_tflops": alg / ms / 1e9,
+            "exec_tflops": executed / ms / 1e9, "exec_frac": executed / ms / 1e9 / peak_tf,
+            "launches_per_call": 6, "device_status": bsa.status_string(rc)}
+
+
 # ---------------------------------------------------------------------- ranks
 
 def shard_batch_offset(rank, wl):
@@ -391,6 +439,10 @@ def main():
                 "kernel": "bsa_fwd_kernel", "peak_source": f"{peak_src} bf16 (burst)",
                 "algorithmic_flops_per_launch": flops}
 
+    bwd = None
+    if args.backward:
+        bwd = time_backward(args, wl, p, pl, q, k, v, stream, peak_tf)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(wl, q_np, k_np, v_np, args.cpu_seconds)
@@ -405,7 +457,7 @@ def main():
             "nnz": nnz, "sparsity": 1.0 - nnz / (wl.B * wl.heads * wl.Nq * wl.Nc),
             "dense_equiv_tflops": 4.0 * wl.B * wl.heads * wl.Nq * 128 * wl.N * wl.d
             / ms_per_step / 1e9,
-            "dense": dense, "roofline": roofline, "cpu_baseline": cpu,
+            "dense": dense, "roofline": roofline, "cpu_baseline": cpu, "backward": bwd,
             "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,

@@ -484,7 +484,7 @@ static EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-bool make_chunk_map(CUtensorMap* tm, const void* base, const Dims& g) {
+bool make_chunk_map(CUtensorMap* tm, const void* base, const Dims& g, int box_t) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[5] = {(cuuint64_t)g.d, (cuuint64_t)g.W, (cuuint64_t)g.H,
@@ -492,7 +492,7 @@ bool make_chunk_map(CUtensorMap* tm, const void* base, const Dims& g) {
     const cuuint64_t strides[4] = {(cuuint64_t)g.d * 2, (cuuint64_t)g.W * g.d * 2,
                                    (cuuint64_t)g.H * g.W * g.d * 2,
                                    (cuuint64_t)g.T * g.H * g.W * g.d * 2};
-    const cuuint32_t box[5] = {64, kChunkW, kChunkH, kChunkT, 1};
+    const cuuint32_t box[5] = {64, kChunkW, kChunkH, (cuuint32_t)box_t, 1};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

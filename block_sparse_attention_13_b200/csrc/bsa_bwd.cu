@@ -39,8 +39,10 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ prep
-// aux[bh][r][0][l] = LSE * log2(e), aux[bh][r][1][l] = <dO, O> for local query l
-// of computed query chunk r (chunk q_skip + r). One CTA per (r, bh).
+// Per computed query chunk r (chunk q_skip + r) of head bh, a 1 KB record in
+// two halves of 64 local queries: aux[bh][r][h][0..63] = LSE * log2(e) and
+// aux[bh][r][h][64..127] = <dO, O> of local queries 64h .. 64h+63. One CTA per
+// (r, bh).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                        const __nv_bfloat16* __restrict__ dout,
@@ -74,13 +76,13 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
         }
 #pragma unroll
         for (int off = VPT / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (dv == 0) dst[128 + l] = acc;
+        if (dv == 0) dst[(l >> 6) * 128 + 64 + (l & 63)] = acc;
     }
     if (tid < 128) {
         const int l = tid;
         const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
         const int64_t tok = (static_cast<int64_t>(ct + lt) * H + (ch + lh)) * W + cw + lw;
-        dst[l] = lse[bh * N + tok] * kLog2e;
+        dst[(l >> 6) * 128 + (l & 63)] = lse[bh * N + tok] * kLog2e;
     }
 }
 
@@ -172,9 +174,9 @@ struct BwdCfg {
     static constexpr int kHalves = D / 64;
     static constexpr int kTileBytes = kHalves * kHalfBytes;
     static constexpr int kMaxList = 2048;            // Nc limit of the library
-    static constexpr int kThreads = 192;             // 4 softmax warps, TMA warp, MMA warp
-    static constexpr int kTmaWarp = 4;
-    static constexpr int kMmaWarp = 5;
+    static constexpr int kThreads = 320;             // 8 softmax warps, TMA warp, MMA warp
+    static constexpr int kTmaWarp = 8;
+    static constexpr int kMmaWarp = 9;
     static constexpr uint32_t kTmemCols = 512;
     // both kernels: six tiles, then 2 KB of per-query-chunk aux, control, list
     static constexpr int kAux = 6 * kTileBytes;
@@ -190,7 +192,7 @@ struct BwdArgs {
     const int32_t* col_ptr;   // CSC (dK/dV kernel): local query rows per key chunk
     const int32_t* row_idx;
     int64_t idx_cap;
-    const float* aux;         // [BH][Nq][2][128]: LSE*log2(e), D
+    const float* aux;         // [BH][Nq][half][LSE*log2(e) x64 | D x64]
     __nv_bfloat16* dq;        // for zero rows / columns written without TMA
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
@@ -208,10 +210,11 @@ struct BwdArgs {
 // scaled by `mul`, rounded to bf16 and written as row m of a 128-byte-swizzled
 // [128][64]-per-half staging tile (the layout of the 5-D TMA box).
 template <int D>
-__device__ __forceinline__ void stage_tmem_rows(uint32_t t_row, uint8_t* stage, int m, float mul) {
+__device__ __forceinline__ void stage_tmem_rows(uint32_t t_row, uint8_t* stage, int m, float mul,
+                                                int g_begin = 0, int g_end = D / 32) {
     constexpr int kHalfBytes = 128 * 64 * 2;
-#pragma unroll
-    for (int g = 0; g < D / 32; ++g) {
+#pragma unroll 1
+    for (int g = g_begin; g < g_end; ++g) {
         uint32_t o[32];
         tmem_ld32(t_row + g * 32, o);
         tmem_wait_ld();
@@ -247,13 +250,17 @@ __device__ __forceinline__ float2 exp2_pair(float2 x, int j) {
 }
 
 // ------------------------------------------------------------------ dQ kernel
-// One CTA per CSR row (query chunk). Shared memory tiles: Q, dO, K[2], V[2].
-// TMEM: S slots at columns 0 and 128 (dS written over the first 64 columns of
-// its slot as packed bf16, the TMEM A operand of dQ += dS K), dP at 256, dQ at
-// 384. MMA issue order per step j: dP(j+1), dQ(j), S(j+2); S(j+1) was issued
-// one step earlier, so the exponentials of step j+1 need only wait for dP(j+1).
+// One CTA per CSR row (query chunk). Shared memory tiles: Q, dO, K[3], V.
+// TMEM: S slots at columns 0 and 128, dP at 256, dQ at 384. The 8 dS warps
+// split each row: warps w and w+4 share TMEM lanes 32(w%4).. and take key
+// columns [0,64) and [64,128); each writes its 32 columns of packed bf16 dS
+// over the first half of the S columns it has just read ([0,32) and [64,96)),
+// the TMEM A operand of dQ += dS K. MMA issue order per step j, once dS(j) is
+// written: dP(j+1), dQ(j), S(j+2); S(j+1) was issued a step earlier. Two
+// producer lanes keep the loads independent: lane 0 refills K slots (K(j+3)
+// after dQ(j)), lane 1 the V tile (V(j+1) after dP(j)).
 struct __align__(8) DqCtl {
-    uint64_t qd_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2];
+    uint64_t qd_full, k_full[3], k_empty[3], v_full, v_empty, s_full[2];
     uint64_t dp_full, ds_full, dq_full, aux;
     int n_valid;
     uint32_t tmem_base;
@@ -261,7 +268,7 @@ struct __align__(8) DqCtl {
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     bsa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                       const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
@@ -272,7 +279,7 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* sQ = smem;
     uint8_t* sdO = smem + C::kTileBytes;
     auto sK = [&](int s) { return smem + (2 + s) * C::kTileBytes; };
-    auto sV = [&](int s) { return smem + (4 + s) * C::kTileBytes; };
+    uint8_t* sV = smem + 5 * C::kTileBytes;
     DqCtl* ctl = reinterpret_cast<DqCtl*>(smem + C::kCtl);
     uint16_t* list = reinterpret_cast<uint16_t*>(smem + C::kList);
     const int warp = threadIdx.x >> 5;
@@ -281,15 +288,16 @@ __global__ void __launch_bounds__(192, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&ctl->qd_full, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < 3; ++s) {
             mbar_init(&ctl->k_full[s], 1);
             mbar_init(&ctl->k_empty[s], 1);
-            mbar_init(&ctl->v_full[s], 1);
-            mbar_init(&ctl->v_empty[s], 1);
-            mbar_init(&ctl->s_full[s], 1);
         }
+        mbar_init(&ctl->v_full, 1);
+        mbar_init(&ctl->v_empty, 1);
+        mbar_init(&ctl->s_full[0], 1);
+        mbar_init(&ctl->s_full[1], 1);
         mbar_init(&ctl->dp_full, 1);
-        mbar_init(&ctl->ds_full, 128);
+        mbar_init(&ctl->ds_full, 256);
         mbar_init(&ctl->dq_full, 1);
         mbar_init(&ctl->aux, 1);
         ctl->abort_flag = 0;
@@ -341,47 +349,60 @@ __global__ void __launch_bounds__(192, 1)
     chunk_origin(a.q_skip + r_local, a.NH, a.NW, q_t, q_h, q_w);
 
     if (warp == C::kTmaWarp) {
-        // ------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ TMA producers
         if (lane == 0 && n > 0) {
+            // Q, dO, then the K ring
             mbar_arrive_expect_tx(&ctl->qd_full, 2 * C::kTileBytes);
 #pragma unroll
-            for (int h = 0; h < C::kHalves; ++h) {
-                tma_load_5d(&tm_q, smem_u32(sQ) + h * C::kHalfBytes, &ctl->qd_full, h * 64, q_w,
+            for (int c = 0; c < C::kHalves; ++c) {
+                tma_load_5d(&tm_q, smem_u32(sQ) + c * C::kHalfBytes, &ctl->qd_full, c * 64, q_w,
                             q_h, q_t, bh);
-                tma_load_5d(&tm_do, smem_u32(sdO) + h * C::kHalfBytes, &ctl->qd_full, h * 64, q_w,
+                tma_load_5d(&tm_do, smem_u32(sdO) + c * C::kHalfBytes, &ctl->qd_full, c * 64, q_w,
                             q_h, q_t, bh);
             }
-            int nk[2] = {0, 0}, nv[2] = {0, 0};
-            auto load = [&](bool is_k, int j) -> bool {
-                if (j >= n) return true;
-                const int s = j & 1;
-                uint64_t* full = is_k ? &ctl->k_full[s] : &ctl->v_full[s];
-                uint64_t* empty = is_k ? &ctl->k_empty[s] : &ctl->v_empty[s];
-                if (j >= 2 && !mbar_wait(empty, ((j - 2) >> 1) & 1, abort_flag, a.status, tmo,
-                                         site(1, is_k ? 1 : 2, s, j)))
-                    return false;
+            int nk[3] = {0, 0, 0};
+            bool ok = true;
+            for (int j = 0; j < n && ok; ++j) {
+                const int s = j % 3;
+                if (j >= 3 && !mbar_wait(&ctl->k_empty[s], ((j - 3) / 3) & 1, abort_flag, a.status,
+                                         tmo, site(1, 1, s, j))) {
+                    ok = false;
+                    break;
+                }
                 int kt, kh, kw;
                 chunk_origin(list[j], a.NH, a.NW, kt, kh, kw);
-                mbar_arrive_expect_tx(full, C::kTileBytes);
-                const uint32_t dst = smem_u32(is_k ? sK(s) : sV(s));
+                mbar_arrive_expect_tx(&ctl->k_full[s], C::kTileBytes);
 #pragma unroll
-                for (int h = 0; h < C::kHalves; ++h)
-                    tma_load_5d(is_k ? &tm_k : &tm_v, dst + h * C::kHalfBytes, full, h * 64, kw, kh,
-                                kt, bh);
-                ++(is_k ? nk : nv)[s];
-                return true;
-            };
-            // consumption order: S(0) dP(0) S(1) | dP(j+1) dQ(j) S(j+2) ...; V(j) is
-            // freed by dP(j), K(j) by dQ(j)
-            bool ok = load(true, 0) && load(false, 0) && load(true, 1) && load(false, 1);
-            for (int j = 0; j + 2 < n && ok; ++j) ok = load(false, j + 2) && load(true, j + 2);
+                for (int c = 0; c < C::kHalves; ++c)
+                    tma_load_5d(&tm_k, smem_u32(sK(s)) + c * C::kHalfBytes, &ctl->k_full[s], c * 64,
+                                kw, kh, kt, bh);
+                ++nk[s];
+            }
             if (!ok || *abort_flag) {
                 drain_wait(&ctl->qd_full, 0, tmo);
-                for (int s = 0; s < 2; ++s) {
+                for (int s = 0; s < 3; ++s)
                     if (nk[s] > 0) drain_wait(&ctl->k_full[s], (nk[s] - 1) & 1, tmo);
-                    if (nv[s] > 0) drain_wait(&ctl->v_full[s], (nv[s] - 1) & 1, tmo);
-                }
             }
+        } else if (lane == 1 && n > 0) {
+            // the V tile: V(j) once dP(j-1) has read V(j-1)
+            int nv = 0;
+            bool ok = true;
+            for (int j = 0; j < n && ok; ++j) {
+                if (j >= 1 && !mbar_wait(&ctl->v_empty, (j - 1) & 1, abort_flag, a.status, tmo,
+                                         site(1, 2, 0, j))) {
+                    ok = false;
+                    break;
+                }
+                int vt, vh, vw;
+                chunk_origin(list[j], a.NH, a.NW, vt, vh, vw);
+                mbar_arrive_expect_tx(&ctl->v_full, C::kTileBytes);
+#pragma unroll
+                for (int c = 0; c < C::kHalves; ++c)
+                    tma_load_5d(&tm_v, smem_u32(sV) + c * C::kHalfBytes, &ctl->v_full, c * 64, vw, vh,
+                                vt, bh);
+                ++nv;
+            }
+            if ((!ok || *abort_flag) && nv > 0) drain_wait(&ctl->v_full, (nv - 1) & 1, tmo);
         }
         __syncwarp();
     } else if (warp == C::kMmaWarp) {
@@ -392,8 +413,7 @@ __global__ void __launch_bounds__(192, 1)
             bool issued = false;
             bool ok = mbar_wait(&ctl->qd_full, 0, abort_flag, a.status, tmo, site(2, 0, 0, 0));
             if (ok) tc_fence_after();
-            auto issue_ss = [&](uint32_t dcol, uint8_t* A, uint8_t* B) {
-                const uint32_t sa = smem_u32(A), sb = smem_u32(B);
+            auto issue_ss = [&](uint32_t dcol, uint32_t sa, uint32_t sb) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
@@ -402,32 +422,32 @@ __global__ void __launch_bounds__(192, 1)
                 }
             };
             auto issue_s = [&](int j) -> bool {
-                const int s = j & 1;
-                if (!mbar_wait(&ctl->k_full[s], (j >> 1) & 1, abort_flag, a.status, tmo, site(2, 1, s, j)))
+                const int s = j % 3, t = j & 1;
+                if (!mbar_wait(&ctl->k_full[s], (j / 3) & 1, abort_flag, a.status, tmo, site(2, 1, s, j)))
                     return false;
                 tc_fence_after();
-                issue_ss(128u * s, sQ, sK(s));
+                issue_ss(128u * t, smem_u32(sQ), smem_u32(sK(s)));
                 issued = true;
-                tc_commit(&ctl->s_full[s]);
+                tc_commit(&ctl->s_full[t]);
                 return true;
             };
             auto issue_dp = [&](int j) -> bool {
-                const int s = j & 1;
-                if (!mbar_wait(&ctl->v_full[s], (j >> 1) & 1, abort_flag, a.status, tmo, site(2, 2, s, j)))
+                if (!mbar_wait(&ctl->v_full, j & 1, abort_flag, a.status, tmo, site(2, 2, 0, j)))
                     return false;
                 tc_fence_after();
-                issue_ss(256u, sdO, sV(s));
+                issue_ss(256u, smem_u32(sdO), smem_u32(sV));
                 issued = true;
-                tc_commit(&ctl->v_empty[s]);
+                tc_commit(&ctl->v_empty);
                 tc_commit(&ctl->dp_full);
                 return true;
             };
+            // dQ += dS(j) K(j): keys 16kk.. of dS sit at column 64*(kk/4) + 8*(kk%4) of the S slot
             auto issue_dq = [&](int j) {
-                const int s = j & 1;
+                const int s = j % 3, t = j & 1;
                 const uint32_t sk = smem_u32(sK(s));
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + 384u, tmem + 128u * s + kk * 8,
+                    mma_ts(tmem + 384u, tmem + 128u * t + 64u * (kk >> 2) + 8u * (kk & 3),
                            sdesc_sw128(sk + kk * 2048, C::kHalfBytes, 1024), kIdQ,
                            (j > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(&ctl->k_empty[s]);
@@ -453,24 +473,27 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ dS + epilogue
-        const int m = threadIdx.x;  // query row = TMEM lane (warps 0-3)
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        const float* aux_row = a.aux + (static_cast<int64_t>(bh) * a.Nq + r_local) * 256;
-        const float lse2 = aux_row[m];
-        const float Dm = aux_row[128 + m];
+        const int grp = warp >> 2;                    // key columns [64*grp, 64*grp + 64)
+        const int m = (warp & 3) * 32 + lane;         // query row = TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const float* aux_row = a.aux + (static_cast<int64_t>(bh) * a.Nq + r_local) * 256 +
+                               (m >> 6) * 128 + (m & 63);
+        const float lse2 = aux_row[0];
+        const float Dm = aux_row[64];
         const float2 cc = make_float2(a.scale_log2, a.scale_log2);
         const float2 nl = make_float2(-lse2, -lse2);
+        const float2 nd = make_float2(-Dm, -Dm);
         bool ok = true;
         for (int j = 0; j < n; ++j) {
-            const int s = j & 1;
-            bool got = mbar_wait(&ctl->s_full[s], (j >> 1) & 1, abort_flag, a.status, tmo, site(3, 4, s, j));
+            const int t = j & 1;
+            bool got = mbar_wait(&ctl->s_full[t], (j >> 1) & 1, abort_flag, a.status, tmo, site(3, 4, t, j));
             got = got && mbar_wait(&ctl->dp_full, j & 1, abort_flag, a.status, tmo, site(3, 5, 0, j));
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t tS = tmem + lane_off + 128u * s;
-            const uint32_t tP = tmem + lane_off + 256u;
+            const uint32_t tS = tmem + lane_off + 128u * t + 64u * grp;
+            const uint32_t tP = tmem + lane_off + 256u + 64u * grp;
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
+            for (int g = 0; g < 2; ++g) {
                 uint32_t sv[32], pv[32];
                 tmem_ld32(tS + g * 32, sv);
                 tmem_ld32(tP + g * 32, pv);
@@ -481,12 +504,12 @@ __global__ void __launch_bounds__(192, 1)
                     const float2 x = __ffma2_rn(
                         make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), cc, nl);
                     const float2 p = exp2_pair(x, e);
-                    const float2 dp = make_float2(__uint_as_float(pv[2 * e]) - Dm,
-                                                  __uint_as_float(pv[2 * e + 1]) - Dm);
+                    const float2 dp = __fadd2_rn(
+                        make_float2(__uint_as_float(pv[2 * e]), __uint_as_float(pv[2 * e + 1])), nd);
                     const float2 ds = __fmul2_rn(p, dp);
                     pk[e] = pack_bf16x2(ds.x, ds.y);
                 }
-                // dS over S columns [16g, 16g+16): those S values are already read
+                // dS over this warp's S columns [16g, 16g+16): already read
                 tmem_st16(tS + g * 16, pk);
             }
             tmem_wait_st();
@@ -497,19 +520,20 @@ __global__ void __launch_bounds__(192, 1)
             const bool got = mbar_wait(&ctl->dq_full, 0, abort_flag, a.status, tmo, site(3, 6, 0, 0));
             ok = __all_sync(0xffffffffu, got);
         }
-        const bool all_ok = bar_red_and(1, 128, ok);
+        const bool all_ok = bar_red_and(1, 256, ok);
         if (all_ok && n > 0) {
             tc_fence_after();
-            stage_tmem_rows<D>(tmem + lane_off + 384u, sQ, m, a.scale);  // Q is dead: all MMAs done
+            // Q is dead once every MMA has completed; each warp group stages half the columns
+            stage_tmem_rows<D>(tmem + lane_off + 384u, sQ, m, a.scale, grp * D / 64, (grp + 1) * D / 64);
             fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (m == 0) {
+            named_bar_sync(1, 256);
+            if (threadIdx.x == 0) {
 #pragma unroll
-                for (int h = 0; h < C::kHalves; ++h)
-                    tma_store_5d(&tm_dq, smem_u32(sQ) + h * C::kHalfBytes, h * 64, q_w, q_h, q_t, bh);
+                for (int c = 0; c < C::kHalves; ++c)
+                    tma_store_5d(&tm_dq, smem_u32(sQ) + c * C::kHalfBytes, c * 64, q_w, q_h, q_t, bh);
                 tma_store_commit_and_wait_all();
             }
-        } else if (all_ok) {
+        } else if (all_ok && grp == 0) {
             zero_token<D>(a.dq, bh, a.N, a.H, a.W, q_t, q_h, q_w, m);  // no selected chunk
         }
     }
@@ -524,28 +548,33 @@ __global__ void __launch_bounds__(192, 1)
 
 // ------------------------------------------------------------------ dK/dV kernel
 // One CTA per key chunk (CSC column). Shared memory tiles: K, V (this key
-// chunk), Q[2], dO[2] (query chunks of the column, double-buffered), and the
-// 1 KB aux record of each buffered query chunk. Thread m of the softmax warps
-// owns key row m. TMEM: S^T = K Q^T and dP^T = V dO^T in two halves of 64
-// queries (S^T half h at column 64h, dP^T half h at 128 + 64h; P^T and dS^T
-// are written back over the first 32 columns of their half as packed bf16),
-// dV accumulates at 256, dK at 384. MMA issue order per step i:
-//   dV,dK(i,a)  S^T,dP^T(i+1,a)  dV,dK(i,b)  S^T,dP^T(i+1,b)
+// chunk) and Q[2], dO[2] (query chunks of the column, double-buffered), each
+// query chunk loaded in two halves of 64 queries (its frames 0-1 and 2-3)
+// together with the matching half of its aux record; a half is released as
+// soon as its last MMA has run. TMEM: S^T = K Q^T and dP^T = V dO^T per half
+// (S^T half h at column 64h, dP^T half h at 128 + 64h), dV accumulates at 256,
+// dK at 384. The 8 softmax warps split each half: warps w and w+4 share TMEM
+// lanes 32(w%4).. (key rows) and take its query columns [0,32) and [32,64),
+// writing packed bf16 P^T / dS^T over the first 16 of the columns they read
+// (the TMEM A operands of dV += P^T dO and dK += dS^T Q).
+// MMA issue order per step i:
+//   dV,dK(i,h0)  S^T,dP^T(i+1,h0)  dV,dK(i,h1)  S^T,dP^T(i+1,h1)
 // so the exponentials of one half run while the tensor core works on the other.
 struct __align__(8) DkvCtl {
-    uint64_t kv_full, qd_full[2], qd_empty[2], sd_full[2], p_full[2], dkv_full, aux;
+    uint64_t kv_full, qd_full[2][2], qd_empty[2][2], sd_full[2], p_full[2], dkv_full, aux;
     int n_valid;
     uint32_t tmem_base;
     int abort_flag;
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
-    bsa_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+__global__ void __launch_bounds__(320, 1)
+    bsa_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_doh,
                        const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                        const BwdArgs a) {
     using C = BwdCfg<D>;
+    constexpr int kHalfTile = C::kTileBytes / 2;  // 64 tokens x D
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -553,7 +582,7 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* sV = smem + C::kTileBytes;
     auto sQ = [&](int s) { return smem + (2 + s) * C::kTileBytes; };
     auto sdO = [&](int s) { return smem + (4 + s) * C::kTileBytes; };
-    float* sAux = reinterpret_cast<float*>(smem + C::kAux);  // [2][2][128]
+    float* sAux = reinterpret_cast<float*>(smem + C::kAux);  // [slot][half][lse2 64 | D 64]
     DkvCtl* ctl = reinterpret_cast<DkvCtl*>(smem + C::kCtl);
     uint16_t* list = reinterpret_cast<uint16_t*>(smem + C::kList);
     const int warp = threadIdx.x >> 5;
@@ -565,10 +594,12 @@ __global__ void __launch_bounds__(192, 1)
     if (threadIdx.x == 0) {
         mbar_init(&ctl->kv_full, 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&ctl->qd_full[s], 1);
-            mbar_init(&ctl->qd_empty[s], 1);
+            for (int h = 0; h < 2; ++h) {
+                mbar_init(&ctl->qd_full[s][h], 1);
+                mbar_init(&ctl->qd_empty[s][h], 1);
+            }
             mbar_init(&ctl->sd_full[s], 1);
-            mbar_init(&ctl->p_full[s], 128);
+            mbar_init(&ctl->p_full[s], 256);
         }
         mbar_init(&ctl->dkv_full, 1);
         mbar_init(&ctl->aux, 1);
@@ -597,10 +628,10 @@ __global__ void __launch_bounds__(192, 1)
         if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.status, kStatusBadIndex);
         if (lane == 0) {
             ctl->n_valid = cnt;
-            prefetch_tensormap(&tm_q);
+            prefetch_tensormap(&tm_qh);
             prefetch_tensormap(&tm_k);
             prefetch_tensormap(&tm_v);
-            prefetch_tensormap(&tm_do);
+            prefetch_tensormap(&tm_doh);
             prefetch_tensormap(&tm_dk);
             prefetch_tensormap(&tm_dv);
         }
@@ -624,40 +655,44 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0 && n > 0) {
             mbar_arrive_expect_tx(&ctl->kv_full, 2 * C::kTileBytes);
 #pragma unroll
-            for (int h = 0; h < C::kHalves; ++h) {
-                tma_load_5d(&tm_k, smem_u32(sK) + h * C::kHalfBytes, &ctl->kv_full, h * 64, k_w, k_h,
+            for (int c = 0; c < C::kHalves; ++c) {
+                tma_load_5d(&tm_k, smem_u32(sK) + c * C::kHalfBytes, &ctl->kv_full, c * 64, k_w, k_h,
                             k_t, bh);
-                tma_load_5d(&tm_v, smem_u32(sV) + h * C::kHalfBytes, &ctl->kv_full, h * 64, k_w, k_h,
+                tma_load_5d(&tm_v, smem_u32(sV) + c * C::kHalfBytes, &ctl->kv_full, c * 64, k_w, k_h,
                             k_t, bh);
             }
-            int nq[2] = {0, 0};
+            int nq[2][2] = {{0, 0}, {0, 0}};
             bool ok = true;
             for (int i = 0; i < n && ok; ++i) {
                 const int s = i & 1;
-                if (i >= 2 && !mbar_wait(&ctl->qd_empty[s], ((i - 2) >> 1) & 1, abort_flag, a.status,
-                                         tmo, site(1, 1, s, i))) {
-                    ok = false;
-                    break;
-                }
                 const int r = list[i];
                 int qt, qh, qw;
                 chunk_origin(a.q_skip + r, a.NH, a.NW, qt, qh, qw);
-                mbar_arrive_expect_tx(&ctl->qd_full[s], 2 * C::kTileBytes + 1024);
+                for (int h = 0; h < 2; ++h) {
+                    if (i >= 2 && !mbar_wait(&ctl->qd_empty[s][h], ((i - 2) >> 1) & 1, abort_flag,
+                                             a.status, tmo, site(1, 1 + h, s, i))) {
+                        ok = false;
+                        break;
+                    }
+                    uint64_t* bar = &ctl->qd_full[s][h];
+                    mbar_arrive_expect_tx(bar, 2 * kHalfTile + 512);
 #pragma unroll
-                for (int h = 0; h < C::kHalves; ++h) {
-                    tma_load_5d(&tm_q, smem_u32(sQ(s)) + h * C::kHalfBytes, &ctl->qd_full[s], h * 64,
-                                qw, qh, qt, bh);
-                    tma_load_5d(&tm_do, smem_u32(sdO(s)) + h * C::kHalfBytes, &ctl->qd_full[s],
-                                h * 64, qw, qh, qt, bh);
+                    for (int c = 0; c < C::kHalves; ++c) {
+                        tma_load_5d(&tm_qh, smem_u32(sQ(s)) + c * C::kHalfBytes + h * 8192, bar, c * 64,
+                                    qw, qh, qt + 2 * h, bh);
+                        tma_load_5d(&tm_doh, smem_u32(sdO(s)) + c * C::kHalfBytes + h * 8192, bar,
+                                    c * 64, qw, qh, qt + 2 * h, bh);
+                    }
+                    bulk_load(smem_u32(sAux + s * 256 + h * 128),
+                              a.aux + (static_cast<int64_t>(bh) * a.Nq + r) * 256 + h * 128, 512, bar);
+                    ++nq[s][h];
                 }
-                bulk_load(smem_u32(sAux + s * 256), a.aux + (static_cast<int64_t>(bh) * a.Nq + r) * 256,
-                          1024, &ctl->qd_full[s]);
-                ++nq[s];
             }
             if (!ok || *abort_flag) {
                 drain_wait(&ctl->kv_full, 0, tmo);
                 for (int s = 0; s < 2; ++s)
-                    if (nq[s] > 0) drain_wait(&ctl->qd_full[s], (nq[s] - 1) & 1, tmo);
+                    for (int h = 0; h < 2; ++h)
+                        if (nq[s][h] > 0) drain_wait(&ctl->qd_full[s][h], (nq[s][h] - 1) & 1, tmo);
             }
         }
         __syncwarp();
@@ -672,12 +707,10 @@ __global__ void __launch_bounds__(192, 1)
             // S^T and dP^T for queries [64h, 64h+64) of step i
             auto issue_sd = [&](int i, int h) -> bool {
                 const int s = i & 1;
-                if (h == 0) {
-                    if (!mbar_wait(&ctl->qd_full[s], (i >> 1) & 1, abort_flag, a.status, tmo,
-                                   site(2, 1, s, i)))
-                        return false;
-                    tc_fence_after();
-                }
+                if (!mbar_wait(&ctl->qd_full[s][h], (i >> 1) & 1, abort_flag, a.status, tmo,
+                               site(2, 1, s * 2 + h, i)))
+                    return false;
+                tc_fence_after();
                 const uint32_t sk = smem_u32(sK), sv = smem_u32(sV);
                 const uint32_t sq = smem_u32(sQ(s)) + h * 8192, sd = smem_u32(sdO(s)) + h * 8192;
 #pragma unroll
@@ -703,17 +736,18 @@ __global__ void __launch_bounds__(192, 1)
                     return false;
                 tc_fence_after();
                 const uint32_t sq = smem_u32(sQ(s)), sd = smem_u32(sdO(s));
+                // queries 16kk.. of half h: column 64h + 32*(kk/2) + 8*(kk%2) of S^T / dP^T
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + 256u, tmem + 64u * h + kk * 8,
+                    mma_ts(tmem + 256u, tmem + 64u * h + 32u * (kk >> 1) + 8u * (kk & 1),
                            sdesc_sw128(sd + (4 * h + kk) * 2048, C::kHalfBytes, 1024), kIdG,
                            (i > 0 || h > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + 384u, tmem + 128u + 64u * h + kk * 8,
+                    mma_ts(tmem + 384u, tmem + 128u + 64u * h + 32u * (kk >> 1) + 8u * (kk & 1),
                            sdesc_sw128(sq + (4 * h + kk) * 2048, C::kHalfBytes, 1024), kIdG,
                            (i > 0 || h > 0 || kk > 0) ? 1u : 0u);
-                if (h == 1) tc_commit(&ctl->qd_empty[s]);
+                tc_commit(&ctl->qd_empty[s][h]);
                 return true;
             };
             ok = ok && issue_sd(0, 0) && issue_sd(0, 1);
@@ -731,33 +765,33 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ P^T, dS^T + epilogue
-        const int m = threadIdx.x;  // key row = TMEM lane (warps 0-3)
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const int grp = warp >> 2;                    // query columns [32*grp, 32*grp + 32) of a half
+        const int m = (warp & 3) * 32 + lane;         // key row = TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const float2 cc = make_float2(a.scale_log2, a.scale_log2);
         bool ok = true;
         for (int i = 0; i < n && ok; ++i) {
             const int s = i & 1;
-            // the aux record arrived with this step's Q/dO copies
-            bool got = mbar_wait(&ctl->qd_full[s], (i >> 1) & 1, abort_flag, a.status, tmo, site(3, 3, s, i));
-            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-            const float* lse2 = sAux + s * 256;
-            const float* Dq = lse2 + 128;
             for (int h = 0; h < 2; ++h) {
-                got = mbar_wait(&ctl->sd_full[h], i & 1, abort_flag, a.status, tmo, site(3, 4, h, i));
+                // this half's aux record arrived with its Q/dO copies
+                bool got = mbar_wait(&ctl->qd_full[s][h], (i >> 1) & 1, abort_flag, a.status, tmo,
+                                     site(3, 3, s * 2 + h, i));
+                got = got && mbar_wait(&ctl->sd_full[h], i & 1, abort_flag, a.status, tmo, site(3, 4, h, i));
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t tS = tmem + lane_off + 64u * h;
-                const uint32_t tP = tmem + lane_off + 128u + 64u * h;
-#pragma unroll
-                for (int g = 0; g < 2; ++g) {
+                const float* lse2 = sAux + s * 256 + h * 128;
+                const float* Dq = lse2 + 64;
+                const uint32_t tS = tmem + lane_off + 64u * h + 32u * grp;
+                const uint32_t tP = tmem + lane_off + 128u + 64u * h + 32u * grp;
+                {
                     uint32_t sv[32], pv[32];
-                    tmem_ld32(tS + g * 32, sv);
-                    tmem_ld32(tP + g * 32, pv);
+                    tmem_ld32(tS, sv);
+                    tmem_ld32(tP, pv);
                     tmem_wait_ld();
                     uint32_t pk[16], dk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const int qi = 64 * h + 32 * g + 2 * e;  // query column of this pair
+                        const int qi = 32 * grp + 2 * e;  // query of this pair within the half
                         const float2 l2 = *reinterpret_cast<const float2*>(lse2 + qi);
                         const float2 dd = *reinterpret_cast<const float2*>(Dq + qi);
                         const float2 x = __ffma2_rn(
@@ -770,8 +804,8 @@ __global__ void __launch_bounds__(192, 1)
                         pk[e] = pack_bf16x2(p.x, p.y);
                         dk[e] = pack_bf16x2(ds.x, ds.y);
                     }
-                    tmem_st16(tS + g * 16, pk);
-                    tmem_st16(tP + g * 16, dk);
+                    tmem_st16(tS, pk);
+                    tmem_st16(tP, dk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -782,26 +816,28 @@ __global__ void __launch_bounds__(192, 1)
             const bool got = mbar_wait(&ctl->dkv_full, 0, abort_flag, a.status, tmo, site(3, 6, 0, 0));
             ok = __all_sync(0xffffffffu, got);
         }
-        const bool all_ok = bar_red_and(1, 128, ok);
+        const bool all_ok = bar_red_and(1, 256, ok);
         if (all_ok && n > 0) {
             tc_fence_after();
-            // K and V tiles are dead once every MMA has completed
-            stage_tmem_rows<D>(tmem + lane_off + 256u, sV, m, 1.0f);
-            stage_tmem_rows<D>(tmem + lane_off + 384u, sK, m, a.scale);
+            // K and V tiles are dead once every MMA has completed: group 0 stages
+            // dV, group 1 dK (scaled)
+            if (grp == 0)
+                stage_tmem_rows<D>(tmem + lane_off + 256u, sV, m, 1.0f);
+            else
+                stage_tmem_rows<D>(tmem + lane_off + 384u, sK, m, a.scale);
             fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (m == 0) {
+            named_bar_sync(1, 256);
+            if (threadIdx.x == 0) {
 #pragma unroll
-                for (int h = 0; h < C::kHalves; ++h) {
-                    tma_store_5d(&tm_dv, smem_u32(sV) + h * C::kHalfBytes, h * 64, k_w, k_h, k_t, bh);
-                    tma_store_5d(&tm_dk, smem_u32(sK) + h * C::kHalfBytes, h * 64, k_w, k_h, k_t, bh);
+                for (int c = 0; c < C::kHalves; ++c) {
+                    tma_store_5d(&tm_dv, smem_u32(sV) + c * C::kHalfBytes, c * 64, k_w, k_h, k_t, bh);
+                    tma_store_5d(&tm_dk, smem_u32(sK) + c * C::kHalfBytes, c * 64, k_w, k_h, k_t, bh);
                 }
                 tma_store_commit_and_wait_all();
             }
         } else if (all_ok) {
             // no query chunk selected this key chunk: zero gradients
-            zero_token<D>(a.dk, bh, a.N, a.H, a.W, k_t, k_h, k_w, m);
-            zero_token<D>(a.dv, bh, a.N, a.H, a.W, k_t, k_h, k_w, m);
+            zero_token<D>(grp ? a.dk : a.dv, bh, a.N, a.H, a.W, k_t, k_h, k_w, m);
         }
     }
 
@@ -829,13 +865,13 @@ cudaError_t launch_bwd_d(const Dims& g, const CUtensorMap* m, const BwdArgs& dq_
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    // m: q, k, v, dout, dq, dk, dv
+    // m: q, k, v, dout, dq, dk, dv (whole chunks), then q and dout (half chunks)
     bsa_bwd_dq_kernel<D><<<static_cast<unsigned>(dq_args.units), C::kThreads, C::kSmemBytes, st>>>(
         m[0], m[1], m[2], m[3], m[4], dq_args);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     bsa_bwd_dkv_kernel<D><<<static_cast<unsigned>(dkv_args.units), C::kThreads, C::kSmemBytes, st>>>(
-        m[0], m[1], m[2], m[3], m[5], m[6], dkv_args);
+        m[7], m[1], m[2], m[8], m[5], m[6], dkv_args);
     return cudaGetLastError();
 }
 
@@ -882,10 +918,12 @@ cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const v
     int32_t* row_idx = reinterpret_cast<int32_t*>(ws + L.row_idx);
     const int64_t cols = g.BH * g.Nc;
 
-    CUtensorMap m[7];
-    const void* bases[7] = {q, k, v, dout, dq, dk, dv};
-    for (int i = 0; i < 7; ++i)
-        if (!make_chunk_map(&m[i], bases[i], g)) return cudaErrorInvalidValue;
+    // whole-chunk maps q, k, v, dout, dq, dk, dv, then half-chunk maps of q and dout
+    CUtensorMap m[9];
+    const void* bases[9] = {q, k, v, dout, dq, dk, dv, q, dout};
+    for (int i = 0; i < 9; ++i)
+        if (!make_chunk_map(&m[i], bases[i], g, i < 7 ? kChunkT : kChunkT / 2))
+            return cudaErrorInvalidValue;
 
     cudaError_t e = cudaMemsetAsync(ws + L.bitmap, 0, L.cnt - L.bitmap, st);  // bitmap + rawcnt
     if (e != cudaSuccess) return e;

@@ -54,7 +54,7 @@ WsLayout ws_layout(const Dims& g, const bsa_params& p);
 // Backward workspace layout (byte offsets).
 struct BwdLayout {
     size_t status;   // uint32 status word (+ padding to 256)
-    size_t aux;      // float [BH][Nq][2][128]: LSE * log2(e), <dO, O>
+    size_t aux;      // float [BH][Nq][2][128]: per half of 64 queries, LSE * log2(e) then <dO, O>
     size_t bitmap;   // uint32 [BH*Nc][words]: query rows per key chunk
     size_t rawcnt;   // int32 [BH*Nc]: entries per key chunk (duplicate check)
     size_t cnt;      // int32 [BH*Nc]: distinct rows per key chunk
@@ -82,8 +82,10 @@ cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const vo
                            void* out, float* lse, uint32_t* status, uint64_t timeout_ns,
                            int debug_flags, cudaStream_t st);
 // 5-D TMA map over a [BH][T][H][W][d] bf16 tensor whose box is one (4,4,8)
-// chunk x 64 channels (128-byte swizzle). False if the driver call failed.
-bool make_chunk_map(CUtensorMap* tm, const void* base, const Dims& g);
+// chunk x 64 channels (128-byte swizzle); box_t = 2 gives half a chunk (its
+// first or last two frames: local tokens 0-63 or 64-127). False if the driver
+// call failed.
+bool make_chunk_map(CUtensorMap* tm, const void* base, const Dims& g, int box_t = kChunkT);
 cudaError_t launch_scan_counts(const int32_t* counts, int64_t n, int32_t* ptr, cudaStream_t st);
 cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const void* v,
                             const void* out, const float* lse, const void* dout,

@@ -18,7 +18,13 @@ pytestmark = pytest.mark.gpu
 
 import block_sparse_attention_13_b200 as bsa  # noqa: E402
 
-# bars: max |gpu - ref| / max |ref| and mean |gpu - ref| / mean |ref|, per tensor
+# bars: max |gpu - ref| / max |ref| and mean |gpu - ref| / mean |ref|, per tensor.
+# Rounding the gradients to bf16 alone costs up to 2^-9 (0.2 %) of an element;
+# P and dS enter the products as bf16 (2^-9 each) and D comes from the bf16
+# output. dQ = scale * sum_j dS_j K_j cancels (sum_j dS_j = 0) while the
+# rounding of dS adds up over the row's keys, so its relative error grows with
+# the row length. Measured: small grids at most 0.5 % max / 0.3 % mean; the
+# 720p grid (5,760 keys per row) 1.04 % / 0.48 % for dQ. Bars: twice that.
 BWD_MAX_REL = 2e-2
 BWD_MEAN_REL = 1e-2
 
