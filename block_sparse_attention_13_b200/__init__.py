@@ -32,6 +32,8 @@ BSA_ERR_CAPACITY = 9
 
 BSA_SEL_TOPK = 0
 BSA_SEL_CDF = 1
+BSA_SEL_TOPK_CDF = 2
+MODES = {"topk": BSA_SEL_TOPK, "cdf": BSA_SEL_CDF, "topk_cdf": BSA_SEL_TOPK_CDF}
 
 EXPORTED = ("bsa_version", "bsa_status_string", "bsa_workspace_size", "bsa_plan_sizes",
             "bsa_plan", "bsa_plan_noalloc", "bsa_forward", "bsa_forward_ex", "bsa_read_status",
@@ -58,7 +60,7 @@ class bsa_params(ctypes.Structure):
 def make_params(B, heads, T, H, W, d, mode="topk", topk=1, cdf_p=0.9, cdf_cap_frac=0.25,
                 t_cond=0, scale=0.0, q_begin=0) -> bsa_params:
     return bsa_params(B, heads, T, H, W, d, 4, 4, 8, float(scale),
-                      BSA_SEL_TOPK if mode == "topk" else BSA_SEL_CDF, int(topk), float(cdf_p),
+                      MODES[mode], int(topk), float(cdf_p),
                       float(cdf_cap_frac), int(t_cond), int(q_begin))
 
 

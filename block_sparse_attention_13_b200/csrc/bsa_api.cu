@@ -26,10 +26,11 @@ WsLayout ws_layout(const Dims& g, const bsa_params& p) {
     off += round_up((size_t)g.BH * g.Nq * g.Nc * sizeof(float), 256);
     L.pad_stride = 0;
     L.counts = L.padded = off;
-    if (p.mode == BSA_SEL_CDF) {
+    if (p.mode != BSA_SEL_TOPK) {
         int cap = (int)std::floor((double)p.cdf_cap_frac * g.Nc);
         if (cap < 1) cap = 1;
         if (cap > g.Nc) cap = g.Nc;
+        if (p.mode == BSA_SEL_TOPK_CDF && p.topk < cap) cap = p.topk;
         L.pad_stride = cap;
         L.counts = off;
         off += round_up((size_t)g.rows * sizeof(int32_t), 256);
@@ -52,13 +53,14 @@ static int make_dims(const bsa_params* p, Dims* g) {
     if (p->t_cond < 0 || p->t_cond % kChunkT || p->t_cond > p->T) return BSA_ERR_SHAPE;
     if (p->q_begin < 0 || p->q_begin % kChunkT || p->q_begin >= p->T) return BSA_ERR_SHAPE;
     if (!(std::isfinite(p->scale)) || p->scale < 0.f) return BSA_ERR_INVALID_ARG;
-    if (p->mode == BSA_SEL_TOPK) {
+    if (p->mode == BSA_SEL_TOPK || p->mode == BSA_SEL_TOPK_CDF) {
         if (p->topk < 1) return BSA_ERR_INVALID_ARG;
-    } else if (p->mode == BSA_SEL_CDF) {
+    } else if (p->mode != BSA_SEL_CDF) {
+        return BSA_ERR_INVALID_ARG;
+    }
+    if (p->mode != BSA_SEL_TOPK) {
         if (!(p->cdf_p > 0.f && p->cdf_p <= 1.f)) return BSA_ERR_INVALID_ARG;
         if (!(p->cdf_cap_frac > 0.f && p->cdf_cap_frac <= 1.f)) return BSA_ERR_INVALID_ARG;
-    } else {
-        return BSA_ERR_INVALID_ARG;
     }
     g->B = p->B;
     g->heads = p->heads;
@@ -104,6 +106,7 @@ static int64_t max_nnz_of(const Dims& g, const bsa_params& p) {
         if (nrows == 0) continue;
         int cap = (int)std::floor((double)p.cdf_cap_frac * na);
         if (cap < 1) cap = 1;
+        if (p.mode == BSA_SEL_TOPK_CDF && p.topk < cap) cap = p.topk;
         total += nrows * cap;
     }
     return g.BH * total;

@@ -304,6 +304,8 @@ __global__ void __launch_bounds__(256) select_kernel(
         if (cap < 1) cap = 1;
         if (cap > pad_stride) cap = pad_stride;
         count = mstar < cap ? mstar : cap;
+        // combination: kept by both rules, i.e. the first min(k, CDF count) chunks
+        if (mode == BSA_SEL_TOPK_CDF && topk < count) count = topk;
     }
 
     // emit the top-`count` chunks by (score desc, index asc), ascending

@@ -55,16 +55,20 @@ typedef enum {
     BSA_ERR_CAPACITY = 9             /* col_idx capacity smaller than the selection needs     */
 } bsa_status;
 
-typedef enum { BSA_SEL_TOPK = 0, BSA_SEL_CDF = 1 } bsa_select_mode;
+/* Selection modes ([P3] "3D Block Sparse Attention": Top-K, CDF threshold and
+ * their combination). TOPK_CDF keeps a chunk when both rules keep it: the
+ * first min(topk, CDF count) chunks of the common descending order (the pages
+ * name the combination without defining it; this is the reading taken). */
+typedef enum { BSA_SEL_TOPK = 0, BSA_SEL_CDF = 1, BSA_SEL_TOPK_CDF = 2 } bsa_select_mode;
 
 typedef struct {
     int32_t B, heads, T, H, W, d; /* d in {64,128}; T%4 == H%4 == W%8 == 0                 */
     int32_t chunk_t, chunk_h, chunk_w; /* must be 4,4,8 ([P3] default chunk shape)          */
     float scale;        /* softmax scale; 0 means 1/sqrt(d) ([P1] scaled dot product)     */
     int32_t mode;       /* bsa_select_mode                                                */
-    int32_t topk;       /* TOPK: key chunks kept per query chunk (clamped to |A(i)|)      */
-    float cdf_p;        /* CDF: cumulative pooled-softmax mass to reach, in (0,1]          */
-    float cdf_cap_frac; /* CDF: at most max(1, floor(cap_frac*|A(i)|)) chunks, in (0,1]   */
+    int32_t topk;       /* TOPK, TOPK_CDF: key chunks kept per query chunk (clamped to |A(i)|) */
+    float cdf_p;        /* CDF, TOPK_CDF: cumulative pooled-softmax mass to reach, in (0,1] */
+    float cdf_cap_frac; /* CDF, TOPK_CDF: at most max(1, floor(cap_frac*|A(i)|)) chunks, (0,1] */
     int32_t t_cond;     /* leading latent frames holding condition tokens; 0 = none; %4==0 */
     int32_t q_begin;    /* first latent frame whose queries are computed; 0 = all; %4==0, < T.
                          * Query chunks of earlier frames are neither read nor written and

@@ -41,6 +41,9 @@ CN = 128
 
 c_i64p = ctypes.POINTER(ctypes.c_int64)
 
+# selection modes: top-k, CDF threshold, and their combination (chunks kept by both)
+MODES = {"topk": 0, "cdf": 1, "topk_cdf": 2}
+
 
 def build(force: bool = False) -> str:
     """Compile liboracle.so (gcc, -O2, OpenMP). Portable flags: no -march."""
@@ -146,7 +149,7 @@ def select(S, T, H, W, mode="topk", topk=0, cdf_p=0.9, cap_frac=0.25, t_cond=0, 
     col_cap = rows * Nc
     col_idx = np.empty(col_cap, dtype=np.int32)
     nnz = _check(_load().oracle_select(S.ctypes.data, B * Hh, T, H, W, int(t_cond),
-                                       0 if mode == "topk" else 1, int(topk), float(cdf_p),
+                                       MODES[mode], int(topk), float(cdf_p),
                                        float(cap_frac), int(fp32), row_ptr.ctypes.data,
                                        col_idx.ctypes.data, col_cap), "oracle_select")
     return row_ptr, col_idx[:nnz].copy()

@@ -156,7 +156,10 @@ static int int_cmp(const void* a, const void* b) {
  * Block selection over the scores S[bh][i][m] -> CSR in row order (bh, i).
  * mode 0 = top-k ([P1] top-r; [P3] Top-K), mode 1 = CDF ([P3] CDF threshold;
  * [P1] "CDF-p mode": descending pooled scores until the cumulative softmax of
- * the scores reaches p). k is clamped to |A(i)|. fp32 != 0 takes the CDF
+ * the scores reaches p), mode 2 = combination ([P3] lists "Top-K, CDF threshold
+ * and combination" modes without a definition; read as: a chunk is kept when
+ * both rules keep it, i.e. the first min(k, CDF count) chunks of the common
+ * descending order). k is clamped to |A(i)|. fp32 != 0 takes the CDF
  * decision in float arithmetic (scores are already float-valued then).
  * Column indices of a row are written in ascending order.
  * Returns nnz >= 0, or -1 on bad arguments, -2 if col_cap is too small.
@@ -165,7 +168,7 @@ int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, 
                       int topk, double cdf_p, double cap_frac, int fp32, int32_t* row_ptr,
                       int32_t* col_idx, int64_t col_cap) {
     if (!S || !row_ptr || !col_idx || BH <= 0 || !grid_ok(T, H, W) || t_cond < 0 ||
-        t_cond % CT != 0 || (mode != 0 && mode != 1) || (mode == 0 && topk <= 0))
+        t_cond % CT != 0 || mode < 0 || mode > 2 || (mode != 1 && topk <= 0))
         return -1;
     const int Nc = (int)((int64_t)T * H * W / CN);
     cand_t* cand = (cand_t*)malloc(sizeof(cand_t) * (size_t)Nc);
@@ -217,6 +220,9 @@ int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, 
                 int cap = (int)floor(cap_frac * na);
                 if (cap < 1) cap = 1;
                 count = mstar < cap ? mstar : cap;
+                /* combination (reading of [P3] "Top-K, CDF and combination"): a chunk is
+                   kept when both rules keep it; both are prefixes of the same order */
+                if (mode == 2 && topk < count) count = topk;
             }
             if (nnz + count > col_cap) {
                 free(cand);

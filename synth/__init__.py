@@ -2,7 +2,7 @@
 
 The C generator in ``synth.c`` is the single implementation used by the CPU
 oracle, the GPU tests and the benchmark. This module builds it on demand,
-exposes it through ctypes and names the five standard workloads.
+exposes it through ctypes and names the standard workloads.
 """
 from __future__ import annotations
 

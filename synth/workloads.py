@@ -1,4 +1,4 @@
-"""The five synthetic workloads (shapes, selection settings, generator knobs).
+"""The synthetic workloads (shapes, selection settings, generator knobs).
 
 Each workload stands in for a latent grid of the video DiT's refinement stage
 ("LongCat-Video Technical Report", sections "Block Sparse Attention (BSA)" and
@@ -20,7 +20,7 @@ class Workload:
     H: int
     W: int
     d: int
-    mode: str = "topk"          # "topk" | "cdf"
+    mode: str = "topk"          # "topk" | "cdf" | "topk_cdf" (chunks kept by both rules)
     topk: int = 0
     cdf_p: float = 0.9
     cdf_cap_frac: float = 0.25
@@ -74,6 +74,12 @@ WORKLOADS = {
     # block-causal video continuation with CDF selection (p = 0.9, cap 25%)
     "causal_cdf": Workload("causal_cdf", B=2, heads=32, T=24, H=48, W=80, d=128,
                            mode="cdf", cdf_p=0.9, cdf_cap_frac=0.25, t_cond=8),
+    # 87.5 % sparsity (r = N_k / 8): 90 of 720 chunks
+    "720p_r8": Workload("720p_r8", B=1, heads=32, T=24, H=48, W=80, d=128, topk=90),
+    # combination of both rules: CDF p = 0.1 (29-66 chunks on these inputs, median 41)
+    # bounded by k = 45, so each rule decides part of the rows
+    "720p_topk_cdf": Workload("720p_topk_cdf", B=1, heads=32, T=24, H=48, W=80, d=128,
+                              mode="topk_cdf", topk=45, cdf_p=0.1, cdf_cap_frac=0.25),
     # the same video-continuation input at a later denoising step: the condition
     # frames' K/V are cached, only the noisy queries (frames >= 8) are computed
     "causal_cdf_kv": Workload("causal_cdf_kv", B=2, heads=32, T=24, H=48, W=80, d=128,

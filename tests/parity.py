@@ -47,13 +47,16 @@ def valid_topk_set(sel, s64, cand):
     return lo >= hi or _tied(lo, hi)
 
 
-def cdf_count_ok(count, s64, cand, p, cap_frac):
-    """count is the CDF count of this row up to mass ties within TIE_REL."""
+def cdf_count_ok(count, s64, cand, p, cap_frac, k=None):
+    """count is the CDF count of this row (bounded by k in the combination
+    mode) up to mass ties within TIE_REL."""
     s = s64[cand]
     w = np.exp(s - s.max())
     w /= w.sum()
     mass = np.cumsum(np.sort(w)[::-1])
     cap = max(1, int(np.floor(cap_frac * len(cand))))
+    if k is not None:
+        cap = min(cap, k)
     mstar = int(np.searchsorted(mass, p, side="left")) + 1  # first prefix with mass >= p
     mstar = min(mstar, len(cand))
     if count == min(mstar, cap):
@@ -67,7 +70,7 @@ def cdf_count_ok(count, s64, cand, p, cap_frac):
 
 
 def compare_csr(gpu_rp, gpu_ci, ora_rp, ora_ci, S64, Nc, n_cond, mode, p=0.9, cap_frac=0.25,
-                rows=None):
+                rows=None, topk=None):
     """Returns (n_rows_checked, n_rows_differing); asserts validity of every row."""
     S64 = np.asarray(S64).reshape(-1, Nc, Nc)
     g_rows, o_rows = rows_of(gpu_rp, gpu_ci), rows_of(ora_rp, ora_ci)
@@ -86,7 +89,8 @@ def compare_csr(gpu_rp, gpu_ci, ora_rp, ora_ci, S64, Nc, n_cond, mode, p=0.9, ca
         if mode == "topk":
             assert len(g) == len(o), f"row {r}: count {len(g)} vs {len(o)}"
         else:
-            assert cdf_count_ok(len(g), s64, cand, p, cap_frac), \
+            k = topk if mode == "topk_cdf" else None
+            assert cdf_count_ok(len(g), s64, cand, p, cap_frac, k), \
                 f"row {r}: cdf count {len(g)} vs oracle {len(o)}"
     return len(idx), ndiff
 

@@ -75,6 +75,20 @@ def test_plan_sizes_topk_and_cdf(L):
     assert (rc, nnz) == (0, 240 * 240 + 480 * 300)
 
 
+def test_plan_sizes_topk_cdf_combination(L):
+    # per row at most min(k, cap): 720 noisy chunks, cap 180, k = 45
+    rc, rows, nnz = rc_sizes(P(heads=32, T=24, H=48, W=80, d=128, mode="topk_cdf", topk=45,
+                               cdf_p=0.1))
+    assert (rc, rows, nnz) == (0, 23040, 23040 * 45)
+    # k above the cap: the cap bounds
+    rc, rows, nnz = rc_sizes(P(heads=1, T=24, H=48, W=80, d=128, mode="topk_cdf", topk=300,
+                               cdf_p=0.9, t_cond=8))
+    assert (rc, nnz) == (0, 240 * 60 + 480 * 180)
+    ws_c = bsa.bsa_workspace_size(P(heads=1, T=24, H=48, W=80, d=128, mode="cdf"))
+    ws_tc = bsa.bsa_workspace_size(P(heads=1, T=24, H=48, W=80, d=128, mode="topk_cdf", topk=45))
+    assert ws_tc < ws_c   # padded rows hold min(k, cap) = 45 instead of 180 entries
+
+
 def test_plan_sizes_kv_cached_step(L):
     # causal_cdf with only the noisy queries (frames >= 8): 480 of 720 rows per head
     rc, rows, nnz = rc_sizes(P(B=2, heads=32, T=24, H=48, W=80, d=128, mode="cdf", t_cond=8,
@@ -100,6 +114,8 @@ def test_plan_sizes_kv_cached_step(L):
     (dict(t_cond=2), bsa.BSA_ERR_SHAPE),
     (dict(t_cond=8), bsa.BSA_ERR_SHAPE),
     (dict(topk=0), bsa.BSA_ERR_INVALID_ARG),
+    (dict(mode="topk_cdf", topk=0), bsa.BSA_ERR_INVALID_ARG),
+    (dict(mode="topk_cdf", cdf_p=0.0), bsa.BSA_ERR_INVALID_ARG),
     (dict(mode="cdf", cdf_p=0.0), bsa.BSA_ERR_INVALID_ARG),
     (dict(mode="cdf", cdf_p=1.5), bsa.BSA_ERR_INVALID_ARG),
     (dict(mode="cdf", cdf_cap_frac=0.0), bsa.BSA_ERR_INVALID_ARG),
@@ -205,3 +221,9 @@ def test_no_cpu_fallback_without_a_gpu(L):
     assert rc == bsa.BSA_ERR_CUDA
     with pytest.raises(bsa.BsaError):
         bsa.bsa_plan_sizes(P(T=6))
+
+
+def test_unknown_selection_mode_rejected(L):
+    p = P()
+    p.mode = 3
+    assert rc_sizes(p)[0] == bsa.BSA_ERR_INVALID_ARG

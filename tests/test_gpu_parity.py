@@ -36,6 +36,12 @@ SMALL = {
                                         t_cond=8),
     "cdf_nocap": W["tiny"].with_(name="cdf_nocap", heads=2, T=8, H=16, W=32, d=64, mode="cdf",
                                  cdf_p=0.5, cdf_cap_frac=1.0),
+    # combination mode where each rule binds on some rows: CDF counts 3-12 against k = 5 or 6
+    "topk_cdf_small": W["tiny"].with_(name="topk_cdf_small", heads=2, T=8, H=16, W=32, d=128,
+                                      mode="topk_cdf", topk=6, cdf_p=0.2, cdf_cap_frac=0.5),
+    "causal_topk_cdf": W["tiny"].with_(name="causal_topk_cdf", B=2, heads=2, T=16, H=16, W=32,
+                                       d=64, mode="topk_cdf", topk=5, cdf_p=0.2,
+                                       cdf_cap_frac=0.25, t_cond=8),
 }
 
 
@@ -78,7 +84,7 @@ def check_case(wl, rows=None, qkv=None):
                                 wl.cdf_cap_frac, wl.t_cond, fp32=True)
     S64 = oracle.scores(oracle.pool(q, wl.T, wl.H, wl.W), oracle.pool(k, wl.T, wl.H, wl.W), scale)
     n_checked, n_diff = compare_csr(rp, ci, o_rp, o_ci, S64, wl.Nc, wl.n_cond, wl.mode,
-                                    wl.cdf_p, wl.cdf_cap_frac)
+                                    wl.cdf_p, wl.cdf_cap_frac, topk=wl.topk)
     assert n_diff <= max(1, n_checked // 100), f"{n_diff} of {n_checked} rows differ (ties)"
     # attention on the GPU's own CSR
     if rows is None:
@@ -298,7 +304,8 @@ def _sample_rows(wl, per_head, seed=0):
 
 
 @pytest.mark.parametrize("name,per_head", [("480p", 8), ("720p", 4), ("long", 2),
-                                           ("causal_cdf", 2)])
+                                           ("causal_cdf", 2), ("720p_r8", 2),
+                                           ("720p_topk_cdf", 2)])
 def test_full_size_workloads(name, per_head):
     wl = W[name]
     check_case(wl, rows=_sample_rows(wl, per_head))

@@ -217,6 +217,24 @@ def test_cdf_bruteforce_minimal_subset(p, cap_frac):
         assert got == sorted(order[:cnt].tolist())
 
 
+@pytest.mark.parametrize("k,p", [(2, 0.5), (4, 0.3), (6, 0.9), (1, 0.05)])
+def test_topk_cdf_combination_is_the_intersection(k, p):
+    """Combination mode keeps the chunks both rules keep: the lexsort top-k set
+    intersected with the brute-force minimal CDF set."""
+    rng = np.random.default_rng(5 + k)
+    Nc = 8
+    S = rng.normal(size=(1, 1, Nc, Nc)) * 1.5
+    S[0, 0, 3, :4] = S[0, 0, 3, 4]                    # a row with ties
+    T, H, W = 4, 8, 32                                  # 1 x 2 x 4 = 8 chunks
+    rp, ci = oracle.select(S, T, H, W, mode="topk_cdf", topk=k, cdf_p=p, cap_frac=1.0)
+    for i in range(Nc):
+        row = S[0, 0, i]
+        order = np.lexsort((np.arange(Nc), -row))      # score desc, index asc
+        topk_set = set(order[:min(k, Nc)].tolist())
+        cdf_set = set(order[:_bruteforce_cdf(row, np.arange(Nc), p, 1.0)].tolist())
+        assert set(ci[rp[i]:rp[i + 1]].tolist()) == (topk_set & cdf_set), i
+
+
 def test_cdf_special_cases():
     T, H, W = 4, 8, 32
     rng = np.random.default_rng(5)
