@@ -55,8 +55,8 @@ typedef enum {
     BSA_ERR_CAPACITY = 9             /* col_idx capacity smaller than the selection needs     */
 } bsa_status;
 
-/* Selection modes ([P3] "3D Block Sparse Attention": Top-K, CDF threshold and
- * their combination). TOPK_CDF keeps a chunk when both rules keep it: the
+/* Selection modes ([P3] "3D Block Sparse Attention": Top-K, the CDF threshold
+ * and a combination of the two). TOPK_CDF keeps a chunk when both rules keep it: the
  * first min(topk, CDF count) chunks of the common descending order (the pages
  * name the combination without defining it; this is the reading taken). */
 typedef enum { BSA_SEL_TOPK = 0, BSA_SEL_CDF = 1, BSA_SEL_TOPK_CDF = 2 } bsa_select_mode;

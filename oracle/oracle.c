@@ -156,8 +156,8 @@ static int int_cmp(const void* a, const void* b) {
  * Block selection over the scores S[bh][i][m] -> CSR in row order (bh, i).
  * mode 0 = top-k ([P1] top-r; [P3] Top-K), mode 1 = CDF ([P3] CDF threshold;
  * [P1] "CDF-p mode": descending pooled scores until the cumulative softmax of
- * the scores reaches p), mode 2 = combination ([P3] lists "Top-K, CDF threshold
- * and combination" modes without a definition; read as: a chunk is kept when
+ * the scores reaches p), mode 2 = combination ([P3] names a combined mode next to Top-K
+ * and the CDF threshold without defining it; read as: a chunk is kept when
  * both rules keep it, i.e. the first min(k, CDF count) chunks of the common
  * descending order). k is clamped to |A(i)|. fp32 != 0 takes the CDF
  * decision in float arithmetic (scores are already float-valued then).
@@ -220,7 +220,7 @@ int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, 
                 int cap = (int)floor(cap_frac * na);
                 if (cap < 1) cap = 1;
                 count = mstar < cap ? mstar : cap;
-                /* combination (reading of [P3] "Top-K, CDF and combination"): a chunk is
+                /* combination (the reading taken of [P3]'s combined mode): a chunk is
                    kept when both rules keep it; both are prefixes of the same order */
                 if (mode == 2 && topk < count) count = topk;
             }
