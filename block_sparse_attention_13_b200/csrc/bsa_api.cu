@@ -49,7 +49,6 @@ static int make_dims(const bsa_params* p, Dims* g) {
     if (p->chunk_t != kChunkT || p->chunk_h != kChunkH || p->chunk_w != kChunkW)
         return BSA_ERR_UNSUPPORTED;
     if (p->d != 64 && p->d != 128) return BSA_ERR_UNSUPPORTED;
-    if (p->T % kChunkT || p->H % kChunkH || p->W % kChunkW) return BSA_ERR_SHAPE;
     if (p->t_cond < 0 || p->t_cond % kChunkT || p->t_cond > p->T) return BSA_ERR_SHAPE;
     if (p->q_begin < 0 || p->q_begin % kChunkT || p->q_begin >= p->T) return BSA_ERR_SHAPE;
     if (!(std::isfinite(p->scale)) || p->scale < 0.f) return BSA_ERR_INVALID_ARG;
@@ -68,9 +67,11 @@ static int make_dims(const bsa_params* p, Dims* g) {
     g->H = p->H;
     g->W = p->W;
     g->d = p->d;
-    g->NT = p->T / kChunkT;
-    g->NH = p->H / kChunkH;
-    g->NW = p->W / kChunkW;
+    // chunks per axis by ceiling division: edge chunks of a grid that is not a
+    // multiple of the chunk shape are partial
+    g->NT = (p->T + kChunkT - 1) / kChunkT;
+    g->NH = (p->H + kChunkH - 1) / kChunkH;
+    g->NW = (p->W + kChunkW - 1) / kChunkW;
     const int64_t nc = (int64_t)g->NT * g->NH * g->NW;
     g->N = (int64_t)p->T * p->H * p->W;
     g->BH = (int64_t)p->B * p->heads;
@@ -137,7 +138,7 @@ const char* bsa_status_string(int s) {
     switch (s) {
         case BSA_OK: return "ok";
         case BSA_ERR_INVALID_ARG: return "invalid argument";
-        case BSA_ERR_SHAPE: return "unsupported shape (T%4, H%4, W%8, t_cond%4 must be 0)";
+        case BSA_ERR_SHAPE: return "invalid shape (sizes must be positive; t_cond, q_begin multiples of 4)";
         case BSA_ERR_UNSUPPORTED: return "unsupported configuration or device";
         case BSA_ERR_ALIGNMENT: return "tensor pointer not 16-byte aligned";
         case BSA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";

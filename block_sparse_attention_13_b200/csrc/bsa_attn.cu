@@ -76,7 +76,7 @@ struct FwdArgs {
     __nv_bfloat16* out;
     float* lse;
     uint32_t* status;
-    int H, W, NH, NW, Nc;
+    int T, H, W, NH, NW, Nc;
     int q_skip, Nq;    // CSR row r is query chunk q_skip + r % Nq of (batch, head) r / Nq
     int64_t N;
     int64_t rows;
@@ -103,8 +103,10 @@ struct __align__(8) Ctl {
 //   PV0(j), S0(j+1), PV1(j), S1(j+1)
 // so each tile's softmax runs while the tensor core works on the other tile.
 // S(j+1) is queued right behind the PV(j) that reads P from the same TMEM
-// columns: tcgen05 MMAs of one CTA execute in issue order.
-template <int D>
+// columns: tcgen05 MMAs of one CTA execute in issue order. kPartial: the grid
+// has partial edge chunks, whose key slots past the grid are masked out of the
+// softmax (a separate instantiation, so full grids keep the unmasked loop).
+template <int D, bool kPartial>
 __global__ void __launch_bounds__(320, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -337,6 +339,25 @@ __global__ void __launch_bounds__(320, 1)
             tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(s + 64));
             tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(s + 96));
             tmem_wait_ld();
+            if constexpr (kPartial) {
+                // A partial edge key chunk (grid not a multiple of the chunk shape): its
+                // slots past the grid were zero-filled by TMA and must not take part in
+                // the softmax. The branch is uniform across the CTA.
+                int kt, kh, kw;
+                chunk_origin(lists[t * C::kMaxChunks + it], a.NH, a.NW, kt, kh, kw);
+                const int nt = a.T - kt, nh = a.H - kh, nw = a.W - kw;
+                if (nt < kChunkT || nh < kChunkH || nw < kChunkW) {
+                    // bit lh*8 + lw: slot (lh, lw) of a 32-column frame exists
+                    uint32_t m32 = 0u;
+                    const uint32_t row8 = nw >= kChunkW ? 0xffu : ((1u << nw) - 1u);
+#pragma unroll
+                    for (int lh = 0; lh < kChunkH; ++lh)
+                        if (lh < nh) m32 |= row8 << (8 * lh);
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if ((c >> 5) >= nt || !((m32 >> (c & 31)) & 1u)) s[c] = 0xff800000u;  // -inf
+                }
+            }
             float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
             float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
 #pragma unroll
@@ -404,6 +425,9 @@ __global__ void __launch_bounds__(320, 1)
             int q_t, q_h, q_w;
             chunk_origin(a.q_skip + static_cast<int>(row % a.Nq), a.NH, a.NW, q_t, q_h, q_w);
             const int lt = m >> 5, lh = (m >> 3) & 3, lw = m & 7;
+            // a query slot of a partial edge chunk past the grid has no output (the TMA
+            // store clips those rows; the direct stores below skip them)
+            const bool q_exists = q_t + lt < a.T && q_h + lh < a.H && q_w + lw < a.W;
             const int64_t tok =
                 (static_cast<int64_t>(q_t + lt) * a.H + (q_h + lh)) * a.W + q_w + lw;
             if (all_ok && n_t > 0) {
@@ -438,9 +462,9 @@ __global__ void __launch_bounds__(320, 1)
                                      q_t, static_cast<int>(bh));
                     tma_store_commit_and_wait_all();
                 }
-                if (a.lse)
+                if (a.lse && q_exists)
                     a.lse[bh * a.N + tok] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
-            } else if (all_ok) {
+            } else if (all_ok && q_exists) {
                 // empty (or rejected) row: zeros, lse = -inf
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
                 uint4* dst = reinterpret_cast<uint4*>(a.out + (bh * a.N + tok) * D);
@@ -502,22 +526,31 @@ bool make_chunk_map(CUtensorMap* tm, const void* base, const Dims& g, int box_t)
 
 namespace {
 
-template <int D>
-cudaError_t launch_fwd_d(const Dims& g, const CUtensorMap& mq, const CUtensorMap& mk,
-                         const CUtensorMap& mv, const CUtensorMap& mo, const FwdArgs& args,
-                         cudaStream_t st) {
+template <int D, bool kPartial>
+cudaError_t launch_fwd_dp(const Dims& g, const CUtensorMap& mq, const CUtensorMap& mk,
+                          const CUtensorMap& mv, const CUtensorMap& mo, const FwdArgs& args,
+                          cudaStream_t st) {
     using C = AttnCfg<D>;
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<D>,
+        cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<D, kPartial>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
     const unsigned grid = static_cast<unsigned>((g.rows + 1) / 2);
-    bsa_fwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mo, args);
+    bsa_fwd_kernel<D, kPartial><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mo, args);
     return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_fwd_d(const Dims& g, const CUtensorMap& mq, const CUtensorMap& mk,
+                         const CUtensorMap& mv, const CUtensorMap& mo, const FwdArgs& args,
+                         cudaStream_t st) {
+    const bool partial = g.T % kChunkT || g.H % kChunkH || g.W % kChunkW;
+    return partial ? launch_fwd_dp<D, true>(g, mq, mk, mv, mo, args, st)
+                   : launch_fwd_dp<D, false>(g, mq, mk, mv, mo, args, st);
 }
 
 __global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y_poly,
@@ -558,6 +591,7 @@ cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const vo
     args.out = static_cast<__nv_bfloat16*>(out);
     args.lse = lse;
     args.status = status;
+    args.T = g.T;
     args.H = g.H;
     args.W = g.W;
     args.NH = g.NH;

@@ -48,7 +48,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
                                                        const __nv_bfloat16* __restrict__ dout,
                                                        const float* __restrict__ lse,
                                                        float* __restrict__ aux, int q_skip, int Nq,
-                                                       int H, int W, int NH, int NW, int64_t N) {
+                                                       int T, int H, int W, int NH, int NW,
+                                                       int64_t N) {
     constexpr int VPT = D / 8;               // 16-byte vectors per token row
     constexpr int ITERS = 128 * VPT / 256;   // vectors per thread
     const int r = blockIdx.x;
@@ -62,9 +63,12 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
         const int vi = it * 256 + tid;
         const int l = vi / VPT, dv = vi % VPT;
         const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
+        // slots of a partial edge chunk past the grid: D = 0 (their dO rows load as zeros)
+        const bool exists = ct + lt < T && ch + lh < H && cw + lw < W;
         const int64_t tok = (static_cast<int64_t>(ct + lt) * H + (ch + lh)) * W + cw + lw;
-        const uint4 a = *reinterpret_cast<const uint4*>(o + (bh * N + tok) * D + dv * 8);
-        const uint4 b = *reinterpret_cast<const uint4*>(dout + (bh * N + tok) * D + dv * 8);
+        const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 a = exists ? *reinterpret_cast<const uint4*>(o + (bh * N + tok) * D + dv * 8) : zero;
+        const uint4 b = exists ? *reinterpret_cast<const uint4*>(dout + (bh * N + tok) * D + dv * 8) : zero;
         const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
         float acc = 0.f;
 #pragma unroll
@@ -81,8 +85,10 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
     if (tid < 128) {
         const int l = tid;
         const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
+        const bool exists = ct + lt < T && ch + lh < H && cw + lw < W;
         const int64_t tok = (static_cast<int64_t>(ct + lt) * H + (ch + lh)) * W + cw + lw;
-        dst[(l >> 6) * 128 + (l & 63)] = lse[bh * N + tok] * kLog2e;
+        // a missing query gets LSE = +inf, so every P of it is exactly zero
+        dst[(l >> 6) * 128 + (l & 63)] = exists ? lse[bh * N + tok] * kLog2e : INFINITY;
     }
 }
 
@@ -197,7 +203,7 @@ struct BwdArgs {
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
     uint32_t* status;
-    int H, W, NH, NW, Nc;
+    int T, H, W, NH, NW, Nc;
     int q_skip, Nq;
     int64_t N;
     int64_t units;            // CTAs: CSR rows (dQ) or key chunks BH*Nc (dK/dV)
@@ -233,11 +239,13 @@ __device__ __forceinline__ void stage_tmem_rows(uint32_t t_row, uint8_t* stage, 
     }
 }
 
-// Zeros for local token m of the chunk at (t0, h0, w0) of head bh.
+// Zeros for local token m of the chunk at (t0, h0, w0) of head bh (nothing for
+// a slot of a partial edge chunk past the grid).
 template <int D>
-__device__ __forceinline__ void zero_token(__nv_bfloat16* base, int64_t bh, int64_t N, int H, int W,
-                                           int t0, int h0, int w0, int m) {
+__device__ __forceinline__ void zero_token(__nv_bfloat16* base, int64_t bh, int64_t N, int T,
+                                           int H, int W, int t0, int h0, int w0, int m) {
     const int lt = m >> 5, lh = (m >> 3) & 3, lw = m & 7;
+    if (t0 + lt >= T || h0 + lh >= H || w0 + lw >= W) return;
     const int64_t tok = (static_cast<int64_t>(t0 + lt) * H + (h0 + lh)) * W + w0 + lw;
     uint4* dst = reinterpret_cast<uint4*>(base + (bh * N + tok) * D);
 #pragma unroll
@@ -534,7 +542,7 @@ __global__ void __launch_bounds__(320, 1)
                 tma_store_commit_and_wait_all();
             }
         } else if (all_ok && grp == 0) {
-            zero_token<D>(a.dq, bh, a.N, a.H, a.W, q_t, q_h, q_w, m);  // no selected chunk
+            zero_token<D>(a.dq, bh, a.N, a.T, a.H, a.W, q_t, q_h, q_w, m);  // no selected chunk
         }
     }
 
@@ -837,7 +845,7 @@ __global__ void __launch_bounds__(320, 1)
             }
         } else if (all_ok) {
             // no query chunk selected this key chunk: zero gradients
-            zero_token<D>(grp ? a.dk : a.dv, bh, a.N, a.H, a.W, k_t, k_h, k_w, m);
+            zero_token<D>(grp ? a.dk : a.dv, bh, a.N, a.T, a.H, a.W, k_t, k_h, k_w, m);
         }
     }
 
@@ -931,11 +939,11 @@ cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const v
     const auto* o16 = static_cast<const __nv_bfloat16*>(out);
     const auto* g16 = static_cast<const __nv_bfloat16*>(dout);
     if (g.d == 128)
-        bwd_prep_kernel<128><<<pgrid, 256, 0, st>>>(o16, g16, lse, aux, g.q_skip, g.Nq, g.H, g.W,
-                                                   g.NH, g.NW, g.N);
+        bwd_prep_kernel<128><<<pgrid, 256, 0, st>>>(o16, g16, lse, aux, g.q_skip, g.Nq, g.T, g.H,
+                                                   g.W, g.NH, g.NW, g.N);
     else
-        bwd_prep_kernel<64><<<pgrid, 256, 0, st>>>(o16, g16, lse, aux, g.q_skip, g.Nq, g.H, g.W,
-                                                  g.NH, g.NW, g.N);
+        bwd_prep_kernel<64><<<pgrid, 256, 0, st>>>(o16, g16, lse, aux, g.q_skip, g.Nq, g.T, g.H,
+                                                  g.W, g.NH, g.NW, g.N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     csc_scatter_kernel<<<static_cast<unsigned>((g.rows + 7) / 8), 256, 0, st>>>(
         row_ptr, col_idx, col_cap, g.rows, g.Nq, g.Nc, L.words, bitmap, rawcnt, status);
@@ -961,6 +969,7 @@ cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const v
     args.dk = static_cast<__nv_bfloat16*>(dk);
     args.dv = static_cast<__nv_bfloat16*>(dv);
     args.status = status;
+    args.T = g.T;
     args.H = g.H;
     args.W = g.W;
     args.NH = g.NH;

@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
                                                    const __nv_bfloat16* __restrict__ x1,
                                                    float* __restrict__ p0, float* __restrict__ p1,
                                                    int c_begin0, int n0, int c_begin1, int n1,
-                                                   int H, int W, int NH, int NW, int64_t N) {
+                                                   int T, int H, int W, int NH, int NW, int64_t N) {
     constexpr int VPT = D / 8;               // 16-byte vectors per token row
     constexpr int ITERS = 128 * VPT / 256;   // vectors per thread
     constexpr int GROUPS = 256 / VPT;        // threads that share one channel group
@@ -59,6 +59,10 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     const int ct = c / (NH * NW), ch = (c / NW) % NH, cw = c % NW;
     const int tid = threadIdx.x;
     const int dvec = tid % VPT;
+    // a partial edge chunk (grid not a multiple of the chunk shape) averages the
+    // tokens it has
+    const int nt = min(kChunkT, T - ct * kChunkT), nh = min(kChunkH, H - ch * kChunkH),
+              nw = min(kChunkW, W - cw * kChunkW);
 
     float acc[8];
 #pragma unroll
@@ -69,6 +73,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
         const int v = it * 256 + tid;
         const int l = v / VPT;  // local token (lt*4 + lh)*8 + lw
         const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
+        if (lt >= nt || lh >= nh || lw >= nw) continue;
         const int64_t tok =
             ((int64_t)(ct * kChunkT + lt) * H + (ch * kChunkH + lh)) * W + cw * kChunkW + lw;
         const uint4 u = ld_nc_v4(base + tok * D + dvec * 8);
@@ -85,19 +90,20 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
         float s = 0.f;
 #pragma unroll
         for (int g2 = 0; g2 < GROUPS; ++g2) s += red[g2][tid];
-        pooled[(bh * n_out + blockIdx.x) * D + tid] = s * (1.0f / kChunkTokens);
+        pooled[(bh * n_out + blockIdx.x) * D + tid] = s * (1.0f / static_cast<float>(nt * nh * nw));
     }
 }
 
 // ------------------------------------------------------------------------
 // 3D rearrangement: a (lt, lh) segment of 8 tokens is contiguous both in the
 // [T,H,W] layout and in the chunk-major layout, so the copy is two streams of
-// contiguous 16-byte vectors.
+// contiguous 16-byte vectors. Slots of a partial edge chunk past the grid are
+// zero in the chunk-major layout and are not written back by the inverse.
 template <int D>
 __global__ void __launch_bounds__(256) rearrange_kernel(const __nv_bfloat16* __restrict__ src,
-                                                        __nv_bfloat16* __restrict__ dst, int H,
-                                                        int W, int NH, int NW, int Nc, int64_t N,
-                                                        int inverse) {
+                                                        __nv_bfloat16* __restrict__ dst, int T,
+                                                        int H, int W, int NH, int NW, int Nc,
+                                                        int64_t N, int inverse) {
     constexpr int VPT = D / 8;
     constexpr int ITERS = 128 * VPT / 256;
     const int c = blockIdx.x;
@@ -108,10 +114,14 @@ __global__ void __launch_bounds__(256) rearrange_kernel(const __nv_bfloat16* __r
         const int v = it * 256 + threadIdx.x;
         const int l = v / VPT, dv = v % VPT;
         const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
-        const int64_t tok =
-            ((int64_t)(ct * kChunkT + lt) * H + (ch * kChunkH + lh)) * W + cw * kChunkW + lw;
-        const int64_t thw = (bh * N + tok) * D + dv * 8;
+        const int t = ct * kChunkT + lt, h = ch * kChunkH + lh, w = cw * kChunkW + lw;
         const int64_t blk = ((bh * Nc + c) * kChunkTokens + l) * D + dv * 8;
+        if (t >= T || h >= H || w >= W) {
+            if (!inverse) *reinterpret_cast<uint4*>(dst + blk) = make_uint4(0u, 0u, 0u, 0u);
+            continue;
+        }
+        const int64_t tok = ((int64_t)t * H + h) * W + w;
+        const int64_t thw = (bh * N + tok) * D + dv * 8;
         const int64_t s_off = inverse ? blk : thw;
         const int64_t d_off = inverse ? thw : blk;
         *reinterpret_cast<uint4*>(dst + d_off) = ld_nc_v4(src + s_off);
@@ -440,11 +450,11 @@ cudaError_t launch_pool(const Dims& g, const void* x0, const void* x1, float* p0
     const auto* b = static_cast<const __nv_bfloat16*>(x1 ? x1 : x0);
     const int c0 = x1 ? g.q_skip : 0, n0 = x1 ? g.Nq : g.Nc;
     if (g.d == 128)
-        pool_kernel<128><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, c0, n0, 0, g.Nc, g.H, g.W,
-                                               g.NH, g.NW, g.N);
+        pool_kernel<128><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, c0, n0, 0, g.Nc, g.T, g.H,
+                                               g.W, g.NH, g.NW, g.N);
     else
-        pool_kernel<64><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, c0, n0, 0, g.Nc, g.H, g.W,
-                                              g.NH, g.NW, g.N);
+        pool_kernel<64><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, c0, n0, 0, g.Nc, g.T, g.H,
+                                              g.W, g.NH, g.NW, g.N);
     return cudaGetLastError();
 }
 
@@ -454,9 +464,11 @@ cudaError_t launch_rearrange(const Dims& g, const void* src, void* dst, int inve
     const auto* s = static_cast<const __nv_bfloat16*>(src);
     auto* d = static_cast<__nv_bfloat16*>(dst);
     if (g.d == 128)
-        rearrange_kernel<128><<<grid, 256, 0, st>>>(s, d, g.H, g.W, g.NH, g.NW, g.Nc, g.N, inverse);
+        rearrange_kernel<128><<<grid, 256, 0, st>>>(s, d, g.T, g.H, g.W, g.NH, g.NW, g.Nc, g.N,
+                                                    inverse);
     else
-        rearrange_kernel<64><<<grid, 256, 0, st>>>(s, d, g.H, g.W, g.NH, g.NW, g.Nc, g.N, inverse);
+        rearrange_kernel<64><<<grid, 256, 0, st>>>(s, d, g.T, g.H, g.W, g.NH, g.NW, g.Nc, g.N,
+                                                   inverse);
     return cudaGetLastError();
 }
 

@@ -17,7 +17,9 @@
  *   - Tensors Q, K, V, O are bf16, contiguous [B, heads, T*H*W, d], tokens in
  *     [T,H,W] order (t slowest, w fastest). DEVICE pointers, 16-byte aligned.
  *   - Chunk c of a (batch, head) covers the (4,4,8) block (ct, ch, cw) with
- *     c = (ct*(H/4) + ch)*(W/8) + cw; its local token l = (lt*4 + lh)*8 + lw.
+ *     c = (ct*NH + ch)*NW + cw, NH = ceil(H/4), NW = ceil(W/8); its local token
+ *     l = (lt*4 + lh)*8 + lw is token (4ct+lt, 4ch+lh, 8cw+lw) when that lies
+ *     inside the grid (a partial edge chunk has fewer than 128 tokens).
  *   - CSR rows are ordered (batch, head, query chunk); row r's key chunks are
  *     col_idx[row_ptr[r] .. row_ptr[r+1]), ascending. int32, DEVICE memory.
  *   - The caller allocates and owns every buffer. The library never allocates
@@ -45,7 +47,7 @@ extern "C" {
 typedef enum {
     BSA_OK = 0,
     BSA_ERR_INVALID_ARG = 1,         /* null pointer, bad enum, k < 1, p outside (0,1] ...   */
-    BSA_ERR_SHAPE = 2,               /* T%4, H%4, W%8 or t_cond%4 != 0, sizes <= 0 ...        */
+    BSA_ERR_SHAPE = 2,               /* sizes <= 0, t_cond or q_begin not a multiple of 4 ... */
     BSA_ERR_UNSUPPORTED = 3,         /* d not in {64,128}, chunk shape != (4,4,8), no sm_100  */
     BSA_ERR_ALIGNMENT = 4,           /* a tensor pointer is not 16-byte aligned               */
     BSA_ERR_WORKSPACE_TOO_SMALL = 5, /* ws_bytes < bsa_workspace_size()                       */
@@ -62,7 +64,12 @@ typedef enum {
 typedef enum { BSA_SEL_TOPK = 0, BSA_SEL_CDF = 1, BSA_SEL_TOPK_CDF = 2 } bsa_select_mode;
 
 typedef struct {
-    int32_t B, heads, T, H, W, d; /* d in {64,128}; T%4 == H%4 == W%8 == 0                 */
+    int32_t B, heads, T, H, W, d; /* d in {64,128}; any T, H, W >= 1: chunks per axis are
+                                   * ceil(T/4), ceil(H/4), ceil(W/8) ([P1] block counts by
+                                   * ceiling division); an edge chunk of a grid that is not a
+                                   * multiple of (4,4,8) is partial: pooling averages its
+                                   * existing tokens, attention uses its existing keys, and
+                                   * outputs exist for its existing queries only            */
     int32_t chunk_t, chunk_h, chunk_w; /* must be 4,4,8 ([P3] default chunk shape)          */
     float scale;        /* softmax scale; 0 means 1/sqrt(d) ([P1] scaled dot product)     */
     int32_t mode;       /* bsa_select_mode                                                */

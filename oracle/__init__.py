@@ -65,6 +65,8 @@ def _load():
             vp, i32, i64, dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
             lib.oracle_token_of.restype = i64
             lib.oracle_token_of.argtypes = [i32, i32, i32, i64, i32]
+            lib.oracle_num_chunks.restype = i64
+            lib.oracle_num_chunks.argtypes = [i32, i32, i32]
             lib.oracle_rearrange.restype = i32
             lib.oracle_rearrange.argtypes = [vp, i32, i32, i32, i32, i32, vp]
             lib.oracle_pool.restype = i32
@@ -106,14 +108,20 @@ def num_threads() -> int:
 
 
 def token_of(T, H, W, c, l) -> int:
+    """Token index of local slot l of chunk c, -1 past the grid edge."""
     return _load().oracle_token_of(T, H, W, c, l)
+
+
+def num_chunks(T, H, W) -> int:
+    """Chunks of the grid: ceil(T/4) * ceil(H/4) * ceil(W/8)."""
+    return _load().oracle_num_chunks(T, H, W)
 
 
 def rearrange(x, T, H, W):
     """THW order [B, heads, N, d] -> chunk-major [B, heads, Nc, 128, d] (bf16 bits)."""
     x = _u16(x)
     B, Hh, N, d = x.shape
-    out = np.empty((B, Hh, N // CN, CN, d), dtype=np.uint16)
+    out = np.empty((B, Hh, num_chunks(T, H, W), CN, d), dtype=np.uint16)
     _check(_load().oracle_rearrange(x.ctypes.data, B * Hh, T, H, W, d, out.ctypes.data),
            "oracle_rearrange")
     return out
@@ -123,7 +131,7 @@ def pool(x, T, H, W, fp32=False):
     """Chunk means [B, heads, Nc, d] (float64; float-valued when fp32)."""
     x = _u16(x)
     B, Hh, N, d = x.shape
-    out = np.empty((B, Hh, N // CN, d), dtype=np.float64)
+    out = np.empty((B, Hh, num_chunks(T, H, W), d), dtype=np.float64)
     _check(_load().oracle_pool(x.ctypes.data, B * Hh, T, H, W, d, int(fp32), out.ctypes.data),
            "oracle_pool")
     return out
@@ -230,5 +238,6 @@ def dense(q, k, v, T, H, W, scale, qtok, t_cond=0, want_lse=True):
 
 
 def chunk_tokens(T, H, W, c):
-    """Token indices (THW order) of the 128 local tokens of chunk c."""
+    """Token indices (THW order) of the 128 local slots of chunk c (-1 for a
+    slot past the grid edge of a partial chunk)."""
     return np.array([token_of(T, H, W, c, l) for l in range(CN)], dtype=np.int64)

@@ -19,6 +19,11 @@
  *
  * Readings where the pages are loose (each also listed in the design notes):
  *   - chunk shape (T,H,W) = (4,4,8), 128 tokens, for queries and keys alike;
+ *   - [P1] counts the blocks per axis with a ceiling division, so a grid whose
+ *     T, H or W is not a multiple of 4, 4, 8 has partial edge chunks: their
+ *     missing tokens (local slots past the grid edge) do not exist -- pooling
+ *     averages the chunk's existing tokens and attention ranges over existing
+ *     keys only;
  *   - chunk index is 0-based over the rearranged sequence: chunk c holds the
  *     tokens of block (ct,ch,cw) with c = (ct*NH + ch)*NW + cw and local index
  *     (lt*4 + lh)*8 + lw (block order [N_T,N_H,N_W], intra-block order [t,h,w]);
@@ -46,43 +51,53 @@ static inline double bf16_to_double(uint16_t b) {
     return (double)f;
 }
 
+static int ceil_div(int n, int c) { return (n + c - 1) / c; }
+
+/* [P1] 3D block partitioning: chunks per axis by ceiling division. */
+int64_t oracle_num_chunks(int T, int H, int W) {
+    return (int64_t)ceil_div(T, CT) * ceil_div(H, CH) * ceil_div(W, CW);
+}
+
 /* [P1] 3D block partitioning: token index (THW order) of local token `l` of
- * chunk `c`. */
+ * chunk `c`, or -1 when that slot of a partial edge chunk lies past the grid. */
 int64_t oracle_token_of(int T, int H, int W, int64_t c, int l) {
-    const int NH = H / CH, NW = W / CW;
+    const int NH = ceil_div(H, CH), NW = ceil_div(W, CW);
     const int64_t ct = c / ((int64_t)NH * NW);
     const int ch = (int)((c / NW) % NH);
     const int cw = (int)(c % NW);
     const int lt = l / (CH * CW), lh = (l / CW) % CH, lw = l % CW;
     const int64_t t = ct * CT + lt, h = (int64_t)ch * CH + lh, w = (int64_t)cw * CW + lw;
-    (void)T;
+    if (t >= T || h >= H || w >= W) return -1;
     return (t * H + h) * W + w;
 }
 
-static int grid_ok(int T, int H, int W) {
-    return T > 0 && H > 0 && W > 0 && T % CT == 0 && H % CH == 0 && W % CW == 0;
-}
+static int grid_ok(int T, int H, int W) { return T > 0 && H > 0 && W > 0; }
 
-/* [P1] "tokens are rearranged in memory so that all tokens within a block are
- * contiguous": out[bh][c][l][:] = x[bh][token_of(c,l)][:] (bf16 bits copied). */
+/* [P1] block-contiguous memory order (the tokens of a block made adjacent, in
+ * [t,h,w] order inside the block): out[bh][c][l][:] = x[bh][token_of(c,l)][:]
+ * (bf16 bits copied); the slots of missing tokens of partial chunks are zero. */
 int oracle_rearrange(const uint16_t* x, int BH, int T, int H, int W, int d, uint16_t* out) {
     if (!x || !out || BH <= 0 || d <= 0 || !grid_ok(T, H, W)) return -1;
-    const int64_t N = (int64_t)T * H * W, Nc = N / CN;
+    const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks(T, H, W);
     for (int bh = 0; bh < BH; ++bh)
         for (int64_t c = 0; c < Nc; ++c)
             for (int l = 0; l < CN; ++l) {
                 const int64_t tok = oracle_token_of(T, H, W, c, l);
-                memcpy(out + (((int64_t)bh * Nc + c) * CN + l) * d, x + ((int64_t)bh * N + tok) * d,
-                       sizeof(uint16_t) * (size_t)d);
+                uint16_t* o = out + (((int64_t)bh * Nc + c) * CN + l) * d;
+                if (tok < 0)
+                    memset(o, 0, sizeof(uint16_t) * (size_t)d);
+                else
+                    memcpy(o, x + ((int64_t)bh * N + tok) * d, sizeof(uint16_t) * (size_t)d);
             }
     return 0;
 }
 
-/* [P1] pooled representations: mean of the n = 128 token vectors of a chunk.
- * pooled[bh][c][:]. fp32 != 0: accumulate in float in local-token order. */
+/* [P1] pooled representations: mean of the token vectors of a chunk (its
+ * existing tokens: 128, fewer for a partial edge chunk). pooled[bh][c][:].
+ * fp32 != 0: accumulate in float in local-token order. */
 int oracle_pool(const uint16_t* x, int BH, int T, int H, int W, int d, int fp32, double* pooled) {
     if (!x || !pooled || BH <= 0 || d <= 0 || !grid_ok(T, H, W)) return -1;
-    const int64_t N = (int64_t)T * H * W, Nc = N / CN;
+    const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks(T, H, W);
 #pragma omp parallel for collapse(2) schedule(static)
     for (int bh = 0; bh < BH; ++bh)
         for (int64_t c = 0; c < Nc; ++c) {
@@ -90,11 +105,15 @@ int oracle_pool(const uint16_t* x, int BH, int T, int H, int W, int d, int fp32,
             for (int e = 0; e < d; ++e) {
                 double acc = 0.0;
                 float accf = 0.0f;
+                int n = 0;
                 for (int l = 0; l < CN; ++l) {
-                    const double v = bf16_to_double(x[((int64_t)bh * N + oracle_token_of(T, H, W, c, l)) * d + e]);
+                    const int64_t tok = oracle_token_of(T, H, W, c, l);
+                    if (tok < 0) continue;
+                    const double v = bf16_to_double(x[((int64_t)bh * N + tok) * d + e]);
                     if (fp32) accf += (float)v; else acc += v;
+                    ++n;
                 }
-                o[e] = fp32 ? (double)(accf * (1.0f / CN)) : acc / CN;
+                o[e] = fp32 ? (double)(accf * (1.0f / (float)n)) : acc / n;
             }
         }
     return 0;
@@ -129,7 +148,7 @@ int oracle_scores(const double* qp, const double* kp, int BH, int Nc, int d, dou
 /* [P1] block-causal attention: a chunk is a condition chunk when every frame of
  * it lies below t_cond. */
 static int is_condition_chunk(int H, int W, int64_t c, int t_cond) {
-    const int64_t ct = c / ((int64_t)(H / CH) * (W / CW));
+    const int64_t ct = c / ((int64_t)ceil_div(H, CH) * ceil_div(W, CW));
     return (ct * CT + CT - 1) < t_cond;
 }
 
@@ -170,7 +189,7 @@ int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, 
     if (!S || !row_ptr || !col_idx || BH <= 0 || !grid_ok(T, H, W) || t_cond < 0 ||
         t_cond % CT != 0 || mode < 0 || mode > 2 || (mode != 1 && topk <= 0))
         return -1;
-    const int Nc = (int)((int64_t)T * H * W / CN);
+    const int Nc = (int)oracle_num_chunks(T, H, W);
     cand_t* cand = (cand_t*)malloc(sizeof(cand_t) * (size_t)Nc);
     int32_t* pick = (int32_t*)malloc(sizeof(int32_t) * (size_t)Nc);
     if (!cand || !pick) {
@@ -247,7 +266,9 @@ int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, 
  * over the tokens of the chunks in CSR row r. All arithmetic in fp64.
  * out[n][l][:] is the output of local query l of rows[n]; lse[n][l] is the
  * natural-log log-sum-exp of the scaled logits (nullable). A row with no
- * selected chunk yields zeros and lse = -inf.
+ * selected chunk yields zeros and lse = -inf. Keys are the existing tokens of
+ * the selected chunks; a local query slot past the grid edge (partial chunk)
+ * has no output: NaN.
  */
 int oracle_attend(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int T, int H,
                   int W, int d, double scale, const int32_t* row_ptr, const int32_t* col_idx,
@@ -255,7 +276,7 @@ int oracle_attend(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B
     if (!q || !k || !v || !row_ptr || !col_idx || !rows || !out || BH <= 0 || d <= 0 ||
         !grid_ok(T, H, W))
         return -1;
-    const int64_t N = (int64_t)T * H * W, Nc = N / CN;
+    const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks(T, H, W);
     int bad = 0;
 #pragma omp parallel
     {
@@ -270,20 +291,22 @@ int oracle_attend(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B
             if (r < 0 || r >= (int64_t)BH * Nc) { bad = 1; continue; }
             const int64_t bh = r / Nc, i = r % Nc;
             const int64_t beg = row_ptr[r], end = row_ptr[r + 1];
-            const int64_t nk = (end - beg) * CN;
-            if (nk > cap_keys) {
+            const int64_t slots = (end - beg) * CN;
+            if (slots > cap_keys) {
                 free(kd); free(vd); free(s);
-                kd = (double*)malloc(sizeof(double) * (size_t)(nk * d));
-                vd = (double*)malloc(sizeof(double) * (size_t)(nk * d));
-                s = (double*)malloc(sizeof(double) * (size_t)nk);
-                cap_keys = nk;
+                kd = (double*)malloc(sizeof(double) * (size_t)(slots * d));
+                vd = (double*)malloc(sizeof(double) * (size_t)(slots * d));
+                s = (double*)malloc(sizeof(double) * (size_t)slots);
+                cap_keys = slots;
             }
-            /* keys: every token of every selected chunk */
+            /* keys: every existing token of every selected chunk */
+            int64_t nk = 0;
             for (int64_t e = beg; e < end; ++e) {
                 const int64_t c = col_idx[e];
                 for (int l = 0; l < CN; ++l) {
                     const int64_t tok = oracle_token_of(T, H, W, c, l);
-                    const int64_t j = (e - beg) * CN + l;
+                    if (tok < 0) continue;
+                    const int64_t j = nk++;
                     for (int x = 0; x < d; ++x) {
                         kd[j * d + x] = bf16_to_double(k[(bh * N + tok) * d + x]);
                         vd[j * d + x] = bf16_to_double(v[(bh * N + tok) * d + x]);
@@ -292,8 +315,13 @@ int oracle_attend(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B
             }
             for (int lq = 0; lq < CN; ++lq) {
                 const int64_t qtok = oracle_token_of(T, H, W, i, lq);
-                for (int x = 0; x < d; ++x) qd[x] = bf16_to_double(q[(bh * N + qtok) * d + x]);
                 double* o = out + (n * CN + lq) * d;
+                if (qtok < 0) {
+                    for (int x = 0; x < d; ++x) o[x] = NAN;
+                    if (lse) lse[n * CN + lq] = NAN;
+                    continue;
+                }
+                for (int x = 0; x < d; ++x) qd[x] = bf16_to_double(q[(bh * N + qtok) * d + x]);
                 if (nk == 0) {
                     for (int x = 0; x < d; ++x) o[x] = 0.0;
                     if (lse) lse[n * CN + lq] = -INFINITY;
@@ -400,7 +428,9 @@ int oracle_dense(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH
  * query l of rows[n]; dk and dv ([BH][N][d], zeroed by the caller) accumulate
  * the contributions of those rows only (complete for a key chunk when every
  * row that selects it is listed). A row with no selected chunk contributes
- * nothing and has dQ = 0. All arithmetic in fp64.
+ * nothing and has dQ = 0. Keys and queries are the existing tokens of their
+ * chunks; a local query slot past the grid edge has no dQ (NaN) and
+ * contributes nothing. All arithmetic in fp64.
  */
 int oracle_attend_bwd(const double* q, const double* k, const double* v, const double* dout,
                       int BH, int T, int H, int W, int d, double scale, const int32_t* row_ptr,
@@ -409,7 +439,7 @@ int oracle_attend_bwd(const double* q, const double* k, const double* v, const d
     if (!q || !k || !v || !dout || !row_ptr || !col_idx || !rows || !dq_rows || !dk || !dv ||
         BH <= 0 || d <= 0 || !grid_ok(T, H, W))
         return -1;
-    const int64_t N = (int64_t)T * H * W, Nc = N / CN;
+    const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks(T, H, W);
     for (int64_t n = 0; n < n_rows; ++n)
         if (rows[n] < 0 || rows[n] >= (int64_t)BH * Nc) return -1;
     int64_t cap_keys = 0;
@@ -420,29 +450,42 @@ int oracle_attend_bwd(const double* q, const double* k, const double* v, const d
         const int64_t r = rows[n];
         const int64_t bh = r / Nc, i = r % Nc;
         const int64_t beg = row_ptr[r], end = row_ptr[r + 1];
-        const int64_t nk = (end - beg) * CN;
+        const int64_t slots = (end - beg) * CN;
         double* dqr = dq_rows + n * CN * d;
+        if (slots > cap_keys) {
+            free(ktok); free(P); free(dS);
+            ktok = (int64_t*)malloc(sizeof(int64_t) * (size_t)slots);
+            P = (double*)malloc(sizeof(double) * (size_t)(CN * slots));
+            dS = (double*)malloc(sizeof(double) * (size_t)(CN * slots));
+            cap_keys = slots;
+        }
+        int64_t nk = 0;  /* existing key tokens of the row */
+        for (int64_t e = beg; e < end; ++e)
+            for (int l = 0; l < CN; ++l) {
+                const int64_t tok = oracle_token_of(T, H, W, col_idx[e], l);
+                if (tok >= 0) ktok[nk++] = bh * N + tok;
+            }
+        for (int lq = 0; lq < CN; ++lq)
+            if (oracle_token_of(T, H, W, i, lq) < 0)
+                for (int x = 0; x < d; ++x) dqr[(int64_t)lq * d + x] = NAN;
         if (nk <= 0) {
-            for (int64_t x = 0; x < (int64_t)CN * d; ++x) dqr[x] = 0.0;
+            for (int lq = 0; lq < CN; ++lq)
+                if (oracle_token_of(T, H, W, i, lq) >= 0)
+                    for (int x = 0; x < d; ++x) dqr[(int64_t)lq * d + x] = 0.0;
             continue;
         }
-        if (nk > cap_keys) {
-            free(ktok); free(P); free(dS);
-            ktok = (int64_t*)malloc(sizeof(int64_t) * (size_t)nk);
-            P = (double*)malloc(sizeof(double) * (size_t)(CN * nk));
-            dS = (double*)malloc(sizeof(double) * (size_t)(CN * nk));
-            cap_keys = nk;
-        }
-        for (int64_t e = beg; e < end; ++e)
-            for (int l = 0; l < CN; ++l)
-                ktok[(e - beg) * CN + l] = bh * N + oracle_token_of(T, H, W, col_idx[e], l);
         /* per query: softmax weights, O, D, dS and dQ */
 #pragma omp parallel for schedule(static)
         for (int lq = 0; lq < CN; ++lq) {
-            const double* qr = q + (bh * N + oracle_token_of(T, H, W, i, lq)) * d;
-            const double* gr = dout + (bh * N + oracle_token_of(T, H, W, i, lq)) * d;
+            const int64_t qtok = oracle_token_of(T, H, W, i, lq);
             double* p = P + (int64_t)lq * nk;
             double* ds = dS + (int64_t)lq * nk;
+            if (qtok < 0) {  /* no such query: no weights */
+                for (int64_t j = 0; j < nk; ++j) p[j] = ds[j] = 0.0;
+                continue;
+            }
+            const double* qr = q + (bh * N + qtok) * d;
+            const double* gr = dout + (bh * N + qtok) * d;
             double mx = -INFINITY;
             for (int64_t j = 0; j < nk; ++j) {
                 const double* kr = k + ktok[j] * d;
@@ -482,7 +525,9 @@ int oracle_attend_bwd(const double* q, const double* k, const double* v, const d
             double* dkr = dk + ktok[j] * d;
             double* dvr = dv + ktok[j] * d;
             for (int lq = 0; lq < CN; ++lq) {
-                const int64_t qt = bh * N + oracle_token_of(T, H, W, i, lq);
+                const int64_t qtok = oracle_token_of(T, H, W, i, lq);
+                if (qtok < 0) continue;
+                const int64_t qt = bh * N + qtok;
                 const double pw = P[(int64_t)lq * nk + j];
                 const double sw = dS[(int64_t)lq * nk + j] * scale;
                 const double* qr = q + qt * d;

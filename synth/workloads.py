@@ -35,18 +35,28 @@ class Workload:
         return self.T * self.H * self.W
 
     @property
+    def NH(self) -> int:
+        return -(-self.H // 4)
+
+    @property
+    def NW(self) -> int:
+        return -(-self.W // 8)
+
+    @property
     def Nc(self) -> int:
-        return (self.T // 4) * (self.H // 4) * (self.W // 8)
+        """Chunks per (batch, head): ceil(T/4) * ceil(H/4) * ceil(W/8); edge chunks of a
+        grid that is not a multiple of (4, 4, 8) are partial."""
+        return -(-self.T // 4) * self.NH * self.NW
 
     @property
     def n_cond(self) -> int:
         """Condition chunks: chunks whose 4 frames all lie below t_cond."""
-        return (self.t_cond // 4) * (self.H // 4) * (self.W // 8)
+        return (self.t_cond // 4) * self.NH * self.NW
 
     @property
     def q_skip(self) -> int:
         """Query chunks before q_begin (not computed)."""
-        return (self.q_begin // 4) * (self.H // 4) * (self.W // 8)
+        return (self.q_begin // 4) * self.NH * self.NW
 
     @property
     def Nq(self) -> int:
@@ -74,6 +84,12 @@ WORKLOADS = {
     # block-causal video continuation with CDF selection (p = 0.9, cap 25%)
     "causal_cdf": Workload("causal_cdf", B=2, heads=32, T=24, H=48, W=80, d=128,
                            mode="cdf", cdf_p=0.9, cdf_cap_frac=0.25, t_cond=8),
+    # the actual 720p token grid of the pages (1280x720 frames at 16x16 compression: 80x45
+    # tokens per latent frame, 93 frames -> 24 latent frames): H = 45 leaves a last chunk
+    # row of one token, so 80 of the 720 chunks are partial (32 of 128 tokens)
+    "720p_real": Workload("720p_real", B=1, heads=32, T=24, H=45, W=80, d=128, topk=45),
+    # 480p the same way (832x480 -> 52x30 tokens): partial chunks along H and W
+    "480p_real": Workload("480p_real", B=1, heads=32, T=24, H=30, W=52, d=128, topk=21),
     # 87.5 % sparsity (r = N_k / 8): 90 of 720 chunks
     "720p_r8": Workload("720p_r8", B=1, heads=32, T=24, H=48, W=80, d=128, topk=90),
     # combination of both rules: CDF p = 0.1 (29-66 chunks on these inputs, median 41)

@@ -89,6 +89,17 @@ def test_plan_sizes_topk_cdf_combination(L):
     assert ws_tc < ws_c   # padded rows hold min(k, cap) = 45 instead of 180 entries
 
 
+def test_plan_sizes_partial_edge_chunks(L):
+    # the actual 720p token grid 24 x 45 x 80: ceil(45/4) = 12 chunk rows, 720 chunks
+    rc, rows, nnz = rc_sizes(P(heads=32, T=24, H=45, W=80, d=128, topk=45))
+    assert (rc, rows, nnz) == (0, 32 * 720, 32 * 720 * 45)
+    # 5 x 7 x 9 tokens: 2 x 2 x 2 chunks, all partial
+    rc, rows, nnz = rc_sizes(P(heads=1, T=5, H=7, W=9, topk=3))
+    assert (rc, rows, nnz) == (0, 8, 24)
+    # a single token
+    assert rc_sizes(P(heads=1, T=1, H=1, W=1, topk=1))[:2] == (0, 1)
+
+
 def test_plan_sizes_kv_cached_step(L):
     # causal_cdf with only the noisy queries (frames >= 8): 480 of 720 rows per head
     rc, rows, nnz = rc_sizes(P(B=2, heads=32, T=24, H=48, W=80, d=128, mode="cdf", t_cond=8,
@@ -106,9 +117,9 @@ def test_plan_sizes_kv_cached_step(L):
     (dict(q_begin=2), bsa.BSA_ERR_SHAPE),
     (dict(q_begin=4), bsa.BSA_ERR_SHAPE),     # q_begin must leave at least one frame (T = 4)
     (dict(q_begin=-4), bsa.BSA_ERR_SHAPE),
-    (dict(T=6), bsa.BSA_ERR_SHAPE),
-    (dict(H=6), bsa.BSA_ERR_SHAPE),
-    (dict(W=12), bsa.BSA_ERR_SHAPE),
+    (dict(T=0), bsa.BSA_ERR_SHAPE),
+    (dict(H=-4), bsa.BSA_ERR_SHAPE),
+    (dict(W=0), bsa.BSA_ERR_SHAPE),
     (dict(B=0), bsa.BSA_ERR_SHAPE),
     (dict(d=96), bsa.BSA_ERR_UNSUPPORTED),
     (dict(t_cond=2), bsa.BSA_ERR_SHAPE),
@@ -187,7 +198,7 @@ def test_backward_workspace_size_layout(L):
     expect = 256 + r256(rows * 256 * 4) + r256(cols * words * 4) + 2 * r256(cols * 4) + \
         r256((cols + 1) * 4) + r256(rows * 720 * 4)
     assert bsa.bsa_backward_workspace_size(p) == expect
-    assert bsa.lib().bsa_backward_workspace_size(ctypes.byref(P(T=6))) == 0
+    assert bsa.lib().bsa_backward_workspace_size(ctypes.byref(P(T=0))) == 0
 
 
 def test_backward_host_checks_before_any_cuda_call(L):
@@ -205,7 +216,7 @@ def test_backward_host_checks_before_any_cuda_call(L):
         bsa.BSA_ERR_ALIGNMENT
     assert f(pp, x, x, x, x, x, x, x, x, 16, x, ws - 1, x, x, x, None) == \
         bsa.BSA_ERR_WORKSPACE_TOO_SMALL
-    assert f(ctypes.byref(P(T=6)), x, x, x, x, x, x, x, x, 16, x, ws, x, x, x, None) == \
+    assert f(ctypes.byref(P(T=0)), x, x, x, x, x, x, x, x, 16, x, ws, x, x, x, None) == \
         bsa.BSA_ERR_SHAPE
 
 
@@ -220,7 +231,7 @@ def test_no_cpu_fallback_without_a_gpu(L):
                     None)
     assert rc == bsa.BSA_ERR_CUDA
     with pytest.raises(bsa.BsaError):
-        bsa.bsa_plan_sizes(P(T=6))
+        bsa.bsa_plan_sizes(P(T=0))
 
 
 def test_unknown_selection_mode_rejected(L):

@@ -32,6 +32,8 @@ BWD_MEAN_REL = 1e-2
 def rel_errors(g, o):
     g = np.asarray(g, dtype=np.float64)
     o = np.asarray(o, dtype=np.float64)
+    live = ~np.isnan(o)            # slots of partial edge chunks past the grid: NaN
+    g, o = g[live], o[live]
     err = np.abs(g - o)
     return float(err.max() / max(np.abs(o).max(), 1e-30)), \
         float(err.mean() / max(np.abs(o).mean(), 1e-30))
@@ -170,12 +172,14 @@ def test_backward_deterministic():
         assert torch.equal(x.view(torch.int16), y.view(torch.int16))
 
 
-def test_backward_full_size_720p_sampled():
-    """Full 720p grid, 32 heads, in the launch configuration of the benchmark:
-    dQ of sampled rows and dK/dV of sampled key chunks of (batch 0, head 0)
-    against the oracle, plus the invariants sum(dK) = 0 and sum(dV) = sum(dO)
-    per head (every row is non-empty under top-k)."""
-    wl = W["720p"]
+@pytest.mark.parametrize("name", ["720p", "720p_real"])
+def test_backward_full_size_720p_sampled(name):
+    """Full 720p grids, 32 heads, in the launch configuration of the benchmark
+    (720p_real has partial edge chunks): dQ of sampled rows and dK/dV of a
+    sampled key chunk of (batch 0, head 0) against the oracle, plus the
+    invariants sum(dK) = 0 and sum(dV) = sum(dO) per head (every row is
+    non-empty under top-k)."""
+    wl = W[name]
     q, k, v = synth.make_qkv(wl)
     g = synth.make_dout(wl)
     scale = 1.0 / math.sqrt(wl.d)

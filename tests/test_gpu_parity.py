@@ -39,6 +39,11 @@ SMALL = {
     # combination mode where each rule binds on some rows: CDF counts 3-12 against k = 5 or 6
     "topk_cdf_small": W["tiny"].with_(name="topk_cdf_small", heads=2, T=8, H=16, W=32, d=128,
                                       mode="topk_cdf", topk=6, cdf_p=0.2, cdf_cap_frac=0.5),
+    # partial edge chunks: grids that are not multiples of (4, 4, 8)
+    "partial_topk": W["tiny"].with_(name="partial_topk", heads=2, T=6, H=10, W=20, d=64, topk=5),
+    "partial_causal_cdf": W["tiny"].with_(name="partial_causal_cdf", B=2, heads=2, T=10, H=13,
+                                          W=28, d=128, mode="cdf", cdf_p=0.9, cdf_cap_frac=0.25,
+                                          t_cond=4),
     "causal_topk_cdf": W["tiny"].with_(name="causal_topk_cdf", B=2, heads=2, T=16, H=16, W=32,
                                        d=64, mode="topk_cdf", topk=5, cdf_p=0.2,
                                        cdf_cap_frac=0.25, t_cond=8),
@@ -68,10 +73,15 @@ def run_gpu(wl, q, k, v):
 
 
 def gather_rows(x_bhnd, wl, rows):
-    """[B,Hh,N,d] (numpy) -> [len(rows), 128, d] in chunk-local order."""
+    """[B,Hh,N,d] (numpy) -> [len(rows), 128, d] in chunk-local order; NaN for the
+    slots of a partial edge chunk past the grid."""
     flat = x_bhnd.reshape(wl.B * wl.heads, wl.N, -1)
-    return np.stack([flat[r // wl.Nc][oracle.chunk_tokens(wl.T, wl.H, wl.W, r % wl.Nc)]
-                     for r in rows])
+    out = np.full((len(rows), 128, flat.shape[-1]), np.nan)
+    for n, r in enumerate(rows):
+        tok = oracle.chunk_tokens(wl.T, wl.H, wl.W, r % wl.Nc)
+        ok = tok >= 0
+        out[n][ok] = flat[r // wl.Nc][tok[ok]]
+    return out
 
 
 def check_case(wl, rows=None, qkv=None):
@@ -303,9 +313,10 @@ def _sample_rows(wl, per_head, seed=0):
     return np.array(sorted(rows), dtype=np.int64)
 
 
-@pytest.mark.parametrize("name,per_head", [("480p", 8), ("720p", 4), ("long", 2),
+@pytest.mark.parametrize("name,per_head", [("480p", 224), ("720p", 64), ("long", 2),
                                            ("causal_cdf", 2), ("720p_r8", 2),
-                                           ("720p_topk_cdf", 2)])
+                                           ("720p_topk_cdf", 2), ("720p_real", 4),
+                                           ("480p_real", 4)])
 def test_full_size_workloads(name, per_head):
     wl = W[name]
     check_case(wl, rows=_sample_rows(wl, per_head))
