@@ -67,12 +67,26 @@ def _load():
             lib.oracle_token_of.argtypes = [i32, i32, i32, i64, i32]
             lib.oracle_num_chunks.restype = i64
             lib.oracle_num_chunks.argtypes = [i32, i32, i32]
+            lib.oracle_num_chunks_shape.restype = i64
+            lib.oracle_num_chunks_shape.argtypes = [i32] * 6
+            lib.oracle_token_of_shape.restype = i64
+            lib.oracle_token_of_shape.argtypes = [i32] * 6 + [i64, i32]
+            lib.oracle_pool_shape.restype = i32
+            lib.oracle_pool_shape.argtypes = [vp] + [i32] * 9 + [vp]
+            lib.oracle_select_shape.restype = i64
+            lib.oracle_select_shape.argtypes = [vp] + [i32] * 10 + [dbl, dbl, i32, vp, vp, i64]
+            lib.oracle_attend_shape.restype = i32
+            lib.oracle_attend_shape.argtypes = [vp, vp, vp] + [i32] * 8 + [dbl, vp, vp, vp, i64,
+                                                                           vp, vp]
+            lib.oracle_attend_bwd_shape.restype = i32
+            lib.oracle_attend_bwd_shape.argtypes = [vp] * 4 + [i32] * 8 + [dbl, vp, vp, vp, i64,
+                                                                          vp, vp, vp]
             lib.oracle_rearrange.restype = i32
             lib.oracle_rearrange.argtypes = [vp, i32, i32, i32, i32, i32, vp]
             lib.oracle_pool.restype = i32
             lib.oracle_pool.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp]
             lib.oracle_scores.restype = i32
-            lib.oracle_scores.argtypes = [vp, vp, i32, i32, i32, dbl, i32, vp]
+            lib.oracle_scores.argtypes = [vp, vp, i32, i32, i32, i32, dbl, i32, vp]
             lib.oracle_select.restype = i64
             lib.oracle_select.argtypes = [vp, i32, i32, i32, i32, i32, i32, i32, dbl, dbl, i32,
                                           vp, vp, i64]
@@ -112,9 +126,9 @@ def token_of(T, H, W, c, l) -> int:
     return _load().oracle_token_of(T, H, W, c, l)
 
 
-def num_chunks(T, H, W) -> int:
-    """Chunks of the grid: ceil(T/4) * ceil(H/4) * ceil(W/8)."""
-    return _load().oracle_num_chunks(T, H, W)
+def num_chunks(T, H, W, chunk=CHUNK) -> int:
+    """Chunks of the grid: ceil(T/ct) * ceil(H/ch) * ceil(W/cw) (default (4,4,8))."""
+    return _load().oracle_num_chunks_shape(T, H, W, *chunk)
 
 
 def rearrange(x, T, H, W):
@@ -127,51 +141,55 @@ def rearrange(x, T, H, W):
     return out
 
 
-def pool(x, T, H, W, fp32=False):
-    """Chunk means [B, heads, Nc, d] (float64; float-valued when fp32)."""
+def pool(x, T, H, W, fp32=False, chunk=CHUNK):
+    """Chunk means [B, heads, Nc, d] (float64; float-valued when fp32) over chunks of
+    shape `chunk` (default the (4,4,8) query chunk)."""
     x = _u16(x)
     B, Hh, N, d = x.shape
-    out = np.empty((B, Hh, num_chunks(T, H, W), d), dtype=np.float64)
-    _check(_load().oracle_pool(x.ctypes.data, B * Hh, T, H, W, d, int(fp32), out.ctypes.data),
-           "oracle_pool")
+    out = np.empty((B, Hh, num_chunks(T, H, W, chunk), d), dtype=np.float64)
+    _check(_load().oracle_pool_shape(x.ctypes.data, B * Hh, T, H, W, *chunk, d, int(fp32),
+                                     out.ctypes.data), "oracle_pool")
     return out
 
 
 def scores(qp, kp, scale, fp32=False):
-    """Pooled scores [B, heads, Nc, Nc] = qp kp^T * scale."""
+    """Pooled scores [B, heads, Nq, Nk] = qp kp^T * scale."""
     qp = np.ascontiguousarray(qp, dtype=np.float64)
     kp = np.ascontiguousarray(kp, dtype=np.float64)
-    B, Hh, Nc, d = qp.shape
-    out = np.empty((B, Hh, Nc, Nc), dtype=np.float64)
-    _check(_load().oracle_scores(qp.ctypes.data, kp.ctypes.data, B * Hh, Nc, d, float(scale),
+    B, Hh, Nq, d = qp.shape
+    Nk = kp.shape[2]
+    out = np.empty((B, Hh, Nq, Nk), dtype=np.float64)
+    _check(_load().oracle_scores(qp.ctypes.data, kp.ctypes.data, B * Hh, Nq, Nk, d, float(scale),
                                  int(fp32), out.ctypes.data), "oracle_scores")
     return out
 
 
-def select(S, T, H, W, mode="topk", topk=0, cdf_p=0.9, cap_frac=0.25, t_cond=0, fp32=False):
-    """CSR (row_ptr int32 [rows+1], col_idx int32 [nnz]) of the selected chunks."""
+def select(S, T, H, W, mode="topk", topk=0, cdf_p=0.9, cap_frac=0.25, t_cond=0, fp32=False,
+           kchunk=CHUNK):
+    """CSR (row_ptr int32 [rows+1], col_idx int32 [nnz]) of the selected key chunks
+    (of shape `kchunk`) per (4,4,8) query chunk; S is [B, heads, Nq, Nk]."""
     S = np.ascontiguousarray(S, dtype=np.float64)
-    B, Hh, Nc, _ = S.shape
-    rows = B * Hh * Nc
+    B, Hh, Nq, Nk = S.shape
+    rows = B * Hh * Nq
     row_ptr = np.zeros(rows + 1, dtype=np.int32)
-    col_cap = rows * Nc
-    col_idx = np.empty(col_cap, dtype=np.int32)
-    nnz = _check(_load().oracle_select(S.ctypes.data, B * Hh, T, H, W, int(t_cond),
-                                       MODES[mode], int(topk), float(cdf_p),
-                                       float(cap_frac), int(fp32), row_ptr.ctypes.data,
-                                       col_idx.ctypes.data, col_cap), "oracle_select")
+    col_cap = rows * Nk
+    col_idx = np.empty(max(col_cap, 1), dtype=np.int32)
+    nnz = _check(_load().oracle_select_shape(S.ctypes.data, B * Hh, T, H, W, *kchunk,
+                                             int(t_cond), MODES[mode], int(topk), float(cdf_p),
+                                             float(cap_frac), int(fp32), row_ptr.ctypes.data,
+                                             col_idx.ctypes.data, col_cap), "oracle_select")
     return row_ptr, col_idx[:nnz].copy()
 
 
 def plan(q, k, T, H, W, scale, mode="topk", topk=0, cdf_p=0.9, cap_frac=0.25, t_cond=0,
-         fp32=False):
+         fp32=False, kchunk=CHUNK):
     """pool -> scores -> select; returns (row_ptr, col_idx, S)."""
-    S = scores(pool(q, T, H, W, fp32), pool(k, T, H, W, fp32), scale, fp32)
-    rp, ci = select(S, T, H, W, mode, topk, cdf_p, cap_frac, t_cond, fp32)
+    S = scores(pool(q, T, H, W, fp32), pool(k, T, H, W, fp32, kchunk), scale, fp32)
+    rp, ci = select(S, T, H, W, mode, topk, cdf_p, cap_frac, t_cond, fp32, kchunk)
     return rp, ci, S
 
 
-def attend(q, k, v, T, H, W, scale, row_ptr, col_idx, rows, want_lse=True):
+def attend(q, k, v, T, H, W, scale, row_ptr, col_idx, rows, want_lse=True, kchunk=CHUNK):
     """Sparse attention for the listed CSR rows: out [n, 128, d] f64, lse [n, 128]."""
     q, k, v = _u16(q), _u16(k), _u16(v)
     B, Hh, N, d = q.shape
@@ -182,10 +200,12 @@ def attend(q, k, v, T, H, W, scale, row_ptr, col_idx, rows, want_lse=True):
         ci = np.zeros(1, dtype=np.int32)
     out = np.empty((rows.size, CN, d), dtype=np.float64)
     lse = np.empty((rows.size, CN), dtype=np.float64) if want_lse else None
-    _check(_load().oracle_attend(q.ctypes.data, k.ctypes.data, v.ctypes.data, B * Hh, T, H, W, d,
-                                 float(scale), rp.ctypes.data, ci.ctypes.data, rows.ctypes.data,
-                                 rows.size, out.ctypes.data,
-                                 lse.ctypes.data if lse is not None else None), "oracle_attend")
+    _check(_load().oracle_attend_shape(q.ctypes.data, k.ctypes.data, v.ctypes.data, B * Hh, T, H,
+                                       W, *kchunk, d, float(scale), rp.ctypes.data,
+                                       ci.ctypes.data, rows.ctypes.data, rows.size,
+                                       out.ctypes.data,
+                                       lse.ctypes.data if lse is not None else None),
+           "oracle_attend")
     return out, lse
 
 
@@ -197,7 +217,7 @@ def _f64(a):
     return np.ascontiguousarray(a, dtype=np.float64)
 
 
-def attend_bwd(q, k, v, dout, T, H, W, scale, row_ptr, col_idx, rows):
+def attend_bwd(q, k, v, dout, T, H, W, scale, row_ptr, col_idx, rows, kchunk=CHUNK):
     """Gradients of ``attend`` for upstream gradient ``dout`` (same shape as q).
 
     Inputs: bf16 bit patterns (uint16) or float arrays [B, heads, N, d].
@@ -215,11 +235,11 @@ def attend_bwd(q, k, v, dout, T, H, W, scale, row_ptr, col_idx, rows):
     dq = np.empty((rows.size, CN, d), dtype=np.float64)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
-    _check(_load().oracle_attend_bwd(q.ctypes.data, k.ctypes.data, v.ctypes.data,
-                                     dout.ctypes.data, B * Hh, T, H, W, d, float(scale),
-                                     rp.ctypes.data, ci.ctypes.data, rows.ctypes.data, rows.size,
-                                     dq.ctypes.data, dk.ctypes.data, dv.ctypes.data),
-           "oracle_attend_bwd")
+    _check(_load().oracle_attend_bwd_shape(q.ctypes.data, k.ctypes.data, v.ctypes.data,
+                                           dout.ctypes.data, B * Hh, T, H, W, *kchunk, d,
+                                           float(scale), rp.ctypes.data, ci.ctypes.data,
+                                           rows.ctypes.data, rows.size, dq.ctypes.data,
+                                           dk.ctypes.data, dv.ctypes.data), "oracle_attend_bwd")
     return dq, dk, dv
 
 
@@ -237,7 +257,9 @@ def dense(q, k, v, T, H, W, scale, qtok, t_cond=0, want_lse=True):
     return out, lse
 
 
-def chunk_tokens(T, H, W, c):
-    """Token indices (THW order) of the 128 local slots of chunk c (-1 for a
-    slot past the grid edge of a partial chunk)."""
-    return np.array([token_of(T, H, W, c, l) for l in range(CN)], dtype=np.int64)
+def chunk_tokens(T, H, W, c, chunk=CHUNK):
+    """Token indices (THW order) of the local slots of chunk c of shape `chunk`
+    (default (4,4,8): 128 slots), -1 for a slot past the grid edge."""
+    n = chunk[0] * chunk[1] * chunk[2]
+    return np.array([_load().oracle_token_of_shape(T, H, W, *chunk, c, l) for l in range(n)],
+                    dtype=np.int64)

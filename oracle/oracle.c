@@ -53,22 +53,33 @@ static inline double bf16_to_double(uint16_t b) {
 
 static int ceil_div(int n, int c) { return (n + c - 1) / c; }
 
-/* [P1] 3D block partitioning: chunks per axis by ceiling division. */
-int64_t oracle_num_chunks(int T, int H, int W) {
-    return (int64_t)ceil_div(T, CT) * ceil_div(H, CH) * ceil_div(W, CW);
+/* [P1] 3D block partitioning with blocks of shape (st, sh, sw): chunks per axis
+ * by ceiling division. */
+int64_t oracle_num_chunks_shape(int T, int H, int W, int st, int sh, int sw) {
+    return (int64_t)ceil_div(T, st) * ceil_div(H, sh) * ceil_div(W, sw);
 }
 
-/* [P1] 3D block partitioning: token index (THW order) of local token `l` of
- * chunk `c`, or -1 when that slot of a partial edge chunk lies past the grid. */
-int64_t oracle_token_of(int T, int H, int W, int64_t c, int l) {
-    const int NH = ceil_div(H, CH), NW = ceil_div(W, CW);
+/* Token index (THW order) of local slot l = (lt*sh + lh)*sw + lw of chunk c of
+ * shape (st, sh, sw), or -1 when that slot of a partial edge chunk lies past
+ * the grid. */
+int64_t oracle_token_of_shape(int T, int H, int W, int st, int sh, int sw, int64_t c, int l) {
+    const int NH = ceil_div(H, sh), NW = ceil_div(W, sw);
     const int64_t ct = c / ((int64_t)NH * NW);
     const int ch = (int)((c / NW) % NH);
     const int cw = (int)(c % NW);
-    const int lt = l / (CH * CW), lh = (l / CW) % CH, lw = l % CW;
-    const int64_t t = ct * CT + lt, h = (int64_t)ch * CH + lh, w = (int64_t)cw * CW + lw;
+    const int lt = l / (sh * sw), lh = (l / sw) % sh, lw = l % sw;
+    const int64_t t = ct * st + lt, h = (int64_t)ch * sh + lh, w = (int64_t)cw * sw + lw;
     if (t >= T || h >= H || w >= W) return -1;
     return (t * H + h) * W + w;
+}
+
+/* The query chunk shape (4,4,8) of [P3]: */
+int64_t oracle_num_chunks(int T, int H, int W) {
+    return oracle_num_chunks_shape(T, H, W, CT, CH, CW);
+}
+
+int64_t oracle_token_of(int T, int H, int W, int64_t c, int l) {
+    return oracle_token_of_shape(T, H, W, CT, CH, CW, c, l);
 }
 
 static int grid_ok(int T, int H, int W) { return T > 0 && H > 0 && W > 0; }
@@ -95,9 +106,12 @@ int oracle_rearrange(const uint16_t* x, int BH, int T, int H, int W, int d, uint
 /* [P1] pooled representations: mean of the token vectors of a chunk (its
  * existing tokens: 128, fewer for a partial edge chunk). pooled[bh][c][:].
  * fp32 != 0: accumulate in float in local-token order. */
-int oracle_pool(const uint16_t* x, int BH, int T, int H, int W, int d, int fp32, double* pooled) {
-    if (!x || !pooled || BH <= 0 || d <= 0 || !grid_ok(T, H, W)) return -1;
-    const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks(T, H, W);
+int oracle_pool_shape(const uint16_t* x, int BH, int T, int H, int W, int st, int sh, int sw,
+                      int d, int fp32, double* pooled) {
+    if (!x || !pooled || BH <= 0 || d <= 0 || !grid_ok(T, H, W) || st <= 0 || sh <= 0 || sw <= 0)
+        return -1;
+    const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks_shape(T, H, W, st, sh, sw);
+    const int n_slots = st * sh * sw;
 #pragma omp parallel for collapse(2) schedule(static)
     for (int bh = 0; bh < BH; ++bh)
         for (int64_t c = 0; c < Nc; ++c) {
@@ -106,8 +120,8 @@ int oracle_pool(const uint16_t* x, int BH, int T, int H, int W, int d, int fp32,
                 double acc = 0.0;
                 float accf = 0.0f;
                 int n = 0;
-                for (int l = 0; l < CN; ++l) {
-                    const int64_t tok = oracle_token_of(T, H, W, c, l);
+                for (int l = 0; l < n_slots; ++l) {
+                    const int64_t tok = oracle_token_of_shape(T, H, W, st, sh, sw, c, l);
                     if (tok < 0) continue;
                     const double v = bf16_to_double(x[((int64_t)bh * N + tok) * d + e]);
                     if (fp32) accf += (float)v; else acc += v;
@@ -119,16 +133,21 @@ int oracle_pool(const uint16_t* x, int BH, int T, int H, int W, int d, int fp32,
     return 0;
 }
 
-/* [P1] S_pool = Q_pool K_pool^T / sqrt(d) (scale passed in). S[bh][i][m]. */
-int oracle_scores(const double* qp, const double* kp, int BH, int Nc, int d, double scale,
+int oracle_pool(const uint16_t* x, int BH, int T, int H, int W, int d, int fp32, double* pooled) {
+    return oracle_pool_shape(x, BH, T, H, W, CT, CH, CW, d, fp32, pooled);
+}
+
+/* [P1] S_pool = Q_pool K_pool^T / sqrt(d) (scale passed in). S[bh][i][m] for Nq
+ * query chunks and Nk key chunks. */
+int oracle_scores(const double* qp, const double* kp, int BH, int Nq, int Nk, int d, double scale,
                   int fp32, double* S) {
-    if (!qp || !kp || !S || BH <= 0 || Nc <= 0 || d <= 0) return -1;
+    if (!qp || !kp || !S || BH <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return -1;
 #pragma omp parallel for collapse(2) schedule(static)
     for (int bh = 0; bh < BH; ++bh)
-        for (int i = 0; i < Nc; ++i) {
-            const double* q = qp + ((int64_t)bh * Nc + i) * d;
-            for (int m = 0; m < Nc; ++m) {
-                const double* k = kp + ((int64_t)bh * Nc + m) * d;
+        for (int i = 0; i < Nq; ++i) {
+            const double* q = qp + ((int64_t)bh * Nq + i) * d;
+            for (int m = 0; m < Nk; ++m) {
+                const double* k = kp + ((int64_t)bh * Nk + m) * d;
                 double s;
                 if (fp32) {
                     float a = 0.0f;
@@ -139,7 +158,7 @@ int oracle_scores(const double* qp, const double* kp, int BH, int Nc, int d, dou
                     for (int e = 0; e < d; ++e) a += q[e] * k[e];
                     s = a * scale;
                 }
-                S[((int64_t)bh * Nc + i) * Nc + m] = s;
+                S[((int64_t)bh * Nq + i) * Nk + m] = s;
             }
         }
     return 0;
@@ -147,9 +166,9 @@ int oracle_scores(const double* qp, const double* kp, int BH, int Nc, int d, dou
 
 /* [P1] block-causal attention: a chunk is a condition chunk when every frame of
  * it lies below t_cond. */
-static int is_condition_chunk(int H, int W, int64_t c, int t_cond) {
-    const int64_t ct = c / ((int64_t)ceil_div(H, CH) * ceil_div(W, CW));
-    return (ct * CT + CT - 1) < t_cond;
+static int is_condition_chunk(int H, int W, int st, int sh, int sw, int64_t c, int t_cond) {
+    const int64_t ct = c / ((int64_t)ceil_div(H, sh) * ceil_div(W, sw));
+    return (ct * st + st - 1) < t_cond;
 }
 
 typedef struct {
@@ -183,15 +202,17 @@ static int int_cmp(const void* a, const void* b) {
  * Column indices of a row are written in ascending order.
  * Returns nnz >= 0, or -1 on bad arguments, -2 if col_cap is too small.
  */
-int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, int mode,
-                      int topk, double cdf_p, double cap_frac, int fp32, int32_t* row_ptr,
-                      int32_t* col_idx, int64_t col_cap) {
+int64_t oracle_select_shape(const double* S, int BH, int T, int H, int W, int kst, int ksh, int ksw,
+                            int t_cond, int mode, int topk, double cdf_p, double cap_frac, int fp32,
+                            int32_t* row_ptr, int32_t* col_idx, int64_t col_cap) {
     if (!S || !row_ptr || !col_idx || BH <= 0 || !grid_ok(T, H, W) || t_cond < 0 ||
-        t_cond % CT != 0 || mode < 0 || mode > 2 || (mode != 1 && topk <= 0))
+        t_cond % CT != 0 || kst <= 0 || ksh <= 0 || ksw <= 0 || t_cond % kst != 0 || mode < 0 ||
+        mode > 2 || (mode != 1 && topk <= 0))
         return -1;
-    const int Nc = (int)oracle_num_chunks(T, H, W);
-    cand_t* cand = (cand_t*)malloc(sizeof(cand_t) * (size_t)Nc);
-    int32_t* pick = (int32_t*)malloc(sizeof(int32_t) * (size_t)Nc);
+    const int Nq = (int)oracle_num_chunks(T, H, W);                       /* query chunks */
+    const int Nk = (int)oracle_num_chunks_shape(T, H, W, kst, ksh, ksw);  /* key chunks */
+    cand_t* cand = (cand_t*)malloc(sizeof(cand_t) * (size_t)Nk);
+    int32_t* pick = (int32_t*)malloc(sizeof(int32_t) * (size_t)Nk);
     if (!cand || !pick) {
         free(cand);
         free(pick);
@@ -200,12 +221,12 @@ int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, 
     int64_t nnz = 0;
     row_ptr[0] = 0;
     for (int bh = 0; bh < BH; ++bh) {
-        for (int i = 0; i < Nc; ++i) {
-            const double* row = S + ((int64_t)bh * Nc + i) * Nc;
-            const int q_cond = t_cond > 0 && is_condition_chunk(H, W, i, t_cond);
+        for (int i = 0; i < Nq; ++i) {
+            const double* row = S + ((int64_t)bh * Nq + i) * Nk;
+            const int q_cond = t_cond > 0 && is_condition_chunk(H, W, CT, CH, CW, i, t_cond);
             int na = 0;
-            for (int m = 0; m < Nc; ++m) {
-                if (q_cond && !is_condition_chunk(H, W, m, t_cond)) continue;
+            for (int m = 0; m < Nk; ++m) {
+                if (q_cond && !is_condition_chunk(H, W, kst, ksh, ksw, m, t_cond)) continue;
                 cand[na].s = row[m];
                 cand[na].idx = m;
                 ++na;
@@ -252,12 +273,19 @@ int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, 
             qsort(pick, (size_t)count, sizeof(int32_t), int_cmp);
             memcpy(col_idx + nnz, pick, sizeof(int32_t) * (size_t)count);
             nnz += count;
-            row_ptr[(int64_t)bh * Nc + i + 1] = (int32_t)nnz;
+            row_ptr[(int64_t)bh * Nq + i + 1] = (int32_t)nnz;
         }
     }
     free(cand);
     free(pick);
     return nnz;
+}
+
+int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, int mode,
+                      int topk, double cdf_p, double cap_frac, int fp32, int32_t* row_ptr,
+                      int32_t* col_idx, int64_t col_cap) {
+    return oracle_select_shape(S, BH, T, H, W, CT, CH, CW, t_cond, mode, topk, cdf_p, cap_frac,
+                               fp32, row_ptr, col_idx, col_cap);
 }
 
 /*
@@ -270,12 +298,14 @@ int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, 
  * the selected chunks; a local query slot past the grid edge (partial chunk)
  * has no output: NaN.
  */
-int oracle_attend(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int T, int H,
-                  int W, int d, double scale, const int32_t* row_ptr, const int32_t* col_idx,
-                  const int64_t* rows, int64_t n_rows, double* out, double* lse) {
+int oracle_attend_shape(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int T,
+                        int H, int W, int kst, int ksh, int ksw, int d, double scale,
+                        const int32_t* row_ptr, const int32_t* col_idx, const int64_t* rows,
+                        int64_t n_rows, double* out, double* lse) {
     if (!q || !k || !v || !row_ptr || !col_idx || !rows || !out || BH <= 0 || d <= 0 ||
-        !grid_ok(T, H, W))
+        !grid_ok(T, H, W) || kst <= 0 || ksh <= 0 || ksw <= 0)
         return -1;
+    const int kn = kst * ksh * ksw;  /* slots of a key chunk */
     const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks(T, H, W);
     int bad = 0;
 #pragma omp parallel
@@ -291,7 +321,7 @@ int oracle_attend(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B
             if (r < 0 || r >= (int64_t)BH * Nc) { bad = 1; continue; }
             const int64_t bh = r / Nc, i = r % Nc;
             const int64_t beg = row_ptr[r], end = row_ptr[r + 1];
-            const int64_t slots = (end - beg) * CN;
+            const int64_t slots = (end - beg) * kn;
             if (slots > cap_keys) {
                 free(kd); free(vd); free(s);
                 kd = (double*)malloc(sizeof(double) * (size_t)(slots * d));
@@ -303,8 +333,8 @@ int oracle_attend(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B
             int64_t nk = 0;
             for (int64_t e = beg; e < end; ++e) {
                 const int64_t c = col_idx[e];
-                for (int l = 0; l < CN; ++l) {
-                    const int64_t tok = oracle_token_of(T, H, W, c, l);
+                for (int l = 0; l < kn; ++l) {
+                    const int64_t tok = oracle_token_of_shape(T, H, W, kst, ksh, ksw, c, l);
                     if (tok < 0) continue;
                     const int64_t j = nk++;
                     for (int x = 0; x < d; ++x) {
@@ -350,6 +380,13 @@ int oracle_attend(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B
         free(kd); free(vd); free(s); free(qd);
     }
     return bad ? -1 : 0;
+}
+
+int oracle_attend(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int T, int H,
+                  int W, int d, double scale, const int32_t* row_ptr, const int32_t* col_idx,
+                  const int64_t* rows, int64_t n_rows, double* out, double* lse) {
+    return oracle_attend_shape(q, k, v, BH, T, H, W, CT, CH, CW, d, scale, row_ptr, col_idx, rows,
+                               n_rows, out, lse);
 }
 
 /*
@@ -432,13 +469,15 @@ int oracle_dense(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH
  * chunks; a local query slot past the grid edge has no dQ (NaN) and
  * contributes nothing. All arithmetic in fp64.
  */
-int oracle_attend_bwd(const double* q, const double* k, const double* v, const double* dout,
-                      int BH, int T, int H, int W, int d, double scale, const int32_t* row_ptr,
-                      const int32_t* col_idx, const int64_t* rows, int64_t n_rows,
-                      double* dq_rows, double* dk, double* dv) {
+int oracle_attend_bwd_shape(const double* q, const double* k, const double* v, const double* dout,
+                            int BH, int T, int H, int W, int kst, int ksh, int ksw, int d,
+                            double scale, const int32_t* row_ptr, const int32_t* col_idx,
+                            const int64_t* rows, int64_t n_rows, double* dq_rows, double* dk,
+                            double* dv) {
     if (!q || !k || !v || !dout || !row_ptr || !col_idx || !rows || !dq_rows || !dk || !dv ||
-        BH <= 0 || d <= 0 || !grid_ok(T, H, W))
+        BH <= 0 || d <= 0 || !grid_ok(T, H, W) || kst <= 0 || ksh <= 0 || ksw <= 0)
         return -1;
+    const int kn = kst * ksh * ksw;  /* slots of a key chunk */
     const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks(T, H, W);
     for (int64_t n = 0; n < n_rows; ++n)
         if (rows[n] < 0 || rows[n] >= (int64_t)BH * Nc) return -1;
@@ -450,7 +489,7 @@ int oracle_attend_bwd(const double* q, const double* k, const double* v, const d
         const int64_t r = rows[n];
         const int64_t bh = r / Nc, i = r % Nc;
         const int64_t beg = row_ptr[r], end = row_ptr[r + 1];
-        const int64_t slots = (end - beg) * CN;
+        const int64_t slots = (end - beg) * kn;
         double* dqr = dq_rows + n * CN * d;
         if (slots > cap_keys) {
             free(ktok); free(P); free(dS);
@@ -461,8 +500,8 @@ int oracle_attend_bwd(const double* q, const double* k, const double* v, const d
         }
         int64_t nk = 0;  /* existing key tokens of the row */
         for (int64_t e = beg; e < end; ++e)
-            for (int l = 0; l < CN; ++l) {
-                const int64_t tok = oracle_token_of(T, H, W, col_idx[e], l);
+            for (int l = 0; l < kn; ++l) {
+                const int64_t tok = oracle_token_of_shape(T, H, W, kst, ksh, ksw, col_idx[e], l);
                 if (tok >= 0) ktok[nk++] = bh * N + tok;
             }
         for (int lq = 0; lq < CN; ++lq)
@@ -541,6 +580,14 @@ int oracle_attend_bwd(const double* q, const double* k, const double* v, const d
     }
     free(ktok); free(P); free(dS);
     return 0;
+}
+
+int oracle_attend_bwd(const double* q, const double* k, const double* v, const double* dout,
+                      int BH, int T, int H, int W, int d, double scale, const int32_t* row_ptr,
+                      const int32_t* col_idx, const int64_t* rows, int64_t n_rows,
+                      double* dq_rows, double* dk, double* dv) {
+    return oracle_attend_bwd_shape(q, k, v, dout, BH, T, H, W, CT, CH, CW, d, scale, row_ptr,
+                                   col_idx, rows, n_rows, dq_rows, dk, dv);
 }
 
 int oracle_num_threads(void) {
