@@ -54,20 +54,23 @@ class bsa_params(ctypes.Structure):
                 ("chunk_w", ctypes.c_int32), ("scale", ctypes.c_float), ("mode", ctypes.c_int32),
                 ("topk", ctypes.c_int32), ("cdf_p", ctypes.c_float),
                 ("cdf_cap_frac", ctypes.c_float), ("t_cond", ctypes.c_int32),
-                ("q_begin", ctypes.c_int32)]
+                ("q_begin", ctypes.c_int32), ("kchunk_t", ctypes.c_int32),
+                ("kchunk_h", ctypes.c_int32), ("kchunk_w", ctypes.c_int32)]
 
 
 def make_params(B, heads, T, H, W, d, mode="topk", topk=1, cdf_p=0.9, cdf_cap_frac=0.25,
-                t_cond=0, scale=0.0, q_begin=0) -> bsa_params:
+                t_cond=0, scale=0.0, q_begin=0, kchunk=(0, 0, 0)) -> bsa_params:
+    """kchunk: key chunk shape (t, h, w); 0 on an axis = the query chunk's (4, 4, 8)."""
     return bsa_params(B, heads, T, H, W, d, 4, 4, 8, float(scale),
                       MODES[mode], int(topk), float(cdf_p),
-                      float(cdf_cap_frac), int(t_cond), int(q_begin))
+                      float(cdf_cap_frac), int(t_cond), int(q_begin), *map(int, kchunk))
 
 
 def params_for(wl) -> bsa_params:
     """Parameters of a workload description (anything with the Workload fields)."""
     return make_params(wl.B, wl.heads, wl.T, wl.H, wl.W, wl.d, wl.mode, wl.topk, wl.cdf_p,
-                       wl.cdf_cap_frac, wl.t_cond, q_begin=getattr(wl, "q_begin", 0))
+                       wl.cdf_cap_frac, wl.t_cond, q_begin=getattr(wl, "q_begin", 0),
+                       kchunk=getattr(wl, "kchunk", (0, 0, 0)))
 
 
 _lib = None

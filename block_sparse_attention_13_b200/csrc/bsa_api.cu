@@ -13,6 +13,8 @@ namespace bsa {
 
 static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+static int64_t max_key_nnz_of(const Dims& g, const bsa_params& p);
+
 WsLayout ws_layout(const Dims& g, const bsa_params& p) {
     WsLayout L{};
     size_t off = 0;
@@ -21,21 +23,32 @@ WsLayout ws_layout(const Dims& g, const bsa_params& p) {
     L.qpool = off;
     off += round_up((size_t)g.BH * g.Nq * g.d * sizeof(float), 256);
     L.kpool = off;
-    off += round_up((size_t)g.BH * g.Nc * g.d * sizeof(float), 256);
+    off += round_up((size_t)g.BH * g.Nk * g.d * sizeof(float), 256);
     L.scores = off;
-    off += round_up((size_t)g.BH * g.Nq * g.Nc * sizeof(float), 256);
+    off += round_up((size_t)g.BH * g.Nq * g.Nk * sizeof(float), 256);
     L.pad_stride = 0;
-    L.counts = L.padded = off;
-    if (p.mode != BSA_SEL_TOPK) {
-        int cap = (int)std::floor((double)p.cdf_cap_frac * g.Nc);
-        if (cap < 1) cap = 1;
-        if (cap > g.Nc) cap = g.Nc;
-        if (p.mode == BSA_SEL_TOPK_CDF && p.topk < cap) cap = p.topk;
-        L.pad_stride = cap;
+    L.counts = L.padded = L.kc_row_ptr = L.kc_col_idx = off;
+    L.kc_cap = 0;
+    if (p.mode != BSA_SEL_TOPK || g.m > 1) {
         L.counts = off;
         off += round_up((size_t)g.rows * sizeof(int32_t), 256);
+    }
+    if (p.mode != BSA_SEL_TOPK) {
+        int cap = (int)std::floor((double)p.cdf_cap_frac * g.Nk);
+        if (cap < 1) cap = 1;
+        if (cap > g.Nk) cap = g.Nk;
+        if (p.mode == BSA_SEL_TOPK_CDF && p.topk < cap) cap = p.topk;
+        L.pad_stride = cap;
         L.padded = off;
         off += round_up((size_t)g.rows * cap * sizeof(int32_t), 256);
+    }
+    if (g.m > 1) {
+        // selection in key chunks first, then the expansion to (4,4,8) boxes
+        L.kc_cap = max_key_nnz_of(g, p);
+        L.kc_row_ptr = off;
+        off += round_up((size_t)(g.rows + 1) * sizeof(int32_t), 256);
+        L.kc_col_idx = off;
+        off += round_up((size_t)(L.kc_cap > 0 ? L.kc_cap : 1) * sizeof(int32_t), 256);
     }
     L.total = off;
     return L;
@@ -50,6 +63,14 @@ static int make_dims(const bsa_params* p, Dims* g) {
         return BSA_ERR_UNSUPPORTED;
     if (p->d != 64 && p->d != 128) return BSA_ERR_UNSUPPORTED;
     if (p->t_cond < 0 || p->t_cond % kChunkT || p->t_cond > p->T) return BSA_ERR_SHAPE;
+    // key chunk shape: 0 = the query chunk's size on that axis; otherwise a
+    // positive multiple of it, at most 8 boxes of (4,4,8) in all
+    const int kt = p->kchunk_t ? p->kchunk_t : kChunkT, kh = p->kchunk_h ? p->kchunk_h : kChunkH,
+              kw = p->kchunk_w ? p->kchunk_w : kChunkW;
+    if (kt < 0 || kh < 0 || kw < 0 || kt % kChunkT || kh % kChunkH || kw % kChunkW)
+        return BSA_ERR_UNSUPPORTED;
+    if ((kt / kChunkT) * (kh / kChunkH) * (kw / kChunkW) > 8) return BSA_ERR_UNSUPPORTED;
+    if (p->t_cond % kt) return BSA_ERR_SHAPE;
     if (p->q_begin < 0 || p->q_begin % kChunkT || p->q_begin >= p->T) return BSA_ERR_SHAPE;
     if (!(std::isfinite(p->scale)) || p->scale < 0.f) return BSA_ERR_INVALID_ARG;
     if (p->mode == BSA_SEL_TOPK || p->mode == BSA_SEL_TOPK_CDF) {
@@ -80,6 +101,15 @@ static int make_dims(const bsa_params* p, Dims* g) {
     // and CSR offsets are int32.
     if (nc > 2048 || g->BH > 65535) return BSA_ERR_UNSUPPORTED;
     g->Nc = (int)nc;
+    g->mT = kt / kChunkT;
+    g->mH = kh / kChunkH;
+    g->mW = kw / kChunkW;
+    g->m = g->mT * g->mH * g->mW;
+    g->NkT = (g->NT + g->mT - 1) / g->mT;
+    g->NkH = (g->NH + g->mH - 1) / g->mH;
+    g->NkW = (g->NW + g->mW - 1) / g->mW;
+    g->Nk = g->NkT * g->NkH * g->NkW;
+    g->n_cond_k = (p->t_cond / kt) * g->NkH * g->NkW;
     g->q_skip = (p->q_begin / kChunkT) * g->NH * g->NW;
     g->Nq = g->Nc - g->q_skip;
     g->rows = g->BH * g->Nq;
@@ -94,15 +124,16 @@ static int make_dims(const bsa_params* p, Dims* g) {
 static int64_t cond_rows(const Dims& g) { return g.n_cond > g.q_skip ? g.n_cond - g.q_skip : 0; }
 static int64_t noisy_rows(const Dims& g) { return g.Nq - cond_rows(g); }
 
-static int64_t max_nnz_of(const Dims& g, const bsa_params& p) {
+// CSR entries in key chunks (exact for TOPK, an upper bound otherwise).
+static int64_t max_key_nnz_of(const Dims& g, const bsa_params& p) {
     if (p.mode == BSA_SEL_TOPK) {
-        const int64_t kc = p.topk < g.n_cond ? p.topk : g.n_cond;
-        const int64_t kn = p.topk < g.Nc ? p.topk : g.Nc;
+        const int64_t kc = p.topk < g.n_cond_k ? p.topk : g.n_cond_k;
+        const int64_t kn = p.topk < g.Nk ? p.topk : g.Nk;
         return g.BH * (cond_rows(g) * kc + noisy_rows(g) * kn);
     }
     int64_t total = 0;
     for (int which = 0; which < 2; ++which) {
-        const int na = which == 0 ? g.n_cond : g.Nc;
+        const int na = which == 0 ? g.n_cond_k : g.Nk;
         const int64_t nrows = which == 0 ? cond_rows(g) : noisy_rows(g);
         if (nrows == 0) continue;
         int cap = (int)std::floor((double)p.cdf_cap_frac * na);
@@ -112,6 +143,9 @@ static int64_t max_nnz_of(const Dims& g, const bsa_params& p) {
     }
     return g.BH * total;
 }
+
+// CSR entries in (4,4,8) boxes: a key chunk covers at most m of them.
+static int64_t max_nnz_of(const Dims& g, const bsa_params& p) { return max_key_nnz_of(g, p) * g.m; }
 
 static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
@@ -187,10 +221,19 @@ int bsa_plan(const bsa_params* p, const void* q, const void* k, void* workspace,
     uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
     if ((rc = cuda_status(launch_pool(g, q, k, qp, kp, st))) != BSA_OK) return rc;
     if ((rc = cuda_status(launch_scores(g, qp, kp, S, st))) != BSA_OK) return rc;
-    return cuda_status(launch_select(g, *p, S, row_ptr, col_idx, col_capacity,
-                                     reinterpret_cast<int32_t*>(ws + L.counts),
-                                     reinterpret_cast<int32_t*>(ws + L.padded), L.pad_stride,
-                                     status, st));
+    int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+    int32_t* padded = reinterpret_cast<int32_t*>(ws + L.padded);
+    if (g.m == 1)
+        return cuda_status(launch_select(g, *p, S, row_ptr, col_idx, col_capacity, counts, padded,
+                                         L.pad_stride, status, st));
+    // key chunks larger than the query chunk: select key chunks, then list their boxes
+    int32_t* kc_rp = reinterpret_cast<int32_t*>(ws + L.kc_row_ptr);
+    int32_t* kc_ci = reinterpret_cast<int32_t*>(ws + L.kc_col_idx);
+    if ((rc = cuda_status(launch_select(g, *p, S, kc_rp, kc_ci, L.kc_cap, counts, padded,
+                                        L.pad_stride, status, st))) != BSA_OK)
+        return rc;
+    return cuda_status(launch_expand_boxes(g, kc_rp, kc_ci, counts, row_ptr, col_idx, col_capacity,
+                                           status, st));
 }
 
 // Internal: forward with a custom wait limit and debug flags (used by the

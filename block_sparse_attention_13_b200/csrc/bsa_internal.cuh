@@ -29,23 +29,30 @@ __host__ __device__ __forceinline__ uint32_t site(int role, int bar, int tile, i
 // Derived sizes of one call.
 struct Dims {
     int B, heads, T, H, W, d;
-    int NT, NH, NW, Nc;
+    int NT, NH, NW, Nc;  // query chunks ((4,4,8) boxes) per axis and per (batch, head)
     int64_t N, BH, rows;
-    int n_cond;      // condition chunks per (batch, head); 0 without block-causal mask
+    int n_cond;      // condition query chunks per (batch, head); 0 without block-causal mask
     int q_skip;      // query chunks before q_begin (not computed)
     int Nq;          // query chunks computed per (batch, head): Nc - q_skip
+    // key chunks: mT x mH x mW boxes each (1x1x1 unless the key chunk is larger)
+    int mT, mH, mW, m;
+    int NkT, NkH, NkW, Nk;
+    int n_cond_k;    // condition key chunks per (batch, head)
     float scale;
 };
 
 // Workspace layout (byte offsets), identical for plan and forward.
 struct WsLayout {
     size_t status;   // uint32 status word (+ padding to 256)
-    size_t qpool;    // float [BH][Nc][d]
-    size_t kpool;    // float [BH][Nc][d]
-    size_t scores;   // float [BH][Nc][Nc]
-    size_t counts;   // int32 [rows]            (CDF only)
+    size_t qpool;    // float [BH][Nq][d]
+    size_t kpool;    // float [BH][Nk][d]
+    size_t scores;   // float [BH][Nq][Nk]
+    size_t counts;   // int32 [rows]            (CDF and box expansion)
     size_t padded;   // int32 [rows][pad_stride] (CDF only)
     int pad_stride;  // max chunks a CDF row may keep
+    size_t kc_row_ptr;  // int32 [rows+1]   key-chunk CSR before box expansion (m > 1)
+    size_t kc_col_idx;  // int32 [kc_cap]
+    int64_t kc_cap;
     size_t total;
 };
 
@@ -87,6 +94,11 @@ cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const vo
 // call failed.
 bool make_chunk_map(CUtensorMap* tm, const void* base, const Dims& g, int box_t = kChunkT);
 cudaError_t launch_scan_counts(const int32_t* counts, int64_t n, int32_t* ptr, cudaStream_t st);
+// Key-chunk CSR -> CSR over the (4,4,8) boxes each selected key chunk covers.
+cudaError_t launch_expand_boxes(const Dims& g, const int32_t* kc_row_ptr,
+                                const int32_t* kc_col_idx, int32_t* counts, int32_t* row_ptr,
+                                int32_t* col_idx, int64_t col_cap, uint32_t* status,
+                                cudaStream_t st);
 cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const void* v,
                             const void* out, const float* lse, const void* dout,
                             const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,

@@ -37,14 +37,22 @@ __device__ __forceinline__ void add_bf16x2(float& a, float& b, uint32_t u) {
 // read consecutive 16-byte vectors, so every warp load is one contiguous
 // 512-byte run. Each thread always covers the same 8 channels and sums them
 // over its tokens in fp32; a shared-memory pass finishes the 128-token sum.
-// Tensor z (blockIdx.z) pools chunks [c_begin_z, c_begin_z + n_z) into rows
-// 0 .. n_z-1 of its output.
+// Tensor z (blockIdx.z) pools chunks [c_begin, c_begin + n_out) of its own
+// chunk grid into rows 0 .. n_out-1 of its output. A chunk is mt x mh x mw
+// (4,4,8) boxes (a key chunk can be larger than the query chunk); a partial
+// edge chunk averages the tokens it has.
+struct PoolSide {
+    int c_begin, n_out;
+    int mt, mh, mw;  // boxes per chunk along t, h, w
+    int NHc, NWc;    // chunks of this grid along h, w
+};
+
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ x0,
                                                    const __nv_bfloat16* __restrict__ x1,
                                                    float* __restrict__ p0, float* __restrict__ p1,
-                                                   int c_begin0, int n0, int c_begin1, int n1,
-                                                   int T, int H, int W, int NH, int NW, int64_t N) {
+                                                   PoolSide s0, PoolSide s1, int T, int H, int W,
+                                                   int64_t N) {
     constexpr int VPT = D / 8;               // 16-byte vectors per token row
     constexpr int ITERS = 128 * VPT / 256;   // vectors per thread
     constexpr int GROUPS = 256 / VPT;        // threads that share one channel group
@@ -52,36 +60,42 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 
     const __nv_bfloat16* x = blockIdx.z ? x1 : x0;
     float* pooled = blockIdx.z ? p1 : p0;
-    const int n_out = blockIdx.z ? n1 : n0;
-    if (static_cast<int>(blockIdx.x) >= n_out) return;
-    const int c = (blockIdx.z ? c_begin1 : c_begin0) + blockIdx.x;
+    const PoolSide sd = blockIdx.z ? s1 : s0;
+    if (static_cast<int>(blockIdx.x) >= sd.n_out) return;
+    const int c = sd.c_begin + blockIdx.x;
     const int64_t bh = blockIdx.y;
-    const int ct = c / (NH * NW), ch = (c / NW) % NH, cw = c % NW;
+    const int ct = c / (sd.NHc * sd.NWc), ch = (c / sd.NWc) % sd.NHc, cw = c % sd.NWc;
     const int tid = threadIdx.x;
     const int dvec = tid % VPT;
-    // a partial edge chunk (grid not a multiple of the chunk shape) averages the
-    // tokens it has
-    const int nt = min(kChunkT, T - ct * kChunkT), nh = min(kChunkH, H - ch * kChunkH),
-              nw = min(kChunkW, W - cw * kChunkW);
 
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
     const __nv_bfloat16* base = x + bh * N * D;
+    int n_tok = 0;
+    for (int bt = 0; bt < sd.mt; ++bt)
+        for (int bhh = 0; bhh < sd.mh; ++bhh)
+            for (int bw = 0; bw < sd.mw; ++bw) {
+                const int t0 = (ct * sd.mt + bt) * kChunkT, h0 = (ch * sd.mh + bhh) * kChunkH,
+                          w0 = (cw * sd.mw + bw) * kChunkW;
+                const int nt = min(kChunkT, T - t0), nh = min(kChunkH, H - h0),
+                          nw = min(kChunkW, W - w0);
+                if (nt <= 0 || nh <= 0 || nw <= 0) continue;  // box past the grid
+                n_tok += nt * nh * nw;
 #pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-        const int v = it * 256 + tid;
-        const int l = v / VPT;  // local token (lt*4 + lh)*8 + lw
-        const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
-        if (lt >= nt || lh >= nh || lw >= nw) continue;
-        const int64_t tok =
-            ((int64_t)(ct * kChunkT + lt) * H + (ch * kChunkH + lh)) * W + cw * kChunkW + lw;
-        const uint4 u = ld_nc_v4(base + tok * D + dvec * 8);
-        add_bf16x2(acc[0], acc[1], u.x);
-        add_bf16x2(acc[2], acc[3], u.y);
-        add_bf16x2(acc[4], acc[5], u.z);
-        add_bf16x2(acc[6], acc[7], u.w);
-    }
+                for (int it = 0; it < ITERS; ++it) {
+                    const int v = it * 256 + tid;
+                    const int l = v / VPT;  // local token (lt*4 + lh)*8 + lw
+                    const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
+                    if (lt >= nt || lh >= nh || lw >= nw) continue;
+                    const int64_t tok = ((int64_t)(t0 + lt) * H + (h0 + lh)) * W + w0 + lw;
+                    const uint4 u = ld_nc_v4(base + tok * D + dvec * 8);
+                    add_bf16x2(acc[0], acc[1], u.x);
+                    add_bf16x2(acc[2], acc[3], u.y);
+                    add_bf16x2(acc[4], acc[5], u.z);
+                    add_bf16x2(acc[6], acc[7], u.w);
+                }
+            }
     const int grp = tid / VPT;
 #pragma unroll
     for (int e = 0; e < 8; ++e) red[grp][dvec * 8 + e] = acc[e];
@@ -90,7 +104,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
         float s = 0.f;
 #pragma unroll
         for (int g2 = 0; g2 < GROUPS; ++g2) s += red[g2][tid];
-        pooled[(bh * n_out + blockIdx.x) * D + tid] = s * (1.0f / static_cast<float>(nt * nh * nw));
+        pooled[(bh * sd.n_out + blockIdx.x) * D + tid] = s * (1.0f / static_cast<float>(n_tok));
     }
 }
 
@@ -236,20 +250,24 @@ __device__ __forceinline__ uint32_t kth_largest_key(const uint32_t (&key)[MAXJ],
     return v;
 }
 
+// One warp per CSR row. Query chunks are numbered on the (4,4,8) grid (Ncq per
+// (batch, head), the first n_cond_q of them condition chunks); candidates are
+// the Nk key chunks (the first n_cond_k of them condition chunks), which are
+// the query chunks themselves unless the key chunk shape is larger.
 template <int MAXJ>
 __global__ void __launch_bounds__(256) select_kernel(
-    const float* __restrict__ S, int Nc, int n_cond, int q_skip, int64_t rows, int mode, int topk,
-    float cdf_p, float cap_frac, int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
-    int64_t col_cap, int32_t* __restrict__ counts, int32_t* __restrict__ padded, int pad_stride,
-    uint32_t* status) {
+    const float* __restrict__ S, int Ncq, int Nk, int n_cond_q, int n_cond_k, int q_skip,
+    int64_t rows, int mode, int topk, float cdf_p, float cap_frac, int32_t* __restrict__ row_ptr,
+    int32_t* __restrict__ col_idx, int64_t col_cap, int32_t* __restrict__ counts,
+    int32_t* __restrict__ padded, int pad_stride, uint32_t* status) {
     const int lane = threadIdx.x & 31;
     const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (w >= rows) return;
-    const int Nq = Nc - q_skip;                 // computed query chunks per (batch, head)
+    const int Nq = Ncq - q_skip;                // computed query chunks per (batch, head)
     const int64_t bh = w / Nq;
     const int i = q_skip + (int)(w % Nq);       // query chunk of this row
-    const int na = (n_cond > 0 && i < n_cond) ? n_cond : Nc;  // candidates are [0, na)
-    const float* srow = S + w * (int64_t)Nc;
+    const int na = (n_cond_q > 0 && i < n_cond_q) ? n_cond_k : Nk;  // candidates are [0, na)
+    const float* srow = S + w * (int64_t)Nk;
 
     uint32_t key[MAXJ];
 #pragma unroll
@@ -329,14 +347,14 @@ __global__ void __launch_bounds__(256) select_kernel(
     int32_t* dst;
     int64_t off;
     if (mode == BSA_SEL_TOPK) {
-        const int kc = topk < n_cond ? topk : n_cond;
-        const int kn = topk < Nc ? topk : Nc;
-        // rows of a (batch, head): condition rows q_skip .. n_cond-1, then noisy rows
-        const int c_rows = n_cond > q_skip ? n_cond - q_skip : 0;
-        const int first_noisy = n_cond > q_skip ? n_cond : q_skip;
-        const int64_t per_bh = (int64_t)c_rows * kc + (int64_t)(Nc - first_noisy) * kn;
-        off = bh * per_bh + (i < n_cond ? (int64_t)(i - q_skip) * kc
-                                        : (int64_t)c_rows * kc + (int64_t)(i - first_noisy) * kn);
+        const int kc = topk < n_cond_k ? topk : n_cond_k;
+        const int kn = topk < Nk ? topk : Nk;
+        // rows of a (batch, head): condition rows q_skip .. n_cond_q-1, then noisy rows
+        const int c_rows = n_cond_q > q_skip ? n_cond_q - q_skip : 0;
+        const int first_noisy = n_cond_q > q_skip ? n_cond_q : q_skip;
+        const int64_t per_bh = (int64_t)c_rows * kc + (int64_t)(Ncq - first_noisy) * kn;
+        off = bh * per_bh + (i < n_cond_q ? (int64_t)(i - q_skip) * kc
+                                          : (int64_t)c_rows * kc + (int64_t)(i - first_noisy) * kn);
         if (off + count > col_cap) {
             if (lane == 0) atomicOr(status, kStatusCapacity);
             return;
@@ -424,6 +442,82 @@ __global__ void __launch_bounds__(256) compact_kernel(const int32_t* __restrict_
     for (int e = lane; e < n; e += 32) col_idx[off + e] = padded[w * (int64_t)pad_stride + e];
 }
 
+// ------------------------------------------------------------------------
+// Key chunks larger than the query chunk: each selected key chunk is replaced
+// by the (4,4,8) boxes it covers inside the grid (box ids on the query-chunk
+// grid), so the attention kernels see a CSR over 128-token boxes.
+struct BoxGrid {
+    int NT, NH, NW;     // boxes per axis
+    int mT, mH, mW;     // boxes per key chunk per axis
+    int NkH, NkW, Nk;   // key chunks along h, w and in total
+};
+
+__device__ __forceinline__ void key_chunk_boxes(const BoxGrid& g, int kc, int& t0, int& h0, int& w0,
+                                                int& nt, int& nh, int& nw) {
+    const int kct = kc / (g.NkH * g.NkW), kch = (kc / g.NkW) % g.NkH, kcw = kc % g.NkW;
+    t0 = kct * g.mT;
+    h0 = kch * g.mH;
+    w0 = kcw * g.mW;
+    nt = min(g.mT, g.NT - t0);
+    nh = min(g.mH, g.NH - h0);
+    nw = min(g.mW, g.NW - w0);
+}
+
+// One warp per row: boxes of the row's key chunks.
+__global__ void __launch_bounds__(256) expand_count_kernel(const int32_t* __restrict__ kc_row_ptr,
+                                                           const int32_t* __restrict__ kc_col_idx,
+                                                           int64_t rows, BoxGrid g,
+                                                           int32_t* __restrict__ counts) {
+    const int lane = threadIdx.x & 31;
+    const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (w >= rows) return;
+    int n = 0;
+    for (int64_t e = kc_row_ptr[w] + lane; e < kc_row_ptr[w + 1]; e += 32) {
+        int t0, h0, w0, nt, nh, nw;
+        key_chunk_boxes(g, kc_col_idx[e], t0, h0, w0, nt, nh, nw);
+        n += nt * nh * nw;
+    }
+    n = __reduce_add_sync(0xffffffffu, n);
+    if (lane == 0) counts[w] = n;
+}
+
+// One warp per row: each lane writes the boxes of one key chunk, key chunks in
+// row order, boxes in (t, h, w) order inside a key chunk.
+__global__ void __launch_bounds__(256) expand_emit_kernel(const int32_t* __restrict__ kc_row_ptr,
+                                                          const int32_t* __restrict__ kc_col_idx,
+                                                          int64_t rows, BoxGrid g,
+                                                          const int32_t* __restrict__ row_ptr,
+                                                          int32_t* __restrict__ col_idx,
+                                                          int64_t col_cap, uint32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (w >= rows) return;
+    if (row_ptr[w + 1] > col_cap) {
+        if (lane == 0) atomicOr(status, kStatusCapacity);
+        return;
+    }
+    int64_t run = row_ptr[w];
+    const int64_t beg = kc_row_ptr[w], end = kc_row_ptr[w + 1];
+    for (int64_t e0 = beg; e0 < end; e0 += 32) {
+        const int64_t e = e0 + lane;
+        int t0 = 0, h0 = 0, w0 = 0, nt = 0, nh = 0, nw = 0;
+        if (e < end) key_chunk_boxes(g, kc_col_idx[e], t0, h0, w0, nt, nh, nw);
+        const int n = nt * nh * nw;
+        int incl = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int64_t pos = run + (incl - n);
+        for (int a = 0; a < nt; ++a)
+            for (int b = 0; b < nh; ++b)
+                for (int c = 0; c < nw; ++c)
+                    col_idx[pos++] = ((t0 + a) * g.NH + (h0 + b)) * g.NW + (w0 + c);
+        run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+}
+
 // One CTA waits on an mbarrier that nothing arrives at; the bounded wait
 // expires, records the timeout and the kernel returns normally.
 __global__ void selftest_timeout_kernel(uint32_t* status, uint64_t timeout_ns) {
@@ -444,17 +538,17 @@ __global__ void selftest_timeout_kernel(uint32_t* status, uint64_t timeout_ns) {
 cudaError_t launch_pool(const Dims& g, const void* x0, const void* x1, float* p0, float* p1,
                         cudaStream_t st) {
     // with two tensors (plan): x0 = Q pools the computed query chunks, x1 = K
-    // pools every chunk; with one tensor it pools every chunk of x0
-    dim3 grid(g.Nc, (unsigned)g.BH, x1 ? 2 : 1);
+    // pools every key chunk; with one tensor it pools every query chunk of x0
+    const PoolSide sq{x1 ? g.q_skip : 0, x1 ? g.Nq : g.Nc, 1, 1, 1, g.NH, g.NW};
+    const PoolSide sk{0, g.Nk, g.mT, g.mH, g.mW, g.NkH, g.NkW};
+    const int nx = x1 ? (g.Nq > g.Nk ? g.Nq : g.Nk) : g.Nc;
+    dim3 grid((unsigned)nx, (unsigned)g.BH, x1 ? 2 : 1);
     const auto* a = static_cast<const __nv_bfloat16*>(x0);
     const auto* b = static_cast<const __nv_bfloat16*>(x1 ? x1 : x0);
-    const int c0 = x1 ? g.q_skip : 0, n0 = x1 ? g.Nq : g.Nc;
     if (g.d == 128)
-        pool_kernel<128><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, c0, n0, 0, g.Nc, g.T, g.H,
-                                               g.W, g.NH, g.NW, g.N);
+        pool_kernel<128><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, sq, sk, g.T, g.H, g.W, g.N);
     else
-        pool_kernel<64><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, c0, n0, 0, g.Nc, g.T, g.H,
-                                              g.W, g.NH, g.NW, g.N);
+        pool_kernel<64><<<grid, 256, 0, st>>>(a, b, p0, p1 ? p1 : p0, sq, sk, g.T, g.H, g.W, g.N);
     return cudaGetLastError();
 }
 
@@ -474,8 +568,8 @@ cudaError_t launch_rearrange(const Dims& g, const void* src, void* dst, int inve
 
 cudaError_t launch_scores(const Dims& g, const float* qp, const float* kp, float* S,
                           cudaStream_t st) {
-    dim3 grid((g.Nc + 63) / 64, (g.Nq + 63) / 64, (unsigned)g.BH);
-    scores_kernel<<<grid, 256, 0, st>>>(qp, kp, S, g.Nq, g.Nc, g.d, g.scale);
+    dim3 grid((g.Nk + 63) / 64, (g.Nq + 63) / 64, (unsigned)g.BH);
+    scores_kernel<<<grid, 256, 0, st>>>(qp, kp, S, g.Nq, g.Nk, g.d, g.scale);
     return cudaGetLastError();
 }
 
@@ -485,13 +579,14 @@ cudaError_t launch_select(const Dims& g, const bsa_params& p, const float* S, in
     const unsigned blocks = (unsigned)((g.rows + 7) / 8);
     const int mode = p.mode;
 #define BSA_SELECT(MJ)                                                                       \
-    select_kernel<MJ><<<blocks, 256, 0, st>>>(S, g.Nc, g.n_cond, g.q_skip, g.rows, mode, p.topk, \
-                                              p.cdf_p, p.cdf_cap_frac, row_ptr, col_idx,    \
-                                              col_cap, counts, padded, pad_stride, status)
-    if (g.Nc <= 32) BSA_SELECT(1);
-    else if (g.Nc <= 256) BSA_SELECT(8);
-    else if (g.Nc <= 1024) BSA_SELECT(32);
-    else if (g.Nc <= 2048) BSA_SELECT(64);
+    select_kernel<MJ><<<blocks, 256, 0, st>>>(S, g.Nc, g.Nk, g.n_cond, g.n_cond_k, g.q_skip,   \
+                                              g.rows, mode, p.topk, p.cdf_p, p.cdf_cap_frac, \
+                                              row_ptr, col_idx, col_cap, counts, padded,     \
+                                              pad_stride, status)
+    if (g.Nk <= 32) BSA_SELECT(1);
+    else if (g.Nk <= 256) BSA_SELECT(8);
+    else if (g.Nk <= 1024) BSA_SELECT(32);
+    else if (g.Nk <= 2048) BSA_SELECT(64);
     else return cudaErrorInvalidValue;
 #undef BSA_SELECT
     cudaError_t e = cudaGetLastError();
@@ -506,6 +601,22 @@ cudaError_t launch_select(const Dims& g, const bsa_params& p, const float* S, in
 
 cudaError_t launch_scan_counts(const int32_t* counts, int64_t n, int32_t* ptr, cudaStream_t st) {
     scan_counts_kernel<<<1, 1024, 0, st>>>(counts, n, ptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_expand_boxes(const Dims& g, const int32_t* kc_row_ptr,
+                                const int32_t* kc_col_idx, int32_t* counts, int32_t* row_ptr,
+                                int32_t* col_idx, int64_t col_cap, uint32_t* status,
+                                cudaStream_t st) {
+    const BoxGrid bg{g.NT, g.NH, g.NW, g.mT, g.mH, g.mW, g.NkH, g.NkW, g.Nk};
+    const unsigned blocks = (unsigned)((g.rows + 7) / 8);
+    expand_count_kernel<<<blocks, 256, 0, st>>>(kc_row_ptr, kc_col_idx, g.rows, bg, counts);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    scan_counts_kernel<<<1, 1024, 0, st>>>(counts, g.rows, row_ptr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    expand_emit_kernel<<<blocks, 256, 0, st>>>(kc_row_ptr, kc_col_idx, g.rows, bg, row_ptr,
+                                               col_idx, col_cap, status);
     return cudaGetLastError();
 }
 

@@ -86,6 +86,16 @@ typedef struct {
                          * [B,heads,T*H*W,d] buffer. Row r of the CSR is query chunk
                          * q_begin/4*(H/4)*(W/8) + r % Nq of (batch, head) r / Nq, where
                          * Nq = Nc - q_begin/4*(H/4)*(W/8). */
+    int32_t kchunk_t, kchunk_h, kchunk_w;
+                        /* key chunk shape; 0 on an axis = the query chunk's size (4, 4, 8).
+                         * Otherwise a multiple of it on that axis, at most 8 (4,4,8) boxes
+                         * in all (key chunks of 128..1024 tokens: [P1]'s block-size
+                         * robustness study; [P3]'s general kernel for key chunks above
+                         * 128 tokens). K is pooled per key chunk, the scores are
+                         * [Nq x Nk] and selection keeps topk KEY chunks per query chunk
+                         * (t_cond must be a multiple of kchunk_t); the CSR that bsa_plan
+                         * writes then lists the (4,4,8) boxes those key chunks cover, the
+                         * unit bsa_forward / bsa_backward attend over. */
 } bsa_params;
 
 /* Library version: major*10000 + minor*100 + patch. */
@@ -100,8 +110,9 @@ BSA_API const char* bsa_status_string(int status);
 BSA_API size_t bsa_workspace_size(const bsa_params* p);
 
 /* CSR sizes for `p`: *n_rows = B*heads*Nq (Nq = query chunks from q_begin on,
- * Nc when q_begin = 0); *max_nnz = col_idx capacity that
- * always suffices (exact for TOPK; upper bound for CDF). Host-only call. */
+ * Nc when q_begin = 0); *max_nnz = col_idx capacity that always suffices, in
+ * (4,4,8) boxes (exact for TOPK with the default key chunk; an upper bound
+ * otherwise). Host-only call. */
 BSA_API int bsa_plan_sizes(const bsa_params* p, int64_t* n_rows, int64_t* max_nnz);
 
 /*

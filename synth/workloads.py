@@ -26,6 +26,7 @@ class Workload:
     cdf_cap_frac: float = 0.25
     t_cond: int = 0             # latent frames of condition tokens (block-causal mask)
     q_begin: int = 0            # first latent frame whose queries are computed (KV-cached step)
+    kchunk: tuple = (4, 4, 8)   # key chunk shape (multiples of the (4,4,8) query chunk)
     tfreq_mult: float = 1.0     # temporal frequency multiplier of the smooth field
     seed: int = 0
     cond_seed: int = 1
@@ -52,6 +53,18 @@ class Workload:
     def n_cond(self) -> int:
         """Condition chunks: chunks whose 4 frames all lie below t_cond."""
         return (self.t_cond // 4) * self.NH * self.NW
+
+    @property
+    def Nk(self) -> int:
+        """Key chunks per (batch, head)."""
+        kt, kh, kw = self.kchunk
+        return -(-self.T // kt) * -(-self.H // kh) * -(-self.W // kw)
+
+    @property
+    def n_cond_k(self) -> int:
+        """Condition key chunks."""
+        kt, kh, kw = self.kchunk
+        return (self.t_cond // kt) * -(-self.H // kh) * -(-self.W // kw)
 
     @property
     def q_skip(self) -> int:
@@ -90,6 +103,9 @@ WORKLOADS = {
     "720p_real": Workload("720p_real", B=1, heads=32, T=24, H=45, W=80, d=128, topk=45),
     # 480p the same way (832x480 -> 52x30 tokens): partial chunks along H and W
     "480p_real": Workload("480p_real", B=1, heads=32, T=24, H=30, W=52, d=128, topk=21),
+    # key chunks of 512 tokens (8,8,8) over the 720p-like grid: 180 key chunks, keep 11 (93.9 %)
+    "720p_k512": Workload("720p_k512", B=1, heads=32, T=24, H=48, W=80, d=128, topk=11,
+                          kchunk=(8, 8, 8)),
     # 87.5 % sparsity (r = N_k / 8): 90 of 720 chunks
     "720p_r8": Workload("720p_r8", B=1, heads=32, T=24, H=48, W=80, d=128, topk=90),
     # combination of both rules: CDF p = 0.1 (29-66 chunks on these inputs, median 41)

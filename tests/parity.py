@@ -24,8 +24,11 @@ def rows_of(row_ptr, col_idx):
     return [ci[rp[r]:rp[r + 1]] for r in range(len(rp) - 1)]
 
 
-def _candidates(i, Nc, n_cond):
-    return np.arange(n_cond if (n_cond > 0 and i < n_cond) else Nc)
+def _candidates(i, Nk, n_cond, n_cond_k=None):
+    """Key chunks a query chunk i may select: the condition key chunks for a
+    condition query chunk, all Nk otherwise."""
+    n_cond_k = n_cond if n_cond_k is None else n_cond_k
+    return np.arange(n_cond_k if (n_cond > 0 and i < n_cond) else Nk)
 
 
 def _tied(a, b):
@@ -70,9 +73,12 @@ def cdf_count_ok(count, s64, cand, p, cap_frac, k=None):
 
 
 def compare_csr(gpu_rp, gpu_ci, ora_rp, ora_ci, S64, Nc, n_cond, mode, p=0.9, cap_frac=0.25,
-                rows=None, topk=None):
-    """Returns (n_rows_checked, n_rows_differing); asserts validity of every row."""
-    S64 = np.asarray(S64).reshape(-1, Nc, Nc)
+                rows=None, topk=None, Nk=None, n_cond_k=None):
+    """Returns (n_rows_checked, n_rows_differing); asserts validity of every row.
+    Rows are (batch, head, query chunk) with Nc query chunks per head; columns are
+    key chunks (Nk of them, Nc unless key chunks are larger)."""
+    Nk = Nc if Nk is None else Nk
+    S64 = np.asarray(S64).reshape(-1, Nc, Nk)
     g_rows, o_rows = rows_of(gpu_rp, gpu_ci), rows_of(ora_rp, ora_ci)
     assert len(g_rows) == len(o_rows)
     idx = range(len(g_rows)) if rows is None else rows
@@ -84,7 +90,7 @@ def compare_csr(gpu_rp, gpu_ci, ora_rp, ora_ci, S64, Nc, n_cond, mode, p=0.9, ca
         ndiff += 1
         i = r % Nc
         s64 = S64[r // Nc, i]
-        cand = _candidates(i, Nc, n_cond)
+        cand = _candidates(i, Nk, n_cond, n_cond_k)
         assert valid_topk_set(g, s64, cand), f"row {r}: gpu {g} vs oracle {o} not a tie"
         if mode == "topk":
             assert len(g) == len(o), f"row {r}: count {len(g)} vs {len(o)}"

@@ -100,6 +100,33 @@ def test_plan_sizes_partial_edge_chunks(L):
     assert rc_sizes(P(heads=1, T=1, H=1, W=1, topk=1))[:2] == (0, 1)
 
 
+def test_plan_sizes_key_chunks(L):
+    # 720p-like grid with (8,8,8) key chunks (2 x 2 x 1 boxes): 180 key chunks, keep 11 -> 44 boxes
+    rc, rows, nnz = rc_sizes(P(heads=32, T=24, H=48, W=80, d=128, topk=11, kchunk=(8, 8, 8)))
+    assert (rc, rows, nnz) == (0, 23040, 23040 * 11 * 4)
+    # (4,8,8) (2 boxes) on the block-causal grid: 360 key chunks, 120 of them condition
+    # chunks; condition rows keep min(k, 120)
+    rc, rows, nnz = rc_sizes(P(heads=1, T=24, H=48, W=80, d=128, topk=150, t_cond=8,
+                               kchunk=(4, 8, 8)))
+    assert (rc, nnz) == (0, (240 * 120 + 480 * 150) * 2)
+    ws = bsa.bsa_workspace_size(P(heads=32, T=24, H=48, W=80, d=128, topk=11, kchunk=(8, 8, 8)))
+    kpool, scores = 32 * 180 * 128 * 4, 32 * 720 * 180 * 4
+    assert ws >= 256 + 32 * 720 * 128 * 4 + kpool + scores
+
+
+@pytest.mark.parametrize("kchunk,code", [((4, 4, 12), bsa.BSA_ERR_UNSUPPORTED),
+                                         ((6, 4, 8), bsa.BSA_ERR_UNSUPPORTED),
+                                         ((8, 8, 16), 0), ((16, 8, 16), bsa.BSA_ERR_UNSUPPORTED),
+                                         ((-4, 4, 8), bsa.BSA_ERR_UNSUPPORTED)])
+def test_key_chunk_shape_validation(L, kchunk, code):
+    assert rc_sizes(P(T=16, H=16, W=32, kchunk=kchunk))[0] == code
+
+
+def test_key_chunk_needs_t_cond_multiple(L):
+    assert rc_sizes(P(T=16, H=16, W=32, t_cond=4, kchunk=(8, 4, 8)))[0] == bsa.BSA_ERR_SHAPE
+    assert rc_sizes(P(T=16, H=16, W=32, t_cond=8, kchunk=(8, 4, 8)))[0] == 0
+
+
 def test_plan_sizes_kv_cached_step(L):
     # causal_cdf with only the noisy queries (frames >= 8): 480 of 720 rows per head
     rc, rows, nnz = rc_sizes(P(B=2, heads=32, T=24, H=48, W=80, d=128, mode="cdf", t_cond=8,

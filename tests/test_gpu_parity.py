@@ -39,6 +39,14 @@ SMALL = {
     # combination mode where each rule binds on some rows: CDF counts 3-12 against k = 5 or 6
     "topk_cdf_small": W["tiny"].with_(name="topk_cdf_small", heads=2, T=8, H=16, W=32, d=128,
                                       mode="topk_cdf", topk=6, cdf_p=0.2, cdf_cap_frac=0.5),
+    # key chunks larger than the query chunk (256, 512, 1024 tokens), incl. partial ones
+    "kchunk_256": W["tiny"].with_(name="kchunk_256", heads=2, T=8, H=16, W=32, d=64, topk=3,
+                                  kchunk=(4, 8, 8)),
+    "kchunk_512_partial": W["tiny"].with_(name="kchunk_512_partial", heads=2, T=10, H=13, W=37,
+                                          d=128, topk=3, kchunk=(8, 8, 8)),
+    "kchunk_1024_causal_cdf": W["tiny"].with_(name="kchunk_1024_causal_cdf", B=2, heads=2, T=16,
+                                              H=16, W=64, d=64, mode="cdf", cdf_p=0.9,
+                                              cdf_cap_frac=0.5, t_cond=8, kchunk=(8, 8, 16)),
     # partial edge chunks: grids that are not multiples of (4, 4, 8)
     "partial_topk": W["tiny"].with_(name="partial_topk", heads=2, T=6, H=10, W=20, d=64, topk=5),
     "partial_causal_cdf": W["tiny"].with_(name="partial_causal_cdf", B=2, heads=2, T=10, H=13,
@@ -84,17 +92,39 @@ def gather_rows(x_bhnd, wl, rows):
     return out
 
 
+def boxes_to_key_chunks(rp, ci, wl):
+    """The GPU's CSR over (4,4,8) boxes -> the key chunks they came from (the boxes of
+    one key chunk are listed consecutively)."""
+    mt, mh, mw = wl.kchunk[0] // 4, wl.kchunk[1] // 4, wl.kchunk[2] // 8
+    NH, NW = wl.NH, wl.NW
+    NkH, NkW = -(-wl.H // wl.kchunk[1]), -(-wl.W // wl.kchunk[2])
+    b = np.asarray(ci, dtype=np.int64)
+    key = ((b // (NH * NW)) // mt * NkH + (b // NW) % NH // mh) * NkW + (b % NW) // mw
+    rows = []
+    for r in range(len(rp) - 1):
+        kr = key[rp[r]:rp[r + 1]]
+        keep = np.ones(len(kr), dtype=bool)
+        keep[1:] = kr[1:] != kr[:-1]
+        rows.append(kr[keep])
+    krp = np.concatenate([[0], np.cumsum([len(x) for x in rows])]).astype(np.int32)
+    return krp, (np.concatenate(rows) if rows else np.zeros(0)).astype(np.int32)
+
+
 def check_case(wl, rows=None, qkv=None):
     q, k, v = synth.make_qkv(wl) if qkv is None else qkv
     scale = 1.0 / math.sqrt(wl.d)
     rp, ci, out, lse, status = run_gpu(wl, q, k, v)
     assert status == bsa.BSA_OK, bsa.status_string(status)
+    kchunk = tuple(wl.kchunk)
     # selection: oracle decides in fp32 (the kernel's precision); ties judged in fp64
     o_rp, o_ci, _ = oracle.plan(q, k, wl.T, wl.H, wl.W, scale, wl.mode, wl.topk, wl.cdf_p,
-                                wl.cdf_cap_frac, wl.t_cond, fp32=True)
-    S64 = oracle.scores(oracle.pool(q, wl.T, wl.H, wl.W), oracle.pool(k, wl.T, wl.H, wl.W), scale)
-    n_checked, n_diff = compare_csr(rp, ci, o_rp, o_ci, S64, wl.Nc, wl.n_cond, wl.mode,
-                                    wl.cdf_p, wl.cdf_cap_frac, topk=wl.topk)
+                                wl.cdf_cap_frac, wl.t_cond, fp32=True, kchunk=kchunk)
+    S64 = oracle.scores(oracle.pool(q, wl.T, wl.H, wl.W),
+                        oracle.pool(k, wl.T, wl.H, wl.W, chunk=kchunk), scale)
+    g_rp, g_ci = (rp, ci) if kchunk == (4, 4, 8) else boxes_to_key_chunks(rp, ci, wl)
+    n_checked, n_diff = compare_csr(g_rp, g_ci, o_rp, o_ci, S64, wl.Nc, wl.n_cond, wl.mode,
+                                    wl.cdf_p, wl.cdf_cap_frac, topk=wl.topk, Nk=wl.Nk,
+                                    n_cond_k=wl.n_cond_k)
     assert n_diff <= max(1, n_checked // 100), f"{n_diff} of {n_checked} rows differ (ties)"
     # attention on the GPU's own CSR
     if rows is None:
@@ -316,7 +346,7 @@ def _sample_rows(wl, per_head, seed=0):
 @pytest.mark.parametrize("name,per_head", [("480p", 224), ("720p", 64), ("long", 2),
                                            ("causal_cdf", 2), ("720p_r8", 2),
                                            ("720p_topk_cdf", 2), ("720p_real", 4),
-                                           ("480p_real", 4)])
+                                           ("480p_real", 4), ("720p_k512", 4)])
 def test_full_size_workloads(name, per_head):
     wl = W[name]
     check_case(wl, rows=_sample_rows(wl, per_head))
