@@ -99,6 +99,8 @@ def _load():
             lib.oracle_attend_bwd.restype = i32
             lib.oracle_attend_bwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, dbl, vp, vp,
                                               vp, i64, vp, vp, vp]
+            lib.oracle_lse_merge.restype = i32
+            lib.oracle_lse_merge.argtypes = [vp, vp, vp, vp, i64, i32]
             lib.oracle_num_threads.restype = i32
             lib.oracle_num_threads.argtypes = []
             _lib = lib
@@ -241,6 +243,19 @@ def attend_bwd(q, k, v, dout, T, H, W, scale, row_ptr, col_idx, rows, kchunk=CHU
                                            rows.ctypes.data, rows.size, dq.ctypes.data,
                                            dk.ctypes.data, dv.ctypes.data), "oracle_attend_bwd")
     return dq, dk, dv
+
+
+def lse_merge(o1, l1, o2, l2):
+    """Merge two partial attention results over disjoint key sets by their
+    log-sum-exps: returns (o, l) float64, o [..., d], l [...]."""
+    o = np.array(o1, dtype=np.float64, copy=True)
+    l = np.array(l1, dtype=np.float64, copy=True)
+    o2 = np.ascontiguousarray(o2, dtype=np.float64)
+    l2 = np.ascontiguousarray(l2, dtype=np.float64)
+    d = o.shape[-1]
+    _check(_load().oracle_lse_merge(o.ctypes.data, l.ctypes.data, o2.ctypes.data, l2.ctypes.data,
+                                    l.size, d), "oracle_lse_merge")
+    return o, l
 
 
 def dense(q, k, v, T, H, W, scale, qtok, t_cond=0, want_lse=True):

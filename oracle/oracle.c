@@ -590,6 +590,36 @@ int oracle_attend_bwd(const double* q, const double* k, const double* v, const d
                                    col_idx, rows, n_rows, dq_rows, dk, dv);
 }
 
+/*
+ * Context-parallel merge of two partial attention results over disjoint key
+ * sets ([P1] ring block sparse attention: the output of a query is assembled
+ * with an online softmax over key partitions; [P3] "开源实现": LSE and output
+ * correction for context parallelism). For each query, with natural-log
+ * log-sum-exps l1, l2 of the two partitions:
+ *   l = log(exp(l1) + exp(l2)),   o = exp(l1 - l) o1 + exp(l2 - l) o2
+ * which is the softmax-weighted output over the union of the key sets. A
+ * partition with no keys has l = -inf and weight 0 (both empty: o = 0,
+ * l = -inf). o1/l1 are overwritten with the merge. fp64.
+ */
+int oracle_lse_merge(double* o1, double* l1, const double* o2, const double* l2, int64_t n, int d) {
+    if (!o1 || !l1 || !o2 || !l2 || n < 0 || d <= 0) return -1;
+    for (int64_t i = 0; i < n; ++i) {
+        const double a = l1[i], b = l2[i];
+        if (b == -INFINITY) continue;
+        if (a == -INFINITY) {
+            for (int x = 0; x < d; ++x) o1[i * d + x] = o2[i * d + x];
+            l1[i] = b;
+            continue;
+        }
+        const double m = a > b ? a : b;
+        const double l = m + log(exp(a - m) + exp(b - m));
+        const double wa = exp(a - l), wb = exp(b - l);
+        for (int x = 0; x < d; ++x) o1[i * d + x] = wa * o1[i * d + x] + wb * o2[i * d + x];
+        l1[i] = l;
+    }
+    return 0;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     extern int omp_get_max_threads(void);
