@@ -38,7 +38,9 @@ MODES = {"topk": BSA_SEL_TOPK, "cdf": BSA_SEL_CDF, "topk_cdf": BSA_SEL_TOPK_CDF}
 EXPORTED = ("bsa_version", "bsa_status_string", "bsa_workspace_size", "bsa_plan_sizes",
             "bsa_plan", "bsa_plan_noalloc", "bsa_forward", "bsa_forward_ex", "bsa_read_status",
             "bsa_rearrange", "bsa_pool", "bsa_scores", "bsa_selftest_exp2",
-            "bsa_selftest_timeout", "bsa_backward_workspace_size", "bsa_backward")
+            "bsa_selftest_timeout", "bsa_backward_workspace_size", "bsa_backward",
+            "bsa_select_pooled", "bsa_csr_slice_workspace_size", "bsa_csr_slice",
+            "bsa_lse_merge")
 
 
 class BsaError(RuntimeError):
@@ -55,15 +57,18 @@ class bsa_params(ctypes.Structure):
                 ("topk", ctypes.c_int32), ("cdf_p", ctypes.c_float),
                 ("cdf_cap_frac", ctypes.c_float), ("t_cond", ctypes.c_int32),
                 ("q_begin", ctypes.c_int32), ("kchunk_t", ctypes.c_int32),
-                ("kchunk_h", ctypes.c_int32), ("kchunk_w", ctypes.c_int32)]
+                ("kchunk_h", ctypes.c_int32), ("kchunk_w", ctypes.c_int32),
+                ("q_end", ctypes.c_int32)]
 
 
 def make_params(B, heads, T, H, W, d, mode="topk", topk=1, cdf_p=0.9, cdf_cap_frac=0.25,
-                t_cond=0, scale=0.0, q_begin=0, kchunk=(0, 0, 0)) -> bsa_params:
-    """kchunk: key chunk shape (t, h, w); 0 on an axis = the query chunk's (4, 4, 8)."""
+                t_cond=0, scale=0.0, q_begin=0, kchunk=(0, 0, 0), q_end=0) -> bsa_params:
+    """kchunk: key chunk shape (t, h, w); 0 on an axis = the query chunk's (4, 4, 8).
+    [q_begin, q_end): latent frames whose queries are computed (q_end 0 = T)."""
     return bsa_params(B, heads, T, H, W, d, 4, 4, 8, float(scale),
                       MODES[mode], int(topk), float(cdf_p),
-                      float(cdf_cap_frac), int(t_cond), int(q_begin), *map(int, kchunk))
+                      float(cdf_cap_frac), int(t_cond), int(q_begin), *map(int, kchunk),
+                      int(q_end))
 
 
 def params_for(wl) -> bsa_params:
@@ -103,6 +108,10 @@ def lib():
             "bsa_selftest_exp2": (i32, [vp, vp, vp, i64, vp]),
             "bsa_selftest_timeout": (i32, [vp, u64, vp]),
             "bsa_backward_workspace_size": (sz, [P]),
+            "bsa_select_pooled": (i32, [P, vp, vp, i32, vp, sz, vp, vp, i64, vp]),
+            "bsa_csr_slice_workspace_size": (sz, [i64]),
+            "bsa_csr_slice": (i32, [i64, vp, vp, i64, i32, i32, vp, sz, vp, vp, i64, vp]),
+            "bsa_lse_merge": (i32, [P, vp, vp, vp, vp, vp]),
             "bsa_backward": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, vp,
                                    vp]),
         }
@@ -199,6 +208,30 @@ def bsa_backward(p, q, k, v, out, lse, dout, row_ptr, col_idx, workspace, dq, dk
                               _ptr(dout), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
                               _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)), "bsa_backward")
+
+
+def bsa_select_pooled(p, qpool, kpool, workspace, row_ptr, col_idx, kshard=0, stream=None):
+    _check(lib().bsa_select_pooled(ctypes.byref(p), _ptr(qpool), _ptr(kpool), int(kshard),
+                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
+                                   _stream(stream)), "bsa_select_pooled")
+
+
+def bsa_csr_slice_workspace_size(n_rows: int) -> int:
+    return lib().bsa_csr_slice_workspace_size(int(n_rows))
+
+
+def bsa_csr_slice(row_ptr, col_idx, lo, hi, workspace, out_row_ptr, out_col_idx, stream=None):
+    _check(lib().bsa_csr_slice(row_ptr.numel() - 1, _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
+                               int(lo), int(hi), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _ptr(out_row_ptr),
+                               _ptr(out_col_idx), out_col_idx.numel(), _stream(stream)),
+           "bsa_csr_slice")
+
+
+def bsa_lse_merge(p, out, lse, out_part, lse_part, stream=None):
+    _check(lib().bsa_lse_merge(ctypes.byref(p), _ptr(out), _ptr(lse), _ptr(out_part),
+                               _ptr(lse_part), _stream(stream)), "bsa_lse_merge")
 
 
 def bsa_read_status(workspace, stream=None) -> int:

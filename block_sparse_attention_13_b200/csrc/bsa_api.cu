@@ -72,6 +72,10 @@ static int make_dims(const bsa_params* p, Dims* g) {
     if ((kt / kChunkT) * (kh / kChunkH) * (kw / kChunkW) > 8) return BSA_ERR_UNSUPPORTED;
     if (p->t_cond % kt) return BSA_ERR_SHAPE;
     if (p->q_begin < 0 || p->q_begin % kChunkT || p->q_begin >= p->T) return BSA_ERR_SHAPE;
+    // q_end: 0 = T; otherwise past q_begin, at most T, a multiple of 4 unless it is T
+    const int q_end = p->q_end ? p->q_end : p->T;
+    if (q_end <= p->q_begin || q_end > p->T || (q_end % kChunkT && q_end != p->T))
+        return BSA_ERR_SHAPE;
     if (!(std::isfinite(p->scale)) || p->scale < 0.f) return BSA_ERR_INVALID_ARG;
     if (p->mode == BSA_SEL_TOPK || p->mode == BSA_SEL_TOPK_CDF) {
         if (p->topk < 1) return BSA_ERR_INVALID_ARG;
@@ -111,7 +115,8 @@ static int make_dims(const bsa_params* p, Dims* g) {
     g->Nk = g->NkT * g->NkH * g->NkW;
     g->n_cond_k = (p->t_cond / kt) * g->NkH * g->NkW;
     g->q_skip = (p->q_begin / kChunkT) * g->NH * g->NW;
-    g->Nq = g->Nc - g->q_skip;
+    const int q_stop = q_end == p->T ? g->Nc : (q_end / kChunkT) * g->NH * g->NW;
+    g->Nq = q_stop - g->q_skip;
     g->rows = g->BH * g->Nq;
     if (g->rows * (int64_t)g->Nc > INT32_MAX) return BSA_ERR_UNSUPPORTED;
     g->n_cond = (p->t_cond / kChunkT) * g->NH * g->NW;
@@ -121,7 +126,10 @@ static int make_dims(const bsa_params* p, Dims* g) {
 
 // Computed rows per (batch, head) that are condition rows (candidates: the
 // n_cond condition chunks) and noisy rows (candidates: all chunks).
-static int64_t cond_rows(const Dims& g) { return g.n_cond > g.q_skip ? g.n_cond - g.q_skip : 0; }
+static int64_t cond_rows(const Dims& g) {
+    const int c_end = g.n_cond < g.q_skip + g.Nq ? g.n_cond : g.q_skip + g.Nq;
+    return c_end > g.q_skip ? c_end - g.q_skip : 0;
+}
 static int64_t noisy_rows(const Dims& g) { return g.Nq - cond_rows(g); }
 
 // CSR entries in key chunks (exact for TOPK, an upper bound otherwise).
@@ -290,6 +298,78 @@ int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* 
     return cuda_status(launch_backward(g, q, k, v, out, lse, dout, row_ptr, col_idx, col_capacity,
                                        workspace, dq, dk, dv, kDefaultTimeoutNs,
                                        static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_select_pooled(const bsa_params* p, const float* qpool, const float* kpool, int32_t kshard,
+                      void* workspace, size_t ws_bytes, int32_t* row_ptr, int32_t* col_idx,
+                      int64_t col_capacity, void* stream) {
+    Dims g;
+    int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!qpool || !kpool || !workspace || !row_ptr || !col_idx) return BSA_ERR_INVALID_ARG;
+    if (kshard < 0 || (kshard > 0 && g.Nk % kshard)) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(qpool) || !aligned16(kpool) || !aligned16(workspace) || !aligned16(row_ptr) ||
+        !aligned16(col_idx))
+        return BSA_ERR_ALIGNMENT;
+    const WsLayout L = ws_layout(g, *p);
+    if (ws_bytes < L.total) return BSA_ERR_WORKSPACE_TOO_SMALL;
+    if (col_capacity < max_nnz_of(g, *p)) return BSA_ERR_CAPACITY;
+    if ((rc = device_ok()) != BSA_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    float* S = reinterpret_cast<float*>(ws + L.scores);
+    uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+    if ((rc = cuda_status(launch_scores(g, qpool, kpool, S, st, kshard))) != BSA_OK) return rc;
+    int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+    int32_t* padded = reinterpret_cast<int32_t*>(ws + L.padded);
+    if (g.m == 1)
+        return cuda_status(launch_select(g, *p, S, row_ptr, col_idx, col_capacity, counts, padded,
+                                         L.pad_stride, status, st));
+    int32_t* kc_rp = reinterpret_cast<int32_t*>(ws + L.kc_row_ptr);
+    int32_t* kc_ci = reinterpret_cast<int32_t*>(ws + L.kc_col_idx);
+    if ((rc = cuda_status(launch_select(g, *p, S, kc_rp, kc_ci, L.kc_cap, counts, padded,
+                                        L.pad_stride, status, st))) != BSA_OK)
+        return rc;
+    return cuda_status(launch_expand_boxes(g, kc_rp, kc_ci, counts, row_ptr, col_idx, col_capacity,
+                                           status, st));
+}
+
+size_t bsa_csr_slice_workspace_size(int64_t n_rows) {
+    if (n_rows < 0) return 0;
+    return 256 + round_up((size_t)n_rows * sizeof(int32_t), 256);
+}
+
+int bsa_csr_slice(int64_t n_rows, const int32_t* row_ptr, const int32_t* col_idx,
+                  int64_t col_capacity, int32_t lo, int32_t hi, void* workspace, size_t ws_bytes,
+                  int32_t* out_row_ptr, int32_t* out_col_idx, int64_t out_capacity, void* stream) {
+    if (n_rows < 0 || !row_ptr || !col_idx || !workspace || !out_row_ptr || !out_col_idx ||
+        col_capacity < 0 || out_capacity < 0 || lo < 0 || hi < lo)
+        return BSA_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return BSA_ERR_ALIGNMENT;
+    if (ws_bytes < bsa_csr_slice_workspace_size(n_rows)) return BSA_ERR_WORKSPACE_TOO_SMALL;
+    int rc = device_ok();
+    if (rc != BSA_OK) return rc;
+    if (n_rows == 0) return BSA_OK;
+    char* ws = static_cast<char*>(workspace);
+    return cuda_status(launch_csr_slice(n_rows, row_ptr, col_idx, col_capacity, lo, hi,
+                                        reinterpret_cast<int32_t*>(ws + 256), out_row_ptr,
+                                        out_col_idx, out_capacity,
+                                        reinterpret_cast<uint32_t*>(ws),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_lse_merge(const bsa_params* p, void* out, float* lse, const void* out_part,
+                  const float* lse_part, void* stream) {
+    Dims g;
+    int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!out || !lse || !out_part || !lse_part) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(out_part) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+        (reinterpret_cast<uintptr_t>(lse_part) & 3u))
+        return BSA_ERR_ALIGNMENT;
+    if ((rc = device_ok()) != BSA_OK) return rc;
+    return cuda_status(launch_lse_merge(g, out, lse, out_part, lse_part,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 int bsa_read_status(void* workspace, void* stream) {

@@ -79,8 +79,10 @@ cudaError_t launch_pool(const Dims& g, const void* x0, const void* x1, float* p0
                         cudaStream_t st);
 cudaError_t launch_rearrange(const Dims& g, const void* src, void* dst, int inverse,
                              cudaStream_t st);
+// kshard > 0: kp is [shard][BH][kshard][d] (gathered pooled keys of a context-
+// parallel group); 0: the plain [BH][Nk][d] layout.
 cudaError_t launch_scores(const Dims& g, const float* qp, const float* kp, float* S,
-                          cudaStream_t st);
+                          cudaStream_t st, int kshard = 0);
 cudaError_t launch_select(const Dims& g, const bsa_params& p, const float* S, int32_t* row_ptr,
                           int32_t* col_idx, int64_t col_cap, int32_t* counts, int32_t* padded,
                           int pad_stride, uint32_t* status, cudaStream_t st);
@@ -104,6 +106,15 @@ cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const v
                             const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
                             void* workspace, void* dq, void* dk, void* dv, uint64_t timeout_ns,
                             cudaStream_t st);
+// Context parallelism: CSR entries with lo <= column < hi, re-indexed to
+// column - lo (order kept); and the log-sum-exp merge of a partial attention
+// result into an accumulator.
+cudaError_t launch_csr_slice(int64_t rows, const int32_t* row_ptr, const int32_t* col_idx,
+                             int64_t col_cap, int lo, int hi, int32_t* counts, int32_t* out_row_ptr,
+                             int32_t* out_col_idx, int64_t out_cap, uint32_t* status,
+                             cudaStream_t st);
+cudaError_t launch_lse_merge(const Dims& g, void* out, float* lse, const void* out_part,
+                             const float* lse_part, cudaStream_t st);
 cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, int64_t n,
                                  cudaStream_t st);
 cudaError_t launch_selftest_timeout(uint32_t* status, uint64_t timeout_ns, cudaStream_t st);

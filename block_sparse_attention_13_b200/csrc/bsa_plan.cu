@@ -146,17 +146,20 @@ __global__ void __launch_bounds__(256) rearrange_kernel(const __nv_bfloat16* __r
 // Pooled scores S[bh][i][m] = <qp[i], kp[m]> * scale in fp32 FMA. 64x64 output
 // tile per CTA, 4x4 register micro-tile per thread, operands staged
 // transposed in shared memory 32 channels at a time.
+// kp holds the key chunks in shards of `kshard` chunks, [shard][BH][kshard][D]
+// (kshard = Nk: one shard, the plain [BH][Nk][D] layout); the gathered pooled
+// keys of a context-parallel group arrive that way.
 __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ qp,
                                                      const float* __restrict__ kp,
                                                      float* __restrict__ S, int Nq, int Nk,
-                                                     int D, float scale) {
+                                                     int kshard, int D, float scale) {
     constexpr int BT = 64, BK = 32, LD = BT + 4;
     __shared__ __align__(16) float As[BK][LD];
     __shared__ __align__(16) float Bs[BK][LD];
     const int64_t bh = blockIdx.z;
     const int i0 = blockIdx.y * BT, m0 = blockIdx.x * BT;
     const float* A = qp + bh * (int64_t)Nq * D;
-    const float* Bm = kp + bh * (int64_t)Nk * D;
+    const int64_t BH = gridDim.z;
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
     float acc[4][4];
 #pragma unroll
@@ -171,7 +174,10 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ q
             const int r = idx / (BK / 4), kq = idx % (BK / 4);
             float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
             if (i0 + r < Nq) va = *reinterpret_cast<const float4*>(A + (int64_t)(i0 + r) * D + k0 + kq * 4);
-            if (m0 + r < Nk) vb = *reinterpret_cast<const float4*>(Bm + (int64_t)(m0 + r) * D + k0 + kq * 4);
+            if (m0 + r < Nk) {
+                const int m = m0 + r, sh = m / kshard, ml = m - sh * kshard;
+                vb = *reinterpret_cast<const float4*>(kp + ((sh * BH + bh) * kshard + ml) * D + k0 + kq * 4);
+            }
             As[kq * 4 + 0][r] = va.x; As[kq * 4 + 1][r] = va.y;
             As[kq * 4 + 2][r] = va.z; As[kq * 4 + 3][r] = va.w;
             Bs[kq * 4 + 0][r] = vb.x; Bs[kq * 4 + 1][r] = vb.y;
@@ -257,13 +263,14 @@ __device__ __forceinline__ uint32_t kth_largest_key(const uint32_t (&key)[MAXJ],
 template <int MAXJ>
 __global__ void __launch_bounds__(256) select_kernel(
     const float* __restrict__ S, int Ncq, int Nk, int n_cond_q, int n_cond_k, int q_skip,
-    int64_t rows, int mode, int topk, float cdf_p, float cap_frac, int32_t* __restrict__ row_ptr,
-    int32_t* __restrict__ col_idx, int64_t col_cap, int32_t* __restrict__ counts,
-    int32_t* __restrict__ padded, int pad_stride, uint32_t* status) {
+    int Nq, int64_t rows, int mode, int topk, float cdf_p, float cap_frac,
+    int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx, int64_t col_cap,
+    int32_t* __restrict__ counts, int32_t* __restrict__ padded, int pad_stride, uint32_t* status) {
     const int lane = threadIdx.x & 31;
     const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (w >= rows) return;
-    const int Nq = Ncq - q_skip;                // computed query chunks per (batch, head)
+    (void)Ncq;
+    // computed query chunks per (batch, head): q_skip .. q_skip + Nq - 1
     const int64_t bh = w / Nq;
     const int i = q_skip + (int)(w % Nq);       // query chunk of this row
     const int na = (n_cond_q > 0 && i < n_cond_q) ? n_cond_k : Nk;  // candidates are [0, na)
@@ -349,10 +356,13 @@ __global__ void __launch_bounds__(256) select_kernel(
     if (mode == BSA_SEL_TOPK) {
         const int kc = topk < n_cond_k ? topk : n_cond_k;
         const int kn = topk < Nk ? topk : Nk;
-        // rows of a (batch, head): condition rows q_skip .. n_cond_q-1, then noisy rows
-        const int c_rows = n_cond_q > q_skip ? n_cond_q - q_skip : 0;
+        // rows of a (batch, head): condition rows q_skip .. min(n_cond_q, q_skip+Nq)-1,
+        // then noisy rows
+        const int q_stop = q_skip + Nq;
+        const int c_end = n_cond_q < q_stop ? n_cond_q : q_stop;
+        const int c_rows = c_end > q_skip ? c_end - q_skip : 0;
         const int first_noisy = n_cond_q > q_skip ? n_cond_q : q_skip;
-        const int64_t per_bh = (int64_t)c_rows * kc + (int64_t)(Ncq - first_noisy) * kn;
+        const int64_t per_bh = (int64_t)c_rows * kc + (int64_t)(Nq - c_rows) * kn;
         off = bh * per_bh + (i < n_cond_q ? (int64_t)(i - q_skip) * kc
                                           : (int64_t)c_rows * kc + (int64_t)(i - first_noisy) * kn);
         if (off + count > col_cap) {
@@ -567,9 +577,10 @@ cudaError_t launch_rearrange(const Dims& g, const void* src, void* dst, int inve
 }
 
 cudaError_t launch_scores(const Dims& g, const float* qp, const float* kp, float* S,
-                          cudaStream_t st) {
+                          cudaStream_t st, int kshard) {
     dim3 grid((g.Nk + 63) / 64, (g.Nq + 63) / 64, (unsigned)g.BH);
-    scores_kernel<<<grid, 256, 0, st>>>(qp, kp, S, g.Nq, g.Nk, g.d, g.scale);
+    scores_kernel<<<grid, 256, 0, st>>>(qp, kp, S, g.Nq, g.Nk, kshard > 0 ? kshard : g.Nk, g.d,
+                                        g.scale);
     return cudaGetLastError();
 }
 
@@ -580,9 +591,9 @@ cudaError_t launch_select(const Dims& g, const bsa_params& p, const float* S, in
     const int mode = p.mode;
 #define BSA_SELECT(MJ)                                                                       \
     select_kernel<MJ><<<blocks, 256, 0, st>>>(S, g.Nc, g.Nk, g.n_cond, g.n_cond_k, g.q_skip,   \
-                                              g.rows, mode, p.topk, p.cdf_p, p.cdf_cap_frac, \
-                                              row_ptr, col_idx, col_cap, counts, padded,     \
-                                              pad_stride, status)
+                                              g.Nq, g.rows, mode, p.topk, p.cdf_p,           \
+                                              p.cdf_cap_frac, row_ptr, col_idx, col_cap,     \
+                                              counts, padded, pad_stride, status)
     if (g.Nk <= 32) BSA_SELECT(1);
     else if (g.Nk <= 256) BSA_SELECT(8);
     else if (g.Nk <= 1024) BSA_SELECT(32);

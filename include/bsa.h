@@ -96,6 +96,10 @@ typedef struct {
                          * (t_cond must be a multiple of kchunk_t); the CSR that bsa_plan
                          * writes then lists the (4,4,8) boxes those key chunks cover, the
                          * unit bsa_forward / bsa_backward attend over. */
+    int32_t q_end;      /* one past the last latent frame whose queries are computed; 0 = T;
+                         * a multiple of 4 unless it is T. The computed query chunks are the
+                         * frames [q_begin, q_end): a rank of a context-parallel group
+                         * computes the rows of its own frame range (bsa_select_pooled). */
 } bsa_params;
 
 /* Library version: major*10000 + minor*100 + patch. */
@@ -189,6 +193,57 @@ BSA_API int bsa_backward(const bsa_params* p, const void* q, const void* k, cons
                          const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
                          void* workspace, size_t ws_bytes, void* dq, void* dk, void* dv,
                          void* stream);
+
+/*
+ * Context parallelism ([P1] ring block sparse attention: the sequence split
+ * across ranks along the latent frames, pooled keys gathered from every rank,
+ * each rank's queries selecting among all key chunks, partial attention over
+ * every rank's K/V shard combined by an online softmax; [P3] "开源实现": LSE
+ * and output correction).
+ *
+ * bsa_select_pooled: selection (scores + top-k / CDF, as bsa_plan) from pooled
+ * inputs. `p` describes the whole group's grid, with [q_begin, q_end) the
+ * frames of this rank's queries. qpool: device fp32 [B,heads,Nq,d] (this
+ * rank's pooled query chunks, e.g. from bsa_pool on its shard). kpool: device
+ * fp32 pooled key chunks of the whole grid, either [B,heads,Nk,d] (kshard = 0)
+ * or, as an all-gather delivers them, [shard][B,heads,kshard,d] with kshard
+ * key chunks per shard (Nk a multiple of kshard). The CSR has this rank's
+ * rows and global chunk ids. Workspace, capacity and errors as bsa_plan.
+ */
+BSA_API int bsa_select_pooled(const bsa_params* p, const float* qpool, const float* kpool,
+                              int32_t kshard, void* workspace, size_t ws_bytes, int32_t* row_ptr,
+                              int32_t* col_idx, int64_t col_capacity, void* stream);
+
+/* Bytes of device workspace bsa_csr_slice needs for n_rows rows (0 if n_rows < 0). */
+BSA_API size_t bsa_csr_slice_workspace_size(int64_t n_rows);
+
+/*
+ * The part of a CSR that falls in one shard of key chunks: for every row, the
+ * entries c with lo <= c < hi, written as c - lo in their original order.
+ * row_ptr/col_idx: device int32 input (n_rows+1, col_capacity); out_row_ptr /
+ * out_col_idx: device int32 output (n_rows+1, out_capacity). workspace: device,
+ * >= bsa_csr_slice_workspace_size(n_rows), 16-byte aligned; its first bytes
+ * are a status block (bsa_read_status: DEVICE_BAD_INDEX for an input row
+ * outside col_capacity, CAPACITY if out_capacity is too small). Errors:
+ * INVALID_ARG, ALIGNMENT, WORKSPACE_TOO_SMALL, CUDA.
+ */
+BSA_API int bsa_csr_slice(int64_t n_rows, const int32_t* row_ptr, const int32_t* col_idx,
+                          int64_t col_capacity, int32_t lo, int32_t hi, void* workspace,
+                          size_t ws_bytes, int32_t* out_row_ptr, int32_t* out_col_idx,
+                          int64_t out_capacity, void* stream);
+
+/*
+ * Merge a partial attention result into an accumulator by log-sum-exp, for
+ * every token of the grid `p` describes: with l1 = lse, l2 = lse_part,
+ *   lse <- log(e^l1 + e^l2),  out <- e^(l1-lse) out + e^(l2-lse) out_part.
+ * A token with lse_part = -inf (no key of that partition) keeps its value;
+ * one with lse = -inf takes the part. out, out_part: device bf16
+ * [B,heads,N,d]; lse, lse_part: device fp32 [B,heads,N] (natural log, as
+ * bsa_forward writes them). Errors: INVALID_ARG, SHAPE, UNSUPPORTED,
+ * ALIGNMENT, CUDA.
+ */
+BSA_API int bsa_lse_merge(const bsa_params* p, void* out, float* lse, const void* out_part,
+                          const float* lse_part, void* stream);
 
 /*
  * bsa_plan without a caller workspace: the same selection as bsa_plan, with

@@ -265,3 +265,41 @@ def test_unknown_selection_mode_rejected(L):
     p = P()
     p.mode = 3
     assert rc_sizes(p)[0] == bsa.BSA_ERR_INVALID_ARG
+
+
+def test_context_parallel_entries_host_checks(L):
+    x = vp(FAKE)
+    # csr slice: workspace size, argument checks
+    assert bsa.bsa_csr_slice_workspace_size(100) == 256 + 512
+    assert L.bsa_csr_slice_workspace_size(-1) == 0
+    ws = bsa.bsa_csr_slice_workspace_size(10)
+    f = L.bsa_csr_slice
+    assert f(10, x, x, 16, 5, 2, x, ws, x, x, 16, None) == bsa.BSA_ERR_INVALID_ARG   # hi < lo
+    assert f(10, x, x, 16, -1, 2, x, ws, x, x, 16, None) == bsa.BSA_ERR_INVALID_ARG
+    assert f(10, x, x, 16, 0, 2, vp(FAKE + 8), ws, x, x, 16, None) == bsa.BSA_ERR_ALIGNMENT
+    assert f(10, x, x, 16, 0, 2, x, ws - 1, x, x, 16, None) == bsa.BSA_ERR_WORKSPACE_TOO_SMALL
+    # lse merge
+    p = P()
+    assert L.bsa_lse_merge(ctypes.byref(p), x, None, x, x, None) == bsa.BSA_ERR_INVALID_ARG
+    assert L.bsa_lse_merge(ctypes.byref(p), x, vp(FAKE + 2), x, x, None) == \
+        bsa.BSA_ERR_ALIGNMENT
+    # select from pooled inputs: kshard must divide the key chunks
+    pr = P(T=16, H=8, W=16, q_begin=4, q_end=8)
+    wsz = bsa.bsa_workspace_size(pr)
+    g = L.bsa_select_pooled
+    assert g(ctypes.byref(pr), x, x, 3, x, wsz, x, x, 64, None) == bsa.BSA_ERR_INVALID_ARG
+    assert g(ctypes.byref(pr), x, x, 2, x, wsz - 1, x, x, 64, None) == \
+        bsa.BSA_ERR_WORKSPACE_TOO_SMALL
+
+
+@pytest.mark.parametrize("kw,code", [(dict(q_begin=4, q_end=4), bsa.BSA_ERR_SHAPE),
+                                     (dict(q_end=6), bsa.BSA_ERR_SHAPE),
+                                     (dict(q_end=20), bsa.BSA_ERR_SHAPE),
+                                     (dict(q_end=8), 0), (dict(T=10, q_end=10), 0)])
+def test_query_frame_range(L, kw, code):
+    base = dict(T=16, H=8, W=16)
+    base.update(kw)
+    rc, rows, _ = rc_sizes(P(**base))
+    assert rc == code
+    if code == 0 and base.get("q_end", 0) == 8:
+        assert rows == 2 * 2 * 2 * 2     # heads 2 x chunk frames [0, 2) x (2 x 2) chunks

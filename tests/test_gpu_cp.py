@@ -1,0 +1,149 @@
+"""GPU checks of the context-parallel (ring) path on one device: the ranks of a
+group of 2 or 4 are run one after the other through the same driver, with a
+communicator that hands each rank what the real all-gather and ring shifts
+would deliver. Every device step runs through the C ABI; the result of each
+rank must equal the rows of the unsplit computation (selection exactly, the
+attention within the rounding of the bf16 partial results) and the oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity import ATT_MAX_ABS, ATT_MEAN_ABS, compare_attention
+from test_gpu_parity import dev, gather_rows, host_f32
+
+pytestmark = pytest.mark.gpu
+
+import block_sparse_attention_13_b200 as bsa  # noqa: E402
+from block_sparse_attention_13_b200.context_parallel import CudaOps, ring_forward  # noqa: E402
+
+
+class SimComm:
+    """What rank `rank` of a `world`-rank group receives: the stacked pooled keys
+    of all shards, and at ring step s the K/V shard of rank (rank - s - 1)."""
+
+    def __init__(self, rank, world, kp_all, k_shards, v_shards):
+        self.rank, self.world = rank, world
+        self.kp_all, self.k, self.v = kp_all, k_shards, v_shards
+        self.step = 0
+
+    def all_gather(self, x):
+        assert torch.equal(x, self.kp_all[self.rank])
+        return self.kp_all
+
+    def start_shift(self, tensors):
+        self.step += 1
+        return (self.rank - self.step) % self.world
+
+    def finish_shift(self, j):
+        return [self.k[j], self.v[j]]
+
+
+def shard(x, world, frames, HW):
+    return [x[:, :, r * frames * HW:(r + 1) * frames * HW].contiguous() for r in range(world)]
+
+
+CASES = {
+    "w2_topk": (synth.WORKLOADS["tiny"].with_(heads=2, T=16, H=16, W=32, d=128, topk=6), 2),
+    "w4_topk": (synth.WORKLOADS["tiny"].with_(heads=2, T=16, H=16, W=32, d=64, topk=9), 4),
+    "w2_causal_cdf": (synth.WORKLOADS["tiny"].with_(B=2, heads=2, T=16, H=16, W=32, d=128,
+                                                    mode="cdf", cdf_p=0.9, cdf_cap_frac=0.25,
+                                                    t_cond=8), 2),
+    "w2_partial": (synth.WORKLOADS["tiny"].with_(heads=2, T=8, H=13, W=37, d=128, topk=5), 2),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_ring_forward_equals_unsplit(name):
+    wl, world = CASES[name]
+    q, k, v = synth.make_qkv(wl)
+    HW = wl.H * wl.W
+    T_l = wl.T // world
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    # the unsplit computation
+    p = bsa.params_for(wl)
+    pl = bsa.allocate(p)
+    bsa.bsa_plan(p, qd, kd, pl.workspace, pl.row_ptr, pl.col_idx)
+    out_g = torch.empty_like(qd)
+    lse_g = torch.empty((wl.B, wl.heads, wl.N), dtype=torch.float32, device="cuda")
+    bsa.bsa_forward(p, qd, kd, vd, pl.row_ptr, pl.col_idx, pl.workspace, out_g, lse_g)
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_OK
+    g_rp = pl.row_ptr.cpu().numpy()
+    g_ci = pl.col_idx[: int(g_rp[-1])].cpu().numpy()
+    # per-rank shards and the pooled keys the all-gather would deliver
+    qs, ks, vs = (shard(x, world, T_l, HW) for x in (qd, kd, vd))
+    ops = CudaOps()
+    p_local = bsa.make_params(wl.B, wl.heads, T_l, wl.H, wl.W, wl.d, wl.mode, wl.topk)
+    kp_all = torch.stack([ops.pool(p_local, ks[r]) for r in range(world)])
+    nc_l = wl.Nc // world
+    scale = 1.0 / math.sqrt(wl.d)
+    for r in range(world):
+        comm = SimComm(r, world, kp_all, ks, vs)
+        probe = CudaOps()
+        out, lse = ring_forward(qs[r], ks[r], vs[r], (T_l, wl.H, wl.W), wl.topk, wl.mode,
+                                wl.cdf_p, wl.cdf_cap_frac, wl.t_cond, comm=comm, ops=probe)
+        # selection: this rank's rows of the unsplit plan, exactly
+        p_rank = bsa.make_params(wl.B, wl.heads, wl.T, wl.H, wl.W, wl.d, wl.mode, wl.topk,
+                                 wl.cdf_p, wl.cdf_cap_frac, wl.t_cond, q_begin=r * T_l,
+                                 q_end=(r + 1) * T_l)
+        rp, ci = CudaOps().select_pooled(p_rank, ops.pool(p_local, qs[r]), kp_all, nc_l)
+        rp, ci = rp.cpu().numpy(), ci.cpu().numpy()
+        for bh in range(wl.B * wl.heads):
+            for i in range(nc_l):
+                row = bh * nc_l + i
+                grow = bh * wl.Nc + r * nc_l + i
+                assert np.array_equal(ci[rp[row]:rp[row + 1]], g_ci[g_rp[grow]:g_rp[grow + 1]])
+        # attention: the unsplit result for these frames. Each shard's partial output is
+        # rounded to bf16 before the merge (half an ulp of the partial, which can exceed
+        # the merged value where partials of opposite sign cancel) and the merge rounds
+        # again; measured up to 2 ulps of the result. Bars: the attention max bar and
+        # half the attention mean bar
+        sl = slice(r * T_l * HW, (r + 1) * T_l * HW)
+        diff = (out.float() - out_g[:, :, sl].float()).abs()
+        assert float(diff.max()) <= ATT_MAX_ABS and float(diff.mean()) <= ATT_MEAN_ABS / 2, \
+            (float(diff.max()), float(diff.mean()))
+        np.testing.assert_allclose(lse.cpu().numpy(), lse_g[:, :, sl].cpu().numpy(), rtol=0,
+                                   atol=1e-4)
+        # and the oracle, on the unsplit CSR rows of this rank
+        rows = np.array([bh * wl.Nc + r * nc_l + i for bh in range(wl.B * wl.heads)
+                         for i in range(nc_l)])
+        o_out, _ = oracle.attend(q, k, v, wl.T, wl.H, wl.W, scale, g_rp, g_ci, rows)
+        full = torch.zeros_like(out_g)
+        full[:, :, sl] = out
+        mx, mean = compare_attention(gather_rows(host_f32(full), wl, rows), o_out)
+        assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+
+
+def test_csr_slice_and_merge_units():
+    """bsa_csr_slice keeps [lo, hi) re-indexed in row order; bsa_lse_merge of a
+    split selection equals the forward over the whole selection."""
+    wl = synth.WORKLOADS["tiny"].with_(heads=2, T=8, H=16, W=32, d=64, topk=7)
+    q, k, v = synth.make_qkv(wl)
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    p = bsa.params_for(wl)
+    pl = bsa.allocate(p)
+    bsa.bsa_plan(p, qd, kd, pl.workspace, pl.row_ptr, pl.col_idx)
+    ops = CudaOps()
+    rp_h = pl.row_ptr.cpu().numpy()
+    ci_h = pl.col_idx[: int(rp_h[-1])].cpu().numpy()
+    outs = []
+    for lo, hi in ((0, 13), (13, 32)):
+        srp, sci = ops.slice(pl.row_ptr, pl.col_idx, lo, hi)
+        srp_h, sci_h = srp.cpu().numpy(), sci.cpu().numpy()
+        for r in range(wl.rows):
+            row = ci_h[rp_h[r]:rp_h[r + 1]]
+            assert np.array_equal(sci_h[srp_h[r]:srp_h[r + 1]], row[(row >= lo) & (row < hi)] - lo)
+        # attention over the slice: shift the key ids back by running on the whole grid
+        back = torch.from_numpy(sci_h[: srp_h[-1]] + lo).cuda() if srp_h[-1] else \
+            torch.zeros(1, dtype=torch.int32, device="cuda")
+        outs.append(ops.forward(p, qd, kd, vd, srp, back.to(torch.int32)))
+    (o, l), (o2, l2) = outs
+    ops.merge(p, o, l, o2, l2)
+    of, lf = ops.forward(p, qd, kd, vd, pl.row_ptr, pl.col_idx)
+    ops.check()
+    diff = (o.float() - of.float()).abs()
+    assert float(diff.max()) <= ATT_MAX_ABS and float(diff.mean()) <= ATT_MEAN_ABS / 2
+    torch.testing.assert_close(l, lf, rtol=0, atol=1e-4)
