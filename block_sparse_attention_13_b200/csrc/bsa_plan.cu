@@ -72,30 +72,53 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
     const __nv_bfloat16* base = x + bh * N * D;
-    int n_tok = 0;
-    for (int bt = 0; bt < sd.mt; ++bt)
-        for (int bhh = 0; bhh < sd.mh; ++bhh)
-            for (int bw = 0; bw < sd.mw; ++bw) {
-                const int t0 = (ct * sd.mt + bt) * kChunkT, h0 = (ch * sd.mh + bhh) * kChunkH,
-                          w0 = (cw * sd.mw + bw) * kChunkW;
-                const int nt = min(kChunkT, T - t0), nh = min(kChunkH, H - h0),
-                          nw = min(kChunkW, W - w0);
-                if (nt <= 0 || nh <= 0 || nw <= 0) continue;  // box past the grid
-                n_tok += nt * nh * nw;
+    // sums the existing tokens of the box at (t0, h0, w0); returns their count
+    auto add_box = [&](int t0, int h0, int w0) -> int {
+        const int nt = min(kChunkT, T - t0), nh = min(kChunkH, H - h0), nw = min(kChunkW, W - w0);
+        if (nt <= 0 || nh <= 0 || nw <= 0) return 0;  // box past the grid
+        if (nt == kChunkT && nh == kChunkH && nw == kChunkW) {
+            // a whole box: every load unconditional, all in flight together
+            uint4 u[ITERS];
 #pragma unroll
-                for (int it = 0; it < ITERS; ++it) {
-                    const int v = it * 256 + tid;
-                    const int l = v / VPT;  // local token (lt*4 + lh)*8 + lw
-                    const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
-                    if (lt >= nt || lh >= nh || lw >= nw) continue;
-                    const int64_t tok = ((int64_t)(t0 + lt) * H + (h0 + lh)) * W + w0 + lw;
-                    const uint4 u = ld_nc_v4(base + tok * D + dvec * 8);
-                    add_bf16x2(acc[0], acc[1], u.x);
-                    add_bf16x2(acc[2], acc[3], u.y);
-                    add_bf16x2(acc[4], acc[5], u.z);
-                    add_bf16x2(acc[6], acc[7], u.w);
-                }
+            for (int it = 0; it < ITERS; ++it) {
+                const int l = (it * 256 + tid) / VPT;  // local token (lt*4 + lh)*8 + lw
+                const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
+                const int64_t tok = ((int64_t)(t0 + lt) * H + (h0 + lh)) * W + w0 + lw;
+                u[it] = ld_nc_v4(base + tok * D + dvec * 8);
             }
+#pragma unroll
+            for (int it = 0; it < ITERS; ++it) {
+                add_bf16x2(acc[0], acc[1], u[it].x);
+                add_bf16x2(acc[2], acc[3], u[it].y);
+                add_bf16x2(acc[4], acc[5], u[it].z);
+                add_bf16x2(acc[6], acc[7], u[it].w);
+            }
+        } else {
+#pragma unroll
+            for (int it = 0; it < ITERS; ++it) {
+                const int l = (it * 256 + tid) / VPT;
+                const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
+                if (lt >= nt || lh >= nh || lw >= nw) continue;
+                const int64_t tok = ((int64_t)(t0 + lt) * H + (h0 + lh)) * W + w0 + lw;
+                const uint4 u = ld_nc_v4(base + tok * D + dvec * 8);
+                add_bf16x2(acc[0], acc[1], u.x);
+                add_bf16x2(acc[2], acc[3], u.y);
+                add_bf16x2(acc[4], acc[5], u.z);
+                add_bf16x2(acc[6], acc[7], u.w);
+            }
+        }
+        return nt * nh * nw;
+    };
+    int n_tok = 0;
+    if (sd.mt * sd.mh * sd.mw == 1) {
+        n_tok = add_box(ct * kChunkT, ch * kChunkH, cw * kChunkW);
+    } else {
+        for (int bt = 0; bt < sd.mt; ++bt)
+            for (int bhh = 0; bhh < sd.mh; ++bhh)
+                for (int bw = 0; bw < sd.mw; ++bw)
+                    n_tok += add_box((ct * sd.mt + bt) * kChunkT, (ch * sd.mh + bhh) * kChunkH,
+                                     (cw * sd.mw + bw) * kChunkW);
+    }
     const int grp = tid / VPT;
 #pragma unroll
     for (int e = 0; e < 8; ++e) red[grp][dvec * 8 + e] = acc[e];
