@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-group", type=int, default=4,
+                    help="(batch, head) pairs per group of the host-buffer pipeline")
+    ap.add_argument("--e2e-streams", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--backward", action="store_true",
@@ -392,21 +395,24 @@ def main():
     total_flops = sum_over_ranks(flops * args.steps)
     value = total_flops / (total_ms / 1e3) / 1e12
 
-    # ---- end to end through the C ABI with host buffers (pinned), per step:
-    # H2D of q, k, v; plan; forward; D2H of the output
+    # ---- end to end with host buffers (pinned) through the public host API: per step
+    # H2D of q, k, v, plan, forward and D2H of the output, in groups of (batch, head)
+    # pairs whose copies overlap the other groups' kernels
+    from block_sparse_attention_13_b200.host import HostForward
     out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    hf = HostForward(p, group=args.e2e_group, streams=args.e2e_streams)
+    hf(host[0], host[1], host[2], out_host)          # warm-up
+    torch.cuda.synchronize()
+    hf.check()
     e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e_s.record(stream)
     for _ in range(max(args.e2e_steps, 1)):
-        q.copy_(host[0], non_blocking=True)
-        k.copy_(host[1], non_blocking=True)
-        v.copy_(host[2], non_blocking=True)
-        step()
-        out_host.copy_(out, non_blocking=True)
+        hf(host[0], host[1], host[2], out_host)
     e_e.record(stream)
     torch.cuda.synchronize()
+    hf.check()
     barrier()
     e2e_ms = max_over_ranks(e_s.elapsed_time(e_e)) / max(args.e2e_steps, 1)
     e2e_value = sum_over_ranks(flops) / (e2e_ms / 1e3) / 1e12
@@ -459,7 +465,9 @@ def main():
             / ms_per_step / 1e9,
             "dense": dense, "roofline": roofline, "cpu_baseline": cpu, "backward": bwd,
             "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "api": "HostForward (pinned host q, k, v -> out)",
+                    "group": args.e2e_group, "streams": args.e2e_streams},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks, "device_status": bsa.status_string(rc),
         }
