@@ -59,7 +59,14 @@ struct AttnCfg {
     static constexpr int kCtl = 6 * kTileBytes;
     static constexpr int kMaxChunks = 2048;                // Nc limit of the library
     static constexpr int kList = kCtl + 512;               // uint16 chunk lists of both tiles
-    static constexpr int kSmemBytes = kList + 2 * kMaxChunks * 2 + 1024;  // + alignment slack
+    // Grids with partial edge chunks: the edge pattern of every listed chunk (uint8),
+    // then the operands of the masking product (see bsa_fwd_kernel): a ones tile and
+    // one bias tile per edge pattern 1..7, each 128 rows x 8 bf16 (2 KB), K-major
+    // without swizzle.
+    static constexpr int kPat = kList + 2 * kMaxChunks * 2;
+    static constexpr int kBias = kPat + 2 * kMaxChunks;
+    static constexpr int kBiasTile = 128 * 16;
+    static constexpr int kSmemBytes = kBias + 8 * kBiasTile + 1024;  // + alignment slack
     // tensor memory: S0 S1 (fp32 128x128; P is written over S as bf16) O0 O1
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t s_col(int t) { return t * 128; }
@@ -103,9 +110,14 @@ struct __align__(8) Ctl {
 //   PV0(j), S0(j+1), PV1(j), S1(j+1)
 // so each tile's softmax runs while the tensor core works on the other tile.
 // S(j+1) is queued right behind the PV(j) that reads P from the same TMEM
-// columns: tcgen05 MMAs of one CTA execute in issue order. kPartial: the grid
-// has partial edge chunks, whose key slots past the grid are masked out of the
-// softmax (a separate instantiation, so full grids keep the unmasked loop).
+// columns: tcgen05 MMAs of one CTA execute in issue order.
+// kPartial: the grid has partial edge chunks. The key slots of such a chunk past
+// the grid (zero-filled by TMA) must not take part in the softmax, so S of a
+// partial key chunk gets one more K = 16 product, ones x bias: A has a 1 in
+// column 0 of every row, B has -inf in column 0 of the rows of missing key
+// slots and 0 elsewhere (one B tile per edge pattern: partial in t, h, w or a
+// combination). Existing slots get exactly +0 and missing ones -inf, as a mask
+// would give, and the softmax loop is the same as for full grids.
 template <int D, bool kPartial>
 __global__ void __launch_bounds__(320, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -120,6 +132,25 @@ __global__ void __launch_bounds__(320, 1)
     const int lane = threadIdx.x & 31;
 
     uint16_t* lists = reinterpret_cast<uint16_t*>(smem + C::kList);  // [2][kMaxChunks]
+    uint8_t* pats = smem + C::kPat;                                   // [2][kMaxChunks]
+
+    if constexpr (kPartial) {
+        // ones tile (tile 0) and bias tiles of edge patterns 1..7: row r (key slot r of a
+        // chunk: frame r / 32, row (r / 8) % 4, column r % 8) holds 8 bf16, only the
+        // first nonzero. Rows are 16 bytes apart, so 8-row core matrices are 128 bytes
+        // apart (SBO); both K groups of the product read the same 8 columns (LBO 0).
+        const int et = a.T % kChunkT, eh = a.H % kChunkH, ew = a.W % kChunkW;
+        for (int i = threadIdx.x; i < 8 * 128; i += blockDim.x) {
+            const int tile = i >> 7, r = i & 127;
+            const int lt = r >> 5, lh = (r >> 3) & 3, lw = r & 7;
+            const bool missing = ((tile & 1) && lt >= et) || ((tile & 2) && lh >= eh) ||
+                                 ((tile & 4) && lw >= ew);
+            // bf16 bits: 1.0 = 0x3f80, -inf = 0xff80
+            const uint32_t first = tile == 0 ? 0x3f80u : (missing ? 0xff80u : 0u);
+            *reinterpret_cast<uint4*>(smem + C::kBias + i * 16) = make_uint4(first, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+    }
 
     if (threadIdx.x == 0) {
         for (int t = 0; t < 2; ++t) {
@@ -161,8 +192,17 @@ __global__ void __launch_bounds__(320, 1)
                 const bool valid = e < end && c >= 0 && c < a.Nc;
                 if (e < end && !valid) bad = true;
                 const uint32_t vb = __ballot_sync(0xffffffffu, valid);
-                if (valid) lists[t * C::kMaxChunks + cnt + __popc(vb & ((1u << lane) - 1u))] =
-                    static_cast<uint16_t>(c);
+                const int slot = t * C::kMaxChunks + cnt + __popc(vb & ((1u << lane) - 1u));
+                if (valid) {
+                    lists[slot] = static_cast<uint16_t>(c);
+                    if constexpr (kPartial) {
+                        int kt, kh, kw;
+                        chunk_origin(c, a.NH, a.NW, kt, kh, kw);
+                        pats[slot] = static_cast<uint8_t>((kt + kChunkT > a.T ? 1 : 0) |
+                                                          (kh + kChunkH > a.H ? 2 : 0) |
+                                                          (kw + kChunkW > a.W ? 4 : 0));
+                    }
+                }
                 cnt += __popc(vb);
             }
             if (lane == 0) ctl->n_valid[t] = cnt;
@@ -277,6 +317,14 @@ __global__ void __launch_bounds__(320, 1)
                     mma_ss(tmem + C::s_col(t), sdesc_sw128(sq + off, 16, 1024),
                            sdesc_sw128(sk + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
                 }
+                if constexpr (kPartial) {
+                    const int pat = pats[t * C::kMaxChunks + j];
+                    if (pat) {
+                        const uint32_t sb = smem_u32(smem + C::kBias);
+                        mma_ss(tmem + C::s_col(t), sdesc_plain(sb, 0, 128),
+                               sdesc_plain(sb + pat * C::kBiasTile, 0, 128), kIdS, 1u);
+                    }
+                }
                 issued = true;
                 tc_commit(&b.k_empty);
                 if (!((a.debug_flags & 1) && j == 0 && t == 0)) tc_commit(&b.s_full);
@@ -339,25 +387,6 @@ __global__ void __launch_bounds__(320, 1)
             tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(s + 64));
             tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(s + 96));
             tmem_wait_ld();
-            if constexpr (kPartial) {
-                // A partial edge key chunk (grid not a multiple of the chunk shape): its
-                // slots past the grid were zero-filled by TMA and must not take part in
-                // the softmax. The branch is uniform across the CTA.
-                int kt, kh, kw;
-                chunk_origin(lists[t * C::kMaxChunks + it], a.NH, a.NW, kt, kh, kw);
-                const int nt = a.T - kt, nh = a.H - kh, nw = a.W - kw;
-                if (nt < kChunkT || nh < kChunkH || nw < kChunkW) {
-                    // bit lh*8 + lw: slot (lh, lw) of a 32-column frame exists
-                    uint32_t m32 = 0u;
-                    const uint32_t row8 = nw >= kChunkW ? 0xffu : ((1u << nw) - 1u);
-#pragma unroll
-                    for (int lh = 0; lh < kChunkH; ++lh)
-                        if (lh < nh) m32 |= row8 << (8 * lh);
-#pragma unroll
-                    for (int c = 0; c < 128; ++c)
-                        if ((c >> 5) >= nt || !((m32 >> (c & 31)) & 1u)) s[c] = 0xff800000u;  // -inf
-                }
-            }
             float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
             float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
 #pragma unroll
