@@ -81,6 +81,9 @@ def _load():
             lib.oracle_attend_bwd_shape.restype = i32
             lib.oracle_attend_bwd_shape.argtypes = [vp] * 4 + [i32] * 8 + [dbl, vp, vp, vp, i64,
                                                                           vp, vp, vp]
+            lib.oracle_attend_bwd_part_shape.restype = i32
+            lib.oracle_attend_bwd_part_shape.argtypes = [vp] * 6 + [i32] * 8 + [dbl, vp, vp, vp,
+                                                                               i64, vp, vp, vp]
             lib.oracle_rearrange.restype = i32
             lib.oracle_rearrange.argtypes = [vp, i32, i32, i32, i32, i32, vp]
             lib.oracle_pool.restype = i32
@@ -242,6 +245,34 @@ def attend_bwd(q, k, v, dout, T, H, W, scale, row_ptr, col_idx, rows, kchunk=CHU
                                            float(scale), rp.ctypes.data, ci.ctypes.data,
                                            rows.ctypes.data, rows.size, dq.ctypes.data,
                                            dk.ctypes.data, dv.ctypes.data), "oracle_attend_bwd")
+    return dq, dk, dv
+
+
+def attend_bwd_part(q, k, v, dout, out, lse, T, H, W, scale, row_ptr, col_idx, rows,
+                    kchunk=CHUNK):
+    """Gradient contributions of the keys of one partition (the chunks the CSR
+    lists), given the full attention's output ``out`` and natural-log ``lse``
+    ([B, heads, N]) for the queries. q, dout, out: the query grid; k, v: the
+    key grid (same T, H, W). Returns dq_rows [n, 128, d] and dk, dv
+    [B, heads, N, d] like ``attend_bwd``; the sums over a partition of the keys
+    equal ``attend_bwd``. float64 throughout."""
+    q, k, v, dout, out = _f64(q), _f64(k), _f64(v), _f64(dout), _f64(out)
+    lse = np.ascontiguousarray(lse, dtype=np.float64)
+    B, Hh, N, d = q.shape
+    assert lse.shape == (B, Hh, N) and out.shape == q.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    rp = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    ci = np.ascontiguousarray(col_idx, dtype=np.int32)
+    if ci.size == 0:
+        ci = np.zeros(1, dtype=np.int32)
+    dq = np.empty((rows.size, CN, d), dtype=np.float64)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    _check(_load().oracle_attend_bwd_part_shape(
+        q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data, out.ctypes.data,
+        lse.ctypes.data, B * Hh, T, H, W, *kchunk, d, float(scale), rp.ctypes.data,
+        ci.ctypes.data, rows.ctypes.data, rows.size, dq.ctypes.data, dk.ctypes.data,
+        dv.ctypes.data), "oracle_attend_bwd_part")
     return dq, dk, dv
 
 

@@ -582,6 +582,123 @@ int oracle_attend_bwd_shape(const double* q, const double* k, const double* v, c
     return 0;
 }
 
+/*
+ * The gradient contributions of one partition of the keys, for context
+ * parallelism ([P1] "Block Sparse Attention (BSA)", ring block sparse
+ * attention: the keys of a query are split across the ranks of the group; [P3]
+ * "开源实现": the trainable BSA's backward kernels and the LSE correction for
+ * context parallelism). The softmax of a query runs over ALL its keys, so its
+ * weights on the keys of one partition need the whole set's log-sum-exp and
+ * the whole output: with lse[q] (natural log) and out[q] of the full
+ * attention,
+ *   P[q,j]  = exp(s[q,j] - lse[q])          for the keys j of this partition
+ *   Dq      = <dout[q], out[q]>
+ *   dS[q,j] = P[q,j] (<dout[q], v_j> - Dq)
+ *   dQ[q]   = scale * sum_j dS[q,j] k_j,  dK[j] += scale * dS[q,j] q,
+ *   dV[j]  += P[q,j] dout[q]
+ * and the gradients of the full attention are the sums of these over the
+ * partitions (every term of the chain rule above is a sum over keys). The CSR
+ * lists the partition's chunks per query row, in the key grid (T,H,W) and key
+ * chunk shape (kst,ksh,ksw); q, dout, out, lse live on the query grid, which
+ * has the same (T,H,W) (one rank's shard of queries against one shard of
+ * keys). Outputs as oracle_attend_bwd_shape: dq_rows for the listed rows
+ * (NaN for query slots past the grid edge, 0 for a row with no chunk of the
+ * partition), dk/dv accumulated. fp64.
+ */
+int oracle_attend_bwd_part_shape(const double* q, const double* k, const double* v,
+                                 const double* dout, const double* out, const double* lse, int BH,
+                                 int T, int H, int W, int kst, int ksh, int ksw, int d,
+                                 double scale, const int32_t* row_ptr, const int32_t* col_idx,
+                                 const int64_t* rows, int64_t n_rows, double* dq_rows, double* dk,
+                                 double* dv) {
+    if (!q || !k || !v || !dout || !out || !lse || !row_ptr || !col_idx || !rows || !dq_rows ||
+        !dk || !dv || BH <= 0 || d <= 0 || !grid_ok(T, H, W) || kst <= 0 || ksh <= 0 || ksw <= 0)
+        return -1;
+    const int kn = kst * ksh * ksw;
+    const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks(T, H, W);
+    for (int64_t n = 0; n < n_rows; ++n)
+        if (rows[n] < 0 || rows[n] >= (int64_t)BH * Nc) return -1;
+    int64_t cap_keys = 0;
+    int64_t* ktok = NULL;
+    double* P = NULL;
+    double* dS = NULL;
+    for (int64_t n = 0; n < n_rows; ++n) {
+        const int64_t r = rows[n];
+        const int64_t bh = r / Nc, i = r % Nc;
+        const int64_t beg = row_ptr[r], end = row_ptr[r + 1];
+        const int64_t slots = (end - beg) * kn;
+        double* dqr = dq_rows + n * CN * d;
+        if (slots > cap_keys) {
+            free(ktok); free(P); free(dS);
+            ktok = (int64_t*)malloc(sizeof(int64_t) * (size_t)slots);
+            P = (double*)malloc(sizeof(double) * (size_t)(CN * slots));
+            dS = (double*)malloc(sizeof(double) * (size_t)(CN * slots));
+            cap_keys = slots;
+        }
+        int64_t nk = 0;
+        for (int64_t e = beg; e < end; ++e)
+            for (int l = 0; l < kn; ++l) {
+                const int64_t tok = oracle_token_of_shape(T, H, W, kst, ksh, ksw, col_idx[e], l);
+                if (tok >= 0) ktok[nk++] = bh * N + tok;
+            }
+        for (int lq = 0; lq < CN; ++lq) {
+            const int exists = oracle_token_of(T, H, W, i, lq) >= 0;
+            for (int x = 0; x < d; ++x) dqr[(int64_t)lq * d + x] = exists ? 0.0 : NAN;
+        }
+        if (nk <= 0) continue;
+#pragma omp parallel for schedule(static)
+        for (int lq = 0; lq < CN; ++lq) {
+            const int64_t qtok = oracle_token_of(T, H, W, i, lq);
+            double* p = P + (int64_t)lq * nk;
+            double* ds = dS + (int64_t)lq * nk;
+            if (qtok < 0) {
+                for (int64_t j = 0; j < nk; ++j) p[j] = ds[j] = 0.0;
+                continue;
+            }
+            const int64_t qt = bh * N + qtok;
+            const double* qr = q + qt * d;
+            const double* gr = dout + qt * d;
+            const double* orow = out + qt * d;
+            double D = 0.0;
+            for (int x = 0; x < d; ++x) D += gr[x] * orow[x];
+            double* dqq = dqr + (int64_t)lq * d;
+            for (int64_t j = 0; j < nk; ++j) {
+                const double* kr = k + ktok[j] * d;
+                const double* vr = v + ktok[j] * d;
+                double s = 0.0, dp = 0.0;
+                for (int x = 0; x < d; ++x) {
+                    s += qr[x] * kr[x];
+                    dp += gr[x] * vr[x];
+                }
+                p[j] = exp(s * scale - lse[qt]);
+                ds[j] = p[j] * (dp - D);
+                for (int x = 0; x < d; ++x) dqq[x] += ds[j] * kr[x];
+            }
+            for (int x = 0; x < d; ++x) dqq[x] *= scale;
+        }
+#pragma omp parallel for schedule(static)
+        for (int64_t j = 0; j < nk; ++j) {
+            double* dkr = dk + ktok[j] * d;
+            double* dvr = dv + ktok[j] * d;
+            for (int lq = 0; lq < CN; ++lq) {
+                const int64_t qtok = oracle_token_of(T, H, W, i, lq);
+                if (qtok < 0) continue;
+                const int64_t qt = bh * N + qtok;
+                const double pw = P[(int64_t)lq * nk + j];
+                const double sw = dS[(int64_t)lq * nk + j] * scale;
+                const double* qr = q + qt * d;
+                const double* gr = dout + qt * d;
+                for (int x = 0; x < d; ++x) {
+                    dvr[x] += pw * gr[x];
+                    dkr[x] += sw * qr[x];
+                }
+            }
+        }
+    }
+    free(ktok); free(P); free(dS);
+    return 0;
+}
+
 int oracle_attend_bwd(const double* q, const double* k, const double* v, const double* dout,
                       int BH, int T, int H, int W, int d, double scale, const int32_t* row_ptr,
                       const int32_t* col_idx, const int64_t* rows, int64_t n_rows,

@@ -64,3 +64,67 @@ def test_merge_is_commutative_associative_and_keeps_empty_parts():
     assert np.array_equal(m, o0) and np.array_equal(lm, l0)
     m, lm = oracle.lse_merge(np.zeros((n, d)), e, o1, e)
     assert not m.any() and np.all(np.isneginf(lm))
+
+
+def _rows_to_tokens(x_rows, T, H, W, B, heads, nc):
+    """[B*heads*nc, 128, ...] chunk rows -> [B, heads, N, ...] THW tokens."""
+    N = T * H * W
+    out = np.zeros((B * heads, N) + x_rows.shape[2:], dtype=np.float64)
+    for c in range(nc):
+        tok = oracle.chunk_tokens(T, H, W, c)
+        ok = tok >= 0
+        for bh in range(B * heads):
+            out[bh, tok[ok]] = x_rows[bh * nc + c][ok]
+    return out.reshape((B, heads, N) + x_rows.shape[2:])
+
+
+def _backward_case(wl, topk):
+    q, k, v = synth.make_qkv(wl)
+    dout = synth.make_dout(wl)
+    scale = 1 / math.sqrt(wl.d)
+    rp, ci, _ = oracle.plan(q, k, wl.T, wl.H, wl.W, scale, "topk", topk)
+    nc = oracle.num_chunks(wl.T, wl.H, wl.W)
+    rows = np.arange(wl.B * wl.heads * nc)
+    o, l = oracle.attend(q, k, v, wl.T, wl.H, wl.W, scale, rp, ci, rows)
+    out = _rows_to_tokens(o, wl.T, wl.H, wl.W, wl.B, wl.heads, nc)
+    lse = _rows_to_tokens(l, wl.T, wl.H, wl.W, wl.B, wl.heads, nc)
+    full = oracle.attend_bwd(q, k, v, dout, wl.T, wl.H, wl.W, scale, rp, ci, rows)
+    return q, k, v, dout, out, lse, scale, rp, ci, rows, full
+
+
+def test_backward_over_key_partitions_sums_to_full_backward():
+    """Ring block sparse attention splits every query's keys across ranks; the
+    gradient terms of the chain rule are sums over keys, so the contributions
+    of disjoint key partitions (each weighted with the whole softmax: the full
+    log-sum-exp and output) must add up to the backward of the unsplit
+    attention (attend_bwd, pinned by finite differences). A partition that used
+    its own softmax instead of the whole one fails this."""
+    for wl, topk in ((synth.WORKLOADS["tiny"].with_(T=16, H=8, W=16, heads=2, d=32), 6),
+                     (synth.WORKLOADS["tiny"].with_(T=10, H=6, W=13, heads=1, d=16), 5)):
+        q, k, v, dout, out, lse, scale, rp, ci, rows, (fq, fk, fv) = _backward_case(wl, topk)
+        nc = oracle.num_chunks(wl.T, wl.H, wl.W)
+        for split in (nc // 2, 1, nc - 1):
+            (ra, ca), (rb, cb) = split_csr(rp, ci, lambda c: c < split)
+            aq, ak, av = oracle.attend_bwd_part(q, k, v, dout, out, lse, wl.T, wl.H, wl.W, scale,
+                                                ra, ca, rows)
+            bq, bk, bv = oracle.attend_bwd_part(q, k, v, dout, out, lse, wl.T, wl.H, wl.W, scale,
+                                                rb, cb, rows)
+            np.testing.assert_allclose(aq + bq, fq, rtol=0, atol=1e-11 * np.nanmax(np.abs(fq)))
+            np.testing.assert_allclose(ak + bk, fk, rtol=0, atol=1e-11 * np.abs(fk).max())
+            np.testing.assert_allclose(av + bv, fv, rtol=0, atol=1e-11 * np.abs(fv).max())
+            # query slots past the grid edge carry no gradient in either
+            assert np.array_equal(np.isnan(aq), np.isnan(fq))
+
+
+def test_backward_of_the_whole_key_set_and_of_an_empty_one():
+    wl = synth.WORKLOADS["tiny"].with_(T=8, H=8, W=16, heads=2, d=32)
+    q, k, v, dout, out, lse, scale, rp, ci, rows, (fq, fk, fv) = _backward_case(wl, 3)
+    aq, ak, av = oracle.attend_bwd_part(q, k, v, dout, out, lse, wl.T, wl.H, wl.W, scale, rp, ci,
+                                        rows)
+    np.testing.assert_allclose(aq, fq, rtol=0, atol=1e-11 * np.abs(fq).max())
+    np.testing.assert_allclose(ak, fk, rtol=0, atol=1e-11 * np.abs(fk).max())
+    np.testing.assert_allclose(av, fv, rtol=0, atol=1e-11 * np.abs(fv).max())
+    empty_rp = np.zeros_like(rp)
+    eq, ek, ev = oracle.attend_bwd_part(q, k, v, dout, out, lse, wl.T, wl.H, wl.W, scale, empty_rp,
+                                        np.zeros(0, np.int32), rows)
+    assert not eq.any() and not ek.any() and not ev.any()
