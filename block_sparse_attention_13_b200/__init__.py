@@ -40,7 +40,7 @@ EXPORTED = ("bsa_version", "bsa_status_string", "bsa_workspace_size", "bsa_plan_
             "bsa_rearrange", "bsa_pool", "bsa_scores", "bsa_selftest_exp2",
             "bsa_selftest_timeout", "bsa_backward_workspace_size", "bsa_backward",
             "bsa_select_pooled", "bsa_csr_slice_workspace_size", "bsa_csr_slice",
-            "bsa_lse_merge")
+            "bsa_lse_merge", "bsa_grad_accumulate", "bsa_grad_finalize")
 
 
 class BsaError(RuntimeError):
@@ -112,6 +112,8 @@ def lib():
             "bsa_csr_slice_workspace_size": (sz, [i64]),
             "bsa_csr_slice": (i32, [i64, vp, vp, i64, i32, i32, vp, sz, vp, vp, i64, vp]),
             "bsa_lse_merge": (i32, [P, vp, vp, vp, vp, vp]),
+            "bsa_grad_accumulate": (i32, [P, vp, vp, i32, vp]),
+            "bsa_grad_finalize": (i32, [P, vp, vp, vp]),
             "bsa_backward": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, vp,
                                    vp]),
         }
@@ -232,6 +234,16 @@ def bsa_csr_slice(row_ptr, col_idx, lo, hi, workspace, out_row_ptr, out_col_idx,
 def bsa_lse_merge(p, out, lse, out_part, lse_part, stream=None):
     _check(lib().bsa_lse_merge(ctypes.byref(p), _ptr(out), _ptr(lse), _ptr(out_part),
                                _ptr(lse_part), _stream(stream)), "bsa_lse_merge")
+
+
+def bsa_grad_accumulate(p, part, acc, overwrite=False, stream=None):
+    _check(lib().bsa_grad_accumulate(ctypes.byref(p), _ptr(part), _ptr(acc), 1 if overwrite else 0,
+                                     _stream(stream)), "bsa_grad_accumulate")
+
+
+def bsa_grad_finalize(p, acc, out, stream=None):
+    _check(lib().bsa_grad_finalize(ctypes.byref(p), _ptr(acc), _ptr(out), _stream(stream)),
+           "bsa_grad_finalize")
 
 
 def bsa_read_status(workspace, stream=None) -> int:

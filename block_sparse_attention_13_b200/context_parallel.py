@@ -9,6 +9,14 @@ computed shard by shard while the K/V shards travel around the ring, the
 partial results being combined by their log-sum-exps ("LongCat-Video
 Technical Report #", section "开源实现": LSE and output correction).
 
+The backward (``ring_backward``) runs the same ring again. At each step a rank
+computes, with bsa_backward, the contributions of the K/V shard it holds to
+its queries' dQ and to that shard's dK and dV, weighted with the merged
+output and LSE of the forward (the softmax over all shards). dQ sums the
+contributions of every shard on the rank (fp32, bsa_grad_accumulate); dK and
+dV of a shard sum the contributions of every rank, which one NCCL
+reduce-scatter of the ranks' fp32 contributions delivers to the shard's owner.
+
 On one node of B200s the gather is an NCCL all-gather of the pooled keys
 (Nc x d floats per head and rank) and the ring step an NCCL send/receive of
 the next K/V shard, posted before the current shard's attention so that the
@@ -21,7 +29,8 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import (BSA_OK, BsaError, bsa_csr_slice, bsa_csr_slice_workspace_size, bsa_forward,
+from . import (BSA_OK, BsaError, backward_workspace, bsa_backward, bsa_csr_slice,
+               bsa_csr_slice_workspace_size, bsa_forward, bsa_grad_accumulate, bsa_grad_finalize,
                bsa_lse_merge, bsa_plan_sizes, bsa_pool, bsa_read_status, bsa_select_pooled,
                bsa_workspace_size, make_params, status_string)
 
@@ -71,6 +80,21 @@ class CudaOps:
     def merge(self, p, out, lse, out_part, lse_part):
         bsa_lse_merge(p, out, lse, out_part, lse_part)
 
+    def backward(self, p, q, k, v, out, lse, dout, row_ptr, col_idx):
+        ws = backward_workspace(p, q.device)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        bsa_backward(p, q, k, v, out, lse, dout, row_ptr, col_idx, ws, dq, dk, dv)
+        self._status.append(ws)
+        return dq, dk, dv
+
+    def accumulate(self, p, part, acc, overwrite):
+        bsa_grad_accumulate(p, part, acc, overwrite)
+
+    def finalize(self, p, acc):
+        out = torch.empty(acc.shape, dtype=torch.bfloat16, device=acc.device)
+        bsa_grad_finalize(p, acc, out)
+        return out
+
     def check(self):
         for ws in self._status:
             rc = bsa_read_status(ws)
@@ -113,16 +137,31 @@ class TorchComm:
             r.wait()
         return recv
 
+    def reduce_scatter(self, x):
+        """x: [world, *shape] on every rank; returns the sum over ranks of their
+        x[rank] slice, on each rank."""
+        out = torch.empty(tuple(x.shape[1:]), dtype=x.dtype, device=x.device)
+        if dist.get_backend(self.group) == "gloo":
+            # gloo has no reduce-scatter: reduce the whole buffer, keep this slice
+            buf = x.contiguous().clone()
+            dist.all_reduce(buf, group=self.group)
+            out.copy_(buf[self.rank])
+        else:
+            dist.reduce_scatter_tensor(out, x.contiguous(), group=self.group)
+        return out
+
 
 def ring_forward(q, k, v, grid, topk=None, mode="topk", cdf_p=0.9, cdf_cap_frac=0.25, t_cond=0,
-                 scale=0.0, comm=None, ops=None):
+                 scale=0.0, comm=None, ops=None, return_csr=False):
     """Block sparse attention of this rank's queries over the whole group's sequence.
 
     q, k, v: this rank's shard, [B, heads, T_l*H*W, d] bf16, holding latent frames
     [rank*T_l, (rank+1)*T_l) of the group's grid (T_l * world, H, W); grid = (T_l, H, W),
     T_l a multiple of 4. topk defaults to 1/16 of the group's key chunks. t_cond counts
     frames of the whole sequence. Returns (out, lse) for the local queries, as
-    bsa_forward would give for these rows of the unsplit sequence.
+    bsa_forward would give for these rows of the unsplit sequence; with
+    return_csr also the rank's selection (row_ptr, col_idx over the key chunks of
+    the whole sequence, shard layout), which ring_backward takes.
     """
     comm = comm or TorchComm()
     ops = ops or CudaOps()
@@ -158,4 +197,67 @@ def ring_forward(q, k, v, grid, topk=None, mode="topk", cdf_p=0.9, cdf_cap_frac=
         if handle is not None:
             k_cur, v_cur = comm.finish_shift(handle)
     ops.check()
+    if return_csr:
+        return out, lse, row_ptr, col_idx
     return out, lse
+
+
+def _local_params(q, grid, scale):
+    B, heads, N, d = q.shape
+    T_l, H, W = grid
+    if T_l % 4:
+        raise ValueError("each rank must hold whole chunks: T_l must be a multiple of 4")
+    if N != T_l * H * W:
+        raise ValueError("q does not hold T_l*H*W tokens")
+    nc_l = (T_l // 4) * ((H + 3) // 4) * ((W + 7) // 8)
+    return make_params(B, heads, T_l, H, W, d, "topk", 1, 0.9, 0.25, 0, scale), nc_l
+
+
+def ring_backward_partials(q, k, v, out, lse, dout, row_ptr, col_idx, grid, scale=0.0,
+                           comm=None, ops=None):
+    """The per-rank part of ring_backward, before the dK/dV reduction.
+
+    Returns (dq_acc, dkv_parts): dq_acc fp32 [B, heads, N_l, d], the complete dQ of
+    the local queries; dkv_parts fp32 [2, world, B, heads, N_l, d], this rank's
+    contributions to dK (index 0) and dV (index 1) of every shard.
+    """
+    comm = comm or TorchComm()
+    ops = ops or CudaOps()
+    world, rank = comm.world, comm.rank
+    p, nc_l = _local_params(q, grid, scale)
+    dq_acc = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dkv_parts = torch.empty((2, world) + tuple(k.shape), dtype=torch.float32, device=k.device)
+    k_cur, v_cur = k, v
+    for s in range(world):
+        j = (rank - s) % world                   # the shard held at this step
+        handle = comm.start_shift([k_cur, v_cur]) if s + 1 < world else None
+        srp, sci = ops.slice(row_ptr, col_idx, j * nc_l, (j + 1) * nc_l)
+        dq_p, dk_p, dv_p = ops.backward(p, q, k_cur, v_cur, out, lse, dout, srp, sci)
+        ops.accumulate(p, dq_p, dq_acc, s == 0)
+        ops.accumulate(p, dk_p, dkv_parts[0, j], True)
+        ops.accumulate(p, dv_p, dkv_parts[1, j], True)
+        if handle is not None:
+            k_cur, v_cur = comm.finish_shift(handle)
+    return dq_acc, dkv_parts
+
+
+def ring_backward(q, k, v, out, lse, dout, row_ptr, col_idx, grid, scale=0.0, comm=None,
+                  ops=None):
+    """Gradients of ring_forward for this rank's upstream gradient dout.
+
+    q, k, v, dout: this rank's shard [B, heads, T_l*H*W, d] bf16; out, lse: what
+    ring_forward returned (the merged output and LSE over all shards); row_ptr,
+    col_idx: the selection ring_forward returned with return_csr. Returns
+    (dq, dk, dv) bf16 for the local queries and the local K/V shard: the rows of
+    the unsplit sequence's gradients, summed in fp32 before the final rounding.
+    """
+    comm = comm or TorchComm()
+    ops = ops or CudaOps()
+    p, _ = _local_params(q, grid, scale)
+    dq_acc, dkv_parts = ring_backward_partials(q, k, v, out, lse, dout, row_ptr, col_idx, grid,
+                                               scale, comm, ops)
+    dk_acc = comm.reduce_scatter(dkv_parts[0])
+    dv_acc = comm.reduce_scatter(dkv_parts[1])
+    dq, dk, dv = ops.finalize(p, dq_acc), ops.finalize(p, dk_acc), ops.finalize(p, dv_acc)
+    ops.check()
+    return dq, dk, dv

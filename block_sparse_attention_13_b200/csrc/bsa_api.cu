@@ -372,6 +372,29 @@ int bsa_lse_merge(const bsa_params* p, void* out, float* lse, const void* out_pa
                                         static_cast<cudaStream_t>(stream)));
 }
 
+int bsa_grad_accumulate(const bsa_params* p, const void* part, float* acc, int overwrite,
+                        void* stream) {
+    Dims g;
+    int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!part || !acc || (overwrite != 0 && overwrite != 1)) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(part) || !aligned16(acc)) return BSA_ERR_ALIGNMENT;
+    if ((rc = device_ok()) != BSA_OK) return rc;
+    return cuda_status(launch_grad_accumulate(g.BH * g.N * g.d, part, acc, overwrite,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_grad_finalize(const bsa_params* p, const float* acc, void* out, void* stream) {
+    Dims g;
+    int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!acc || !out) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(acc) || !aligned16(out)) return BSA_ERR_ALIGNMENT;
+    if ((rc = device_ok()) != BSA_OK) return rc;
+    return cuda_status(launch_grad_finalize(g.BH * g.N * g.d, acc, out,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 int bsa_read_status(void* workspace, void* stream) {
     if (!workspace) return BSA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -6,7 +6,9 @@
 // attends over each rank's K/V shard in turn and folds the partial results
 // together with their log-sum-exps. This file holds the two device steps that
 // are specific to that: slicing the selection to one shard's key chunks, and
-// merging a partial result into the running one.
+// merging a partial result into the running one. For the backward of the ring
+// it holds the fp32 accumulation of the per-shard gradient contributions and
+// their final rounding to bf16.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -116,7 +118,70 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(__nv_bfloat16* __restric
     if (v % VPT == 0) lse[tok] = l;
 }
 
+// acc (fp32) = part (bf16), or acc += part; 8 elements per thread and step.
+__global__ void __launch_bounds__(256) grad_accumulate_kernel(const uint4* __restrict__ part,
+                                                              float4* __restrict__ acc,
+                                                              int64_t n8, int overwrite) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 pv = part[i];
+        const uint32_t w[4] = {pv.x, pv.y, pv.z, pv.w};
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {  // bf16 -> fp32 is exact: the bits move up 16 places
+            f[2 * e] = __uint_as_float(w[e] << 16);
+            f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+        }
+        float4 a0 = make_float4(f[0], f[1], f[2], f[3]), a1 = make_float4(f[4], f[5], f[6], f[7]);
+        if (!overwrite) {
+            const float4 b0 = acc[2 * i], b1 = acc[2 * i + 1];
+            a0 = make_float4(b0.x + a0.x, b0.y + a0.y, b0.z + a0.z, b0.w + a0.w);
+            a1 = make_float4(b1.x + a1.x, b1.y + a1.y, b1.z + a1.z, b1.w + a1.w);
+        }
+        acc[2 * i] = a0;
+        acc[2 * i + 1] = a1;
+    }
+}
+
+// out (bf16, round to nearest even) = acc (fp32).
+__global__ void __launch_bounds__(256) grad_finalize_kernel(const float4* __restrict__ acc,
+                                                            uint4* __restrict__ out, int64_t n8) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 a0 = acc[2 * i], a1 = acc[2 * i + 1];
+        out[i] = make_uint4(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w),
+                            pack_bf16x2(a1.x, a1.y), pack_bf16x2(a1.z, a1.w));
+    }
+}
+
+// Elementwise passes over HBM: at most 8 resident 256-thread blocks per SM,
+// grid-striding over the rest.
+unsigned stream_blocks(int64_t n8) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (n8 + 255) / 256, cap = static_cast<int64_t>(sms) * 8;
+    return static_cast<unsigned>(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
 }  // namespace
+
+cudaError_t launch_grad_accumulate(int64_t n, const void* part, float* acc, int overwrite,
+                                   cudaStream_t st) {
+    const int64_t n8 = n / 8;
+    if (n8 == 0) return cudaSuccess;
+    grad_accumulate_kernel<<<stream_blocks(n8), 256, 0, st>>>(
+        static_cast<const uint4*>(part), reinterpret_cast<float4*>(acc), n8, overwrite);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_grad_finalize(int64_t n, const float* acc, void* out, cudaStream_t st) {
+    const int64_t n8 = n / 8;
+    if (n8 == 0) return cudaSuccess;
+    grad_finalize_kernel<<<stream_blocks(n8), 256, 0, st>>>(reinterpret_cast<const float4*>(acc),
+                                                            static_cast<uint4*>(out), n8);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_csr_slice(int64_t rows, const int32_t* row_ptr, const int32_t* col_idx,
                              int64_t col_cap, int lo, int hi, int32_t* counts, int32_t* out_row_ptr,

@@ -115,6 +115,9 @@ cudaError_t launch_csr_slice(int64_t rows, const int32_t* row_ptr, const int32_t
                              cudaStream_t st);
 cudaError_t launch_lse_merge(const Dims& g, void* out, float* lse, const void* out_part,
                              const float* lse_part, cudaStream_t st);
+cudaError_t launch_grad_accumulate(int64_t n, const void* part, float* acc, int overwrite,
+                                   cudaStream_t st);
+cudaError_t launch_grad_finalize(int64_t n, const float* acc, void* out, cudaStream_t st);
 cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, int64_t n,
                                  cudaStream_t st);
 cudaError_t launch_selftest_timeout(uint32_t* status, uint64_t timeout_ns, cudaStream_t st);

@@ -246,6 +246,30 @@ BSA_API int bsa_lse_merge(const bsa_params* p, void* out, float* lse, const void
                           const float* lse_part, void* stream);
 
 /*
+ * Backward of the ring ([P1] ring block sparse attention; [P3] "开源实现":
+ * the trainable BSA's backward kernels and the LSE correction for context
+ * parallelism). bsa_backward over one K/V shard, given the merged output and
+ * LSE of the whole ring, yields that shard's contributions to dQ, dK and dV;
+ * each gradient is the sum of its contributions over the shards (dQ) or over
+ * the ranks (dK, dV). These two calls keep that sum in fp32:
+ *
+ * acc <- part (overwrite = 1) or acc <- acc + part (overwrite = 0), for the
+ * B*heads*N*d elements of the grid `p` describes. part: device bf16
+ * [B,heads,N,d] (a gradient as bsa_backward writes it); acc: device fp32 of
+ * the same shape. Both 16-byte aligned. Errors: INVALID_ARG, SHAPE,
+ * UNSUPPORTED, ALIGNMENT, CUDA.
+ */
+BSA_API int bsa_grad_accumulate(const bsa_params* p, const void* part, float* acc, int overwrite,
+                                void* stream);
+
+/*
+ * out <- acc rounded to bf16 (nearest even), for the grid `p` describes.
+ * acc: device fp32 [B,heads,N,d]; out: device bf16 of the same shape. Both
+ * 16-byte aligned. Errors: INVALID_ARG, SHAPE, UNSUPPORTED, ALIGNMENT, CUDA.
+ */
+BSA_API int bsa_grad_finalize(const bsa_params* p, const float* acc, void* out, void* stream);
+
+/*
  * bsa_plan without a caller workspace: the same selection as bsa_plan, with
  * its scratch held in a fixed array inside this library, for callers that
  * cannot allocate device memory (a plug-in whose host engine owns the memory

@@ -90,6 +90,32 @@ class OracleOps:
         out.copy_(torch.from_numpy(m))
         lse.copy_(torch.from_numpy(lm))
 
+    def backward(self, p, q, k, v, out, lse, dout, rp, ci):
+        T, H, W = p.T, p.H, p.W
+        nc = oracle.num_chunks(T, H, W)
+        rows = np.arange(p.B * p.heads * nc)
+        dq_rows, dk, dv = oracle.attend_bwd_part(_bits(q), _bits(k), _bits(v), _bits(dout),
+                                                 out.numpy(), lse.numpy(), T, H, W,
+                                                 1.0 / math.sqrt(p.d), rp.numpy(), ci.numpy(),
+                                                 rows)
+        N = T * H * W
+        dq = np.zeros((p.B * p.heads, N, p.d))
+        for r in rows:
+            tok = oracle.chunk_tokens(T, H, W, r % nc)
+            ok = tok >= 0
+            dq[r // nc][tok[ok]] = dq_rows[r][ok]
+        return (torch.from_numpy(dq.reshape(p.B, p.heads, N, p.d)), torch.from_numpy(dk),
+                torch.from_numpy(dv))
+
+    def accumulate(self, p, part, acc, overwrite):
+        if overwrite:
+            acc.copy_(part)
+        else:
+            acc.add_(part.to(acc.dtype))
+
+    def finalize(self, p, acc):
+        return acc.double()
+
     def check(self):
         pass
 
@@ -101,7 +127,7 @@ WORKLOADS = {
 }
 
 
-def _worker(rank, world, port, name, result_dir):
+def _worker(rank, world, port, name, result_dir, backward=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
     try:
@@ -112,11 +138,19 @@ def _worker(rank, world, port, name, result_dir):
         T_l = wl.T // world
         sl = slice(rank * T_l * HW, (rank + 1) * T_l * HW)
         qs, ks, vs = (torch.from_numpy(x[:, :, sl].copy()).view(torch.bfloat16) for x in (q, k, v))
-        out, lse = ring_forward(qs, ks, vs, (T_l, wl.H, wl.W), wl.topk, wl.mode, wl.cdf_p,
-                                wl.cdf_cap_frac, wl.t_cond, comm=TorchComm(),
-                                ops=OracleOps(wl, world))
+        comm, ops = TorchComm(), OracleOps(wl, world)
+        out, lse, rp, ci = ring_forward(qs, ks, vs, (T_l, wl.H, wl.W), wl.topk, wl.mode,
+                                        wl.cdf_p, wl.cdf_cap_frac, wl.t_cond, comm=comm, ops=ops,
+                                        return_csr=True)
         np.save(os.path.join(result_dir, f"out{rank}.npy"), out.numpy())
         np.save(os.path.join(result_dir, f"lse{rank}.npy"), lse.numpy())
+        if backward:
+            from block_sparse_attention_13_b200.context_parallel import ring_backward
+            dout = torch.from_numpy(synth.make_dout(wl)[:, :, sl].copy()).view(torch.bfloat16)
+            dq, dk, dv = ring_backward(qs, ks, vs, out, lse, dout, rp, ci, (T_l, wl.H, wl.W),
+                                       comm=comm, ops=ops)
+            for nm, x in (("dq", dq), ("dk", dk), ("dv", dv)):
+                np.save(os.path.join(result_dir, f"{nm}{rank}.npy"), x.numpy())
     finally:
         dist.destroy_process_group()
 
@@ -145,3 +179,36 @@ def test_ring_forward_on_gloo_ranks(tmp_path, name, world):
         got_l = np.load(tmp_path / f"lse{rank}.npy").reshape(wl.B * wl.heads, -1)
         np.testing.assert_allclose(got, full[:, sl], rtol=0, atol=1e-12)
         np.testing.assert_allclose(got_l, full_l[:, sl], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("name,world", [("topk", 2), ("topk", 4), ("causal_cdf", 2)])
+def test_ring_backward_on_gloo_ranks(tmp_path, name, world):
+    """dQ of each rank's queries and dK, dV of each rank's shard must equal the
+    rows of the unsplit oracle backward: the shard contributions weighted with
+    the merged softmax, dQ summed over the ring's steps and dK/dV over the
+    ranks by the reduce-scatter."""
+    mp.spawn(_worker, args=(world, _free_port(), name, str(tmp_path), True), nprocs=world,
+             join=True)
+    wl = WORKLOADS[name]
+    q, k, v = synth.make_qkv(wl)
+    dout = synth.make_dout(wl)
+    scale = 1.0 / math.sqrt(wl.d)
+    rp, ci, _ = oracle.plan(q, k, wl.T, wl.H, wl.W, scale, wl.mode, wl.topk, wl.cdf_p,
+                            wl.cdf_cap_frac, wl.t_cond)
+    rows = np.arange(wl.rows)
+    dq_rows, dk, dv = oracle.attend_bwd(q, k, v, dout, wl.T, wl.H, wl.W, scale, rp, ci, rows)
+    dq = np.zeros((wl.B * wl.heads, wl.N, wl.d))
+    for r in rows:
+        tok = oracle.chunk_tokens(wl.T, wl.H, wl.W, r % wl.Nc)
+        dq[r // wl.Nc][tok] = dq_rows[r]
+    full = {"dq": dq, "dk": dk.reshape(wl.B * wl.heads, wl.N, wl.d),
+            "dv": dv.reshape(wl.B * wl.heads, wl.N, wl.d)}
+    HW = wl.H * wl.W
+    T_l = wl.T // world
+    for rank in range(world):
+        sl = slice(rank * T_l * HW, (rank + 1) * T_l * HW)
+        for nm in ("dq", "dk", "dv"):
+            got = np.load(tmp_path / f"{nm}{rank}.npy").reshape(wl.B * wl.heads, -1, wl.d)
+            ref = full[nm][:, sl]
+            # fp32 accumulators of fp64 contributions
+            np.testing.assert_allclose(got, ref, rtol=0, atol=2e-6 * np.abs(full[nm]).max())

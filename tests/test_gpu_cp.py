@@ -18,7 +18,9 @@ from test_gpu_parity import dev, gather_rows, host_f32
 pytestmark = pytest.mark.gpu
 
 import block_sparse_attention_13_b200 as bsa  # noqa: E402
-from block_sparse_attention_13_b200.context_parallel import CudaOps, ring_forward  # noqa: E402
+from block_sparse_attention_13_b200.context_parallel import (CudaOps, ring_backward,  # noqa: E402
+                                                            ring_backward_partials, ring_forward)
+from test_gpu_backward import BWD_MAX_REL, BWD_MEAN_REL, rel_errors  # noqa: E402
 
 
 class SimComm:
@@ -40,6 +42,11 @@ class SimComm:
 
     def finish_shift(self, j):
         return [self.k[j], self.v[j]]
+
+    def reduce_scatter(self, x):
+        # only a one-rank group can be answered without the other ranks' buffers
+        assert self.world == 1
+        return x[0].clone()
 
 
 def shard(x, world, frames, HW):
@@ -147,3 +154,116 @@ def test_csr_slice_and_merge_units():
     diff = (o.float() - of.float()).abs()
     assert float(diff.max()) <= ATT_MAX_ABS and float(diff.mean()) <= ATT_MEAN_ABS / 2
     torch.testing.assert_close(l, lf, rtol=0, atol=1e-4)
+
+
+def _unsplit_backward(wl, qd, kd, vd, gd):
+    p = bsa.params_for(wl)
+    pl = bsa.allocate(p)
+    bsa.bsa_plan(p, qd, kd, pl.workspace, pl.row_ptr, pl.col_idx)
+    out = torch.empty_like(qd)
+    lse = torch.empty((wl.B, wl.heads, wl.N), dtype=torch.float32, device="cuda")
+    bsa.bsa_forward(p, qd, kd, vd, pl.row_ptr, pl.col_idx, pl.workspace, out, lse)
+    ws = bsa.backward_workspace(p)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    bsa.bsa_backward(p, qd, kd, vd, out, lse, gd, pl.row_ptr, pl.col_idx, ws, dq, dk, dv)
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_OK
+    assert bsa.bsa_read_status(ws) == bsa.BSA_OK
+    rp = pl.row_ptr.cpu().numpy()
+    return rp, pl.col_idx[: int(rp[-1])].cpu().numpy(), dq, dk, dv
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_ring_backward_equals_unsplit(name):
+    """Each rank's ring backward, run one rank after another with the K/V shards
+    each step would deliver, and the dK/dV contributions summed over the ranks as
+    the reduce-scatter would: the gradients must match the unsplit backward and
+    the oracle within the backward bars (the shard contributions are rounded to
+    bf16 before their fp32 sum)."""
+    wl, world = CASES[name]
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    HW = wl.H * wl.W
+    T_l = wl.T // world
+    qd, kd, vd, gd = dev(q), dev(k), dev(v), dev(g)
+    g_rp, g_ci, dq_g, dk_g, dv_g = _unsplit_backward(wl, qd, kd, vd, gd)
+    qs, ks, vs, gs = (shard(x, world, T_l, HW) for x in (qd, kd, vd, gd))
+    ops = CudaOps()
+    p_local = bsa.make_params(wl.B, wl.heads, T_l, wl.H, wl.W, wl.d, wl.mode, wl.topk)
+    kp_all = torch.stack([ops.pool(p_local, ks[r]) for r in range(world)])
+    grid = (T_l, wl.H, wl.W)
+    dq_full = torch.empty_like(qd)
+    parts = []
+    for r in range(world):
+        out, lse, rp, ci = ring_forward(qs[r], ks[r], vs[r], grid, wl.topk, wl.mode, wl.cdf_p,
+                                        wl.cdf_cap_frac, wl.t_cond,
+                                        comm=SimComm(r, world, kp_all, ks, vs), ops=CudaOps(),
+                                        return_csr=True)
+        bops = CudaOps()
+        dq_acc, dkv = ring_backward_partials(qs[r], ks[r], vs[r], out, lse, gs[r], rp, ci, grid,
+                                             comm=SimComm(r, world, kp_all, ks, vs), ops=bops)
+        bops.check()
+        dq_full[:, :, r * T_l * HW:(r + 1) * T_l * HW] = bops.finalize(p_local, dq_acc)
+        parts.append(dkv)
+    dk_full, dv_full = torch.empty_like(kd), torch.empty_like(vd)
+    for j in range(world):
+        sl = slice(j * T_l * HW, (j + 1) * T_l * HW)
+        dk_full[:, :, sl] = ops.finalize(p_local, sum(pt[0, j] for pt in parts).contiguous())
+        dv_full[:, :, sl] = ops.finalize(p_local, sum(pt[1, j] for pt in parts).contiguous())
+    rows = np.arange(wl.rows)
+    scale = 1.0 / math.sqrt(wl.d)
+    o_dq, o_dk, o_dv = oracle.attend_bwd(q, k, v, g, wl.T, wl.H, wl.W, scale, g_rp, g_ci, rows)
+    errs = {"dq": rel_errors(gather_rows(host_f32(dq_full), wl, rows), o_dq),
+            "dk": rel_errors(host_f32(dk_full), o_dk),
+            "dv": rel_errors(host_f32(dv_full), o_dv)}
+    for nm, (mx, mean) in errs.items():
+        assert mx <= BWD_MAX_REL and mean <= BWD_MEAN_REL, (nm, errs)
+    # and against the unsplit GPU backward, within the same bars
+    ref = {"dq": gather_rows(host_f32(dq_g), wl, rows), "dk": host_f32(dk_g),
+           "dv": host_f32(dv_g)}
+    got = {"dq": gather_rows(host_f32(dq_full), wl, rows), "dk": host_f32(dk_full),
+           "dv": host_f32(dv_full)}
+    for nm in ref:
+        mx, mean = rel_errors(got[nm], ref[nm])
+        assert mx <= BWD_MAX_REL and mean <= BWD_MEAN_REL, (nm, mx, mean)
+
+
+def test_ring_backward_one_rank_is_the_backward():
+    """A group of one: ring_backward (forward CSR, one shard, reduce-scatter of
+    one) must give the unsplit backward up to the fp32 round trip, i.e. exactly."""
+    wl = synth.WORKLOADS["tiny"].with_(heads=2, T=8, H=13, W=37, d=128, topk=5)
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    qd, kd, vd, gd = dev(q), dev(k), dev(v), dev(g)
+    _, _, dq_g, dk_g, dv_g = _unsplit_backward(wl, qd, kd, vd, gd)
+    ops = CudaOps()
+    p = bsa.make_params(wl.B, wl.heads, wl.T, wl.H, wl.W, wl.d, wl.mode, wl.topk)
+    kp_all = torch.stack([ops.pool(p, kd)])
+    comm = SimComm(0, 1, kp_all, [kd], [vd])
+    out, lse, rp, ci = ring_forward(qd, kd, vd, (wl.T, wl.H, wl.W), wl.topk, comm=comm, ops=ops,
+                                    return_csr=True)
+    dq, dk, dv = ring_backward(qd, kd, vd, out, lse, gd, rp, ci, (wl.T, wl.H, wl.W),
+                               comm=SimComm(0, 1, kp_all, [kd], [vd]), ops=CudaOps())
+    # bf16 -> fp32 -> bf16 is the identity
+    for a, b in ((dq, dq_g), (dk, dk_g), (dv, dv_g)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_grad_accumulate_and_finalize_units():
+    """The fp32 accumulation of bf16 parts equals the fp32 sums taken in the same
+    order (bf16 widens exactly), and the final rounding is round-to-nearest-even
+    (torch's bf16 cast)."""
+    wl = synth.WORKLOADS["tiny"].with_(heads=2, T=4, H=4, W=8, d=64)
+    p = bsa.make_params(wl.B, wl.heads, wl.T, wl.H, wl.W, wl.d, "topk", 1)
+    shape = (wl.B, wl.heads, wl.N, wl.d)
+    gen = torch.Generator(device="cpu").manual_seed(5)
+    parts = [torch.randn(shape, generator=gen).to(torch.bfloat16).cuda() for _ in range(3)]
+    acc = torch.full(shape, float("nan"), dtype=torch.float32, device="cuda")
+    bsa.bsa_grad_accumulate(p, parts[0], acc, overwrite=True)
+    for x in parts[1:]:
+        bsa.bsa_grad_accumulate(p, x, acc, overwrite=False)
+    ref = parts[0].float() + parts[1].float() + parts[2].float()
+    assert torch.equal(acc, ref)
+    acc2 = torch.randn(shape, generator=gen).cuda() * 3
+    out = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    bsa.bsa_grad_finalize(p, acc2, out)
+    assert torch.equal(out.view(torch.int16), acc2.to(torch.bfloat16).view(torch.int16))
