@@ -386,7 +386,9 @@ __global__ void __launch_bounds__(320, 1)
             tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
             tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(s + 64));
             tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(s + 96));
-            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                tmem_wait_ld_tie(*reinterpret_cast<uint32_t(*)[32]>(s + 32 * c));
             float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
             float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
 #pragma unroll
@@ -432,7 +434,7 @@ __global__ void __launch_bounds__(320, 1)
                 for (int g = 0; g < D / 32; ++g) {
                     uint32_t o[32];
                     tmem_ld32(tO + g * 32, o);
-                    tmem_wait_ld();
+                    tmem_wait_ld_tie(o);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
                     tmem_st32(tO + g * 32, o);
@@ -467,7 +469,7 @@ __global__ void __launch_bounds__(320, 1)
                 for (int g = 0; g < D / 32; ++g) {
                     uint32_t o[32];
                     tmem_ld32(tO + g * 32, o);
-                    tmem_wait_ld();
+                    tmem_wait_ld_tie(o);
                     const int half = (g * 32) / 64;
                     const int chunk0 = ((g * 32) % 64) / 8;
 #pragma unroll

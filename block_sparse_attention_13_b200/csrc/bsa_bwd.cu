@@ -223,7 +223,7 @@ __device__ __forceinline__ void stage_tmem_rows(uint32_t t_row, uint8_t* stage, 
     for (int g = g_begin; g < g_end; ++g) {
         uint32_t o[32];
         tmem_ld32(t_row + g * 32, o);
-        tmem_wait_ld();
+        tmem_wait_ld_tie(o);
         const int half = (g * 32) / 64;
         const int chunk0 = ((g * 32) % 64) / 8;
 #pragma unroll
@@ -505,7 +505,8 @@ __global__ void __launch_bounds__(320, 1)
                 uint32_t sv[32], pv[32];
                 tmem_ld32(tS + g * 32, sv);
                 tmem_ld32(tP + g * 32, pv);
-                tmem_wait_ld();
+                tmem_wait_ld_tie(sv);
+                tmem_wait_ld_tie(pv);
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -795,7 +796,8 @@ __global__ void __launch_bounds__(320, 1)
                     uint32_t sv[32], pv[32];
                     tmem_ld32(tS, sv);
                     tmem_ld32(tP, pv);
-                    tmem_wait_ld();
+                    tmem_wait_ld_tie(sv);
+                    tmem_wait_ld_tie(pv);
                     uint32_t pk[16], dk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
