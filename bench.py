@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--e2e-group", type=int, default=4,
+    ap.add_argument("--e2e-group", type=int, default=2,
                     help="(batch, head) pairs per group of the host-buffer pipeline")
     ap.add_argument("--e2e-streams", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=15.0,

@@ -29,7 +29,7 @@ class HostForward:
     group: (batch, head) pairs per group; streams: groups in flight.
     """
 
-    def __init__(self, p: bsa_params, group: int = 4, streams: int = 3, device="cuda"):
+    def __init__(self, p: bsa_params, group: int = 2, streams: int = 3, device="cuda"):
         self.p = p
         self.BH = p.B * p.heads
         self.group = max(1, min(group, self.BH))
