@@ -166,9 +166,10 @@ __global__ void __launch_bounds__(256) rearrange_kernel(const __nv_bfloat16* __r
 }
 
 // ------------------------------------------------------------------------
-// Pooled scores S[bh][i][m] = <qp[i], kp[m]> * scale in fp32 FMA. 64x64 output
-// tile per CTA, 4x4 register micro-tile per thread, operands staged
-// transposed in shared memory 32 channels at a time.
+// Pooled scores S[bh][i][m] = <qp[i], kp[m]> * scale in fp32 FMA. 128x128
+// output tile per CTA, 8x8 register micro-tile per thread (64 FMAs per 16
+// values read from shared memory), operands staged transposed in shared
+// memory 16 channels at a time.
 // kp holds the key chunks in shards of `kshard` chunks, [shard][BH][kshard][D]
 // (kshard = Nk: one shard, the plain [BH][Nk][D] layout); the gathered pooled
 // keys of a context-parallel group arrive that way.
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ q
                                                      const float* __restrict__ kp,
                                                      float* __restrict__ S, int Nq, int Nk,
                                                      int kshard, int D, float scale) {
-    constexpr int BT = 64, BK = 32, LD = BT + 4;
+    constexpr int BT = 128, BK = 16, LD = BT + 4;
     __shared__ __align__(16) float As[BK][LD];
     __shared__ __align__(16) float Bs[BK][LD];
     const int64_t bh = blockIdx.z;
@@ -184,16 +185,16 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ q
     const float* A = qp + bh * (int64_t)Nq * D;
     const int64_t BH = gridDim.z;
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
-    float acc[4][4];
+    float acc[8][8];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+        for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
 
     for (int k0 = 0; k0 < D; k0 += BK) {
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-            const int idx = tid + 256 * j;  // 512 float4 per 64x32 tile
+            const int idx = tid + 256 * j;  // 512 float4 per 128x16 tile
             const int r = idx / (BK / 4), kq = idx % (BK / 4);
             float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
             if (i0 + r < Nq) va = *reinterpret_cast<const float4*>(A + (int64_t)(i0 + r) * D + k0 + kq * 4);
@@ -207,32 +208,39 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ q
             Bs[kq * 4 + 2][r] = vb.z; Bs[kq * 4 + 3][r] = vb.w;
         }
         __syncthreads();
-#pragma unroll 8
+#pragma unroll
         for (int kk = 0; kk < BK; ++kk) {
-            const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-            const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
-            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+            const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 8]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][ty * 8 + 4]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8 + 4]);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int p = 0; p < 4; ++p)
+            for (int p = 0; p < 8; ++p)
 #pragma unroll
-                for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
+                for (int q = 0; q < 8; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
         }
         __syncthreads();
     }
     float* out = S + bh * (int64_t)Nq * Nk;
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const int i = i0 + ty * 4 + p;
+    for (int p = 0; p < 8; ++p) {
+        const int i = i0 + ty * 8 + p;
         if (i >= Nq) continue;
-        const int m = m0 + tx * 4;
-        float* o = out + (int64_t)i * Nk + m;
-        if ((Nk & 3) == 0 && m + 3 < Nk) {
-            *reinterpret_cast<float4*>(o) = make_float4(acc[p][0] * scale, acc[p][1] * scale,
-                                                        acc[p][2] * scale, acc[p][3] * scale);
-        } else {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (m + q < Nk) o[q] = acc[p][q] * scale;
+        for (int h = 0; h < 2; ++h) {
+            const int m = m0 + tx * 8 + h * 4;
+            float* o = out + (int64_t)i * Nk + m;
+            if ((Nk & 3) == 0 && m + 3 < Nk) {
+                *reinterpret_cast<float4*>(o) =
+                    make_float4(acc[p][h * 4 + 0] * scale, acc[p][h * 4 + 1] * scale,
+                                acc[p][h * 4 + 2] * scale, acc[p][h * 4 + 3] * scale);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (m + q < Nk) o[q] = acc[p][h * 4 + q] * scale;
+            }
         }
     }
 }
@@ -601,7 +609,7 @@ cudaError_t launch_rearrange(const Dims& g, const void* src, void* dst, int inve
 
 cudaError_t launch_scores(const Dims& g, const float* qp, const float* kp, float* S,
                           cudaStream_t st, int kshard) {
-    dim3 grid((g.Nk + 63) / 64, (g.Nq + 63) / 64, (unsigned)g.BH);
+    dim3 grid((g.Nk + 127) / 128, (g.Nq + 127) / 128, (unsigned)g.BH);
     scores_kernel<<<grid, 256, 0, st>>>(qp, kp, S, g.Nq, g.Nk, kshard > 0 ? kshard : g.Nk, g.d,
                                         g.scale);
     return cudaGetLastError();
