@@ -338,8 +338,8 @@ def block_sparse_attention(q, k, v, topk=None, mode="topk", cdf_p=0.9, cdf_cap_f
     B, heads, N, d = q.shape
     T, H, W = grid
     assert T * H * W == N
-    if topk is None:
-        topk = max(1, ((T // 4) * (H // 4) * (W // 8)) // 16)
+    if topk is None:  # 1/16 of the key chunks (ceil counts: edge chunks may be partial)
+        topk = max(1, (-(-T // 4) * -(-H // 4) * -(-W // 8)) // 16)
     p = make_params(B, heads, T, H, W, d, mode, topk, cdf_p, cdf_cap_frac, t_cond)
     pl = plan(p, q, k)
     lse = torch.empty((B, heads, N), dtype=torch.float32, device=q.device) if want_lse else None
