@@ -52,8 +52,10 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--backward", action="store_true",
-                    help="also time bsa_backward (dQ, dK, dV) on the same plan")
-    ap.add_argument("--bwd-steps", type=int, default=20)
+                    help="time bsa_backward (dQ, dK, dV) on the same plan (the default)")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward timing")
+    ap.add_argument("--bwd-steps", type=int, default=10)
     return ap.parse_args()
 
 
@@ -446,7 +448,7 @@ def main():
                 "algorithmic_flops_per_launch": flops}
 
     bwd = None
-    if args.backward:
+    if not args.no_backward:
         bwd = time_backward(args, wl, p, pl, q, k, v, stream, peak_tf)
 
     cpu = None
