@@ -169,51 +169,81 @@ __global__ void __launch_bounds__(256) rearrange_kernel(const __nv_bfloat16* __r
 // Pooled scores S[bh][i][m] = <qp[i], kp[m]> * scale in fp32 FMA. 128x128
 // output tile per CTA, 8x8 register micro-tile per thread (64 FMAs per 16
 // values read from shared memory), operands staged transposed in shared
-// memory 16 channels at a time.
+// memory 16 channels at a time, two stages deep.
 // kp holds the key chunks in shards of `kshard` chunks, [shard][BH][kshard][D]
 // (kshard = Nk: one shard, the plain [BH][Nk][D] layout); the gathered pooled
 // keys of a context-parallel group arrive that way.
-__global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ qp,
+__global__ void __launch_bounds__(256, 2) scores_kernel(const float* __restrict__ qp,
                                                      const float* __restrict__ kp,
                                                      float* __restrict__ S, int Nq, int Nk,
                                                      int kshard, int D, float scale) {
     constexpr int BT = 128, BK = 16, LD = BT + 4;
-    __shared__ __align__(16) float As[BK][LD];
-    __shared__ __align__(16) float Bs[BK][LD];
+    // two stages: the next 16 channels are fetched into registers while the
+    // current ones are multiplied, then stored into the other stage
+    __shared__ __align__(16) float As[2][BK][LD];
+    __shared__ __align__(16) float Bs[2][BK][LD];
     const int64_t bh = blockIdx.z;
     const int i0 = blockIdx.y * BT, m0 = blockIdx.x * BT;
     const float* A = qp + bh * (int64_t)Nq * D;
     const int64_t BH = gridDim.z;
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+    // the two rows (of A and of B) this thread stages, and their channel quad
+    const float* arow[2];
+    const float* brow[2];
+    int rr[2], kq[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int idx = tid + 256 * j;  // 512 float4 per 128x16 tile
+        rr[j] = idx / (BK / 4);
+        kq[j] = idx % (BK / 4);
+        arow[j] = i0 + rr[j] < Nq ? A + (int64_t)(i0 + rr[j]) * D : nullptr;
+        const int m = m0 + rr[j];
+        if (m < Nk) {
+            const int sh = m / kshard, ml = m - sh * kshard;
+            brow[j] = kp + ((sh * BH + bh) * kshard + ml) * D;
+        } else {
+            brow[j] = nullptr;
+        }
+    }
+    float4 ra[2], rb[2];
+    auto fetch = [&](int k0) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            ra[j] = arow[j] ? *reinterpret_cast<const float4*>(arow[j] + k0 + kq[j] * 4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            rb[j] = brow[j] ? *reinterpret_cast<const float4*>(brow[j] + k0 + kq[j] * 4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    auto stage = [&](int st) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int r = rr[j], c = kq[j] * 4;
+            As[st][c + 0][r] = ra[j].x; As[st][c + 1][r] = ra[j].y;
+            As[st][c + 2][r] = ra[j].z; As[st][c + 3][r] = ra[j].w;
+            Bs[st][c + 0][r] = rb[j].x; Bs[st][c + 1][r] = rb[j].y;
+            Bs[st][c + 2][r] = rb[j].z; Bs[st][c + 3][r] = rb[j].w;
+        }
+    };
     float acc[8][8];
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
         for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
 
-    for (int k0 = 0; k0 < D; k0 += BK) {
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int idx = tid + 256 * j;  // 512 float4 per 128x16 tile
-            const int r = idx / (BK / 4), kq = idx % (BK / 4);
-            float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
-            if (i0 + r < Nq) va = *reinterpret_cast<const float4*>(A + (int64_t)(i0 + r) * D + k0 + kq * 4);
-            if (m0 + r < Nk) {
-                const int m = m0 + r, sh = m / kshard, ml = m - sh * kshard;
-                vb = *reinterpret_cast<const float4*>(kp + ((sh * BH + bh) * kshard + ml) * D + k0 + kq * 4);
-            }
-            As[kq * 4 + 0][r] = va.x; As[kq * 4 + 1][r] = va.y;
-            As[kq * 4 + 2][r] = va.z; As[kq * 4 + 3][r] = va.w;
-            Bs[kq * 4 + 0][r] = vb.x; Bs[kq * 4 + 1][r] = vb.y;
-            Bs[kq * 4 + 2][r] = vb.z; Bs[kq * 4 + 3][r] = vb.w;
-        }
-        __syncthreads();
+    fetch(0);
+    stage(0);
+    __syncthreads();
+    const int nk = D / BK;
+    for (int c = 0; c < nk; ++c) {
+        const int st = c & 1;
+        if (c + 1 < nk) fetch((c + 1) * BK);
 #pragma unroll
         for (int kk = 0; kk < BK; ++kk) {
-            const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 8]);
-            const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][ty * 8 + 4]);
-            const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8]);
-            const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8 + 4]);
+            const float4 a0 = *reinterpret_cast<const float4*>(&As[st][kk][ty * 8]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&As[st][kk][ty * 8 + 4]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&Bs[st][kk][tx * 8]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&Bs[st][kk][tx * 8 + 4]);
             const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -221,6 +251,7 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ q
 #pragma unroll
                 for (int q = 0; q < 8; ++q) acc[p][q] = fmaf(av[p], bv[q], acc[p][q]);
         }
+        if (c + 1 < nk) stage(st ^ 1);  // the other stage was last read before the previous sync
         __syncthreads();
     }
     float* out = S + bh * (int64_t)Nq * Nk;
