@@ -656,9 +656,16 @@ cudaError_t launch_select(const Dims& g, const bsa_params& p, const float* S, in
                                               g.Nq, g.rows, mode, p.topk, p.cdf_p,           \
                                               p.cdf_cap_frac, row_ptr, col_idx, col_cap,     \
                                               counts, padded, pad_stride, status)
+    // keys per lane: the smallest instantiation that holds the row (the searches
+    // cost one compare per key slot and step, so padding slots are not free)
     if (g.Nk <= 32) BSA_SELECT(1);
     else if (g.Nk <= 256) BSA_SELECT(8);
+    else if (g.Nk <= 512) BSA_SELECT(16);
+    else if (g.Nk <= 768) BSA_SELECT(24);
     else if (g.Nk <= 1024) BSA_SELECT(32);
+    else if (g.Nk <= 1280) BSA_SELECT(40);
+    else if (g.Nk <= 1536) BSA_SELECT(48);
+    else if (g.Nk <= 1792) BSA_SELECT(56);
     else if (g.Nk <= 2048) BSA_SELECT(64);
     else return cudaErrorInvalidValue;
 #undef BSA_SELECT
