@@ -290,6 +290,16 @@ def test_context_parallel_entries_host_checks(L):
     assert g(ctypes.byref(pr), x, x, 3, x, wsz, x, x, 64, None) == bsa.BSA_ERR_INVALID_ARG
     assert g(ctypes.byref(pr), x, x, 2, x, wsz - 1, x, x, 64, None) == \
         bsa.BSA_ERR_WORKSPACE_TOO_SMALL
+    # gradient accumulation of the ring backward: arguments, overwrite flag, alignment
+    a = L.bsa_grad_accumulate
+    assert a(ctypes.byref(p), None, x, 1, None) == bsa.BSA_ERR_INVALID_ARG
+    assert a(ctypes.byref(p), x, None, 0, None) == bsa.BSA_ERR_INVALID_ARG
+    assert a(ctypes.byref(p), x, x, 2, None) == bsa.BSA_ERR_INVALID_ARG
+    assert a(ctypes.byref(p), vp(FAKE + 4), x, 1, None) == bsa.BSA_ERR_ALIGNMENT
+    assert a(ctypes.byref(P(T=0)), x, x, 1, None) == bsa.BSA_ERR_SHAPE
+    fz = L.bsa_grad_finalize
+    assert fz(ctypes.byref(p), None, x, None) == bsa.BSA_ERR_INVALID_ARG
+    assert fz(ctypes.byref(p), x, vp(FAKE + 8), None) == bsa.BSA_ERR_ALIGNMENT
 
 
 @pytest.mark.parametrize("kw,code", [(dict(q_begin=4, q_end=4), bsa.BSA_ERR_SHAPE),
