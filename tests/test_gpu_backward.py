@@ -162,6 +162,24 @@ def test_backward_kv_cached_rows():
     assert torch.all(dq[:, :, : wl.q_begin * HW] == 7.0)
 
 
+def test_autograd_op_matches_the_c_abi_calls():
+    """block_sparse_attention_train (torch.autograd) runs the same plan, forward and
+    backward as the direct C-ABI calls: outputs and gradients bit for bit."""
+    from block_sparse_attention_13_b200.autograd import block_sparse_attention_train
+    wl = SMALL["ragged135_d128"]
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    rp, ci, out, lse, dq, dk, dv, st_f, st_b = gpu_fwd_bwd(wl, q, k, v, g)
+    assert st_f == bsa.BSA_OK and st_b == bsa.BSA_OK
+    qt, kt, vt = (dev(x).requires_grad_(True) for x in (q, k, v))
+    o = block_sparse_attention_train(qt, kt, vt, (wl.T, wl.H, wl.W), topk=wl.topk, mode=wl.mode,
+                                     cdf_p=wl.cdf_p, cdf_cap_frac=wl.cdf_cap_frac,
+                                     t_cond=wl.t_cond)
+    o.backward(dev(g))
+    for a, b in ((o.detach(), out), (qt.grad, dq), (kt.grad, dk), (vt.grad, dv)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 def test_backward_deterministic():
     wl = SMALL["ragged135_d128"]
     q, k, v = synth.make_qkv(wl)
