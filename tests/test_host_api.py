@@ -80,3 +80,19 @@ def test_ring_backward_visits_every_shard_once_in_ring_order():
     # dQ: overwrite on the first step only; dK and dV: each shard's slot written once
     assert acc == [True, True, True] + [False, True, True] * (world - 1)
     assert parts.shape == (2, world) + tuple(q.shape)
+
+
+def test_product_modules_never_import_the_oracle():
+    """The library's Python modules (binding, host pipeline, autograd op, ring driver)
+    must not load the CPU oracle: it is test infrastructure, and a product path that
+    reached it would be a CPU fallback."""
+    import subprocess
+    import sys
+    code = ("import sys\n"
+            "import block_sparse_attention_13_b200, block_sparse_attention_13_b200.host\n"
+            "import block_sparse_attention_13_b200.autograd\n"
+            "import block_sparse_attention_13_b200.context_parallel\n"
+            "assert 'oracle' not in sys.modules, sorted(m for m in sys.modules if 'oracle' in m)\n")
+    root = __file__.rsplit("/tests/", 1)[0]
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
