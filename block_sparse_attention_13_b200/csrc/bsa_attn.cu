@@ -524,18 +524,18 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver entry point is looked up once per process (a function-local static
+// is initialised exactly once, also under concurrent first calls).
 static EncodeTiledFn get_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    static const EncodeTiledFn fn = [] {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q{};
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+            return reinterpret_cast<EncodeTiledFn>(p);
+        return static_cast<EncodeTiledFn>(nullptr);
+    }();
     return fn;
 }
 
@@ -562,14 +562,9 @@ cudaError_t launch_fwd_dp(const Dims& g, const CUtensorMap& mq, const CUtensorMa
                           const CUtensorMap& mv, const CUtensorMap& mo, const FwdArgs& args,
                           cudaStream_t st) {
     using C = AttnCfg<D>;
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<D, kPartial>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
+    static std::atomic<uint64_t> attr_done{0};
+    const cudaError_t e = raise_smem_limit(bsa_fwd_kernel<D, kPartial>, C::kSmemBytes, attr_done);
+    if (e != cudaSuccess) return e;
     const unsigned grid = static_cast<unsigned>((g.rows + 1) / 2);
     bsa_fwd_kernel<D, kPartial><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mo, args);
     return cudaGetLastError();

@@ -859,21 +859,15 @@ __global__ void __launch_bounds__(320, 1)
     }
 }
 
-template <typename K>
-cudaError_t set_smem(K kernel, int bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-}
-
 template <int D>
 cudaError_t launch_bwd_d(const Dims& g, const CUtensorMap* m, const BwdArgs& dq_args,
                          const BwdArgs& dkv_args, cudaStream_t st) {
     using C = BwdCfg<D>;
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = set_smem(bsa_bwd_dq_kernel<D>, C::kSmemBytes);
-        if (e == cudaSuccess) e = set_smem(bsa_bwd_dkv_kernel<D>, C::kSmemBytes);
+    static std::atomic<uint64_t> dq_attr{0}, dkv_attr{0};
+    {
+        cudaError_t e = raise_smem_limit(bsa_bwd_dq_kernel<D>, C::kSmemBytes, dq_attr);
+        if (e == cudaSuccess) e = raise_smem_limit(bsa_bwd_dkv_kernel<D>, C::kSmemBytes, dkv_attr);
         if (e != cudaSuccess) return e;
-        attr_done = true;
     }
     // m: q, k, v, dout, dq, dk, dv (whole chunks), then q and dout (half chunks)
     bsa_bwd_dq_kernel<D><<<static_cast<unsigned>(dq_args.units), C::kThreads, C::kSmemBytes, st>>>(

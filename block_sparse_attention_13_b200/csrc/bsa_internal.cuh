@@ -2,11 +2,28 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 #include "../../include/bsa.h"
 
 namespace bsa {
+
+// Raises a kernel's dynamic shared-memory limit on the current device. The
+// attribute belongs to that device's context, so `done` keeps one bit per device
+// (a device numbered 64 or above sets it on every call). Two threads that race on
+// the first launch both set it, which is harmless.
+template <typename Kernel>
+inline cudaError_t raise_smem_limit(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t{1} << dev) : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
 
 constexpr int kChunkT = 4, kChunkH = 4, kChunkW = 8;
 constexpr int kChunkTokens = kChunkT * kChunkH * kChunkW;  // 128

@@ -23,7 +23,9 @@
  *   - CSR rows are ordered (batch, head, query chunk); row r's key chunks are
  *     col_idx[row_ptr[r] .. row_ptr[r+1]), ascending. int32, DEVICE memory.
  *   - The caller allocates and owns every buffer. The library never allocates
- *     device memory and holds no global state beyond cached driver entry points.
+ *     device memory. Its only process-wide state is the cached tensor-map entry
+ *     point and, per device, whether each kernel's shared-memory limit has been
+ *     raised; both are safe to reach from several host threads at once.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Launches are
  *     asynchronous; errors found on the device are read with bsa_read_status.
  *   - Return value: BSA_OK (0) or a bsa_status code. No exception crosses the ABI.
