@@ -156,6 +156,8 @@ static int64_t max_key_nnz_of(const Dims& g, const bsa_params& p) {
 static int64_t max_nnz_of(const Dims& g, const bsa_params& p) { return max_key_nnz_of(g, p) * g.m; }
 
 static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+// int32 CSR arrays and fp32 vectors are read element by element: 4-byte alignment
+static bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
 
 static int cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
 
@@ -256,7 +258,8 @@ int bsa_forward_ex(const bsa_params* p, const void* q, const void* k, const void
     if (!q || !k || !v || !row_ptr || !col_idx || !workspace || !out || col_capacity < 0)
         return BSA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-        !aligned16(workspace) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        !aligned16(workspace) || (lse && !aligned4(lse)) || !aligned4(row_ptr) ||
+        !aligned4(col_idx))
         return BSA_ERR_ALIGNMENT;
     if (ws_bytes < 256) return BSA_ERR_WORKSPACE_TOO_SMALL;
     if ((rc = device_ok()) != BSA_OK) return rc;
@@ -291,7 +294,7 @@ int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* 
         return BSA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) ||
-        (reinterpret_cast<uintptr_t>(lse) & 3u))
+        !aligned4(lse) || !aligned4(row_ptr) || !aligned4(col_idx))
         return BSA_ERR_ALIGNMENT;
     if (ws_bytes < bwd_layout(g).total) return BSA_ERR_WORKSPACE_TOO_SMALL;
     if ((rc = device_ok()) != BSA_OK) return rc;
@@ -345,7 +348,9 @@ int bsa_csr_slice(int64_t n_rows, const int32_t* row_ptr, const int32_t* col_idx
     if (n_rows < 0 || !row_ptr || !col_idx || !workspace || !out_row_ptr || !out_col_idx ||
         col_capacity < 0 || out_capacity < 0 || lo < 0 || hi < lo)
         return BSA_ERR_INVALID_ARG;
-    if (!aligned16(workspace)) return BSA_ERR_ALIGNMENT;
+    if (!aligned16(workspace) || !aligned4(row_ptr) || !aligned4(col_idx) ||
+        !aligned4(out_row_ptr) || !aligned4(out_col_idx))
+        return BSA_ERR_ALIGNMENT;
     if (ws_bytes < bsa_csr_slice_workspace_size(n_rows)) return BSA_ERR_WORKSPACE_TOO_SMALL;
     int rc = device_ok();
     if (rc != BSA_OK) return rc;
@@ -364,8 +369,7 @@ int bsa_lse_merge(const bsa_params* p, void* out, float* lse, const void* out_pa
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
     if (!out || !lse || !out_part || !lse_part) return BSA_ERR_INVALID_ARG;
-    if (!aligned16(out) || !aligned16(out_part) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
-        (reinterpret_cast<uintptr_t>(lse_part) & 3u))
+    if (!aligned16(out) || !aligned16(out_part) || !aligned4(lse) || !aligned4(lse_part))
         return BSA_ERR_ALIGNMENT;
     if ((rc = device_ok()) != BSA_OK) return rc;
     return cuda_status(launch_lse_merge(g, out, lse, out_part, lse_part,
@@ -442,6 +446,7 @@ int bsa_scores(const bsa_params* p, const float* qp, const float* kp, float* S, 
 
 int bsa_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n, void* stream) {
     if (!x || !y_poly || !y_mufu || n < 0 || (n & 1)) return BSA_ERR_INVALID_ARG;
+    if (!aligned4(x) || !aligned4(y_poly) || !aligned4(y_mufu)) return BSA_ERR_ALIGNMENT;
     const int rc = device_ok();
     if (rc != BSA_OK) return rc;
     return cuda_status(launch_exp2_selftest(x, y_poly, y_mufu, n, static_cast<cudaStream_t>(stream)));

@@ -21,7 +21,9 @@
  *     l = (lt*4 + lh)*8 + lw is token (4ct+lt, 4ch+lh, 8cw+lw) when that lies
  *     inside the grid (a partial edge chunk has fewer than 128 tokens).
  *   - CSR rows are ordered (batch, head, query chunk); row r's key chunks are
- *     col_idx[row_ptr[r] .. row_ptr[r+1]), ascending. int32, DEVICE memory.
+ *     col_idx[row_ptr[r] .. row_ptr[r+1]), ascending. int32, DEVICE memory,
+ *     4-byte aligned (16 where bsa_plan or bsa_select_pooled writes them); an
+ *     fp32 lse array is 4-byte aligned.
  *   - The caller allocates and owns every buffer. The library never allocates
  *     device memory. Its only process-wide state is the cached tensor-map entry
  *     point and, per device, whether each kernel's shared-memory limit has been
@@ -51,7 +53,8 @@ typedef enum {
     BSA_ERR_INVALID_ARG = 1,         /* null pointer, bad enum, k < 1, p outside (0,1] ...   */
     BSA_ERR_SHAPE = 2,               /* sizes <= 0, t_cond or q_begin not a multiple of 4 ... */
     BSA_ERR_UNSUPPORTED = 3,         /* d not in {64,128}, chunk shape != (4,4,8), no sm_100  */
-    BSA_ERR_ALIGNMENT = 4,           /* a tensor pointer is not 16-byte aligned               */
+    BSA_ERR_ALIGNMENT = 4,           /* a bf16 tensor or workspace pointer is not 16-byte
+                                        aligned, or an int32 / fp32 array not 4-byte aligned */
     BSA_ERR_WORKSPACE_TOO_SMALL = 5, /* ws_bytes < bsa_workspace_size()                       */
     BSA_ERR_CUDA = 6,                /* a CUDA runtime/driver call or launch failed           */
     BSA_ERR_DEVICE_BAD_INDEX = 7,    /* device saw an out-of-range CSR row or column index    */
@@ -334,7 +337,8 @@ BSA_API int bsa_scores(const bsa_params* p, const float* qp, const float* kp, fl
 /* Device self-test of the softmax exponentials: for n (even) floats x, writes
  * the FMA-pipe polynomial 2^x that the forward kernel uses for part of the
  * softmax numerators into y_poly, and the MUFU ex2.approx value into y_mufu.
- * Device pointers. Used to check the polynomial against exact 2^x. */
+ * Device pointers, 4-byte aligned. Used to check the polynomial against exact
+ * 2^x. Errors: INVALID_ARG (n odd or negative), ALIGNMENT, UNSUPPORTED, CUDA. */
 BSA_API int bsa_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n,
                               void* stream);
 

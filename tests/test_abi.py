@@ -216,6 +216,11 @@ def test_forward_host_checks_before_any_cuda_call(L):
     assert f(pp, *a, 16, vp(FAKE), 255, vp(FAKE), None, None) == \
         bsa.BSA_ERR_WORKSPACE_TOO_SMALL
     assert f(pp, *a, -1, vp(FAKE), 256, vp(FAKE), None, None) == bsa.BSA_ERR_INVALID_ARG
+    # int32 CSR arrays and the fp32 lse are read element by element: 4-byte alignment
+    x, odd = vp(FAKE), vp(FAKE + 2)
+    assert f(pp, x, x, x, odd, x, 16, x, 256, x, None, None) == bsa.BSA_ERR_ALIGNMENT
+    assert f(pp, x, x, x, x, odd, 16, x, 256, x, None, None) == bsa.BSA_ERR_ALIGNMENT
+    assert f(pp, x, x, x, x, x, 16, x, 256, x, odd, None) == bsa.BSA_ERR_ALIGNMENT
 
 
 def test_backward_workspace_size_layout(L):
@@ -243,6 +248,9 @@ def test_backward_host_checks_before_any_cuda_call(L):
         bsa.BSA_ERR_ALIGNMENT
     assert f(pp, x, x, x, x, x, x, x, x, 16, x, ws - 1, x, x, x, None) == \
         bsa.BSA_ERR_WORKSPACE_TOO_SMALL
+    odd = vp(FAKE + 2)
+    assert f(pp, x, x, x, x, x, x, odd, x, 16, x, ws, x, x, x, None) == bsa.BSA_ERR_ALIGNMENT
+    assert f(pp, x, x, x, x, x, x, x, odd, 16, x, ws, x, x, x, None) == bsa.BSA_ERR_ALIGNMENT
     assert f(ctypes.byref(P(T=0)), x, x, x, x, x, x, x, x, 16, x, ws, x, x, x, None) == \
         bsa.BSA_ERR_SHAPE
 
@@ -278,6 +286,12 @@ def test_context_parallel_entries_host_checks(L):
     assert f(10, x, x, 16, -1, 2, x, ws, x, x, 16, None) == bsa.BSA_ERR_INVALID_ARG
     assert f(10, x, x, 16, 0, 2, vp(FAKE + 8), ws, x, x, 16, None) == bsa.BSA_ERR_ALIGNMENT
     assert f(10, x, x, 16, 0, 2, x, ws - 1, x, x, 16, None) == bsa.BSA_ERR_WORKSPACE_TOO_SMALL
+    odd = vp(FAKE + 2)
+    for i in range(4):   # row_ptr, col_idx, out_row_ptr, out_col_idx
+        arrs = [x, x, x, x]
+        arrs[i] = odd
+        assert f(10, arrs[0], arrs[1], 16, 0, 2, x, ws, arrs[2], arrs[3], 16, None) == \
+            bsa.BSA_ERR_ALIGNMENT
     # lse merge
     p = P()
     assert L.bsa_lse_merge(ctypes.byref(p), x, None, x, x, None) == bsa.BSA_ERR_INVALID_ARG
@@ -300,6 +314,16 @@ def test_context_parallel_entries_host_checks(L):
     fz = L.bsa_grad_finalize
     assert fz(ctypes.byref(p), None, x, None) == bsa.BSA_ERR_INVALID_ARG
     assert fz(ctypes.byref(p), x, vp(FAKE + 8), None) == bsa.BSA_ERR_ALIGNMENT
+
+
+def test_exp2_selftest_host_checks(L):
+    x = vp(FAKE)
+    e = L.bsa_selftest_exp2
+    assert e(x, x, x, 3, None) == bsa.BSA_ERR_INVALID_ARG          # n must be even
+    assert e(x, x, x, -2, None) == bsa.BSA_ERR_INVALID_ARG
+    assert e(None, x, x, 2, None) == bsa.BSA_ERR_INVALID_ARG
+    assert e(vp(FAKE + 2), x, x, 2, None) == bsa.BSA_ERR_ALIGNMENT
+    assert e(x, x, vp(FAKE + 1), 2, None) == bsa.BSA_ERR_ALIGNMENT
 
 
 @pytest.mark.parametrize("kw,code", [(dict(q_begin=4, q_end=4), bsa.BSA_ERR_SHAPE),
