@@ -40,7 +40,11 @@ EXPORTED = ("bsa_version", "bsa_status_string", "bsa_workspace_size", "bsa_plan_
             "bsa_rearrange", "bsa_pool", "bsa_scores", "bsa_selftest_exp2",
             "bsa_selftest_timeout", "bsa_backward_workspace_size", "bsa_backward",
             "bsa_select_pooled", "bsa_csr_slice_workspace_size", "bsa_csr_slice",
-            "bsa_lse_merge", "bsa_grad_accumulate", "bsa_grad_finalize")
+            "bsa_lse_merge", "bsa_grad_accumulate", "bsa_grad_finalize", "bsa_shape_info")
+
+# Scratch array of bsa_plan_noalloc inside the library (include/bsa.h: 32 MiB);
+# a plan whose workspace exceeds it is rejected by the library before any CUDA call.
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class BsaError(RuntimeError):
@@ -59,6 +63,13 @@ class bsa_params(ctypes.Structure):
                 ("q_begin", ctypes.c_int32), ("kchunk_t", ctypes.c_int32),
                 ("kchunk_h", ctypes.c_int32), ("kchunk_w", ctypes.c_int32),
                 ("q_end", ctypes.c_int32)]
+
+
+class bsa_shape(ctypes.Structure):
+    """Element counts of the tensors of a call (include/bsa.h, bsa_shape_info)."""
+    _fields_ = [("BH", ctypes.c_int64), ("N", ctypes.c_int64), ("rows", ctypes.c_int64),
+                ("d", ctypes.c_int32), ("Nc", ctypes.c_int32), ("Nq", ctypes.c_int32),
+                ("Nk", ctypes.c_int32)]
 
 
 def make_params(B, heads, T, H, W, d, mode="topk", topk=1, cdf_p=0.9, cdf_cap_frac=0.25,
@@ -97,6 +108,7 @@ def lib():
             "bsa_status_string": (ctypes.c_char_p, [i32]),
             "bsa_workspace_size": (sz, [P]),
             "bsa_plan_sizes": (i32, [P, ctypes.POINTER(i64), ctypes.POINTER(i64)]),
+            "bsa_shape_info": (i32, [P, ctypes.POINTER(bsa_shape)]),
             "bsa_plan": (i32, [P, vp, vp, vp, sz, vp, vp, i64, vp]),
             "bsa_plan_noalloc": (i32, [P, vp, vp, vp, vp, i64, vp]),
             "bsa_forward": (i32, [P, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, vp]),
@@ -138,6 +150,46 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _tensors(what, *specs):
+    """Checks the tensors of one call before their pointers are passed on.
+
+    Each spec is (name, tensor or None, dtype or None, minimum size). A tensor
+    the library reads or writes must have that dtype, be contiguous, hold at
+    least that many elements (bytes when dtype is None: a workspace) and live on
+    the current CUDA device: anything else would reach the kernels as a bad
+    address. Raises BsaError: INVALID_ARG for the kind of tensor, SHAPE for its
+    size; the device is checked after every tensor's kind and size. None entries
+    (optional outputs) are skipped.
+    """
+    import torch
+    given = [(name, t, dtype, need) for name, t, dtype, need in specs if t is not None]
+    for name, t, dtype, need in given:
+        if not isinstance(t, torch.Tensor):
+            raise BsaError(BSA_ERR_INVALID_ARG, f"{what}: {name} is not a torch.Tensor")
+        if dtype is not None and t.dtype != dtype:
+            raise BsaError(BSA_ERR_INVALID_ARG, f"{what}: {name} is {t.dtype}, expected {dtype}")
+        if not t.is_contiguous():
+            raise BsaError(BSA_ERR_INVALID_ARG, f"{what}: {name} is not contiguous")
+        have = t.numel() if dtype is not None else t.numel() * t.element_size()
+        if have < need:
+            unit = "elements" if dtype is not None else "bytes"
+            raise BsaError(BSA_ERR_SHAPE, f"{what}: {name} holds {have} {unit}, needs {need}")
+    cur = None
+    for name, t, _, _ in given:
+        if not t.is_cuda:
+            raise BsaError(BSA_ERR_INVALID_ARG, f"{what}: {name} is not a CUDA tensor")
+        if cur is None:
+            cur = torch.cuda.current_device()
+        if t.device.index != cur:
+            raise BsaError(BSA_ERR_INVALID_ARG,
+                           f"{what}: {name} is on {t.device}, the current device is cuda:{cur}")
+
+
+def _dtypes():
+    import torch
+    return torch.bfloat16, torch.float32, torch.int32
+
+
 def _stream(stream):
     if stream is None:
         import torch
@@ -167,7 +219,18 @@ def bsa_plan_sizes(p: bsa_params):
     return rows.value, nnz.value
 
 
+def bsa_shape_info(p: bsa_params) -> bsa_shape:
+    s = bsa_shape()
+    _check(lib().bsa_shape_info(ctypes.byref(p), ctypes.byref(s)), "bsa_shape_info")
+    return s
+
+
 def bsa_plan(p, q, k, workspace, row_ptr, col_idx, stream=None):
+    bf, _, i32 = _dtypes()
+    s = bsa_shape_info(p)
+    x = s.BH * s.N * s.d
+    _tensors("bsa_plan", ("q", q, bf, x), ("k", k, bf, x), ("workspace", workspace, None, 0),
+             ("row_ptr", row_ptr, i32, s.rows + 1), ("col_idx", col_idx, i32, 0))
     _check(lib().bsa_plan(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _ptr(row_ptr),
                           _ptr(col_idx), col_idx.numel(), _stream(stream)), "bsa_plan")
@@ -176,12 +239,30 @@ def bsa_plan(p, q, k, workspace, row_ptr, col_idx, stream=None):
 def bsa_plan_noalloc(p, q, k, row_ptr, col_idx, stream=None):
     """bsa_plan with the library's fixed scratch array instead of a workspace,
     for callers that cannot allocate device memory (see include/bsa.h)."""
+    bf, _, i32 = _dtypes()
+    if lib().bsa_workspace_size(ctypes.byref(p)) <= NOALLOC_SCRATCH_BYTES:
+        s = bsa_shape_info(p)
+        x, rows = s.BH * s.N * s.d, s.rows + 1
+    else:
+        x = rows = 0          # the library rejects this plan before touching any pointer
+    _tensors("bsa_plan_noalloc", ("q", q, bf, x), ("k", k, bf, x), ("row_ptr", row_ptr, i32, rows),
+             ("col_idx", col_idx, i32, 0))
     _check(lib().bsa_plan_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(row_ptr),
                                   _ptr(col_idx), col_idx.numel(), _stream(stream)),
            "bsa_plan_noalloc")
 
 
+def _forward_tensors(what, p, q, k, v, row_ptr, col_idx, workspace, out, lse):
+    bf, f32, i32 = _dtypes()
+    s = bsa_shape_info(p)
+    x = s.BH * s.N * s.d
+    _tensors(what, ("q", q, bf, x), ("k", k, bf, x), ("v", v, bf, x), ("out", out, bf, x),
+             ("lse", lse, f32, s.BH * s.N), ("row_ptr", row_ptr, i32, s.rows + 1),
+             ("col_idx", col_idx, i32, 0), ("workspace", workspace, None, 0))
+
+
 def bsa_forward(p, q, k, v, row_ptr, col_idx, workspace, out, lse=None, stream=None):
+    _forward_tensors("bsa_forward", p, q, k, v, row_ptr, col_idx, workspace, out, lse)
     _check(lib().bsa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
                              _ptr(col_idx), col_idx.numel(), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse),
@@ -190,6 +271,7 @@ def bsa_forward(p, q, k, v, row_ptr, col_idx, workspace, out, lse=None, stream=N
 
 def bsa_forward_ex(p, q, k, v, row_ptr, col_idx, workspace, out, lse=None, timeout_ns=0,
                    debug_flags=0, stream=None):
+    _forward_tensors("bsa_forward_ex", p, q, k, v, row_ptr, col_idx, workspace, out, lse)
     _check(lib().bsa_forward_ex(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
                                 _ptr(col_idx), col_idx.numel(), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), _ptr(out),
@@ -206,6 +288,14 @@ def bsa_backward_workspace_size(p: bsa_params) -> int:
 
 def bsa_backward(p, q, k, v, out, lse, dout, row_ptr, col_idx, workspace, dq, dk, dv,
                  stream=None):
+    bf, f32, i32 = _dtypes()
+    s = bsa_shape_info(p)
+    x = s.BH * s.N * s.d
+    _tensors("bsa_backward", ("q", q, bf, x), ("k", k, bf, x), ("v", v, bf, x), ("out", out, bf, x),
+             ("lse", lse, f32, s.BH * s.N), ("dout", dout, bf, x),
+             ("row_ptr", row_ptr, i32, s.rows + 1), ("col_idx", col_idx, i32, 0),
+             ("workspace", workspace, None, 0), ("dq", dq, bf, x), ("dk", dk, bf, x),
+             ("dv", dv, bf, x))
     _check(lib().bsa_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
                               _ptr(dout), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
                               _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -213,6 +303,11 @@ def bsa_backward(p, q, k, v, out, lse, dout, row_ptr, col_idx, workspace, dq, dk
 
 
 def bsa_select_pooled(p, qpool, kpool, workspace, row_ptr, col_idx, kshard=0, stream=None):
+    _, f32, i32 = _dtypes()
+    s = bsa_shape_info(p)
+    _tensors("bsa_select_pooled", ("qpool", qpool, f32, s.BH * s.Nq * s.d),
+             ("kpool", kpool, f32, s.BH * s.Nk * s.d), ("workspace", workspace, None, 0),
+             ("row_ptr", row_ptr, i32, s.rows + 1), ("col_idx", col_idx, i32, 0))
     _check(lib().bsa_select_pooled(ctypes.byref(p), _ptr(qpool), _ptr(kpool), int(kshard),
                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
                                    _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
@@ -224,6 +319,10 @@ def bsa_csr_slice_workspace_size(n_rows: int) -> int:
 
 
 def bsa_csr_slice(row_ptr, col_idx, lo, hi, workspace, out_row_ptr, out_col_idx, stream=None):
+    _, _, i32 = _dtypes()
+    _tensors("bsa_csr_slice", ("row_ptr", row_ptr, i32, 1), ("col_idx", col_idx, i32, 0),
+             ("workspace", workspace, None, 0),
+             ("out_row_ptr", out_row_ptr, i32, row_ptr.numel()), ("out_col_idx", out_col_idx, i32, 0))
     _check(lib().bsa_csr_slice(row_ptr.numel() - 1, _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
                                int(lo), int(hi), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _ptr(out_row_ptr),
@@ -232,44 +331,74 @@ def bsa_csr_slice(row_ptr, col_idx, lo, hi, workspace, out_row_ptr, out_col_idx,
 
 
 def bsa_lse_merge(p, out, lse, out_part, lse_part, stream=None):
+    bf, f32, _ = _dtypes()
+    s = bsa_shape_info(p)
+    x = s.BH * s.N * s.d
+    _tensors("bsa_lse_merge", ("out", out, bf, x), ("lse", lse, f32, s.BH * s.N),
+             ("out_part", out_part, bf, x), ("lse_part", lse_part, f32, s.BH * s.N))
     _check(lib().bsa_lse_merge(ctypes.byref(p), _ptr(out), _ptr(lse), _ptr(out_part),
                                _ptr(lse_part), _stream(stream)), "bsa_lse_merge")
 
 
 def bsa_grad_accumulate(p, part, acc, overwrite=False, stream=None):
+    bf, f32, _ = _dtypes()
+    s = bsa_shape_info(p)
+    x = s.BH * s.N * s.d
+    _tensors("bsa_grad_accumulate", ("part", part, bf, x), ("acc", acc, f32, x))
     _check(lib().bsa_grad_accumulate(ctypes.byref(p), _ptr(part), _ptr(acc), 1 if overwrite else 0,
                                      _stream(stream)), "bsa_grad_accumulate")
 
 
 def bsa_grad_finalize(p, acc, out, stream=None):
+    bf, f32, _ = _dtypes()
+    s = bsa_shape_info(p)
+    x = s.BH * s.N * s.d
+    _tensors("bsa_grad_finalize", ("acc", acc, f32, x), ("out", out, bf, x))
     _check(lib().bsa_grad_finalize(ctypes.byref(p), _ptr(acc), _ptr(out), _stream(stream)),
            "bsa_grad_finalize")
 
 
 def bsa_read_status(workspace, stream=None) -> int:
+    _tensors("bsa_read_status", ("workspace", workspace, None, 4))
     return lib().bsa_read_status(_ptr(workspace), _stream(stream))
 
 
 def bsa_rearrange(p, x, out, inverse=False, stream=None):
+    bf, _, _ = _dtypes()
+    s = bsa_shape_info(p)
+    thw, blk = s.BH * s.N * s.d, s.BH * s.Nc * 128 * s.d
+    _tensors("bsa_rearrange", ("x", x, bf, blk if inverse else thw),
+             ("out", out, bf, thw if inverse else blk))
     _check(lib().bsa_rearrange(ctypes.byref(p), _ptr(x), _ptr(out), 1 if inverse else 0,
                                _stream(stream)), "bsa_rearrange")
 
 
 def bsa_pool(p, x, pooled, stream=None):
+    bf, f32, _ = _dtypes()
+    s = bsa_shape_info(p)
+    _tensors("bsa_pool", ("x", x, bf, s.BH * s.N * s.d), ("pooled", pooled, f32, s.BH * s.Nc * s.d))
     _check(lib().bsa_pool(ctypes.byref(p), _ptr(x), _ptr(pooled), _stream(stream)), "bsa_pool")
 
 
 def bsa_scores(p, qp, kp, S, stream=None):
+    _, f32, _ = _dtypes()
+    s = bsa_shape_info(p)
+    _tensors("bsa_scores", ("qp", qp, f32, s.BH * s.Nq * s.d), ("kp", kp, f32, s.BH * s.Nk * s.d),
+             ("S", S, f32, s.BH * s.Nq * s.Nk))
     _check(lib().bsa_scores(ctypes.byref(p), _ptr(qp), _ptr(kp), _ptr(S), _stream(stream)),
            "bsa_scores")
 
 
 def bsa_selftest_exp2(x, y_poly, y_mufu, stream=None):
+    _, f32, _ = _dtypes()
+    _tensors("bsa_selftest_exp2", ("x", x, f32, 0), ("y_poly", y_poly, f32, x.numel()),
+             ("y_mufu", y_mufu, f32, x.numel()))
     _check(lib().bsa_selftest_exp2(_ptr(x), _ptr(y_poly), _ptr(y_mufu), x.numel(),
                                    _stream(stream)), "bsa_selftest_exp2")
 
 
 def bsa_selftest_timeout(workspace, timeout_ns, stream=None):
+    _tensors("bsa_selftest_timeout", ("workspace", workspace, None, 256))
     _check(lib().bsa_selftest_timeout(_ptr(workspace), int(timeout_ns), _stream(stream)),
            "bsa_selftest_timeout")
 

@@ -210,6 +210,21 @@ int bsa_plan_sizes(const bsa_params* p, int64_t* n_rows, int64_t* max_nnz) {
     return BSA_OK;
 }
 
+int bsa_shape_info(const bsa_params* p, bsa_shape* out) {
+    Dims g;
+    const int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!out) return BSA_ERR_INVALID_ARG;
+    out->BH = g.BH;
+    out->N = g.N;
+    out->rows = g.rows;
+    out->d = g.d;
+    out->Nc = g.Nc;
+    out->Nq = g.Nq;
+    out->Nk = g.Nk;
+    return BSA_OK;
+}
+
 int bsa_plan(const bsa_params* p, const void* q, const void* k, void* workspace, size_t ws_bytes,
              int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, void* stream) {
     Dims g;

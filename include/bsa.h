@@ -124,6 +124,27 @@ BSA_API size_t bsa_workspace_size(const bsa_params* p);
  * otherwise). Host-only call. */
 BSA_API int bsa_plan_sizes(const bsa_params* p, int64_t* n_rows, int64_t* max_nnz);
 
+/* Element counts of the tensors a call for `p` reads and writes, so a binding
+ * can check caller buffers before anything reaches the device:
+ *   BH*N*d   q, k, v, out, dout, dq, dk, dv ([T,H,W] order, bf16);
+ *   BH*N     lse (fp32);
+ *   BH*Nc*128*d  the chunk-major side of bsa_rearrange (partial edge chunks
+ *            padded to 128 slots);
+ *   BH*Nc*d  bsa_pool's output; BH*Nq*d pooled queries and BH*Nk*d pooled
+ *            keys of bsa_scores / bsa_select_pooled; BH*Nq*Nk their scores;
+ *   rows+1   row_ptr.
+ * Host-only call; SHAPE, UNSUPPORTED or INVALID_ARG as for bsa_plan_sizes. */
+typedef struct {
+    int64_t BH;    /* B*heads */
+    int64_t N;     /* tokens per (batch, head): T*H*W */
+    int64_t rows;  /* CSR rows: BH*Nq */
+    int32_t d;     /* head dimension */
+    int32_t Nc;    /* (4,4,8) chunks per (batch, head), partial edge chunks included */
+    int32_t Nq;    /* query chunks computed per (batch, head): frames [q_begin, q_end) */
+    int32_t Nk;    /* key chunks per (batch, head) (of the key chunk shape) */
+} bsa_shape;
+BSA_API int bsa_shape_info(const bsa_params* p, bsa_shape* out);
+
 /*
  * Block selection ([P1] pooled block similarity + top-r; [P3] Top-K / CDF):
  *   1. mean-pool every (4,4,8) chunk of Q and K in fp32 ([P1] Q_pool, K_pool);

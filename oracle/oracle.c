@@ -193,8 +193,8 @@ static int int_cmp(const void* a, const void* b) {
 /*
  * Block selection over the scores S[bh][i][m] -> CSR in row order (bh, i).
  * mode 0 = top-k ([P1] top-r; [P3] Top-K), mode 1 = CDF ([P3] CDF threshold;
- * [P1] "CDF-p mode": descending pooled scores until the cumulative softmax of
- * the scores reaches p), mode 2 = combination ([P3] names a combined mode next to Top-K
+ * [P1] CDF-p: walk the chunks from the highest pooled score down and stop as
+ * soon as their softmax mass adds up to p or more), mode 2 = combination ([P3] names a combined mode next to Top-K
  * and the CDF threshold without defining it; read as: a chunk is kept when
  * both rules keep it, i.e. the first min(k, CDF count) chunks of the common
  * descending order). k is clamped to |A(i)|. fp32 != 0 takes the CDF

@@ -96,3 +96,131 @@ def test_product_modules_never_import_the_oracle():
     root = __file__.rsplit("/tests/", 1)[0]
     r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+# ------------------------------------------------------------------ tensor shapes and checks
+
+import ctypes  # noqa: E402
+
+import block_sparse_attention_13_b200 as bsa  # noqa: E402
+
+
+@pytest.mark.parametrize("kw,want", [
+    # 8x8x16 grid: 2x2x2 chunks of 128 tokens
+    (dict(B=1, heads=2, T=8, H=8, W=16, d=64), dict(BH=2, N=1024, Nc=8, Nq=8, Nk=8, rows=16)),
+    # partial edge chunks: ceil(10/4) x ceil(13/4) x ceil(37/8) = 3 x 4 x 5
+    (dict(B=2, heads=3, T=10, H=13, W=37, d=128), dict(BH=6, N=4810, Nc=60, Nq=60, Nk=60,
+                                                         rows=360)),
+    # frames [4, 8) of 16: query chunks 4..7 of 16
+    (dict(B=1, heads=2, T=16, H=8, W=16, d=64, q_begin=4, q_end=8),
+     dict(BH=2, N=2048, Nc=16, Nq=4, Nk=16, rows=8)),
+    # key chunks of (8,8,8): 2 x 1 x 2 of them over 4 x 2 x 2 query chunks
+    (dict(B=1, heads=1, T=16, H=8, W=16, d=128, kchunk=(8, 8, 8)),
+     dict(BH=1, N=2048, Nc=16, Nq=16, Nk=4, rows=16)),
+])
+def test_shape_info(kw, want):
+    kw = dict(kw)
+    p = bsa.make_params(kw.pop("B"), kw.pop("heads"), kw.pop("T"), kw.pop("H"), kw.pop("W"),
+                        kw.pop("d"), **kw)
+    s = bsa.bsa_shape_info(p)
+    assert {k: getattr(s, k) for k in want} == want
+    assert s.rows == bsa.bsa_plan_sizes(p)[0]
+
+
+def test_shape_info_rejects_invalid_params():
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.bsa_shape_info(bsa.make_params(1, 1, 0, 8, 8, 64))
+    assert e.value.code == bsa.BSA_ERR_SHAPE
+    p = bsa.make_params(1, 1, 8, 8, 8, 64)
+    assert bsa.lib().bsa_shape_info(ctypes.byref(p), None) == bsa.BSA_ERR_INVALID_ARG
+
+
+def _raises(fn):
+    with pytest.raises(bsa.BsaError) as e:
+        fn()
+    return e.value.code, str(e.value)
+
+
+def test_binding_checks_tensors_before_the_library_sees_them():
+    """Every mirror checks dtype, contiguity, size and device before it hands a
+    pointer to the library (a CPU or undersized tensor would otherwise reach the
+    kernels as a bad address). Here, without a GPU, a tensor of the right kind
+    and size fails on the device check."""
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    p = bsa.make_params(1, 2, 8, 8, 16, 64)
+    x = 2 * 1024 * 64
+    q = torch.zeros(x, dtype=bf)
+    rp, ci = torch.zeros(17, dtype=i32), torch.zeros(64, dtype=i32)
+    ws = torch.zeros(bsa.bsa_workspace_size(p), dtype=torch.uint8)
+    lse = torch.zeros(2 * 1024, dtype=f32)
+    INV, SHAPE = bsa.BSA_ERR_INVALID_ARG, bsa.BSA_ERR_SHAPE
+
+    assert _raises(lambda: bsa.bsa_plan(p, q.float(), q, ws, rp, ci))[0] == INV
+    strided = torch.zeros(2 * x, dtype=bf)[::2]
+    c, m = _raises(lambda: bsa.bsa_plan(p, strided, q, ws, rp, ci))
+    assert c == INV and "contiguous" in m
+    c, m = _raises(lambda: bsa.bsa_plan(p, q, q[:-1], ws, rp, ci))
+    assert c == SHAPE and "k holds" in m
+    c, m = _raises(lambda: bsa.bsa_plan(p, q, q, ws, rp[:-1], ci))
+    assert c == SHAPE and "row_ptr" in m
+    c, m = _raises(lambda: bsa.bsa_plan(p, q, q, ws, rp, ci))
+    assert c == INV and "not a CUDA tensor" in m
+    assert _raises(lambda: bsa.bsa_plan(p, q, q, "ws", rp, ci))[0] == INV
+
+    c, m = _raises(lambda: bsa.bsa_forward(p, q, q, q, rp, ci, ws, q, lse[:-1]))
+    assert c == SHAPE and "lse" in m
+    assert _raises(lambda: bsa.bsa_forward(p, q, q, q, rp, ci.long(), ws, q))[0] == INV
+    assert _raises(lambda: bsa.bsa_forward_ex(p, q, q, q, rp, ci, ws, q[:-8]))[0] == SHAPE
+    c, m = _raises(lambda: bsa.bsa_forward(p, q, q, q, rp, ci, ws, q, lse))
+    assert c == INV and "not a CUDA tensor" in m
+
+    c, m = _raises(lambda: bsa.bsa_backward(p, q, q, q, q, lse, q, rp, ci, ws, q, q, q.float()))
+    assert c == INV and "dv" in m
+    c, m = _raises(lambda: bsa.bsa_backward(p, q, q, q, q, lse, q[:-1], rp, ci, ws, q, q, q))
+    assert c == SHAPE and "dout" in m
+
+    # the chunk-major side of the rearrangement holds Nc x 128 slots (partial chunks padded)
+    pr = bsa.make_params(1, 1, 10, 13, 37, 64)
+    tok, blk = 10 * 13 * 37 * 64, 60 * 128 * 64
+    t_tok, t_blk = torch.zeros(tok, dtype=bf), torch.zeros(blk, dtype=bf)
+    c, m = _raises(lambda: bsa.bsa_rearrange(pr, t_tok, t_tok))
+    assert c == SHAPE and "out" in m
+    c, m = _raises(lambda: bsa.bsa_rearrange(pr, t_tok, t_blk, inverse=True))
+    assert c == SHAPE and "x holds" in m
+    assert _raises(lambda: bsa.bsa_rearrange(pr, t_tok, t_blk))[0] == INV       # not CUDA
+
+    c, m = _raises(lambda: bsa.bsa_pool(p, q, torch.zeros(2 * 8 * 64 - 1, dtype=f32)))
+    assert c == SHAPE and "pooled" in m
+    pooled = torch.zeros(2 * 8 * 64, dtype=f32)
+    c, m = _raises(lambda: bsa.bsa_scores(p, pooled, pooled, torch.zeros(2 * 8 * 8 - 1, dtype=f32)))
+    assert c == SHAPE and "S holds" in m
+    c, m = _raises(lambda: bsa.bsa_select_pooled(p, pooled, pooled[:-1], ws, rp, ci))
+    assert c == SHAPE and "kpool" in m
+    c, m = _raises(lambda: bsa.bsa_csr_slice(rp, ci, 0, 4, ws, rp[:-1], ci))
+    assert c == SHAPE and "out_row_ptr" in m
+    c, m = _raises(lambda: bsa.bsa_lse_merge(p, q, lse, q, lse[:-1]))
+    assert c == SHAPE and "lse_part" in m
+    assert _raises(lambda: bsa.bsa_grad_accumulate(p, q, q))[0] == INV        # acc must be fp32
+    acc = torch.zeros(x, dtype=f32)
+    assert _raises(lambda: bsa.bsa_grad_finalize(p, acc[:-1], q))[0] == SHAPE
+    assert _raises(lambda: bsa.bsa_read_status(torch.zeros(3, dtype=torch.uint8)))[0] == SHAPE
+    assert _raises(lambda: bsa.bsa_selftest_timeout(torch.zeros(255, dtype=torch.uint8),
+                                                    1000))[0] == SHAPE
+    y = torch.zeros(8, dtype=f32)
+    assert _raises(lambda: bsa.bsa_selftest_exp2(y, y[:-2], y))[0] == SHAPE
+
+
+def test_noalloc_binding_relies_on_the_library_rejecting_large_plans():
+    """bsa_plan_noalloc's wrapper checks tensor sizes only for plans that fit the
+    library's scratch: larger ones must be rejected by the library itself, before
+    any pointer is used. Pins that the library's limit is not above the binding's."""
+    p = None
+    for heads in range(1, 256):
+        cand = bsa.make_params(1, heads, 16, 48, 80, 128)
+        if bsa.bsa_workspace_size(cand) > bsa.NOALLOC_SCRATCH_BYTES:
+            p = cand
+            break
+    assert p is not None
+    fake = ctypes.c_void_p(0x10000)   # never dereferenced: the call fails on the host
+    rc = bsa.lib().bsa_plan_noalloc(ctypes.byref(p), fake, fake, fake, fake, 1 << 30, None)
+    assert rc == bsa.BSA_ERR_WORKSPACE_TOO_SMALL
