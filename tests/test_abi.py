@@ -337,3 +337,30 @@ def test_query_frame_range(L, kw, code):
     assert rc == code
     if code == 0 and base.get("q_end", 0) == 8:
         assert rows == 2 * 2 * 2 * 2     # heads 2 x chunk frames [0, 2) x (2 x 2) chunks
+
+
+def test_plain_c_program_uses_the_header_and_library(L, tmp_path):
+    """The header compiles as strict C99 and a C program linked against libbsa.so
+    gets the same host-side answers as the Python binding."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(bsa.LIB_PATH)
+    exe = str(tmp_path / "c_consumer")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c_consumer.c"),
+                    "-L", libdir, "-lbsa", f"-Wl,-rpath,{libdir}", "-o", exe], check=True)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {ln.split()[0]: ln.split()[1:] for ln in out if ln.strip()}
+    p = bsa.make_params(1, 32, 24, 48, 80, 128, "topk", 45)
+    rows, nnz = bsa.bsa_plan_sizes(p)
+    s = bsa.bsa_shape_info(p)
+    assert got["plan_sizes"] == ["0", str(rows), str(nnz)]
+    assert got["shape"] == ["0"] + [str(getattr(s, f)) for f in ("BH", "N", "rows", "d", "Nc",
+                                                                    "Nq", "Nk")]
+    assert got["workspace"] == [str(bsa.bsa_workspace_size(p)),
+                                str(bsa.bsa_backward_workspace_size(p))]
+    assert got["null_q"] == [str(bsa.BSA_ERR_INVALID_ARG)]
+    assert got["bad_d"][0] == str(bsa.BSA_ERR_UNSUPPORTED)
+    assert got["version"] == [str(bsa.bsa_version())]
