@@ -6,10 +6,22 @@
 #include <cstdint>
 #include <cstring>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "bsa_internal.cuh"
 #include "bsa_ptx.cuh"
 
 namespace bsa {
+
+// NVTX range over the host side of one call (argument checks and launches), so
+// a profiler's timeline groups each entry point's kernels under its name. The
+// calls cost a few nanoseconds when no profiler is attached.
+struct TraceRange {
+    explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+    TraceRange(const TraceRange&) = delete;
+    TraceRange& operator=(const TraceRange&) = delete;
+};
 
 static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -227,6 +239,7 @@ int bsa_shape_info(const bsa_params* p, bsa_shape* out) {
 
 int bsa_plan(const bsa_params* p, const void* q, const void* k, void* workspace, size_t ws_bytes,
              int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, void* stream) {
+    TraceRange trace("bsa_plan");
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
@@ -244,8 +257,15 @@ int bsa_plan(const bsa_params* p, const void* q, const void* k, void* workspace,
     float* kp = reinterpret_cast<float*>(ws + L.kpool);
     float* S = reinterpret_cast<float*>(ws + L.scores);
     uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
-    if ((rc = cuda_status(launch_pool(g, q, k, qp, kp, st))) != BSA_OK) return rc;
-    if ((rc = cuda_status(launch_scores(g, qp, kp, S, st))) != BSA_OK) return rc;
+    {
+        TraceRange stage("bsa_plan.pool");
+        if ((rc = cuda_status(launch_pool(g, q, k, qp, kp, st))) != BSA_OK) return rc;
+    }
+    {
+        TraceRange stage("bsa_plan.scores");
+        if ((rc = cuda_status(launch_scores(g, qp, kp, S, st))) != BSA_OK) return rc;
+    }
+    TraceRange select_stage("bsa_plan.select");
     int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
     int32_t* padded = reinterpret_cast<int32_t*>(ws + L.padded);
     if (g.m == 1)
@@ -267,6 +287,7 @@ int bsa_forward_ex(const bsa_params* p, const void* q, const void* k, const void
                    const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
                    void* workspace, size_t ws_bytes, void* out, float* lse, uint64_t timeout_ns,
                    int debug_flags, void* stream) {
+    TraceRange trace("bsa_forward");
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
@@ -301,6 +322,7 @@ int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* 
                  const void* out, const float* lse, const void* dout, const int32_t* row_ptr,
                  const int32_t* col_idx, int64_t col_capacity, void* workspace, size_t ws_bytes,
                  void* dq, void* dk, void* dv, void* stream) {
+    TraceRange trace("bsa_backward");
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
@@ -321,6 +343,7 @@ int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* 
 int bsa_select_pooled(const bsa_params* p, const float* qpool, const float* kpool, int32_t kshard,
                       void* workspace, size_t ws_bytes, int32_t* row_ptr, int32_t* col_idx,
                       int64_t col_capacity, void* stream) {
+    TraceRange trace("bsa_select_pooled");
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
@@ -360,6 +383,7 @@ size_t bsa_csr_slice_workspace_size(int64_t n_rows) {
 int bsa_csr_slice(int64_t n_rows, const int32_t* row_ptr, const int32_t* col_idx,
                   int64_t col_capacity, int32_t lo, int32_t hi, void* workspace, size_t ws_bytes,
                   int32_t* out_row_ptr, int32_t* out_col_idx, int64_t out_capacity, void* stream) {
+    TraceRange trace("bsa_csr_slice");
     if (n_rows < 0 || !row_ptr || !col_idx || !workspace || !out_row_ptr || !out_col_idx ||
         col_capacity < 0 || out_capacity < 0 || lo < 0 || hi < lo)
         return BSA_ERR_INVALID_ARG;
@@ -380,6 +404,7 @@ int bsa_csr_slice(int64_t n_rows, const int32_t* row_ptr, const int32_t* col_idx
 
 int bsa_lse_merge(const bsa_params* p, void* out, float* lse, const void* out_part,
                   const float* lse_part, void* stream) {
+    TraceRange trace("bsa_lse_merge");
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
@@ -393,6 +418,7 @@ int bsa_lse_merge(const bsa_params* p, void* out, float* lse, const void* out_pa
 
 int bsa_grad_accumulate(const bsa_params* p, const void* part, float* acc, int overwrite,
                         void* stream) {
+    TraceRange trace("bsa_grad_accumulate");
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
@@ -404,6 +430,7 @@ int bsa_grad_accumulate(const bsa_params* p, const void* part, float* acc, int o
 }
 
 int bsa_grad_finalize(const bsa_params* p, const float* acc, void* out, void* stream) {
+    TraceRange trace("bsa_grad_finalize");
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
@@ -430,6 +457,7 @@ int bsa_read_status(void* workspace, void* stream) {
 }
 
 int bsa_rearrange(const bsa_params* p, const void* x, void* out, int inverse, void* stream) {
+    TraceRange trace("bsa_rearrange");
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
@@ -440,6 +468,7 @@ int bsa_rearrange(const bsa_params* p, const void* x, void* out, int inverse, vo
 }
 
 int bsa_pool(const bsa_params* p, const void* x, float* pooled, void* stream) {
+    TraceRange trace("bsa_pool");
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
@@ -450,6 +479,7 @@ int bsa_pool(const bsa_params* p, const void* x, float* pooled, void* stream) {
 }
 
 int bsa_scores(const bsa_params* p, const float* qp, const float* kp, float* S, void* stream) {
+    TraceRange trace("bsa_scores");
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
