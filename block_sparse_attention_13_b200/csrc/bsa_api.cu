@@ -188,7 +188,7 @@ using namespace bsa;
 
 extern "C" {
 
-int bsa_version(void) { return 100; }
+int bsa_version(void) { return 200; }
 
 const char* bsa_status_string(int s) {
     switch (s) {

@@ -89,8 +89,9 @@ typedef struct {
                          * only the noisy queries are evaluated, against the cached
                          * condition K/V plus the noisy K/V, which stay in one
                          * [B,heads,T*H*W,d] buffer. Row r of the CSR is query chunk
-                         * q_begin/4*(H/4)*(W/8) + r % Nq of (batch, head) r / Nq, where
-                         * Nq = Nc - q_begin/4*(H/4)*(W/8). */
+                         * q_begin/4*NH*NW + r % Nq of (batch, head) r / Nq, where Nq is
+                         * the number of chunks in frames [q_begin, q_end) (Nc -
+                         * q_begin/4*NH*NW when q_end = T; bsa_shape_info reports it). */
     int32_t kchunk_t, kchunk_h, kchunk_w;
                         /* key chunk shape; 0 on an axis = the query chunk's size (4, 4, 8).
                          * Otherwise a multiple of it on that axis, at most 8 (4,4,8) boxes
@@ -107,7 +108,7 @@ typedef struct {
                          * computes the rows of its own frame range (bsa_select_pooled). */
 } bsa_params;
 
-/* Library version: major*10000 + minor*100 + patch. */
+/* Library version: major*10000 + minor*100 + patch (0.2.0: bsa_shape_info added). */
 BSA_API int bsa_version(void);
 
 /* Text for a status code (static storage; never NULL). */
@@ -118,8 +119,8 @@ BSA_API const char* bsa_status_string(int status);
  * invalid. The same workspace serves both calls. */
 BSA_API size_t bsa_workspace_size(const bsa_params* p);
 
-/* CSR sizes for `p`: *n_rows = B*heads*Nq (Nq = query chunks from q_begin on,
- * Nc when q_begin = 0); *max_nnz = col_idx capacity that always suffices, in
+/* CSR sizes for `p`: *n_rows = B*heads*Nq (Nq = query chunks of frames
+ * [q_begin, q_end), Nc for the whole grid); *max_nnz = col_idx capacity that always suffices, in
  * (4,4,8) boxes (exact for TOPK with the default key chunk; an upper bound
  * otherwise). Host-only call. */
 BSA_API int bsa_plan_sizes(const bsa_params* p, int64_t* n_rows, int64_t* max_nnz);
