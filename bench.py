@@ -72,7 +72,7 @@ def load_peaks():
 def kernel_hash():
     h = hashlib.sha256()
     for f in sorted(os.listdir(os.path.dirname(KERNEL_SRC))):
-        if f in ("bsa_attn.cu", "bsa_ptx.cuh"):
+        if f in ("bsa_attn.cu", "bsa_ptx.cuh", "bsa_internal.cuh"):   # the kernel's sources
             with open(os.path.join(os.path.dirname(KERNEL_SRC), f), "rb") as fh:
                 h.update(fh.read())
     return h.hexdigest()[:16]
