@@ -52,7 +52,9 @@ typedef enum {
     BSA_OK = 0,
     BSA_ERR_INVALID_ARG = 1,         /* null pointer, bad enum, k < 1, p outside (0,1] ...   */
     BSA_ERR_SHAPE = 2,               /* sizes <= 0, t_cond or q_begin not a multiple of 4 ... */
-    BSA_ERR_UNSUPPORTED = 3,         /* d not in {64,128}, chunk shape != (4,4,8), no sm_100  */
+    BSA_ERR_UNSUPPORTED = 3,         /* d not in {64,128}, chunk shape != (4,4,8), no sm_100,
+                                        or beyond the limits: Nc <= 2048 chunks per (batch,
+                                        head), B*heads <= 65535, CSR rows*Nc < 2^31          */
     BSA_ERR_ALIGNMENT = 4,           /* a bf16 tensor or workspace pointer is not 16-byte
                                         aligned, or an int32 / fp32 array not 4-byte aligned */
     BSA_ERR_WORKSPACE_TOO_SMALL = 5, /* ws_bytes < bsa_workspace_size()                       */
