@@ -166,6 +166,19 @@ def test_invalid_params(L, kw, code):
     assert bsa.lib().bsa_workspace_size(ctypes.byref(p)) == 0
 
 
+def test_size_limits_at_their_boundaries(L):
+    # 2,048 chunks per (batch, head) is the largest grid; one more chunk axis step is rejected
+    assert rc_sizes(P(T=4 * 32, H=4 * 8, W=8 * 8))[0] == 0                  # Nc = 2048
+    assert rc_sizes(P(T=4 * 32, H=4 * 8, W=8 * 8 + 1))[0] == bsa.BSA_ERR_UNSUPPORTED
+    # B * heads <= 65535
+    assert rc_sizes(P(B=5, heads=13107, T=4, H=4, W=8))[0] == 0             # 65535
+    assert rc_sizes(P(B=2, heads=32768, T=4, H=4, W=8))[0] == bsa.BSA_ERR_UNSUPPORTED
+    # CSR offsets are int32: rows * Nc <= 2^31 - 1 (rows = heads * 2048 here)
+    assert rc_sizes(P(B=1, heads=511, T=4 * 32, H=4 * 8, W=8 * 8))[0] == 0
+    assert rc_sizes(P(B=1, heads=512, T=4 * 32, H=4 * 8, W=8 * 8))[0] == \
+        bsa.BSA_ERR_UNSUPPORTED                                               # exactly 2^31
+
+
 def test_chunk_shape_other_than_448_unsupported(L):
     p = P()
     p.chunk_w = 4
