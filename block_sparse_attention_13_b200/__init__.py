@@ -40,7 +40,8 @@ EXPORTED = ("bsa_version", "bsa_status_string", "bsa_workspace_size", "bsa_plan_
             "bsa_rearrange", "bsa_pool", "bsa_scores", "bsa_selftest_exp2",
             "bsa_selftest_timeout", "bsa_backward_workspace_size", "bsa_backward",
             "bsa_select_pooled", "bsa_csr_slice_workspace_size", "bsa_csr_slice",
-            "bsa_lse_merge", "bsa_grad_accumulate", "bsa_grad_finalize", "bsa_shape_info")
+            "bsa_lse_merge", "bsa_grad_accumulate", "bsa_grad_finalize", "bsa_shape_info",
+            "bsa_forward_host_workspace_size", "bsa_forward_host")
 
 # Scratch array of bsa_plan_noalloc inside the library (include/bsa.h: 32 MiB);
 # a plan whose workspace exceeds it is rejected by the library before any CUDA call.
@@ -109,6 +110,9 @@ def lib():
             "bsa_workspace_size": (sz, [P]),
             "bsa_plan_sizes": (i32, [P, ctypes.POINTER(i64), ctypes.POINTER(i64)]),
             "bsa_shape_info": (i32, [P, ctypes.POINTER(bsa_shape)]),
+            "bsa_forward_host_workspace_size": (sz, [P, ctypes.c_int32, ctypes.c_int32]),
+            "bsa_forward_host": (i32, [P, vp, vp, vp, vp, ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.POINTER(vp), vp, sz, vp]),
             "bsa_plan": (i32, [P, vp, vp, vp, sz, vp, vp, i64, vp]),
             "bsa_plan_noalloc": (i32, [P, vp, vp, vp, vp, i64, vp]),
             "bsa_forward": (i32, [P, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, vp]),
@@ -150,16 +154,17 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _tensors(what, *specs):
+def _tensors(what, *specs, where="cuda"):
     """Checks the tensors of one call before their pointers are passed on.
 
     Each spec is (name, tensor or None, dtype or None, minimum size). A tensor
     the library reads or writes must have that dtype, be contiguous, hold at
     least that many elements (bytes when dtype is None: a workspace) and live on
-    the current CUDA device: anything else would reach the kernels as a bad
-    address. Raises BsaError: INVALID_ARG for the kind of tensor, SHAPE for its
-    size; the device is checked after every tensor's kind and size. None entries
-    (optional outputs) are skipped.
+    the current CUDA device (where="cpu": in host memory): anything else would
+    reach the kernels or the copies as a bad address. Raises BsaError:
+    INVALID_ARG for the kind of tensor, SHAPE for its size; the device is
+    checked after every tensor's kind and size. None entries (optional outputs)
+    are skipped.
     """
     import torch
     given = [(name, t, dtype, need) for name, t, dtype, need in specs if t is not None]
@@ -174,6 +179,11 @@ def _tensors(what, *specs):
         if have < need:
             unit = "elements" if dtype is not None else "bytes"
             raise BsaError(BSA_ERR_SHAPE, f"{what}: {name} holds {have} {unit}, needs {need}")
+    if where == "cpu":
+        for name, t, _, _ in given:
+            if t.device.type != "cpu":
+                raise BsaError(BSA_ERR_INVALID_ARG, f"{what}: {name} is not in host memory")
+        return
     cur = None
     for name, t, _, _ in given:
         if not t.is_cuda:
@@ -300,6 +310,31 @@ def bsa_backward(p, q, k, v, out, lse, dout, row_ptr, col_idx, workspace, dq, dk
                               _ptr(dout), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
                               _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)), "bsa_backward")
+
+
+def bsa_forward_host_workspace_size(p: bsa_params, group: int, slots: int) -> int:
+    n = lib().bsa_forward_host_workspace_size(ctypes.byref(p), int(group), int(slots))
+    if n == 0:
+        raise BsaError(BSA_ERR_INVALID_ARG, "bsa_forward_host_workspace_size")
+    return n
+
+
+def bsa_forward_host(p, q, k, v, out, group, streams, workspace, stream=None):
+    """plan + forward for q, k, v, out in host memory (CPU tensors, pinned for
+    overlap): groups of `group` (batch, head) pairs run on `streams` (torch
+    streams or raw handles), staged in `workspace` (device, status block
+    zeroed before the first call). The caller's stream waits for all of it."""
+    bf, _, _ = _dtypes()
+    s = bsa_shape_info(p)
+    x = s.BH * s.N * s.d
+    _tensors("bsa_forward_host", ("q", q, bf, x), ("k", k, bf, x), ("v", v, bf, x),
+             ("out", out, bf, x), where="cpu")
+    _tensors("bsa_forward_host", ("workspace", workspace, None, 0))
+    handles = (ctypes.c_void_p * len(streams))(*[_stream(st).value for st in streams])
+    _check(lib().bsa_forward_host(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                  int(group), len(streams), handles, _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)),
+           "bsa_forward_host")
 
 
 def bsa_select_pooled(p, qpool, kpool, workspace, row_ptr, col_idx, kshard=0, stream=None):

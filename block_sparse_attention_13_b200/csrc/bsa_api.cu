@@ -6,22 +6,10 @@
 #include <cstdint>
 #include <cstring>
 
-#include <nvtx3/nvToolsExt.h>
-
 #include "bsa_internal.cuh"
 #include "bsa_ptx.cuh"
 
 namespace bsa {
-
-// NVTX range over the host side of one call (argument checks and launches), so
-// a profiler's timeline groups each entry point's kernels under its name. The
-// calls cost a few nanoseconds when no profiler is attached.
-struct TraceRange {
-    explicit TraceRange(const char* name) { nvtxRangePushA(name); }
-    ~TraceRange() { nvtxRangePop(); }
-    TraceRange(const TraceRange&) = delete;
-    TraceRange& operator=(const TraceRange&) = delete;
-};
 
 static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -67,7 +55,7 @@ WsLayout ws_layout(const Dims& g, const bsa_params& p) {
 }
 
 // Validates `p` and fills the derived sizes. Host only, no CUDA calls.
-static int make_dims(const bsa_params* p, Dims* g) {
+int make_dims(const bsa_params* p, Dims* g) {
     if (!p || !g) return BSA_ERR_INVALID_ARG;
     if (p->B <= 0 || p->heads <= 0 || p->T <= 0 || p->H <= 0 || p->W <= 0 || p->d <= 0)
         return BSA_ERR_SHAPE;
@@ -165,7 +153,7 @@ static int64_t max_key_nnz_of(const Dims& g, const bsa_params& p) {
 }
 
 // CSR entries in (4,4,8) boxes: a key chunk covers at most m of them.
-static int64_t max_nnz_of(const Dims& g, const bsa_params& p) { return max_key_nnz_of(g, p) * g.m; }
+int64_t max_nnz_of(const Dims& g, const bsa_params& p) { return max_key_nnz_of(g, p) * g.m; }
 
 static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 // int32 CSR arrays and fp32 vectors are read element by element: 4-byte alignment
@@ -173,7 +161,7 @@ static bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr)
 
 static int cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
 
-static int device_ok() {
+int device_ok() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
     int major = 0;

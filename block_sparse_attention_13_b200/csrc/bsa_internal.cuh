@@ -2,12 +2,24 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
+
 #include <atomic>
 #include <cstdint>
 
 #include "../../include/bsa.h"
 
 namespace bsa {
+
+// NVTX range over the host side of one call (argument checks and launches), so
+// a profiler's timeline groups each entry point's kernels under its name. The
+// calls cost a few nanoseconds when no profiler is attached.
+struct TraceRange {
+    explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+    TraceRange(const TraceRange&) = delete;
+    TraceRange& operator=(const TraceRange&) = delete;
+};
 
 // Raises a kernel's dynamic shared-memory limit on the current device. The
 // attribute belongs to that device's context, so `done` keeps one bit per device
@@ -74,6 +86,13 @@ struct WsLayout {
 };
 
 WsLayout ws_layout(const Dims& g, const bsa_params& p);
+
+// Host-side checks shared by the entry points (no CUDA call except device_ok):
+// parameter validation into derived sizes, the CSR capacity a plan needs, and
+// whether the current device is an sm_100 part (BSA_OK, UNSUPPORTED or CUDA).
+int make_dims(const bsa_params* p, Dims* g);
+int64_t max_nnz_of(const Dims& g, const bsa_params& p);
+int device_ok();
 
 // Backward workspace layout (byte offsets).
 struct BwdLayout {

@@ -110,7 +110,8 @@ typedef struct {
                          * computes the rows of its own frame range (bsa_select_pooled). */
 } bsa_params;
 
-/* Library version: major*10000 + minor*100 + patch (0.2.0: bsa_shape_info added). */
+/* Library version: major*10000 + minor*100 + patch (0.2.0: bsa_shape_info and
+ * bsa_forward_host added). */
 BSA_API int bsa_version(void);
 
 /* Text for a status code (static storage; never NULL). */
@@ -324,6 +325,32 @@ BSA_API int bsa_grad_finalize(const bsa_params* p, const float* acc, void* out, 
  */
 BSA_API int bsa_plan_noalloc(const bsa_params* p, const void* q, const void* k, int32_t* row_ptr,
                              int32_t* col_idx, int64_t col_capacity, void* stream);
+
+/*
+ * Selection and sparse attention (bsa_plan + bsa_forward) for q, k, v and out in
+ * HOST memory, [B,heads,N,d] bf16 (pinned memory lets the copies run
+ * asynchronously and overlap the kernels; pageable memory works but
+ * serialises them). Each (batch, head) pair is an independent problem ([P1]
+ * section "Block Sparse Attention (BSA)": blocks, pooled scores and the kept
+ * set are per head), so the pairs are split into groups of `group`, and group
+ * i runs on streams[i % slots]: its Q of the computed frames [q_begin, q_end),
+ * its K and V are copied in, the plan's kernels and the forward kernel run on
+ * staging buffers in the workspace, and its output of the computed frames is
+ * copied out (out elsewhere is left as it was). Every slot stream first waits
+ * for the work queued on `stream`, and `stream` waits for every slot at the
+ * end: work queued on `stream` afterwards sees the finished output (read it on
+ * the host after synchronising `stream`). Host buffers must not be touched until then.
+ * group: 1..B*heads. slots: 1..16 streams (cudaStream_t; NULL entries are the
+ * legacy default stream). workspace: device, 256-byte aligned,
+ * >= bsa_forward_host_workspace_size(p, group, slots), owned by the caller;
+ * its first 256 bytes are the status block that bsa_read_status reads (zero
+ * it before the first call). Device errors of every group land there.
+ * Errors: INVALID_ARG, SHAPE, UNSUPPORTED, ALIGNMENT, WORKSPACE_TOO_SMALL, CUDA.
+ */
+BSA_API size_t bsa_forward_host_workspace_size(const bsa_params* p, int32_t group, int32_t slots);
+BSA_API int bsa_forward_host(const bsa_params* p, const void* q, const void* k, const void* v,
+                             void* out, int32_t group, int32_t slots, void* const* streams,
+                             void* workspace, size_t ws_bytes, void* stream);
 
 /* bsa_forward with an explicit limit for every device-side wait (timeout_ns;
  * 0 = the default of 2 s) and debug flags (bit 0: the MMA warp withholds its

@@ -377,3 +377,64 @@ def test_plain_c_program_uses_the_header_and_library(L, tmp_path):
     assert got["null_q"] == [str(bsa.BSA_ERR_INVALID_ARG)]
     assert got["bad_d"][0] == str(bsa.BSA_ERR_UNSUPPORTED)
     assert got["version"] == [str(bsa.bsa_version())]
+
+
+def _r256(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("kw,group,slots", [
+    (dict(B=1, heads=32, T=24, H=48, W=80, d=128, topk=45), 2, 3),
+    (dict(B=2, heads=3, T=10, H=13, W=37, d=64, mode="cdf"), 4, 2),
+    (dict(B=1, heads=5, T=16, H=8, W=16, d=128, topk=3, kchunk=(8, 8, 8)), 5, 1),
+])
+def test_forward_host_workspace_layout(L, kw, group, slots):
+    """256-byte status block, then per slot: Q, K, V, O of one group, the plan's
+    workspace and CSR of one group, each rounded up to 256 bytes."""
+    p = P(**kw)
+    N = p.T * p.H * p.W
+    pg = P(**dict(kw, B=1, heads=group))
+    rows, nnz = bsa.bsa_plan_sizes(pg)
+    slot = (4 * _r256(group * N * p.d * 2) + _r256(bsa.bsa_workspace_size(pg)) +
+            _r256((rows + 1) * 4) + _r256(max(nnz, 1) * 4))
+    assert bsa.bsa_forward_host_workspace_size(p, group, slots) == 256 + slots * slot
+
+
+def test_forward_host_host_checks(L):
+    p = P(B=1, heads=4, T=8, H=8, W=16, d=64)
+    f = L.bsa_forward_host_workspace_size
+    assert f(ctypes.byref(p), 0, 1) == 0                    # group < 1
+    assert f(ctypes.byref(p), 5, 1) == 0                    # group > B*heads
+    assert f(ctypes.byref(p), 2, 0) == 0 and f(ctypes.byref(p), 2, 17) == 0
+    assert f(ctypes.byref(P(T=0)), 1, 1) == 0
+    ws = f(ctypes.byref(p), 2, 2)
+    x = vp(FAKE)
+    streams = (ctypes.c_void_p * 2)(None, None)
+    g = L.bsa_forward_host
+    pp = ctypes.byref(p)
+    # q, k, v, out, group, slots, streams, workspace, ws_bytes, stream
+    assert g(pp, None, x, x, x, 2, 2, streams, x, ws, None) == bsa.BSA_ERR_INVALID_ARG
+    assert g(pp, x, x, x, x, 2, 2, None, x, ws, None) == bsa.BSA_ERR_INVALID_ARG
+    assert g(pp, x, x, x, x, 0, 2, streams, x, ws, None) == bsa.BSA_ERR_INVALID_ARG
+    assert g(pp, x, x, x, x, 2, 17, streams, x, ws, None) == bsa.BSA_ERR_INVALID_ARG
+    assert g(pp, x, x, x, x, 2, 2, streams, vp(FAKE + 16), ws, None) == bsa.BSA_ERR_ALIGNMENT
+    assert g(pp, x, x, x, x, 2, 2, streams, x, ws - 1, None) == \
+        bsa.BSA_ERR_WORKSPACE_TOO_SMALL
+    assert g(ctypes.byref(P(T=0)), x, x, x, x, 2, 2, streams, x, ws, None) == bsa.BSA_ERR_SHAPE
+
+
+def test_forward_host_binding_checks():
+    import torch
+    p = bsa.make_params(1, 2, 8, 8, 16, 64)
+    x = 2 * 1024 * 64
+    h = torch.zeros(x, dtype=torch.bfloat16)
+    ws = torch.zeros(bsa.bsa_forward_host_workspace_size(p, 1, 2), dtype=torch.uint8)
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.bsa_forward_host(p, h, h, h, h[:-1], 1, [None, None], ws)
+    assert e.value.code == bsa.BSA_ERR_SHAPE and "out" in str(e.value)
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.bsa_forward_host(p, h, h, h.float(), h, 1, [None, None], ws)
+    assert e.value.code == bsa.BSA_ERR_INVALID_ARG
+    with pytest.raises(bsa.BsaError) as e:      # the staging workspace must be on the device
+        bsa.bsa_forward_host(p, h, h, h, h, 1, [None, None], ws)
+    assert e.value.code == bsa.BSA_ERR_INVALID_ARG and "CUDA" in str(e.value)
