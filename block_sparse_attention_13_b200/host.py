@@ -26,7 +26,10 @@ def _params_for_group(p: bsa_params, heads: int) -> bsa_params:
 class HostForward:
     """plan + forward for q, k, v in pinned host memory, [B, heads, T*H*W, d] bf16.
 
-    group: (batch, head) pairs per group; streams: groups in flight.
+    group: (batch, head) pairs per group; streams: groups in flight. Whole
+    slices are copied back, so with q_begin > 0 the host output of the skipped
+    frames is overwritten with unspecified values (the C entry bsa_forward_host
+    copies only the computed frames).
     """
 
     def __init__(self, p: bsa_params, group: int = 2, streams: int = 3, device="cuda"):
