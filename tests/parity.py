@@ -2,8 +2,8 @@
 
 Selection: the GPU's chunk lists must equal the oracle's (decided in fp32, the
 kernel's precision) except where pooled scores tie within 1e-5 relative (or,
-for CDF, where the cumulative mass sits within 1e-5 of p); every GPU row must
-then still be a valid selection under the oracle's fp64 scores.
+for CDF, where the cumulative mass sits within 1e-5 of p); every GPU row, equal
+or not, must also be a valid selection under the oracle's fp64 scores.
 
 Attention: GPU bf16 output vs the fp64 oracle evaluated on the GPU's own CSR,
 max-abs <= 2e-2 and mean-abs <= 2e-3 (fp32 accumulation, bf16 inputs,
@@ -85,15 +85,17 @@ def compare_csr(gpu_rp, gpu_ci, ora_rp, ora_ci, S64, Nc, n_cond, mode, p=0.9, ca
     ndiff = 0
     for r in idx:
         g, o = g_rows[r], o_rows[r]
-        if len(g) == len(o) and np.array_equal(g, o):
-            continue
-        ndiff += 1
+        same = len(g) == len(o) and np.array_equal(g, o)
+        ndiff += not same
+        # every row, equal to the oracle's or not, must be a valid selection under the
+        # fp64 scores, so a mistake shared by the kernel and the oracle's float mode fails
         i = r % Nc
         s64 = S64[r // Nc, i]
         cand = _candidates(i, Nk, n_cond, n_cond_k)
         assert valid_topk_set(g, s64, cand), f"row {r}: gpu {g} vs oracle {o} not a tie"
         if mode == "topk":
-            assert len(g) == len(o), f"row {r}: count {len(g)} vs {len(o)}"
+            assert len(g) == min(topk, len(cand)) if topk else len(g) == len(o), \
+                f"row {r}: count {len(g)} vs {len(o)}"
         else:
             k = topk if mode == "topk_cdf" else None
             assert cdf_count_ok(len(g), s64, cand, p, cap_frac, k), \
