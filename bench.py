@@ -9,9 +9,12 @@ inputs resident in HBM. Prints one JSON line (rank 0).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 720p]
   python bench.py --impl reference ...   # the CPU oracle on the host cores
 
-Multi-GPU: one process per GPU (torchrun); every rank runs an independent
-problem (its own batch element), there is no collective on the data path;
-timing is the max over ranks.
+Multi-GPU: one process per GPU (torchrun). By default the heads of the one
+call are split across the ranks (every (batch, head) pair is an independent
+problem for pooling, selection and attention, so there is no collective on the
+data path; strong scaling: the total work is the same for every N). With
+--partition replicas every rank runs its own copy of the problem (its own batch
+element; weak scaling). Timing is the max over ranks.
 """
 from __future__ import annotations
 
@@ -57,6 +60,11 @@ def parse():
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward timing")
     ap.add_argument("--bwd-steps", type=int, default=10)
+    ap.add_argument("--partition", default="heads", choices=["heads", "replicas"],
+                    help="N > 1: split the heads of the one call (default) or run replicas")
+    ap.add_argument("--per-config", default="480p,long,causal_cdf",
+                    help="other workloads timed after the main one (N = 1; '' for none)")
+    ap.add_argument("--per-config-steps", type=int, default=10)
     return ap.parse_args()
 
 
@@ -114,7 +122,7 @@ class ClockSampler:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "25"],
                 stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -208,26 +216,35 @@ def cpu_oracle_sample(wl, q, k, v, target_s):
 
 
 def run_reference(args, wl, rank, world):
+    """The oracle as it stands, on the host cores. Each timed step is one
+    bounded sample of the workload (plan on one (batch, head) pair, attention
+    on a growing set of that head's query chunks); the line reports what ran:
+    `steps` samples of `ms_per_step` wall time each, and the throughput the
+    sample extrapolates to for the full workload (`extrapolated`)."""
     if rank != 0:
         return 0
-    import numpy as np  # noqa: F401
     import synth
     q, k, v = synth.make_qkv(wl.with_(B=1, heads=1))
     per_step = max(1.0, min(args.cpu_seconds, 100.0 / max(1, args.steps + args.warmup)))
-    vals = []
+    vals, secs = [], []
     cb = None
+    t_run0 = time.perf_counter()
     for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         cb = cpu_oracle_sample(wl, q, k, v, per_step)
         if s >= args.warmup:
             vals.append(cb["value"])
+            secs.append(time.perf_counter() - t0)
     value = statistics.median(vals)
     cb["value"] = value
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": cb["est_full_step_s"] * 1e3, "higher_is_better": True,
+        "steps": len(secs), "warmup": args.warmup,
+        "ms_per_step": statistics.mean(secs) * 1e3, "higher_is_better": True,
+        "extrapolated": True, "est_full_step_s": cb["est_full_step_s"],
+        "wall_s": time.perf_counter() - t_run0,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(wl, world),
+        "config": workload_config(wl, world, "oracle"),
         "cpu_baseline": cb,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -236,19 +253,19 @@ def run_reference(args, wl, rank, world):
     return 0
 
 
-def workload_config(wl, world):
+def workload_config(wl, world, parallelism):
     return {"workload": wl.name, "B": wl.B, "heads": wl.heads, "grid_thw": [wl.T, wl.H, wl.W],
             "d": wl.d, "chunk_thw": [4, 4, 8], "mode": wl.mode,
-            "topk": wl.topk if wl.mode == "topk" else None,
-            "cdf_p": wl.cdf_p if wl.mode == "cdf" else None,
-            "t_cond": wl.t_cond, "q_begin": wl.q_begin, "parallelism": f"replicas{world}",
+            "topk": wl.topk if wl.mode != "cdf" else None,
+            "cdf_p": wl.cdf_p if wl.mode != "topk" else None,
+            "t_cond": wl.t_cond, "q_begin": wl.q_begin, "parallelism": parallelism,
             "l2": "inputs larger than L2 (Q+K+V per step "
                   f"{3 * wl.B * wl.heads * wl.N * wl.d * 2 / 1e9:.2f} GB)"}
 
 
 # ---------------------------------------------------------------------- backward
 
-def time_backward(args, wl, p, pl, q, k, v, stream, peak_tf):
+def time_backward(args, wl, p, pl, q, k, v, stream, peak_tf, batch_offset=0, head_offset=0):
     """bsa_backward on the plan of the timed forward: forward once with LSE,
     then K timed backward calls (events on the launching stream). Algorithmic
     FLOPs are the five products of the gradient (S, dP, dV, dS K, dS^T Q:
@@ -257,8 +274,7 @@ def time_backward(args, wl, p, pl, q, k, v, stream, peak_tf):
     import torch
     import synth
     import block_sparse_attention_13_b200 as bsa
-    g_np = synth.make_dout(wl, batch_offset=shard_batch_offset(
-        int(os.environ.get("RANK", "0")), wl))
+    g_np = synth.make_dout(wl, batch_offset=batch_offset, head_offset=head_offset)
     dout = torch.from_numpy(g_np).view(torch.bfloat16).to("cuda")
     out = torch.empty_like(q)
     lse = torch.empty((wl.B, wl.heads, wl.N), dtype=torch.float32, device="cuda")
@@ -291,12 +307,80 @@ def time_backward(args, wl, p, pl, q, k, v, stream, peak_tf):
             "launches_per_call": 6, "device_status": bsa.status_string(rc)}
 
 
+# ---------------------------------------------------------------------- other workloads
+
+def time_config(wl, steps, peak_tf, stream):
+    """plan + forward on another workload (inputs resident, larger than L2):
+    CUDA events per kernel group on the launching stream, `steps` timed steps
+    after 3 warm-up steps."""
+    import torch
+    import synth
+    import block_sparse_attention_13_b200 as bsa
+    host = synth.make_qkv(wl)
+    q, k, v = (torch.from_numpy(a).view(torch.bfloat16).to("cuda") for a in host)
+    del host
+    p = bsa.params_for(wl)
+    pl = bsa.allocate(p)
+    out = torch.empty_like(q)
+    for _ in range(3):
+        bsa.bsa_plan(p, q, k, pl.workspace, pl.row_ptr, pl.col_idx)
+        bsa.bsa_forward(p, q, k, v, pl.row_ptr, pl.col_idx, pl.workspace, out)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for e in ev:
+        e[0].record(stream)
+        bsa.bsa_plan(p, q, k, pl.workspace, pl.row_ptr, pl.col_idx)
+        e[1].record(stream)
+        bsa.bsa_forward(p, q, k, v, pl.row_ptr, pl.col_idx, pl.workspace, out)
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    rc = bsa.bsa_read_status(pl.workspace)
+    nnz = int(pl.row_ptr[-1].item())
+    plan_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    tf = exec_flops(wl, nnz) / fwd_ms / 1e9
+    res = {"plan_ms": plan_ms, "fwd_ms": fwd_ms, "step_ms": plan_ms + fwd_ms,
+           "fwd_exec_tflops": tf, "frac": tf / peak_tf, "nnz": nnz,
+           "sparsity": 1.0 - nnz / (wl.B * wl.heads * wl.Nq * wl.Nc), "steps": steps,
+           "config": workload_config(wl, 1, "single"), "device_status": bsa.status_string(rc)}
+    del q, k, v, out, pl
+    torch.cuda.empty_cache()
+    return res
+
+
 # ---------------------------------------------------------------------- ranks
 
 def shard_batch_offset(rank, wl):
-    """Batch index of this rank's first element: every rank runs its own
-    independent problem (weak scaling, no data exchange)."""
+    """Batch index of this rank's first element when every rank runs its own
+    independent replica of the problem (weak scaling, no data exchange)."""
     return rank * wl.B
+
+
+def shard_heads(rank, world, heads):
+    """Heads [h0, h0 + n) of the call that this rank computes: the heads split as
+    evenly as possible, the first `heads % world` ranks taking one more. Every
+    (batch, head) pair is an independent problem for pooling, selection and
+    attention, so the ranks exchange nothing."""
+    base, extra = divmod(heads, world)
+    n = base + (1 if rank < extra else 0)
+    h0 = rank * base + min(rank, extra)
+    return h0, n
+
+
+def rank_problem(wl, rank, world, partition):
+    """(this rank's workload, batch offset, head offset) of its inputs."""
+    if partition == "heads" and world > 1:
+        h0, n = shard_heads(rank, world, wl.heads)
+        if n == 0:
+            raise ValueError(f"{world} ranks for {wl.heads} heads: rank {rank} has none")
+        return wl.with_(heads=n), 0, h0
+    return wl, shard_batch_offset(rank, wl), 0
+
+
+def parallelism_of(partition, world):
+    if world == 1:
+        return "single"
+    return f"heads/{world}" if partition == "heads" else f"replicas{world}"
 
 
 def reduce_over_ranks(value, op, world, device):
@@ -346,8 +430,11 @@ def main():
     def sum_over_ranks(x):
         return reduce_over_ranks(x, "sum", world, "cuda")
 
-    # inputs: this rank's own problem (batch offset = rank), pinned host + device copies
-    q_np, k_np, v_np = synth.make_qkv(wl, batch_offset=shard_batch_offset(rank, wl))
+    # inputs: this rank's part of the call (its heads) or its own replica, pinned host +
+    # device copies
+    wl_full = wl
+    wl, b_off, h_off = rank_problem(wl_full, rank, world, args.partition)
+    q_np, k_np, v_np = synth.make_qkv(wl, batch_offset=b_off, head_offset=h_off)
     host = [torch.from_numpy(a).view(torch.bfloat16).pin_memory() for a in (q_np, k_np, v_np)]
     q, k, v = (h.to("cuda", non_blocking=False) for h in host)
     p = bsa.params_for(wl)
@@ -398,9 +485,10 @@ def main():
     total_flops = sum_over_ranks(flops * args.steps)
     value = total_flops / (total_ms / 1e3) / 1e12
 
-    # ---- end to end with host buffers (pinned) through the public host API: per step
-    # H2D of q, k, v, plan, forward and D2H of the output, in groups of (batch, head)
-    # pairs whose copies overlap the other groups' kernels
+    # ---- end to end with host buffers (pinned) through the C ABI's host-buffer entry
+    # (bsa_forward_host, via HostForward): per step H2D of q, k, v, plan, forward and D2H
+    # of the output, in groups of (batch, head) pairs whose copies overlap the other
+    # groups' kernels
     from block_sparse_attention_13_b200.host import HostForward
     out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     hf = HostForward(p, group=args.e2e_group, streams=args.e2e_streams)
@@ -450,18 +538,28 @@ def main():
 
     bwd = None
     if not args.no_backward:
-        bwd = time_backward(args, wl, p, pl, q, k, v, stream, peak_tf)
+        bwd = time_backward(args, wl, p, pl, q, k, v, stream, peak_tf, b_off, h_off)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(wl, q_np, k_np, v_np, args.cpu_seconds)
 
+    per_config = None
+    if world == 1 and args.per_config:
+        per_config = {}
+        del hf, out_host
+        for name in [x for x in args.per_config.split(",") if x]:
+            per_config[name] = time_config(synth.WORKLOADS[name], args.per_config_steps,
+                                           peak_tf, stream)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": workload_config(wl, world),
+            "higher_is_better": True,
+            "scaling": "strong" if (args.partition == "heads" and world > 1) else "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(wl_full, world, parallelism_of(args.partition, world)),
             "plan_ms": plan_ms, "fwd_ms": fwd_ms, "fwd_exec_tflops": fwd_tflops,
             "nnz": nnz, "sparsity": 1.0 - nnz / (wl.B * wl.heads * wl.Nq * wl.Nc),
             "dense_equiv_tflops": 4.0 * wl.B * wl.heads * wl.Nq * 128 * wl.N * wl.d
@@ -469,10 +567,12 @@ def main():
             "dense": dense, "roofline": roofline, "cpu_baseline": cpu, "backward": bwd,
             "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "api": "HostForward (pinned host q, k, v -> out)",
+                    "api": "bsa_forward_host (C ABI, via HostForward; pinned host q, k, v "
+                           "-> out)",
                     "group": args.e2e_group, "streams": args.e2e_streams},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks, "device_status": bsa.status_string(rc),
+            "per_config": per_config,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -86,8 +86,8 @@ def make_params(B, heads, T, H, W, d, mode="topk", topk=1, cdf_p=0.9, cdf_cap_fr
 def params_for(wl) -> bsa_params:
     """Parameters of a workload description (anything with the Workload fields)."""
     return make_params(wl.B, wl.heads, wl.T, wl.H, wl.W, wl.d, wl.mode, wl.topk, wl.cdf_p,
-                       wl.cdf_cap_frac, wl.t_cond, q_begin=getattr(wl, "q_begin", 0),
-                       kchunk=getattr(wl, "kchunk", (0, 0, 0)))
+                       wl.cdf_cap_frac, wl.t_cond, scale=getattr(wl, "scale", 0.0),
+                       q_begin=getattr(wl, "q_begin", 0), kchunk=getattr(wl, "kchunk", (0, 0, 0)))
 
 
 _lib = None

@@ -170,15 +170,20 @@ int bsa_forward_host(const bsa_params* p, const void* q, const void* k, const vo
     const char* vh = static_cast<const char*>(v);
     char* oh = static_cast<char*>(out);
 
+    // A failure part way through stops queueing further groups, but the work
+    // already queued on the slot streams still runs: the caller's stream is
+    // made to wait for it on every return path after this point, so the host
+    // buffers are not written after the caller has synchronised `stream`.
+    int err = BSA_OK;
     int i = 0;
-    for (int64_t g0 = 0; g0 < g.BH; g0 += group, ++i) {
+    for (int64_t g0 = 0; g0 < g.BH && err == BSA_OK; g0 += group, ++i) {
         const int n = static_cast<int>(g.BH - g0 < group ? g.BH - g0 : group);
         const int s = i % slots;
         cudaStream_t st = static_cast<cudaStream_t>(streams[s]);
         char* slot = ws + L.slot0 + static_cast<size_t>(s) * L.slot_bytes;
         const bsa_params pg = group_params(*p, n);
         Dims gd;
-        if ((rc = make_dims(&pg, &gd)) != BSA_OK) return rc;
+        if ((err = make_dims(&pg, &gd)) != BSA_OK) break;
         const size_t src = static_cast<size_t>(g0) * pair_bytes;
         // Q of the computed frames, K and V whole (the candidates span every frame)
         if (cudaMemcpy2DAsync(slot + L.q + q_off, pair_bytes, qh + src + q_off, pair_bytes, q_len,
@@ -186,28 +191,37 @@ int bsa_forward_host(const bsa_params* p, const void* q, const void* k, const vo
             cudaMemcpyAsync(slot + L.k, kh + src, n * pair_bytes, cudaMemcpyHostToDevice, st) !=
                 cudaSuccess ||
             cudaMemcpyAsync(slot + L.v, vh + src, n * pair_bytes, cudaMemcpyHostToDevice, st) !=
-                cudaSuccess)
-            return BSA_ERR_CUDA;
+                cudaSuccess) {
+            err = BSA_ERR_CUDA;
+            break;
+        }
         int32_t* rp = reinterpret_cast<int32_t*>(slot + L.row_ptr);
         int32_t* ci = reinterpret_cast<int32_t*>(slot + L.col_idx);
         if (plan_group(gd, pg, slot + L.q, slot + L.k, slot + L.plan_ws, rp, ci, L.col_cap, status,
-                       st) != cudaSuccess)
-            return BSA_ERR_CUDA;
-        if (launch_forward(gd, slot + L.q, slot + L.k, slot + L.v, rp, ci, L.col_cap,
-                           slot + L.out, nullptr, status, kDefaultTimeoutNs, 0, st) != cudaSuccess)
-            return BSA_ERR_CUDA;
+                       st) != cudaSuccess ||
+            launch_forward(gd, slot + L.q, slot + L.k, slot + L.v, rp, ci, L.col_cap,
+                           slot + L.out, nullptr, status, kDefaultTimeoutNs, 0, st) !=
+                cudaSuccess) {
+            err = BSA_ERR_CUDA;
+            break;
+        }
         // the output of the computed frames; the others stay as the caller left them
         if (cudaMemcpy2DAsync(oh + src + q_off, pair_bytes, slot + L.out + q_off, pair_bytes, q_len,
-                              n, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-            return BSA_ERR_CUDA;
+                              n, cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+            err = BSA_ERR_CUDA;
+            break;
+        }
     }
-    // the caller's stream continues once every slot's last copy is done
+    // the caller's stream continues once every slot's last operation is done
     for (int s = 0; s < slots; ++s) {
         if (cudaEventRecord(events.ev[s], static_cast<cudaStream_t>(streams[s])) != cudaSuccess ||
-            cudaStreamWaitEvent(main_st, events.ev[s], 0) != cudaSuccess)
-            return BSA_ERR_CUDA;
+            cudaStreamWaitEvent(main_st, events.ev[s], 0) != cudaSuccess) {
+            // cannot order the caller's stream after this slot: wait for it here
+            (void)cudaStreamSynchronize(static_cast<cudaStream_t>(streams[s]));
+            if (err == BSA_OK) err = BSA_ERR_CUDA;
+        }
     }
-    return BSA_OK;
+    return err;
 }
 
 }  // extern "C"

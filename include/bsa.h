@@ -308,12 +308,16 @@ BSA_API int bsa_grad_finalize(const bsa_params* p, const float* acc, void* out, 
  * the device). The paper has no counterpart; this is an interface convenience.
  *   - Limit: 32 MiB of scratch (bsa_workspace_size(p) must not exceed it,
  *     about the 480p-like grid with 32 heads); larger plans return
- *     BSA_ERR_WORKSPACE_TOO_SMALL before any CUDA call. The array occupies
+ *     BSA_ERR_WORKSPACE_TOO_SMALL. All of bsa_plan's host checks (shape,
+ *     pointers, alignment, capacity, device) run before any CUDA call, with
+ *     bsa_plan's error codes. The array occupies
  *     32 MiB on every GPU that loads this library's device code, until exit.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
- *   - The first call on a device looks up the array's device address (once
- *     per device, with that device current); make that first call before any
- *     stream capture.
+ *   - Every call looks up the array's device address in the current context
+ *     (an address belongs to the context it was looked up in, and a caller may
+ *     switch contexts on one device). The first call in a context also loads
+ *     this library's device code into it; make that first call on each device
+ *     before any stream capture.
  *   - Every call reuses the same array, which keeps the previous call's
  *     contents; the call clears the part that must start at zero. Calls whose
  *     work overlaps on the GPU (e.g. on two streams without ordering) race on
@@ -346,6 +350,10 @@ BSA_API int bsa_plan_noalloc(const bsa_params* p, const void* q, const void* k, 
  * its first 256 bytes are the status block that bsa_read_status reads (zero
  * it before the first call). Device errors of every group land there.
  * Errors: INVALID_ARG, SHAPE, UNSUPPORTED, ALIGNMENT, WORKSPACE_TOO_SMALL, CUDA.
+ * A CUDA error part way through stops queueing further groups; `stream` still
+ * waits for whatever was already queued on the slot streams (or the call waits
+ * for it on the host), so after synchronising `stream` nothing writes the host
+ * buffers any more, also when the call returned an error.
  */
 BSA_API size_t bsa_forward_host_workspace_size(const bsa_params* p, int32_t group, int32_t slots);
 BSA_API int bsa_forward_host(const bsa_params* p, const void* q, const void* k, const void* v,

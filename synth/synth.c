@@ -106,27 +106,30 @@ static void make_components(component_t* cp, uint64_t seed, uint32_t tensor, uin
 
 /*
  * Fill out[B][heads][T][H][W][d] (bf16 bit patterns) for one tensor. Batch
- * element b uses stream batch index b + b_offset, so disjoint slices of a large
- * virtual batch can be generated independently (e.g. one per rank).
+ * element b uses stream batch index b + b_offset and head hd stream head index
+ * hd + h_offset, so disjoint slices of a large virtual problem (a range of batch
+ * elements, or a range of heads of one batch element) can be generated
+ * independently, e.g. one per rank.
  * tensor: 0 = Q, 1 = K, 2 = V (selects the stream; also any other id works).
  * rms_norm: 1 to RMS-normalise each token (Q, K), 0 for V.
  * Returns 0 on success, -1 on bad arguments.
  */
-int synth_field_bf16(uint16_t* out, int B, int b_offset, int heads, int T, int H, int W,
-                     int d, uint64_t seed, uint32_t tensor, int rms_norm, double tfreq_mult,
-                     int cond_frames, uint64_t cond_seed) {
-    if (!out || B <= 0 || b_offset < 0 || heads <= 0 || T <= 0 || H <= 0 || W <= 0 || d <= 0 || d > MAX_D ||
-        (d & 1))
+int synth_field_bf16_slice(uint16_t* out, int B, int b_offset, int heads, int h_offset, int T,
+                           int H, int W, int d, uint64_t seed, uint32_t tensor, int rms_norm,
+                           double tfreq_mult, int cond_frames, uint64_t cond_seed) {
+    if (!out || B <= 0 || b_offset < 0 || heads <= 0 || h_offset < 0 || T <= 0 || H <= 0 ||
+        W <= 0 || d <= 0 || d > MAX_D || (d & 1))
         return -1;
     const int64_t N = (int64_t)T * H * W;
     for (int b = 0; b < B; ++b) {
         for (int hd = 0; hd < heads; ++hd) {
             component_t comp_main[NCOMP], comp_cond[NCOMP];
             const uint32_t bs = (uint32_t)(b + b_offset);
-            make_components(comp_main, seed, tensor, bs, (uint32_t)hd, d, tfreq_mult);
-            make_components(comp_cond, cond_seed, tensor, bs, (uint32_t)hd, d, tfreq_mult);
-            const uint64_t nkey_main = stream_key(seed, tensor, bs, (uint32_t)hd, NOISE_COMPONENT);
-            const uint64_t nkey_cond = stream_key(cond_seed, tensor, bs, (uint32_t)hd, NOISE_COMPONENT);
+            const uint32_t hs = (uint32_t)(hd + h_offset);
+            make_components(comp_main, seed, tensor, bs, hs, d, tfreq_mult);
+            make_components(comp_cond, cond_seed, tensor, bs, hs, d, tfreq_mult);
+            const uint64_t nkey_main = stream_key(seed, tensor, bs, hs, NOISE_COMPONENT);
+            const uint64_t nkey_cond = stream_key(cond_seed, tensor, bs, hs, NOISE_COMPONENT);
             uint16_t* base = out + ((int64_t)b * heads + hd) * N * d;
 #pragma omp parallel for schedule(static)
             for (int64_t tok = 0; tok < N; ++tok) {
@@ -165,6 +168,14 @@ int synth_field_bf16(uint16_t* out, int B, int b_offset, int heads, int T, int H
         }
     }
     return 0;
+}
+
+/* The whole head range of batch elements [b_offset, b_offset + B). */
+int synth_field_bf16(uint16_t* out, int B, int b_offset, int heads, int T, int H, int W,
+                     int d, uint64_t seed, uint32_t tensor, int rms_norm, double tfreq_mult,
+                     int cond_frames, uint64_t cond_seed) {
+    return synth_field_bf16_slice(out, B, b_offset, heads, 0, T, H, W, d, seed, tensor, rms_norm,
+                                  tfreq_mult, cond_frames, cond_seed);
 }
 
 /* Raw access to the counter generator, for tests of the generator itself. */

@@ -27,9 +27,19 @@ class Workload:
     t_cond: int = 0             # latent frames of condition tokens (block-causal mask)
     q_begin: int = 0            # first latent frame whose queries are computed (KV-cached step)
     kchunk: tuple = (4, 4, 8)   # key chunk shape (multiples of the (4,4,8) query chunk)
+    scale: float = 0.0          # softmax scale; 0 = 1/sqrt(d)
     tfreq_mult: float = 1.0     # temporal frequency multiplier of the smooth field
     seed: int = 0
     cond_seed: int = 1
+
+    @property
+    def softmax_scale(self) -> float:
+        """The scale the library applies: the given one rounded to float, else
+        1/sqrt(d) (the library takes the scale as a float)."""
+        import numpy as np
+        if self.scale:
+            return float(np.float32(self.scale))
+        return 1.0 / self.d ** 0.5
 
     @property
     def N(self) -> int:

@@ -39,6 +39,10 @@ def test_reference_arm_prints_one_contract_line():
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert line["gpu_launches"] == 0
+    # the line says what ran: `steps` bounded samples of ms_per_step each, whose
+    # throughput is extrapolated to the full workload
+    assert line["extrapolated"] is True and line["est_full_step_s"] > 0
+    assert line["steps"] * line["ms_per_step"] / 1e3 <= line["wall_s"] + 1e-6
 
 
 def test_reference_arm_prints_on_rank_zero_only():

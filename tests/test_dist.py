@@ -1,8 +1,9 @@
-"""Multi-rank host logic on CPU (gloo, world size 2).
+"""Multi-rank host logic on CPU (gloo, world size 2 and 3).
 
-The operator shards with no exchange: each rank runs its own problem (its own
-batch element) and only the timing is reduced over ranks. The ranks here run
-the CPU oracle as a stand-in for their GPU step, so this needs no GPU.
+The operator shards with no exchange. By default the heads of the one call are
+split across the ranks; with replicas each rank runs its own problem (its own
+batch element). Only the timing is reduced over ranks. The ranks here run the
+CPU oracle as a stand-in for their GPU step, so this needs no GPU.
 """
 import math
 import os
@@ -66,3 +67,58 @@ def test_two_ranks_shard_independent_problems(tmp_path):
     for i in range(world):
         np.testing.assert_array_equal(r[i]["q"][0], q2[i])
         np.testing.assert_array_equal(r[i]["out"], out2[i * per_rank:(i + 1) * per_rank])
+
+
+def _head_worker(rank, world, port, result_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=timedelta(seconds=60))
+    try:
+        full = synth.WORKLOADS["tiny"].with_(heads=5, T=8, mode="cdf", t_cond=4)
+        wl, b_off, h_off = bench.rank_problem(full, rank, world, "heads")
+        q, k, v = synth.make_qkv(wl, batch_offset=b_off, head_offset=h_off)
+        scale = 1 / math.sqrt(wl.d)
+        rp, ci, _ = oracle.plan(q, k, wl.T, wl.H, wl.W, scale, wl.mode, wl.topk, wl.cdf_p,
+                                wl.cdf_cap_frac, wl.t_cond)
+        out, lse = oracle.attend(q, k, v, wl.T, wl.H, wl.W, scale, rp, ci, np.arange(wl.rows))
+        # gather every rank's heads (the caller's optional all-gather of O over heads)
+        parts = [None] * world
+        dist.all_gather_object(parts, (h_off, out, lse))
+        np.savez(os.path.join(result_dir, f"h{rank}.npz"),
+                 offsets=np.array([p[0] for p in parts]),
+                 out=np.concatenate([p[1] for p in sorted(parts, key=lambda x: x[0])]),
+                 lse=np.concatenate([p[2] for p in sorted(parts, key=lambda x: x[0])]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world", [2, 3])
+def test_head_split_shards_concatenate_to_the_unsplit_call(tmp_path, world):
+    """5 heads over 2 or 3 ranks (uneven shards): every rank draws exactly its
+    heads of the one problem, and the shards' outputs, in head order, equal the
+    oracle's output of the unsplit call."""
+    mp.start_processes(_head_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       start_method="spawn", join=True)
+    full = synth.WORKLOADS["tiny"].with_(heads=5, T=8, mode="cdf", t_cond=4)
+    q, k, v = synth.make_qkv(full)
+    scale = 1 / math.sqrt(full.d)
+    rp, ci, _ = oracle.plan(q, k, full.T, full.H, full.W, scale, full.mode, full.topk,
+                            full.cdf_p, full.cdf_cap_frac, full.t_cond)
+    out, lse = oracle.attend(q, k, v, full.T, full.H, full.W, scale, rp, ci,
+                             np.arange(full.rows))
+    for r in range(world):
+        got = np.load(tmp_path / f"h{r}.npz")
+        assert list(got["offsets"]) == [bench.shard_heads(i, world, 5)[0] for i in range(world)]
+        np.testing.assert_array_equal(got["out"], out)
+        np.testing.assert_array_equal(got["lse"], lse)
+
+
+def test_shard_heads_covers_every_head_once():
+    for heads in (1, 5, 32):
+        for world in range(1, heads + 1):
+            spans = [bench.shard_heads(r, world, heads) for r in range(world)]
+            assert spans[0][0] == 0 and all(n >= 1 for _, n in spans)
+            assert all(spans[i][0] + spans[i][1] == spans[i + 1][0] for i in range(world - 1))
+            assert spans[-1][0] + spans[-1][1] == heads
+            assert max(n for _, n in spans) - min(n for _, n in spans) <= 1

@@ -70,7 +70,7 @@ def gpu_fwd_bwd(wl, q, k, v, g, csr=None, sentinel=None):
 def check_bwd(wl, csr=None):
     q, k, v = synth.make_qkv(wl)
     g = synth.make_dout(wl)
-    scale = 1.0 / math.sqrt(wl.d)
+    scale = wl.softmax_scale
     rp, ci, out, lse, dq, dk, dv, st_f, st_b = gpu_fwd_bwd(wl, q, k, v, g, csr)
     assert st_f == bsa.BSA_OK and st_b == bsa.BSA_OK, (st_f, st_b)
     rows = np.arange(wl.rows)

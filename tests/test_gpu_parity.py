@@ -55,6 +55,13 @@ SMALL = {
     "causal_topk_cdf": W["tiny"].with_(name="causal_topk_cdf", B=2, heads=2, T=16, H=16, W=32,
                                        d=64, mode="topk_cdf", topk=5, cdf_p=0.2,
                                        cdf_cap_frac=0.25, t_cond=8),
+    # a softmax scale other than 1/sqrt(d): sharper (CDF counts and the attention's
+    # softmax both change) and flatter than the default
+    "scale_sharp_cdf": W["tiny"].with_(name="scale_sharp_cdf", B=2, heads=2, T=16, H=16, W=32,
+                                       d=128, mode="cdf", cdf_p=0.9, cdf_cap_frac=0.25,
+                                       t_cond=8, scale=0.3),
+    "scale_flat_topk": W["tiny"].with_(name="scale_flat_topk", heads=2, T=8, H=16, W=32, d=64,
+                                       topk=5, scale=0.02),
 }
 
 
@@ -112,7 +119,7 @@ def boxes_to_key_chunks(rp, ci, wl):
 
 def check_case(wl, rows=None, qkv=None):
     q, k, v = synth.make_qkv(wl) if qkv is None else qkv
-    scale = 1.0 / math.sqrt(wl.d)
+    scale = wl.softmax_scale
     rp, ci, out, lse, status = run_gpu(wl, q, k, v)
     assert status == bsa.BSA_OK, bsa.status_string(status)
     kchunk = tuple(wl.kchunk)
@@ -199,7 +206,7 @@ def test_kv_cached_step_equals_rows_of_the_full_computation(case):
     rp = pl.row_ptr.cpu().numpy()
     ci = pl.col_idx[: int(rp[-1])].cpu().numpy()
     assert len(rp) == wl.rows + 1
-    scale = 1.0 / math.sqrt(wl.d)
+    scale = wl.softmax_scale
     o_rp, o_ci, _ = oracle.plan(q, k, wl.T, wl.H, wl.W, scale, wl.mode, wl.topk, wl.cdf_p,
                                 wl.cdf_cap_frac, wl.t_cond, fp32=True)
     # place the GPU's rows at their positions in the full plan (the oracle's rows elsewhere)
@@ -333,6 +340,35 @@ def test_bounded_wait_selftest_reports_timeout():
     check_case(SMALL["tiny"])  # the context is still usable
 
 
+def test_forward_kernel_abort_path_reports_timeout():
+    """The forward kernel's own bounded waits: with debug flag 0 the MMA warp
+    withholds the first S-ready signal of tile 0, so that tile's softmax warps
+    (and then every role) wait until the 20 ms limit, record the timeout, drain
+    their copies and products, free TMEM and return. The status must say
+    DEVICE_TIMEOUT, and the next calls must work."""
+    wl = SMALL["tiny"]
+    q, k, v = synth.make_qkv(wl)
+    p = bsa.params_for(wl)
+    pl = bsa.allocate(p)
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    bsa.bsa_plan(p, qd, kd, pl.workspace, pl.row_ptr, pl.col_idx)
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_OK
+    out = torch.zeros_like(qd)
+    bsa.bsa_forward_ex(p, qd, kd, vd, pl.row_ptr, pl.col_idx, pl.workspace, out,
+                       timeout_ns=20_000_000, debug_flags=1)
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_ERR_DEVICE_TIMEOUT
+    # the same buffers give the right result on the next call, and so does a fresh case
+    bsa.bsa_forward(p, qd, kd, vd, pl.row_ptr, pl.col_idx, pl.workspace, out)
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_OK
+    rp = pl.row_ptr.cpu().numpy()
+    ci = pl.col_idx[: int(rp[-1])].cpu().numpy()
+    rows = np.arange(wl.rows)
+    o_out, _ = oracle.attend(q, k, v, wl.T, wl.H, wl.W, wl.softmax_scale, rp, ci, rows)
+    mx, mean = compare_attention(gather_rows(host_f32(out), wl, rows), o_out)
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+    check_case(SMALL["causal_cdf_small"])
+
+
 # ------------------------------------------------------------------ full-size workloads
 
 def _sample_rows(wl, per_head, seed=0):
@@ -343,10 +379,19 @@ def _sample_rows(wl, per_head, seed=0):
     return np.array(sorted(rows), dtype=np.int64)
 
 
-@pytest.mark.parametrize("name,per_head", [("480p", 224), ("720p", 64), ("long", 2),
-                                           ("causal_cdf", 2), ("720p_r8", 2),
-                                           ("720p_topk_cdf", 2), ("720p_real", 4),
+@pytest.mark.parametrize("name,per_head", [("480p", 224), ("720p", 64), ("long", 16),
+                                           ("causal_cdf", 16), ("720p_r8", 4),
+                                           ("720p_topk_cdf", 4), ("720p_real", 4),
                                            ("480p_real", 4), ("720p_k512", 4)])
 def test_full_size_workloads(name, per_head):
     wl = W[name]
     check_case(wl, rows=_sample_rows(wl, per_head))
+
+
+def test_grid_of_1920_chunks():
+    """A grid near the library's limit of 2,048 chunks per (batch, head):
+    64 x 48 x 80 latent tokens, 1,920 chunks, k = 120 (93.75 % sparse). Its
+    rows take the selector's widest instantiation (64 keys per lane)."""
+    wl = W["720p"].with_(name="grid1920", heads=1, T=64, topk=120)
+    assert 1792 < wl.Nc <= 2048
+    check_case(wl, rows=_sample_rows(wl, 32))

@@ -56,6 +56,30 @@ def test_plan_noalloc_matches_plan_on_two_calls_in_a_row():
 
 
 @pytest.mark.gpu
+def test_plan_noalloc_allocates_no_device_memory():
+    """A warm call changes neither the device's free memory nor torch's
+    allocator: the scratch is the library's fixed array, nothing else."""
+    wl = W["tiny"].with_(heads=2, T=16, H=16, W=32, d=128, topk=5)
+    q, k, _ = synth.make_qkv(wl)
+    qd, kd = _dev(q), _dev(k)
+    p = bsa.params_for(wl)
+    rows, nnz = bsa.bsa_plan_sizes(p)
+    row_ptr = torch.empty((rows + 1,), dtype=torch.int32, device="cuda")
+    col_idx = torch.empty((max(nnz, 1),), dtype=torch.int32, device="cuda")
+    bsa.bsa_plan_noalloc(p, qd, kd, row_ptr, col_idx)   # first call in this context
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0, reserved0 = torch.cuda.memory_allocated(), torch.cuda.memory_reserved()
+    for _ in range(3):
+        bsa.bsa_plan_noalloc(p, qd, kd, row_ptr, col_idx)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert torch.cuda.memory_allocated() == alloc0
+    assert torch.cuda.memory_reserved() == reserved0
+
+
+@pytest.mark.gpu
 def test_plan_noalloc_rejects_plans_beyond_its_scratch():
     p = bsa.params_for(W["720p"])  # needs ~90 MB of scratch > 32 MiB
     assert bsa.bsa_workspace_size(p) > (32 << 20)
