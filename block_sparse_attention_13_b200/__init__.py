@@ -41,7 +41,8 @@ EXPORTED = ("bsa_version", "bsa_status_string", "bsa_workspace_size", "bsa_plan_
             "bsa_selftest_timeout", "bsa_backward_workspace_size", "bsa_backward",
             "bsa_select_pooled", "bsa_csr_slice_workspace_size", "bsa_csr_slice",
             "bsa_lse_merge", "bsa_grad_accumulate", "bsa_grad_finalize", "bsa_shape_info",
-            "bsa_forward_host_workspace_size", "bsa_forward_host")
+            "bsa_forward_host_workspace_size", "bsa_forward_host", "bsa_forward_partial",
+            "bsa_lse_merge_f32")
 
 # Scratch array of bsa_plan_noalloc inside the library (include/bsa.h: 32 MiB);
 # a plan whose workspace exceeds it is rejected by the library before any CUDA call.
@@ -128,6 +129,8 @@ def lib():
             "bsa_csr_slice_workspace_size": (sz, [i64]),
             "bsa_csr_slice": (i32, [i64, vp, vp, i64, i32, i32, vp, sz, vp, vp, i64, vp]),
             "bsa_lse_merge": (i32, [P, vp, vp, vp, vp, vp]),
+            "bsa_lse_merge_f32": (i32, [P, vp, vp, vp, vp, vp]),
+            "bsa_forward_partial": (i32, [P, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, vp]),
             "bsa_grad_accumulate": (i32, [P, vp, vp, i32, vp]),
             "bsa_grad_finalize": (i32, [P, vp, vp, vp]),
             "bsa_backward": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, vp,
@@ -289,6 +292,23 @@ def bsa_forward_ex(p, q, k, v, row_ptr, col_idx, workspace, out, lse=None, timeo
            "bsa_forward_ex")
 
 
+def bsa_forward_partial(p, q, k, v, row_ptr, col_idx, workspace, out_f32, lse, stream=None):
+    """bsa_forward with an fp32 output (a partial result to merge by LSE)."""
+    bf, f32, i32 = _dtypes()
+    s = bsa_shape_info(p)
+    x = s.BH * s.N * s.d
+    _tensors("bsa_forward_partial", ("q", q, bf, x), ("k", k, bf, x), ("v", v, bf, x),
+             ("out_f32", out_f32, f32, x), ("lse", lse, f32, s.BH * s.N),
+             ("row_ptr", row_ptr, i32, s.rows + 1), ("col_idx", col_idx, i32, 0),
+             ("workspace", workspace, None, 0))
+    if out_f32 is None or lse is None:
+        raise BsaError(BSA_ERR_INVALID_ARG, "bsa_forward_partial: out_f32 and lse are required")
+    _check(lib().bsa_forward_partial(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
+                                     _ptr(col_idx), col_idx.numel(), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _ptr(out_f32),
+                                     _ptr(lse), _stream(stream)), "bsa_forward_partial")
+
+
 def bsa_backward_workspace_size(p: bsa_params) -> int:
     n = lib().bsa_backward_workspace_size(ctypes.byref(p))
     if n == 0:
@@ -373,6 +393,16 @@ def bsa_lse_merge(p, out, lse, out_part, lse_part, stream=None):
              ("out_part", out_part, bf, x), ("lse_part", lse_part, f32, s.BH * s.N))
     _check(lib().bsa_lse_merge(ctypes.byref(p), _ptr(out), _ptr(lse), _ptr(out_part),
                                _ptr(lse_part), _stream(stream)), "bsa_lse_merge")
+
+
+def bsa_lse_merge_f32(p, out, lse, out_part, lse_part, stream=None):
+    _, f32, _ = _dtypes()
+    s = bsa_shape_info(p)
+    x = s.BH * s.N * s.d
+    _tensors("bsa_lse_merge_f32", ("out", out, f32, x), ("lse", lse, f32, s.BH * s.N),
+             ("out_part", out_part, f32, x), ("lse_part", lse_part, f32, s.BH * s.N))
+    _check(lib().bsa_lse_merge_f32(ctypes.byref(p), _ptr(out), _ptr(lse), _ptr(out_part),
+                                   _ptr(lse_part), _stream(stream)), "bsa_lse_merge_f32")
 
 
 def bsa_grad_accumulate(p, part, acc, overwrite=False, stream=None):

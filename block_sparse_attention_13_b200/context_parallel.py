@@ -7,7 +7,8 @@ keys of all ranks are gathered, each rank scores its query chunks against all
 of them and keeps the top-k (or CDF) key chunks, and the attention is then
 computed shard by shard while the K/V shards travel around the ring, the
 partial results being combined by their log-sum-exps ("LongCat-Video
-Technical Report #", section "开源实现": LSE and output correction).
+Technical Report #", section "开源实现": LSE and output correction). The
+partial outputs stay in fp32 through the merges and are rounded to bf16 once.
 
 The backward (``ring_backward``) runs the same ring again. At each step a rank
 computes, with bsa_backward, the contributions of the K/V shard it holds to
@@ -21,7 +22,8 @@ On one node of B200s the gather is an NCCL all-gather of the pooled keys
 (Nc x d floats per head and rank) and the ring step an NCCL send/receive of
 the next K/V shard, posted before the current shard's attention so that the
 transfer overlaps it. Every computation runs in the library's kernels
-(bsa_pool, bsa_select_pooled, bsa_csr_slice, bsa_forward, bsa_lse_merge);
+(bsa_pool, bsa_select_pooled, bsa_csr_slice, bsa_forward_partial,
+bsa_lse_merge_f32, bsa_grad_finalize);
 torch.distributed only moves data.
 """
 from __future__ import annotations
@@ -30,9 +32,9 @@ import torch
 import torch.distributed as dist
 
 from . import (BSA_OK, BsaError, backward_workspace, bsa_backward, bsa_csr_slice,
-               bsa_csr_slice_workspace_size, bsa_forward, bsa_grad_accumulate, bsa_grad_finalize,
-               bsa_lse_merge, bsa_plan_sizes, bsa_pool, bsa_read_status, bsa_select_pooled,
-               bsa_workspace_size, make_params, status_string)
+               bsa_csr_slice_workspace_size, bsa_forward_partial, bsa_grad_accumulate,
+               bsa_grad_finalize, bsa_lse_merge_f32, bsa_plan_sizes, bsa_pool, bsa_read_status,
+               bsa_select_pooled, bsa_workspace_size, make_params, status_string)
 
 
 class CudaOps:
@@ -69,16 +71,18 @@ class CudaOps:
         return out_rp, out_ci
 
     def forward(self, p, q, k, v, row_ptr, col_idx):
+        """Partial attention over one K/V shard: fp32 output and LSE."""
         ws = torch.zeros(256, dtype=torch.uint8, device=q.device)
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
         B, heads, N, _ = q.shape
         lse = torch.empty((B, heads, N), dtype=torch.float32, device=q.device)
-        bsa_forward(p, q, k, v, row_ptr, col_idx, ws, out, lse)
+        bsa_forward_partial(p, q, k, v, row_ptr, col_idx, ws, out, lse)
         self._status.append(ws)
         return out, lse
 
     def merge(self, p, out, lse, out_part, lse_part):
-        bsa_lse_merge(p, out, lse, out_part, lse_part)
+        """fp32 accumulator <- LSE merge with an fp32 partial result."""
+        bsa_lse_merge_f32(p, out, lse, out_part, lse_part)
 
     def backward(self, p, q, k, v, out, lse, dout, row_ptr, col_idx):
         ws = backward_workspace(p, q.device)
@@ -196,6 +200,8 @@ def ring_forward(q, k, v, grid, topk=None, mode="topk", cdf_p=0.9, cdf_cap_frac=
             ops.merge(p_local, out, lse, o_part, l_part)
         if handle is not None:
             k_cur, v_cur = comm.finish_shift(handle)
+    # the partial results were merged in fp32; round once, as the unsplit call does
+    out = ops.finalize(p_local, out)
     ops.check()
     if return_csr:
         return out, lse, row_ptr, col_idx

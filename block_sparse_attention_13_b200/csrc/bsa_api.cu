@@ -293,6 +293,28 @@ int bsa_forward_ex(const bsa_params* p, const void* q, const void* k, const void
                                       static_cast<cudaStream_t>(stream)));
 }
 
+int bsa_forward_partial(const bsa_params* p, const void* q, const void* k, const void* v,
+                        const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
+                        void* workspace, size_t ws_bytes, float* out_f32, float* lse,
+                        void* stream) {
+    TraceRange trace("bsa_forward_partial");
+    Dims g;
+    int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!q || !k || !v || !row_ptr || !col_idx || !workspace || !out_f32 || !lse ||
+        col_capacity < 0)
+        return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out_f32) ||
+        !aligned16(workspace) || !aligned4(lse) || !aligned4(row_ptr) || !aligned4(col_idx))
+        return BSA_ERR_ALIGNMENT;
+    if (ws_bytes < 256) return BSA_ERR_WORKSPACE_TOO_SMALL;
+    if ((rc = device_ok()) != BSA_OK) return rc;
+    uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace));
+    return cuda_status(launch_forward(g, q, k, v, row_ptr, col_idx, col_capacity, nullptr, lse,
+                                      status, kDefaultTimeoutNs, 0,
+                                      static_cast<cudaStream_t>(stream), out_f32));
+}
+
 int bsa_forward(const bsa_params* p, const void* q, const void* k, const void* v,
                 const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
                 void* workspace, size_t ws_bytes, void* out, float* lse, void* stream) {
@@ -402,6 +424,20 @@ int bsa_lse_merge(const bsa_params* p, void* out, float* lse, const void* out_pa
     if ((rc = device_ok()) != BSA_OK) return rc;
     return cuda_status(launch_lse_merge(g, out, lse, out_part, lse_part,
                                         static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_lse_merge_f32(const bsa_params* p, float* out, float* lse, const float* out_part,
+                      const float* lse_part, void* stream) {
+    TraceRange trace("bsa_lse_merge_f32");
+    Dims g;
+    int rc = make_dims(p, &g);
+    if (rc != BSA_OK) return rc;
+    if (!out || !lse || !out_part || !lse_part) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(out_part) || !aligned4(lse) || !aligned4(lse_part))
+        return BSA_ERR_ALIGNMENT;
+    if ((rc = device_ok()) != BSA_OK) return rc;
+    return cuda_status(launch_lse_merge_f32(g, out, lse, out_part, lse_part,
+                                            static_cast<cudaStream_t>(stream)));
 }
 
 int bsa_grad_accumulate(const bsa_params* p, const void* part, float* acc, int overwrite,

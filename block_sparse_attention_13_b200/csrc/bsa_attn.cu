@@ -81,6 +81,7 @@ struct FwdArgs {
     const int32_t* col_idx;
     int64_t col_cap;
     __nv_bfloat16* out;
+    float* out_f32;    // non-null: O is written here in fp32 instead of bf16 to `out`
     float* lse;
     uint32_t* status;
     int T, H, W, NH, NW, Nc;
@@ -461,7 +462,30 @@ __global__ void __launch_bounds__(320, 1)
             const bool q_exists = q_t + lt < a.T && q_h + lh < a.H && q_w + lw < a.W;
             const int64_t tok =
                 (static_cast<int64_t>(q_t + lt) * a.H + (q_h + lh)) * a.W + q_w + lw;
-            if (all_ok && n_t > 0) {
+            if (all_ok && n_t > 0 && a.out_f32) {
+                // fp32 output (a partial result that is merged later): each thread
+                // stores its own row, 128-bit stores; tcgen05.ld is warp-collective,
+                // so every lane loads and only existing query slots store
+                tc_fence_after();
+                const float inv_l = 1.0f / l_run;
+                float4* dst = reinterpret_cast<float4*>(a.out_f32 + (bh * a.N + tok) * D);
+#pragma unroll
+                for (int g = 0; g < D / 32; ++g) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + g * 32, o);
+                    tmem_wait_ld_tie(o);
+                    if (q_exists) {
+#pragma unroll
+                        for (int c4 = 0; c4 < 8; ++c4)
+                            dst[g * 8 + c4] = make_float4(__uint_as_float(o[c4 * 4 + 0]) * inv_l,
+                                                          __uint_as_float(o[c4 * 4 + 1]) * inv_l,
+                                                          __uint_as_float(o[c4 * 4 + 2]) * inv_l,
+                                                          __uint_as_float(o[c4 * 4 + 3]) * inv_l);
+                    }
+                }
+                if (a.lse && q_exists)
+                    a.lse[bh * a.N + tok] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+            } else if (all_ok && n_t > 0) {
                 tc_fence_after();
                 const float inv_l = 1.0f / l_run;
                 uint8_t* stage = smem + C::q_off(t);  // Q of this tile is dead once O is final
@@ -498,9 +522,15 @@ __global__ void __launch_bounds__(320, 1)
             } else if (all_ok && q_exists) {
                 // empty (or rejected) row: zeros, lse = -inf
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-                uint4* dst = reinterpret_cast<uint4*>(a.out + (bh * a.N + tok) * D);
+                if (a.out_f32) {
+                    uint4* dst = reinterpret_cast<uint4*>(a.out_f32 + (bh * a.N + tok) * D);
 #pragma unroll
-                for (int j = 0; j < D / 8; ++j) dst[j] = z;
+                    for (int j = 0; j < D / 4; ++j) dst[j] = z;
+                } else {
+                    uint4* dst = reinterpret_cast<uint4*>(a.out + (bh * a.N + tok) * D);
+#pragma unroll
+                    for (int j = 0; j < D / 8; ++j) dst[j] = z;
+                }
                 if (a.lse) a.lse[bh * a.N + tok] = -INFINITY;
             }
         }
@@ -605,16 +635,19 @@ cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, i
 cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const void* v,
                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
                            void* out, float* lse, uint32_t* status, uint64_t timeout_ns,
-                           int debug_flags, cudaStream_t st) {
+                           int debug_flags, cudaStream_t st, float* out_f32) {
+    if (!out && !out_f32) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv, mo;
+    // with an fp32 output the bf16 output map is never used (built over q)
     if (!make_chunk_map(&mq, q, g) || !make_chunk_map(&mk, k, g) || !make_chunk_map(&mv, v, g) ||
-        !make_chunk_map(&mo, out, g))
+        !make_chunk_map(&mo, out_f32 ? q : out, g))
         return cudaErrorInvalidValue;
     FwdArgs args;
     args.row_ptr = row_ptr;
     args.col_idx = col_idx;
     args.col_cap = col_cap;
     args.out = static_cast<__nv_bfloat16*>(out);
+    args.out_f32 = out_f32;
     args.lse = lse;
     args.status = status;
     args.T = g.T;

@@ -118,6 +118,45 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(__nv_bfloat16* __restric
     if (v % VPT == 0) lse[tok] = l;
 }
 
+// The same merge with an fp32 accumulator and an fp32 partial result (4
+// elements per thread): the partial outputs are rounded only once, when the
+// merged result is finally converted to bf16.
+template <int D>
+__global__ void __launch_bounds__(256) lse_merge_f32_kernel(float* __restrict__ out,
+                                                            float* __restrict__ lse,
+                                                            const float* __restrict__ part,
+                                                            const float* __restrict__ lse_part,
+                                                            int64_t tokens) {
+    constexpr int VPT = D / 4;
+    const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool valid = v < tokens * VPT;
+    const int64_t tok = valid ? v / VPT : 0;
+    const float a = valid ? lse[tok] : 0.f, b = valid ? lse_part[tok] : -INFINITY;
+    // every lane of a token (VPT consecutive lanes of one warp) has read lse[tok]
+    // before its first lane overwrites it
+    __syncwarp();
+    if (!valid || b == -INFINITY) return;
+    float4* po = reinterpret_cast<float4*>(out) + v;
+    const float4 y = reinterpret_cast<const float4*>(part)[v];
+    float l;
+    float4 r;
+    if (a == -INFINITY) {
+        r = y;
+        l = b;
+    } else {
+        const float m = fmaxf(a, b);
+        const float ea = __expf(a - m), eb = __expf(b - m);
+        const float inv = 1.0f / (ea + eb);
+        const float wa = ea * inv, wb = eb * inv;
+        l = m + __logf(ea + eb);
+        const float4 x = *po;
+        r = make_float4(fmaf(wa, x.x, wb * y.x), fmaf(wa, x.y, wb * y.y), fmaf(wa, x.z, wb * y.z),
+                        fmaf(wa, x.w, wb * y.w));
+    }
+    *po = r;
+    if (v % VPT == 0) lse[tok] = l;
+}
+
 // acc (fp32) = part (bf16), or acc += part; 8 elements per thread and step.
 __global__ void __launch_bounds__(256) grad_accumulate_kernel(const uint4* __restrict__ part,
                                                               float4* __restrict__ acc,
@@ -209,6 +248,18 @@ cudaError_t launch_lse_merge(const Dims& g, void* out, float* lse, const void* o
         lse_merge_kernel<128><<<blocks, 256, 0, st>>>(o, lse, p, lse_part, tokens);
     else
         lse_merge_kernel<64><<<blocks, 256, 0, st>>>(o, lse, p, lse_part, tokens);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lse_merge_f32(const Dims& g, float* out, float* lse, const float* out_part,
+                                 const float* lse_part, cudaStream_t st) {
+    const int64_t tokens = g.BH * g.N;
+    const int64_t vecs = tokens * (g.d / 4);
+    const unsigned blocks = static_cast<unsigned>((vecs + 255) / 256);
+    if (g.d == 128)
+        lse_merge_f32_kernel<128><<<blocks, 256, 0, st>>>(out, lse, out_part, lse_part, tokens);
+    else
+        lse_merge_f32_kernel<64><<<blocks, 256, 0, st>>>(out, lse, out_part, lse_part, tokens);
     return cudaGetLastError();
 }
 

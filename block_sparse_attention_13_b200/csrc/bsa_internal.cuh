@@ -122,10 +122,11 @@ cudaError_t launch_scores(const Dims& g, const float* qp, const float* kp, float
 cudaError_t launch_select(const Dims& g, const bsa_params& p, const float* S, int32_t* row_ptr,
                           int32_t* col_idx, int64_t col_cap, int32_t* counts, int32_t* padded,
                           int pad_stride, uint32_t* status, cudaStream_t st);
+// out_f32 non-null: O is written there in fp32 (and `out` is not used).
 cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const void* v,
                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
                            void* out, float* lse, uint32_t* status, uint64_t timeout_ns,
-                           int debug_flags, cudaStream_t st);
+                           int debug_flags, cudaStream_t st, float* out_f32 = nullptr);
 // 5-D TMA map over a [BH][T][H][W][d] bf16 tensor whose box is one (4,4,8)
 // chunk x 64 channels (128-byte swizzle); box_t = 2 gives half a chunk (its
 // first or last two frames: local tokens 0-63 or 64-127). False if the driver
@@ -151,6 +152,9 @@ cudaError_t launch_csr_slice(int64_t rows, const int32_t* row_ptr, const int32_t
                              cudaStream_t st);
 cudaError_t launch_lse_merge(const Dims& g, void* out, float* lse, const void* out_part,
                              const float* lse_part, cudaStream_t st);
+// The same merge with fp32 accumulator and fp32 partial result.
+cudaError_t launch_lse_merge_f32(const Dims& g, float* out, float* lse, const float* out_part,
+                                 const float* lse_part, cudaStream_t st);
 cudaError_t launch_grad_accumulate(int64_t n, const void* part, float* acc, int overwrite,
                                    cudaStream_t st);
 cudaError_t launch_grad_finalize(int64_t n, const float* acc, void* out, cudaStream_t st);

@@ -189,6 +189,21 @@ BSA_API int bsa_forward(const bsa_params* p, const void* q, const void* k, const
                 void* workspace, size_t ws_bytes, void* out, float* lse, void* stream);
 
 /*
+ * bsa_forward with the output kept in fp32: a partial result over one
+ * partition of the keys, to be merged with the others by log-sum-exp
+ * (bsa_lse_merge_f32) and rounded to bf16 only once at the end ([P1] ring
+ * block sparse attention; [P3] "开源实现": LSE and output correction). Same
+ * computation, arguments and errors as bsa_forward except: out_f32: device
+ * fp32 [B,heads,N,d], 16-byte aligned, written in [T,H,W] token order
+ * (normalised by the partition's own softmax sum; zeros for an empty row);
+ * lse: required.
+ */
+BSA_API int bsa_forward_partial(const bsa_params* p, const void* q, const void* k, const void* v,
+                                const int32_t* row_ptr, const int32_t* col_idx,
+                                int64_t col_capacity, void* workspace, size_t ws_bytes,
+                                float* out_f32, float* lse, void* stream);
+
+/*
  * Bytes of device workspace that bsa_backward needs for `p` (0 if `p` is
  * invalid): a status block, LSE and <dO,O> per computed query token, and the
  * column-major (CSC) copy of a block mask of at most one entry per (row, key
@@ -276,6 +291,15 @@ BSA_API int bsa_lse_merge(const bsa_params* p, void* out, float* lse, const void
                           const float* lse_part, void* stream);
 
 /*
+ * bsa_lse_merge with out and out_part in fp32 (device fp32 [B,heads,N,d],
+ * 16-byte aligned), as bsa_forward_partial writes them: the merged result is
+ * rounded once, by bsa_grad_finalize, after the last partition. Errors as for
+ * bsa_lse_merge.
+ */
+BSA_API int bsa_lse_merge_f32(const bsa_params* p, float* out, float* lse, const float* out_part,
+                              const float* lse_part, void* stream);
+
+/*
  * Backward of the ring ([P1] ring block sparse attention; [P3] "开源实现":
  * the trainable BSA's backward kernels and the LSE correction for context
  * parallelism). bsa_backward over one K/V shard, given the merged output and
@@ -293,7 +317,8 @@ BSA_API int bsa_grad_accumulate(const bsa_params* p, const void* part, float* ac
                                 void* stream);
 
 /*
- * out <- acc rounded to bf16 (nearest even), for the grid `p` describes.
+ * out <- acc rounded to bf16 (nearest even), for the grid `p` describes (the
+ * last step of the ring's fp32 gradients, and of its fp32 merged output).
  * acc: device fp32 [B,heads,N,d]; out: device bf16 of the same shape. Both
  * 16-byte aligned. Errors: INVALID_ARG, SHAPE, UNSUPPORTED, ALIGNMENT, CUDA.
  */

@@ -310,6 +310,21 @@ def test_context_parallel_entries_host_checks(L):
     assert L.bsa_lse_merge(ctypes.byref(p), x, None, x, x, None) == bsa.BSA_ERR_INVALID_ARG
     assert L.bsa_lse_merge(ctypes.byref(p), x, vp(FAKE + 2), x, x, None) == \
         bsa.BSA_ERR_ALIGNMENT
+    # the fp32 merge and the fp32-output forward of the ring's partial results
+    m32 = L.bsa_lse_merge_f32
+    assert m32(ctypes.byref(p), x, x, None, x, None) == bsa.BSA_ERR_INVALID_ARG
+    assert m32(ctypes.byref(p), vp(FAKE + 8), x, x, x, None) == bsa.BSA_ERR_ALIGNMENT
+    assert m32(ctypes.byref(p), x, x, x, vp(FAKE + 2), None) == bsa.BSA_ERR_ALIGNMENT
+    assert m32(ctypes.byref(P(W=0)), x, x, x, x, None) == bsa.BSA_ERR_SHAPE
+    fp = L.bsa_forward_partial
+    assert fp(ctypes.byref(p), x, x, x, x, x, 16, x, 256, None, x, None) == \
+        bsa.BSA_ERR_INVALID_ARG                                   # out_f32 required
+    assert fp(ctypes.byref(p), x, x, x, x, x, 16, x, 256, x, None, None) == \
+        bsa.BSA_ERR_INVALID_ARG                                   # lse required
+    assert fp(ctypes.byref(p), x, x, x, x, x, 16, x, 256, vp(FAKE + 4), x, None) == \
+        bsa.BSA_ERR_ALIGNMENT
+    assert fp(ctypes.byref(p), x, x, x, x, x, 16, x, 255, x, x, None) == \
+        bsa.BSA_ERR_WORKSPACE_TOO_SMALL
     # select from pooled inputs: kshard must divide the key chunks
     pr = P(T=16, H=8, W=16, q_begin=4, q_end=8)
     wsz = bsa.bsa_workspace_size(pr)

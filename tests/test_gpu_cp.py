@@ -103,15 +103,18 @@ def test_ring_forward_equals_unsplit(name):
                 row = bh * nc_l + i
                 grow = bh * wl.Nc + r * nc_l + i
                 assert np.array_equal(ci[rp[row]:rp[row + 1]], g_ci[g_rp[grow]:g_rp[grow + 1]])
-        # attention: the unsplit result for these frames. Each shard's partial output is
-        # rounded to bf16 before the merge (half an ulp of the partial, which can exceed
-        # the merged value where partials of opposite sign cancel) and the merge rounds
-        # again; measured up to 2 ulps of the result. Bars: the attention max bar and
-        # half the attention mean bar
+        # attention: the unsplit result for these frames. The partial outputs stay in
+        # fp32 through the merges and are rounded to bf16 once, as the unsplit call's
+        # output is. What remains is the bf16 rounding of the softmax numerators P,
+        # taken against each shard's own running max instead of the whole row's (about
+        # 2^-9 of each P, averaged over the row's keys): within one bf16 ulp of the
+        # unsplit value, plus 2^-13 absolute where that value is near zero
         sl = slice(r * T_l * HW, (r + 1) * T_l * HW)
-        diff = (out.float() - out_g[:, :, sl].float()).abs()
-        assert float(diff.max()) <= ATT_MAX_ABS and float(diff.mean()) <= ATT_MEAN_ABS / 2, \
-            (float(diff.max()), float(diff.mean()))
+        ref = out_g[:, :, sl].float()
+        diff = (out.float() - ref).abs()
+        ulp = torch.exp2(torch.floor(torch.log2(ref.abs().clamp_min(2.0 ** -100))) - 7)
+        worst = float((diff / (ulp + 2.0 ** -13)).max())
+        assert worst <= 1.0, (worst, float(diff.max()))
         np.testing.assert_allclose(lse.cpu().numpy(), lse_g[:, :, sl].cpu().numpy(), rtol=0,
                                    atol=1e-4)
         # and the oracle, on the unsplit CSR rows of this rank
@@ -148,12 +151,20 @@ def test_csr_slice_and_merge_units():
             torch.zeros(1, dtype=torch.int32, device="cuda")
         outs.append(ops.forward(p, qd, kd, vd, srp, back.to(torch.int32)))
     (o, l), (o2, l2) = outs
+    assert o.dtype == torch.float32 and o2.dtype == torch.float32   # fp32 partial results
     ops.merge(p, o, l, o2, l2)
     of, lf = ops.forward(p, qd, kd, vd, pl.row_ptr, pl.col_idx)
     ops.check()
-    diff = (o.float() - of.float()).abs()
-    assert float(diff.max()) <= ATT_MAX_ABS and float(diff.mean()) <= ATT_MEAN_ABS / 2
+    # fp32 against fp32: only the bf16 rounding of P against different running maxima
+    diff = (o - of).abs()
+    assert float(diff.max()) <= 2e-3 and float(diff.mean()) <= 1e-4, \
+        (float(diff.max()), float(diff.mean()))
     torch.testing.assert_close(l, lf, rtol=0, atol=1e-4)
+    # and the merged fp32 result against the oracle
+    rows = np.arange(wl.rows)
+    o_out, _ = oracle.attend(q, k, v, wl.T, wl.H, wl.W, 1 / math.sqrt(wl.d), rp_h, ci_h, rows)
+    mx, mean = compare_attention(gather_rows(o.cpu().numpy(), wl, rows), o_out)
+    assert mx <= ATT_MAX_ABS / 4 and mean <= ATT_MEAN_ABS / 4, (mx, mean)
 
 
 def _unsplit_backward(wl, qd, kd, vd, gd):
