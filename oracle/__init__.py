@@ -75,6 +75,11 @@ def _load():
             lib.oracle_pool_shape.argtypes = [vp] + [i32] * 9 + [vp]
             lib.oracle_select_shape.restype = i64
             lib.oracle_select_shape.argtypes = [vp] + [i32] * 10 + [dbl, dbl, i32, vp, vp, i64]
+            lib.oracle_select_qk.restype = i64
+            lib.oracle_select_qk.argtypes = [vp] + [i32] * 13 + [dbl, dbl, i32, vp, vp, i64]
+            lib.oracle_attend_qk.restype = i32
+            lib.oracle_attend_qk.argtypes = [vp, vp, vp] + [i32] * 11 + [dbl, vp, vp, vp, i64,
+                                                                        vp, vp]
             lib.oracle_attend_shape.restype = i32
             lib.oracle_attend_shape.argtypes = [vp, vp, vp] + [i32] * 8 + [dbl, vp, vp, vp, i64,
                                                                            vp, vp]
@@ -170,46 +175,49 @@ def scores(qp, kp, scale, fp32=False):
 
 
 def select(S, T, H, W, mode="topk", topk=0, cdf_p=0.9, cap_frac=0.25, t_cond=0, fp32=False,
-           kchunk=CHUNK):
+           kchunk=CHUNK, qchunk=CHUNK):
     """CSR (row_ptr int32 [rows+1], col_idx int32 [nnz]) of the selected key chunks
-    (of shape `kchunk`) per (4,4,8) query chunk; S is [B, heads, Nq, Nk]."""
+    (of shape `kchunk`) per query chunk (of shape `qchunk`); S is [B, heads, Nq, Nk]."""
     S = np.ascontiguousarray(S, dtype=np.float64)
     B, Hh, Nq, Nk = S.shape
     rows = B * Hh * Nq
     row_ptr = np.zeros(rows + 1, dtype=np.int32)
     col_cap = rows * Nk
     col_idx = np.empty(max(col_cap, 1), dtype=np.int32)
-    nnz = _check(_load().oracle_select_shape(S.ctypes.data, B * Hh, T, H, W, *kchunk,
-                                             int(t_cond), MODES[mode], int(topk), float(cdf_p),
-                                             float(cap_frac), int(fp32), row_ptr.ctypes.data,
-                                             col_idx.ctypes.data, col_cap), "oracle_select")
+    nnz = _check(_load().oracle_select_qk(S.ctypes.data, B * Hh, T, H, W, *qchunk, *kchunk,
+                                          int(t_cond), MODES[mode], int(topk), float(cdf_p),
+                                          float(cap_frac), int(fp32), row_ptr.ctypes.data,
+                                          col_idx.ctypes.data, col_cap), "oracle_select")
     return row_ptr, col_idx[:nnz].copy()
 
 
 def plan(q, k, T, H, W, scale, mode="topk", topk=0, cdf_p=0.9, cap_frac=0.25, t_cond=0,
-         fp32=False, kchunk=CHUNK):
+         fp32=False, kchunk=CHUNK, qchunk=CHUNK):
     """pool -> scores -> select; returns (row_ptr, col_idx, S)."""
-    S = scores(pool(q, T, H, W, fp32), pool(k, T, H, W, fp32, kchunk), scale, fp32)
-    rp, ci = select(S, T, H, W, mode, topk, cdf_p, cap_frac, t_cond, fp32, kchunk)
+    S = scores(pool(q, T, H, W, fp32, qchunk), pool(k, T, H, W, fp32, kchunk), scale, fp32)
+    rp, ci = select(S, T, H, W, mode, topk, cdf_p, cap_frac, t_cond, fp32, kchunk, qchunk)
     return rp, ci, S
 
 
-def attend(q, k, v, T, H, W, scale, row_ptr, col_idx, rows, want_lse=True, kchunk=CHUNK):
-    """Sparse attention for the listed CSR rows: out [n, 128, d] f64, lse [n, 128]."""
+def attend(q, k, v, T, H, W, scale, row_ptr, col_idx, rows, want_lse=True, kchunk=CHUNK,
+           qchunk=CHUNK):
+    """Sparse attention for the listed CSR rows: out [n, slots, d] f64, lse [n, slots],
+    slots = the query chunk's token count (128 for (4,4,8))."""
     q, k, v = _u16(q), _u16(k), _u16(v)
     B, Hh, N, d = q.shape
+    qn = qchunk[0] * qchunk[1] * qchunk[2]
     rows = np.ascontiguousarray(rows, dtype=np.int64)
     rp = np.ascontiguousarray(row_ptr, dtype=np.int32)
     ci = np.ascontiguousarray(col_idx, dtype=np.int32)
     if ci.size == 0:
         ci = np.zeros(1, dtype=np.int32)
-    out = np.empty((rows.size, CN, d), dtype=np.float64)
-    lse = np.empty((rows.size, CN), dtype=np.float64) if want_lse else None
-    _check(_load().oracle_attend_shape(q.ctypes.data, k.ctypes.data, v.ctypes.data, B * Hh, T, H,
-                                       W, *kchunk, d, float(scale), rp.ctypes.data,
-                                       ci.ctypes.data, rows.ctypes.data, rows.size,
-                                       out.ctypes.data,
-                                       lse.ctypes.data if lse is not None else None),
+    out = np.empty((rows.size, qn, d), dtype=np.float64)
+    lse = np.empty((rows.size, qn), dtype=np.float64) if want_lse else None
+    _check(_load().oracle_attend_qk(q.ctypes.data, k.ctypes.data, v.ctypes.data, B * Hh, T, H,
+                                    W, *qchunk, *kchunk, d, float(scale), rp.ctypes.data,
+                                    ci.ctypes.data, rows.ctypes.data, rows.size,
+                                    out.ctypes.data,
+                                    lse.ctypes.data if lse is not None else None),
            "oracle_attend")
     return out, lse
 

@@ -191,7 +191,10 @@ static int int_cmp(const void* a, const void* b) {
 }
 
 /*
- * Block selection over the scores S[bh][i][m] -> CSR in row order (bh, i).
+ * Block selection over the scores S[bh][i][m] -> CSR in row order (bh, i), for
+ * query chunks of shape (qst, qsh, qsw) and key chunks of shape (kst, ksh, ksw)
+ * ([P1] block-size robustness: query blocks of 64 or 128 tokens, key blocks of
+ * 64 to 1024).
  * mode 0 = top-k ([P1] top-r; [P3] Top-K), mode 1 = CDF ([P3] CDF threshold;
  * [P1] CDF-p: walk the chunks from the highest pooled score down and stop as
  * soon as their softmax mass adds up to p or more), mode 2 = combination ([P3] names a combined mode next to Top-K
@@ -202,14 +205,15 @@ static int int_cmp(const void* a, const void* b) {
  * Column indices of a row are written in ascending order.
  * Returns nnz >= 0, or -1 on bad arguments, -2 if col_cap is too small.
  */
-int64_t oracle_select_shape(const double* S, int BH, int T, int H, int W, int kst, int ksh, int ksw,
-                            int t_cond, int mode, int topk, double cdf_p, double cap_frac, int fp32,
-                            int32_t* row_ptr, int32_t* col_idx, int64_t col_cap) {
-    if (!S || !row_ptr || !col_idx || BH <= 0 || !grid_ok(T, H, W) || t_cond < 0 ||
-        t_cond % CT != 0 || kst <= 0 || ksh <= 0 || ksw <= 0 || t_cond % kst != 0 || mode < 0 ||
-        mode > 2 || (mode != 1 && topk <= 0))
+int64_t oracle_select_qk(const double* S, int BH, int T, int H, int W, int qst, int qsh, int qsw,
+                         int kst, int ksh, int ksw, int t_cond, int mode, int topk, double cdf_p,
+                         double cap_frac, int fp32, int32_t* row_ptr, int32_t* col_idx,
+                         int64_t col_cap) {
+    if (!S || !row_ptr || !col_idx || BH <= 0 || !grid_ok(T, H, W) || t_cond < 0 || qst <= 0 ||
+        qsh <= 0 || qsw <= 0 || t_cond % qst != 0 || kst <= 0 || ksh <= 0 || ksw <= 0 ||
+        t_cond % kst != 0 || mode < 0 || mode > 2 || (mode != 1 && topk <= 0))
         return -1;
-    const int Nq = (int)oracle_num_chunks(T, H, W);                       /* query chunks */
+    const int Nq = (int)oracle_num_chunks_shape(T, H, W, qst, qsh, qsw);  /* query chunks */
     const int Nk = (int)oracle_num_chunks_shape(T, H, W, kst, ksh, ksw);  /* key chunks */
     cand_t* cand = (cand_t*)malloc(sizeof(cand_t) * (size_t)Nk);
     int32_t* pick = (int32_t*)malloc(sizeof(int32_t) * (size_t)Nk);
@@ -223,7 +227,7 @@ int64_t oracle_select_shape(const double* S, int BH, int T, int H, int W, int ks
     for (int bh = 0; bh < BH; ++bh) {
         for (int i = 0; i < Nq; ++i) {
             const double* row = S + ((int64_t)bh * Nq + i) * Nk;
-            const int q_cond = t_cond > 0 && is_condition_chunk(H, W, CT, CH, CW, i, t_cond);
+            const int q_cond = t_cond > 0 && is_condition_chunk(H, W, qst, qsh, qsw, i, t_cond);
             int na = 0;
             for (int m = 0; m < Nk; ++m) {
                 if (q_cond && !is_condition_chunk(H, W, kst, ksh, ksw, m, t_cond)) continue;
@@ -281,6 +285,14 @@ int64_t oracle_select_shape(const double* S, int BH, int T, int H, int W, int ks
     return nnz;
 }
 
+/* Query chunks of the [P3] shape (4,4,8), key chunks (kst, ksh, ksw). */
+int64_t oracle_select_shape(const double* S, int BH, int T, int H, int W, int kst, int ksh, int ksw,
+                            int t_cond, int mode, int topk, double cdf_p, double cap_frac, int fp32,
+                            int32_t* row_ptr, int32_t* col_idx, int64_t col_cap) {
+    return oracle_select_qk(S, BH, T, H, W, CT, CH, CW, kst, ksh, ksw, t_cond, mode, topk, cdf_p,
+                            cap_frac, fp32, row_ptr, col_idx, col_cap);
+}
+
 int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, int mode,
                       int topk, double cdf_p, double cap_frac, int fp32, int32_t* row_ptr,
                       int32_t* col_idx, int64_t col_cap) {
@@ -290,23 +302,25 @@ int64_t oracle_select(const double* S, int BH, int T, int H, int W, int t_cond, 
 
 /*
  * [P1] sparse attention: O = softmax(Q K^T / sqrt(d) with non-selected logits
- * at -inf) V, evaluated for the query chunks listed in rows[] (row r = bh*Nc+i)
- * over the tokens of the chunks in CSR row r. All arithmetic in fp64.
- * out[n][l][:] is the output of local query l of rows[n]; lse[n][l] is the
+ * at -inf) V, evaluated for the query chunks (shape (qst, qsh, qsw), Nc of them
+ * per (batch, head)) listed in rows[] (row r = bh*Nc+i) over the tokens of the
+ * key chunks (shape (kst, ksh, ksw)) in CSR row r. All arithmetic in fp64.
+ * out[n][l][:] (l < qst*qsh*qsw) is the output of local query l of rows[n]; lse[n][l] is the
  * natural-log log-sum-exp of the scaled logits (nullable). A row with no
  * selected chunk yields zeros and lse = -inf. Keys are the existing tokens of
  * the selected chunks; a local query slot past the grid edge (partial chunk)
  * has no output: NaN.
  */
-int oracle_attend_shape(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int T,
-                        int H, int W, int kst, int ksh, int ksw, int d, double scale,
-                        const int32_t* row_ptr, const int32_t* col_idx, const int64_t* rows,
-                        int64_t n_rows, double* out, double* lse) {
+int oracle_attend_qk(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int T,
+                     int H, int W, int qst, int qsh, int qsw, int kst, int ksh, int ksw, int d,
+                     double scale, const int32_t* row_ptr, const int32_t* col_idx,
+                     const int64_t* rows, int64_t n_rows, double* out, double* lse) {
     if (!q || !k || !v || !row_ptr || !col_idx || !rows || !out || BH <= 0 || d <= 0 ||
-        !grid_ok(T, H, W) || kst <= 0 || ksh <= 0 || ksw <= 0)
+        !grid_ok(T, H, W) || qst <= 0 || qsh <= 0 || qsw <= 0 || kst <= 0 || ksh <= 0 || ksw <= 0)
         return -1;
     const int kn = kst * ksh * ksw;  /* slots of a key chunk */
-    const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks(T, H, W);
+    const int qn = qst * qsh * qsw;  /* slots of a query chunk */
+    const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks_shape(T, H, W, qst, qsh, qsw);
     int bad = 0;
 #pragma omp parallel
     {
@@ -343,18 +357,18 @@ int oracle_attend_shape(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                     }
                 }
             }
-            for (int lq = 0; lq < CN; ++lq) {
-                const int64_t qtok = oracle_token_of(T, H, W, i, lq);
-                double* o = out + (n * CN + lq) * d;
+            for (int lq = 0; lq < qn; ++lq) {
+                const int64_t qtok = oracle_token_of_shape(T, H, W, qst, qsh, qsw, i, lq);
+                double* o = out + (n * qn + lq) * d;
                 if (qtok < 0) {
                     for (int x = 0; x < d; ++x) o[x] = NAN;
-                    if (lse) lse[n * CN + lq] = NAN;
+                    if (lse) lse[n * qn + lq] = NAN;
                     continue;
                 }
                 for (int x = 0; x < d; ++x) qd[x] = bf16_to_double(q[(bh * N + qtok) * d + x]);
                 if (nk == 0) {
                     for (int x = 0; x < d; ++x) o[x] = 0.0;
-                    if (lse) lse[n * CN + lq] = -INFINITY;
+                    if (lse) lse[n * qn + lq] = -INFINITY;
                     continue;
                 }
                 double mx = -INFINITY;
@@ -374,12 +388,21 @@ int oracle_attend_shape(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                     const double w = s[j] / z;
                     for (int x = 0; x < d; ++x) o[x] += w * vd[j * d + x];
                 }
-                if (lse) lse[n * CN + lq] = mx + log(z);
+                if (lse) lse[n * qn + lq] = mx + log(z);
             }
         }
         free(kd); free(vd); free(s); free(qd);
     }
     return bad ? -1 : 0;
+}
+
+/* Query chunks of the [P3] shape (4,4,8), key chunks (kst, ksh, ksw). */
+int oracle_attend_shape(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int T,
+                        int H, int W, int kst, int ksh, int ksw, int d, double scale,
+                        const int32_t* row_ptr, const int32_t* col_idx, const int64_t* rows,
+                        int64_t n_rows, double* out, double* lse) {
+    return oracle_attend_qk(q, k, v, BH, T, H, W, CT, CH, CW, kst, ksh, ksw, d, scale, row_ptr,
+                            col_idx, rows, n_rows, out, lse);
 }
 
 int oracle_attend(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH, int T, int H,
