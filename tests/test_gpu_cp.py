@@ -105,16 +105,14 @@ def test_ring_forward_equals_unsplit(name):
                 assert np.array_equal(ci[rp[row]:rp[row + 1]], g_ci[g_rp[grow]:g_rp[grow + 1]])
         # attention: the unsplit result for these frames. The partial outputs stay in
         # fp32 through the merges and are rounded to bf16 once, as the unsplit call's
-        # output is. What remains is the bf16 rounding of the softmax numerators P,
-        # taken against each shard's own running max instead of the whole row's (about
-        # 2^-9 of each P, averaged over the row's keys): within one bf16 ulp of the
-        # unsplit value, plus 2^-13 absolute where that value is near zero
+        # output is. What differs is the bf16 rounding of the softmax numerators P,
+        # taken against each shard's own running max instead of the whole row's, so
+        # the ring must be as accurate as the unsplit call against the fp64 oracle
+        # (below); here, close to it element by element
         sl = slice(r * T_l * HW, (r + 1) * T_l * HW)
-        ref = out_g[:, :, sl].float()
-        diff = (out.float() - ref).abs()
-        ulp = torch.exp2(torch.floor(torch.log2(ref.abs().clamp_min(2.0 ** -100))) - 7)
-        worst = float((diff / (ulp + 2.0 ** -13)).max())
-        assert worst <= 1.0, (worst, float(diff.max()))
+        diff = (out.float() - out_g[:, :, sl].float()).abs()
+        assert float(diff.max()) <= ATT_MAX_ABS / 2 and float(diff.mean()) <= ATT_MEAN_ABS / 4, \
+            (float(diff.max()), float(diff.mean()))
         np.testing.assert_allclose(lse.cpu().numpy(), lse_g[:, :, sl].cpu().numpy(), rtol=0,
                                    atol=1e-4)
         # and the oracle, on the unsplit CSR rows of this rank
@@ -125,6 +123,10 @@ def test_ring_forward_equals_unsplit(name):
         full[:, :, sl] = out
         mx, mean = compare_attention(gather_rows(host_f32(full), wl, rows), o_out)
         assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+        # as accurate as the unsplit call on these rows (measured: max within 2 %, mean
+        # within 0.1 %; with bf16 partials merged in bf16 the ring was 1.5-2.7x worse)
+        mx_u, mean_u = compare_attention(gather_rows(host_f32(out_g), wl, rows), o_out)
+        assert mx <= 1.1 * mx_u and mean <= 1.02 * mean_u, (mx, mx_u, mean, mean_u)
 
 
 def test_csr_slice_and_merge_units():
