@@ -62,7 +62,7 @@ def parse():
     ap.add_argument("--bwd-steps", type=int, default=10)
     ap.add_argument("--partition", default="heads", choices=["heads", "replicas"],
                     help="N > 1: split the heads of the one call (default) or run replicas")
-    ap.add_argument("--per-config", default="480p,long,causal_cdf",
+    ap.add_argument("--per-config", default="480p,long,causal_cdf,720p_q64",
                     help="other workloads timed after the main one (N = 1; '' for none)")
     ap.add_argument("--per-config-steps", type=int, default=10)
     return ap.parse_args()
@@ -100,8 +100,39 @@ def load_traffic(workload):
 
 
 def exec_flops(wl, nnz):
-    """Executed attention FLOPs: QK^T and PV over 128x128 tiles of kept chunks."""
-    return 4.0 * wl.d * 128 * 128 * nnz
+    """Attention FLOPs of the kept chunk pairs: QK^T and PV over the query chunk's
+    and the key chunk's tokens. With 128-token query chunks the plan's CSR lists
+    (4,4,8) boxes (128 x 128 per entry); with 64-token query chunks it lists key
+    chunks of 64 or 128 tokens."""
+    qc = tuple(getattr(wl, "qchunk", (4, 4, 8)))
+    if qc == (4, 4, 8):
+        return 4.0 * wl.d * 128 * 128 * nnz
+    kc = tuple(wl.kchunk)
+    return 4.0 * wl.d * (qc[0] * qc[1] * qc[2]) * (kc[0] * kc[1] * kc[2]) * nnz
+
+
+def sparsity(wl, nnz):
+    """1 - (attended query-key pairs) / (all query-key pairs of the computed rows)."""
+    qc = tuple(getattr(wl, "qchunk", (4, 4, 8)))
+    qn = qc[0] * qc[1] * qc[2]
+    return 1.0 - exec_flops(wl, nnz) / (4.0 * wl.d * wl.rows * qn * wl.N)
+
+
+def q64_box_entries(wl, row_ptr, col_idx):
+    """64-token query chunks: the (query box, key box) pairs the kernel computes
+    (each a 128 x 128 tile), i.e. the union over a box's two query chunks."""
+    import numpy as np
+    rp = np.asarray(row_ptr, dtype=np.int64)
+    ci = np.asarray(col_idx[: rp[-1]], dtype=np.int64)
+    NH, NW, NWq = wl.NH, wl.NW, wl.NWq
+    rows = np.repeat(np.arange(len(rp) - 1), np.diff(rp))
+    bh, q = rows // wl.Nc, rows % wl.Nc
+    qbox = bh * (wl.Nc // NWq * NW) + (q // NWq) * NW + (q % NWq) // 2
+    if tuple(wl.kchunk) == (4, 4, 4):
+        kbox = (ci // NWq) * NW + (ci % NWq) // 2
+    else:
+        kbox = ci
+    return int(np.unique(qbox * (1 << 20) + kbox).size)
 
 
 class ClockSampler:
@@ -255,7 +286,8 @@ def run_reference(args, wl, rank, world):
 
 def workload_config(wl, world, parallelism):
     return {"workload": wl.name, "B": wl.B, "heads": wl.heads, "grid_thw": [wl.T, wl.H, wl.W],
-            "d": wl.d, "chunk_thw": [4, 4, 8], "mode": wl.mode,
+            "d": wl.d, "chunk_thw": list(getattr(wl, "qchunk", (4, 4, 8))),
+            "key_chunk_thw": list(getattr(wl, "kchunk", (4, 4, 8))), "mode": wl.mode,
             "topk": wl.topk if wl.mode != "cdf" else None,
             "cdf_p": wl.cdf_p if wl.mode != "topk" else None,
             "t_cond": wl.t_cond, "q_begin": wl.q_begin, "parallelism": parallelism,
@@ -341,8 +373,16 @@ def time_config(wl, steps, peak_tf, stream):
     tf = exec_flops(wl, nnz) / fwd_ms / 1e9
     res = {"plan_ms": plan_ms, "fwd_ms": fwd_ms, "step_ms": plan_ms + fwd_ms,
            "fwd_exec_tflops": tf, "frac": tf / peak_tf, "nnz": nnz,
-           "sparsity": 1.0 - nnz / (wl.B * wl.heads * wl.Nq * wl.Nc), "steps": steps,
+           "sparsity": sparsity(wl, nnz), "steps": steps,
            "config": workload_config(wl, 1, "single"), "device_status": bsa.status_string(rc)}
+    if tuple(wl.qchunk) != (4, 4, 8):
+        # the kernel's tiles: (query box, key box) pairs of the two chunks' union
+        n_box = q64_box_entries(wl, pl.row_ptr.cpu().numpy(), pl.col_idx.cpu().numpy())
+        tile_tf = 4.0 * wl.d * 128 * 128 * n_box / fwd_ms / 1e9
+        res.update({"fwd_exec_tflops_note": "algorithmic: 4*d*64*64 per kept chunk pair",
+                    "box_tiles": n_box, "tile_tflops": tile_tf, "tile_frac": tile_tf / peak_tf,
+                    "useful_share_of_tiles": exec_flops(wl, nnz) / (4.0 * wl.d * 128 * 128 *
+                                                                    n_box)})
     del q, k, v, out, pl
     torch.cuda.empty_cache()
     return res
@@ -561,7 +601,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(wl_full, world, parallelism_of(args.partition, world)),
             "plan_ms": plan_ms, "fwd_ms": fwd_ms, "fwd_exec_tflops": fwd_tflops,
-            "nnz": nnz, "sparsity": 1.0 - nnz / (wl.B * wl.heads * wl.Nq * wl.Nc),
+            "nnz": nnz, "sparsity": sparsity(wl, nnz),
             "dense_equiv_tflops": 4.0 * wl.B * wl.heads * wl.Nq * 128 * wl.N * wl.d
             / ms_per_step / 1e9,
             "dense": dense, "roofline": roofline, "cpu_baseline": cpu, "backward": bwd,

@@ -75,10 +75,12 @@ class bsa_shape(ctypes.Structure):
 
 
 def make_params(B, heads, T, H, W, d, mode="topk", topk=1, cdf_p=0.9, cdf_cap_frac=0.25,
-                t_cond=0, scale=0.0, q_begin=0, kchunk=(0, 0, 0), q_end=0) -> bsa_params:
-    """kchunk: key chunk shape (t, h, w); 0 on an axis = the query chunk's (4, 4, 8).
-    [q_begin, q_end): latent frames whose queries are computed (q_end 0 = T)."""
-    return bsa_params(B, heads, T, H, W, d, 4, 4, 8, float(scale),
+                t_cond=0, scale=0.0, q_begin=0, kchunk=(0, 0, 0), q_end=0,
+                chunk=(4, 4, 8)) -> bsa_params:
+    """chunk: query chunk shape, (4, 4, 8) or (4, 4, 4) (64-token chunks). kchunk: key
+    chunk shape (t, h, w); 0 on an axis = the query chunk's. [q_begin, q_end): latent
+    frames whose queries are computed (q_end 0 = T)."""
+    return bsa_params(B, heads, T, H, W, d, *map(int, chunk), float(scale),
                       MODES[mode], int(topk), float(cdf_p),
                       float(cdf_cap_frac), int(t_cond), int(q_begin), *map(int, kchunk),
                       int(q_end))
@@ -88,7 +90,8 @@ def params_for(wl) -> bsa_params:
     """Parameters of a workload description (anything with the Workload fields)."""
     return make_params(wl.B, wl.heads, wl.T, wl.H, wl.W, wl.d, wl.mode, wl.topk, wl.cdf_p,
                        wl.cdf_cap_frac, wl.t_cond, scale=getattr(wl, "scale", 0.0),
-                       q_begin=getattr(wl, "q_begin", 0), kchunk=getattr(wl, "kchunk", (0, 0, 0)))
+                       q_begin=getattr(wl, "q_begin", 0), kchunk=getattr(wl, "kchunk", (0, 0, 0)),
+                       chunk=getattr(wl, "qchunk", (4, 4, 8)))
 
 
 _lib = None

@@ -50,6 +50,22 @@ WsLayout ws_layout(const Dims& g, const bsa_params& p) {
         L.kc_col_idx = off;
         off += round_up((size_t)(L.kc_cap > 0 ? L.kc_cap : 1) * sizeof(int32_t), 256);
     }
+    L.box_counts = L.box_row_ptr = L.box_col_idx = L.box_pat = off;
+    L.box_cap = 0;
+    if (g.qw != kChunkW) {
+        // a query box's list is the union of its two chunks' lists: at most their sum
+        L.box_cap = max_key_nnz_of(g, p);
+        if (L.box_cap < 1) L.box_cap = 1;
+        const size_t box_rows = (size_t)g.BH * g.NB;
+        L.box_counts = off;
+        off += round_up(box_rows * sizeof(int32_t), 256);
+        L.box_row_ptr = off;
+        off += round_up((box_rows + 1) * sizeof(int32_t), 256);
+        L.box_col_idx = off;
+        off += round_up((size_t)L.box_cap * sizeof(int32_t), 256);
+        L.box_pat = off;
+        off += round_up((size_t)L.box_cap, 256);
+    }
     L.total = off;
     return L;
 }
@@ -59,23 +75,36 @@ int make_dims(const bsa_params* p, Dims* g) {
     if (!p || !g) return BSA_ERR_INVALID_ARG;
     if (p->B <= 0 || p->heads <= 0 || p->T <= 0 || p->H <= 0 || p->W <= 0 || p->d <= 0)
         return BSA_ERR_SHAPE;
-    if (p->chunk_t != kChunkT || p->chunk_h != kChunkH || p->chunk_w != kChunkW)
+    // query chunks: (4,4,8), the [P3] default, or (4,4,4), the 64-token blocks of
+    // [P1]'s block-size robustness study
+    if (p->chunk_t != kChunkT || p->chunk_h != kChunkH ||
+        (p->chunk_w != kChunkW && p->chunk_w != kChunkW / 2))
         return BSA_ERR_UNSUPPORTED;
+    const bool q64 = p->chunk_w == kChunkW / 2;
     if (p->d != 64 && p->d != 128) return BSA_ERR_UNSUPPORTED;
     if (p->t_cond < 0 || p->t_cond % kChunkT || p->t_cond > p->T) return BSA_ERR_SHAPE;
     // key chunk shape: 0 = the query chunk's size on that axis; otherwise a
-    // positive multiple of it, at most 8 boxes of (4,4,8) in all
+    // positive multiple of it, at most 8 boxes of (4,4,8) in all. With 64-token
+    // query chunks the key chunk is (4,4,4) or (4,4,8).
     const int kt = p->kchunk_t ? p->kchunk_t : kChunkT, kh = p->kchunk_h ? p->kchunk_h : kChunkH,
-              kw = p->kchunk_w ? p->kchunk_w : kChunkW;
-    if (kt < 0 || kh < 0 || kw < 0 || kt % kChunkT || kh % kChunkH || kw % kChunkW)
-        return BSA_ERR_UNSUPPORTED;
-    if ((kt / kChunkT) * (kh / kChunkH) * (kw / kChunkW) > 8) return BSA_ERR_UNSUPPORTED;
+              kw = p->kchunk_w ? p->kchunk_w : p->chunk_w;
+    if (q64) {
+        if (kt != kChunkT || kh != kChunkH || (kw != kChunkW && kw != kChunkW / 2))
+            return BSA_ERR_UNSUPPORTED;
+    } else {
+        if (kt < 0 || kh < 0 || kw < 0 || kt % kChunkT || kh % kChunkH || kw % kChunkW)
+            return BSA_ERR_UNSUPPORTED;
+        if ((kt / kChunkT) * (kh / kChunkH) * (kw / kChunkW) > 8) return BSA_ERR_UNSUPPORTED;
+    }
     if (p->t_cond % kt) return BSA_ERR_SHAPE;
     if (p->q_begin < 0 || p->q_begin % kChunkT || p->q_begin >= p->T) return BSA_ERR_SHAPE;
     // q_end: 0 = T; otherwise past q_begin, at most T, a multiple of 4 unless it is T
     const int q_end = p->q_end ? p->q_end : p->T;
     if (q_end <= p->q_begin || q_end > p->T || (q_end % kChunkT && q_end != p->T))
         return BSA_ERR_SHAPE;
+    // 64-token query chunks: every query chunk is computed (no KV-cached step, no
+    // context-parallel row range)
+    if (q64 && (p->q_begin != 0 || q_end != p->T)) return BSA_ERR_UNSUPPORTED;
     if (!(std::isfinite(p->scale)) || p->scale < 0.f) return BSA_ERR_INVALID_ARG;
     if (p->mode == BSA_SEL_TOPK || p->mode == BSA_SEL_TOPK_CDF) {
         if (p->topk < 1) return BSA_ERR_INVALID_ARG;
@@ -96,30 +125,45 @@ int make_dims(const bsa_params* p, Dims* g) {
     // multiple of the chunk shape are partial
     g->NT = (p->T + kChunkT - 1) / kChunkT;
     g->NH = (p->H + kChunkH - 1) / kChunkH;
-    g->NW = (p->W + kChunkW - 1) / kChunkW;
-    const int64_t nc = (int64_t)g->NT * g->NH * g->NW;
+    g->NW = (p->W + kChunkW - 1) / kChunkW;          // (4,4,8) boxes along w
+    g->qw = p->chunk_w;
+    g->NWq = (p->W + g->qw - 1) / g->qw;              // query chunks along w
+    const int64_t nb = (int64_t)g->NT * g->NH * g->NW;
+    const int64_t nc = (int64_t)g->NT * g->NH * g->NWq;
     g->N = (int64_t)p->T * p->H * p->W;
     g->BH = (int64_t)p->B * p->heads;
     // Limits of this implementation: selection keeps a row of scores in one
-    // warp's registers (Nc <= 2048), grids index batch*heads in y (<= 65535),
+    // warp's registers (Nc, Nk <= 2048), grids index batch*heads in y (<= 65535),
     // and CSR offsets are int32.
     if (nc > 2048 || g->BH > 65535) return BSA_ERR_UNSUPPORTED;
     g->Nc = (int)nc;
-    g->mT = kt / kChunkT;
-    g->mH = kh / kChunkH;
-    g->mW = kw / kChunkW;
-    g->m = g->mT * g->mH * g->mW;
-    g->NkT = (g->NT + g->mT - 1) / g->mT;
-    g->NkH = (g->NH + g->mH - 1) / g->mH;
-    g->NkW = (g->NW + g->mW - 1) / g->mW;
+    g->NB = (int)nb;
+    if (q64) {
+        // key chunks are (4,4,4) half-boxes or whole (4,4,8) boxes; no expansion
+        g->kw64 = kw == kChunkW / 2;
+        g->mT = g->mH = g->mW = g->m = 1;
+        g->NkT = g->NT;
+        g->NkH = g->NH;
+        g->NkW = g->kw64 ? g->NWq : g->NW;
+    } else {
+        g->kw64 = 0;
+        g->mT = kt / kChunkT;
+        g->mH = kh / kChunkH;
+        g->mW = kw / kChunkW;
+        g->m = g->mT * g->mH * g->mW;
+        g->NkT = (g->NT + g->mT - 1) / g->mT;
+        g->NkH = (g->NH + g->mH - 1) / g->mH;
+        g->NkW = (g->NW + g->mW - 1) / g->mW;
+    }
     g->Nk = g->NkT * g->NkH * g->NkW;
     g->n_cond_k = (p->t_cond / kt) * g->NkH * g->NkW;
-    g->q_skip = (p->q_begin / kChunkT) * g->NH * g->NW;
-    const int q_stop = q_end == p->T ? g->Nc : (q_end / kChunkT) * g->NH * g->NW;
+    g->q_skip = (p->q_begin / kChunkT) * g->NH * g->NWq;
+    const int q_stop = q_end == p->T ? g->Nc : (q_end / kChunkT) * g->NH * g->NWq;
     g->Nq = q_stop - g->q_skip;
     g->rows = g->BH * g->Nq;
-    if (g->rows * (int64_t)g->Nc > INT32_MAX) return BSA_ERR_UNSUPPORTED;
-    g->n_cond = (p->t_cond / kChunkT) * g->NH * g->NW;
+    const int nmax = g->Nc > g->Nk ? g->Nc : g->Nk;
+    if (g->rows * (int64_t)nmax > INT32_MAX) return BSA_ERR_UNSUPPORTED;
+    g->n_cond = (p->t_cond / kChunkT) * g->NH * g->NWq;
     g->scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt((float)p->d);
     return BSA_OK;
 }
@@ -161,6 +205,34 @@ static bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr)
 
 static int cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
 
+cudaError_t launch_forward_any(const Dims& g, const bsa_params& p, const void* q, const void* k,
+                               const void* v, const int32_t* row_ptr, const int32_t* col_idx,
+                               int64_t col_cap, char* ws, uint32_t* status, void* out, float* lse,
+                               uint64_t timeout_ns, int debug_flags, cudaStream_t st,
+                               float* out_f32) {
+    if (g.qw == kChunkW)
+        return launch_forward(g, q, k, v, row_ptr, col_idx, col_cap, out, lse, status, timeout_ns,
+                              debug_flags, st, out_f32);
+    // 64-token query chunks: one tile per (4,4,8) box of queries, over the union of
+    // its two chunks' key boxes with a quadrant pattern per entry
+    const WsLayout L = ws_layout(g, p);
+    int32_t* bcnt = reinterpret_cast<int32_t*>(ws + L.box_counts);
+    int32_t* brp = reinterpret_cast<int32_t*>(ws + L.box_row_ptr);
+    int32_t* bci = reinterpret_cast<int32_t*>(ws + L.box_col_idx);
+    uint8_t* bpat = reinterpret_cast<uint8_t*>(ws + L.box_pat);
+    cudaError_t e = launch_quad_union(g, row_ptr, col_idx, col_cap, bcnt, brp, bci, bpat,
+                                      L.box_cap, status, st);
+    if (e != cudaSuccess) return e;
+    Dims gb = g;
+    gb.Nc = gb.Nq = g.NB;
+    gb.q_skip = 0;
+    gb.rows = g.BH * g.NB;
+    gb.qw = kChunkW;
+    gb.NWq = g.NW;
+    return launch_forward(gb, q, k, v, brp, bci, L.box_cap, out, lse, status, timeout_ns,
+                          debug_flags, st, out_f32, bpat);
+}
+
 int device_ok() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
@@ -170,13 +242,19 @@ int device_ok() {
     return major == 10 ? BSA_OK : BSA_ERR_UNSUPPORTED;
 }
 
+// Workspace bsa_forward needs: the status block, plus the box CSR for 64-token
+// query chunks (the plan's workspace, bsa_workspace_size, holds both).
+static size_t forward_ws_bytes(const Dims& g, const bsa_params& p) {
+    return g.qw == kChunkW ? 256 : ws_layout(g, p).total;
+}
+
 }  // namespace bsa
 
 using namespace bsa;
 
 extern "C" {
 
-int bsa_version(void) { return 200; }
+int bsa_version(void) { return 300; }
 
 const char* bsa_status_string(int s) {
     switch (s) {
@@ -285,12 +363,13 @@ int bsa_forward_ex(const bsa_params* p, const void* q, const void* k, const void
         !aligned16(workspace) || (lse && !aligned4(lse)) || !aligned4(row_ptr) ||
         !aligned4(col_idx))
         return BSA_ERR_ALIGNMENT;
-    if (ws_bytes < 256) return BSA_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_bytes < forward_ws_bytes(g, *p)) return BSA_ERR_WORKSPACE_TOO_SMALL;
     if ((rc = device_ok()) != BSA_OK) return rc;
-    uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace));
-    return cuda_status(launch_forward(g, q, k, v, row_ptr, col_idx, col_capacity, out, lse, status,
-                                      timeout_ns ? timeout_ns : kDefaultTimeoutNs, debug_flags,
-                                      static_cast<cudaStream_t>(stream)));
+    char* ws = static_cast<char*>(workspace);
+    return cuda_status(launch_forward_any(g, *p, q, k, v, row_ptr, col_idx, col_capacity, ws,
+                                          reinterpret_cast<uint32_t*>(ws), out, lse,
+                                          timeout_ns ? timeout_ns : kDefaultTimeoutNs, debug_flags,
+                                          static_cast<cudaStream_t>(stream), nullptr));
 }
 
 int bsa_forward_partial(const bsa_params* p, const void* q, const void* k, const void* v,
@@ -307,12 +386,13 @@ int bsa_forward_partial(const bsa_params* p, const void* q, const void* k, const
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out_f32) ||
         !aligned16(workspace) || !aligned4(lse) || !aligned4(row_ptr) || !aligned4(col_idx))
         return BSA_ERR_ALIGNMENT;
-    if (ws_bytes < 256) return BSA_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_bytes < forward_ws_bytes(g, *p)) return BSA_ERR_WORKSPACE_TOO_SMALL;
     if ((rc = device_ok()) != BSA_OK) return rc;
-    uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace));
-    return cuda_status(launch_forward(g, q, k, v, row_ptr, col_idx, col_capacity, nullptr, lse,
-                                      status, kDefaultTimeoutNs, 0,
-                                      static_cast<cudaStream_t>(stream), out_f32));
+    char* ws = static_cast<char*>(workspace);
+    return cuda_status(launch_forward_any(g, *p, q, k, v, row_ptr, col_idx, col_capacity, ws,
+                                          reinterpret_cast<uint32_t*>(ws), nullptr, lse,
+                                          kDefaultTimeoutNs, 0, static_cast<cudaStream_t>(stream),
+                                          out_f32));
 }
 
 int bsa_forward(const bsa_params* p, const void* q, const void* k, const void* v,
@@ -324,7 +404,7 @@ int bsa_forward(const bsa_params* p, const void* q, const void* k, const void* v
 
 size_t bsa_backward_workspace_size(const bsa_params* p) {
     Dims g;
-    if (make_dims(p, &g) != BSA_OK) return 0;
+    if (make_dims(p, &g) != BSA_OK || g.qw != kChunkW) return 0;
     return bwd_layout(g).total;
 }
 
@@ -336,6 +416,7 @@ int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* 
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
+    if (g.qw != kChunkW) return BSA_ERR_UNSUPPORTED;  // 64-token chunks: forward only
     if (!q || !k || !v || !out || !lse || !dout || !row_ptr || !col_idx || !workspace || !dq ||
         !dk || !dv || col_capacity < 0)
         return BSA_ERR_INVALID_ARG;
@@ -357,6 +438,7 @@ int bsa_select_pooled(const bsa_params* p, const float* qpool, const float* kpoo
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
+    if (g.qw != kChunkW) return BSA_ERR_UNSUPPORTED;  // the ring uses (4,4,8) chunks
     if (!qpool || !kpool || !workspace || !row_ptr || !col_idx) return BSA_ERR_INVALID_ARG;
     if (kshard < 0 || (kshard > 0 && g.Nk % kshard)) return BSA_ERR_INVALID_ARG;
     if (!aligned16(qpool) || !aligned16(kpool) || !aligned16(workspace) || !aligned16(row_ptr) ||
@@ -485,6 +567,7 @@ int bsa_rearrange(const bsa_params* p, const void* x, void* out, int inverse, vo
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
+    if (g.qw != kChunkW) return BSA_ERR_UNSUPPORTED;  // chunk-major copy of (4,4,8) chunks
     if (!x || !out || (inverse != 0 && inverse != 1)) return BSA_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(out)) return BSA_ERR_ALIGNMENT;
     if ((rc = device_ok()) != BSA_OK) return rc;

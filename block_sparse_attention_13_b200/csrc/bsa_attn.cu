@@ -33,6 +33,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "bsa_internal.cuh"
 #include "bsa_ptx.cuh"
 
@@ -82,6 +84,7 @@ struct FwdArgs {
     int64_t col_cap;
     __nv_bfloat16* out;
     float* out_f32;    // non-null: O is written here in fp32 instead of bf16 to `out`
+    const uint8_t* quad;  // 64-token query chunks: quadrant pattern of every CSR entry
     float* lse;
     uint32_t* status;
     int T, H, W, NH, NW, Nc;
@@ -119,7 +122,13 @@ struct __align__(8) Ctl {
 // slots and 0 elsewhere (one B tile per edge pattern: partial in t, h, w or a
 // combination). Existing slots get exactly +0 and missing ones -inf, as a mask
 // would give, and the softmax loop is the same as for full grids.
-template <int D, bool kPartial>
+// kQuad: 64-token query (and key) chunks. A tile is a (4,4,8) box of queries, i.e.
+// two w-adjacent query chunks (rows with lw < 4 and lw >= 4), and its CSR row is the
+// union of the key boxes they selected; each entry's quadrant pattern says which key
+// halves (key slots with lw < 4, lw >= 4) each query half attends to. The softmax
+// threads set the logits of the other key halves to -inf before the row max, so the
+// result is exactly the attention of each query chunk over its own key chunks.
+template <int D, bool kPartial, bool kQuad>
 __global__ void __launch_bounds__(320, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -196,13 +205,16 @@ __global__ void __launch_bounds__(320, 1)
                 const int slot = t * C::kMaxChunks + cnt + __popc(vb & ((1u << lane) - 1u));
                 if (valid) {
                     lists[slot] = static_cast<uint16_t>(c);
+                    // bits 0-2: edge pattern of a partial key box; bits 3-6: quadrant pattern
+                    uint32_t pv = 0;
                     if constexpr (kPartial) {
                         int kt, kh, kw;
                         chunk_origin(c, a.NH, a.NW, kt, kh, kw);
-                        pats[slot] = static_cast<uint8_t>((kt + kChunkT > a.T ? 1 : 0) |
-                                                          (kh + kChunkH > a.H ? 2 : 0) |
-                                                          (kw + kChunkW > a.W ? 4 : 0));
+                        pv = (kt + kChunkT > a.T ? 1u : 0u) | (kh + kChunkH > a.H ? 2u : 0u) |
+                             (kw + kChunkW > a.W ? 4u : 0u);
                     }
+                    if constexpr (kQuad) pv |= static_cast<uint32_t>(a.quad[e] & 15u) << 3;
+                    if constexpr (kPartial || kQuad) pats[slot] = static_cast<uint8_t>(pv);
                 }
                 cnt += __popc(vb);
             }
@@ -319,7 +331,7 @@ __global__ void __launch_bounds__(320, 1)
                            sdesc_sw128(sk + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
                 }
                 if constexpr (kPartial) {
-                    const int pat = pats[t * C::kMaxChunks + j];
+                    const int pat = pats[t * C::kMaxChunks + j] & 7;
                     if (pat) {
                         const uint32_t sb = smem_u32(smem + C::kBias);
                         mma_ss(tmem + C::s_col(t), sdesc_plain(sb, 0, 128),
@@ -376,6 +388,7 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t tO = tmem + lane_off + C::o_col(t);
         const float c2 = a.scale_log2;
         float m_run = -INFINITY;
+        bool has_key = false;  // a step with keys for this row has been seen
         float2 l2 = make_float2(0.f, 0.f), l2b = make_float2(0.f, 0.f);
         bool ok = true;
         for (int it = 0; it < n_t; ++it) {
@@ -390,38 +403,72 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 tmem_wait_ld_tie(*reinterpret_cast<uint32_t(*)[32]>(s + 32 * c));
-            float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
-            float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
+            // Row max in four chains: key slots with lw in {0,1}, {2,3} (the key box's
+            // left half, lw < 4) and {4,5}, {6,7} (its right half).
+            float ha0 = fmaxf(__uint_as_float(s[0]), __uint_as_float(s[1]));
+            float ha1 = fmaxf(__uint_as_float(s[2]), __uint_as_float(s[3]));
+            float hb0 = fmaxf(__uint_as_float(s[4]), __uint_as_float(s[5]));
+            float hb1 = fmaxf(__uint_as_float(s[6]), __uint_as_float(s[7]));
 #pragma unroll
-            for (int j = 4; j < 128; j += 8) {
-                mx0 = fmax3(mx0, __uint_as_float(s[j]), __uint_as_float(s[j + 1]));
-                mx1 = fmax3(mx1, __uint_as_float(s[j + 2]), __uint_as_float(s[j + 3]));
-                mx2 = fmax3(mx2, __uint_as_float(s[j + 4]), __uint_as_float(s[j + 5]));
-                mx3 = fmax3(mx3, __uint_as_float(s[j + 6]), __uint_as_float(s[j + 7]));
+            for (int j = 8; j < 128; j += 8) {
+                ha0 = fmax3(ha0, __uint_as_float(s[j]), __uint_as_float(s[j + 1]));
+                ha1 = fmax3(ha1, __uint_as_float(s[j + 2]), __uint_as_float(s[j + 3]));
+                hb0 = fmax3(hb0, __uint_as_float(s[j + 4]), __uint_as_float(s[j + 5]));
+                hb1 = fmax3(hb1, __uint_as_float(s[j + 6]), __uint_as_float(s[j + 7]));
             }
-            const float m_new = fmax3(fmaxf(mx0, mx1), mx2, mx3) * c2;
-            // Lazy rescale: move the reference max only when it grows by > 2^8.
-            const bool rescale = it > 0 && m_new > m_run + 8.0f;
+            const float mx_a = fmaxf(ha0, ha1), mx_b = fmaxf(hb0, hb1);
+            // kQuad: the key halves this query row attends to in this box (its query
+            // half is the lw of row m). The masked logits never enter any arithmetic:
+            // the max is taken over the kept halves and masked numerators are zeroed.
+            bool keep_a = true, keep_b = true;
+            if constexpr (kQuad) {
+                const uint32_t qp = pats[t * C::kMaxChunks + it] >> 3;
+                const uint32_t mine = (qp >> ((m & 4) ? 2 : 0)) & 3u;
+                keep_a = mine & 1u;
+                keep_b = mine & 2u;
+            }
+            const bool step_has = keep_a || keep_b;
+            const float m_new =
+                (keep_a && keep_b ? fmaxf(mx_a, mx_b) : (keep_a ? mx_a : mx_b)) * c2;
+            // Lazy rescale: move the reference max only when it grows by > 2^8. The
+            // first step with a key sets it (it == 0 unless rows skip steps).
+            const bool first = !has_key && step_has;
+            const bool rescale = has_key && step_has && m_new > m_run + 8.0f;
             const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
-            if (it == 0 || rescale) m_run = m_new;
+            if (first || rescale) m_run = m_new;
+            has_key = has_key || step_has;
             l2.x *= alpha;
             l2.y *= alpha;
             l2b.x *= alpha;
             l2b.y *= alpha;
             const float2 cc = make_float2(c2, c2);
-            const float2 nm = make_float2(-m_run, -m_run);
+            // no key yet (kQuad): every numerator of this step is zeroed below
+            const float m_ref = has_key ? m_run : 0.0f;
+            const float2 nm = make_float2(-m_ref, -m_ref);
+            const bool masked = kQuad && __any_sync(0xffffffffu, !(keep_a && keep_b));
             uint32_t pk[64];
+            auto exp_pairs = [&](auto mask_tag) {
+                constexpr bool kMask = decltype(mask_tag)::value;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                const float2 x = __ffma2_rn(
-                    make_float2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), cc, nm);
-                // alternate pairs between the MUFU unit and the FMA-pipe polynomial
-                const float2 pp = (kPolyEvery > 0 && j % kPolyEvery == 0)
-                                      ? exp2_poly2(x)
-                                      : make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                if (j & 1) l2b = __fadd2_rn(l2b, pp); else l2 = __fadd2_rn(l2, pp);
-                pk[j] = pack_bf16x2(pp.x, pp.y);
-            }
+                for (int j = 0; j < 64; ++j) {
+                    const float2 x = __ffma2_rn(
+                        make_float2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), cc,
+                        nm);
+                    // alternate pairs between the MUFU unit and the FMA-pipe polynomial
+                    float2 pp = (kPolyEvery > 0 && j % kPolyEvery == 0)
+                                    ? exp2_poly2(x)
+                                    : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    // pair j holds key slots 2j, 2j+1: lw of both is < 4 iff (j & 2) == 0
+                    if constexpr (kMask)
+                        if (!((j & 2) ? keep_b : keep_a)) pp = make_float2(0.0f, 0.0f);
+                    if (j & 1) l2b = __fadd2_rn(l2b, pp); else l2 = __fadd2_rn(l2, pp);
+                    pk[j] = pack_bf16x2(pp.x, pp.y);
+                }
+            };
+            if (masked)
+                exp_pairs(std::true_type{});
+            else
+                exp_pairs(std::false_type{});
             // P over S columns [0, 64): every S value is already in registers
             tmem_st32(tS + 0, *reinterpret_cast<const uint32_t(*)[32]>(pk + 0));
             tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
@@ -467,7 +514,9 @@ __global__ void __launch_bounds__(320, 1)
                 // stores its own row, 128-bit stores; tcgen05.ld is warp-collective,
                 // so every lane loads and only existing query slots store
                 tc_fence_after();
-                const float inv_l = 1.0f / l_run;
+                // a row without any key (kQuad: its query chunk kept none of the box's
+                // keys): zeros, lse = -inf
+                const float inv_l = has_key ? 1.0f / l_run : 0.0f;
                 float4* dst = reinterpret_cast<float4*>(a.out_f32 + (bh * a.N + tok) * D);
 #pragma unroll
                 for (int g = 0; g < D / 32; ++g) {
@@ -484,10 +533,11 @@ __global__ void __launch_bounds__(320, 1)
                     }
                 }
                 if (a.lse && q_exists)
-                    a.lse[bh * a.N + tok] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+                    a.lse[bh * a.N + tok] =
+                        has_key ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
             } else if (all_ok && n_t > 0) {
                 tc_fence_after();
-                const float inv_l = 1.0f / l_run;
+                const float inv_l = has_key ? 1.0f / l_run : 0.0f;
                 uint8_t* stage = smem + C::q_off(t);  // Q of this tile is dead once O is final
 #pragma unroll
                 for (int g = 0; g < D / 32; ++g) {
@@ -518,7 +568,8 @@ __global__ void __launch_bounds__(320, 1)
                     tma_store_commit_and_wait_all();
                 }
                 if (a.lse && q_exists)
-                    a.lse[bh * a.N + tok] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+                    a.lse[bh * a.N + tok] =
+                        has_key ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
             } else if (all_ok && q_exists) {
                 // empty (or rejected) row: zeros, lse = -inf
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
@@ -587,16 +638,18 @@ bool make_chunk_map(CUtensorMap* tm, const void* base, const Dims& g, int box_t)
 
 namespace {
 
-template <int D, bool kPartial>
+template <int D, bool kPartial, bool kQuad>
 cudaError_t launch_fwd_dp(const Dims& g, const CUtensorMap& mq, const CUtensorMap& mk,
                           const CUtensorMap& mv, const CUtensorMap& mo, const FwdArgs& args,
                           cudaStream_t st) {
     using C = AttnCfg<D>;
     static std::atomic<uint64_t> attr_done{0};
-    const cudaError_t e = raise_smem_limit(bsa_fwd_kernel<D, kPartial>, C::kSmemBytes, attr_done);
+    const cudaError_t e =
+        raise_smem_limit(bsa_fwd_kernel<D, kPartial, kQuad>, C::kSmemBytes, attr_done);
     if (e != cudaSuccess) return e;
     const unsigned grid = static_cast<unsigned>((g.rows + 1) / 2);
-    bsa_fwd_kernel<D, kPartial><<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mo, args);
+    bsa_fwd_kernel<D, kPartial, kQuad>
+        <<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mo, args);
     return cudaGetLastError();
 }
 
@@ -605,8 +658,11 @@ cudaError_t launch_fwd_d(const Dims& g, const CUtensorMap& mq, const CUtensorMap
                          const CUtensorMap& mv, const CUtensorMap& mo, const FwdArgs& args,
                          cudaStream_t st) {
     const bool partial = g.T % kChunkT || g.H % kChunkH || g.W % kChunkW;
-    return partial ? launch_fwd_dp<D, true>(g, mq, mk, mv, mo, args, st)
-                   : launch_fwd_dp<D, false>(g, mq, mk, mv, mo, args, st);
+    if (args.quad)
+        return partial ? launch_fwd_dp<D, true, true>(g, mq, mk, mv, mo, args, st)
+                       : launch_fwd_dp<D, false, true>(g, mq, mk, mv, mo, args, st);
+    return partial ? launch_fwd_dp<D, true, false>(g, mq, mk, mv, mo, args, st)
+                   : launch_fwd_dp<D, false, false>(g, mq, mk, mv, mo, args, st);
 }
 
 __global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y_poly,
@@ -635,7 +691,8 @@ cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, i
 cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const void* v,
                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
                            void* out, float* lse, uint32_t* status, uint64_t timeout_ns,
-                           int debug_flags, cudaStream_t st, float* out_f32) {
+                           int debug_flags, cudaStream_t st, float* out_f32,
+                           const uint8_t* quad) {
     if (!out && !out_f32) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv, mo;
     // with an fp32 output the bf16 output map is never used (built over q)
@@ -648,6 +705,7 @@ cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const vo
     args.col_cap = col_cap;
     args.out = static_cast<__nv_bfloat16*>(out);
     args.out_f32 = out_f32;
+    args.quad = quad;
     args.lse = lse;
     args.status = status;
     args.T = g.T;

@@ -199,9 +199,9 @@ int bsa_forward_host(const bsa_params* p, const void* q, const void* k, const vo
         int32_t* ci = reinterpret_cast<int32_t*>(slot + L.col_idx);
         if (plan_group(gd, pg, slot + L.q, slot + L.k, slot + L.plan_ws, rp, ci, L.col_cap, status,
                        st) != cudaSuccess ||
-            launch_forward(gd, slot + L.q, slot + L.k, slot + L.v, rp, ci, L.col_cap,
-                           slot + L.out, nullptr, status, kDefaultTimeoutNs, 0, st) !=
-                cudaSuccess) {
+            launch_forward_any(gd, pg, slot + L.q, slot + L.k, slot + L.v, rp, ci, L.col_cap,
+                               slot + L.plan_ws, status, slot + L.out, nullptr, kDefaultTimeoutNs,
+                               0, st, nullptr) != cudaSuccess) {
             err = BSA_ERR_CUDA;
             break;
         }

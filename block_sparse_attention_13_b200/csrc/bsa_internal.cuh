@@ -58,7 +58,11 @@ __host__ __device__ __forceinline__ uint32_t site(int role, int bar, int tile, i
 // Derived sizes of one call.
 struct Dims {
     int B, heads, T, H, W, d;
-    int NT, NH, NW, Nc;  // query chunks ((4,4,8) boxes) per axis and per (batch, head)
+    int NT, NH, NW;      // (4,4,8) boxes per axis (the unit of the attention kernels' tiles)
+    int Nc;              // query chunks per (batch, head) (= boxes, unless 64-token chunks)
+    int qw, NWq;         // query chunk width along w (8, or 4 for 64-token chunks); chunks along w
+    int NB;              // (4,4,8) boxes per (batch, head)
+    int kw64;            // key chunks are (4,4,4) half-boxes (64-token query chunks only)
     int64_t N, BH, rows;
     int n_cond;      // condition query chunks per (batch, head); 0 without block-causal mask
     int q_skip;      // query chunks before q_begin (not computed)
@@ -82,6 +86,13 @@ struct WsLayout {
     size_t kc_row_ptr;  // int32 [rows+1]   key-chunk CSR before box expansion (m > 1)
     size_t kc_col_idx;  // int32 [kc_cap]
     int64_t kc_cap;
+    // 64-token query chunks: the forward's CSR over (4,4,8) boxes, one row per query
+    // box (its two query chunks), with a quadrant pattern per entry
+    size_t box_counts;  // int32 [BH*NB]
+    size_t box_row_ptr; // int32 [BH*NB+1]
+    size_t box_col_idx; // int32 [box_cap]
+    size_t box_pat;     // uint8 [box_cap]
+    int64_t box_cap;
     size_t total;
 };
 
@@ -122,11 +133,14 @@ cudaError_t launch_scores(const Dims& g, const float* qp, const float* kp, float
 cudaError_t launch_select(const Dims& g, const bsa_params& p, const float* S, int32_t* row_ptr,
                           int32_t* col_idx, int64_t col_cap, int32_t* counts, int32_t* padded,
                           int pad_stride, uint32_t* status, cudaStream_t st);
-// out_f32 non-null: O is written there in fp32 (and `out` is not used).
+// out_f32 non-null: O is written there in fp32 (and `out` is not used). quad
+// non-null: rows are query boxes of 64-token chunks, with a quadrant pattern per
+// CSR entry (launch_quad_union); g then describes boxes (Nc = Nq = NB).
 cudaError_t launch_forward(const Dims& g, const void* q, const void* k, const void* v,
                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
                            void* out, float* lse, uint32_t* status, uint64_t timeout_ns,
-                           int debug_flags, cudaStream_t st, float* out_f32 = nullptr);
+                           int debug_flags, cudaStream_t st, float* out_f32 = nullptr,
+                           const uint8_t* quad = nullptr);
 // 5-D TMA map over a [BH][T][H][W][d] bf16 tensor whose box is one (4,4,8)
 // chunk x 64 channels (128-byte swizzle); box_t = 2 gives half a chunk (its
 // first or last two frames: local tokens 0-63 or 64-127). False if the driver
@@ -138,6 +152,22 @@ cudaError_t launch_expand_boxes(const Dims& g, const int32_t* kc_row_ptr,
                                 const int32_t* kc_col_idx, int32_t* counts, int32_t* row_ptr,
                                 int32_t* col_idx, int64_t col_cap, uint32_t* status,
                                 cudaStream_t st);
+// 64-token query chunks: the chunk CSR (rows = query chunks) -> a CSR over
+// (4,4,8) boxes with one row per query box and a 4-bit quadrant pattern per
+// entry (bits 0-1: key halves the box's left query chunk attends to, bits 2-3:
+// the right one's).
+cudaError_t launch_quad_union(const Dims& g, const int32_t* row_ptr, const int32_t* col_idx,
+                              int64_t col_cap, int32_t* counts, int32_t* box_row_ptr,
+                              int32_t* box_col, uint8_t* box_pat, int64_t box_cap,
+                              uint32_t* status, cudaStream_t st);
+// The forward of one call on device buffers: for 64-token query chunks the box
+// CSR is built first, in the regions ws_layout(g, p) gives inside `ws` (a
+// workspace of at least that size; unused otherwise). Device errors go to status.
+cudaError_t launch_forward_any(const Dims& g, const bsa_params& p, const void* q, const void* k,
+                               const void* v, const int32_t* row_ptr, const int32_t* col_idx,
+                               int64_t col_cap, char* ws, uint32_t* status, void* out, float* lse,
+                               uint64_t timeout_ns, int debug_flags, cudaStream_t st,
+                               float* out_f32);
 cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const void* v,
                             const void* out, const float* lse, const void* dout,
                             const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,

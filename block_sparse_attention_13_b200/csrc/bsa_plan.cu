@@ -39,12 +39,14 @@ __device__ __forceinline__ void add_bf16x2(float& a, float& b, uint32_t u) {
 // over its tokens in fp32; a shared-memory pass finishes the 128-token sum.
 // Tensor z (blockIdx.z) pools chunks [c_begin, c_begin + n_out) of its own
 // chunk grid into rows 0 .. n_out-1 of its output. A chunk is mt x mh x mw
-// (4,4,8) boxes (a key chunk can be larger than the query chunk); a partial
-// edge chunk averages the tokens it has.
+// boxes of (4,4,bw) tokens, bw = 8 or 4 (a key chunk can be larger than the
+// query chunk; 64-token chunks are single (4,4,4) boxes); a partial edge chunk
+// averages the tokens it has.
 struct PoolSide {
     int c_begin, n_out;
     int mt, mh, mw;  // boxes per chunk along t, h, w
     int NHc, NWc;    // chunks of this grid along h, w
+    int bw;          // box width along w: 8, or 4 for 64-token chunks
 };
 
 template <int D>
@@ -74,7 +76,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     const __nv_bfloat16* base = x + bh * N * D;
     // sums the existing tokens of the box at (t0, h0, w0); returns their count
     auto add_box = [&](int t0, int h0, int w0) -> int {
-        const int nt = min(kChunkT, T - t0), nh = min(kChunkH, H - h0), nw = min(kChunkW, W - w0);
+        const int nt = min(kChunkT, T - t0), nh = min(kChunkH, H - h0), nw = min(sd.bw, W - w0);
         if (nt <= 0 || nh <= 0 || nw <= 0) return 0;  // box past the grid
         if (nt == kChunkT && nh == kChunkH && nw == kChunkW) {
             // a whole box: every load unconditional, all in flight together
@@ -94,10 +96,14 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
                 add_bf16x2(acc[6], acc[7], u[it].w);
             }
         } else {
+            // a partial box, or a (4,4,4) box of 64 tokens: local token l is
+            // (lt*4 + lh)*bw + lw
+            const int lb = sd.bw == kChunkW ? 3 : 2;  // log2(bw)
 #pragma unroll
             for (int it = 0; it < ITERS; ++it) {
                 const int l = (it * 256 + tid) / VPT;
-                const int lt = l >> 5, lh = (l >> 3) & 3, lw = l & 7;
+                if (l >= (16 << lb)) continue;
+                const int lt = l >> (lb + 2), lh = (l >> lb) & 3, lw = l & ((1 << lb) - 1);
                 if (lt >= nt || lh >= nh || lw >= nw) continue;
                 const int64_t tok = ((int64_t)(t0 + lt) * H + (h0 + lh)) * W + w0 + lw;
                 const uint4 u = ld_nc_v4(base + tok * D + dvec * 8);
@@ -111,13 +117,13 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     };
     int n_tok = 0;
     if (sd.mt * sd.mh * sd.mw == 1) {
-        n_tok = add_box(ct * kChunkT, ch * kChunkH, cw * kChunkW);
+        n_tok = add_box(ct * kChunkT, ch * kChunkH, cw * sd.bw);
     } else {
         for (int bt = 0; bt < sd.mt; ++bt)
             for (int bhh = 0; bhh < sd.mh; ++bhh)
                 for (int bw = 0; bw < sd.mw; ++bw)
                     n_tok += add_box((ct * sd.mt + bt) * kChunkT, (ch * sd.mh + bhh) * kChunkH,
-                                     (cw * sd.mw + bw) * kChunkW);
+                                     (cw * sd.mw + bw) * sd.bw);
     }
     const int grp = tid / VPT;
 #pragma unroll
@@ -590,6 +596,111 @@ __global__ void __launch_bounds__(256) expand_emit_kernel(const int32_t* __restr
     }
 }
 
+// ------------------------------------------------------------------------
+// 64-token query chunks: the attention kernel works on (4,4,8) boxes of
+// queries, i.e. on the two w-adjacent query chunks of a box at once. Each box
+// row lists the union of the key boxes its two chunks selected, in ascending
+// order, with a 4-bit quadrant pattern per entry: bits 0-1 are the key halves
+// (lw < 4, lw >= 4) the box's left query chunk attends to, bits 2-3 those of
+// its right query chunk. One thread per box row merges the two sorted chunk
+// rows (a key chunk's box index grows with the key chunk index).
+struct QuadGrid {
+    int NH, NW, NWq;   // boxes along h, w; query chunks along w
+    int NkW;           // key chunks along w
+    int kw64;          // key chunks are (4,4,4) half-boxes (else whole boxes)
+    int Nq, Nk, NB;    // query chunks, key chunks, boxes per (batch, head)
+    int64_t rows;      // box rows: batch*heads * NB
+};
+
+__device__ __forceinline__ void key_box_of(const QuadGrid& g, int kc, int& box, int& bits) {
+    if (g.kw64) {
+        const int kt = kc / (g.NH * g.NkW), kh = (kc / g.NkW) % g.NH, kw4 = kc % g.NkW;
+        box = (kt * g.NH + kh) * g.NW + (kw4 >> 1);
+        bits = 1 << (kw4 & 1);
+    } else {
+        box = kc;
+        bits = 3;
+    }
+}
+
+template <bool kEmit>
+__global__ void __launch_bounds__(256) quad_union_kernel(
+    const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx, int64_t col_cap,
+    QuadGrid g, int32_t* __restrict__ counts, const int32_t* __restrict__ box_row_ptr,
+    int32_t* __restrict__ box_col, uint8_t* __restrict__ box_pat, int64_t box_cap,
+    uint32_t* status) {
+    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= g.rows) return;
+    const int64_t bh = r / g.NB;
+    const int b = (int)(r % g.NB);
+    const int bt = b / (g.NH * g.NW), bhh = (b / g.NW) % g.NH, bw = b % g.NW;
+    const int q0 = (bt * g.NH + bhh) * g.NWq + 2 * bw;  // the box's left query chunk
+    bool bad = false;
+    int64_t pos[2], end[2];
+    for (int side = 0; side < 2; ++side) {
+        pos[side] = end[side] = 0;
+        if (side == 1 && 2 * bw + 1 >= g.NWq) continue;  // no right chunk at the grid edge
+        const int64_t row = bh * g.Nq + q0 + side;
+        const int64_t beg = row_ptr[row], e = row_ptr[row + 1];
+        if (beg >= 0 && e >= beg && e <= col_cap && e - beg <= g.Nk) {
+            pos[side] = beg;
+            end[side] = e;
+        } else {
+            bad = true;
+        }
+    }
+    int64_t out = 0;
+    if (kEmit) {
+        out = box_row_ptr[r];
+        if (box_row_ptr[r + 1] > box_cap) {
+            atomicOr(status, kStatusCapacity);
+            return;
+        }
+    }
+    // next key box of a side (INT32_MAX when exhausted), skipping invalid entries
+    auto peek = [&](int side, int& box, int& bits) {
+        while (pos[side] < end[side]) {
+            const int c = col_idx[pos[side]];
+            if (c >= 0 && c < g.Nk) {
+                key_box_of(g, c, box, bits);
+                return;
+            }
+            bad = true;
+            ++pos[side];
+        }
+        box = INT32_MAX;
+        bits = 0;
+    };
+    int n = 0, prev = -1;
+    while (true) {
+        int b0, t0, b1, t1;
+        peek(0, b0, t0);
+        peek(1, b1, t1);
+        const int bx = b0 < b1 ? b0 : b1;
+        if (bx == INT32_MAX) break;
+        int pat = 0;
+        // every entry of either row in box bx (a row holds at most its two halves)
+        for (int side = 0; side < 2; ++side) {
+            while (true) {
+                int bb, bits;
+                peek(side, bb, bits);
+                if (bb != bx) break;
+                pat |= bits << (2 * side);
+                ++pos[side];
+            }
+        }
+        if (bx <= prev) bad = true;  // a row that is not ascending
+        prev = bx;
+        if (kEmit) {
+            box_col[out + n] = bx;
+            box_pat[out + n] = static_cast<uint8_t>(pat);
+        }
+        ++n;
+    }
+    if (!kEmit) counts[r] = n;
+    if (bad) atomicOr(status, kStatusBadIndex);
+}
+
 // One CTA waits on an mbarrier that nothing arrives at; the bounded wait
 // expires, records the timeout and the kernel returns normally.
 __global__ void selftest_timeout_kernel(uint32_t* status, uint64_t timeout_ns) {
@@ -611,8 +722,8 @@ cudaError_t launch_pool(const Dims& g, const void* x0, const void* x1, float* p0
                         cudaStream_t st) {
     // with two tensors (plan): x0 = Q pools the computed query chunks, x1 = K
     // pools every key chunk; with one tensor it pools every query chunk of x0
-    const PoolSide sq{x1 ? g.q_skip : 0, x1 ? g.Nq : g.Nc, 1, 1, 1, g.NH, g.NW};
-    const PoolSide sk{0, g.Nk, g.mT, g.mH, g.mW, g.NkH, g.NkW};
+    const PoolSide sq{x1 ? g.q_skip : 0, x1 ? g.Nq : g.Nc, 1, 1, 1, g.NH, g.NWq, g.qw};
+    const PoolSide sk{0, g.Nk, g.mT, g.mH, g.mW, g.NkH, g.NkW, g.kw64 ? kChunkW / 2 : kChunkW};
     const int nx = x1 ? (g.Nq > g.Nk ? g.Nq : g.Nk) : g.Nc;
     dim3 grid((unsigned)nx, (unsigned)g.BH, x1 ? 2 : 1);
     const auto* a = static_cast<const __nv_bfloat16*>(x0);
@@ -697,6 +808,24 @@ cudaError_t launch_expand_boxes(const Dims& g, const int32_t* kc_row_ptr,
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     expand_emit_kernel<<<blocks, 256, 0, st>>>(kc_row_ptr, kc_col_idx, g.rows, bg, row_ptr,
                                                col_idx, col_cap, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quad_union(const Dims& g, const int32_t* row_ptr, const int32_t* col_idx,
+                              int64_t col_cap, int32_t* counts, int32_t* box_row_ptr,
+                              int32_t* box_col, uint8_t* box_pat, int64_t box_cap,
+                              uint32_t* status, cudaStream_t st) {
+    const QuadGrid qg{g.NH, g.NW, g.NWq, g.NkW, g.kw64, g.Nq, g.Nk, g.NB, g.BH * g.NB};
+    const unsigned blocks = (unsigned)((qg.rows + 255) / 256);
+    quad_union_kernel<false><<<blocks, 256, 0, st>>>(row_ptr, col_idx, col_cap, qg, counts,
+                                                     nullptr, nullptr, nullptr, 0, status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    scan_counts_kernel<<<1, 1024, 0, st>>>(counts, qg.rows, box_row_ptr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    quad_union_kernel<true><<<blocks, 256, 0, st>>>(row_ptr, col_idx, col_cap, qg, counts,
+                                                    box_row_ptr, box_col, box_pat, box_cap,
+                                                    status);
     return cudaGetLastError();
 }
 

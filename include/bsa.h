@@ -111,7 +111,8 @@ typedef struct {
 } bsa_params;
 
 /* Library version: major*10000 + minor*100 + patch (0.2.0: bsa_shape_info and
- * bsa_forward_host added). */
+ * bsa_forward_host added; 0.3.0: 64-token chunks, bsa_forward_partial and
+ * bsa_lse_merge_f32). */
 BSA_API int bsa_version(void);
 
 /* Text for a status code (static storage; never NULL). */

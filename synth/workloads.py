@@ -27,6 +27,7 @@ class Workload:
     t_cond: int = 0             # latent frames of condition tokens (block-causal mask)
     q_begin: int = 0            # first latent frame whose queries are computed (KV-cached step)
     kchunk: tuple = (4, 4, 8)   # key chunk shape (multiples of the (4,4,8) query chunk)
+    qchunk: tuple = (4, 4, 8)   # query chunk shape: (4,4,8), or (4,4,4) for 64-token chunks
     scale: float = 0.0          # softmax scale; 0 = 1/sqrt(d)
     tfreq_mult: float = 1.0     # temporal frequency multiplier of the smooth field
     seed: int = 0
@@ -51,18 +52,24 @@ class Workload:
 
     @property
     def NW(self) -> int:
+        """(4,4,8) boxes along w."""
         return -(-self.W // 8)
 
     @property
+    def NWq(self) -> int:
+        """Query chunks along w."""
+        return -(-self.W // self.qchunk[2])
+
+    @property
     def Nc(self) -> int:
-        """Chunks per (batch, head): ceil(T/4) * ceil(H/4) * ceil(W/8); edge chunks of a
-        grid that is not a multiple of (4, 4, 8) are partial."""
-        return -(-self.T // 4) * self.NH * self.NW
+        """Query chunks per (batch, head): ceil(T/4) * ceil(H/4) * ceil(W/qw); edge
+        chunks of a grid that is not a multiple of the chunk shape are partial."""
+        return -(-self.T // 4) * self.NH * self.NWq
 
     @property
     def n_cond(self) -> int:
         """Condition chunks: chunks whose 4 frames all lie below t_cond."""
-        return (self.t_cond // 4) * self.NH * self.NW
+        return (self.t_cond // 4) * self.NH * self.NWq
 
     @property
     def Nk(self) -> int:
@@ -79,7 +86,7 @@ class Workload:
     @property
     def q_skip(self) -> int:
         """Query chunks before q_begin (not computed)."""
-        return (self.q_begin // 4) * self.NH * self.NW
+        return (self.q_begin // 4) * self.NH * self.NWq
 
     @property
     def Nq(self) -> int:
@@ -122,6 +129,10 @@ WORKLOADS = {
     # bounded by k = 45, so each rule decides part of the rows
     "720p_topk_cdf": Workload("720p_topk_cdf", B=1, heads=32, T=24, H=48, W=80, d=128,
                               mode="topk_cdf", topk=45, cdf_p=0.1, cdf_cap_frac=0.25),
+    # 64-token query and key chunks (4,4,4) over the 720p-like grid ([P1] block-size
+    # robustness): 1,440 chunks per head, keep 90 (93.75 %)
+    "720p_q64": Workload("720p_q64", B=1, heads=32, T=24, H=48, W=80, d=128, topk=90,
+                         qchunk=(4, 4, 4), kchunk=(4, 4, 4)),
     # the same video-continuation input at a later denoising step: the condition
     # frames' K/V are cached, only the noisy queries (frames >= 8) are computed
     "causal_cdf_kv": Workload("causal_cdf_kv", B=2, heads=32, T=24, H=48, W=80, d=128,

@@ -42,7 +42,7 @@ def test_library_exports_nothing_else():
 
 
 def test_version_and_strings(L):
-    assert bsa.bsa_version() == 200
+    assert bsa.bsa_version() == 300
     for code in range(0, 10):
         s = bsa.status_string(code)
         assert s and s != "unknown status"
@@ -122,6 +122,64 @@ def test_key_chunk_shape_validation(L, kchunk, code):
     assert rc_sizes(P(T=16, H=16, W=32, kchunk=kchunk))[0] == code
 
 
+def test_plan_sizes_64_token_chunks(L):
+    # 720p-like grid in 64-token chunks: 6 x 12 x 20 = 1,440 query chunks per head
+    q64 = dict(heads=32, T=24, H=48, W=80, d=128, chunk=(4, 4, 4))
+    rc, rows, nnz = rc_sizes(P(topk=90, **q64))
+    assert (rc, rows, nnz) == (0, 32 * 1440, 32 * 1440 * 90)
+    # with 128-token key chunks: 720 key chunks
+    rc, rows, nnz = rc_sizes(P(topk=45, kchunk=(4, 4, 8), **q64))
+    assert (rc, rows, nnz) == (0, 32 * 1440, 32 * 1440 * 45)
+    # block-causal CDF: 480 condition chunks capped at 120, 960 noisy capped at 360
+    rc, rows, nnz = rc_sizes(P(mode="cdf", t_cond=8, **q64))
+    assert (rc, rows, nnz) == (0, 32 * 1440, 32 * (480 * 120 + 960 * 360))
+    # the plan's workspace also holds the forward's CSR over (4,4,8) boxes: a row per
+    # query box (720 per head) and at most the chunk CSR's entries
+    p = P(topk=90, **q64)
+    base = 256 + 2 * 32 * 1440 * 128 * 4 + 32 * 1440 * 1440 * 4
+    assert bsa.bsa_workspace_size(p) >= base + 32 * 720 * 8 + 32 * 1440 * 90 * 5
+    si = bsa.bsa_shape_info(p)
+    assert (si.Nc, si.Nq, si.Nk, si.rows) == (1440, 1440, 1440, 32 * 1440)
+    # W = 20: 5 chunk columns of 4 (boxes: 3, the last holding one chunk)
+    assert rc_sizes(P(heads=1, T=4, H=4, W=20, topk=2, chunk=(4, 4, 4)))[:2] == (0, 5)
+    # partial chunks: W = 10 -> 3 chunk columns, the last of 2 tokens
+    assert rc_sizes(P(heads=1, T=4, H=4, W=10, topk=2, chunk=(4, 4, 4)))[:2] == (0, 3)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(chunk=(4, 4, 4)), 0),
+    (dict(chunk=(4, 4, 4), kchunk=(4, 4, 8)), 0),
+    (dict(chunk=(4, 4, 4), kchunk=(4, 8, 8)), bsa.BSA_ERR_UNSUPPORTED),   # not (4,4,4)/(4,4,8)
+    (dict(chunk=(4, 4, 4), kchunk=(8, 4, 4)), bsa.BSA_ERR_UNSUPPORTED),
+    (dict(chunk=(4, 4, 4), q_begin=4), bsa.BSA_ERR_UNSUPPORTED),          # every row computed
+    (dict(chunk=(4, 4, 4), q_end=8), bsa.BSA_ERR_UNSUPPORTED),
+    (dict(chunk=(4, 4, 2)), bsa.BSA_ERR_UNSUPPORTED),
+    (dict(chunk=(4, 4, 16)), bsa.BSA_ERR_UNSUPPORTED),
+    (dict(chunk=(8, 4, 4)), bsa.BSA_ERR_UNSUPPORTED),
+])
+def test_query_chunk_shape_validation(L, kw, code):
+    assert rc_sizes(P(T=16, H=16, W=32, **kw))[0] == code
+
+
+def test_64_token_chunks_limits_and_forward_only_entries(L):
+    # chunks per (batch, head) are limited to 2,048: the long grid in 64-token chunks
+    # (14 x 12 x 20 = 3,360) is not supported
+    assert rc_sizes(P(T=56, H=48, W=80, d=128, topk=5, chunk=(4, 4, 4)))[0] == \
+        bsa.BSA_ERR_UNSUPPORTED
+    p = P(T=16, H=16, W=32, chunk=(4, 4, 4))
+    x = vp(FAKE)
+    assert L.bsa_backward_workspace_size(ctypes.byref(p)) == 0
+    assert L.bsa_backward(ctypes.byref(p), x, x, x, x, x, x, x, x, 64, x, 1 << 20, x, x, x,
+                          None) == bsa.BSA_ERR_UNSUPPORTED
+    assert L.bsa_rearrange(ctypes.byref(p), x, x, 0, None) == bsa.BSA_ERR_UNSUPPORTED
+    assert L.bsa_select_pooled(ctypes.byref(p), x, x, 0, x, 1 << 30, x, x, 1 << 20, None) == \
+        bsa.BSA_ERR_UNSUPPORTED
+    # the forward needs the plan's workspace (it builds the box CSR there)
+    ws = bsa.bsa_workspace_size(p)
+    assert L.bsa_forward(ctypes.byref(p), x, x, x, x, x, 64, x, ws - 1, x, None, None) == \
+        bsa.BSA_ERR_WORKSPACE_TOO_SMALL
+
+
 def test_key_chunk_needs_t_cond_multiple(L):
     assert rc_sizes(P(T=16, H=16, W=32, t_cond=4, kchunk=(8, 4, 8)))[0] == bsa.BSA_ERR_SHAPE
     assert rc_sizes(P(T=16, H=16, W=32, t_cond=8, kchunk=(8, 4, 8)))[0] == 0
@@ -179,10 +237,11 @@ def test_size_limits_at_their_boundaries(L):
         bsa.BSA_ERR_UNSUPPORTED                                               # exactly 2^31
 
 
-def test_chunk_shape_other_than_448_unsupported(L):
-    p = P()
-    p.chunk_w = 4
-    assert rc_sizes(p)[0] == bsa.BSA_ERR_UNSUPPORTED
+def test_chunk_shapes_other_than_448_and_444_unsupported(L):
+    for shape in ((4, 4, 6), (4, 8, 8), (2, 4, 8), (4, 4, 12)):
+        p = P()
+        p.chunk_t, p.chunk_h, p.chunk_w = shape
+        assert rc_sizes(p)[0] == bsa.BSA_ERR_UNSUPPORTED, shape
 
 
 def test_workspace_size_layout(L):

@@ -32,6 +32,9 @@ CASES = [
     (T_.with_(B=1, heads=3, T=16, H=16, W=32, d=128, mode="cdf", t_cond=8, q_begin=8), 2, 2),
     # key chunks of 512 tokens, one slot
     (T_.with_(B=1, heads=3, T=8, H=16, W=32, d=128, topk=2, kchunk=(8, 8, 8)), 2, 1),
+    # 64-token query and key chunks
+    (T_.with_(B=1, heads=3, T=8, H=16, W=20, d=64, topk=5, qchunk=(4, 4, 4), kchunk=(4, 4, 4)),
+     2, 2),
 ]
 
 

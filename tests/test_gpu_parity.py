@@ -62,6 +62,22 @@ SMALL = {
                                        t_cond=8, scale=0.3),
     "scale_flat_topk": W["tiny"].with_(name="scale_flat_topk", heads=2, T=8, H=16, W=32, d=64,
                                        topk=5, scale=0.02),
+    # 64-token query and key chunks (4,4,4): the kernel's tile is a (4,4,8) box of two
+    # query chunks over the union of their key boxes, masked per quadrant
+    "q64_k64": W["tiny"].with_(name="q64_k64", heads=2, T=8, H=16, W=32, d=128, topk=6,
+                               qchunk=(4, 4, 4), kchunk=(4, 4, 4)),
+    "q64_k128": W["tiny"].with_(name="q64_k128", heads=2, T=8, H=16, W=32, d=64, topk=4,
+                                qchunk=(4, 4, 4), kchunk=(4, 4, 8)),
+    # W = 20: the last box holds one query chunk; block-causal CDF
+    "q64_odd_w_causal_cdf": W["tiny"].with_(name="q64_odd_w_causal_cdf", B=2, heads=2, T=12,
+                                            H=16, W=20, d=128, mode="cdf", cdf_p=0.9,
+                                            cdf_cap_frac=0.25, t_cond=4, qchunk=(4, 4, 4),
+                                            kchunk=(4, 4, 4)),
+    # partial chunks in h and w (H = 13, W = 30: the last chunk column holds 2 tokens)
+    "q64_partial_topk_cdf": W["tiny"].with_(name="q64_partial_topk_cdf", heads=2, T=10, H=13,
+                                            W=30, d=64, mode="topk_cdf", topk=7, cdf_p=0.3,
+                                            cdf_cap_frac=0.5, qchunk=(4, 4, 4),
+                                            kchunk=(4, 4, 4)),
 }
 
 
@@ -88,12 +104,14 @@ def run_gpu(wl, q, k, v):
 
 
 def gather_rows(x_bhnd, wl, rows):
-    """[B,Hh,N,d] (numpy) -> [len(rows), 128, d] in chunk-local order; NaN for the
-    slots of a partial edge chunk past the grid."""
+    """[B,Hh,N,d] (numpy) -> [len(rows), slots, d] in chunk-local order (slots: the
+    query chunk's tokens, 128 or 64); NaN for the slots of a partial edge chunk past
+    the grid."""
     flat = x_bhnd.reshape(wl.B * wl.heads, wl.N, -1)
-    out = np.full((len(rows), 128, flat.shape[-1]), np.nan)
+    qc = tuple(getattr(wl, "qchunk", (4, 4, 8)))
+    out = np.full((len(rows), qc[0] * qc[1] * qc[2], flat.shape[-1]), np.nan)
     for n, r in enumerate(rows):
-        tok = oracle.chunk_tokens(wl.T, wl.H, wl.W, r % wl.Nc)
+        tok = oracle.chunk_tokens(wl.T, wl.H, wl.W, r % wl.Nc, qc)
         ok = tok >= 0
         out[n][ok] = flat[r // wl.Nc][tok[ok]]
     return out
@@ -122,13 +140,18 @@ def check_case(wl, rows=None, qkv=None):
     scale = wl.softmax_scale
     rp, ci, out, lse, status = run_gpu(wl, q, k, v)
     assert status == bsa.BSA_OK, bsa.status_string(status)
-    kchunk = tuple(wl.kchunk)
+    kchunk, qchunk = tuple(wl.kchunk), tuple(wl.qchunk)
+    q64 = qchunk == (4, 4, 4)
     # selection: oracle decides in fp32 (the kernel's precision); ties judged in fp64
     o_rp, o_ci, _ = oracle.plan(q, k, wl.T, wl.H, wl.W, scale, wl.mode, wl.topk, wl.cdf_p,
-                                wl.cdf_cap_frac, wl.t_cond, fp32=True, kchunk=kchunk)
-    S64 = oracle.scores(oracle.pool(q, wl.T, wl.H, wl.W),
+                                wl.cdf_cap_frac, wl.t_cond, fp32=True, kchunk=kchunk,
+                                qchunk=qchunk)
+    S64 = oracle.scores(oracle.pool(q, wl.T, wl.H, wl.W, chunk=qchunk),
                         oracle.pool(k, wl.T, wl.H, wl.W, chunk=kchunk), scale)
-    g_rp, g_ci = (rp, ci) if kchunk == (4, 4, 8) else boxes_to_key_chunks(rp, ci, wl)
+    # the plan's CSR lists key chunks, except with larger key chunks of 128-token query
+    # chunks, where it lists the (4,4,8) boxes they cover
+    direct = kchunk == (4, 4, 8) or q64
+    g_rp, g_ci = (rp, ci) if direct else boxes_to_key_chunks(rp, ci, wl)
     n_checked, n_diff = compare_csr(g_rp, g_ci, o_rp, o_ci, S64, wl.Nc, wl.n_cond, wl.mode,
                                     wl.cdf_p, wl.cdf_cap_frac, topk=wl.topk, Nk=wl.Nk,
                                     n_cond_k=wl.n_cond_k)
@@ -136,7 +159,8 @@ def check_case(wl, rows=None, qkv=None):
     # attention on the GPU's own CSR
     if rows is None:
         rows = np.arange(wl.rows)
-    o_out, o_lse = oracle.attend(q, k, v, wl.T, wl.H, wl.W, scale, rp, ci, rows)
+    o_out, o_lse = oracle.attend(q, k, v, wl.T, wl.H, wl.W, scale, rp, ci, rows,
+                                 **(dict(kchunk=kchunk, qchunk=qchunk) if q64 else {}))
     g_out = gather_rows(host_f32(out), wl, rows)
     mx, mean = compare_attention(g_out, o_out)
     assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
@@ -382,10 +406,47 @@ def _sample_rows(wl, per_head, seed=0):
 @pytest.mark.parametrize("name,per_head", [("480p", 224), ("720p", 64), ("long", 16),
                                            ("causal_cdf", 16), ("720p_r8", 4),
                                            ("720p_topk_cdf", 4), ("720p_real", 4),
-                                           ("480p_real", 4), ("720p_k512", 4)])
+                                           ("480p_real", 4), ("720p_k512", 4),
+                                           ("720p_q64", 16)])
 def test_full_size_workloads(name, per_head):
     wl = W[name]
     check_case(wl, rows=_sample_rows(wl, per_head))
+
+
+def test_64_token_chunks_caller_csr_with_an_empty_half():
+    """A caller CSR where one of the two query chunks of a box selects nothing: its
+    rows are zeros with LSE -inf while its neighbour's rows are exact; out-of-order
+    rows are reported."""
+    wl = SMALL["q64_k64"].with_(heads=1)
+    q, k, v = synth.make_qkv(wl)
+    p = bsa.params_for(wl)
+    pl = bsa.allocate(p)
+    nc = wl.Nc                                  # 2 x 4 x 8 = 64 query chunks
+    rows = [[] if i % 3 == 1 else sorted({(i * 7) % nc, (i * 5 + 3) % nc, i}) for i in range(nc)]
+    rp = np.concatenate([[0], np.cumsum([len(r) for r in rows])]).astype(np.int32)
+    ci = np.concatenate([np.array(r, dtype=np.int32) for r in rows]).astype(np.int32)
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    out = torch.full_like(qd, 7.0)
+    lse = torch.zeros((1, 1, wl.N), dtype=torch.float32, device="cuda")
+    bsa.bsa_forward(p, qd, kd, vd, torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda(),
+                    pl.workspace, out, lse)
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_OK
+    full = [i for i in range(nc) if rows[i]]
+    o_out, o_lse = oracle.attend(q, k, v, wl.T, wl.H, wl.W, wl.softmax_scale, rp, ci, full,
+                                 kchunk=(4, 4, 4), qchunk=(4, 4, 4))
+    mx, mean = compare_attention(gather_rows(host_f32(out), wl, full), o_out)
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+    g_lse = gather_rows(lse.cpu().numpy()[..., None], wl, full)[..., 0]
+    np.testing.assert_allclose(g_lse, o_lse, rtol=0, atol=2e-3)
+    empty = [i for i in range(nc) if not rows[i]]
+    assert np.all(gather_rows(host_f32(out), wl, empty) == 0)
+    assert np.all(np.isneginf(gather_rows(lse.cpu().numpy()[..., None], wl, empty)))
+    # a row out of order is reported (and still computed)
+    ci_bad = ci.copy()
+    ci_bad[0], ci_bad[1] = ci[1], ci[0]
+    bsa.bsa_forward(p, qd, kd, vd, torch.from_numpy(rp).cuda(), torch.from_numpy(ci_bad).cuda(),
+                    pl.workspace, out, lse)
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_ERR_DEVICE_BAD_INDEX
 
 
 def test_grid_of_1920_chunks():
