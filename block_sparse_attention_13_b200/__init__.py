@@ -526,18 +526,23 @@ def backward(pl: Plan, q, k, v, out, lse, dout, workspace=None, dq=None, dk=None
 
 
 def block_sparse_attention(q, k, v, topk=None, mode="topk", cdf_p=0.9, cdf_cap_frac=0.25,
-                           t_cond=0, grid=None, want_lse=False):
+                           t_cond=0, grid=None, want_lse=False, chunk=(4, 4, 8), kchunk=(0, 0, 0),
+                           scale=0.0):
     """One call: plan + forward for q, k, v [B, heads, T*H*W, d] bf16 on the GPU.
 
-    grid = (T, H, W) of the latent video. Returns out (and lse if asked).
+    grid = (T, H, W) of the latent video; chunk = the query chunk shape, (4, 4, 8) or
+    (4, 4, 4); kchunk = the key chunk shape (0 = the query chunk's). Returns out (and
+    lse if asked).
     """
     import torch
     B, heads, N, d = q.shape
     T, H, W = grid
     assert T * H * W == N
     if topk is None:  # 1/16 of the key chunks (ceil counts: edge chunks may be partial)
-        topk = max(1, (-(-T // 4) * -(-H // 4) * -(-W // 8)) // 16)
-    p = make_params(B, heads, T, H, W, d, mode, topk, cdf_p, cdf_cap_frac, t_cond)
+        kc = tuple(c if c else q_ for c, q_ in zip(kchunk, chunk))
+        topk = max(1, (-(-T // kc[0]) * -(-H // kc[1]) * -(-W // kc[2])) // 16)
+    p = make_params(B, heads, T, H, W, d, mode, topk, cdf_p, cdf_cap_frac, t_cond, scale=scale,
+                    kchunk=kchunk, chunk=chunk)
     pl = plan(p, q, k)
     lse = torch.empty((B, heads, N), dtype=torch.float32, device=q.device) if want_lse else None
     out = forward(pl, q, k, v, lse=lse)

@@ -602,8 +602,10 @@ __global__ void __launch_bounds__(256) expand_emit_kernel(const int32_t* __restr
 // row lists the union of the key boxes its two chunks selected, in ascending
 // order, with a 4-bit quadrant pattern per entry: bits 0-1 are the key halves
 // (lw < 4, lw >= 4) the box's left query chunk attends to, bits 2-3 those of
-// its right query chunk. One thread per box row merges the two sorted chunk
-// rows (a key chunk's box index grows with the key chunk index).
+// its right query chunk. One warp per box row: its lanes read the two chunk
+// rows (coalesced) into four bitmaps over the key boxes, one per quadrant, in
+// shared memory; the union is their OR, emitted in ascending box order. The
+// order of a row's entries does not matter and duplicates collapse.
 struct QuadGrid {
     int NH, NW, NWq;   // boxes along h, w; query chunks along w
     int NkW;           // key chunks along w
@@ -611,6 +613,8 @@ struct QuadGrid {
     int Nq, Nk, NB;    // query chunks, key chunks, boxes per (batch, head)
     int64_t rows;      // box rows: batch*heads * NB
 };
+
+constexpr int kQuadMaxWords = 64;  // 32-bit words per quadrant bitmap: up to 2,048 key boxes
 
 __device__ __forceinline__ void key_box_of(const QuadGrid& g, int kc, int& box, int& bits) {
     if (g.kw64) {
@@ -629,76 +633,77 @@ __global__ void __launch_bounds__(256) quad_union_kernel(
     QuadGrid g, int32_t* __restrict__ counts, const int32_t* __restrict__ box_row_ptr,
     int32_t* __restrict__ box_col, uint8_t* __restrict__ box_pat, int64_t box_cap,
     uint32_t* status) {
-    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (r >= g.rows) return;
+    __shared__ uint32_t bitmap[8][4][kQuadMaxWords];  // [warp][quadrant][word]
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int64_t r = (int64_t)blockIdx.x * 8 + wib;
+    if (r >= g.rows) return;  // warp-uniform
+    uint32_t (*bm)[kQuadMaxWords] = bitmap[wib];
+    const int words = (g.NB + 31) >> 5;
+    for (int w = lane; w < words; w += 32)
+        for (int qd = 0; qd < 4; ++qd) bm[qd][w] = 0u;
+    __syncwarp();
     const int64_t bh = r / g.NB;
     const int b = (int)(r % g.NB);
     const int bt = b / (g.NH * g.NW), bhh = (b / g.NW) % g.NH, bw = b % g.NW;
     const int q0 = (bt * g.NH + bhh) * g.NWq + 2 * bw;  // the box's left query chunk
     bool bad = false;
-    int64_t pos[2], end[2];
     for (int side = 0; side < 2; ++side) {
-        pos[side] = end[side] = 0;
         if (side == 1 && 2 * bw + 1 >= g.NWq) continue;  // no right chunk at the grid edge
         const int64_t row = bh * g.Nq + q0 + side;
-        const int64_t beg = row_ptr[row], e = row_ptr[row + 1];
-        if (beg >= 0 && e >= beg && e <= col_cap && e - beg <= g.Nk) {
-            pos[side] = beg;
-            end[side] = e;
-        } else {
+        const int64_t beg = row_ptr[row], end = row_ptr[row + 1];
+        if (!(beg >= 0 && end >= beg && end <= col_cap && end - beg <= g.Nk)) {
             bad = true;
+            continue;
+        }
+        for (int64_t e = beg + lane; e < end; e += 32) {
+            const int c = col_idx[e];
+            if (c < 0 || c >= g.Nk) {
+                bad = true;
+                continue;
+            }
+            int box, bits;
+            key_box_of(g, c, box, bits);
+            for (int kh = 0; kh < 2; ++kh)
+                if (bits & (1 << kh)) atomicOr(&bm[2 * side + kh][box >> 5], 1u << (box & 31));
         }
     }
-    int64_t out = 0;
-    if (kEmit) {
-        out = box_row_ptr[r];
-        if (box_row_ptr[r + 1] > box_cap) {
-            atomicOr(status, kStatusCapacity);
-            return;
-        }
+    __syncwarp();
+    if (kEmit && box_row_ptr[r + 1] > box_cap) {
+        if (lane == 0) atomicOr(status, kStatusCapacity);
+        return;
     }
-    // next key box of a side (INT32_MAX when exhausted), skipping invalid entries
-    auto peek = [&](int side, int& box, int& bits) {
-        while (pos[side] < end[side]) {
-            const int c = col_idx[pos[side]];
-            if (c >= 0 && c < g.Nk) {
-                key_box_of(g, c, box, bits);
-                return;
-            }
-            bad = true;
-            ++pos[side];
+    int64_t run = kEmit ? box_row_ptr[r] : 0;
+    int total = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {  // ascending: word w0 + lane per round
+        const int w = w0 + lane;
+        const uint32_t a0 = w < words ? bm[0][w] : 0u, a1 = w < words ? bm[1][w] : 0u;
+        const uint32_t a2 = w < words ? bm[2][w] : 0u, a3 = w < words ? bm[3][w] : 0u;
+        uint32_t any = a0 | a1 | a2 | a3;
+        const int n = __popc(any);
+        int incl = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
         }
-        box = INT32_MAX;
-        bits = 0;
-    };
-    int n = 0, prev = -1;
-    while (true) {
-        int b0, t0, b1, t1;
-        peek(0, b0, t0);
-        peek(1, b1, t1);
-        const int bx = b0 < b1 ? b0 : b1;
-        if (bx == INT32_MAX) break;
-        int pat = 0;
-        // every entry of either row in box bx (a row holds at most its two halves)
-        for (int side = 0; side < 2; ++side) {
-            while (true) {
-                int bb, bits;
-                peek(side, bb, bits);
-                if (bb != bx) break;
-                pat |= bits << (2 * side);
-                ++pos[side];
-            }
-        }
-        if (bx <= prev) bad = true;  // a row that is not ascending
-        prev = bx;
         if (kEmit) {
-            box_col[out + n] = bx;
-            box_pat[out + n] = static_cast<uint8_t>(pat);
+            int64_t pos = run + (incl - n);
+            while (any) {
+                const int bit = __ffs(any) - 1;
+                any &= any - 1;
+                const uint32_t m = 1u << bit;
+                box_col[pos] = w * 32 + bit;
+                box_pat[pos] = static_cast<uint8_t>(((a0 & m) ? 1 : 0) | ((a1 & m) ? 2 : 0) |
+                                                    ((a2 & m) ? 4 : 0) | ((a3 & m) ? 8 : 0));
+                ++pos;
+            }
         }
-        ++n;
+        const int round = __shfl_sync(0xffffffffu, incl, 31);
+        run += round;
+        total += round;
     }
-    if (!kEmit) counts[r] = n;
-    if (bad) atomicOr(status, kStatusBadIndex);
+    if (!kEmit && lane == 0) counts[r] = total;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, kStatusBadIndex);
 }
 
 // One CTA waits on an mbarrier that nothing arrives at; the bounded wait
@@ -816,7 +821,8 @@ cudaError_t launch_quad_union(const Dims& g, const int32_t* row_ptr, const int32
                               int32_t* box_col, uint8_t* box_pat, int64_t box_cap,
                               uint32_t* status, cudaStream_t st) {
     const QuadGrid qg{g.NH, g.NW, g.NWq, g.NkW, g.kw64, g.Nq, g.Nk, g.NB, g.BH * g.NB};
-    const unsigned blocks = (unsigned)((qg.rows + 255) / 256);
+    if (g.NB > 32 * kQuadMaxWords) return cudaErrorInvalidValue;  // not reachable: NB <= Nc
+    const unsigned blocks = (unsigned)((qg.rows + 7) / 8);          // a warp per box row
     quad_union_kernel<false><<<blocks, 256, 0, st>>>(row_ptr, col_idx, col_cap, qg, counts,
                                                      nullptr, nullptr, nullptr, 0, status);
     cudaError_t e = cudaGetLastError();

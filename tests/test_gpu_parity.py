@@ -415,8 +415,7 @@ def test_full_size_workloads(name, per_head):
 
 def test_64_token_chunks_caller_csr_with_an_empty_half():
     """A caller CSR where one of the two query chunks of a box selects nothing: its
-    rows are zeros with LSE -inf while its neighbour's rows are exact; out-of-order
-    rows are reported."""
+    rows are zeros with LSE -inf while its neighbour's rows are exact."""
     wl = SMALL["q64_k64"].with_(heads=1)
     q, k, v = synth.make_qkv(wl)
     p = bsa.params_for(wl)
@@ -441,12 +440,37 @@ def test_64_token_chunks_caller_csr_with_an_empty_half():
     empty = [i for i in range(nc) if not rows[i]]
     assert np.all(gather_rows(host_f32(out), wl, empty) == 0)
     assert np.all(np.isneginf(gather_rows(lse.cpu().numpy()[..., None], wl, empty)))
-    # a row out of order is reported (and still computed)
-    ci_bad = ci.copy()
-    ci_bad[0], ci_bad[1] = ci[1], ci[0]
-    bsa.bsa_forward(p, qd, kd, vd, torch.from_numpy(rp).cuda(), torch.from_numpy(ci_bad).cuda(),
-                    pl.workspace, out, lse)
-    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_ERR_DEVICE_BAD_INDEX
+    # the union of a box's rows does not depend on the order of their entries:
+    # a shuffled row and a repeated entry give the same output bit for bit
+    ci_shuf = ci.copy()
+    ci_shuf[0], ci_shuf[1] = ci[1], ci[0]
+    ci_shuf[rp[2]] = ci_shuf[rp[2] + 1]
+    out2 = torch.full_like(qd, 7.0)
+    bsa.bsa_forward(p, qd, kd, vd, torch.from_numpy(rp).cuda(), torch.from_numpy(ci_shuf).cuda(),
+                    pl.workspace, out2)
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_OK
+    ref_rows = [r for r in range(nc) if set(rows[r]) == set(ci_shuf[rp[r]:rp[r + 1]])]
+    assert 0 in ref_rows
+    g1, g2 = gather_rows(host_f32(out), wl, ref_rows), gather_rows(host_f32(out2), wl, ref_rows)
+    assert np.array_equal(np.nan_to_num(g1), np.nan_to_num(g2))
+
+
+@pytest.mark.parametrize("name", ["causal_cdf_small", "q64_k64", "scale_sharp_cdf"])
+def test_one_call_api_equals_plan_and_forward(name):
+    """block_sparse_attention (plan + forward in one call) gives the explicit
+    calls' output bit for bit."""
+    wl = SMALL[name]
+    q, k, v = synth.make_qkv(wl)
+    rp, ci, out, lse, status = run_gpu(wl, q, k, v)
+    assert status == bsa.BSA_OK
+    o1, l1 = bsa.block_sparse_attention(dev(q), dev(k), dev(v), topk=wl.topk or None,
+                                        mode=wl.mode, cdf_p=wl.cdf_p,
+                                        cdf_cap_frac=wl.cdf_cap_frac, t_cond=wl.t_cond,
+                                        grid=(wl.T, wl.H, wl.W), want_lse=True,
+                                        chunk=tuple(wl.qchunk), kchunk=tuple(wl.kchunk),
+                                        scale=wl.scale)
+    assert torch.equal(o1.view(torch.int16), out.view(torch.int16))
+    assert torch.equal(l1, lse)
 
 
 def test_grid_of_1920_chunks():
