@@ -14,12 +14,13 @@
 //   1. prep:  D = rowsum(dO * O) and LSE * log2(e), chunk-major per query chunk;
 //   2. CSC:   the CSR block mask transposed (per key chunk, the query chunks
 //             that selected it, ascending) through a per-column bitmap;
-//   3. dQ:    one CTA per query chunk (CSR row): S = Q K^T and dP = dO V^T per
-//             selected key chunk, dS in TMEM, dQ += dS K accumulated in TMEM;
+//   3. dQ:    one CTA per query chunk (CSR row): Q and dO copied to TMEM once,
+//             then S = Q K^T and dP = dO V^T per selected key chunk, dS in
+//             TMEM, dQ += dS K accumulated in TMEM;
 //   4. dK/dV: one CTA per key chunk (CSC column): S^T = K Q^T and
-//             dP^T = V dO^T per query chunk that selected it, in two halves of
-//             64 queries so the exponentials of one half overlap the tensor
-//             core's work on the other; dV += P^T dO and dK += dS^T Q in TMEM.
+//             dP^T = V dO^T per query chunk that selected it; P^T and dS^T
+//             written back to TMEM in two phases so the exponentials overlap
+//             the tensor core's work; dV += P^T dO and dK += dS^T Q in TMEM.
 // Q, K, V, dO and the gradients stay in [T,H,W] token order; the same 5-D TMA
 // box as the forward lands one chunk in shared memory in chunk-local order.
 //
@@ -184,9 +185,9 @@ struct BwdCfg {
     static constexpr int kTmaWarp = 8;
     static constexpr int kMmaWarp = 9;
     static constexpr uint32_t kTmemCols = 512;
-    // both kernels: six tiles, then 2 KB of per-query-chunk aux, control, list
+    // every kernel: six tiles, then three 1 KB per-query-chunk aux records, control, list
     static constexpr int kAux = 6 * kTileBytes;
-    static constexpr int kCtl = kAux + 2048;
+    static constexpr int kCtl = kAux + 3 * 1024;
     static constexpr int kList = kCtl + 512;
     static constexpr int kSmemBytes = kList + kMaxList * 2 + 1024;  // + alignment slack
 };
@@ -252,28 +253,75 @@ __device__ __forceinline__ void zero_token(__nv_bfloat16* base, int64_t bh, int6
     for (int j = 0; j < D / 8; ++j) dst[j] = make_uint4(0u, 0u, 0u, 0u);
 }
 
+// An mbarrier arrive that the 32 registers r depend on, and an empty statement
+// that does the same for another 32: arithmetic on r cannot be scheduled above
+// them, so an early release (S loaded, its TMEM columns free) is not delayed
+// behind the work that follows it.
+__device__ __forceinline__ void mbar_arrive_tied(uint64_t* bar, uint32_t (&r)[32]) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%32];"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 : "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void reg_tie(uint32_t (&r)[32]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
 // exp2 of a pair: every 4th pair on the FMA-pipe polynomial, the rest on MUFU.
 __device__ __forceinline__ float2 exp2_pair(float2 x, int j) {
     return (j % 4 == 0) ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
 }
 
 // ------------------------------------------------------------------ dQ kernel
-// One CTA per CSR row (query chunk). Shared memory tiles: Q, dO, K[3], V.
-// TMEM: S slots at columns 0 and 128, dP at 256, dQ at 384. The 8 dS warps
-// split each row: warps w and w+4 share TMEM lanes 32(w%4).. and take key
-// columns [0,64) and [64,128); each writes its 32 columns of packed bf16 dS
-// over the first half of the S columns it has just read ([0,32) and [64,96)),
-// the TMEM A operand of dQ += dS K. MMA issue order per step j, once dS(j) is
-// written: dP(j+1), dQ(j), S(j+2); S(j+1) was issued a step earlier. Two
-// producer lanes keep the loads independent: lane 0 refills K slots (K(j+3)
-// after dQ(j)), lane 1 the V tile (V(j+1) after dP(j)).
+// One CTA per CSR row (query chunk). Q and dO are the A operands of every S and
+// dP of the row, so after the TMA lands them the dS warps copy both into TMEM
+// (bf16 pairs, one row per lane): S = Q K^T and dP = dO V^T then read only
+// their B operand from shared memory. TMEM: Q at columns [0,64), dO at
+// [64,128), S at [128,256), dP at [256,384), dQ at [384,512). Shared memory:
+// Q's tile (a V slot once copied), dO's tile (dQ staging at the end), a
+// three-slot K ring and a second V slot.
+//
+// The 8 dS warps split each row: warps w and w+4 share TMEM lanes 32(w%4)..
+// and take key columns [0,64) and [64,128). A step has two phases. First they
+// load S, release it (s_free: S of the next key chunk is computed in its place)
+// and compute P = exp2(S * scale * log2(e) - LSE * log2(e)) into registers;
+// then they load dP and write dS = P (dP - D) as packed bf16 over the first
+// half of their dP columns, the TMEM A operand of dQ += dS K. MMA issue order
+// per step j: S(j+1) once S(j) is loaded, dQ(j) once dS(j) is written, then
+// dP(j+1) (the tensor core executes in issue order, so dP(j+1) overwrites dS(j)
+// only after dQ(j) has read it). While the warps compute P(j+1), dQ(j) and
+// dP(j+1) are queued. Two producer lanes keep the loads independent: lane 0
+// refills K slots (K(j+3) after dQ(j)), lane 1 the V slots (V(j+2) after
+// dP(j)).
 struct __align__(8) DqCtl {
-    uint64_t qd_full, k_full[3], k_empty[3], v_full, v_empty, s_full[2];
-    uint64_t dp_full, ds_full, dq_full, aux;
+    uint64_t qd_full, qt_full, k_full[3], k_empty[3], v_full[2], v_empty[2];
+    uint64_t s_full, s_free, dp_full, ds_full, dq_full, aux;
     int n_valid;
     uint32_t tmem_base;
     int abort_flag;
 };
+
+// Copy row m of a [128][64]-per-half 128-byte-swizzled bf16 tile (the layout of
+// the 5-D TMA box), channels [64*half, 64*half + 64), into 32 TMEM columns as
+// bf16 pairs (even channel in the low half), the layout of an A operand.
+__device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int half, int m, uint32_t taddr) {
+    constexpr int kHalfBytes = 128 * 64 * 2;
+    const uint8_t* row = tile + half * kHalfBytes + m * 128;
+    uint32_t r[32];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + ((c ^ (m & 7)) << 4));
+        r[4 * c + 0] = v.x;
+        r[4 * c + 1] = v.y;
+        r[4 * c + 2] = v.z;
+        r[4 * c + 3] = v.w;
+    }
+    tmem_st32(taddr, r);
+}
 
 template <int D>
 __global__ void __launch_bounds__(320, 1)
@@ -281,13 +329,14 @@ __global__ void __launch_bounds__(320, 1)
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                       const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
     using C = BwdCfg<D>;
+    constexpr uint32_t kQt = 0, kDOt = 64, kS = 128, kDP = 256, kDQ = 384;  // TMEM columns
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t* sQ = smem;
-    uint8_t* sdO = smem + C::kTileBytes;
+    uint8_t* sQ = smem;                    // then V slot 1
+    uint8_t* sdO = smem + C::kTileBytes;   // then dQ staging
     auto sK = [&](int s) { return smem + (2 + s) * C::kTileBytes; };
-    uint8_t* sV = smem + 5 * C::kTileBytes;
+    auto sV = [&](int s) { return s == 0 ? smem + 5 * C::kTileBytes : sQ; };
     DqCtl* ctl = reinterpret_cast<DqCtl*>(smem + C::kCtl);
     uint16_t* list = reinterpret_cast<uint16_t*>(smem + C::kList);
     const int warp = threadIdx.x >> 5;
@@ -296,14 +345,17 @@ __global__ void __launch_bounds__(320, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&ctl->qd_full, 1);
+        mbar_init(&ctl->qt_full, 256);
         for (int s = 0; s < 3; ++s) {
             mbar_init(&ctl->k_full[s], 1);
             mbar_init(&ctl->k_empty[s], 1);
         }
-        mbar_init(&ctl->v_full, 1);
-        mbar_init(&ctl->v_empty, 1);
-        mbar_init(&ctl->s_full[0], 1);
-        mbar_init(&ctl->s_full[1], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&ctl->v_full[s], 1);
+            mbar_init(&ctl->v_empty[s], 1);
+        }
+        mbar_init(&ctl->s_full, 1);
+        mbar_init(&ctl->s_free, 256);
         mbar_init(&ctl->dp_full, 1);
         mbar_init(&ctl->ds_full, 256);
         mbar_init(&ctl->dq_full, 1);
@@ -392,84 +444,103 @@ __global__ void __launch_bounds__(320, 1)
                     if (nk[s] > 0) drain_wait(&ctl->k_full[s], (nk[s] - 1) & 1, tmo);
             }
         } else if (lane == 1 && n > 0) {
-            // the V tile: V(j) once dP(j-1) has read V(j-1)
-            int nv = 0;
+            // the V slots: V(0) in its own tile, V(1) in Q's once Q is in TMEM, then
+            // V(j) once dP(j-2) has read V(j-2)
+            int nv[2] = {0, 0};
             bool ok = true;
             for (int j = 0; j < n && ok; ++j) {
-                if (j >= 1 && !mbar_wait(&ctl->v_empty, (j - 1) & 1, abort_flag, a.status, tmo,
-                                         site(1, 2, 0, j))) {
+                const int s = j & 1;
+                if (j == 1 && !mbar_wait(&ctl->qt_full, 0, abort_flag, a.status, tmo, site(1, 3, 0, j))) {
+                    ok = false;
+                    break;
+                }
+                if (j >= 2 && !mbar_wait(&ctl->v_empty[s], ((j - 2) >> 1) & 1, abort_flag, a.status,
+                                         tmo, site(1, 2, s, j))) {
                     ok = false;
                     break;
                 }
                 int vt, vh, vw;
                 chunk_origin(list[j], a.NH, a.NW, vt, vh, vw);
-                mbar_arrive_expect_tx(&ctl->v_full, C::kTileBytes);
+                mbar_arrive_expect_tx(&ctl->v_full[s], C::kTileBytes);
 #pragma unroll
                 for (int c = 0; c < C::kHalves; ++c)
-                    tma_load_5d(&tm_v, smem_u32(sV) + c * C::kHalfBytes, &ctl->v_full, c * 64, vw, vh,
-                                vt, bh);
-                ++nv;
+                    tma_load_5d(&tm_v, smem_u32(sV(s)) + c * C::kHalfBytes, &ctl->v_full[s], c * 64,
+                                vw, vh, vt, bh);
+                ++nv[s];
             }
-            if ((!ok || *abort_flag) && nv > 0) drain_wait(&ctl->v_full, (nv - 1) & 1, tmo);
+            if (!ok || *abort_flag)
+                for (int s = 0; s < 2; ++s)
+                    if (nv[s] > 0) drain_wait(&ctl->v_full[s], (nv[s] - 1) & 1, tmo);
         }
         __syncwarp();
     } else if (warp == C::kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && n > 0) {
-            constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);  // both operands K-major
+            constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);  // A from TMEM, B K-major
             constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, 0, 1);    // dS from TMEM, K MN-major
             bool issued = false;
-            bool ok = mbar_wait(&ctl->qd_full, 0, abort_flag, a.status, tmo, site(2, 0, 0, 0));
+            bool ok = mbar_wait(&ctl->qt_full, 0, abort_flag, a.status, tmo, site(2, 0, 0, 0));
             if (ok) tc_fence_after();
-            auto issue_ss = [&](uint32_t dcol, uint32_t sa, uint32_t sb) {
+            // G = A B^T over the D channels: A (Q or dO) in TMEM at acol, B in shared memory
+            auto issue_tk = [&](uint32_t dcol, uint32_t acol, uint32_t sb) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-                    mma_ss(tmem + dcol, sdesc_sw128(sa + off, 16, 1024), sdesc_sw128(sb + off, 16, 1024),
-                           kIdS, kk > 0 ? 1u : 0u);
+                    mma_ts(tmem + dcol, tmem + acol + 8u * kk, sdesc_sw128(sb + off, 16, 1024), kIdS,
+                           kk > 0 ? 1u : 0u);
                 }
             };
             auto issue_s = [&](int j) -> bool {
-                const int s = j % 3, t = j & 1;
+                const int s = j % 3;
                 if (!mbar_wait(&ctl->k_full[s], (j / 3) & 1, abort_flag, a.status, tmo, site(2, 1, s, j)))
                     return false;
                 tc_fence_after();
-                issue_ss(128u * t, smem_u32(sQ), smem_u32(sK(s)));
+                issue_tk(kS, kQt, smem_u32(sK(s)));
                 issued = true;
-                tc_commit(&ctl->s_full[t]);
+                tc_commit(&ctl->s_full);
                 return true;
             };
+            // dP(j) = dO V(j)^T
             auto issue_dp = [&](int j) -> bool {
-                if (!mbar_wait(&ctl->v_full, j & 1, abort_flag, a.status, tmo, site(2, 2, 0, j)))
+                const int s = j & 1;
+                if (!mbar_wait(&ctl->v_full[s], (j >> 1) & 1, abort_flag, a.status, tmo, site(2, 2, s, j)))
                     return false;
                 tc_fence_after();
-                issue_ss(256u, smem_u32(sdO), smem_u32(sV));
+                issue_tk(kDP, kDOt, smem_u32(sV(s)));
                 issued = true;
-                tc_commit(&ctl->v_empty);
+                tc_commit(&ctl->v_empty[s]);
                 tc_commit(&ctl->dp_full);
                 return true;
             };
-            // dQ += dS(j) K(j): keys 16kk.. of dS sit at column 64*(kk/4) + 8*(kk%4) of the S slot
+            // dQ += dS(j) K(j): keys 16kk.. of dS sit at column 64*(kk/4) + 8*(kk%4) of dP's block
             auto issue_dq = [&](int j) {
-                const int s = j % 3, t = j & 1;
+                const int s = j % 3;
                 const uint32_t sk = smem_u32(sK(s));
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + 384u, tmem + 128u * t + 64u * (kk >> 2) + 8u * (kk & 3),
+                    mma_ts(tmem + kDQ, tmem + kDP + 64u * (kk >> 2) + 8u * (kk & 3),
                            sdesc_sw128(sk + kk * 2048, C::kHalfBytes, 1024), kIdQ,
                            (j > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(&ctl->k_empty[s]);
             };
-            ok = ok && issue_s(0) && issue_dp(0) && (n < 2 || issue_s(1));
+            ok = ok && issue_s(0) && issue_dp(0);
             for (int j = 0; j < n && ok; ++j) {
+                if (j + 1 < n) {
+                    // S(j) is in the dS warps' registers: compute S(j+1) in its place
+                    if (!mbar_wait(&ctl->s_free, j & 1, abort_flag, a.status, tmo, site(2, 4, 0, j))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (!issue_s(j + 1)) { ok = false; break; }
+                }
                 if (!mbar_wait(&ctl->ds_full, j & 1, abort_flag, a.status, tmo, site(2, 3, 0, j))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                if (j + 1 < n && !issue_dp(j + 1)) { ok = false; break; }
                 issue_dq(j);
-                if (j + 2 < n && !issue_s(j + 2)) { ok = false; break; }
+                if (j + 1 < n && !issue_dp(j + 1)) { ok = false; break; }
             }
             if (ok) {
                 tc_commit(&ctl->dq_full);
@@ -480,7 +551,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ dS + epilogue
+        // ------------------------------------------------------------ Q, dO to TMEM; dS; epilogue
         const int grp = warp >> 2;                    // key columns [64*grp, 64*grp + 64)
         const int m = (warp & 3) * 32 + lane;         // query row = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -492,35 +563,72 @@ __global__ void __launch_bounds__(320, 1)
         const float2 nl = make_float2(-lse2, -lse2);
         const float2 nd = make_float2(-Dm, -Dm);
         bool ok = true;
-        for (int j = 0; j < n; ++j) {
-            const int t = j & 1;
-            bool got = mbar_wait(&ctl->s_full[t], (j >> 1) & 1, abort_flag, a.status, tmo, site(3, 4, t, j));
-            got = got && mbar_wait(&ctl->dp_full, j & 1, abort_flag, a.status, tmo, site(3, 5, 0, j));
+        if (n > 0) {
+            // warp group g copies channel half g of Q and dO (D = 64: group 0 only)
+            const bool got = mbar_wait(&ctl->qd_full, 0, abort_flag, a.status, tmo, site(3, 0, 0, 0));
+            ok = __all_sync(0xffffffffu, got);
+            if (ok && grp < C::kHalves) {
+                tile_row_to_tmem(sQ, grp, m, tmem + lane_off + kQt + 32u * grp);
+                tile_row_to_tmem(sdO, grp, m, tmem + lane_off + kDOt + 32u * grp);
+                tmem_wait_st();
+            }
+            if (ok) {
+                tc_fence_before();
+                mbar_arrive(&ctl->qt_full);
+            }
+        }
+        const uint32_t tS = tmem + lane_off + kS + 64u * grp;
+        const uint32_t tP = tmem + lane_off + kDP + 64u * grp;
+        for (int j = 0; j < n && ok; ++j) {
+            // P phase
+            bool got = mbar_wait(&ctl->s_full, j & 1, abort_flag, a.status, tmo, site(3, 4, 0, j));
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t tS = tmem + lane_off + 128u * t + 64u * grp;
-            const uint32_t tP = tmem + lane_off + 256u + 64u * grp;
+            float p[64];
+            {
+                uint32_t sv0[32], sv1[32];
+                tmem_ld32(tS, sv0);
+                tmem_ld32(tS + 32, sv1);
+                tmem_wait_ld_tie(sv0);
+                tmem_wait_ld_tie(sv1);
+                // S of this step is in registers: its columns may be overwritten
+                tc_fence_before();
+                mbar_arrive_tied(&ctl->s_free, sv0);
+                reg_tie(sv1);
 #pragma unroll
-            for (int g = 0; g < 2; ++g) {
-                uint32_t sv[32], pv[32];
-                tmem_ld32(tS + g * 32, sv);
-                tmem_ld32(tP + g * 32, pv);
-                tmem_wait_ld_tie(sv);
-                tmem_wait_ld_tie(pv);
-                uint32_t pk[16];
+                for (int e = 0; e < 32; ++e) {
+                    const uint32_t* sv = e < 16 ? sv0 : sv1;
+                    const int o = 2 * (e & 15);
+                    const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[o]), __uint_as_float(sv[o + 1])),
+                                                cc, nl);
+                    const float2 pe = exp2_pair(x, e);
+                    p[2 * e] = pe.x;
+                    p[2 * e + 1] = pe.y;
+                }
+            }
+            // dS phase
+            got = mbar_wait(&ctl->dp_full, j & 1, abort_flag, a.status, tmo, site(3, 5, 0, j));
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t pk[32];
+            {
+                uint32_t dv0[32], dv1[32];
+                tmem_ld32(tP, dv0);
+                tmem_ld32(tP + 32, dv1);
+                tmem_wait_ld_tie(dv0);
+                tmem_wait_ld_tie(dv1);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float2 x = __ffma2_rn(
-                        make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), cc, nl);
-                    const float2 p = exp2_pair(x, e);
-                    const float2 dp = __fadd2_rn(
-                        make_float2(__uint_as_float(pv[2 * e]), __uint_as_float(pv[2 * e + 1])), nd);
-                    const float2 ds = __fmul2_rn(p, dp);
+                for (int e = 0; e < 32; ++e) {
+                    const uint32_t* dv = e < 16 ? dv0 : dv1;
+                    const int o = 2 * (e & 15);
+                    const float2 dp = __fadd2_rn(make_float2(__uint_as_float(dv[o]), __uint_as_float(dv[o + 1])),
+                                                 nd);
+                    const float2 ds = __fmul2_rn(make_float2(p[2 * e], p[2 * e + 1]), dp);
                     pk[e] = pack_bf16x2(ds.x, ds.y);
                 }
-                // dS over this warp's S columns [16g, 16g+16): already read
-                tmem_st16(tS + g * 16, pk);
             }
+            // dS over the first 32 of this warp's dP columns: both halves are in registers
+            tmem_st32(tP, pk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&ctl->ds_full);
@@ -532,14 +640,14 @@ __global__ void __launch_bounds__(320, 1)
         const bool all_ok = bar_red_and(1, 256, ok);
         if (all_ok && n > 0) {
             tc_fence_after();
-            // Q is dead once every MMA has completed; each warp group stages half the columns
-            stage_tmem_rows<D>(tmem + lane_off + 384u, sQ, m, a.scale, grp * D / 64, (grp + 1) * D / 64);
+            // dO's tile is dead once it is in TMEM; each warp group stages half the columns
+            stage_tmem_rows<D>(tmem + lane_off + kDQ, sdO, m, a.scale, grp * D / 64, (grp + 1) * D / 64);
             fence_proxy_async_smem();
             named_bar_sync(1, 256);
             if (threadIdx.x == 0) {
 #pragma unroll
                 for (int c = 0; c < C::kHalves; ++c)
-                    tma_store_5d(&tm_dq, smem_u32(sQ) + c * C::kHalfBytes, c * 64, q_w, q_h, q_t, bh);
+                    tma_store_5d(&tm_dq, smem_u32(sdO) + c * C::kHalfBytes, c * 64, q_w, q_h, q_t, bh);
                 tma_store_commit_and_wait_all();
             }
         } else if (all_ok && grp == 0) {
@@ -556,34 +664,64 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // ------------------------------------------------------------------ dK/dV kernel
-// One CTA per key chunk (CSC column). Shared memory tiles: K, V (this key
-// chunk) and Q[2], dO[2] (query chunks of the column, double-buffered), each
-// query chunk loaded in two halves of 64 queries (its frames 0-1 and 2-3)
-// together with the matching half of its aux record; a half is released as
-// soon as its last MMA has run. TMEM: S^T = K Q^T and dP^T = V dO^T per half
-// (S^T half h at column 64h, dP^T half h at 128 + 64h), dV accumulates at 256,
-// dK at 384. The 8 softmax warps split each half: warps w and w+4 share TMEM
-// lanes 32(w%4).. (key rows) and take its query columns [0,32) and [32,64),
-// writing packed bf16 P^T / dS^T over the first 16 of the columns they read
-// (the TMEM A operands of dV += P^T dO and dK += dS^T Q).
-// MMA issue order per step i:
-//   dV,dK(i,h0)  S^T,dP^T(i+1,h0)  dV,dK(i,h1)  S^T,dP^T(i+1,h1)
-// so the exponentials of one half run while the tensor core works on the other.
+// One CTA per key chunk (CSC column). K and V stay resident; the query chunks
+// that selected the key chunk come through two-slot Q and dO rings, each Q with
+// its 1 KB aux record (LSE * log2(e) and D of its 128 queries: column q of S^T,
+// half q / 64). The 8 exponential warps split each step: warps w and w+4 share
+// TMEM lanes 32(w%4).. (key rows) and take query columns [0,64) and [64,128),
+// the halves of the aux record. All four products are M = 128 keys x N = 128.
+//
+// TMEM: S^T = K Q^T at [0,128), dP^T = V dO^T at [128,256), dV at [256,384), dK
+// at [384,512). A step has two phases on separate barriers. P phase: the warps
+// load S^T, write P^T = exp2(S^T * scale * log2(e) - LSE * log2(e)) as packed
+// bf16 over the first half of their S^T columns (the TMEM A operand of
+// dV += P^T dO) and keep P in registers. dS phase: they load dP^T and write
+// dS^T = P^T (dP^T - D) over the first half of their dP^T columns (the A operand
+// of dK += dS^T Q). MMA issue order per step i: dV(i) and S^T(i+1) once P^T(i)
+// is written, then dK(i) and dP^T(i+1) once dS^T(i) is written. The tensor
+// core executes in issue order, so S^T(i+1) overwrites P^T(i) only after dV(i)
+// has read it (and likewise dP^T(i+1) after dK(i)); while the warps run the dS
+// phase of step i, dV(i) and S^T(i+1) are queued, and while they run the P
+// phase of step i+1, dK(i) and dP^T(i+1).
 struct __align__(8) DkvCtl {
-    uint64_t kv_full, qd_full[2][2], qd_empty[2][2], sd_full[2], p_full[2], dkv_full, aux;
+    uint64_t kv_full, q_full[2], q_empty[2], do_full[2], do_empty[2];
+    uint64_t s_full, dp_full, p_full, ds_full, dkv_full, aux;
     int n_valid;
     uint32_t tmem_base;
     int abort_flag;
 };
 
+// Stage a CSC column's query rows in shared memory (out-of-range entries dropped
+// and reported); returns the count on lane 0 (every lane of the calling warp
+// takes part).
+__device__ __forceinline__ int stage_column(const BwdArgs& a, int64_t col, uint16_t* list, int lane) {
+    bool bad = false;
+    int64_t beg = a.col_ptr[col], end = a.col_ptr[col + 1];
+    if (!(beg >= 0 && end >= beg && end <= a.idx_cap && end - beg <= a.Nq)) {
+        bad = true;
+        beg = end = 0;
+    }
+    int cnt = 0;
+    for (int64_t e0 = beg; e0 < end; e0 += 32) {
+        const int64_t e = e0 + lane;
+        const int r = e < end ? a.row_idx[e] : 0;
+        const bool valid = e < end && r >= 0 && r < a.Nq;
+        if (e < end && !valid) bad = true;
+        const uint32_t vb = __ballot_sync(0xffffffffu, valid);
+        if (valid) list[cnt + __popc(vb & ((1u << lane) - 1u))] = static_cast<uint16_t>(r);
+        cnt += __popc(vb);
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.status, kStatusBadIndex);
+    return cnt;
+}
+
 template <int D>
 __global__ void __launch_bounds__(320, 1)
-    bsa_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_doh,
+    bsa_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                        const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                        const BwdArgs a) {
     using C = BwdCfg<D>;
-    constexpr int kHalfTile = C::kTileBytes / 2;  // 64 tokens x D
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -603,13 +741,15 @@ __global__ void __launch_bounds__(320, 1)
     if (threadIdx.x == 0) {
         mbar_init(&ctl->kv_full, 1);
         for (int s = 0; s < 2; ++s) {
-            for (int h = 0; h < 2; ++h) {
-                mbar_init(&ctl->qd_full[s][h], 1);
-                mbar_init(&ctl->qd_empty[s][h], 1);
-            }
-            mbar_init(&ctl->sd_full[s], 1);
-            mbar_init(&ctl->p_full[s], 256);
+            mbar_init(&ctl->q_full[s], 1);
+            mbar_init(&ctl->q_empty[s], 1);
+            mbar_init(&ctl->do_full[s], 1);
+            mbar_init(&ctl->do_empty[s], 1);
         }
+        mbar_init(&ctl->s_full, 1);
+        mbar_init(&ctl->dp_full, 1);
+        mbar_init(&ctl->p_full, 256);
+        mbar_init(&ctl->ds_full, 256);
         mbar_init(&ctl->dkv_full, 1);
         mbar_init(&ctl->aux, 1);
         ctl->abort_flag = 0;
@@ -617,30 +757,13 @@ __global__ void __launch_bounds__(320, 1)
         fence_proxy_async_smem();
     }
     if (warp == C::kTmaWarp) {
-        // stage the column's query rows (out-of-range entries dropped and reported)
-        bool bad = false;
-        int64_t beg = a.col_ptr[col], end = a.col_ptr[col + 1];
-        if (!(beg >= 0 && end >= beg && end <= a.idx_cap && end - beg <= a.Nq)) {
-            bad = true;
-            beg = end = 0;
-        }
-        int cnt = 0;
-        for (int64_t e0 = beg; e0 < end; e0 += 32) {
-            const int64_t e = e0 + lane;
-            const int r = e < end ? a.row_idx[e] : 0;
-            const bool valid = e < end && r >= 0 && r < a.Nq;
-            if (e < end && !valid) bad = true;
-            const uint32_t vb = __ballot_sync(0xffffffffu, valid);
-            if (valid) list[cnt + __popc(vb & ((1u << lane) - 1u))] = static_cast<uint16_t>(r);
-            cnt += __popc(vb);
-        }
-        if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.status, kStatusBadIndex);
+        const int cnt = stage_column(a, col, list, lane);
         if (lane == 0) {
             ctl->n_valid = cnt;
-            prefetch_tensormap(&tm_qh);
+            prefetch_tensormap(&tm_q);
             prefetch_tensormap(&tm_k);
             prefetch_tensormap(&tm_v);
-            prefetch_tensormap(&tm_doh);
+            prefetch_tensormap(&tm_do);
             prefetch_tensormap(&tm_dk);
             prefetch_tensormap(&tm_dv);
         }
@@ -660,8 +783,10 @@ __global__ void __launch_bounds__(320, 1)
     chunk_origin(kc, a.NH, a.NW, k_t, k_h, k_w);
 
     if (warp == C::kTmaWarp) {
-        // ------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ TMA producers
         if (lane == 0 && n > 0) {
+            // K and V, then the Q ring with each query chunk's aux record (Q(i+2) once
+            // dK(i) has read Q(i); the warps have read the record by then)
             mbar_arrive_expect_tx(&ctl->kv_full, 2 * C::kTileBytes);
 #pragma unroll
             for (int c = 0; c < C::kHalves; ++c) {
@@ -670,99 +795,125 @@ __global__ void __launch_bounds__(320, 1)
                 tma_load_5d(&tm_v, smem_u32(sV) + c * C::kHalfBytes, &ctl->kv_full, c * 64, k_w, k_h,
                             k_t, bh);
             }
-            int nq[2][2] = {{0, 0}, {0, 0}};
+            int nq[2] = {0, 0};
             bool ok = true;
             for (int i = 0; i < n && ok; ++i) {
                 const int s = i & 1;
+                if (i >= 2 && !mbar_wait(&ctl->q_empty[s], ((i - 2) >> 1) & 1, abort_flag, a.status,
+                                         tmo, site(1, 1, s, i))) {
+                    ok = false;
+                    break;
+                }
                 const int r = list[i];
                 int qt, qh, qw;
                 chunk_origin(a.q_skip + r, a.NH, a.NW, qt, qh, qw);
-                for (int h = 0; h < 2; ++h) {
-                    if (i >= 2 && !mbar_wait(&ctl->qd_empty[s][h], ((i - 2) >> 1) & 1, abort_flag,
-                                             a.status, tmo, site(1, 1 + h, s, i))) {
-                        ok = false;
-                        break;
-                    }
-                    uint64_t* bar = &ctl->qd_full[s][h];
-                    mbar_arrive_expect_tx(bar, 2 * kHalfTile + 512);
+                mbar_arrive_expect_tx(&ctl->q_full[s], C::kTileBytes + 1024);
 #pragma unroll
-                    for (int c = 0; c < C::kHalves; ++c) {
-                        tma_load_5d(&tm_qh, smem_u32(sQ(s)) + c * C::kHalfBytes + h * 8192, bar, c * 64,
-                                    qw, qh, qt + 2 * h, bh);
-                        tma_load_5d(&tm_doh, smem_u32(sdO(s)) + c * C::kHalfBytes + h * 8192, bar,
-                                    c * 64, qw, qh, qt + 2 * h, bh);
-                    }
-                    bulk_load(smem_u32(sAux + s * 256 + h * 128),
-                              a.aux + (static_cast<int64_t>(bh) * a.Nq + r) * 256 + h * 128, 512, bar);
-                    ++nq[s][h];
-                }
+                for (int c = 0; c < C::kHalves; ++c)
+                    tma_load_5d(&tm_q, smem_u32(sQ(s)) + c * C::kHalfBytes, &ctl->q_full[s], c * 64,
+                                qw, qh, qt, bh);
+                bulk_load(smem_u32(sAux + s * 256), a.aux + (static_cast<int64_t>(bh) * a.Nq + r) * 256,
+                          1024, &ctl->q_full[s]);
+                ++nq[s];
             }
             if (!ok || *abort_flag) {
                 drain_wait(&ctl->kv_full, 0, tmo);
                 for (int s = 0; s < 2; ++s)
-                    for (int h = 0; h < 2; ++h)
-                        if (nq[s][h] > 0) drain_wait(&ctl->qd_full[s][h], (nq[s][h] - 1) & 1, tmo);
+                    if (nq[s] > 0) drain_wait(&ctl->q_full[s], (nq[s] - 1) & 1, tmo);
             }
+        } else if (lane == 1 && n > 0) {
+            // the dO ring: dO(i+2) once dV(i) has read dO(i)
+            int nd[2] = {0, 0};
+            bool ok = true;
+            for (int i = 0; i < n && ok; ++i) {
+                const int s = i & 1;
+                if (i >= 2 && !mbar_wait(&ctl->do_empty[s], ((i - 2) >> 1) & 1, abort_flag, a.status,
+                                         tmo, site(1, 2, s, i))) {
+                    ok = false;
+                    break;
+                }
+                int qt, qh, qw;
+                chunk_origin(a.q_skip + list[i], a.NH, a.NW, qt, qh, qw);
+                mbar_arrive_expect_tx(&ctl->do_full[s], C::kTileBytes);
+#pragma unroll
+                for (int c = 0; c < C::kHalves; ++c)
+                    tma_load_5d(&tm_do, smem_u32(sdO(s)) + c * C::kHalfBytes, &ctl->do_full[s], c * 64,
+                                qw, qh, qt, bh);
+                ++nd[s];
+            }
+            if (!ok || *abort_flag)
+                for (int s = 0; s < 2; ++s)
+                    if (nd[s] > 0) drain_wait(&ctl->do_full[s], (nd[s] - 1) & 1, tmo);
         }
         __syncwarp();
     } else if (warp == C::kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && n > 0) {
-            constexpr uint32_t kIdS = idesc_bf16_f32(128, 64, 0, 0);  // keys x 64 queries, K-major
-            constexpr uint32_t kIdG = idesc_bf16_f32(128, D, 0, 1);   // P^T/dS^T from TMEM, MN-major
+            constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);  // both operands K-major
+            constexpr uint32_t kIdG = idesc_bf16_f32(128, D, 0, 1);    // A from TMEM, B MN-major
             bool issued = false;
             bool ok = mbar_wait(&ctl->kv_full, 0, abort_flag, a.status, tmo, site(2, 0, 0, 0));
             if (ok) tc_fence_after();
-            // S^T and dP^T for queries [64h, 64h+64) of step i
-            auto issue_sd = [&](int i, int h) -> bool {
+            auto issue_ss = [&](uint32_t dcol, uint32_t sa, uint32_t sb) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
+                    mma_ss(tmem + dcol, sdesc_sw128(sa + off, 16, 1024), sdesc_sw128(sb + off, 16, 1024),
+                           kIdS, kk > 0 ? 1u : 0u);
+                }
+            };
+            // G += A B over 128 queries: queries 16kk.. of A sit at column 64*(kk/4) + 8*(kk%4)
+            // of the TMEM block at acol; B is the query chunk's tile at sb
+            auto issue_ts = [&](uint32_t dcol, uint32_t acol, uint32_t sb, bool first) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + dcol, tmem + acol + 64u * (kk >> 2) + 8u * (kk & 3),
+                           sdesc_sw128(sb + kk * 2048, C::kHalfBytes, 1024), kIdG,
+                           (!first || kk > 0) ? 1u : 0u);
+            };
+            // S^T(i) = K Q(i)^T
+            auto issue_st = [&](int i) -> bool {
                 const int s = i & 1;
-                if (!mbar_wait(&ctl->qd_full[s][h], (i >> 1) & 1, abort_flag, a.status, tmo,
-                               site(2, 1, s * 2 + h, i)))
+                if (!mbar_wait(&ctl->q_full[s], (i >> 1) & 1, abort_flag, a.status, tmo,
+                               site(2, 1, s, i)))
                     return false;
                 tc_fence_after();
-                const uint32_t sk = smem_u32(sK), sv = smem_u32(sV);
-                const uint32_t sq = smem_u32(sQ(s)) + h * 8192, sd = smem_u32(sdO(s)) + h * 8192;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-                    mma_ss(tmem + 64u * h, sdesc_sw128(sk + off, 16, 1024),
-                           sdesc_sw128(sq + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-                    mma_ss(tmem + 128u + 64u * h, sdesc_sw128(sv + off, 16, 1024),
-                           sdesc_sw128(sd + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-                }
+                issue_ss(0u, smem_u32(sK), smem_u32(sQ(s)));
                 issued = true;
-                tc_commit(&ctl->sd_full[h]);
+                tc_commit(&ctl->s_full);
                 return true;
             };
-            // dV += P^T dO and dK += dS^T Q over queries [64h, 64h+64) of step i
-            auto issue_pg = [&](int i, int h) -> bool {
+            // dP^T(i) = V dO(i)^T
+            auto issue_dpt = [&](int i) -> bool {
                 const int s = i & 1;
-                if (!mbar_wait(&ctl->p_full[h], i & 1, abort_flag, a.status, tmo, site(2, 2, h, i)))
+                if (!mbar_wait(&ctl->do_full[s], (i >> 1) & 1, abort_flag, a.status, tmo,
+                               site(2, 2, s, i)))
                     return false;
                 tc_fence_after();
-                const uint32_t sq = smem_u32(sQ(s)), sd = smem_u32(sdO(s));
-                // queries 16kk.. of half h: column 64h + 32*(kk/2) + 8*(kk%2) of S^T / dP^T
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + 256u, tmem + 64u * h + 32u * (kk >> 1) + 8u * (kk & 1),
-                           sdesc_sw128(sd + (4 * h + kk) * 2048, C::kHalfBytes, 1024), kIdG,
-                           (i > 0 || h > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + 384u, tmem + 128u + 64u * h + 32u * (kk >> 1) + 8u * (kk & 1),
-                           sdesc_sw128(sq + (4 * h + kk) * 2048, C::kHalfBytes, 1024), kIdG,
-                           (i > 0 || h > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(&ctl->qd_empty[s][h]);
+                issue_ss(128u, smem_u32(sV), smem_u32(sdO(s)));
+                issued = true;
+                tc_commit(&ctl->dp_full);
                 return true;
             };
-            ok = ok && issue_sd(0, 0) && issue_sd(0, 1);
+            ok = ok && issue_st(0) && issue_dpt(0);
             for (int i = 0; i < n && ok; ++i) {
-                ok = issue_pg(i, 0) && (i + 1 >= n || issue_sd(i + 1, 0)) && issue_pg(i, 1) &&
-                     (i + 1 >= n || issue_sd(i + 1, 1));
+                const int s = i & 1;
+                if (!mbar_wait(&ctl->p_full, i & 1, abort_flag, a.status, tmo, site(2, 3, 0, i))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                issue_ts(256u, 0u, smem_u32(sdO(s)), i == 0);   // dV += P^T(i) dO(i)
+                tc_commit(&ctl->do_empty[s]);
+                if (i + 1 < n && !issue_st(i + 1)) { ok = false; break; }
+                if (!mbar_wait(&ctl->ds_full, i & 1, abort_flag, a.status, tmo, site(2, 4, 0, i))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                issue_ts(384u, 128u, smem_u32(sQ(s)), i == 0);  // dK += dS^T(i) Q(i)
+                tc_commit(&ctl->q_empty[s]);
+                if (i + 1 < n && !issue_dpt(i + 1)) { ok = false; break; }
             }
             if (ok) {
                 tc_commit(&ctl->dkv_full);
@@ -774,53 +925,88 @@ __global__ void __launch_bounds__(320, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ P^T, dS^T + epilogue
-        const int grp = warp >> 2;                    // query columns [32*grp, 32*grp + 32) of a half
+        const int grp = warp >> 2;                    // query columns [64*grp, 64*grp + 64)
         const int m = (warp & 3) * 32 + lane;         // key row = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + 64u * grp;
+        const uint32_t tP = tS + 128u;
         const float2 cc = make_float2(a.scale_log2, a.scale_log2);
         bool ok = true;
-        for (int i = 0; i < n && ok; ++i) {
+        for (int i = 0; i < n; ++i) {
             const int s = i & 1;
-            for (int h = 0; h < 2; ++h) {
-                // this half's aux record arrived with its Q/dO copies
-                bool got = mbar_wait(&ctl->qd_full[s][h], (i >> 1) & 1, abort_flag, a.status, tmo,
-                                     site(3, 3, s * 2 + h, i));
-                got = got && mbar_wait(&ctl->sd_full[h], i & 1, abort_flag, a.status, tmo, site(3, 4, h, i));
-                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-                tc_fence_after();
-                const float* lse2 = sAux + s * 256 + h * 128;
-                const float* Dq = lse2 + 64;
-                const uint32_t tS = tmem + lane_off + 64u * h + 32u * grp;
-                const uint32_t tP = tmem + lane_off + 128u + 64u * h + 32u * grp;
-                {
-                    uint32_t sv[32], pv[32];
-                    tmem_ld32(tS, sv);
-                    tmem_ld32(tP, pv);
-                    tmem_wait_ld_tie(sv);
-                    tmem_wait_ld_tie(pv);
-                    uint32_t pk[16], dk[16];
+            // P phase. The aux record arrived with Q(i), before S^T(i) could start: its 64
+            // LSE * log2(e) values for this group's queries are loaded while S^T(i) runs.
+            bool got = mbar_wait(&ctl->q_full[s], (i >> 1) & 1, abort_flag, a.status, tmo,
+                                 site(3, 3, s, i));
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            const float* lse2 = sAux + s * 256 + grp * 128;  // this group's 64 queries
+            const float* Dq = lse2 + 64;
+            float4 l4v[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int qi = 32 * grp + 2 * e;  // query of this pair within the half
-                        const float2 l2 = *reinterpret_cast<const float2*>(lse2 + qi);
-                        const float2 dd = *reinterpret_cast<const float2*>(Dq + qi);
+            for (int e4 = 0; e4 < 16; ++e4) l4v[e4] = *reinterpret_cast<const float4*>(lse2 + 4 * e4);
+            got = mbar_wait(&ctl->s_full, i & 1, abort_flag, a.status, tmo, site(3, 4, 0, i));
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            tc_fence_after();
+            float p[64];
+            uint32_t pk[32];
+            {
+                uint32_t sv0[32], sv1[32];
+                tmem_ld32(tS, sv0);
+                tmem_ld32(tS + 32, sv1);
+                tmem_wait_ld_tie(sv0);
+                tmem_wait_ld_tie(sv1);
+#pragma unroll
+                for (int e4 = 0; e4 < 16; ++e4) {
+                    const float4 l4 = l4v[e4];
+                    const uint32_t* sv = e4 < 8 ? sv0 : sv1;
+                    const int o = (e4 & 7) * 4;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
                         const float2 x = __ffma2_rn(
-                            make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), cc,
-                            make_float2(-l2.x, -l2.y));
-                        const float2 p = exp2_pair(x, e);
-                        const float2 dp = make_float2(__uint_as_float(pv[2 * e]) - dd.x,
-                                                      __uint_as_float(pv[2 * e + 1]) - dd.y);
-                        const float2 ds = __fmul2_rn(p, dp);
-                        pk[e] = pack_bf16x2(p.x, p.y);
-                        dk[e] = pack_bf16x2(ds.x, ds.y);
+                            make_float2(__uint_as_float(sv[o + 2 * h]), __uint_as_float(sv[o + 2 * h + 1])),
+                            cc, h == 0 ? make_float2(-l4.x, -l4.y) : make_float2(-l4.z, -l4.w));
+                        const float2 pe = exp2_pair(x, 2 * e4 + h);
+                        p[4 * e4 + 2 * h] = pe.x;
+                        p[4 * e4 + 2 * h + 1] = pe.y;
+                        pk[2 * e4 + h] = pack_bf16x2(pe.x, pe.y);
                     }
-                    tmem_st16(tS, pk);
-                    tmem_st16(tP, dk);
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&ctl->p_full[h]);
             }
+            // P^T over the first 32 of this warp's S^T columns: both halves were read
+            tmem_st32(tS, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&ctl->p_full);
+            // dS phase
+            got = mbar_wait(&ctl->dp_full, i & 1, abort_flag, a.status, tmo, site(3, 5, 0, i));
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            tc_fence_after();
+            {
+                uint32_t dv0[32], dv1[32];
+                tmem_ld32(tP, dv0);
+                tmem_ld32(tP + 32, dv1);
+                tmem_wait_ld_tie(dv0);
+                tmem_wait_ld_tie(dv1);
+#pragma unroll
+                for (int e4 = 0; e4 < 16; ++e4) {
+                    const float4 d4 = *reinterpret_cast<const float4*>(Dq + 4 * e4);
+                    const uint32_t* dv = e4 < 8 ? dv0 : dv1;
+                    const int o = (e4 & 7) * 4;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float2 dp = __fadd2_rn(
+                            make_float2(__uint_as_float(dv[o + 2 * h]), __uint_as_float(dv[o + 2 * h + 1])),
+                            h == 0 ? make_float2(-d4.x, -d4.y) : make_float2(-d4.z, -d4.w));
+                        const float2 ds = __fmul2_rn(
+                            make_float2(p[4 * e4 + 2 * h], p[4 * e4 + 2 * h + 1]), dp);
+                        pk[2 * e4 + h] = pack_bf16x2(ds.x, ds.y);
+                    }
+                }
+            }
+            tmem_st32(tP, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&ctl->ds_full);
         }
         if (ok && n > 0) {
             const bool got = mbar_wait(&ctl->dkv_full, 0, abort_flag, a.status, tmo, site(3, 6, 0, 0));
@@ -829,25 +1015,24 @@ __global__ void __launch_bounds__(320, 1)
         const bool all_ok = bar_red_and(1, 256, ok);
         if (all_ok && n > 0) {
             tc_fence_after();
-            // K and V tiles are dead once every MMA has completed: group 0 stages
-            // dV, group 1 dK (scaled)
-            if (grp == 0)
-                stage_tmem_rows<D>(tmem + lane_off + 256u, sV, m, 1.0f);
-            else
-                stage_tmem_rows<D>(tmem + lane_off + 384u, sK, m, a.scale);
+            // K and V are dead once every MMA has completed; each warp group stages half
+            // the columns of dK (into K's tile) and dV (into V's)
+            stage_tmem_rows<D>(tmem + lane_off + 384u, sK, m, a.scale, grp * D / 64, (grp + 1) * D / 64);
+            stage_tmem_rows<D>(tmem + lane_off + 256u, sV, m, 1.0f, grp * D / 64, (grp + 1) * D / 64);
             fence_proxy_async_smem();
             named_bar_sync(1, 256);
             if (threadIdx.x == 0) {
 #pragma unroll
                 for (int c = 0; c < C::kHalves; ++c) {
-                    tma_store_5d(&tm_dv, smem_u32(sV) + c * C::kHalfBytes, c * 64, k_w, k_h, k_t, bh);
                     tma_store_5d(&tm_dk, smem_u32(sK) + c * C::kHalfBytes, c * 64, k_w, k_h, k_t, bh);
+                    tma_store_5d(&tm_dv, smem_u32(sV) + c * C::kHalfBytes, c * 64, k_w, k_h, k_t, bh);
                 }
                 tma_store_commit_and_wait_all();
             }
+        } else if (all_ok && grp == 0) {
+            zero_token<D>(a.dk, bh, a.N, a.T, a.H, a.W, k_t, k_h, k_w, m);  // never selected
         } else if (all_ok) {
-            // no query chunk selected this key chunk: zero gradients
-            zero_token<D>(grp ? a.dk : a.dv, bh, a.N, a.T, a.H, a.W, k_t, k_h, k_w, m);
+            zero_token<D>(a.dv, bh, a.N, a.T, a.H, a.W, k_t, k_h, k_w, m);
         }
     }
 
@@ -869,13 +1054,13 @@ cudaError_t launch_bwd_d(const Dims& g, const CUtensorMap* m, const BwdArgs& dq_
         if (e == cudaSuccess) e = raise_smem_limit(bsa_bwd_dkv_kernel<D>, C::kSmemBytes, dkv_attr);
         if (e != cudaSuccess) return e;
     }
-    // m: q, k, v, dout, dq, dk, dv (whole chunks), then q and dout (half chunks)
+    // m: q, k, v, dout, dq, dk, dv (whole chunks)
     bsa_bwd_dq_kernel<D><<<static_cast<unsigned>(dq_args.units), C::kThreads, C::kSmemBytes, st>>>(
         m[0], m[1], m[2], m[3], m[4], dq_args);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     bsa_bwd_dkv_kernel<D><<<static_cast<unsigned>(dkv_args.units), C::kThreads, C::kSmemBytes, st>>>(
-        m[7], m[1], m[2], m[8], m[5], m[6], dkv_args);
+        m[0], m[1], m[2], m[3], m[5], m[6], dkv_args);
     return cudaGetLastError();
 }
 
@@ -922,12 +1107,11 @@ cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const v
     int32_t* row_idx = reinterpret_cast<int32_t*>(ws + L.row_idx);
     const int64_t cols = g.BH * g.Nc;
 
-    // whole-chunk maps q, k, v, dout, dq, dk, dv, then half-chunk maps of q and dout
-    CUtensorMap m[9];
-    const void* bases[9] = {q, k, v, dout, dq, dk, dv, q, dout};
-    for (int i = 0; i < 9; ++i)
-        if (!make_chunk_map(&m[i], bases[i], g, i < 7 ? kChunkT : kChunkT / 2))
-            return cudaErrorInvalidValue;
+    // whole-chunk maps q, k, v, dout, dq, dk, dv
+    CUtensorMap m[7];
+    const void* bases[7] = {q, k, v, dout, dq, dk, dv};
+    for (int i = 0; i < 7; ++i)
+        if (!make_chunk_map(&m[i], bases[i], g)) return cudaErrorInvalidValue;
 
     cudaError_t e = cudaMemsetAsync(ws + L.bitmap, 0, L.cnt - L.bitmap, st);  // bitmap + rawcnt
     if (e != cudaSuccess) return e;
