@@ -185,7 +185,7 @@ struct BwdCfg {
     static constexpr int kTmaWarp = 8;
     static constexpr int kMmaWarp = 9;
     static constexpr uint32_t kTmemCols = 512;
-    // every kernel: six tiles, then three 1 KB per-query-chunk aux records, control, list
+    // six tiles, then (dK/dV kernel) three 1 KB per-query-chunk aux records, control, list
     static constexpr int kAux = 6 * kTileBytes;
     static constexpr int kCtl = kAux + 3 * 1024;
     static constexpr int kList = kCtl + 512;
@@ -490,22 +490,23 @@ __global__ void __launch_bounds__(320, 1)
                            kk > 0 ? 1u : 0u);
                 }
             };
+            // S(j) = Q K(j)^T. Past the first step the dS warps have seen K(j) land before
+            // releasing S(j-1), so the wait on s_free covers it.
             auto issue_s = [&](int j) -> bool {
                 const int s = j % 3;
-                if (!mbar_wait(&ctl->k_full[s], (j / 3) & 1, abort_flag, a.status, tmo, site(2, 1, s, j)))
+                if (j == 0 && !mbar_wait(&ctl->k_full[s], 0, abort_flag, a.status, tmo, site(2, 1, s, j)))
                     return false;
-                tc_fence_after();
                 issue_tk(kS, kQt, smem_u32(sK(s)));
                 issued = true;
                 tc_commit(&ctl->s_full);
                 return true;
             };
-            // dP(j) = dO V(j)^T
+            // dP(j) = dO V(j)^T. Past the first step the dS warps have seen V(j) land before
+            // arriving on ds_full for step j-1.
             auto issue_dp = [&](int j) -> bool {
                 const int s = j & 1;
-                if (!mbar_wait(&ctl->v_full[s], (j >> 1) & 1, abort_flag, a.status, tmo, site(2, 2, s, j)))
+                if (j == 0 && !mbar_wait(&ctl->v_full[s], 0, abort_flag, a.status, tmo, site(2, 2, s, j)))
                     return false;
-                tc_fence_after();
                 issue_tk(kDP, kDOt, smem_u32(sV(s)));
                 issued = true;
                 tc_commit(&ctl->v_empty[s]);
@@ -591,7 +592,11 @@ __global__ void __launch_bounds__(320, 1)
                 tmem_ld32(tS + 32, sv1);
                 tmem_wait_ld_tie(sv0);
                 tmem_wait_ld_tie(sv1);
-                // S of this step is in registers: its columns may be overwritten
+                // S of this step is in registers: its columns may be overwritten. K(j+1) has
+                // landed (seen here, so the MMA thread need not wait for it) before S(j+1).
+                const bool k_in = j + 1 >= n || mbar_wait(&ctl->k_full[(j + 1) % 3], ((j + 1) / 3) & 1,
+                                                          abort_flag, a.status, tmo, site(3, 1, (j + 1) % 3, j));
+                if (!__all_sync(0xffffffffu, k_in)) { ok = false; break; }
                 tc_fence_before();
                 mbar_arrive_tied(&ctl->s_free, sv0);
                 reg_tie(sv1);
@@ -630,6 +635,10 @@ __global__ void __launch_bounds__(320, 1)
             // dS over the first 32 of this warp's dP columns: both halves are in registers
             tmem_st32(tP, pk);
             tmem_wait_st();
+            // V(j+1) has landed (seen here for the MMA thread) before dP(j+1)
+            const bool v_in = j + 1 >= n || mbar_wait(&ctl->v_full[(j + 1) & 1], ((j + 1) >> 1) & 1,
+                                                      abort_flag, a.status, tmo, site(3, 2, (j + 1) & 1, j));
+            if (!__all_sync(0xffffffffu, v_in)) { ok = false; break; }
             tc_fence_before();
             mbar_arrive(&ctl->ds_full);
         }
@@ -682,7 +691,9 @@ __global__ void __launch_bounds__(320, 1)
 // core executes in issue order, so S^T(i+1) overwrites P^T(i) only after dV(i)
 // has read it (and likewise dP^T(i+1) after dK(i)); while the warps run the dS
 // phase of step i, dV(i) and S^T(i+1) are queued, and while they run the P
-// phase of step i+1, dK(i) and dP^T(i+1).
+// phase of step i+1, dK(i) and dP^T(i+1). Before their dS-phase arrival the
+// warps check that dO(i+1) has landed (requested a step earlier), so the MMA
+// thread does not wait for it.
 struct __align__(8) DkvCtl {
     uint64_t kv_full, q_full[2], q_empty[2], do_full[2], do_empty[2];
     uint64_t s_full, dp_full, p_full, ds_full, dkv_full, aux;
@@ -883,13 +894,12 @@ __global__ void __launch_bounds__(320, 1)
                 tc_commit(&ctl->s_full);
                 return true;
             };
-            // dP^T(i) = V dO(i)^T
+            // dP^T(i) = V dO(i)^T. Past the first step the warps have seen dO(i) land before
+            // arriving on ds_full for step i-1.
             auto issue_dpt = [&](int i) -> bool {
                 const int s = i & 1;
-                if (!mbar_wait(&ctl->do_full[s], (i >> 1) & 1, abort_flag, a.status, tmo,
-                               site(2, 2, s, i)))
+                if (i == 0 && !mbar_wait(&ctl->do_full[0], 0, abort_flag, a.status, tmo, site(2, 2, 0, 0)))
                     return false;
-                tc_fence_after();
                 issue_ss(128u, smem_u32(sV), smem_u32(sdO(s)));
                 issued = true;
                 tc_commit(&ctl->dp_full);
@@ -1005,6 +1015,10 @@ __global__ void __launch_bounds__(320, 1)
             }
             tmem_st32(tP, pk);
             tmem_wait_st();
+            // dO(i+1) has landed (seen here for the MMA thread) before dP^T(i+1)
+            got = i + 1 >= n || mbar_wait(&ctl->do_full[(i + 1) & 1], ((i + 1) >> 1) & 1, abort_flag,
+                                          a.status, tmo, site(3, 2, (i + 1) & 1, i));
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_before();
             mbar_arrive(&ctl->ds_full);
         }
