@@ -336,7 +336,8 @@ def time_backward(args, wl, p, pl, q, k, v, stream, peak_tf, batch_offset=0, hea
     return {"bwd_ms": ms, "steps": args.bwd_steps, "algorithmic_flops": alg,
             "executed_flops": executed, "alg_tflops": alg / ms / 1e9,
             "exec_tflops": executed / ms / 1e9, "exec_frac": executed / ms / 1e9 / peak_tf,
-            "launches_per_call": 6, "device_status": bsa.status_string(rc)}
+            # prep, CSR->CSC (scatter, count, scan, emit), dQ, dK/dV
+            "launches_per_call": 7, "device_status": bsa.status_string(rc)}
 
 
 # ---------------------------------------------------------------------- other workloads
