@@ -83,6 +83,9 @@ def _load():
             lib.oracle_attend_shape.restype = i32
             lib.oracle_attend_shape.argtypes = [vp, vp, vp] + [i32] * 8 + [dbl, vp, vp, vp, i64,
                                                                            vp, vp]
+            lib.oracle_attend_bwd_qk.restype = i32
+            lib.oracle_attend_bwd_qk.argtypes = [vp] * 4 + [i32] * 11 + [dbl, vp, vp, vp, i64,
+                                                                       vp, vp, vp]
             lib.oracle_attend_bwd_shape.restype = i32
             lib.oracle_attend_bwd_shape.argtypes = [vp] * 4 + [i32] * 8 + [dbl, vp, vp, vp, i64,
                                                                           vp, vp, vp]
@@ -230,13 +233,15 @@ def _f64(a):
     return np.ascontiguousarray(a, dtype=np.float64)
 
 
-def attend_bwd(q, k, v, dout, T, H, W, scale, row_ptr, col_idx, rows, kchunk=CHUNK):
+def attend_bwd(q, k, v, dout, T, H, W, scale, row_ptr, col_idx, rows, kchunk=CHUNK,
+               qchunk=CHUNK):
     """Gradients of ``attend`` for upstream gradient ``dout`` (same shape as q).
 
     Inputs: bf16 bit patterns (uint16) or float arrays [B, heads, N, d].
-    Returns dq_rows [n, 128, d] for the listed CSR rows and dk, dv [B, heads, N, d]
-    holding the contributions of those rows (complete for every key chunk whose
-    selecting rows are all listed). float64 throughout.
+    Returns dq_rows [n, slots, d] for the listed CSR rows (slots = the query
+    chunk's token count) and dk, dv [B, heads, N, d] holding the contributions
+    of those rows (complete for every key chunk whose selecting rows are all
+    listed). float64 throughout.
     """
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
     B, Hh, N, d = q.shape
@@ -245,14 +250,15 @@ def attend_bwd(q, k, v, dout, T, H, W, scale, row_ptr, col_idx, rows, kchunk=CHU
     ci = np.ascontiguousarray(col_idx, dtype=np.int32)
     if ci.size == 0:
         ci = np.zeros(1, dtype=np.int32)
-    dq = np.empty((rows.size, CN, d), dtype=np.float64)
+    qn = qchunk[0] * qchunk[1] * qchunk[2]
+    dq = np.empty((rows.size, qn, d), dtype=np.float64)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
-    _check(_load().oracle_attend_bwd_shape(q.ctypes.data, k.ctypes.data, v.ctypes.data,
-                                           dout.ctypes.data, B * Hh, T, H, W, *kchunk, d,
-                                           float(scale), rp.ctypes.data, ci.ctypes.data,
-                                           rows.ctypes.data, rows.size, dq.ctypes.data,
-                                           dk.ctypes.data, dv.ctypes.data), "oracle_attend_bwd")
+    _check(_load().oracle_attend_bwd_qk(q.ctypes.data, k.ctypes.data, v.ctypes.data,
+                                        dout.ctypes.data, B * Hh, T, H, W, *qchunk, *kchunk, d,
+                                        float(scale), rp.ctypes.data, ci.ctypes.data,
+                                        rows.ctypes.data, rows.size, dq.ctypes.data,
+                                        dk.ctypes.data, dv.ctypes.data), "oracle_attend_bwd")
     return dq, dk, dv
 
 

@@ -483,7 +483,9 @@ int oracle_dense(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH
  *   dQ[q]   = scale * sum_j dS[q,j] k_j
  *   dK[j]  += scale * dS[q,j] q
  * Inputs are fp64 [BH][N][d] in THW token order (callers widen bf16 exactly),
- * so the same routine serves finite-difference checks. The rows listed in
+ * so the same routine serves finite-difference checks. Query chunks have shape
+ * (qst,qsh,qsw) and key chunks (kst,ksh,ksw) ([P1] block-size robustness: query
+ * blocks of 64 or 128 tokens); Nc counts the query chunks. The rows listed in
  * rows[] (r = bh*Nc + i) are processed: dq_rows[n][l][:] receives dQ of local
  * query l of rows[n]; dk and dv ([BH][N][d], zeroed by the caller) accumulate
  * the contributions of those rows only (complete for a key chunk when every
@@ -492,16 +494,18 @@ int oracle_dense(const uint16_t* q, const uint16_t* k, const uint16_t* v, int BH
  * chunks; a local query slot past the grid edge has no dQ (NaN) and
  * contributes nothing. All arithmetic in fp64.
  */
-int oracle_attend_bwd_shape(const double* q, const double* k, const double* v, const double* dout,
-                            int BH, int T, int H, int W, int kst, int ksh, int ksw, int d,
-                            double scale, const int32_t* row_ptr, const int32_t* col_idx,
-                            const int64_t* rows, int64_t n_rows, double* dq_rows, double* dk,
-                            double* dv) {
+int oracle_attend_bwd_qk(const double* q, const double* k, const double* v, const double* dout,
+                         int BH, int T, int H, int W, int qst, int qsh, int qsw, int kst, int ksh,
+                         int ksw, int d, double scale, const int32_t* row_ptr,
+                         const int32_t* col_idx, const int64_t* rows, int64_t n_rows,
+                         double* dq_rows, double* dk, double* dv) {
     if (!q || !k || !v || !dout || !row_ptr || !col_idx || !rows || !dq_rows || !dk || !dv ||
-        BH <= 0 || d <= 0 || !grid_ok(T, H, W) || kst <= 0 || ksh <= 0 || ksw <= 0)
+        BH <= 0 || d <= 0 || !grid_ok(T, H, W) || qst <= 0 || qsh <= 0 || qsw <= 0 || kst <= 0 ||
+        ksh <= 0 || ksw <= 0)
         return -1;
     const int kn = kst * ksh * ksw;  /* slots of a key chunk */
-    const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks(T, H, W);
+    const int CQ = qst * qsh * qsw;  /* slots of a query chunk */
+    const int64_t N = (int64_t)T * H * W, Nc = oracle_num_chunks_shape(T, H, W, qst, qsh, qsw);
     for (int64_t n = 0; n < n_rows; ++n)
         if (rows[n] < 0 || rows[n] >= (int64_t)BH * Nc) return -1;
     int64_t cap_keys = 0;
@@ -513,12 +517,12 @@ int oracle_attend_bwd_shape(const double* q, const double* k, const double* v, c
         const int64_t bh = r / Nc, i = r % Nc;
         const int64_t beg = row_ptr[r], end = row_ptr[r + 1];
         const int64_t slots = (end - beg) * kn;
-        double* dqr = dq_rows + n * CN * d;
+        double* dqr = dq_rows + n * CQ * d;
         if (slots > cap_keys) {
             free(ktok); free(P); free(dS);
             ktok = (int64_t*)malloc(sizeof(int64_t) * (size_t)slots);
-            P = (double*)malloc(sizeof(double) * (size_t)(CN * slots));
-            dS = (double*)malloc(sizeof(double) * (size_t)(CN * slots));
+            P = (double*)malloc(sizeof(double) * (size_t)(CQ * slots));
+            dS = (double*)malloc(sizeof(double) * (size_t)(CQ * slots));
             cap_keys = slots;
         }
         int64_t nk = 0;  /* existing key tokens of the row */
@@ -527,19 +531,19 @@ int oracle_attend_bwd_shape(const double* q, const double* k, const double* v, c
                 const int64_t tok = oracle_token_of_shape(T, H, W, kst, ksh, ksw, col_idx[e], l);
                 if (tok >= 0) ktok[nk++] = bh * N + tok;
             }
-        for (int lq = 0; lq < CN; ++lq)
-            if (oracle_token_of(T, H, W, i, lq) < 0)
+        for (int lq = 0; lq < CQ; ++lq)
+            if (oracle_token_of_shape(T, H, W, qst, qsh, qsw, i, lq) < 0)
                 for (int x = 0; x < d; ++x) dqr[(int64_t)lq * d + x] = NAN;
         if (nk <= 0) {
-            for (int lq = 0; lq < CN; ++lq)
-                if (oracle_token_of(T, H, W, i, lq) >= 0)
+            for (int lq = 0; lq < CQ; ++lq)
+                if (oracle_token_of_shape(T, H, W, qst, qsh, qsw, i, lq) >= 0)
                     for (int x = 0; x < d; ++x) dqr[(int64_t)lq * d + x] = 0.0;
             continue;
         }
         /* per query: softmax weights, O, D, dS and dQ */
 #pragma omp parallel for schedule(static)
-        for (int lq = 0; lq < CN; ++lq) {
-            const int64_t qtok = oracle_token_of(T, H, W, i, lq);
+        for (int lq = 0; lq < CQ; ++lq) {
+            const int64_t qtok = oracle_token_of_shape(T, H, W, qst, qsh, qsw, i, lq);
             double* p = P + (int64_t)lq * nk;
             double* ds = dS + (int64_t)lq * nk;
             if (qtok < 0) {  /* no such query: no weights */
@@ -586,8 +590,8 @@ int oracle_attend_bwd_shape(const double* q, const double* k, const double* v, c
         for (int64_t j = 0; j < nk; ++j) {
             double* dkr = dk + ktok[j] * d;
             double* dvr = dv + ktok[j] * d;
-            for (int lq = 0; lq < CN; ++lq) {
-                const int64_t qtok = oracle_token_of(T, H, W, i, lq);
+            for (int lq = 0; lq < CQ; ++lq) {
+                const int64_t qtok = oracle_token_of_shape(T, H, W, qst, qsh, qsw, i, lq);
                 if (qtok < 0) continue;
                 const int64_t qt = bh * N + qtok;
                 const double pw = P[(int64_t)lq * nk + j];
@@ -603,6 +607,15 @@ int oracle_attend_bwd_shape(const double* q, const double* k, const double* v, c
     }
     free(ktok); free(P); free(dS);
     return 0;
+}
+
+int oracle_attend_bwd_shape(const double* q, const double* k, const double* v, const double* dout,
+                            int BH, int T, int H, int W, int kst, int ksh, int ksw, int d,
+                            double scale, const int32_t* row_ptr, const int32_t* col_idx,
+                            const int64_t* rows, int64_t n_rows, double* dq_rows, double* dk,
+                            double* dv) {
+    return oracle_attend_bwd_qk(q, k, v, dout, BH, T, H, W, CT, CH, CW, kst, ksh, ksw, d, scale,
+                                row_ptr, col_idx, rows, n_rows, dq_rows, dk, dv);
 }
 
 /*

@@ -6,12 +6,15 @@ to 1024 tokens; the blocks of its partitioning are t = h = w = 4, i.e. (4,4,4)
 blocks of 64 tokens. The oracle takes the query chunk shape as a parameter of
 selection and attention; these tests tie that generalisation to numpy
 reshapes, sorts and a token-level masked softmax, to dense attention when
-every chunk is kept, and to hand-built block-causal candidate sets.
+every chunk is kept, and to hand-built block-causal candidate sets. The
+backward (gradients over 64-token query chunks) is tied to torch float64
+autograd of the token-masked dense attention and to the (4,4,8) backward.
 """
 import math
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 import synth
@@ -164,3 +167,84 @@ def test_64_token_query_rows_are_the_halves_of_128_token_rows_when_keys_agree():
     for c in range(4):
         np.testing.assert_allclose(out4[2 * c], out8[c][lw < 4], rtol=0, atol=1e-12)
         np.testing.assert_allclose(out4[2 * c + 1], out8[c][lw >= 4], rtol=0, atol=1e-12)
+
+
+def _q64_maps(wl, kchunk):
+    """Token index of every (chunk, slot) for (4,4,4) query chunks and the given
+    key chunks, from numpy reshapes, and the inverse (token -> chunk) maps."""
+    iota = np.arange(wl.N).reshape(1, 1, -1, 1)
+    qtok = numpy_rearrange64(iota, wl.T, wl.H, wl.W)[0, 0, :, :, 0]
+    kt, kh, kw = kchunk
+    kv = iota.reshape(wl.T // kt, kt, wl.H // kh, kh, wl.W // kw, kw)
+    ktok = kv.transpose(0, 2, 4, 1, 3, 5).reshape(-1, kt * kh * kw)
+    qchunk_of = np.empty(wl.N, dtype=np.int64)
+    qchunk_of[qtok.reshape(-1)] = np.repeat(np.arange(qtok.shape[0]), qtok.shape[1])
+    kchunk_of = np.empty(wl.N, dtype=np.int64)
+    kchunk_of[ktok.reshape(-1)] = np.repeat(np.arange(ktok.shape[0]), ktok.shape[1])
+    return qtok, qchunk_of, kchunk_of
+
+
+@pytest.mark.parametrize("kchunk", [Q64, (4, 4, 8)])
+def test_backward_of_64_token_query_chunks_equals_torch_autograd(kchunk):
+    """The oracle's gradients with (4,4,4) query chunks against torch float64
+    autograd of the dense softmax attention under the chunk mask lifted to
+    tokens with numpy reshapes; one query chunk selects nothing (its queries
+    have no output and no gradient)."""
+    wl = W0.with_(T=8, H=8, W=16, heads=1, d=32)
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    scale = 0.3
+    rp, ci, _ = oracle.plan(q, k, wl.T, wl.H, wl.W, scale, "topk", 3, kchunk=kchunk, qchunk=Q64)
+    nq = oracle.num_chunks(wl.T, wl.H, wl.W, Q64)
+    nk = oracle.num_chunks(wl.T, wl.H, wl.W, kchunk)
+    lists = [list(ci[rp[i]:rp[i + 1]]) for i in range(nq)]
+    lists[5] = []                                            # an empty row
+    rp = np.concatenate([[0], np.cumsum([len(r) for r in lists])]).astype(np.int32)
+    ci = np.array([c for r in lists for c in r], dtype=np.int32)
+    dq_rows, dk, dv = oracle.attend_bwd(q, k, v, g, wl.T, wl.H, wl.W, scale, rp, ci,
+                                        np.arange(nq), kchunk=kchunk, qchunk=Q64)
+    assert dq_rows.shape == (nq, 64, wl.d)
+    qtok, qchunk_of, kchunk_of = _q64_maps(wl, kchunk)
+    dq = np.zeros((wl.N, wl.d))
+    for i in range(nq):
+        dq[qtok[i]] = dq_rows[i]
+    M = np.zeros((nq, nk), dtype=bool)
+    for i in range(nq):
+        M[i, lists[i]] = True
+    tm = torch.from_numpy(M[qchunk_of][:, kchunk_of])
+    Q, K, V = (torch.tensor(bf(x)[0, 0], dtype=torch.float64, requires_grad=True)
+               for x in (q, k, v))
+    G = torch.tensor(bf(g)[0, 0], dtype=torch.float64)
+    live = tm.any(-1)
+    s = (Q @ K.T) * scale
+    s = s.masked_fill(~tm, float("-inf"))
+    s = torch.where(live[:, None], s, torch.zeros_like(s))
+    w = torch.softmax(s, -1) * live[:, None]
+    (G * (w @ V)).sum().backward()
+    np.testing.assert_allclose(dq, Q.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk[0, 0], K.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv[0, 0], V.grad.numpy(), rtol=0, atol=1e-12)
+    assert np.all(dq[qtok[5]] == 0) and np.abs(dq).max() > 1e-3 and np.abs(dk).max() > 1e-3
+
+
+def test_backward_of_64_token_rows_equals_128_token_rows_when_keys_agree():
+    """Selections written for the 8 query chunks of (4,4,4) that give both
+    w-halves of every (4,4,8) chunk the same keys: dQ of each 64-token chunk is
+    the matching half of the (4,4,8) chunk's dQ, and dK, dV are the same."""
+    wl = W0.with_(T=8, H=8, W=16, heads=1)
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    scale = 1 / math.sqrt(wl.d)
+    rp8 = np.array([0, 2, 4, 6, 8], dtype=np.int32)
+    ci8 = np.array([0, 3, 1, 2, 0, 2, 1, 3], dtype=np.int32)
+    dq8, dk8, dv8 = oracle.attend_bwd(q, k, v, g, wl.T, wl.H, wl.W, scale, rp8, ci8, np.arange(4))
+    rp4 = np.arange(0, 17, 2, dtype=np.int32)
+    ci4 = np.repeat(ci8.reshape(4, 2), 2, axis=0).reshape(-1).astype(np.int32)
+    dq4, dk4, dv4 = oracle.attend_bwd(q, k, v, g, wl.T, wl.H, wl.W, scale, rp4, ci4, np.arange(8),
+                                      kchunk=(4, 4, 8), qchunk=Q64)
+    lw = np.arange(128) % 8
+    for c in range(4):
+        np.testing.assert_allclose(dq4[2 * c], dq8[c][lw < 4], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dq4[2 * c + 1], dq8[c][lw >= 4], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk4, dk8, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv4, dv8, rtol=0, atol=1e-12)
