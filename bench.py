@@ -384,6 +384,34 @@ def time_config(wl, steps, peak_tf, stream):
                     "box_tiles": n_box, "tile_tflops": tile_tf, "tile_frac": tile_tf / peak_tf,
                     "useful_share_of_tiles": exec_flops(wl, nnz) / (4.0 * wl.d * 128 * 128 *
                                                                     n_box)})
+        # the backward over the same box tiles: 7 products of 2*d*128*128 FLOP per
+        # (query box, key box) pair executed; 5 per kept chunk pair are the gradient's
+        dout = torch.from_numpy(synth.make_dout(wl)).view(torch.bfloat16).to("cuda")
+        lse = torch.empty((wl.B, wl.heads, wl.N), dtype=torch.float32, device="cuda")
+        bsa.bsa_forward(p, q, k, v, pl.row_ptr, pl.col_idx, pl.workspace, out, lse)
+        ws = bsa.backward_workspace(p)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def bwd():
+            bsa.bsa_backward(p, q, k, v, out, lse, dout, pl.row_ptr, pl.col_idx, ws, dq, dk, dv)
+
+        for _ in range(3):
+            bwd()
+        torch.cuda.synchronize()
+        bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for a, b in bev:
+            a.record(stream)
+            bwd()
+            b.record(stream)
+        torch.cuda.synchronize()
+        bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in bev)
+        bwd_tile_tf = 3.5 * 4.0 * wl.d * 128 * 128 * n_box / bwd_ms / 1e9
+        res["backward"] = {"bwd_ms": bwd_ms, "steps": steps,
+                           "alg_tflops": 2.5 * exec_flops(wl, nnz) / bwd_ms / 1e9,
+                           "tile_tflops": bwd_tile_tf, "tile_frac": bwd_tile_tf / peak_tf,
+                           "device_status": bsa.status_string(bsa.bsa_read_status(ws))}
+        del dout, lse, ws, dq, dk, dv
     del q, k, v, out, pl
     torch.cuda.empty_cache()
     return res

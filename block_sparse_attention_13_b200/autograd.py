@@ -51,16 +51,20 @@ class _BlockSparseAttention(torch.autograd.Function):
 
 
 def block_sparse_attention_train(q, k, v, grid, topk=None, mode="topk", cdf_p=0.9,
-                                 cdf_cap_frac=0.25, t_cond=0, scale=0.0):
+                                 cdf_cap_frac=0.25, t_cond=0, scale=0.0, chunk=(4, 4, 8),
+                                 kchunk=(0, 0, 0)):
     """Differentiable block sparse attention of q, k, v [B, heads, T*H*W, d] bf16
-    (CUDA tensors, tokens in [T,H,W] order). grid = (T, H, W); topk defaults to
-    1/16 of the key chunks. Returns out; out.backward(...) fills q.grad, k.grad and
-    v.grad through bsa_backward."""
+    (CUDA tensors, tokens in [T,H,W] order). grid = (T, H, W); chunk = the query
+    chunk shape, (4, 4, 8) or (4, 4, 4); kchunk = the key chunk shape (0 = the query
+    chunk's); topk defaults to 1/16 of the key chunks. Returns out; out.backward(...)
+    fills q.grad, k.grad and v.grad through bsa_backward."""
     B, heads, N, d = q.shape
     T, H, W = grid
     if T * H * W != N:
         raise ValueError("grid does not match the token count")
     if topk is None:
-        topk = max(1, (-(-T // 4) * -(-H // 4) * -(-W // 8)) // 16)
-    p = make_params(B, heads, T, H, W, d, mode, topk, cdf_p, cdf_cap_frac, t_cond, scale)
+        kc = tuple(c if c else q_ for c, q_ in zip(kchunk, chunk))
+        topk = max(1, (-(-T // kc[0]) * -(-H // kc[1]) * -(-W // kc[2])) // 16)
+    p = make_params(B, heads, T, H, W, d, mode, topk, cdf_p, cdf_cap_frac, t_cond, scale,
+                    kchunk=kchunk, chunk=chunk)
     return _BlockSparseAttention.apply(q, k, v, p)

@@ -223,12 +223,7 @@ cudaError_t launch_forward_any(const Dims& g, const bsa_params& p, const void* q
     cudaError_t e = launch_quad_union(g, row_ptr, col_idx, col_cap, bcnt, brp, bci, bpat,
                                       L.box_cap, status, st);
     if (e != cudaSuccess) return e;
-    Dims gb = g;
-    gb.Nc = gb.Nq = g.NB;
-    gb.q_skip = 0;
-    gb.rows = g.BH * g.NB;
-    gb.qw = kChunkW;
-    gb.NWq = g.NW;
+    const Dims gb = box_dims(g);
     return launch_forward(gb, q, k, v, brp, bci, L.box_cap, out, lse, status, timeout_ns,
                           debug_flags, st, out_f32, bpat);
 }
@@ -254,7 +249,7 @@ using namespace bsa;
 
 extern "C" {
 
-int bsa_version(void) { return 300; }
+int bsa_version(void) { return 301; }
 
 const char* bsa_status_string(int s) {
     switch (s) {
@@ -404,8 +399,8 @@ int bsa_forward(const bsa_params* p, const void* q, const void* k, const void* v
 
 size_t bsa_backward_workspace_size(const bsa_params* p) {
     Dims g;
-    if (make_dims(p, &g) != BSA_OK || g.qw != kChunkW) return 0;
-    return bwd_layout(g).total;
+    if (make_dims(p, &g) != BSA_OK) return 0;
+    return bwd_layout(g, *p).total;
 }
 
 int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* v,
@@ -416,7 +411,6 @@ int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* 
     Dims g;
     int rc = make_dims(p, &g);
     if (rc != BSA_OK) return rc;
-    if (g.qw != kChunkW) return BSA_ERR_UNSUPPORTED;  // 64-token chunks: forward only
     if (!q || !k || !v || !out || !lse || !dout || !row_ptr || !col_idx || !workspace || !dq ||
         !dk || !dv || col_capacity < 0)
         return BSA_ERR_INVALID_ARG;
@@ -424,9 +418,9 @@ int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* 
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) ||
         !aligned4(lse) || !aligned4(row_ptr) || !aligned4(col_idx))
         return BSA_ERR_ALIGNMENT;
-    if (ws_bytes < bwd_layout(g).total) return BSA_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_bytes < bwd_layout(g, *p).total) return BSA_ERR_WORKSPACE_TOO_SMALL;
     if ((rc = device_ok()) != BSA_OK) return rc;
-    return cuda_status(launch_backward(g, q, k, v, out, lse, dout, row_ptr, col_idx, col_capacity,
+    return cuda_status(launch_backward(g, *p, q, k, v, out, lse, dout, row_ptr, col_idx, col_capacity,
                                        workspace, dq, dk, dv, kDefaultTimeoutNs,
                                        static_cast<cudaStream_t>(stream)));
 }

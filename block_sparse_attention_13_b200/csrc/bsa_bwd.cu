@@ -189,7 +189,8 @@ struct BwdCfg {
     static constexpr int kAux = 6 * kTileBytes;
     static constexpr int kCtl = kAux + 3 * 1024;
     static constexpr int kList = kCtl + 512;
-    static constexpr int kSmemBytes = kList + kMaxList * 2 + 1024;  // + alignment slack
+    static constexpr int kPat = kList + kMaxList * 2;    // quadrant pattern per list entry
+    static constexpr int kSmemBytes = kPat + kMaxList + 1024;  // + alignment slack
 };
 
 struct BwdArgs {
@@ -200,6 +201,11 @@ struct BwdArgs {
     const int32_t* row_idx;
     int64_t idx_cap;
     const float* aux;         // [BH][Nq][half][LSE*log2(e) x64 | D x64]
+    // 64-token query chunks (rows and key chunks are (4,4,8) boxes): the quadrant
+    // pattern of every CSR entry and of every CSC entry (bit 2*hq + hk: the query
+    // box's half hq attends to the key box's half hk; halves split w at 4)
+    const uint8_t* row_pat;
+    const uint8_t* col_pat;
     __nv_bfloat16* dq;        // for zero rows / columns written without TMA
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
@@ -323,7 +329,7 @@ __device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int half, 
     tmem_st32(taddr, r);
 }
 
-template <int D>
+template <int D, bool kQuad>
 __global__ void __launch_bounds__(320, 1)
     bsa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -339,6 +345,7 @@ __global__ void __launch_bounds__(320, 1)
     auto sV = [&](int s) { return s == 0 ? smem + 5 * C::kTileBytes : sQ; };
     DqCtl* ctl = reinterpret_cast<DqCtl*>(smem + C::kCtl);
     uint16_t* list = reinterpret_cast<uint16_t*>(smem + C::kList);
+    uint8_t* plist = smem + C::kPat;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t row = blockIdx.x;
@@ -379,7 +386,11 @@ __global__ void __launch_bounds__(320, 1)
             const bool valid = e < end && c >= 0 && c < a.Nc;
             if (e < end && !valid) bad = true;
             const uint32_t vb = __ballot_sync(0xffffffffu, valid);
-            if (valid) list[cnt + __popc(vb & ((1u << lane) - 1u))] = static_cast<uint16_t>(c);
+            if (valid) {
+                const int slot = cnt + __popc(vb & ((1u << lane) - 1u));
+                list[slot] = static_cast<uint16_t>(c);
+                if constexpr (kQuad) plist[slot] = a.row_pat[e];
+            }
             cnt += __popc(vb);
         }
         if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.status, kStatusBadIndex);
@@ -585,6 +596,15 @@ __global__ void __launch_bounds__(320, 1)
             bool got = mbar_wait(&ctl->s_full, j & 1, abort_flag, a.status, tmo, site(3, 4, 0, j));
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
+            // 64-token query chunks: the key halves this query row attends to in this box
+            // (its query half is bit 2 of its w index); masked weights are set to 0
+            // after the exponential, so they never enter any arithmetic
+            bool keep_a = true, keep_b = true;
+            if constexpr (kQuad) {
+                const uint32_t mine = (plist[j] >> ((m & 4) ? 2 : 0)) & 3u;
+                keep_a = mine & 1u;
+                keep_b = mine & 2u;
+            }
             float p[64];
             {
                 uint32_t sv0[32], sv1[32];
@@ -606,7 +626,10 @@ __global__ void __launch_bounds__(320, 1)
                     const int o = 2 * (e & 15);
                     const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[o]), __uint_as_float(sv[o + 1])),
                                                 cc, nl);
-                    const float2 pe = exp2_pair(x, e);
+                    float2 pe = exp2_pair(x, e);
+                    // pair e holds key slots whose w index has bit 2 equal to bit 1 of e
+                    if constexpr (kQuad)
+                        if (!((e & 2) ? keep_b : keep_a)) pe = make_float2(0.0f, 0.0f);
                     p[2 * e] = pe.x;
                     p[2 * e + 1] = pe.y;
                 }
@@ -702,10 +725,13 @@ struct __align__(8) DkvCtl {
     int abort_flag;
 };
 
-// Stage a CSC column's query rows in shared memory (out-of-range entries dropped
-// and reported); returns the count on lane 0 (every lane of the calling warp
-// takes part).
-__device__ __forceinline__ int stage_column(const BwdArgs& a, int64_t col, uint16_t* list, int lane) {
+// Stage a CSC column's query rows (and, for 64-token query chunks, their
+// quadrant patterns) in shared memory (out-of-range entries dropped and
+// reported); returns the count on lane 0 (every lane of the calling warp takes
+// part).
+template <bool kQuad>
+__device__ __forceinline__ int stage_column(const BwdArgs& a, int64_t col, uint16_t* list,
+                                            uint8_t* plist, int lane) {
     bool bad = false;
     int64_t beg = a.col_ptr[col], end = a.col_ptr[col + 1];
     if (!(beg >= 0 && end >= beg && end <= a.idx_cap && end - beg <= a.Nq)) {
@@ -719,14 +745,18 @@ __device__ __forceinline__ int stage_column(const BwdArgs& a, int64_t col, uint1
         const bool valid = e < end && r >= 0 && r < a.Nq;
         if (e < end && !valid) bad = true;
         const uint32_t vb = __ballot_sync(0xffffffffu, valid);
-        if (valid) list[cnt + __popc(vb & ((1u << lane) - 1u))] = static_cast<uint16_t>(r);
+        if (valid) {
+            const int slot = cnt + __popc(vb & ((1u << lane) - 1u));
+            list[slot] = static_cast<uint16_t>(r);
+            if constexpr (kQuad) plist[slot] = a.col_pat[e];
+        }
         cnt += __popc(vb);
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.status, kStatusBadIndex);
     return cnt;
 }
 
-template <int D>
+template <int D, bool kQuad>
 __global__ void __launch_bounds__(320, 1)
     bsa_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -743,6 +773,7 @@ __global__ void __launch_bounds__(320, 1)
     float* sAux = reinterpret_cast<float*>(smem + C::kAux);  // [slot][half][lse2 64 | D 64]
     DkvCtl* ctl = reinterpret_cast<DkvCtl*>(smem + C::kCtl);
     uint16_t* list = reinterpret_cast<uint16_t*>(smem + C::kList);
+    uint8_t* plist = smem + C::kPat;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t col = blockIdx.x;
@@ -768,7 +799,7 @@ __global__ void __launch_bounds__(320, 1)
         fence_proxy_async_smem();
     }
     if (warp == C::kTmaWarp) {
-        const int cnt = stage_column(a, col, list, lane);
+        const int cnt = stage_column<kQuad>(a, col, list, plist, lane);
         if (lane == 0) {
             ctl->n_valid = cnt;
             prefetch_tensormap(&tm_q);
@@ -957,6 +988,15 @@ __global__ void __launch_bounds__(320, 1)
             got = mbar_wait(&ctl->s_full, i & 1, abort_flag, a.status, tmo, site(3, 4, 0, i));
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
+            // 64-token query chunks: which query halves this key row (its half is bit 2
+            // of its w index) is attended by in this box pair; masked weights are set
+            // to 0 after the exponential
+            bool keep_q0 = true, keep_q1 = true;
+            if constexpr (kQuad) {
+                const uint32_t pat = plist[i], hk = (m & 4) ? 1u : 0u;
+                keep_q0 = (pat >> hk) & 1u;
+                keep_q1 = (pat >> (2u + hk)) & 1u;
+            }
             float p[64];
             uint32_t pk[32];
             {
@@ -975,7 +1015,10 @@ __global__ void __launch_bounds__(320, 1)
                         const float2 x = __ffma2_rn(
                             make_float2(__uint_as_float(sv[o + 2 * h]), __uint_as_float(sv[o + 2 * h + 1])),
                             cc, h == 0 ? make_float2(-l4.x, -l4.y) : make_float2(-l4.z, -l4.w));
-                        const float2 pe = exp2_pair(x, 2 * e4 + h);
+                        float2 pe = exp2_pair(x, 2 * e4 + h);
+                        // columns 4*e4 + 2h, +1: query w index with bit 2 equal to bit 0 of e4
+                        if constexpr (kQuad)
+                            if (!((e4 & 1) ? keep_q1 : keep_q0)) pe = make_float2(0.0f, 0.0f);
                         p[4 * e4 + 2 * h] = pe.x;
                         p[4 * e4 + 2 * h + 1] = pe.y;
                         pk[2 * e4 + h] = pack_bf16x2(pe.x, pe.y);
@@ -1058,30 +1101,81 @@ __global__ void __launch_bounds__(320, 1)
     }
 }
 
-template <int D>
-cudaError_t launch_bwd_d(const Dims& g, const CUtensorMap* m, const BwdArgs& dq_args,
-                         const BwdArgs& dkv_args, cudaStream_t st) {
+// 64-token query chunks: the quadrant pattern of every CSC entry (column c, query
+// box r) is the pattern of the box CSR entry (r, c), found by binary search in
+// row r's ascending list. One warp per column.
+__global__ void __launch_bounds__(256) csc_pattern_kernel(
+    const int32_t* __restrict__ col_ptr, const int32_t* __restrict__ row_idx, int64_t idx_cap,
+    const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx, int64_t col_cap,
+    const uint8_t* __restrict__ row_pat, int64_t cols, int Nq, int Nc, uint8_t* __restrict__ col_pat,
+    uint32_t* status) {
+    const int64_t c = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (c >= cols) return;
+    const int64_t bh = c / Nc;
+    const int kc = static_cast<int>(c % Nc);
+    int64_t beg = col_ptr[c], end = col_ptr[c + 1];
+    if (!(beg >= 0 && end >= beg && end <= idx_cap)) {
+        if (lane == 0) atomicOr(status, kStatusBadIndex);
+        return;
+    }
+    for (int64_t e = beg + lane; e < end; e += 32) {
+        const int r = row_idx[e];
+        uint8_t pat = 0;
+        if (r >= 0 && r < Nq) {
+            const int64_t row = bh * Nq + r;
+            int64_t lo = row_ptr[row], hi = row_ptr[row + 1];
+            if (lo >= 0 && hi >= lo && hi <= col_cap) {
+                while (lo < hi) {  // first entry >= kc
+                    const int64_t mid = (lo + hi) >> 1;
+                    if (col_idx[mid] < kc) lo = mid + 1; else hi = mid;
+                }
+                if (lo < row_ptr[row + 1] && col_idx[lo] == kc) pat = row_pat[lo];
+                else atomicOr(status, kStatusBadIndex);
+            } else {
+                atomicOr(status, kStatusBadIndex);
+            }
+        }
+        col_pat[e] = pat;
+    }
+}
+
+template <int D, bool kQuad>
+cudaError_t launch_bwd_dq(const CUtensorMap* m, const BwdArgs& dq_args, const BwdArgs& dkv_args,
+                          cudaStream_t st) {
     using C = BwdCfg<D>;
     static std::atomic<uint64_t> dq_attr{0}, dkv_attr{0};
     {
-        cudaError_t e = raise_smem_limit(bsa_bwd_dq_kernel<D>, C::kSmemBytes, dq_attr);
-        if (e == cudaSuccess) e = raise_smem_limit(bsa_bwd_dkv_kernel<D>, C::kSmemBytes, dkv_attr);
+        cudaError_t e = raise_smem_limit(bsa_bwd_dq_kernel<D, kQuad>, C::kSmemBytes, dq_attr);
+        if (e == cudaSuccess)
+            e = raise_smem_limit(bsa_bwd_dkv_kernel<D, kQuad>, C::kSmemBytes, dkv_attr);
         if (e != cudaSuccess) return e;
     }
     // m: q, k, v, dout, dq, dk, dv (whole chunks)
-    bsa_bwd_dq_kernel<D><<<static_cast<unsigned>(dq_args.units), C::kThreads, C::kSmemBytes, st>>>(
-        m[0], m[1], m[2], m[3], m[4], dq_args);
+    bsa_bwd_dq_kernel<D, kQuad>
+        <<<static_cast<unsigned>(dq_args.units), C::kThreads, C::kSmemBytes, st>>>(
+            m[0], m[1], m[2], m[3], m[4], dq_args);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bsa_bwd_dkv_kernel<D><<<static_cast<unsigned>(dkv_args.units), C::kThreads, C::kSmemBytes, st>>>(
-        m[0], m[1], m[2], m[3], m[5], m[6], dkv_args);
+    bsa_bwd_dkv_kernel<D, kQuad>
+        <<<static_cast<unsigned>(dkv_args.units), C::kThreads, C::kSmemBytes, st>>>(
+            m[0], m[1], m[2], m[3], m[5], m[6], dkv_args);
     return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const CUtensorMap* m, const BwdArgs& dq_args, const BwdArgs& dkv_args,
+                         bool quad, cudaStream_t st) {
+    return quad ? launch_bwd_dq<D, true>(m, dq_args, dkv_args, st)
+                : launch_bwd_dq<D, false>(m, dq_args, dkv_args, st);
 }
 
 }  // namespace
 
-BwdLayout bwd_layout(const Dims& g) {
+BwdLayout bwd_layout(const Dims& g0, const bsa_params& p) {
     auto round_up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const bool quad = g0.qw != kChunkW;
+    const Dims g = quad ? box_dims(g0) : g0;
     BwdLayout L{};
     L.words = (g.Nq + 31) / 32;
     L.idx_cap = g.rows * static_cast<int64_t>(g.Nc);  // every (row, chunk) pair
@@ -1101,16 +1195,36 @@ BwdLayout bwd_layout(const Dims& g) {
     off += round_up((cols + 1) * sizeof(int32_t));
     L.row_idx = off;
     off += round_up(static_cast<size_t>(L.idx_cap) * sizeof(int32_t));
+    L.box_counts = L.box_row_ptr = L.box_col_idx = L.box_pat = L.csc_pat = off;
+    L.box_cap = 0;
+    if (quad) {
+        L.box_cap = ws_layout(g0, p).box_cap;  // the forward's bound on a box row's union
+        const size_t box_rows = static_cast<size_t>(g0.BH) * g0.NB;
+        L.box_counts = off;
+        off += round_up(box_rows * sizeof(int32_t));
+        L.box_row_ptr = off;
+        off += round_up((box_rows + 1) * sizeof(int32_t));
+        L.box_col_idx = off;
+        off += round_up(static_cast<size_t>(L.box_cap) * sizeof(int32_t));
+        L.box_pat = off;
+        off += round_up(static_cast<size_t>(L.box_cap));
+        L.csc_pat = off;
+        off += round_up(static_cast<size_t>(L.idx_cap));
+    }
     L.total = off;
     return L;
 }
 
-cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const void* v,
-                            const void* out, const float* lse, const void* dout,
+cudaError_t launch_backward(const Dims& g0, const bsa_params& p, const void* q, const void* k,
+                            const void* v, const void* out, const float* lse, const void* dout,
                             const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
                             void* workspace, void* dq, void* dk, void* dv, uint64_t timeout_ns,
                             cudaStream_t st) {
-    const BwdLayout L = bwd_layout(g);
+    const BwdLayout L = bwd_layout(g0, p);
+    // 64-token query chunks: the attention kernels work on (4,4,8) boxes, over the
+    // box CSR with a quadrant pattern per entry (the forward's own construction)
+    const bool quad = g0.qw != kChunkW;
+    const Dims g = quad ? box_dims(g0) : g0;
     char* ws = static_cast<char*>(workspace);
     uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
     float* aux = reinterpret_cast<float*>(ws + L.aux);
@@ -1129,6 +1243,25 @@ cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const v
 
     cudaError_t e = cudaMemsetAsync(ws + L.bitmap, 0, L.cnt - L.bitmap, st);  // bitmap + rawcnt
     if (e != cudaSuccess) return e;
+    const int32_t* rp = row_ptr;
+    const int32_t* ci = col_idx;
+    int64_t cap = col_cap;
+    const uint8_t* rpat = nullptr;
+    uint8_t* cpat = nullptr;
+    if (quad) {
+        int32_t* bcnt = reinterpret_cast<int32_t*>(ws + L.box_counts);
+        int32_t* brp = reinterpret_cast<int32_t*>(ws + L.box_row_ptr);
+        int32_t* bci = reinterpret_cast<int32_t*>(ws + L.box_col_idx);
+        uint8_t* bpat = reinterpret_cast<uint8_t*>(ws + L.box_pat);
+        if ((e = launch_quad_union(g0, row_ptr, col_idx, col_cap, bcnt, brp, bci, bpat, L.box_cap,
+                                   status, st)) != cudaSuccess)
+            return e;
+        rp = brp;
+        ci = bci;
+        cap = L.box_cap;
+        rpat = bpat;
+        cpat = reinterpret_cast<uint8_t*>(ws + L.csc_pat);
+    }
     dim3 pgrid(static_cast<unsigned>(g.Nq), static_cast<unsigned>(g.BH));
     const auto* o16 = static_cast<const __nv_bfloat16*>(out);
     const auto* g16 = static_cast<const __nv_bfloat16*>(dout);
@@ -1140,7 +1273,7 @@ cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const v
                                                   g.W, g.NH, g.NW, g.N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     csc_scatter_kernel<<<static_cast<unsigned>((g.rows + 7) / 8), 256, 0, st>>>(
-        row_ptr, col_idx, col_cap, g.rows, g.Nq, g.Nc, L.words, bitmap, rawcnt, status);
+        rp, ci, cap, g.rows, g.Nq, g.Nc, L.words, bitmap, rawcnt, status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     csc_count_kernel<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(bitmap, rawcnt,
                                                                                L.words, cols, cnt,
@@ -1150,15 +1283,22 @@ cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const v
     csc_emit_kernel<<<static_cast<unsigned>((cols + 7) / 8), 256, 0, st>>>(
         bitmap, L.words, cols, col_ptr, row_idx, L.idx_cap, status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (quad) {
+        csc_pattern_kernel<<<static_cast<unsigned>((cols + 7) / 8), 256, 0, st>>>(
+            col_ptr, row_idx, L.idx_cap, rp, ci, cap, rpat, cols, g.Nq, g.Nc, cpat, status);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
 
     BwdArgs args{};
-    args.row_ptr = row_ptr;
-    args.col_idx = col_idx;
-    args.col_cap = col_cap;
+    args.row_ptr = rp;
+    args.col_idx = ci;
+    args.col_cap = cap;
     args.col_ptr = col_ptr;
     args.row_idx = row_idx;
     args.idx_cap = L.idx_cap;
     args.aux = aux;
+    args.row_pat = rpat;
+    args.col_pat = cpat;
     args.dq = static_cast<__nv_bfloat16*>(dq);
     args.dk = static_cast<__nv_bfloat16*>(dk);
     args.dv = static_cast<__nv_bfloat16*>(dv);
@@ -1178,8 +1318,8 @@ cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const v
     BwdArgs dq_args = args, dkv_args = args;
     dq_args.units = g.rows;
     dkv_args.units = cols;
-    return g.d == 128 ? launch_bwd_d<128>(g, m, dq_args, dkv_args, st)
-                      : launch_bwd_d<64>(g, m, dq_args, dkv_args, st);
+    return g.d == 128 ? launch_bwd_d<128>(m, dq_args, dkv_args, quad, st)
+                      : launch_bwd_d<64>(m, dq_args, dkv_args, quad, st);
 }
 
 }  // namespace bsa

@@ -105,7 +105,20 @@ int make_dims(const bsa_params* p, Dims* g);
 int64_t max_nnz_of(const Dims& g, const bsa_params& p);
 int device_ok();
 
-// Backward workspace layout (byte offsets).
+// 64-token query chunks: the dims of the attention kernels, whose rows are
+// (4,4,8) boxes of two query chunks and whose key chunks are (4,4,8) boxes.
+inline Dims box_dims(const Dims& g) {
+    Dims gb = g;
+    gb.Nc = gb.Nq = g.NB;
+    gb.q_skip = 0;
+    gb.rows = g.BH * g.NB;
+    gb.qw = kChunkW;
+    gb.NWq = g.NW;
+    return gb;
+}
+
+// Backward workspace layout (byte offsets). With 64-token query chunks every
+// size below is over boxes (box_dims), after the box CSR of the call.
 struct BwdLayout {
     size_t status;   // uint32 status word (+ padding to 256)
     size_t aux;      // float [BH][Nq][2][128]: per half of 64 queries, LSE * log2(e) then <dO, O>
@@ -116,10 +129,18 @@ struct BwdLayout {
     size_t row_idx;  // int32 [idx_cap]
     int words;       // ceil(Nq / 32)
     int64_t idx_cap; // BH * Nq * Nc
+    // 64-token query chunks only: the box CSR (launch_quad_union) and the quadrant
+    // pattern of every CSC entry
+    size_t box_counts;  // int32 [BH*NB]
+    size_t box_row_ptr; // int32 [BH*NB+1]
+    size_t box_col_idx; // int32 [box_cap]
+    size_t box_pat;     // uint8 [box_cap]
+    int64_t box_cap;
+    size_t csc_pat;     // uint8 [idx_cap]
     size_t total;
 };
 
-BwdLayout bwd_layout(const Dims& g);
+BwdLayout bwd_layout(const Dims& g, const bsa_params& p);
 
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_pool(const Dims& g, const void* x0, const void* x1, float* p0, float* p1,
@@ -168,8 +189,8 @@ cudaError_t launch_forward_any(const Dims& g, const bsa_params& p, const void* q
                                int64_t col_cap, char* ws, uint32_t* status, void* out, float* lse,
                                uint64_t timeout_ns, int debug_flags, cudaStream_t st,
                                float* out_f32);
-cudaError_t launch_backward(const Dims& g, const void* q, const void* k, const void* v,
-                            const void* out, const float* lse, const void* dout,
+cudaError_t launch_backward(const Dims& g, const bsa_params& p, const void* q, const void* k,
+                            const void* v, const void* out, const float* lse, const void* dout,
                             const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
                             void* workspace, void* dq, void* dk, void* dv, uint64_t timeout_ns,
                             cudaStream_t st);

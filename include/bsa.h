@@ -112,7 +112,7 @@ typedef struct {
 
 /* Library version: major*10000 + minor*100 + patch (0.2.0: bsa_shape_info and
  * bsa_forward_host added; 0.3.0: 64-token chunks, bsa_forward_partial and
- * bsa_lse_merge_f32). */
+ * bsa_lse_merge_f32; 0.3.1: bsa_backward for 64-token chunks). */
 BSA_API int bsa_version(void);
 
 /* Text for a status code (static storage; never NULL). */
@@ -208,7 +208,9 @@ BSA_API int bsa_forward_partial(const bsa_params* p, const void* q, const void* 
  * Bytes of device workspace that bsa_backward needs for `p` (0 if `p` is
  * invalid): a status block, LSE and <dO,O> per computed query token, and the
  * column-major (CSC) copy of a block mask of at most one entry per (row, key
- * chunk) pair. Host-only call.
+ * chunk) pair; for 64-token query chunks these are over (4,4,8) boxes, after
+ * the box CSR (as the forward builds it) and a quadrant pattern per CSC
+ * entry. Host-only call.
  */
 BSA_API size_t bsa_backward_workspace_size(const bsa_params* p);
 
@@ -219,7 +221,10 @@ BSA_API size_t bsa_backward_workspace_size(const bsa_params* p);
  * With P = exp(QK^T*scale - lse) over the selected keys and D = <dout, out>
  * per query: dV = P^T dout, dS = P * (dout V^T - D), dQ = scale dS K,
  * dK = scale dS^T Q, each summed over the chunks of the CSR only. The block
- * selection itself has no gradient.
+ * selection itself has no gradient. 64-token query chunks ([P1] block-size
+ * robustness) are supported as in bsa_forward: the kernels run over (4,4,8)
+ * boxes of two query chunks and the union of their key boxes, each query
+ * attending only to the key chunks its own chunk selected.
  * q, k, v, out, dout: device bf16 [B,heads,N,d] (out and lse exactly as
  * bsa_forward wrote them for the same CSR). lse: device fp32 [B,heads,N].
  * dq, dk, dv: device bf16 [B,heads,N,d], written in [T,H,W] token order:

@@ -42,7 +42,7 @@ def test_library_exports_nothing_else():
 
 
 def test_version_and_strings(L):
-    assert bsa.bsa_version() == 300
+    assert bsa.bsa_version() == 301
     for code in range(0, 10):
         s = bsa.status_string(code)
         assert s and s != "unknown status"
@@ -161,16 +161,20 @@ def test_query_chunk_shape_validation(L, kw, code):
     assert rc_sizes(P(T=16, H=16, W=32, **kw))[0] == code
 
 
-def test_64_token_chunks_limits_and_forward_only_entries(L):
+def test_64_token_chunks_limits_and_entries_that_take_128_token_chunks(L):
     # chunks per (batch, head) are limited to 2,048: the long grid in 64-token chunks
     # (14 x 12 x 20 = 3,360) is not supported
     assert rc_sizes(P(T=56, H=48, W=80, d=128, topk=5, chunk=(4, 4, 4)))[0] == \
         bsa.BSA_ERR_UNSUPPORTED
     p = P(T=16, H=16, W=32, chunk=(4, 4, 4))
     x = vp(FAKE)
-    assert L.bsa_backward_workspace_size(ctypes.byref(p)) == 0
-    assert L.bsa_backward(ctypes.byref(p), x, x, x, x, x, x, x, x, 64, x, 1 << 20, x, x, x,
-                          None) == bsa.BSA_ERR_UNSUPPORTED
+    # the backward works on (4,4,8) boxes: its workspace holds the box CSR and the
+    # backward layout over boxes, and it is checked before any CUDA call
+    p128 = P(T=16, H=16, W=32)
+    ws = L.bsa_backward_workspace_size(ctypes.byref(p))
+    assert ws > L.bsa_backward_workspace_size(ctypes.byref(p128)) > 0
+    assert L.bsa_backward(ctypes.byref(p), x, x, x, x, x, x, x, x, 64, x, ws - 1, x, x, x,
+                          None) == bsa.BSA_ERR_WORKSPACE_TOO_SMALL
     assert L.bsa_rearrange(ctypes.byref(p), x, x, 0, None) == bsa.BSA_ERR_UNSUPPORTED
     assert L.bsa_select_pooled(ctypes.byref(p), x, x, 0, x, 1 << 30, x, x, 1 << 20, None) == \
         bsa.BSA_ERR_UNSUPPORTED

@@ -74,7 +74,12 @@ def check_bwd(wl, csr=None):
     rp, ci, out, lse, dq, dk, dv, st_f, st_b = gpu_fwd_bwd(wl, q, k, v, g, csr)
     assert st_f == bsa.BSA_OK and st_b == bsa.BSA_OK, (st_f, st_b)
     rows = np.arange(wl.rows)
-    o_dq, o_dk, o_dv = oracle.attend_bwd(q, k, v, g, wl.T, wl.H, wl.W, scale, rp, ci, rows)
+    # 64-token query chunks: the plan's CSR is over the chunks themselves (the library
+    # builds the box CSR inside the forward and backward); otherwise it is over boxes
+    shapes = dict(kchunk=tuple(wl.kchunk), qchunk=tuple(wl.qchunk)) \
+        if tuple(wl.qchunk) == (4, 4, 4) else {}
+    o_dq, o_dk, o_dv = oracle.attend_bwd(q, k, v, g, wl.T, wl.H, wl.W, scale, rp, ci, rows,
+                                         **shapes)
     errs = {
         "dq": rel_errors(gather_rows(host_f32(dq), wl, rows), o_dq),
         "dk": rel_errors(host_f32(dk), o_dk),
@@ -85,9 +90,35 @@ def check_bwd(wl, csr=None):
     return errs
 
 
-@pytest.mark.parametrize("name", sorted(n for n in SMALL if tuple(SMALL[n].qchunk) == (4, 4, 8)))
+@pytest.mark.parametrize("name", sorted(SMALL))
 def test_backward_small_cases(name):
     check_bwd(SMALL[name])
+
+
+def test_backward_64_token_chunks_with_an_empty_chunk_and_unselected_halves():
+    """64-token query chunks with a caller CSR: one query chunk selects nothing
+    (its queries have no output: dQ exactly 0) and some 64-token key chunks no
+    query chunk selects (dK, dV exactly 0), beside chunks whose box partner
+    selected different keys."""
+    wl = SMALL["q64_k64"]
+    q, k, v = synth.make_qkv(wl)
+    rp, ci, _ = oracle.plan(q, k, wl.T, wl.H, wl.W, wl.softmax_scale, wl.mode, wl.topk,
+                            kchunk=tuple(wl.kchunk), qchunk=tuple(wl.qchunk))
+    lists = [list(ci[rp[r]:rp[r + 1]]) for r in range(wl.rows)]
+    lists[3] = []                                        # head 0, chunk 3: no keys
+    unused = {5, 6}                                      # key chunks 5, 6 of head 0: never kept
+    lists = [[c for c in row if not (r < wl.Nc and c in unused)] for r, row in enumerate(lists)]
+    rp2 = np.concatenate([[0], np.cumsum([len(r) for r in lists])]).astype(np.int32)
+    ci2 = np.array([c for row in lists for c in row], dtype=np.int32)
+    check_bwd(wl, csr=(rp2, ci2))
+    g = synth.make_dout(wl)
+    _, _, _, _, dq, dk, dv, _, _ = gpu_fwd_bwd(wl, q, k, v, g, csr=(rp2, ci2))
+    dqh = gather_rows(host_f32(dq), wl, np.array([3]))
+    assert np.all(dqh == 0)
+    for c in unused:
+        toks = oracle.chunk_tokens(wl.T, wl.H, wl.W, c, tuple(wl.kchunk))
+        toks = toks[toks >= 0]
+        assert np.all(host_f32(dk)[0, 0][toks] == 0) and np.all(host_f32(dv)[0, 0][toks] == 0)
 
 
 def test_backward_all_chunks_selected():
@@ -190,14 +221,16 @@ def test_backward_deterministic():
         assert torch.equal(x.view(torch.int16), y.view(torch.int16))
 
 
-@pytest.mark.parametrize("name", ["720p", "720p_real"])
+@pytest.mark.parametrize("name", ["720p", "720p_real", "720p_q64"])
 def test_backward_full_size_720p_sampled(name):
     """Full 720p grids, 32 heads, in the launch configuration of the benchmark
-    (720p_real has partial edge chunks): dQ of sampled rows and dK/dV of a
-    sampled key chunk of (batch 0, head 0) against the oracle, plus the
-    invariants sum(dK) = 0 and sum(dV) = sum(dO) per head (every row is
-    non-empty under top-k)."""
+    (720p_real has partial edge chunks, 720p_q64 64-token query and key chunks):
+    dQ of sampled rows and dK/dV of a sampled key chunk of (batch 0, head 0)
+    against the oracle, plus the invariants sum(dK) = 0 and sum(dV) = sum(dO)
+    per head (every row is non-empty under top-k)."""
     wl = W[name]
+    q64 = tuple(wl.qchunk) == (4, 4, 4)
+    shapes = dict(kchunk=tuple(wl.kchunk), qchunk=tuple(wl.qchunk)) if q64 else {}
     q, k, v = synth.make_qkv(wl)
     g = synth.make_dout(wl)
     scale = 1.0 / math.sqrt(wl.d)
@@ -220,11 +253,13 @@ def test_backward_full_size_720p_sampled(name):
     col_rows = np.array([r for r in range(wl.Nc) if col in ci0[rp0[r]:rp0[r + 1]]])
     rows = np.unique(np.concatenate([sample_rows, col_rows]))
     w1 = wl.with_(heads=1)
-    o_dq, o_dk, o_dv = oracle.attend_bwd(q0, k0, v0, g0, wl.T, wl.H, wl.W, scale, rp0, ci0, rows)
+    o_dq, o_dk, o_dv = oracle.attend_bwd(q0, k0, v0, g0, wl.T, wl.H, wl.W, scale, rp0, ci0, rows,
+                                         **shapes)
     sel = np.isin(rows, sample_rows)
     mx, mean = rel_errors(gather_rows(host_f32(dq[:, :1]), w1, sample_rows), o_dq[sel])
     assert mx <= BWD_MAX_REL and mean <= BWD_MEAN_REL, ("dq", mx, mean)
-    toks = oracle.chunk_tokens(wl.T, wl.H, wl.W, col)
+    toks = oracle.chunk_tokens(wl.T, wl.H, wl.W, col, *([tuple(wl.kchunk)] if q64 else []))
+    toks = toks[toks >= 0]
     for name, gx, ox in (("dk", dk, o_dk), ("dv", dv, o_dv)):
         mx, mean = rel_errors(host_f32(gx[0, 0, toks]), ox[0, 0, toks])
         assert mx <= BWD_MAX_REL and mean <= BWD_MEAN_REL, (name, col, mx, mean)
