@@ -193,11 +193,13 @@ def test_backward_kv_cached_rows():
     assert torch.all(dq[:, :, : wl.q_begin * HW] == 7.0)
 
 
-def test_autograd_op_matches_the_c_abi_calls():
+@pytest.mark.parametrize("name", ["ragged135_d128", "q64_k128"])
+def test_autograd_op_matches_the_c_abi_calls(name):
     """block_sparse_attention_train (torch.autograd) runs the same plan, forward and
-    backward as the direct C-ABI calls: outputs and gradients bit for bit."""
+    backward as the direct C-ABI calls: outputs and gradients bit for bit (also with
+    64-token query chunks)."""
     from block_sparse_attention_13_b200.autograd import block_sparse_attention_train
-    wl = SMALL["ragged135_d128"]
+    wl = SMALL[name]
     q, k, v = synth.make_qkv(wl)
     g = synth.make_dout(wl)
     rp, ci, out, lse, dq, dk, dv, st_f, st_b = gpu_fwd_bwd(wl, q, k, v, g)
@@ -205,7 +207,8 @@ def test_autograd_op_matches_the_c_abi_calls():
     qt, kt, vt = (dev(x).requires_grad_(True) for x in (q, k, v))
     o = block_sparse_attention_train(qt, kt, vt, (wl.T, wl.H, wl.W), topk=wl.topk, mode=wl.mode,
                                      cdf_p=wl.cdf_p, cdf_cap_frac=wl.cdf_cap_frac,
-                                     t_cond=wl.t_cond)
+                                     t_cond=wl.t_cond, chunk=tuple(wl.qchunk),
+                                     kchunk=tuple(wl.kchunk))
     o.backward(dev(g))
     for a, b in ((o.detach(), out), (qt.grad, dq), (kt.grad, dk), (vt.grad, dv)):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
