@@ -24,6 +24,13 @@
 // Q, K, V, dO and the gradients stay in [T,H,W] token order; the same 5-D TMA
 // box as the forward lands one chunk in shared memory in chunk-local order.
 //
+// 64-token query chunks ("LongCat-Video Technical Report", block-size
+// robustness): as in the forward, the rows and key chunks of steps 1-4 are
+// (4,4,8) boxes (two query chunks; the union of their key boxes), and every
+// CSR and CSC entry carries a 4-bit quadrant pattern; the exponential warps set
+// the weights of the quadrants a box's chunks did not select to zero, which
+// leaves exactly the gradients of each chunk's own attention.
+//
 // Every mbarrier wait is bounded; on expiry the CTA records a timeout in the
 // status word, drains its in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -185,7 +192,8 @@ struct BwdCfg {
     static constexpr int kTmaWarp = 8;
     static constexpr int kMmaWarp = 9;
     static constexpr uint32_t kTmemCols = 512;
-    // six tiles, then (dK/dV kernel) three 1 KB per-query-chunk aux records, control, list
+    // six tiles, then (dK/dV kernel) three 1 KB per-query-chunk aux records, control, the
+    // chunk list and (64-token query chunks) the quadrant pattern of each list entry
     static constexpr int kAux = 6 * kTileBytes;
     static constexpr int kCtl = kAux + 3 * 1024;
     static constexpr int kList = kCtl + 512;
