@@ -38,7 +38,7 @@ MODES = {"topk": BSA_SEL_TOPK, "cdf": BSA_SEL_CDF, "topk_cdf": BSA_SEL_TOPK_CDF}
 EXPORTED = ("bsa_version", "bsa_status_string", "bsa_workspace_size", "bsa_plan_sizes",
             "bsa_plan", "bsa_plan_noalloc", "bsa_forward", "bsa_forward_ex", "bsa_read_status",
             "bsa_rearrange", "bsa_pool", "bsa_scores", "bsa_selftest_exp2",
-            "bsa_selftest_timeout", "bsa_backward_workspace_size", "bsa_backward",
+            "bsa_selftest_timeout", "bsa_backward_workspace_size", "bsa_backward", "bsa_backward_ex",
             "bsa_select_pooled", "bsa_csr_slice_workspace_size", "bsa_csr_slice",
             "bsa_lse_merge", "bsa_grad_accumulate", "bsa_grad_finalize", "bsa_shape_info",
             "bsa_forward_host_workspace_size", "bsa_forward_host", "bsa_forward_partial",
@@ -138,6 +138,8 @@ def lib():
             "bsa_grad_finalize": (i32, [P, vp, vp, vp]),
             "bsa_backward": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, vp,
                                    vp]),
+            "bsa_backward_ex": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, sz, vp, vp, vp,
+                                      u64, i32, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -321,18 +323,31 @@ def bsa_backward_workspace_size(p: bsa_params) -> int:
 
 def bsa_backward(p, q, k, v, out, lse, dout, row_ptr, col_idx, workspace, dq, dk, dv,
                  stream=None):
+    _backward("bsa_backward", p, q, k, v, out, lse, dout, row_ptr, col_idx, workspace, dq, dk,
+              dv, stream)
+
+
+def bsa_backward_ex(p, q, k, v, out, lse, dout, row_ptr, col_idx, workspace, dq, dk, dv,
+                    timeout_ns=0, debug_flags=0, stream=None):
+    """bsa_backward with an explicit device wait limit and debug flags."""
+    _backward("bsa_backward_ex", p, q, k, v, out, lse, dout, row_ptr, col_idx, workspace, dq, dk,
+              dv, stream, (int(timeout_ns), int(debug_flags)))
+
+
+def _backward(name, p, q, k, v, out, lse, dout, row_ptr, col_idx, workspace, dq, dk, dv, stream,
+              extra=()):
     bf, f32, i32 = _dtypes()
     s = bsa_shape_info(p)
     x = s.BH * s.N * s.d
-    _tensors("bsa_backward", ("q", q, bf, x), ("k", k, bf, x), ("v", v, bf, x), ("out", out, bf, x),
+    _tensors(name, ("q", q, bf, x), ("k", k, bf, x), ("v", v, bf, x), ("out", out, bf, x),
              ("lse", lse, f32, s.BH * s.N), ("dout", dout, bf, x),
              ("row_ptr", row_ptr, i32, s.rows + 1), ("col_idx", col_idx, i32, 0),
              ("workspace", workspace, None, 0), ("dq", dq, bf, x), ("dk", dk, bf, x),
              ("dv", dv, bf, x))
-    _check(lib().bsa_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
-                              _ptr(dout), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
-                              _ptr(workspace), workspace.numel() * workspace.element_size(),
-                              _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)), "bsa_backward")
+    _check(getattr(lib(), name)(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                _ptr(dout), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _ptr(dq), _ptr(dk), _ptr(dv), *extra, _stream(stream)), name)
 
 
 def bsa_forward_host_workspace_size(p: bsa_params, group: int, slots: int) -> int:

@@ -249,7 +249,7 @@ using namespace bsa;
 
 extern "C" {
 
-int bsa_version(void) { return 301; }
+int bsa_version(void) { return 302; }
 
 const char* bsa_status_string(int s) {
     switch (s) {
@@ -403,10 +403,11 @@ size_t bsa_backward_workspace_size(const bsa_params* p) {
     return bwd_layout(g, *p).total;
 }
 
-int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* v,
-                 const void* out, const float* lse, const void* dout, const int32_t* row_ptr,
-                 const int32_t* col_idx, int64_t col_capacity, void* workspace, size_t ws_bytes,
-                 void* dq, void* dk, void* dv, void* stream) {
+int bsa_backward_ex(const bsa_params* p, const void* q, const void* k, const void* v,
+                    const void* out, const float* lse, const void* dout, const int32_t* row_ptr,
+                    const int32_t* col_idx, int64_t col_capacity, void* workspace, size_t ws_bytes,
+                    void* dq, void* dk, void* dv, uint64_t timeout_ns, int debug_flags,
+                    void* stream) {
     TraceRange trace("bsa_backward");
     Dims g;
     int rc = make_dims(p, &g);
@@ -421,8 +422,17 @@ int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* 
     if (ws_bytes < bwd_layout(g, *p).total) return BSA_ERR_WORKSPACE_TOO_SMALL;
     if ((rc = device_ok()) != BSA_OK) return rc;
     return cuda_status(launch_backward(g, *p, q, k, v, out, lse, dout, row_ptr, col_idx, col_capacity,
-                                       workspace, dq, dk, dv, kDefaultTimeoutNs,
+                                       workspace, dq, dk, dv,
+                                       timeout_ns ? timeout_ns : kDefaultTimeoutNs, debug_flags,
                                        static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* v,
+                 const void* out, const float* lse, const void* dout, const int32_t* row_ptr,
+                 const int32_t* col_idx, int64_t col_capacity, void* workspace, size_t ws_bytes,
+                 void* dq, void* dk, void* dv, void* stream) {
+    return bsa_backward_ex(p, q, k, v, out, lse, dout, row_ptr, col_idx, col_capacity, workspace,
+                           ws_bytes, dq, dk, dv, 0, 0, stream);
 }
 
 int bsa_select_pooled(const bsa_params* p, const float* qpool, const float* kpool, int32_t kshard,

@@ -240,6 +240,10 @@ __global__ void __launch_bounds__(320, 1)
     const int nmax = n0 > n1 ? n0 : n1;
     volatile int* abort_flag = &ctl->abort_flag;
     const uint64_t tmo = a.timeout_ns;
+    // what this thread put in flight (K and V copies per tile; any product), for
+    // the drain after an abort
+    int nk[2] = {0, 0}, nvv[2] = {0, 0};
+    bool issued = false;
 
     if (warp == C::kTmaWarp) {
         // ------------------------------------------------------------ TMA producer
@@ -261,7 +265,6 @@ __global__ void __launch_bounds__(320, 1)
             // (its issue order), so the loads go out in that order too: V0(j),
             // K0(j+1), V1(j), K1(j+1). Each wait depends only on loads issued by
             // earlier steps of this loop.
-            int nk[2] = {0, 0}, nvv[2] = {0, 0};
             auto load_k = [&](int t, int j) -> bool {
                 if (j >= n[t]) return true;
                 TileBars& b = ctl->tb[t];
@@ -297,15 +300,6 @@ __global__ void __launch_bounds__(320, 1)
             bool aborted = !(load_k(0, 0) && load_k(1, 0));
             for (int j = 0; j < nmax && !aborted; ++j)
                 aborted = !(load_v(0, j) && load_k(0, j + 1) && load_v(1, j) && load_k(1, j + 1));
-            if (aborted || *abort_flag) {
-                // let the copies already issued land before shared memory is released
-                for (int t = 0; t < 2; ++t) {
-                    if (n[t] == 0) continue;
-                    drain_wait(&ctl->tb[t].q_full, 0, tmo);
-                    if (nk[t] > 0) drain_wait(&ctl->tb[t].k_full, (nk[t] - 1) & 1, tmo);
-                    if (nvv[t] > 0) drain_wait(&ctl->tb[t].v_full, (nvv[t] - 1) & 1, tmo);
-                }
-            }
         }
         __syncwarp();
     } else if (warp == C::kMmaWarp) {
@@ -314,7 +308,7 @@ __global__ void __launch_bounds__(320, 1)
             constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);  // Q, K both K-major
             constexpr uint32_t kIdO = idesc_bf16_f32(128, D, 0, 1);    // P from TMEM, V MN-major
             const int n[2] = {n0, n1};
-            bool aborted = false, issued = false;
+            bool aborted = false;
             for (int t = 0; t < 2 && !aborted; ++t)
                 if (n[t] > 0 && !mbar_wait(&ctl->tb[t].q_full, 0, abort_flag, a.status, tmo, site(2, 0, t, 0)))
                     aborted = true;
@@ -370,10 +364,6 @@ __global__ void __launch_bounds__(320, 1)
                         tc_commit(&ctl->tb[t].o_full);
                     }
                 }
-            }
-            if (aborted && issued) {
-                tc_commit(&ctl->aux);
-                drain_wait(&ctl->aux, 0, tmo);
             }
         }
         __syncwarp();
@@ -589,7 +579,24 @@ __global__ void __launch_bounds__(320, 1)
 
     tc_fence_before();
     __syncthreads();
+    // After an abort (the flag no longer changes here, whichever role gave up and
+    // whenever), the copies and products still in flight land before the CTA's
+    // shared memory and TMEM are released.
+    if (*abort_flag) {
+        if (warp == C::kTmaWarp && lane == 0) {
+            for (int t = 0; t < 2; ++t) {
+                if ((t ? n1 : n0) == 0) continue;
+                drain_wait(&ctl->tb[t].q_full, 0, tmo);
+                if (nk[t] > 0) drain_wait(&ctl->tb[t].k_full, (nk[t] - 1) & 1, tmo);
+                if (nvv[t] > 0) drain_wait(&ctl->tb[t].v_full, (nvv[t] - 1) & 1, tmo);
+            }
+        } else if (warp == C::kMmaWarp && issued) {
+            tc_commit(&ctl->aux);
+            drain_wait(&ctl->aux, 0, tmo);
+        }
+    }
     if (warp == C::kMmaWarp) {
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }

@@ -225,6 +225,8 @@ struct BwdArgs {
     float scale;
     float scale_log2;
     uint64_t timeout_ns;
+    int debug_flags;          // bit 0: the dQ kernel, bit 1: the dK/dV kernel withholds
+                              // its first S-ready signal (tests of the bounded waits)
 };
 
 // Rows of a 128 x D fp32 TMEM block (this thread's lane, columns from t_row)
@@ -426,6 +428,10 @@ __global__ void __launch_bounds__(320, 1)
     const int r_local = static_cast<int>(row % a.Nq);
     int q_t, q_h, q_w;
     chunk_origin(a.q_skip + r_local, a.NH, a.NW, q_t, q_h, q_w);
+    // what this thread put in flight (K and V copies per slot; any product), for
+    // the drain after an abort
+    int nk[3] = {0, 0, 0}, nv[2] = {0, 0};
+    bool issued = false;
 
     if (warp == C::kTmaWarp) {
         // ------------------------------------------------------------ TMA producers
@@ -439,7 +445,6 @@ __global__ void __launch_bounds__(320, 1)
                 tma_load_5d(&tm_do, smem_u32(sdO) + c * C::kHalfBytes, &ctl->qd_full, c * 64, q_w,
                             q_h, q_t, bh);
             }
-            int nk[3] = {0, 0, 0};
             bool ok = true;
             for (int j = 0; j < n && ok; ++j) {
                 const int s = j % 3;
@@ -457,15 +462,9 @@ __global__ void __launch_bounds__(320, 1)
                                 kw, kh, kt, bh);
                 ++nk[s];
             }
-            if (!ok || *abort_flag) {
-                drain_wait(&ctl->qd_full, 0, tmo);
-                for (int s = 0; s < 3; ++s)
-                    if (nk[s] > 0) drain_wait(&ctl->k_full[s], (nk[s] - 1) & 1, tmo);
-            }
         } else if (lane == 1 && n > 0) {
             // the V slots: V(0) in its own tile, V(1) in Q's once Q is in TMEM, then
             // V(j) once dP(j-2) has read V(j-2)
-            int nv[2] = {0, 0};
             bool ok = true;
             for (int j = 0; j < n && ok; ++j) {
                 const int s = j & 1;
@@ -487,9 +486,6 @@ __global__ void __launch_bounds__(320, 1)
                                 vw, vh, vt, bh);
                 ++nv[s];
             }
-            if (!ok || *abort_flag)
-                for (int s = 0; s < 2; ++s)
-                    if (nv[s] > 0) drain_wait(&ctl->v_full[s], (nv[s] - 1) & 1, tmo);
         }
         __syncwarp();
     } else if (warp == C::kMmaWarp) {
@@ -497,7 +493,6 @@ __global__ void __launch_bounds__(320, 1)
         if (lane == 0 && n > 0) {
             constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);  // A from TMEM, B K-major
             constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, 0, 1);    // dS from TMEM, K MN-major
-            bool issued = false;
             bool ok = mbar_wait(&ctl->qt_full, 0, abort_flag, a.status, tmo, site(2, 0, 0, 0));
             if (ok) tc_fence_after();
             // G = A B^T over the D channels: A (Q or dO) in TMEM at acol, B in shared memory
@@ -517,7 +512,7 @@ __global__ void __launch_bounds__(320, 1)
                     return false;
                 issue_tk(kS, kQt, smem_u32(sK(s)));
                 issued = true;
-                tc_commit(&ctl->s_full);
+                if (!((a.debug_flags & 1) && j == 0)) tc_commit(&ctl->s_full);
                 return true;
             };
             // dP(j) = dO V(j)^T. Past the first step the dS warps have seen V(j) land before
@@ -562,12 +557,7 @@ __global__ void __launch_bounds__(320, 1)
                 issue_dq(j);
                 if (j + 1 < n && !issue_dp(j + 1)) { ok = false; break; }
             }
-            if (ok) {
-                tc_commit(&ctl->dq_full);
-            } else if (issued) {
-                tc_commit(&ctl->aux);
-                drain_wait(&ctl->aux, 0, tmo);
-            }
+            if (ok) tc_commit(&ctl->dq_full);
         }
         __syncwarp();
     } else {
@@ -697,7 +687,23 @@ __global__ void __launch_bounds__(320, 1)
 
     tc_fence_before();
     __syncthreads();
+    // After an abort (the flag no longer changes here, whichever role gave up and
+    // whenever), the copies and products still in flight land before the CTA's
+    // shared memory and TMEM are released.
+    if (*abort_flag) {
+        if (warp == C::kTmaWarp) {
+            if (lane == 0 && n > 0) drain_wait(&ctl->qd_full, 0, tmo);
+            for (int s = 0; s < 3; ++s)
+                if (nk[s] > 0) drain_wait(&ctl->k_full[s], (nk[s] - 1) & 1, tmo);
+            for (int s = 0; s < 2; ++s)
+                if (nv[s] > 0) drain_wait(&ctl->v_full[s], (nv[s] - 1) & 1, tmo);
+        } else if (warp == C::kMmaWarp && issued) {
+            tc_commit(&ctl->aux);
+            drain_wait(&ctl->aux, 0, tmo);
+        }
+    }
     if (warp == C::kMmaWarp) {
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
@@ -831,6 +837,10 @@ __global__ void __launch_bounds__(320, 1)
     const uint64_t tmo = a.timeout_ns;
     int k_t, k_h, k_w;
     chunk_origin(kc, a.NH, a.NW, k_t, k_h, k_w);
+    // what this thread put in flight (Q and dO copies per slot; any product), for
+    // the drain after an abort
+    int nq[2] = {0, 0}, nd[2] = {0, 0};
+    bool issued = false;
 
     if (warp == C::kTmaWarp) {
         // ------------------------------------------------------------ TMA producers
@@ -845,7 +855,6 @@ __global__ void __launch_bounds__(320, 1)
                 tma_load_5d(&tm_v, smem_u32(sV) + c * C::kHalfBytes, &ctl->kv_full, c * 64, k_w, k_h,
                             k_t, bh);
             }
-            int nq[2] = {0, 0};
             bool ok = true;
             for (int i = 0; i < n && ok; ++i) {
                 const int s = i & 1;
@@ -866,14 +875,8 @@ __global__ void __launch_bounds__(320, 1)
                           1024, &ctl->q_full[s]);
                 ++nq[s];
             }
-            if (!ok || *abort_flag) {
-                drain_wait(&ctl->kv_full, 0, tmo);
-                for (int s = 0; s < 2; ++s)
-                    if (nq[s] > 0) drain_wait(&ctl->q_full[s], (nq[s] - 1) & 1, tmo);
-            }
         } else if (lane == 1 && n > 0) {
             // the dO ring: dO(i+2) once dV(i) has read dO(i)
-            int nd[2] = {0, 0};
             bool ok = true;
             for (int i = 0; i < n && ok; ++i) {
                 const int s = i & 1;
@@ -891,9 +894,6 @@ __global__ void __launch_bounds__(320, 1)
                                 qw, qh, qt, bh);
                 ++nd[s];
             }
-            if (!ok || *abort_flag)
-                for (int s = 0; s < 2; ++s)
-                    if (nd[s] > 0) drain_wait(&ctl->do_full[s], (nd[s] - 1) & 1, tmo);
         }
         __syncwarp();
     } else if (warp == C::kMmaWarp) {
@@ -901,7 +901,6 @@ __global__ void __launch_bounds__(320, 1)
         if (lane == 0 && n > 0) {
             constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);  // both operands K-major
             constexpr uint32_t kIdG = idesc_bf16_f32(128, D, 0, 1);    // A from TMEM, B MN-major
-            bool issued = false;
             bool ok = mbar_wait(&ctl->kv_full, 0, abort_flag, a.status, tmo, site(2, 0, 0, 0));
             if (ok) tc_fence_after();
             auto issue_ss = [&](uint32_t dcol, uint32_t sa, uint32_t sb) {
@@ -930,7 +929,7 @@ __global__ void __launch_bounds__(320, 1)
                 tc_fence_after();
                 issue_ss(0u, smem_u32(sK), smem_u32(sQ(s)));
                 issued = true;
-                tc_commit(&ctl->s_full);
+                if (!((a.debug_flags & 2) && i == 0)) tc_commit(&ctl->s_full);
                 return true;
             };
             // dP^T(i) = V dO(i)^T. Past the first step the warps have seen dO(i) land before
@@ -964,12 +963,7 @@ __global__ void __launch_bounds__(320, 1)
                 tc_commit(&ctl->q_empty[s]);
                 if (i + 1 < n && !issue_dpt(i + 1)) { ok = false; break; }
             }
-            if (ok) {
-                tc_commit(&ctl->dkv_full);
-            } else if (issued) {
-                tc_commit(&ctl->aux);
-                drain_wait(&ctl->aux, 0, tmo);
-            }
+            if (ok) tc_commit(&ctl->dkv_full);
         }
         __syncwarp();
     } else {
@@ -1103,7 +1097,22 @@ __global__ void __launch_bounds__(320, 1)
 
     tc_fence_before();
     __syncthreads();
+    // After an abort (final here), the copies and products still in flight land
+    // before the CTA's shared memory and TMEM are released.
+    if (*abort_flag) {
+        if (warp == C::kTmaWarp) {
+            if (lane == 0 && n > 0) drain_wait(&ctl->kv_full, 0, tmo);
+            for (int s = 0; s < 2; ++s) {
+                if (nq[s] > 0) drain_wait(&ctl->q_full[s], (nq[s] - 1) & 1, tmo);
+                if (nd[s] > 0) drain_wait(&ctl->do_full[s], (nd[s] - 1) & 1, tmo);
+            }
+        } else if (warp == C::kMmaWarp && issued) {
+            tc_commit(&ctl->aux);
+            drain_wait(&ctl->aux, 0, tmo);
+        }
+    }
     if (warp == C::kMmaWarp) {
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
@@ -1227,7 +1236,7 @@ cudaError_t launch_backward(const Dims& g0, const bsa_params& p, const void* q, 
                             const void* v, const void* out, const float* lse, const void* dout,
                             const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
                             void* workspace, void* dq, void* dk, void* dv, uint64_t timeout_ns,
-                            cudaStream_t st) {
+                            int debug_flags, cudaStream_t st) {
     const BwdLayout L = bwd_layout(g0, p);
     // 64-token query chunks: the attention kernels work on (4,4,8) boxes, over the
     // box CSR with a quadrant pattern per entry (the forward's own construction)
@@ -1323,6 +1332,7 @@ cudaError_t launch_backward(const Dims& g0, const bsa_params& p, const void* q, 
     args.scale = g.scale;
     args.scale_log2 = g.scale * kLog2e;
     args.timeout_ns = timeout_ns;
+    args.debug_flags = debug_flags;
     BwdArgs dq_args = args, dkv_args = args;
     dq_args.units = g.rows;
     dkv_args.units = cols;

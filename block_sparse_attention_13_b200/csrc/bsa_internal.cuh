@@ -193,7 +193,7 @@ cudaError_t launch_backward(const Dims& g, const bsa_params& p, const void* q, c
                             const void* v, const void* out, const float* lse, const void* dout,
                             const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
                             void* workspace, void* dq, void* dk, void* dv, uint64_t timeout_ns,
-                            cudaStream_t st);
+                            int debug_flags, cudaStream_t st);
 // Context parallelism: CSR entries with lo <= column < hi, re-indexed to
 // column - lo (order kept); and the log-sum-exp merge of a partial attention
 // result into an accumulator.

@@ -112,7 +112,8 @@ typedef struct {
 
 /* Library version: major*10000 + minor*100 + patch (0.2.0: bsa_shape_info and
  * bsa_forward_host added; 0.3.0: 64-token chunks, bsa_forward_partial and
- * bsa_lse_merge_f32; 0.3.1: bsa_backward for 64-token chunks). */
+ * bsa_lse_merge_f32; 0.3.1: bsa_backward for 64-token chunks; 0.3.2:
+ * bsa_backward_ex). */
 BSA_API int bsa_version(void);
 
 /* Text for a status code (static storage; never NULL). */
@@ -244,6 +245,20 @@ BSA_API int bsa_backward(const bsa_params* p, const void* q, const void* k, cons
                          const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
                          void* workspace, size_t ws_bytes, void* dq, void* dk, void* dv,
                          void* stream);
+
+/* bsa_backward with an explicit limit for every device-side wait (timeout_ns;
+ * 0 = the default of 2 s) and debug flags (bit 0: the dQ kernel's MMA thread,
+ * bit 1: the dK/dV kernel's, withholds its first "scores ready" signal, so the
+ * exponential warps' bounded wait expires, every role stops, the copies and
+ * products in flight are waited for and TMEM is freed, and the call reports
+ * DEVICE_TIMEOUT through bsa_read_status(workspace) without faulting or
+ * hanging; the gradients are then not meaningful; used by the
+ * failure-detection tests). Same contract as bsa_backward otherwise. */
+BSA_API int bsa_backward_ex(const bsa_params* p, const void* q, const void* k, const void* v,
+                            const void* out, const float* lse, const void* dout,
+                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
+                            void* workspace, size_t ws_bytes, void* dq, void* dk, void* dv,
+                            uint64_t timeout_ns, int debug_flags, void* stream);
 
 /*
  * Context parallelism ([P1] ring block sparse attention: the sequence split

@@ -42,7 +42,7 @@ def test_library_exports_nothing_else():
 
 
 def test_version_and_strings(L):
-    assert bsa.bsa_version() == 301
+    assert bsa.bsa_version() == 302
     for code in range(0, 10):
         s = bsa.status_string(code)
         assert s and s != "unknown status"

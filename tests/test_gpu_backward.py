@@ -95,6 +95,46 @@ def test_backward_small_cases(name):
     check_bwd(SMALL[name])
 
 
+@pytest.mark.parametrize("name,flags", [("tiny", 1), ("tiny", 2), ("q64_k64", 3)])
+def test_backward_kernel_abort_paths_report_timeout(name, flags):
+    """The backward kernels' own bounded waits: debug bit 0 makes the dQ
+    kernel's MMA thread, bit 1 the dK/dV kernel's, withhold its first
+    S-ready signal, so that kernel's exponential warps (and then every role)
+    wait until the 20 ms limit, record the timeout, and the CTA waits for its
+    copies and products in flight before freeing TMEM and returning. The status
+    must say DEVICE_TIMEOUT, and the next call on the same buffers must give
+    the right gradients."""
+    wl = SMALL[name]
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    p = bsa.params_for(wl)
+    qd, kd, vd, gd = dev(q), dev(k), dev(v), dev(g)
+    pl = bsa.allocate(p)
+    bsa.bsa_plan(p, qd, kd, pl.workspace, pl.row_ptr, pl.col_idx)
+    out = torch.empty_like(qd)
+    lse = torch.empty((wl.B, wl.heads, wl.N), dtype=torch.float32, device="cuda")
+    bsa.bsa_forward(p, qd, kd, vd, pl.row_ptr, pl.col_idx, pl.workspace, out, lse)
+    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_OK
+    ws = bsa.backward_workspace(p)
+    dq, dk, dv = (torch.full_like(qd, float("nan")) for _ in range(3))
+    args = (p, qd, kd, vd, out, lse, gd, pl.row_ptr, pl.col_idx, ws, dq, dk, dv)
+    bsa.bsa_backward_ex(*args, timeout_ns=20_000_000, debug_flags=flags)
+    assert bsa.bsa_read_status(ws) == bsa.BSA_ERR_DEVICE_TIMEOUT
+    bsa.bsa_backward(*args)
+    assert bsa.bsa_read_status(ws) == bsa.BSA_OK
+    rp = pl.row_ptr.cpu().numpy()
+    ci = pl.col_idx[: int(rp[-1])].cpu().numpy()
+    rows = np.arange(wl.rows)
+    shapes = dict(kchunk=tuple(wl.kchunk), qchunk=tuple(wl.qchunk)) \
+        if tuple(wl.qchunk) == (4, 4, 4) else {}
+    refs = oracle.attend_bwd(q, k, v, g, wl.T, wl.H, wl.W, wl.softmax_scale, rp, ci, rows,
+                             **shapes)
+    gots = (gather_rows(host_f32(dq), wl, rows), host_f32(dk), host_f32(dv))
+    for nm, got, ref in zip(("dq", "dk", "dv"), gots, refs):
+        mx, mean = rel_errors(got, ref)
+        assert mx <= BWD_MAX_REL and mean <= BWD_MEAN_REL, (nm, mx, mean)
+
+
 def test_backward_64_token_chunks_with_an_empty_chunk_and_unselected_halves():
     """64-token query chunks with a caller CSR: one query chunk selects nothing
     (its queries have no output: dQ exactly 0) and some 64-token key chunks no
