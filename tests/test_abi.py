@@ -309,10 +309,14 @@ def test_backward_workspace_size_layout(L):
     assert bsa.lib().bsa_backward_workspace_size(ctypes.byref(P(T=0))) == 0
 
 
-def test_backward_host_checks_before_any_cuda_call(L):
+@pytest.mark.parametrize("entry", ["bsa_backward", "bsa_backward_ex"])
+def test_backward_host_checks_before_any_cuda_call(L, entry):
     p = P()
     ws = bsa.bsa_backward_workspace_size(p)
-    f = L.bsa_backward
+    if entry == "bsa_backward":
+        f = L.bsa_backward
+    else:  # the same checks, with a wait limit and debug flags before the stream
+        f = lambda *a: L.bsa_backward_ex(*a[:-1], 0, 1, a[-1])
     pp = ctypes.byref(p)
     x = vp(FAKE)
     # q, k, v, out, lse, dout, row_ptr, col_idx, cap, ws, ws_bytes, dq, dk, dv, stream
@@ -341,6 +345,10 @@ def test_no_cpu_fallback_without_a_gpu(L):
     rc = L.bsa_plan(ctypes.byref(p), vp(FAKE), vp(FAKE), vp(FAKE), ws, vp(FAKE), vp(FAKE), 16,
                     None)
     assert rc == bsa.BSA_ERR_CUDA
+    x = vp(FAKE)
+    bws = bsa.bsa_backward_workspace_size(p)
+    assert L.bsa_backward_ex(ctypes.byref(p), x, x, x, x, x, x, x, x, 16, x, bws, x, x, x,
+                             20_000_000, 3, None) == bsa.BSA_ERR_CUDA
     with pytest.raises(bsa.BsaError):
         bsa.bsa_plan_sizes(P(T=0))
 
