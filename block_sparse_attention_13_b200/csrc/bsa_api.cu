@@ -558,7 +558,8 @@ int bsa_read_status(void* workspace, void* stream) {
     if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return BSA_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return BSA_ERR_CUDA;
-    if (cudaMemsetAsync(workspace, 0, sizeof(word), st) != cudaSuccess) return BSA_ERR_CUDA;
+    // the status word and the record of the first expired wait (words 0 to 5)
+    if (cudaMemsetAsync(workspace, 0, 6 * sizeof(uint32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return BSA_ERR_CUDA;
     if (word & kStatusTimeout) return BSA_ERR_DEVICE_TIMEOUT;
     if (word & kStatusBadIndex) return BSA_ERR_DEVICE_BAD_INDEX;

@@ -409,15 +409,22 @@ BSA_API int bsa_forward_host(const bsa_params* p, const void* q, const void* k, 
 /* bsa_forward with an explicit limit for every device-side wait (timeout_ns;
  * 0 = the default of 2 s) and debug flags (bit 0: the MMA warp withholds its
  * first "scores ready" signal, so the softmax warps' bounded wait expires and
- * the kernel reports DEVICE_TIMEOUT without faulting or hanging; used by the
- * failure-detection tests). Same contract as bsa_forward otherwise. */
+ * the kernel reports DEVICE_TIMEOUT without faulting or hanging; bit 1: every
+ * CTA adds 1 to status word 8 as it returns; used by the failure-detection
+ * tests). Same contract as bsa_forward otherwise. */
 BSA_API int bsa_forward_ex(const bsa_params* p, const void* q, const void* k, const void* v,
                    const int32_t* row_ptr, const int32_t* col_idx, int64_t col_capacity,
                    void* workspace, size_t ws_bytes, void* out, float* lse, uint64_t timeout_ns,
                    int debug_flags, void* stream);
 
 /* Synchronise `stream`, return the first device-side error recorded in the
- * workspace status word since the last call (BSA_OK if none) and clear it. */
+ * workspace status word since the last call (BSA_OK if none) and clear it.
+ * The status block (the first 256 bytes of every workspace) holds uint32
+ * words: [0] error bits; [1] number of bounded waits that expired; [2] 1 once
+ * [3..5] hold the first expired wait: its site code ((role*100 + barrier*10 +
+ * tile)*10000 + step, role 1 = copy producer, 2 = MMA issuer, 3 = exponential
+ * warps), the CTA index and the phase parity; [8] CTAs that finished, counted
+ * only by bsa_forward_ex with debug bit 1. This call clears words 0 to 5. */
 BSA_API int bsa_read_status(void* workspace, void* stream);
 
 /*

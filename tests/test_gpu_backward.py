@@ -12,7 +12,7 @@ import torch
 import oracle
 import synth
 from parity import rows_of
-from test_gpu_parity import SMALL, W, dev, gather_rows, host_f32
+from test_gpu_parity import SMALL, W, check_timeout_record, dev, gather_rows, host_f32
 
 pytestmark = pytest.mark.gpu
 
@@ -119,7 +119,7 @@ def test_backward_kernel_abort_paths_report_timeout(name, flags):
     dq, dk, dv = (torch.full_like(qd, float("nan")) for _ in range(3))
     args = (p, qd, kd, vd, out, lse, gd, pl.row_ptr, pl.col_idx, ws, dq, dk, dv)
     bsa.bsa_backward_ex(*args, timeout_ns=20_000_000, debug_flags=flags)
-    assert bsa.bsa_read_status(ws) == bsa.BSA_ERR_DEVICE_TIMEOUT
+    check_timeout_record(ws)
     bsa.bsa_backward(*args)
     assert bsa.bsa_read_status(ws) == bsa.BSA_OK
     rp = pl.row_ptr.cpu().numpy()

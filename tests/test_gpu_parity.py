@@ -364,12 +364,28 @@ def test_bounded_wait_selftest_reports_timeout():
     check_case(SMALL["tiny"])  # the context is still usable
 
 
+def status_words(ws):
+    """The first 16 uint32 words of a workspace's status block."""
+    return ws[:64].cpu().numpy().view(np.uint32).copy()
+
+
+def check_timeout_record(ws):
+    """The record of the first expired wait, then its clearing by bsa_read_status."""
+    w = status_words(ws)
+    assert w[1] >= 1 and w[2] == 1, w[:6]          # expired waits; a site was recorded
+    assert w[3] // 1_000_000 in (1, 2, 3), w[3]     # role: producer, MMA issuer or warps
+    assert bsa.bsa_read_status(ws) == bsa.BSA_ERR_DEVICE_TIMEOUT
+    assert not status_words(ws)[:6].any()
+    return w
+
+
 def test_forward_kernel_abort_path_reports_timeout():
-    """The forward kernel's own bounded waits: with debug flag 0 the MMA warp
+    """The forward kernel's own bounded waits: with debug bit 0 the MMA warp
     withholds the first S-ready signal of tile 0, so that tile's softmax warps
     (and then every role) wait until the 20 ms limit, record the timeout, drain
-    their copies and products, free TMEM and return. The status must say
-    DEVICE_TIMEOUT, and the next calls must work."""
+    their copies and products, free TMEM and return; with bit 1 every CTA
+    counts itself on the way out. The status must say DEVICE_TIMEOUT, every CTA
+    must have returned, and the next calls must work."""
     wl = SMALL["tiny"]
     q, k, v = synth.make_qkv(wl)
     p = bsa.params_for(wl)
@@ -379,8 +395,10 @@ def test_forward_kernel_abort_path_reports_timeout():
     assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_OK
     out = torch.zeros_like(qd)
     bsa.bsa_forward_ex(p, qd, kd, vd, pl.row_ptr, pl.col_idx, pl.workspace, out,
-                       timeout_ns=20_000_000, debug_flags=1)
-    assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_ERR_DEVICE_TIMEOUT
+                       timeout_ns=20_000_000, debug_flags=3)
+    w = check_timeout_record(pl.workspace)
+    ctas = (wl.rows + 1) // 2                       # two query chunks per CTA
+    assert w[8] == ctas and w[4] < ctas, (w[8], w[4])
     # the same buffers give the right result on the next call, and so does a fresh case
     bsa.bsa_forward(p, qd, kd, vd, pl.row_ptr, pl.col_idx, pl.workspace, out)
     assert bsa.bsa_read_status(pl.workspace) == bsa.BSA_OK
