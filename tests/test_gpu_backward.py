@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from parity import rows_of
+from parity import ATT_MAX_ABS, ATT_MEAN_ABS, compare_attention, rows_of
 from test_gpu_parity import SMALL, W, check_timeout_record, dev, gather_rows, host_f32
 
 pytestmark = pytest.mark.gpu
@@ -133,6 +133,65 @@ def test_backward_kernel_abort_paths_report_timeout(name, flags):
     for nm, got, ref in zip(("dq", "dk", "dv"), gots, refs):
         mx, mean = rel_errors(got, ref)
         assert mx <= BWD_MAX_REL and mean <= BWD_MEAN_REL, (nm, mx, mean)
+
+
+def test_64_token_chunks_with_masked_quadrants_of_huge_logits():
+    """64-token chunks whose box partner selected a key chunk they did not: the
+    kernels compute those quadrants of the (4,4,8) box tile and must keep them
+    out of every result. Key chunk 11 of head 0 has K scaled by 64 (exact in
+    bf16), so its logits reach about +-200 and exp() of them overflows fp32: a
+    masked logit that entered the row max would underflow the row's kept
+    weights to 0, and one that reached an exponential before the mask would
+    give inf * 0 = NaN. Query chunk 20 keeps 10 (the other half of 11's box)
+    while 21 keeps 11; 36 keeps neither while 37 keeps 11; 45 and 44 keep 11
+    together with the rest of their own selection. Forward O and LSE must match
+    the oracle on every row and every gradient must be finite. The gradient
+    bars: the usual ones wherever the hot chunk is not attended (every masked
+    quadrant is there); where it is, only the max bar against the tensor's own
+    largest gradient. Those rows put nearly all their weight on the hot keys,
+    so their exact dS, and hence dQ and the hot keys' dK, cancel to near zero,
+    while D = sum(dO * O) comes from the bf16 output: its 2^-9 rounding, times
+    K scaled by 64, is then most of what is left."""
+    wl = SMALL["q64_k64"]
+    q, k, v = synth.make_qkv(wl)
+    g = synth.make_dout(wl)
+    hot, partner = 11, 10                                 # key chunks sharing one (4,4,8) box
+    toks = oracle.chunk_tokens(wl.T, wl.H, wl.W, hot, (4, 4, 4))
+    kf = (k[0, 0, toks].astype(np.uint32) << 16).view(np.float32) * np.float32(64.0)
+    k = k.copy()
+    k[0, 0, toks] = (kf.view(np.uint32) >> 16).astype(np.uint16)  # exact: a power of two
+    rp, ci, _ = oracle.plan(q, k, wl.T, wl.H, wl.W, wl.softmax_scale, wl.mode, wl.topk,
+                            kchunk=tuple(wl.kchunk), qchunk=tuple(wl.qchunk))
+    lists = [set(ci[rp[r]:rp[r + 1]]) for r in range(wl.rows)]
+    for r, add, drop in ((20, {partner}, {hot}), (21, {hot}, set()), (36, set(), {hot, partner}),
+                         (37, {hot}, set()), (44, {hot}, set()), (45, {hot}, set())):
+        lists[r] = (lists[r] - drop) | add
+    rp2 = np.concatenate([[0], np.cumsum([len(x) for x in lists])]).astype(np.int32)
+    ci2 = np.array([c for x in lists for c in sorted(x)], dtype=np.int32)
+    rows = np.arange(wl.rows)
+    shapes = dict(kchunk=tuple(wl.kchunk), qchunk=tuple(wl.qchunk))
+    _, _, out, lse, dq, dk, dv, st_f, st_b = gpu_fwd_bwd(wl, q, k, v, g, csr=(rp2, ci2))
+    assert st_f == bsa.BSA_OK and st_b == bsa.BSA_OK, (st_f, st_b)
+    o_out, o_lse = oracle.attend(q, k, v, wl.T, wl.H, wl.W, wl.softmax_scale, rp2, ci2, rows,
+                                 **shapes)
+    mx, mean = compare_attention(gather_rows(host_f32(out), wl, rows), o_out)
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+    g_lse = gather_rows(lse.cpu().numpy()[..., None], wl, rows)[..., 0]
+    # LSE: the forward's bar, plus fp32 accumulation of logits that are 64 times larger
+    np.testing.assert_array_less(np.abs(g_lse - o_lse), 2e-3 + 2e-5 * np.abs(o_lse))
+    assert np.abs(o_lse).max() > 50                       # the hot chunk's logits are in play
+    refs = oracle.attend_bwd(q, k, v, g, wl.T, wl.H, wl.W, wl.softmax_scale, rp2, ci2, rows,
+                             **shapes)
+    gots = (gather_rows(host_f32(dq), wl, rows), host_f32(dk), host_f32(dv))
+    hot_rows = np.array([r < wl.Nc and hot in lists[r] for r in range(wl.rows)])  # head 0
+    hot_keys = np.zeros((wl.B, wl.heads, wl.N), dtype=bool)
+    hot_keys[0, 0, toks] = True
+    for nm, got, ref, sel in zip(("dq", "dk", "dv"), gots, refs, (hot_rows, hot_keys, hot_keys)):
+        assert np.isfinite(got[~np.isnan(ref)]).all(), nm
+        mx, mean = rel_errors(got[~sel], ref[~sel])
+        assert mx <= BWD_MAX_REL and mean <= BWD_MEAN_REL, (nm, "elsewhere", mx, mean)
+        err = np.abs(got[sel] - ref[sel])
+        assert np.nanmax(err) <= BWD_MAX_REL * np.nanmax(np.abs(ref)), (nm, "hot")
 
 
 def test_backward_64_token_chunks_with_an_empty_chunk_and_unselected_halves():
