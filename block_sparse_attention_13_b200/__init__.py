@@ -442,7 +442,7 @@ def bsa_grad_finalize(p, acc, out, stream=None):
 
 
 def bsa_read_status(workspace, stream=None) -> int:
-    _tensors("bsa_read_status", ("workspace", workspace, None, 4))
+    _tensors("bsa_read_status", ("workspace", workspace, None, 256))  # the status block
     return lib().bsa_read_status(_ptr(workspace), _stream(stream))
 
 

@@ -424,7 +424,9 @@ BSA_API int bsa_forward_ex(const bsa_params* p, const void* q, const void* k, co
  * [3..5] hold the first expired wait: its site code ((role*100 + barrier*10 +
  * tile)*10000 + step, role 1 = copy producer, 2 = MMA issuer, 3 = exponential
  * warps), the CTA index and the phase parity; [8] CTAs that finished, counted
- * only by bsa_forward_ex with debug bit 1. This call clears words 0 to 5. */
+ * only by bsa_forward_ex with debug bit 1. This call clears words 0 to 5.
+ * workspace: device, the workspace (at least 256 bytes) of one of the calls
+ * above. Errors: INVALID_ARG (NULL workspace), CUDA. */
 BSA_API int bsa_read_status(void* workspace, void* stream);
 
 /*

@@ -178,6 +178,11 @@ def test_binding_checks_tensors_before_the_library_sees_them():
     assert c == INV and "dv" in m
     c, m = _raises(lambda: bsa.bsa_backward(p, q, q, q, q, lse, q[:-1], rp, ci, ws, q, q, q))
     assert c == SHAPE and "dout" in m
+    c, m = _raises(lambda: bsa.bsa_backward_ex(p, q, q, q, q, lse, q, rp, ci, ws, q[:-1], q, q,
+                                               timeout_ns=1000, debug_flags=1))
+    assert c == SHAPE and "bsa_backward_ex" in m and "dq" in m
+    c, m = _raises(lambda: bsa.bsa_backward_ex(p, q, q, q, q, lse, q, rp, ci, ws, q, q, q))
+    assert c == INV and "not a CUDA tensor" in m
 
     # the chunk-major side of the rearrangement holds Nc x 128 slots (partial chunks padded)
     pr = bsa.make_params(1, 1, 10, 13, 37, 64)
@@ -203,7 +208,7 @@ def test_binding_checks_tensors_before_the_library_sees_them():
     assert _raises(lambda: bsa.bsa_grad_accumulate(p, q, q))[0] == INV        # acc must be fp32
     acc = torch.zeros(x, dtype=f32)
     assert _raises(lambda: bsa.bsa_grad_finalize(p, acc[:-1], q))[0] == SHAPE
-    assert _raises(lambda: bsa.bsa_read_status(torch.zeros(3, dtype=torch.uint8)))[0] == SHAPE
+    assert _raises(lambda: bsa.bsa_read_status(torch.zeros(255, dtype=torch.uint8)))[0] == SHAPE
     assert _raises(lambda: bsa.bsa_selftest_timeout(torch.zeros(255, dtype=torch.uint8),
                                                     1000))[0] == SHAPE
     y = torch.zeros(8, dtype=f32)
