@@ -34,18 +34,19 @@ class _BlockSparseAttention(torch.autograd.Function):
         bsa_forward(p, q, k, v, pl.row_ptr, pl.col_idx, pl.workspace, out, lse)
         _check(pl.workspace)
         ctx.p = p
-        ctx.plan = pl
+        # only the selection is kept for the backward, not the plan's workspace
+        # (tens to hundreds of MB per call on video grids)
+        ctx.csr = (pl.row_ptr, pl.col_idx)
         ctx.save_for_backward(q, k, v, out, lse)
         return out
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, out, lse = ctx.saved_tensors
-        pl = ctx.plan
+        row_ptr, col_idx = ctx.csr
         ws = backward_workspace(ctx.p, q.device)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        bsa_backward(ctx.p, q, k, v, out, lse, dout.contiguous(), pl.row_ptr, pl.col_idx, ws, dq,
-                     dk, dv)
+        bsa_backward(ctx.p, q, k, v, out, lse, dout.contiguous(), row_ptr, col_idx, ws, dq, dk, dv)
         _check(ws)
         return dq, dk, dv, None
 

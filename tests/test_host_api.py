@@ -13,6 +13,49 @@ def test_autograd_op_rejects_a_grid_that_does_not_match_the_tokens():
         block_sparse_attention_train(q, q, q, (4, 8, 8))
 
 
+def test_autograd_op_keeps_only_the_selection_for_the_backward(monkeypatch):
+    """The op's host plumbing, with the library calls replaced by recorders: the
+    backward gets the forward's own CSR tensors, the gradients it writes come
+    back to q, k, v, and the plan's workspace is released once the forward
+    has returned (only row_ptr and col_idx stay with the graph)."""
+    import weakref
+    from block_sparse_attention_13_b200 import Plan, autograd
+    seen, held = {}, []
+
+    def allocate(p, device="cuda"):
+        pl = Plan(p, torch.zeros(4096, dtype=torch.uint8), torch.zeros(9, dtype=torch.int32),
+                  torch.zeros(16, dtype=torch.int32))
+        held.append(weakref.ref(pl.workspace))
+        seen["csr"] = (pl.row_ptr, pl.col_idx)
+        return pl
+
+    def forward(p, q, k, v, row_ptr, col_idx, ws, out, lse, stream=None):
+        out.copy_(v)
+        lse.zero_()
+
+    def backward(p, q, k, v, out, lse, dout, row_ptr, col_idx, ws, dq, dk, dv, stream=None):
+        seen["bwd_csr"] = (row_ptr, col_idx)
+        dq.fill_(1.0)
+        dk.fill_(2.0)
+        dv.copy_(dout)
+
+    monkeypatch.setattr(autograd, "allocate", allocate)
+    monkeypatch.setattr(autograd, "bsa_plan", lambda *a, **kw: None)
+    monkeypatch.setattr(autograd, "bsa_forward", forward)
+    monkeypatch.setattr(autograd, "bsa_backward", backward)
+    monkeypatch.setattr(autograd, "bsa_read_status", lambda ws, stream=None: autograd.BSA_OK)
+    monkeypatch.setattr(autograd, "backward_workspace",
+                        lambda p, device="cuda": torch.zeros(256, dtype=torch.uint8))
+    q, k, v = (torch.randn(1, 2, 4 * 8 * 16, 64).to(torch.bfloat16).requires_grad_(True)
+               for _ in range(3))
+    out = block_sparse_attention_train(q, k, v, (4, 8, 16), topk=2)
+    assert held and held[0]() is None                  # the plan's workspace is gone
+    g = torch.randn_like(out)
+    out.backward(g)
+    assert seen["bwd_csr"][0] is seen["csr"][0] and seen["bwd_csr"][1] is seen["csr"][1]
+    assert torch.all(q.grad == 1) and torch.all(k.grad == 2) and torch.equal(v.grad, g)
+
+
 def test_ring_shards_must_hold_whole_chunks():
     q = torch.zeros(1, 2, 6 * 8 * 16, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
