@@ -255,7 +255,9 @@ def ring_backward(q, k, v, out, lse, dout, row_ptr, col_idx, grid, scale=0.0, co
     ring_forward returned (the merged output and LSE over all shards); row_ptr,
     col_idx: the selection ring_forward returned with return_csr. Returns
     (dq, dk, dv) bf16 for the local queries and the local K/V shard: the rows of
-    the unsplit sequence's gradients, summed in fp32 before the final rounding.
+    the unsplit sequence's gradients. Each shard's contribution comes out of
+    bsa_backward in bf16; the contributions are summed in fp32 and the sums
+    rounded once more.
     """
     comm = comm or TorchComm()
     ops = ops or CudaOps()
