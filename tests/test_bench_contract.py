@@ -59,3 +59,38 @@ def test_gpu_arm_fails_loudly_without_a_gpu():
     r = _run(["--workload", "tiny", "--steps", "1", "--warmup", "3", "--no-cpu-baseline"])
     assert r.returncode != 0
     assert '"metric"' not in r.stdout
+
+
+def test_clock_summary_takes_the_median_and_the_active_reasons_in_the_window(tmp_path):
+    """The clock record of the JSON line, from nvidia-smi's CSV rows: only rows
+    inside the timed region count; the SM clock is their median; a throttle
+    reason is listed when any counted row shows it active."""
+    import datetime
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    t0 = datetime.datetime(2026, 1, 1, 12, 0, 0)
+
+    def row(dt_s, sm, reasons):
+        ts = (t0 + datetime.timedelta(seconds=dt_s)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        flags = ["Active" if r in reasons else "Not Active"
+                 for r in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                           "sw_power_cap")]
+        return ", ".join([ts, "0", str(sm), "1965", "700.0", "0x0"] + flags)
+
+    path = tmp_path / "clocks.csv"
+    path.write_text("\n".join([
+        row(0.0, 900, {"hw_slowdown"}),          # before the window: ignored
+        row(1.0, 1700, set()),
+        row(1.5, 1600, {"sw_power_cap"}),
+        row(2.0, 1800, set()),
+        "garbled line",
+        row(9.0, 500, {"sw_thermal_slowdown"}),  # after the window: ignored
+    ]) + "\n")
+    s = bench.ClockSampler(0)
+    s.proc, s.path = object(), str(path)        # as if nvidia-smi had written the file
+    got = s.summary((t0 + datetime.timedelta(seconds=0.5)).timestamp(),
+                    (t0 + datetime.timedelta(seconds=2.5)).timestamp())
+    assert got == {"sm_mhz": 1700.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                   "samples": 3}
