@@ -26,6 +26,9 @@ int main(void) {
 
     /* argument errors come back as status codes, before any device work */
     printf("null_q %d\n", bsa_plan(&p, NULL, NULL, NULL, 0, NULL, NULL, 0, NULL));
+    printf("null_bwd_ex %d\n", bsa_backward_ex(&p, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL,
+                                                0, NULL, 0, NULL, NULL, NULL, 20000000u, 3, NULL));
+    printf("null_status %d\n", bsa_read_status(NULL, NULL));
     p.d = 96;
     printf("bad_d %d %s\n", bsa_plan_sizes(&p, &rows, &nnz), bsa_status_string(BSA_ERR_UNSUPPORTED));
     printf("version %d\n", bsa_version());

@@ -461,6 +461,8 @@ def test_plain_c_program_uses_the_header_and_library(L, tmp_path):
     assert got["workspace"] == [str(bsa.bsa_workspace_size(p)),
                                 str(bsa.bsa_backward_workspace_size(p))]
     assert got["null_q"] == [str(bsa.BSA_ERR_INVALID_ARG)]
+    assert got["null_bwd_ex"] == [str(bsa.BSA_ERR_INVALID_ARG)]
+    assert got["null_status"] == [str(bsa.BSA_ERR_INVALID_ARG)]
     assert got["bad_d"][0] == str(bsa.BSA_ERR_UNSUPPORTED)
     assert got["version"] == [str(bsa.bsa_version())]
 
