@@ -183,7 +183,9 @@ BSA_API int bsa_plan(const bsa_params* p, const void* q, const void* k, void* wo
  * query (-inf for an empty row). row_ptr/col_idx: CSR as written by bsa_plan,
  * or any caller CSR with col_capacity entries; rows or columns out of range
  * are skipped (their output is zero) and reported as DEVICE_BAD_INDEX by
- * bsa_read_status. Errors: INVALID_ARG, SHAPE, UNSUPPORTED, ALIGNMENT,
+ * bsa_read_status. Every device-side wait is bounded (2 s); one that expires
+ * stops its CTA cleanly and is reported as DEVICE_TIMEOUT (bsa_forward_ex sets
+ * the limit). Errors: INVALID_ARG, SHAPE, UNSUPPORTED, ALIGNMENT,
  * WORKSPACE_TOO_SMALL, CUDA.
  */
 BSA_API int bsa_forward(const bsa_params* p, const void* q, const void* k, const void* v,
@@ -235,9 +237,11 @@ BSA_API size_t bsa_backward_workspace_size(const bsa_params* p);
  * (no atomic accumulation). row_ptr/col_idx/col_capacity: the CSR given to
  * bsa_forward; rows or columns out of range, and a chunk listed twice in one
  * row, are reported as DEVICE_BAD_INDEX by bsa_read_status(workspace) (the
- * affected gradients are then not meaningful). workspace: device, >=
+ * affected gradients are then not meaningful). Every device-side wait is
+ * bounded (2 s); one that expires stops its CTA cleanly and is reported as
+ * DEVICE_TIMEOUT (bsa_backward_ex sets the limit). workspace: device, >=
  * bsa_backward_workspace_size(p), 16-byte aligned, owned by the caller; its
- * first bytes are the status block that bsa_read_status reads. Errors:
+ * first 256 bytes are the status block that bsa_read_status reads. Errors:
  * INVALID_ARG, SHAPE, UNSUPPORTED, ALIGNMENT, WORKSPACE_TOO_SMALL, CUDA.
  */
 BSA_API int bsa_backward(const bsa_params* p, const void* q, const void* k, const void* v,
