@@ -86,17 +86,22 @@ def kernel_hash():
     return h.hexdigest()[:16]
 
 
-def load_traffic(workload):
-    """DRAM bytes per forward launch from a committed ncu capture, if the
-    kernel source is unchanged since that capture."""
+def load_traffic(wl):
+    """DRAM bytes per forward launch of workload `wl` from a committed ncu
+    capture, if the kernel source is unchanged since that capture. The record
+    is for the named workload's whole call; a rank's launch over part of its
+    (batch, head) pairs moves that share of it (each pair reads its own Q, K,
+    V and writes its own O)."""
+    import synth
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         rec = json.load(f)
-    ent = rec.get(workload)
+    ent = rec.get(wl.name)
     if not ent or ent.get("kernel_hash") != kernel_hash():
         return None
-    return ent.get("bytes_per_launch")
+    full = synth.WORKLOADS[wl.name]
+    return ent["bytes_per_launch"] * (wl.B * wl.heads) / (full.B * full.heads)
 
 
 def exec_flops(wl, nnz):
@@ -601,7 +606,7 @@ def main():
     peak_tf, peak_hbm, peak_src = load_peaks()
     fwd_tflops = flops / (fwd_ms / 1e3) / 1e12
     roofline = {"bound": "tensor", "achieved": fwd_tflops, "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": fwd_tflops / peak_tf, "traffic": load_traffic(wl.name),
+                "frac": fwd_tflops / peak_tf, "traffic": load_traffic(wl),
                 "kernel": "bsa_fwd_kernel", "peak_source": f"{peak_src} bf16 (burst)",
                 "algorithmic_flops_per_launch": flops}
 

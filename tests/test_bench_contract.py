@@ -94,3 +94,26 @@ def test_clock_summary_takes_the_median_and_the_active_reasons_in_the_window(tmp
                     (t0 + datetime.timedelta(seconds=2.5)).timestamp())
     assert got == {"sm_mhz": 1700.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
                    "samples": 3}
+
+
+def test_roofline_traffic_scales_with_a_rank_share_of_the_heads():
+    """The committed DRAM record is for a whole call; a rank that runs 32/N of
+    the heads reports that share per launch, a replica the whole."""
+    import importlib.util
+    import json as _json
+    import synth
+    spec = importlib.util.spec_from_file_location("bench_mod2", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    with open(bench.TRAFFIC_FILE) as f:
+        rec = _json.load(f)["720p"]
+    if rec["kernel_hash"] != bench.kernel_hash():
+        pytest.skip("the record predates the current kernel source")
+    wl = synth.WORKLOADS["720p"]
+    assert bench.load_traffic(wl) == rec["bytes_per_launch"]
+    for world in (2, 4, 8):
+        part, _, _ = bench.rank_problem(wl, 1, world, "heads")
+        assert bench.load_traffic(part) == rec["bytes_per_launch"] / world
+    rep, _, _ = bench.rank_problem(wl, 1, 2, "replicas")
+    assert bench.load_traffic(rep) == rec["bytes_per_launch"]
+    assert bench.load_traffic(synth.WORKLOADS["tiny"]) is None     # no record
