@@ -626,6 +626,8 @@ def main():
             per_config[name] = time_config(synth.WORKLOADS[name], args.per_config_steps,
                                            peak_tf, stream)
 
+    # the whole job's dense-equivalent work (every rank reaches this collective)
+    dense_equiv = sum_over_ranks(4.0 * wl.B * wl.heads * wl.Nq * 128 * wl.N * wl.d)
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -636,8 +638,7 @@ def main():
             "config": workload_config(wl_full, world, parallelism_of(args.partition, world)),
             "plan_ms": plan_ms, "fwd_ms": fwd_ms, "fwd_exec_tflops": fwd_tflops,
             "nnz": nnz, "sparsity": sparsity(wl, nnz),
-            "dense_equiv_tflops": 4.0 * wl.B * wl.heads * wl.Nq * 128 * wl.N * wl.d
-            / ms_per_step / 1e9,
+            "dense_equiv_tflops": dense_equiv / ms_per_step / 1e9,
             "dense": dense, "roofline": roofline, "cpu_baseline": cpu, "backward": bwd,
             "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
