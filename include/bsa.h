@@ -27,7 +27,9 @@
  *   - The caller allocates and owns every buffer. The library never allocates
  *     device memory. Its only process-wide state is the cached tensor-map entry
  *     point and, per device, whether each kernel's shared-memory limit has been
- *     raised; both are safe to reach from several host threads at once.
+ *     raised; both are safe to reach from several host threads at once. The
+ *     second is kept per device number: after making another context current
+ *     on a device, or resetting it, the attention calls return BSA_ERR_CUDA.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Launches are
  *     asynchronous; errors found on the device are read with bsa_read_status.
  *   - Return value: BSA_OK (0) or a bsa_status code. No exception crosses the ABI.
